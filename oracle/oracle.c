@@ -1,0 +1,402 @@
+/*
+ * oracle.c -- plain, slow, single-threaded CPU oracle of the routed-expert MoE
+ * layer.  TEST INFRASTRUCTURE ONLY (see oracle.h): the product path never
+ * links or calls it, and it shares no code with the CUDA kernels.
+ *
+ * Build: gcc -O2 -std=c99 -ffp-contract=off -fPIC -shared oracle.c -lm
+ * (-ffp-contract=off: a*b+c is two roundings unless fmaf() is written.)
+ *
+ * Page citations are given per function.  The pages describe the engine
+ * (colibri) in prose only and print no listing of these steps; where they are
+ * silent, the reading taken is stated at the function.
+ */
+#include "oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* Weight container.                                                         */
+/* int4 weights, one fp16 scale per group of 64 along the input dimension:   */
+/* "gs64 group-scaled" container of colibri (tantan.ink), "我看到的几个坑";   */
+/* gate / up / down of an expert stored next to each other so that one read  */
+/* fetches the expert: colibri (tantan.ink), "几个关键工程动作".              */
+/* Byte layout (this library's reading; the pages give none):                */
+/*   row-major [N][K/2] packed bytes; group g of row n = bytes [32g, 32g+32); */
+/*   byte j of a group: low nibble = element 64g+j, high = element 64g+32+j; */
+/*   nibble u = w + 8 (offset binary), w in [-8, 7];                         */
+/*   then [N][K/64] IEEE fp16 scales; dequantised weight = w * scale.        */
+/* ------------------------------------------------------------------------ */
+
+size_t or_matrix_bytes(int N, int K) {
+  return (size_t)N * (size_t)(K / 2) + (size_t)N * (size_t)(K / 64) * 2u;
+}
+
+size_t or_expert_bytes(int H, int I) {
+  return 2u * or_matrix_bytes(I, H) + or_matrix_bytes(H, I);
+}
+
+int or_weight(const uint8_t *mat, int N, int K, int n, int k) {
+  (void)N;
+  int g = k / 64, j = k % 64;
+  uint8_t byte = mat[(size_t)n * (size_t)(K / 2) + (size_t)(32 * g + (j % 32))];
+  int u = (j < 32) ? (byte & 0x0F) : (byte >> 4);
+  return u - 8;
+}
+
+float or_half_to_float(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int ex = (h >> 10) & 0x1F;
+  int man = h & 0x3FF;
+  float v;
+  if (ex == 0) {
+    v = ldexpf((float)man, -24); /* subnormal: man * 2^-24, exact */
+  } else if (ex == 31) {
+    v = man ? NAN : INFINITY;
+  } else {
+    v = ldexpf((float)(man + 1024), ex - 25); /* (1024+man) * 2^(ex-15-10) */
+  }
+  return sign ? -v : v;
+}
+
+float or_scale(const uint8_t *mat, int N, int K, int n, int g) {
+  const uint8_t *s = mat + (size_t)N * (size_t)(K / 2);
+  size_t o = ((size_t)n * (size_t)(K / 64) + (size_t)g) * 2u;
+  uint16_t h = (uint16_t)(s[o] | (s[o + 1] << 8)); /* little-endian */
+  return or_half_to_float(h);
+}
+
+void or_pack_matrix(const int8_t *w, const uint16_t *s16, int N, int K, uint8_t *mat) {
+  size_t rowb = (size_t)(K / 2);
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < K / 64; ++g) {
+      for (int j = 0; j < 32; ++j) {
+        int lo = w[(size_t)n * K + 64 * g + j] + 8;
+        int hi = w[(size_t)n * K + 64 * g + 32 + j] + 8;
+        mat[(size_t)n * rowb + 32 * g + j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+      }
+    }
+  }
+  uint8_t *s = mat + (size_t)N * rowb;
+  for (size_t i = 0; i < (size_t)N * (size_t)(K / 64); ++i) {
+    s[2 * i] = (uint8_t)(s16[i] & 0xFF);
+    s[2 * i + 1] = (uint8_t)(s16[i] >> 8);
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Q8_0 activations: int8 values in blocks of 32 with one fp32 scale per      */
+/* block -- Colibri article (alphamatch.ai), "優化整數核心".                  */
+/* Reading: d = amax / 127 (one IEEE division), q = round-half-even(x / d);   */
+/* a block with d == 0 quantises to all zeros.                                */
+/* ------------------------------------------------------------------------ */
+
+void or_quant_q8_0(const float *x, int64_t n, int8_t *q, float *d) {
+  for (int64_t b = 0; b < n / 32; ++b) {
+    const float *xb = x + 32 * b;
+    float amax = 0.0f;
+    for (int i = 0; i < 32; ++i) {
+      float a = fabsf(xb[i]);
+      if (a > amax) amax = a;
+    }
+    float db = amax / 127.0f;
+    d[b] = db;
+    for (int i = 0; i < 32; ++i) {
+      int v = 0;
+      if (db != 0.0f) {
+        float r = rintf(xb[i] / db);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        v = (int)r;
+      }
+      q[32 * b + i] = (int8_t)v;
+    }
+  }
+}
+
+/* ------------------------------------------------------------------------ */
+/* exp and SiLU.                                                             */
+/* exp by the Cody-Waite method: x = k ln2 + r with k = rint(x log2 e), ln2   */
+/* split into a 16-bit head (so k*head is exact) and a tail, |r| <= ln2/2;    */
+/* exp(r) by its Taylor series to degree 7 in Horner form; then exp(x) =      */
+/* exp(r) * 2^k with one rounding.  Truncation error r^8/8! < 1e-8 relative.  */
+/* The constants are the mathematical values rounded to binary32.             */
+/* ------------------------------------------------------------------------ */
+
+static float pow2i(int k) { /* 2^k for -126 <= k <= 127, exact */
+  return ldexpf(1.0f, k);
+}
+
+float or_expf(float x) {
+  if (x != x) return x;
+  if (x > 100.0f) return INFINITY;
+  if (x < -104.0f) return 0.0f;
+  const float log2e = 1.44269502162933349609375f;   /* binary32(1/ln 2) */
+  const float ln2_hi = 0.693145751953125f;          /* ln 2, 16 significant bits */
+  const float ln2_lo = 1.428606765330187045037746e-06f; /* binary32(ln 2 - ln2_hi) */
+  float kf = rintf(x * log2e);
+  int k = (int)kf;
+  float r = fmaf(-kf, ln2_hi, x);
+  r = fmaf(-kf, ln2_lo, r);
+  float p = 1.0f / 5040.0f;
+  p = fmaf(p, r, 1.0f / 720.0f);
+  p = fmaf(p, r, 1.0f / 120.0f);
+  p = fmaf(p, r, 1.0f / 24.0f);
+  p = fmaf(p, r, 1.0f / 6.0f);
+  p = fmaf(p, r, 0.5f);
+  p = fmaf(p, r, 1.0f);
+  p = fmaf(p, r, 1.0f);
+  if (k > 126) return (p * pow2i(126)) * pow2i(k - 126);
+  if (k < -126) return (p * pow2i(k + 126)) * pow2i(-126);
+  return p * pow2i(k);
+}
+
+/* SwiGLU expert FFN, SiLU(gate) * up: the experts of the models the pages run
+ * (GLM-5.2 MoE layers; colibri (tantan.ink), "它的核心判断"). */
+float or_silu(float g) {
+  float e = or_expf(-g);
+  float den = 1.0f + e;
+  return g / den;
+}
+
+void or_expf_n(const float *x, float *y, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) y[i] = or_expf(x[i]);
+}
+
+void or_silu_n(const float *x, float *y, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) y[i] = or_silu(x[i]);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Router: per-token scores over the routed experts (256 per layer for       */
+/* GLM-5.2: colibri (tantan.ink), "它的核心判断"), softmax top-k.             */
+/* Fixed order (a reading; the pages give none): 32 chains, chain l sums      */
+/* x[h]*Wr[h] for h = 32i + l, i ascending, with fmaf from 0; then for        */
+/* off = 16,8,4,2,1 every chain becomes c[l] + c[l^off]; the logit is c[0].   */
+/* Routing must not change with placement (colibri deep review, design rule   */
+/* "never silently change precision or router semantics"), so both sides    */
+/* use this one order and the selected experts are reproducible bit for bit. */
+/* ------------------------------------------------------------------------ */
+
+float or_router_logit(const float *x, const float *wr, int H) {
+  float c[32], t[32];
+  for (int l = 0; l < 32; ++l) {
+    float p = 0.0f;
+    for (int i = 0; 32 * i + l < H; ++i) p = fmaf(x[32 * i + l], wr[32 * i + l], p);
+    c[l] = p;
+  }
+  for (int off = 16; off >= 1; off >>= 1) {
+    for (int l = 0; l < 32; ++l) t[l] = c[l] + c[l ^ off];
+    memcpy(c, t, sizeof c);
+  }
+  return c[0];
+}
+
+void or_router_logits(const float *x, const float *Wr, int T, int H, int E, float *logits) {
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e)
+      logits[(size_t)t * E + e] = or_router_logit(x + (size_t)t * H, Wr + (size_t)e * H, H);
+}
+
+/* Top-k: the k largest logits, a tie going to the lower expert index, listed
+ * by descending logit.  Weights: softmax over the k kept logits, i.e. the full
+ * softmax renormalised over the selection:
+ *   m = l[idx0]; e_s = exp(l_s - m); Z = ((e_0 + e_1) + e_2) + ...; w_s = e_s / Z. */
+void or_topk_softmax(const float *logits, int T, int E, int k, int32_t *idx, float *w) {
+  unsigned char *taken = (unsigned char *)malloc((size_t)E);
+  float *ev = (float *)malloc(sizeof(float) * (size_t)k);
+  for (int t = 0; t < T; ++t) {
+    const float *l = logits + (size_t)t * E;
+    memset(taken, 0, (size_t)E);
+    for (int s = 0; s < k; ++s) {
+      int best = -1;
+      for (int e = 0; e < E; ++e)
+        if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+      taken[best] = 1;
+      idx[(size_t)t * k + s] = best;
+    }
+    float m = l[idx[(size_t)t * k]];
+    float z = 0.0f;
+    for (int s = 0; s < k; ++s) {
+      ev[s] = or_expf(l[idx[(size_t)t * k + s]] - m);
+      z = (s == 0) ? ev[0] : z + ev[s];
+    }
+    for (int s = 0; s < k; ++s) w[(size_t)t * k + s] = ev[s] / z;
+  }
+  free(ev);
+  free(taken);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Batch union: the experts picked by the batch, each listed once, so each is */
+/* fetched once -- colibri (tantan.ink), "几个关键工程动作" (Batch union), and */
+/* the batched-union MoE of prefill, Colibri article (alphamatch.ai).         */
+/* cnt[e] = pairs routed to e; off = exclusive prefix sum (off[E] = T*k);     */
+/* uni = experts with cnt > 0 ascending; perm = pair ids p = t*k+s grouped by */
+/* expert, ascending p inside each group (a stable counting sort).            */
+/* ------------------------------------------------------------------------ */
+
+void or_bucket(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *off,
+               int32_t *uni, int32_t *n_uni, int32_t *perm) {
+  int P = T * k;
+  for (int e = 0; e < E; ++e) cnt[e] = 0;
+  for (int p = 0; p < P; ++p) cnt[idx[p]] += 1;
+  off[0] = 0;
+  for (int e = 0; e < E; ++e) off[e + 1] = off[e] + cnt[e];
+  int nu = 0;
+  for (int e = 0; e < E; ++e)
+    if (cnt[e] > 0) uni[nu++] = e;
+  *n_uni = nu;
+  int32_t *cur = (int32_t *)malloc(sizeof(int32_t) * (size_t)(E > 0 ? E : 1));
+  for (int e = 0; e < E; ++e) cur[e] = off[e];
+  for (int p = 0; p < P; ++p) perm[cur[idx[p]]++] = p;
+  free(cur);
+}
+
+/* ------------------------------------------------------------------------ */
+/* int4 x int8 dot products (the integer kernels of the engine: Colibri       */
+/* article (alphamatch.ai), "優化整數核心").                                  */
+/* Row n of a [N][K] matrix against a Q8_0 vector (q, d):                     */
+/*   S_b = sum over the 32 elements of block b of w*q          (exact int32) */
+/*   group g (blocks 2g, 2g+1, scale s_g):                                    */
+/*     a = float(S_2g) * d_2g;  b = fmaf(float(S_2g+1), d_2g+1, a)            */
+/*   the G = K/64 groups are cut into chunks of csz = ceil(G/32) consecutive  */
+/*   groups; inside a chunk acc = fmaf(s_g, b, acc) from 0, g ascending;      */
+/*   the chunk sums are added left to right.  (Fixed order, this library's    */
+/*   reading: the hidden state h feeds a second quantisation, so both sides   */
+/*   must produce it bit for bit.)                                            */
+/* ------------------------------------------------------------------------ */
+
+int32_t or_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q) {
+  int32_t s = 0;
+  for (int i = 0; i < 32; ++i) s += or_weight(mat, N, K, n, 32 * b + i) * (int32_t)q[32 * b + i];
+  return s;
+}
+
+float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {
+  int G = K / 64;
+  int csz = (G + 31) / 32;
+  int nch = (G + csz - 1) / csz;
+  float total = 0.0f;
+  for (int c = 0; c < nch; ++c) {
+    float acc = 0.0f;
+    int g1 = (c + 1) * csz < G ? (c + 1) * csz : G;
+    for (int g = c * csz; g < g1; ++g) {
+      int32_t s0 = or_block_dot(mat, N, K, n, 2 * g, q);
+      int32_t s1 = or_block_dot(mat, N, K, n, 2 * g + 1, q);
+      float a = (float)s0 * d[2 * g];
+      float b = fmaf((float)s1, d[2 * g + 1], a);
+      acc = fmaf(or_scale(mat, N, K, n, g), b, acc);
+    }
+    total = (c == 0) ? acc : total + acc;
+  }
+  return total;
+}
+
+void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
+                   float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
+  const uint8_t *gate = blob;
+  const uint8_t *up = blob + or_matrix_bytes(I, H);
+  const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
+  float *hh = (float *)malloc(sizeof(float) * (size_t)I);
+  int8_t *q = (int8_t *)malloc((size_t)I);
+  float *dd = (float *)malloc(sizeof(float) * (size_t)(I / 32));
+  for (int n = 0; n < I; ++n) {
+    float gv = or_expert_dot(gate, I, H, n, xq, xd);
+    float uv = or_expert_dot(up, I, H, n, xq, xd);
+    if (g) g[n] = gv;
+    if (u) u[n] = uv;
+    hh[n] = or_silu(gv) * uv;
+  }
+  or_quant_q8_0(hh, I, q, dd);
+  if (h) memcpy(h, hh, sizeof(float) * (size_t)I);
+  if (hq) memcpy(hq, q, (size_t)I);
+  if (hd) memcpy(hd, dd, sizeof(float) * (size_t)(I / 32));
+  if (y)
+    for (int m = 0; m < H; ++m) y[m] = or_expert_dot(down, H, I, m, q, dd);
+  free(dd);
+  free(q);
+  free(hh);
+}
+
+/* ------------------------------------------------------------------------ */
+/* The layer: shared expert (part of the resident dense weights, colibri      */
+/* (tantan.ink), "它的核心判断") plus the router-weighted routed experts.      */
+/* out[t] = y_shared; then for s = 0..k-1: out = fmaf(w[t,s], y_s, out).      */
+/* No residual add, no norm: the input is the already normalised hidden       */
+/* state (reading).  The shared expert has weight 1 (reading).               */
+/* ------------------------------------------------------------------------ */
+
+static int dims_ok(int H, int I, int E, int k) {
+  return H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0 && E >= 1 && k >= 1 && k <= E;
+}
+
+static void token_forward(int H, int I, int E, int k, const float *xt, const float *Wr,
+                          const uint8_t *const *blobs, float *out, int8_t *xq_o, float *xd_o,
+                          float *logit_o, int32_t *idx_o, float *w_o, int8_t *hq_o,
+                          float *hd_o, float *y_o) {
+  int8_t *xq = (int8_t *)malloc((size_t)H);
+  float *xd = (float *)malloc(sizeof(float) * (size_t)(H / 32));
+  float *lg = (float *)malloc(sizeof(float) * (size_t)E);
+  int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+  float *w = (float *)malloc(sizeof(float) * (size_t)k);
+  float *y = (float *)malloc(sizeof(float) * (size_t)H);
+  or_quant_q8_0(xt, H, xq, xd);
+  or_router_logits(xt, Wr, 1, H, E, lg);
+  or_topk_softmax(lg, 1, E, k, idx, w);
+  /* shared expert first (slot k in the trace) */
+  or_expert_ffn(blobs[E], H, I, xq, xd, NULL, NULL, NULL, hq_o ? hq_o + (size_t)k * I : NULL,
+                hd_o ? hd_o + (size_t)k * (I / 32) : NULL, y);
+  if (y_o) memcpy(y_o + (size_t)k * H, y, sizeof(float) * (size_t)H);
+  memcpy(out, y, sizeof(float) * (size_t)H);
+  for (int s = 0; s < k; ++s) {
+    or_expert_ffn(blobs[idx[s]], H, I, xq, xd, NULL, NULL, NULL, hq_o ? hq_o + (size_t)s * I : NULL,
+                  hd_o ? hd_o + (size_t)s * (I / 32) : NULL, y);
+    if (y_o) memcpy(y_o + (size_t)s * H, y, sizeof(float) * (size_t)H);
+    for (int m = 0; m < H; ++m) out[m] = fmaf(w[s], y[m], out[m]);
+  }
+  if (xq_o) memcpy(xq_o, xq, (size_t)H);
+  if (xd_o) memcpy(xd_o, xd, sizeof(float) * (size_t)(H / 32));
+  if (logit_o) memcpy(logit_o, lg, sizeof(float) * (size_t)E);
+  if (idx_o) memcpy(idx_o, idx, sizeof(int32_t) * (size_t)k);
+  if (w_o) memcpy(w_o, w, sizeof(float) * (size_t)k);
+  free(y);
+  free(w);
+  free(idx);
+  free(lg);
+  free(xd);
+  free(xq);
+}
+
+int or_moe_layer(int H, int I, int E, int k, int T, const float *x, const float *Wr,
+                 const uint8_t *const *blobs, float *out, or_layer_trace *tr) {
+  if (!dims_ok(H, I, E, k) || T < 0) return -1;
+  int32_t *idx_all = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T * k : 1));
+  for (int t = 0; t < T; ++t) {
+    size_t tk = (size_t)t * (size_t)(k + 1);
+    token_forward(H, I, E, k, x + (size_t)t * H, Wr, blobs, out + (size_t)t * H,
+                  tr && tr->xq ? tr->xq + (size_t)t * H : NULL,
+                  tr && tr->xd ? tr->xd + (size_t)t * (H / 32) : NULL,
+                  tr && tr->logits ? tr->logits + (size_t)t * E : NULL, idx_all + (size_t)t * k,
+                  tr && tr->w ? tr->w + (size_t)t * k : NULL,
+                  tr && tr->hq ? tr->hq + tk * I : NULL,
+                  tr && tr->hd ? tr->hd + tk * (I / 32) : NULL,
+                  tr && tr->y ? tr->y + tk * H : NULL);
+  }
+  if (tr && tr->idx) memcpy(tr->idx, idx_all, sizeof(int32_t) * (size_t)T * k);
+  if (tr && tr->cnt && tr->off && tr->uni && tr->n_uni && tr->perm)
+    or_bucket(idx_all, T, k, E, tr->cnt, tr->off, tr->uni, tr->n_uni, tr->perm);
+  free(idx_all);
+  return 0;
+}
+
+int or_moe_layer_tokens(int H, int I, int E, int k, const float *x, const float *Wr,
+                        const uint8_t *const *blobs, const int32_t *tok, int n_tok,
+                        float *out) {
+  if (!dims_ok(H, I, E, k) || n_tok < 0) return -1;
+  for (int i = 0; i < n_tok; ++i)
+    token_forward(H, I, E, k, x + (size_t)tok[i] * H, Wr, blobs, out + (size_t)i * H, NULL,
+                  NULL, NULL, NULL, NULL, NULL, NULL, NULL);
+  return 0;
+}
