@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark of the routed-expert MoE layer on B200.
+
+Default workload: one GLM-5.2-shaped MoE layer in decode (H=6144, 256 routed
+experts of SwiGLU intermediate 2048 + 1 shared, top-8 softmax routing, batch 1,
+all 257 int4 gs64 experts resident in HBM).  A step is one moe_layer_forward
+(router + top-k + bucket, fused gate/up + SwiGLU + requant, down + combine) on
+one token drawn from a pool of 64 seeded hidden states, so the routed union
+varies from step to step.
+
+Metric: expert-weight GB/s of the layer = (|union| + 1) * 20,054,016 bytes per
+step / device time of the step (plus us per token-layer and the per-kernel
+roofline).  L2 is flushed (256 MiB write) before every timed step, outside the
+step's CUDA events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own replica of
+the layer on its own tokens (the path has no cross-token exchange), timing is
+the max over ranks, value = bytes all ranks streamed / that time ("weak").
+--impl reference times the CPU oracle (single thread, plain C) on a bounded
+sample of the same workload on this machine's host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import moe_inputs as mi  # noqa: E402
+
+METRIC = "MoE layer µs/token & expert-weight GB/s vs HBM peak; prefill int8 TOPS"
+POOL = 64
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.f = None
+
+    def __enter__(self):
+        try:
+            self.f = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.f.seek(0)
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allreduce_max(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def allreduce_sum(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- oracle timing
+def oracle_sample(w: mi.Workload, x_pool, Wr_h, blob_fn, budget_s: float, max_tokens: int):
+    """Times the CPU oracle token-layer by token-layer until the budget is spent.
+    Returns (bytes, seconds, tokens)."""
+    import numpy as np
+
+    import oracle as orc
+    blob_bytes = w.blob_bytes
+    total_b, total_s, n = 0, 0.0, 0
+    cache = {}
+    for i in range(max_tokens):
+        xt = x_pool[i % len(x_pool)].reshape(1, -1)
+        lg = orc.router_logits(xt, Wr_h)
+        idx, _ = orc.topk_softmax(lg, w.k)
+        need = sorted(set(idx.reshape(-1).tolist()) | {w.E})
+        for e in need:
+            if e not in cache:
+                cache[e] = blob_fn(e)
+        dummy = np.zeros(16, np.uint8)
+        blist = [cache.get(e, dummy) for e in range(w.E + 1)]
+        t0 = time.perf_counter()
+        orc.moe_layer(xt, Wr_h, blist, w.H, w.I, w.E, w.k)
+        dt = time.perf_counter() - t0
+        total_b += len(need) * blob_bytes
+        total_s += dt
+        n += 1
+        if total_s >= budget_s:
+            break
+    return total_b, total_s, n
+
+
+# ----------------------------------------------------------------- native arm
+def run_native(args, ws_n, rank, local):
+    import int4_routed_expert_softmax_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = mi.WORKLOADS[args.workload]
+    seed = w.seed + 1000 * rank
+    wl = mi.shrink(w, seed=seed)
+    T = w.T
+    Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), dev)
+    blobs = mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, 0, 3), dev)
+    xpool = mi.make_x(POOL * T, w.H, mi.sub_seed(seed, 0, 1), dev).view(POOL, T, w.H)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    ws = moe.alloc_workspace(d, T, dev)
+    table = moe.expert_table(blobs)
+    out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    view = moe.moe_workspace_view(d, T, ws)
+    nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
+    status_t = moe.ws_slice(ws, view.status, (4,), torch.int32)
+    blob_b = w.blob_bytes
+    gu_b = 2 * mi.matrix_bytes(w.I, w.H)
+    dn_b = mi.matrix_bytes(w.H, w.I)
+    router_b = w.E * w.H * 4
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        moe.moe_layer_forward(d, xpool[i % POOL], Wr, table, out, ws)
+
+    moe.moe_profile_enable(True)
+    for i in range(args.warmup):
+        flush.zero_()
+        step(i)
+    torch.cuda.synchronize()
+    if int(status_t[0].item()) != 0:
+        raise RuntimeError(f"device status {status_t.tolist()}")
+
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    layer_ms, prof, nuni = [], [], []
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev0[i].record(stream)
+            step(args.warmup + i)
+            ev1[i].record(stream)
+            prof.append(moe.moe_profile_last())       # waits for this step
+            nuni.append(int(nuni_t.item()))
+        torch.cuda.synchronize()
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    for i in range(K):
+        layer_ms.append(ev0[i].elapsed_time(ev1[i]))
+    moe.moe_profile_enable(False)
+    if int(status_t[0].item()) != 0:
+        raise RuntimeError(f"device status {status_t.tolist()}")
+
+    my_bytes = sum((u + 1) * blob_b for u in nuni)
+    my_ms = sum(layer_ms)
+    max_ms = allreduce_max(my_ms, ws_n)
+    all_bytes = allreduce_sum(float(my_bytes), ws_n)
+    value = all_bytes / (max_ms * 1e-3) / 1e9
+    ms_per_step = max_ms / K
+
+    gu_ms = sum(p[1] for p in prof)
+    dn_ms = sum(p[2] for p in prof)
+    rt_ms = sum(p[0] for p in prof)
+    gu_bytes = sum((u + 1) * gu_b for u in nuni)
+    dn_bytes = sum((u + 1) * dn_b for u in nuni)
+    peak, peak_src = peaks()
+    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "k_gateup_decode", "achieved": round(gu_gbs, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(gu_gbs / peak, 4),
+                "peak_source": peak_src, "traffic": None,
+                "bytes_per_launch": round(gu_bytes / K), "us_per_launch": round(gu_ms / K * 1e3, 2)}
+    kernels = {
+        "k_route_decode": {"us": round(rt_ms / K * 1e3, 2),
+                           "GB/s": round(router_b * K / (rt_ms * 1e-3) / 1e9, 1)},
+        "k_gateup_decode": {"us": round(gu_ms / K * 1e3, 2), "GB/s": round(gu_gbs, 1)},
+        "k_down_decode": {"us": round(dn_ms / K * 1e3, 2),
+                          "GB/s": round(dn_bytes / (dn_ms * 1e-3) / 1e9, 1)},
+    }
+
+    # ---- end to end: host buffers through moe_layer_forward_host
+    e2e = None
+    if not args.no_e2e:
+        xh = xpool.cpu().pin_memory()
+        oh = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
+        for i in range(args.warmup):
+            moe.moe_layer_forward_host(d, xh[i % POOL], Wr, table, oh, ws)
+        torch.cuda.synchronize()
+        e_ms, e_bytes = 0.0, 0
+        barrier(ws_n)
+        torch.cuda.synchronize()
+        for i in range(K):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            moe.moe_layer_forward_host(d, xh[(args.warmup + i) % POOL], Wr, table, oh, ws)
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+            e_bytes += (int(nuni_t.item()) + 1) * blob_b
+        barrier(ws_n)
+        e_max = allreduce_max(e_ms, ws_n)
+        e_all = allreduce_sum(float(e_bytes), ws_n)
+        e2e = {"value": round(e_all / (e_max * 1e-3) / 1e9, 1), "unit": "GB/s",
+               "h2d_bytes_per_step": T * w.H * 4, "d2h_bytes_per_step": T * w.H * 4,
+               "us_per_token_layer": round(e_max / K / T * 1e3, 2)}
+
+    # ---- CPU oracle baseline (rank 0, single GPU only)
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu:
+        xh = xpool.cpu().numpy()
+        Wr_h = Wr.cpu().numpy()
+        nb, ns, nt = oracle_sample(w, xh.reshape(POOL * T, w.H), Wr_h,
+                                   lambda e: blobs[e].cpu().numpy(), args.cpu_seconds, 64)
+        cpu = {"value": round(nb / ns / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "us_per_token_layer": round(ns / nt * 1e6, 1),
+               "sample": f"{nt} token-layers of the decode workload (pool draws 0..{nt - 1}), "
+                         f"single-threaded C oracle"}
+
+    clocks = clk.summary()
+    return dict(
+        metric=METRIC, value=round(value, 1), unit="GB/s", n_gpus=ws_n, steps=K, warmup=args.warmup,
+        ms_per_step=round(ms_per_step, 5), higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="int4xint8->fp32", data="synthetic",
+        config={"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
+                            "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
+                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": T, "global_batch": T * ws_n,
+                "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
+                "x_pool": POOL},
+        us_per_token_layer=round(ms_per_step / T * 1e3, 2),
+        union_mean=round(sum(nuni) / len(nuni), 2),
+        roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clocks,
+        gpu_launches=3 * K, wall_s=round(wall, 3))
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, ws_n, rank):
+    """The CPU oracle on a bounded sample of the same workload (rank 0 only)."""
+    if rank != 0:
+        return None
+    import numpy as np  # noqa: F401
+
+    import oracle as orc  # noqa: F401
+    w = mi.WORKLOADS[args.workload]
+    seed = w.seed
+    Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), "cpu").numpy()
+    xpool = mi.make_x(POOL * w.T, w.H, mi.sub_seed(seed, 0, 1), "cpu").numpy()
+    cache = {}
+
+    def blob_fn(e):
+        if e not in cache:
+            b = torch.empty(w.blob_bytes, dtype=torch.uint8)
+            mi.fill_blob(b, w.H, w.I, mi.blob_seed(mi.sub_seed(seed, 0, 3), e))
+            cache[e] = b.numpy()
+        return cache[e]
+
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    mi_ = 0
+    for _ in range(args.warmup):
+        oracle_sample(w, xpool[mi_:mi_ + 1], Wr, blob_fn, 0.0, 1)
+        mi_ += 1
+    tb, ts, tn = 0, 0.0, 0
+    for i in range(args.steps):
+        b, s, n = oracle_sample(w, xpool[(mi_ + i) % POOL:(mi_ + i) % POOL + 1], Wr, blob_fn, per_step, 1)
+        tb, ts, tn = tb + b, ts + s, tn + n
+    value = tb / ts / 1e9
+    cpu = {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"{tn} token-layers of the decode workload, single-threaded C oracle"}
+    return dict(
+        impl="reference", metric=METRIC, value=round(value, 4), unit="GB/s", n_gpus=ws_n,
+        steps=args.steps, warmup=args.warmup, ms_per_step=round(ts / max(1, tn) * 1e3, 3),
+        higher_is_better=True, scaling="weak", vs_baseline=None, dtype="int4xint8->fp32",
+        data="synthetic",
+        config={"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
+                            "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
+                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T},
+        us_per_token_layer=round(ts / max(1, tn) * 1e6, 1), cpu_baseline=cpu,
+        e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        ws_n = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        res = run_reference(args, ws_n, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    ws_n, rank, local = dist_setup()
+    try:
+        res = run_native(args, ws_n, rank, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if ws_n > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+/*
+ * moe.h -- C ABI of libmoe: the routed-expert MoE layer (softmax top-k router,
+ * batch union, int4 gs64 x Q8_0 SwiGLU experts, shared expert, weighted
+ * combine) on NVIDIA B200 (sm_100a).
+ *
+ * What the layer is, by page and section of the sources:
+ *  - MoE layer with 256 routed experts per layer plus shared experts kept in
+ *    the resident dense part; only the routed experts are streamed:
+ *    "colibrì：把 744B 模型当数据流流到 25GB 的笔记本上跑" (tantan.ink),
+ *    section 它的核心判断.
+ *  - int4 weights with one scale per group of 64 ("gs64 group-scaled"): same
+ *    page, section 我看到的几个坑.
+ *  - int8 activations in 32-wide blocks with one scale per block ("Q8_0
+ *    style") and an integer dot kernel: "Colibri：革命性 AI 引擎" (alphamatch.ai),
+ *    section 優化整數核心.
+ *  - batch union (each selected expert read once per batch) and gate/up/down
+ *    stored next to each other: tantan.ink page, section 几个关键工程动作.
+ *  - per-layer LRU cache, learned pins from route counts, one-layer-ahead
+ *    prefetch: same section, and "colibri deep review" (ai-tools-nav), the
+ *    "权重 JIT" row of its technique table.
+ *
+ * Conventions (every entry point):
+ *  - Returns MOE_OK (0) or a negative MOE_ERR_* code.  Argument and shape
+ *    errors are detected on the host before anything is enqueued.
+ *  - Tensor pointers are DEVICE pointers owned by the caller unless the
+ *    parameter says "host".  The library never frees caller memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream.
+ *  - Device-side failures (a bounded wait that ran out, a misaligned expert
+ *    pointer) are written to the status word of the workspace (see
+ *    moe_workspace_view); kernels never trap.
+ *  - Not thread-safe for concurrent calls sharing one workspace.
+ *
+ * Data layouts (row-major, little-endian):
+ *  - Expert blob: gate [I][H] | up [I][H] | down [H][I], each matrix
+ *    [N][K] stored as N*K/2 packed bytes then N*K/64 fp16 scales.
+ *    Group g of row n = bytes [32g, 32g+32) of the row; byte j holds element
+ *    64g+j in its low nibble and element 64g+32+j in its high nibble; a
+ *    nibble u encodes w = u - 8 in [-8, 7]; dequantised weight = w * scale.
+ *    Blob pointers must be 16-byte aligned.
+ *  - Q8_0 vectors: int8 codes [n] and fp32 scales [n/32]; d = amax/127,
+ *    q = round-half-even(x/d), all-zero codes when d == 0.
+ *  - Shapes: H % 128 == 0, I % 128 == 0, H <= 8192, I <= 4096,
+ *    1 <= k <= min(E, 32), E <= 1024.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOE_GROUP 64 /* int4 weights per fp16 scale */
+#define MOE_BLOCK 32 /* int8 activations per fp32 scale */
+#define MOE_MAX_E 1024
+#define MOE_DECODE_T_MAX 16 /* largest batch the decode (GEMV) kernels take */
+
+enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_BAD_ARG = -1,     /* NULL pointer, negative size, bad enum */
+  MOE_ERR_SHAPE = -2,       /* dims outside the accepted shapes */
+  MOE_ERR_CUDA = -3,        /* a CUDA runtime call failed */
+  MOE_ERR_WORKSPACE = -4,   /* workspace too small or misaligned */
+  MOE_ERR_CACHE_FULL = -5,  /* every cache slot is pinned or in use */
+  MOE_ERR_NOT_RESIDENT = -6,/* expert not in the cache */
+  MOE_ERR_TIMEOUT = -7,     /* a device-side bounded wait ran out */
+  MOE_ERR_DEVICE = -8,      /* device-side check failed (see status word) */
+  MOE_ERR_ALLOC = -9        /* host or device allocation failed */
+};
+
+typedef struct moe_dims {
+  int32_t H; /* hidden size */
+  int32_t I; /* SwiGLU intermediate size of every expert (routed and shared) */
+  int32_t E; /* routed experts */
+  int32_t k; /* experts kept per token */
+} moe_dims;
+
+enum moe_path {
+  MOE_PATH_AUTO = 0,    /* decode kernels for T <= MOE_DECODE_T_MAX, else prefill */
+  MOE_PATH_DECODE = 1,  /* GEMV kernels, T processed in chunks of MOE_DECODE_T_MAX */
+  MOE_PATH_PREFILL = 2  /* grouped GEMM over the expert union */
+};
+
+/* Human-readable name of a status code (static string). */
+const char *moe_status_string(int status);
+
+/* MOE_OK if the dims are accepted, else MOE_ERR_SHAPE / MOE_ERR_BAD_ARG. */
+int moe_check_dims(const moe_dims *dims);
+
+/* Bytes of one expert blob: 3*H*I/2 + 3*H*I/32 (20,054,016 for H=6144,
+ * I=2048).  0 if the dims are not accepted. */
+size_t moe_expert_bytes(const moe_dims *dims);
+
+/* Device workspace needed by moe_layer_forward for batches of up to T_max
+ * tokens (256-byte aligned segments).  0 if the dims are not accepted. */
+size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max);
+
+/* Q8_0 quantisation of rows x T x cols fp32 (cols % 32 == 0):
+ * q [rows][cols] int8, d [rows][cols/32] fp32.  Bit-exact definition above.
+ * (Q8_0-style activations: alphamatch.ai page, section 優化整數核心.) */
+int moe_quant_q8_0(const float *x, int64_t rows, int32_t cols, int8_t *q, float *d,
+                   void *stream);
+
+/* Router: logits[t][e] = x[t] . Wr[e] in the library's fixed fp32 order
+ * (32 strided fmaf chains, xor tree), then top-k per token (ties to the lower
+ * expert index, listed by descending logit) and the softmax over the k kept
+ * logits.  x [T][H] fp32, Wr [E][H] fp32 (both 16-byte aligned), idx [T][k]
+ * int32, w [T][k] fp32, logits [T][E] fp32 (written; also the scratch the
+ * top-k reads), route_counts_opt [E] int32 or NULL
+ * (incremented by one per selection: the route-count record behind learned
+ * pins, tantan.ink page section 几个关键工程动作). */
+int moe_router_topk(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                    int32_t *idx, float *w, float *logits, int32_t *route_counts_opt,
+                    void *stream);
+
+/* Batch union (tantan.ink page, section 几个关键工程动作): counting sort of the
+ * T*k (token, slot) pairs by expert.  idx [T][k] int32 ->
+ *   cnt [E]      pairs per expert
+ *   off [E+1]    exclusive prefix sum, off[E] = T*k
+ *   uni [E]      experts with cnt > 0, ascending (first *n_uni entries)
+ *   n_uni [1]    union size
+ *   perm [T*k]   pair ids t*k+s grouped by expert, ascending inside a group.
+ * All outputs are bit-exact (one correct answer). */
+int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt,
+               int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm, void *stream);
+
+/* The whole layer on T tokens:
+ *   x [T][H] fp32 (the normalised hidden state; no residual, no norm here),
+ *   Wr [E][H] fp32,
+ *   expert_table: DEVICE array of E+1 device pointers to expert blobs;
+ *                 entry E is the shared expert (weight 1),
+ *   out [T][H] fp32 = shared(x) + sum_s w[t,s] * expert_{idx[t,s]}(x),
+ *   ws / ws_bytes: device workspace of at least moe_workspace_bytes(dims, T),
+ *                  256-byte aligned; holds every intermediate (see view),
+ *   route_counts_opt [E] int32 or NULL (incremented per selection),
+ *   path: enum moe_path.
+ * Every step runs in the library's kernels; nothing is synchronised with the
+ * host.  Results do not depend on the path. */
+int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                      const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                      int32_t *route_counts_opt, int32_t path, void *stream);
+
+/* Same as moe_layer_forward with x_host [T][H] and out_host [T][H] in HOST
+ * memory (pinned for overlap; pageable works but serialises).  The copies in
+ * and out are enqueued on `stream` around the layer; the call returns after
+ * enqueueing (synchronise the stream before reading out_host). */
+int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
+                           const float *Wr, const void *const *expert_table, float *out_host,
+                           void *ws, size_t ws_bytes, int32_t *route_counts_opt, int32_t path,
+                           void *stream);
+
+/* Device pointers to the intermediates a moe_layer_forward call leaves in its
+ * workspace (for tests and tools).  Pair positions: the T*k routed pairs in
+ * bucket order (position off[e]+i for the i-th pair of expert e), then T
+ * shared-expert pairs at positions T*k + t. */
+typedef struct moe_ws_view {
+  int32_t *status;   /* [4]: [0] = MOE_OK or a device error code, [1] = detail */
+  int8_t *xq;        /* [T][H] */
+  float *xd;         /* [T][H/32] */
+  float *logits;     /* [T][E] */
+  int32_t *idx;      /* [T][k] */
+  float *w;          /* [T][k] */
+  int32_t *cnt;      /* [E] */
+  int32_t *off;      /* [E+1] */
+  int32_t *uni;      /* [E+1]: union ascending, then E (the shared expert) */
+  int32_t *n_uni;    /* [1] */
+  int32_t *perm;     /* [T*k] */
+  int32_t *pos;      /* [T*k]: position of pair t*k+s */
+  int32_t *pair_tok; /* [T*(k+1)]: token of each position */
+  int8_t *hq;        /* [T*(k+1)][I] Q8_0 codes of SiLU(g)*u per position */
+  float *hd;         /* [T*(k+1)][I/32] */
+  int32_t T_max;
+} moe_ws_view;
+
+int moe_workspace_view(const moe_dims *dims, int32_t T_max, void *ws, moe_ws_view *view);
+
+/* Number of streaming multiprocessors the kernels size their grids for
+ * (device of the current context), or a negative status. */
+int moe_device_sms(void);
+
+/* Per-kernel timing.  moe_profile_enable(1) makes every following
+ * moe_layer_forward record CUDA events on its stream around each of its
+ * kernels (library-owned events of the current device); moe_profile_enable(0)
+ * stops it.  moe_profile_last(ms, n) waits for the events of the most recent
+ * forward call and writes up to n durations in milliseconds:
+ *   ms[0] router + top-k + bucket, ms[1] gate/up (+ SwiGLU + requant),
+ *   ms[2] down + combine.
+ * Returns the number of durations written, or a negative status. */
+int moe_profile_enable(int on);
+int moe_profile_last(float *ms, int n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

@@ -1,0 +1,198 @@
+"""ctypes binding of libmoe.so (include/moe.h).  Argument marshalling only:
+every step of the layer runs in the library's CUDA kernels.  Torch is used for
+device memory and streams; the functions take torch tensors and pass their
+data pointers and the current CUDA stream.
+
+Importing never falls back to anything else: if libmoe.so is missing or does not
+load, the first call raises."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmoe.so")
+
+MOE_OK = 0
+MOE_PATH_AUTO, MOE_PATH_DECODE, MOE_PATH_PREFILL = 0, 1, 2
+MOE_DECODE_T_MAX = 16
+
+
+class MoeDims(ctypes.Structure):
+    _fields_ = [("H", ctypes.c_int32), ("I", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32)]
+
+
+class MoeWsView(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in (
+        "status", "xq", "xd", "logits", "idx", "w", "cnt", "off", "uni", "n_uni", "perm", "pos",
+        "pair_tok", "hq", "hd")] + [("T_max", ctypes.c_int32)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status} ({status_string(status)})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libmoe.so not built ({LIB_PATH}); run "
+                               "python -m int4_routed_expert_softmax_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        D = ctypes.POINTER(MoeDims)
+        sig = {
+            "moe_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "moe_check_dims": (ctypes.c_int, [D]),
+            "moe_expert_bytes": (sz, [D]),
+            "moe_workspace_bytes": (sz, [D, i32]),
+            "moe_workspace_view": (ctypes.c_int, [D, i32, P, ctypes.POINTER(MoeWsView)]),
+            "moe_device_sms": (ctypes.c_int, []),
+            "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+            "moe_profile_last": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
+            "moe_quant_q8_0": (ctypes.c_int, [P, i64, i32, P, P, P]),
+            "moe_router_topk": (ctypes.c_int, [D, i32, P, P, P, P, P, P, P]),
+            "moe_bucket": (ctypes.c_int, [D, i32, P, P, P, P, P, P, P]),
+            "moe_layer_forward": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
+            "moe_layer_forward_host": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    assert t.is_contiguous(), "tensors passed to libmoe must be contiguous"
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, rc: int):
+    if rc != MOE_OK:
+        raise MoeError(fn, rc)
+
+
+def dims(H: int, I: int, E: int, k: int) -> MoeDims:
+    return MoeDims(H, I, E, k)
+
+
+def status_string(status: int) -> str:
+    return lib().moe_status_string(status).decode()
+
+
+def moe_check_dims(d: MoeDims) -> int:
+    return lib().moe_check_dims(ctypes.byref(d))
+
+
+def moe_expert_bytes(d: MoeDims) -> int:
+    return int(lib().moe_expert_bytes(ctypes.byref(d)))
+
+
+def moe_workspace_bytes(d: MoeDims, T_max: int) -> int:
+    return int(lib().moe_workspace_bytes(ctypes.byref(d), T_max))
+
+
+def moe_device_sms() -> int:
+    return int(lib().moe_device_sms())
+
+
+def moe_profile_enable(on: bool) -> None:
+    lib().moe_profile_enable(1 if on else 0)
+
+
+def moe_profile_last() -> list:
+    """Per-kernel ms of the last forward: [router+bucket, gate/up, down]."""
+    buf = (ctypes.c_float * 3)()
+    n = lib().moe_profile_last(buf, 3)
+    if n < 0:
+        raise MoeError("moe_profile_last", n)
+    return [float(buf[i]) for i in range(n)]
+
+
+def moe_quant_q8_0(x: torch.Tensor, q: torch.Tensor, d: torch.Tensor, stream=None):
+    rows, cols = x.shape
+    _check("moe_quant_q8_0", lib().moe_quant_q8_0(_ptr(x), rows, cols, _ptr(q), _ptr(d), _stream(stream)))
+
+
+def moe_router_topk(d: MoeDims, x, Wr, idx, w, logits, route_counts=None, stream=None):
+    _check("moe_router_topk", lib().moe_router_topk(
+        ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(idx), _ptr(w), _ptr(logits),
+        _ptr(route_counts), _stream(stream)))
+
+
+def moe_bucket(d: MoeDims, idx, cnt, off, uni, n_uni, perm, stream=None):
+    _check("moe_bucket", lib().moe_bucket(
+        ctypes.byref(d), idx.shape[0], _ptr(idx), _ptr(cnt), _ptr(off), _ptr(uni), _ptr(n_uni),
+        _ptr(perm), _stream(stream)))
+
+
+def moe_layer_forward(d: MoeDims, x, Wr, table, out, ws, route_counts=None,
+                      path: int = MOE_PATH_AUTO, stream=None):
+    _check("moe_layer_forward", lib().moe_layer_forward(
+        ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
+
+
+def moe_layer_forward_host(d: MoeDims, x_host, Wr, table, out_host, ws, route_counts=None,
+                           path: int = MOE_PATH_AUTO, stream=None):
+    _check("moe_layer_forward_host", lib().moe_layer_forward_host(
+        ctypes.byref(d), x_host.shape[0], _ptr(x_host), _ptr(Wr), _ptr(table), _ptr(out_host),
+        _ptr(ws), ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
+
+
+def moe_workspace_view(d: MoeDims, T: int, ws: torch.Tensor) -> MoeWsView:
+    v = MoeWsView()
+    _check("moe_workspace_view", lib().moe_workspace_view(ctypes.byref(d), T, _ptr(ws), ctypes.byref(v)))
+    return v
+
+
+# ----------------------------------------------------------------- helpers
+def alloc_workspace(d: MoeDims, T_max: int, device="cuda") -> torch.Tensor:
+    """Device workspace for batches of up to T_max tokens (256-byte aligned)."""
+    n = moe_workspace_bytes(d, T_max)
+    if n == 0:
+        raise MoeError("moe_workspace_bytes", -2)
+    ws = torch.empty(n + 256, dtype=torch.uint8, device=device)
+    off = (-ws.data_ptr()) % 256
+    return ws[off:off + n]
+
+
+def expert_table(blobs: torch.Tensor | list) -> torch.Tensor:
+    """Device array of blob pointers (int64) from a [E+1][bytes] uint8 tensor
+    or a list of 1-D uint8 device tensors (entry E = shared expert)."""
+    if isinstance(blobs, torch.Tensor):
+        dev = blobs.device
+        ptrs = [blobs[i].data_ptr() for i in range(blobs.shape[0])]
+    else:
+        dev = blobs[0].device
+        ptrs = [b.data_ptr() for b in blobs]
+    return torch.tensor(ptrs, dtype=torch.int64, device=dev)
+
+
+def ws_slice(ws: torch.Tensor, ptr: int, shape, dtype) -> torch.Tensor:
+    """The workspace region at device address `ptr` (from moe_workspace_view)
+    as a tensor view of `shape` / `dtype`."""
+    n = 1
+    for s_ in shape:
+        n *= s_
+    itemsize = torch.empty((), dtype=dtype).element_size()
+    off = ptr - ws.data_ptr()
+    assert 0 <= off and off + n * itemsize <= ws.numel(), "pointer outside the workspace"
+    return ws[off:off + n * itemsize].view(dtype).view(*shape)

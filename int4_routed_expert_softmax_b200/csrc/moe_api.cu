@@ -1,0 +1,364 @@
+// moe_api.cu -- the C ABI of libmoe (declared in include/moe.h): argument
+// checks, workspace carving and the launch sequence of the layer.
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "moe_internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxDevices = 64;
+int g_sms[kMaxDevices] = {0};
+std::mutex g_mu;
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    g_sms[dev] = n;
+  }
+  return g_sms[dev];
+}
+
+bool dims_shape_ok(const moe_dims &d) {
+  return d.H > 0 && d.I > 0 && d.H % 128 == 0 && d.I % 128 == 0 && d.H <= 8192 && d.I <= 4096 &&
+         d.E >= 1 && d.E <= MOE_MAX_E && d.k >= 1 && d.k <= d.E && d.k <= kMaxK;
+}
+
+// ---- optional per-kernel events (moe_profile_enable)
+bool g_prof = false;
+cudaEvent_t g_ev[kMaxDevices][4] = {};
+int g_ev_dev = -1;
+
+void prof_record(int i, cudaStream_t s) {
+  if (!g_prof) return;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
+  if (g_ev[dev][i] == nullptr && cudaEventCreate(&g_ev[dev][i]) != cudaSuccess) return;
+  cudaEventRecord(g_ev[dev][i], s);
+  g_ev_dev = dev;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return MOE_OK;
+  std::fprintf(stderr, "libmoe: CUDA error %d (%s)\n", (int)e, cudaGetErrorString(e));
+  return MOE_ERR_CUDA;
+}
+
+template <typename T>
+T *at(void *ws, size_t off) {
+  return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
+}
+
+// Decode path on Tc <= kDecodeTMax tokens.  Per-token arrays (xq, xd, logits,
+// idx, w) are at token offset t0 of the layout L; pair arrays are chunk-local.
+int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
+                 const float *Wr, const void *const *table, float *out, void *ws,
+                 int32_t *counts, cudaStream_t s) {
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  int32_t *status = at<int32_t>(ws, L.status);
+  const size_t H = d.H, E = d.E, K = d.k;
+
+  RouteArgs ra{};
+  ra.H = d.H;
+  ra.E = d.E;
+  ra.k = d.k;
+  ra.T = Tc;
+  ra.x = x + (size_t)t0 * H;
+  ra.Wr = Wr;
+  ra.xq = at<int8_t>(ws, L.xq) + (size_t)t0 * H;
+  ra.xd = at<float>(ws, L.xd) + (size_t)t0 * (H / 32);
+  ra.logits = at<float>(ws, L.logits) + (size_t)t0 * E;
+  ra.idx = at<int32_t>(ws, L.idx) + (size_t)t0 * K;
+  ra.w = at<float>(ws, L.w) + (size_t)t0 * K;
+  ra.route_counts = counts;
+  ra.cnt = at<int32_t>(ws, L.cnt);
+  ra.off = at<int32_t>(ws, L.off);
+  ra.uni = at<int32_t>(ws, L.uni);
+  ra.n_uni = at<int32_t>(ws, L.n_uni);
+  ra.perm = at<int32_t>(ws, L.perm);
+  ra.pos = at<int32_t>(ws, L.pos);
+  ra.pair_tok = at<int32_t>(ws, L.pair_tok);
+  ra.done = at<unsigned int>(ws, L.ctrl);
+  ra.status = status;
+  ra.do_quant = 1;
+  ra.do_bucket = 1;
+  ra.epc = 2;
+  ra.tt = Tc < 2 ? Tc : 2;
+  prof_record(0, s);
+  cudaError_t err = launch_route_decode(ra, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(1, s);
+
+  GateUpArgs ga{};
+  ga.H = d.H;
+  ga.I = d.I;
+  ga.E = d.E;
+  ga.k = d.k;
+  ga.T = Tc;
+  ga.table = table;
+  ga.uni = ra.uni;
+  ga.n_uni = ra.n_uni;
+  ga.off = ra.off;
+  ga.pair_tok = ra.pair_tok;
+  ga.xq = ra.xq;
+  ga.xd = ra.xd;
+  ga.hq = at<int8_t>(ws, L.hq);
+  ga.hqs = at<int32_t>(ws, L.hqs);
+  ga.hd = at<float>(ws, L.hd);
+  ga.status = status;
+  ga.nstage = gateup_max_stages(d.H, Tc);
+  ga.use_pdl = 0;
+  if (ga.nstage < 2) return MOE_ERR_SHAPE;
+  err = launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.nstage), s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(2, s);
+
+  DownArgs da{};
+  da.H = d.H;
+  da.I = d.I;
+  da.E = d.E;
+  da.k = d.k;
+  da.T = Tc;
+  da.table = table;
+  da.uni = ra.uni;
+  da.n_uni = ra.n_uni;
+  da.off = ra.off;
+  da.pos = ra.pos;
+  da.w = ra.w;
+  da.hq = ga.hq;
+  da.hqs = ga.hqs;
+  da.hd = ga.hd;
+  da.out = out + (size_t)t0 * H;
+  da.status = status;
+  const int sb = d.I / 32;  // scale bytes per down row
+  int g = 16;
+  {
+    int a = sb, b = 16;
+    while (b) {
+      const int t = a % b;
+      a = b;
+      b = t;
+    }
+    g = a;
+  }
+  da.rg = 16 / g;
+  const int nrg = d.H / da.rg;
+  const int grid = nrg < sms ? nrg : sms;
+  da.rows_max = ((nrg + grid - 1) / grid) * da.rg;
+  // rows per stage: the CTA's whole range if three stages fit, else halves
+  da.rs = da.rows_max;
+  while (da.rs > da.rg && down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs) < 3)
+    da.rs = ((da.rs / 2 + da.rg - 1) / da.rg) * da.rg;
+  da.nstage = down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs);
+  da.use_pdl = 0;
+  if (da.nstage < 2) return MOE_ERR_SHAPE;
+  err = launch_down_decode(
+      da, grid, down_smem_bytes(d.H, d.I, d.k, Tc, da.rows_max, da.rs, da.nstage), s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(3, s);
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_status_string(int status) {
+  switch (status) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_BAD_ARG: return "bad argument";
+    case MOE_ERR_SHAPE: return "unsupported shape";
+    case MOE_ERR_CUDA: return "CUDA runtime error";
+    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MOE_ERR_CACHE_FULL: return "expert cache full";
+    case MOE_ERR_NOT_RESIDENT: return "expert not resident";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE: return "device-side check failed";
+    case MOE_ERR_ALLOC: return "allocation failed";
+    default: return "unknown status";
+  }
+}
+
+int moe_check_dims(const moe_dims *dims) {
+  if (dims == nullptr) return MOE_ERR_BAD_ARG;
+  return dims_shape_ok(*dims) ? MOE_OK : MOE_ERR_SHAPE;
+}
+
+size_t moe_expert_bytes(const moe_dims *dims) {
+  if (moe_check_dims(dims) != MOE_OK) return 0;
+  return expert_bytes(dims->H, dims->I);
+}
+
+size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max) {
+  if (moe_check_dims(dims) != MOE_OK || T_max < 0) return 0;
+  return ws_layout(*dims, T_max).total;
+}
+
+int moe_workspace_view(const moe_dims *dims, int32_t T, void *ws, moe_ws_view *v) {
+  if (moe_check_dims(dims) != MOE_OK) return MOE_ERR_SHAPE;
+  if (ws == nullptr || v == nullptr || T < 0) return MOE_ERR_BAD_ARG;
+  const int Tl = T > kDecodeTMax ? T : T;
+  const WsLayout L = ws_layout(*dims, Tl);
+  v->status = at<int32_t>(ws, L.status);
+  v->xq = at<int8_t>(ws, L.xq);
+  v->xd = at<float>(ws, L.xd);
+  v->logits = at<float>(ws, L.logits);
+  v->idx = at<int32_t>(ws, L.idx);
+  v->w = at<float>(ws, L.w);
+  v->cnt = at<int32_t>(ws, L.cnt);
+  v->off = at<int32_t>(ws, L.off);
+  v->uni = at<int32_t>(ws, L.uni);
+  v->n_uni = at<int32_t>(ws, L.n_uni);
+  v->perm = at<int32_t>(ws, L.perm);
+  v->pos = at<int32_t>(ws, L.pos);
+  v->pair_tok = at<int32_t>(ws, L.pair_tok);
+  v->hq = at<int8_t>(ws, L.hq);
+  v->hd = at<float>(ws, L.hd);
+  v->T_max = T;
+  return MOE_OK;
+}
+
+int moe_device_sms(void) {
+  const int n = device_sms();
+  return n > 0 ? n : MOE_ERR_CUDA;
+}
+
+int moe_profile_enable(int on) {
+  g_prof = on != 0;
+  return MOE_OK;
+}
+
+int moe_profile_last(float *ms, int n) {
+  if (ms == nullptr || n < 0) return MOE_ERR_BAD_ARG;
+  const int dev = g_ev_dev;
+  if (dev < 0) return 0;
+  for (int i = 0; i < 4; ++i)
+    if (g_ev[dev][i] == nullptr) return 0;
+  cudaError_t e = cudaEventSynchronize(g_ev[dev][3]);
+  if (e != cudaSuccess) return cuda_status(e);
+  int w = 0;
+  for (int i = 0; i < 3 && w < n; ++i) {
+    float t = 0.0f;
+    e = cudaEventElapsedTime(&t, g_ev[dev][i], g_ev[dev][i + 1]);
+    if (e != cudaSuccess) return cuda_status(e);
+    ms[w++] = t;
+  }
+  return w;
+}
+
+int moe_quant_q8_0(const float *x, int64_t rows, int32_t cols, int8_t *q, float *d, void *stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_SHAPE;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !d) return MOE_ERR_BAD_ARG;
+  QuantArgs a{x, q, d, rows * (int64_t)(cols / 32)};
+  return cuda_status(launch_quant(a, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_router_topk(const moe_dims *dims, int32_t T, const float *x, const float *Wr, int32_t *idx,
+                    float *w, float *logits, int32_t *route_counts_opt, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !idx || !w || !logits) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16)) return MOE_ERR_BAD_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  RouteArgs ra{};
+  ra.H = dims->H;
+  ra.E = dims->E;
+  ra.k = dims->k;
+  ra.T = T;
+  ra.x = x;
+  ra.Wr = Wr;
+  ra.logits = logits;
+  ra.epc = 2;
+  ra.tt = T < 2 ? T : 2;
+  ra.done = nullptr;
+  ra.status = nullptr;
+  cudaError_t err = launch_route_decode(ra, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  return cuda_status(launch_topk(logits, T, dims->E, dims->k, idx, w, route_counts_opt, s));
+}
+
+int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt, int32_t *off,
+               int32_t *uni, int32_t *n_uni, int32_t *perm, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0) return MOE_ERR_BAD_ARG;
+  if (!cnt || !off || !uni || !n_uni || (T > 0 && (!idx || !perm))) return MOE_ERR_BAD_ARG;
+  BucketArgs a{};
+  a.E = dims->E;
+  a.k = dims->k;
+  a.T = T;
+  a.idx = idx;
+  a.cnt = cnt;
+  a.off = off;
+  a.uni = uni;
+  a.n_uni = n_uni;
+  a.perm = perm;
+  a.pos = nullptr;
+  a.pair_tok = nullptr;
+  return cuda_status(launch_bucket(a, static_cast<cudaStream_t>(stream)));
+}
+
+int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                      const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                      int32_t *route_counts_opt, int32_t path, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !expert_table || !out || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(out, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // status word and the router's arrival counter start at zero on every call
+  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
+    const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
+    rc = decode_chunk(*dims, t0, Tc, T <= kDecodeTMax ? L : ws_layout(*dims, T), x, Wr,
+                      expert_table, out, ws, route_counts_opt, s);
+    if (rc != MOE_OK) return rc;
+  }
+  return MOE_OK;
+}
+
+int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host, const float *Wr,
+                           const void *const *expert_table, float *out_host, void *ws,
+                           size_t ws_bytes, int32_t *route_counts_opt, int32_t path, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x_host || !out_host || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *xd = at<float>(ws, L.xin);
+  float *yd = at<float>(ws, L.yout);
+  const size_t bytes = (size_t)T * dims->H * sizeof(float);
+  cudaError_t err = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  rc = moe_layer_forward(dims, T, xd, Wr, expert_table, yd, ws, ws_bytes, route_counts_opt, path,
+                         stream);
+  if (rc != MOE_OK) return rc;
+  return cuda_status(cudaMemcpyAsync(out_host, yd, bytes, cudaMemcpyDeviceToHost, s));
+}
+
+}  // extern "C"

@@ -1,0 +1,154 @@
+// moe_internal.h -- definitions shared by the libmoe host code and kernels:
+// workspace layout, kernel argument blocks, launcher declarations.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+constexpr int kMaxK = 32;                              // kernels keep <= 32 slots per token
+constexpr int kDecodeTMax = MOE_DECODE_T_MAX;
+constexpr int kMaxSmem = 227 * 1024 - 1024;            // dynamic shared memory per CTA (sm_100 opt-in limit, minus static)
+
+// Device-side error details (status[1]) -- which wait or check failed.
+enum Detail : int32_t {
+  kDetRouteBar = 1,
+  kDetGuFull = 10,
+  kDetGuEmpty = 11,
+  kDetGuDrain = 12,
+  kDetGuAlign = 13,
+  kDetDnFull = 20,
+  kDetDnEmpty = 21,
+  kDetDnDrain = 22,
+  kDetDnAlign = 23,
+  kDetPfAlign = 30,
+  kDetPfWait = 31,
+};
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline size_t matrix_bytes(int N, int K) {
+  return (size_t)N * (size_t)(K / 2) + (size_t)N * (size_t)(K / 64) * 2;
+}
+inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matrix_bytes(H, I); }
+
+// Byte offsets of the workspace segments for batches of up to T tokens.
+struct WsLayout {
+  size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
+      pair_tok, hq, hqs, hd, total;
+};
+
+inline WsLayout ws_layout(const moe_dims &d, int T) {
+  WsLayout L{};
+  const size_t P = (size_t)T * (size_t)(d.k + 1);
+  size_t o = 0;
+  auto seg = [&](size_t bytes) {
+    size_t at = o;
+    o = align_up(o + (bytes ? bytes : 1), 256);
+    return at;
+  };
+  L.status = seg(16);
+  L.ctrl = seg(64);
+  L.xin = seg((size_t)T * d.H * 4);
+  L.yout = seg((size_t)T * d.H * 4);
+  L.xq = seg((size_t)T * d.H);
+  L.xd = seg((size_t)T * (d.H / 32) * 4);
+  L.logits = seg((size_t)T * d.E * 4);
+  L.idx = seg((size_t)T * d.k * 4);
+  L.w = seg((size_t)T * d.k * 4);
+  L.cnt = seg((size_t)d.E * 4);
+  L.off = seg((size_t)(d.E + 1) * 4);
+  L.uni = seg((size_t)(d.E + 1) * 4);
+  L.n_uni = seg(16);
+  L.perm = seg((size_t)T * d.k * 4);
+  L.pos = seg((size_t)T * d.k * 4);
+  L.pair_tok = seg(P * 4);
+  L.hq = seg(P * d.I);
+  L.hqs = seg(P * (d.I / 32) * 4);
+  L.hd = seg(P * (d.I / 32) * 4);
+  L.total = o;
+  return L;
+}
+
+struct QuantArgs {
+  const float *x;
+  int8_t *q;
+  float *d;
+  int64_t nblk;
+};
+
+struct RouteArgs {
+  int H, E, k, T;
+  const float *x, *Wr;
+  int8_t *xq;
+  float *xd, *logits, *w;
+  int32_t *idx, *route_counts;
+  int32_t *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok;
+  unsigned int *done;
+  int32_t *status;
+  int do_quant;
+  int do_bucket;
+  int epc;  // experts per CTA
+  int tt;   // tokens per x tile
+};
+
+struct BucketArgs {
+  int E, k, T;
+  const int32_t *idx;
+  int32_t *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok;
+};
+
+struct GateUpArgs {
+  int H, I, E, k, T;
+  const void *const *table;
+  const int32_t *uni, *n_uni, *off, *pair_tok;
+  const int8_t *xq;
+  const float *xd;
+  int8_t *hq;
+  int32_t *hqs;
+  float *hd;
+  int32_t *status;
+  int nstage;
+  int use_pdl;
+};
+
+struct DownArgs {
+  int H, I, E, k, T;
+  const void *const *table;
+  const int32_t *uni, *n_uni, *off, *pos;
+  const float *w;
+  const int8_t *hq;
+  const int32_t *hqs;
+  const float *hd;
+  float *out;
+  int32_t *status;
+  int nstage;
+  int rg;        // row granularity (scale bytes of a row group are a multiple of 16)
+  int rows_max;  // most output rows any CTA owns
+  int rs;        // rows per stage (a multiple of rg)
+  int use_pdl;
+};
+
+// Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
+cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s);
+cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s);
+cudaError_t launch_bucket(const BucketArgs &a, cudaStream_t s);
+cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,
+                        int32_t *counts, cudaStream_t s);
+cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s);
+cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s);
+
+// Shared-memory plans (host side, moe_kernels.cu).
+size_t route_smem_bytes(int H, int epc, int tt);
+size_t gateup_smem_bytes(int H, int T, int nstage);
+size_t down_smem_bytes(int H, int I, int k, int T, int rows_max, int rs, int nstage);
+int gateup_max_stages(int H, int T);
+int down_max_stages(int H, int I, int k, int T, int rows_max, int rs);
+
+}  // namespace moe

@@ -89,29 +89,33 @@ def sub_seed(seed: int, layer: int, role: int) -> int:
     return (seed * 1_000_003 + layer * 10_007 + role * 101) & 0x7FFF_FFFF
 
 
-def fill_blobs(out: torch.Tensor, H: int, I: int, seed: int) -> torch.Tensor:
-    """Fill a uint8 tensor [n][expert_bytes] with random experts in place."""
-    n, nb = out.shape
-    assert nb == expert_bytes(H, I) and out.dtype == torch.uint8
+def fill_blob(out: torch.Tensor, H: int, I: int, seed: int) -> torch.Tensor:
+    """Fill one expert blob (uint8 [expert_bytes]) in place from its own seed."""
+    assert out.numel() == expert_bytes(H, I) and out.dtype == torch.uint8
     dev = out.device
     g = _gen(seed, dev)
     out.random_(0, 256, generator=g)
     mg = matrix_bytes(I, H)
-    regions = [(0, I, H), (mg, I, H), (2 * mg, H, I)]
-    for base, N, K in regions:
+    for base, N, K in ((0, I, H), (mg, I, H), (2 * mg, H, I)):
         s0 = base + N * (K // 2)
         cnt = N * (K // GROUP)
-        for i0 in range(0, n, 16):
-            i1 = min(n, i0 + 16)
-            z = torch.randn((i1 - i0, cnt), generator=g, device=dev, dtype=torch.float32)
-            s = torch.exp(z * 0.3 + math.log(0.02)).to(torch.float16)
-            out[i0:i1, s0:s0 + 2 * cnt] = s.view(torch.uint8).view(i1 - i0, 2 * cnt)
+        z = torch.randn(cnt, generator=g, device=dev, dtype=torch.float32)
+        s = torch.exp(z * 0.3 + math.log(0.02)).to(torch.float16)
+        out[s0:s0 + 2 * cnt] = s.view(torch.uint8)
     return out
 
 
-def make_blobs(H: int, I: int, n: int, seed: int, device="cpu") -> torch.Tensor:
-    out = torch.empty((n, expert_bytes(H, I)), dtype=torch.uint8, device=device)
-    return fill_blobs(out, H, I, seed)
+def blob_seed(seed: int, e: int) -> int:
+    return (seed * 7919 + e * 104_729 + 13) & 0x7FFF_FFFF
+
+
+def make_blobs(H: int, I: int, n: int, seed: int, device="cpu", only=None) -> torch.Tensor:
+    """Expert blobs [n][expert_bytes]; blob e is drawn from its own seed, so any
+    subset can be regenerated alone.  `only`: fill just these rows (others 0)."""
+    out = torch.zeros((n, expert_bytes(H, I)), dtype=torch.uint8, device=device)
+    for e in (range(n) if only is None else only):
+        fill_blob(out[e], H, I, blob_seed(seed, e))
+    return out
 
 
 def zipf_bias(E: int, H: int, s: float, seed: int) -> torch.Tensor:

@@ -1,0 +1,251 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Bit-exact: Q8_0 codes and scales, router logits, top-k indices and weights,
+bucket counts / offsets / union / permutation, the Q8_0 codes of SiLU(g)*u.
+Final outputs: within rel-L2 <= 1e-4 and max-abs <= 2e-3 * rms(ref) (the kernels
+follow the oracle's fixed order, so they are expected to match bit for bit as
+well; that is asserted separately)."""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs as mi
+import oracle as orc
+from tests._common import gpu_layer, hq_by_slot, oracle_layer_from_device, within_tolerance, ws_trace
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _moe():
+    import int4_routed_expert_softmax_b200 as moe
+    return moe
+
+
+# ----------------------------------------------------------------- Q8_0
+@pytest.mark.parametrize("rows,cols,scale", [(1, 256, 1.0), (7, 6144, 1.0), (33, 384, 1e-3),
+                                             (2, 128, 1e4), (1, 32, 0.0)])
+def test_quant_q8_0_bit_exact(rows, cols, scale):
+    moe = _moe()
+    x = mi.make_x(rows, cols, 11 + rows, DEV) * scale
+    x[0, :32] = 0.0                       # a zero block
+    if rows > 1:
+        x[1, 5] = 1e-30                   # tiny amax
+    q = torch.empty((rows, cols), dtype=torch.int8, device=DEV)
+    d = torch.empty((rows, cols // 32), dtype=torch.float32, device=DEV)
+    moe.moe_quant_q8_0(x, q, d)
+    torch.cuda.synchronize()
+    qo, do = orc.quant_q8_0(x.cpu().numpy())
+    assert np.array_equal(q.cpu().numpy(), qo)
+    assert np.array_equal(d.cpu().numpy().view(np.uint32), do.view(np.uint32))
+
+
+# ----------------------------------------------------------------- router
+@pytest.mark.parametrize("name,T", [("tiny", 4), ("decode", 1), ("decode", 16), ("decode", 37)])
+def test_router_topk_bit_exact(name, T):
+    moe = _moe()
+    w = mi.WORKLOADS[name]
+    x = mi.make_x(T, w.H, 5 + T, DEV)
+    Wr = mi.make_router(w.E, w.H, 6, DEV)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    idx = torch.empty((T, w.k), dtype=torch.int32, device=DEV)
+    wt = torch.empty((T, w.k), dtype=torch.float32, device=DEV)
+    lg = torch.empty((T, w.E), dtype=torch.float32, device=DEV)
+    cnt = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    moe.moe_router_topk(d, x, Wr, idx, wt, lg, cnt)
+    torch.cuda.synchronize()
+    lo = orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy())
+    io, wo = orc.topk_softmax(lo, w.k)
+    assert np.array_equal(lg.cpu().numpy().view(np.uint32), lo.view(np.uint32))
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert np.array_equal(wt.cpu().numpy().view(np.uint32), wo.view(np.uint32))
+    assert np.array_equal(cnt.cpu().numpy(), np.bincount(io.reshape(-1), minlength=w.E))
+
+
+def test_router_ties_lower_index_first():
+    moe = _moe()
+    H, E, k, T = 256, 16, 4, 3
+    Wr = mi.make_router(E, H, 9, DEV)
+    Wr[5] = Wr[2]
+    Wr[9] = Wr[2]            # experts 2, 5, 9 always tie
+    Wr[12] = Wr[3]
+    x = mi.make_x(T, H, 10, DEV)
+    x[2] = 0.0               # every logit is zero: ties everywhere
+    d = moe.dims(H, 128, E, k)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    wt = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    lg = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    moe.moe_router_topk(d, x, Wr, idx, wt, lg)
+    torch.cuda.synchronize()
+    io, wo = orc.topk_softmax(orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy()), k)
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert list(io[2]) == [0, 1, 2, 3]
+    assert np.array_equal(wt.cpu().numpy(), wo)
+
+
+# ----------------------------------------------------------------- bucket
+@pytest.mark.parametrize("T,k,E", [(1, 8, 256), (4, 2, 16), (16, 8, 256), (300, 8, 256),
+                                   (2048, 8, 256), (5, 3, 3), (64, 1, 1)])
+def test_bucket_bit_exact(T, k, E):
+    moe = _moe()
+    rng = np.random.default_rng(T * 31 + E)
+    if T >= 300:   # skewed popularity like the prefill workload
+        p = 1.0 / np.arange(1, E + 1) ** 1.1
+        p /= p.sum()
+        io = np.array([rng.choice(E, size=k, replace=False, p=p) for _ in range(T)], np.int32)
+    else:
+        io = np.array([rng.permutation(E)[:k] for _ in range(T)], np.int32).reshape(T, k)
+    d = moe.dims(128, 128, E, k)
+    idx = torch.from_numpy(io).to(DEV)
+    cnt = torch.empty(E, dtype=torch.int32, device=DEV)
+    off = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    uni = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    nu = torch.empty(1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(max(T * k, 1), dtype=torch.int32, device=DEV)
+    moe.moe_bucket(d, idx, cnt, off, uni, nu, perm)
+    torch.cuda.synchronize()
+    c, o, u, n, pm = orc.bucket(io, E)
+    assert int(nu.item()) == n
+    assert np.array_equal(cnt.cpu().numpy(), c)
+    assert np.array_equal(off.cpu().numpy(), o)
+    assert np.array_equal(uni.cpu().numpy()[:n], u)
+    assert np.array_equal(perm.cpu().numpy()[:T * k], pm)
+
+
+# ----------------------------------------------------------------- whole layer
+def _check_layer(w, x, Wr, blobs, path=0, exact=True):
+    T = x.shape[0]
+    out, ws, d = gpu_layer(w, x, Wr, blobs, path=path)
+    ref, tr = oracle_layer_from_device(x, Wr, blobs, w.H, w.I, w.E, w.k)
+    g = ws_trace(ws, d, min(T, 16)) if T <= 16 else None
+    got = out.cpu().numpy()
+    ok, rel, mrel = within_tolerance(got, ref)
+    assert ok, (rel, mrel)
+    if g is not None:
+        assert g["status"][0] == 0, g["status"]
+        assert np.array_equal(g["xq"], tr["xq"])
+        assert np.array_equal(g["xd"].view(np.uint32), tr["xd"].view(np.uint32))
+        assert np.array_equal(g["logits"].view(np.uint32), tr["logits"].view(np.uint32))
+        assert np.array_equal(g["idx"], tr["idx"])
+        assert np.array_equal(g["w"].view(np.uint32), tr["w"].view(np.uint32))
+        assert np.array_equal(g["cnt"], tr["cnt"])
+        assert np.array_equal(g["off"], tr["off"])
+        assert g["n_uni"] == tr["n_uni"] and np.array_equal(g["uni"], tr["uni"])
+        assert np.array_equal(g["perm"], tr["perm"])
+        hq, hd = hq_by_slot(g, T, w.k)
+        assert np.array_equal(hq, tr["hq"])
+        assert np.array_equal(hd.view(np.uint32), tr["hd"].view(np.uint32))
+    if exact:
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+    return out, ref
+
+
+def test_layer_tiny():
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    _check_layer(w, x, Wr, blobs)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_layer_decode_glm_T1(seed):
+    w = mi.shrink(mi.WORKLOADS["decode"], seed=100 + seed)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    _check_layer(w, x, Wr, blobs)
+
+
+@pytest.mark.parametrize("T", [4, 16])
+def test_layer_stacked_batches(T):
+    w = mi.WORKLOADS["stacked"]
+    x, Wr, blobs = mi.make_layer(w, 3, DEV, T=T)
+    _check_layer(w, x, Wr, blobs)
+
+
+@pytest.mark.parametrize("H,I,E,k,T", [
+    (384, 384, 5, 5, 3),      # k = E, ragged group count (G = 6 per row)
+    (128, 128, 1, 1, 2),      # a single expert
+    (256, 128, 16, 2, 1),
+    (1024, 256, 64, 8, 16),
+    (8192, 4096, 8, 2, 2),    # widest accepted shape
+])
+def test_layer_shapes(H, I, E, k, T):
+    w = mi.Workload("shape", H=H, I=I, E=E, k=k, T=T, seed=H + I + E + k + T)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    _check_layer(w, x, Wr, blobs)
+
+
+def test_layer_zero_rows_and_repeat():
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    x[1] = 0.0                        # all-zero hidden state: every block has d = 0
+    out1, _ = _check_layer(w, x, Wr, blobs)
+    out2, _, _ = gpu_layer(w, x, Wr, blobs)
+    assert torch.equal(out1, out2)    # bitwise reproducible
+
+
+def test_layer_T0_is_noop():
+    moe = _moe()
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    ws = moe.alloc_workspace(d, 1)
+    out = torch.empty((0, w.H), device=DEV)
+    moe.moe_layer_forward(d, x[:0], Wr, moe.expert_table(blobs), out, ws)
+
+
+def test_layer_chunked_decode_path_T40():
+    """T > 16 on the decode path runs in chunks of 16 tokens."""
+    w = mi.shrink(mi.WORKLOADS["decode"], seed=77)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV, T=40)
+    out, ws, d = gpu_layer(w, x, Wr, blobs, path=1)
+    toks = [0, 15, 16, 31, 39]
+    ref = oracle_layer_from_device(x, Wr, blobs, w.H, w.I, w.E, w.k, tokens=toks)
+    got = out.cpu().numpy()[toks]
+    ok, rel, mrel = within_tolerance(got, ref)
+    assert ok, (rel, mrel)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_layer_forward_host_matches_device():
+    moe = _moe()
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    out_dev, ws, d = gpu_layer(w, x, Wr, blobs)
+    xh = x.cpu().pin_memory()
+    oh = torch.empty((x.shape[0], w.H), dtype=torch.float32).pin_memory()
+    moe.moe_layer_forward_host(d, xh, Wr, moe.expert_table(blobs), oh, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out_dev.cpu())
+
+
+def test_route_counts_accumulate():
+    moe = _moe()
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    ws = moe.alloc_workspace(d, x.shape[0])
+    cnt = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    out = torch.empty((x.shape[0], w.H), device=DEV)
+    for _ in range(3):
+        moe.moe_layer_forward(d, x, Wr, moe.expert_table(blobs), out, ws, route_counts=cnt)
+    torch.cuda.synchronize()
+    io, _ = orc.topk_softmax(orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy()), w.k)
+    assert np.array_equal(cnt.cpu().numpy(), 3 * np.bincount(io.reshape(-1), minlength=w.E))
+
+
+def test_misaligned_blob_reports_device_error():
+    """A 16-byte-misaligned expert pointer is refused by the kernels' own
+    check (status word), never dereferenced by a bulk copy."""
+    moe = _moe()
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    raw = torch.empty(blobs.numel() + 64, dtype=torch.uint8, device=DEV)
+    base = raw[8:8 + blobs.numel()].view(w.E + 1, -1)
+    base.copy_(blobs)
+    ws = moe.alloc_workspace(d, x.shape[0])
+    out = torch.zeros((x.shape[0], w.H), device=DEV)
+    moe.moe_layer_forward(d, x, Wr, moe.expert_table(base), out, ws)
+    torch.cuda.synchronize()
+    st = moe.ws_slice(ws, moe.moe_workspace_view(d, x.shape[0], ws).status, (4,), torch.int32).cpu()
+    assert int(st[0]) == -8   # MOE_ERR_DEVICE
