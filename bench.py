@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="routed experts per layer (profiling: a small pool, same per-step work)")
     return ap.parse_args()
 
 
@@ -195,6 +197,8 @@ def run_native(args, ws_n, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = mi.WORKLOADS[args.workload]
+    if args.experts:
+        w = mi.shrink(w, E=args.experts)
     seed = w.seed + 1000 * rank
     wl = mi.shrink(w, seed=seed)
     T = w.T

@@ -152,6 +152,116 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
                            void *ws, size_t ws_bytes, int32_t *route_counts_opt, int32_t path,
                            void *stream);
 
+/* The layer in two halves, for callers that must place the experts between
+ * routing and the FFN (the tiered cache below):
+ *   moe_layer_route:   Q8_0 of x, router + top-k + softmax, batch union into ws
+ *                      (T <= MOE_DECODE_T_MAX);
+ *   moe_read_union:    copies the union of that call to host memory
+ *                      (synchronises `stream`): host_uni [E], *host_n;
+ *   moe_layer_experts: gate/up + SwiGLU + requant and down + combine for the
+ *                      routing held in ws; expert_table entries are read only
+ *                      for the union experts and the shared expert (E).
+ * moe_layer_route + moe_layer_experts == moe_layer_forward, bit for bit. */
+int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws,
+                    size_t ws_bytes, int32_t *route_counts_opt, void *stream);
+int moe_read_union(const moe_dims *dims, int32_t T, void *ws, int32_t *host_uni, int32_t *host_n,
+                   void *stream);
+int moe_layer_experts(const moe_dims *dims, int32_t T, const void *const *expert_table, float *out,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * HBM expert cache over host memory: the VRAM tier above host RAM
+ * ("三层 memory hierarchy", tantan.ink page, section 它的核心判断), with a
+ * per-layer LRU, pins learned from route counts and one-layer-ahead
+ * prefetch (section 几个关键工程动作; "colibri deep review", 权重 JIT row).
+ *
+ * The cache owns a pool of expert-sized slots in HBM (allocated once at
+ * create), split evenly between the layers; each layer keeps its own LRU
+ * order and pin set.  Copies host -> HBM are cudaMemcpyAsync of whole blobs
+ * (one blob = gate|up|down, one transfer) on the stream given to the call;
+ * a slot is never overwritten before the kernels that last read it are done
+ * (an event recorded by expert_cache_release).  Placement changes speed,
+ * never results: the tiered output is bitwise the resident output.
+ * host_blobs: [n_layers][E+1] host pointers (pinned memory for async copies;
+ * entry E of a layer = its shared expert), owned by the caller, alive until
+ * destroy.  backend MOE_CACHE_HOST runs the same policy with host memory as
+ * the "HBM" pool and memcpy copies (no GPU; for tests of the policy).
+ * ------------------------------------------------------------------------ */
+typedef struct moe_cache moe_cache;
+
+enum moe_cache_backend { MOE_CACHE_DEVICE = 0, MOE_CACHE_HOST = 1 };
+
+/* fault kinds for expert_cache_inject_fault (host side, never on the GPU) */
+enum moe_cache_fault {
+  MOE_FAULT_NONE = 0,
+  MOE_FAULT_COPY = 1,   /* the next `count` blob copies report an error */
+  MOE_FAULT_ALLOC = 2   /* the next create() pool allocation fails (global) */
+};
+
+typedef struct moe_cache_stats {
+  uint64_t hits;            /* requested experts already resident */
+  uint64_t misses;          /* requested experts copied on demand */
+  uint64_t prefetches;      /* blobs copied by expert_cache_prefetch */
+  uint64_t prefetch_hits;   /* requested experts resident thanks to a prefetch */
+  uint64_t evictions;
+  uint64_t bytes_h2d;       /* bytes copied host -> pool */
+  uint64_t copy_errors;
+  int32_t slots;            /* slots in the pool */
+  int32_t slots_per_layer;
+  int32_t pinned;           /* pinned experts, all layers */
+  int32_t resident;         /* resident experts, all layers */
+} moe_cache_stats;
+
+int expert_cache_create(const moe_dims *dims, int32_t n_layers, const void *const *host_blobs,
+                        size_t hbm_bytes, int32_t backend, moe_cache **out);
+void expert_cache_destroy(moe_cache *cache);
+/* Pin: make resident (copied on `stream` if needed) and never evict. */
+int expert_cache_pin(moe_cache *cache, int32_t layer, const int32_t *experts, int32_t n,
+                     void *stream);
+int expert_cache_unpin(moe_cache *cache, int32_t layer, const int32_t *experts, int32_t n);
+/* Evict (unpinned, resident) experts now; pinned ones are skipped. */
+int expert_cache_evict(moe_cache *cache, int32_t layer, const int32_t *experts, int32_t n);
+/* Start copies of the listed experts that are not resident on `side_stream`
+ * (one-layer-ahead prefetch); returns the number of copies started.  Never
+ * evicts pinned experts; gives up (returning what it started) when the
+ * layer has no evictable slot. */
+int expert_cache_prefetch(moe_cache *cache, int32_t layer, const int32_t *experts, int32_t n,
+                          void *side_stream);
+/* Make the listed experts (and the shared expert E) resident -- misses are
+ * copied on `copy_stream` -- and return in *d_table a device table of E+1
+ * blob pointers for the layer (NULL for experts not resident), valid until
+ * the next acquire of the same layer.  `compute_stream` is made to wait for
+ * every copy the listed experts depend on.  MOE_ERR_CACHE_FULL if the layer
+ * cannot hold them all. */
+int expert_cache_acquire(moe_cache *cache, int32_t layer, const int32_t *experts, int32_t n,
+                         void *copy_stream, void *compute_stream, const void **d_table);
+/* Record on `compute_stream` that the kernels reading the layer's last
+ * acquired experts have been enqueued (their slots may be reused after). */
+int expert_cache_release(moe_cache *cache, int32_t layer, void *compute_stream);
+/* Learned pins: unpin the layer, then pin its n_pin most routed experts by
+ * the host counts [E] (ties to the lower index). */
+int expert_cache_learn_pins(moe_cache *cache, int32_t layer, const int32_t *host_counts,
+                            int32_t n_pin, void *stream);
+int expert_cache_resident(const moe_cache *cache, int32_t layer, int32_t expert);
+int expert_cache_pinned(const moe_cache *cache, int32_t layer, int32_t expert);
+int expert_cache_stats(const moe_cache *cache, moe_cache_stats *stats);
+/* Host-side fault injection for failure tests (see enum moe_cache_fault);
+ * cache may be NULL for MOE_FAULT_ALLOC. */
+int expert_cache_inject_fault(moe_cache *cache, int32_t kind, int32_t count);
+
+/* One tiered decode layer (native runtime of the cache):
+ * route(x) -> read union -> acquire (misses copied on side_stream, compute
+ * waits) -> if Wr_next is given, route the same x with the next layer's
+ * router into ws_pred and prefetch that union for layer+1 on side_stream ->
+ * experts -> release.  Synchronises with the host once per call (the union
+ * read) and once more when predicting.  prefetch_out_opt (host, 2 ints):
+ * [0] copies started for layer+1, [1] predicted union size. */
+int moe_tiered_layer_forward(moe_cache *cache, int32_t layer, const moe_dims *dims, int32_t T,
+                             const float *x, const float *Wr, const float *Wr_next_opt, float *out,
+                             void *ws, size_t ws_bytes, void *ws_pred, size_t ws_pred_bytes,
+                             int32_t *route_counts_opt, void *compute_stream, void *side_stream,
+                             int32_t *prefetch_out_opt);
+
 /* Device pointers to the intermediates a moe_layer_forward call leaves in its
  * workspace (for tests and tools).  Pair positions: the T*k routed pairs in
  * bucket order (position off[e]+i for the i-th pair of expert e), then T

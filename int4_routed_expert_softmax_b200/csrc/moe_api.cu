@@ -57,38 +57,66 @@ T *at(void *ws, size_t off) {
   return reinterpret_cast<T *>(static_cast<unsigned char *>(ws) + off);
 }
 
-// Decode path on Tc <= kDecodeTMax tokens.  Per-token arrays (xq, xd, logits,
+// Routing half of the decode path on Tc <= kDecodeTMax tokens: Q8_0 of x,
+// logits, top-k + softmax, batch union.  Per-token arrays (xq, xd, logits,
 // idx, w) are at token offset t0 of the layout L; pair arrays are chunk-local.
-int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
-                 const float *Wr, const void *const *table, float *out, void *ws,
-                 int32_t *counts, cudaStream_t s) {
-  const int sms = device_sms();
-  if (sms <= 0) return MOE_ERR_CUDA;
-  int32_t *status = at<int32_t>(ws, L.status);
-  const size_t H = d.H, E = d.E, K = d.k;
+struct ChunkPtrs {
+  int8_t *xq;
+  float *xd, *logits, *w;
+  int32_t *idx, *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok, *hqs, *status;
+  int8_t *hq;
+  float *hd;
+  unsigned int *done;
+};
 
+ChunkPtrs chunk_ptrs(const moe_dims &d, int t0, const WsLayout &L, void *ws) {
+  const size_t H = d.H, E = d.E, K = d.k;
+  ChunkPtrs p{};
+  p.xq = at<int8_t>(ws, L.xq) + (size_t)t0 * H;
+  p.xd = at<float>(ws, L.xd) + (size_t)t0 * (H / 32);
+  p.logits = at<float>(ws, L.logits) + (size_t)t0 * E;
+  p.idx = at<int32_t>(ws, L.idx) + (size_t)t0 * K;
+  p.w = at<float>(ws, L.w) + (size_t)t0 * K;
+  p.cnt = at<int32_t>(ws, L.cnt);
+  p.off = at<int32_t>(ws, L.off);
+  p.uni = at<int32_t>(ws, L.uni);
+  p.n_uni = at<int32_t>(ws, L.n_uni);
+  p.perm = at<int32_t>(ws, L.perm);
+  p.pos = at<int32_t>(ws, L.pos);
+  p.pair_tok = at<int32_t>(ws, L.pair_tok);
+  p.hq = at<int8_t>(ws, L.hq);
+  p.hqs = at<int32_t>(ws, L.hqs);
+  p.hd = at<float>(ws, L.hd);
+  p.status = at<int32_t>(ws, L.status);
+  p.done = at<unsigned int>(ws, L.ctrl);
+  return p;
+}
+
+int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
+                const float *Wr, void *ws, int32_t *counts, cudaStream_t s) {
+  const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
   RouteArgs ra{};
   ra.H = d.H;
   ra.E = d.E;
   ra.k = d.k;
   ra.T = Tc;
-  ra.x = x + (size_t)t0 * H;
+  ra.x = x + (size_t)t0 * d.H;
   ra.Wr = Wr;
-  ra.xq = at<int8_t>(ws, L.xq) + (size_t)t0 * H;
-  ra.xd = at<float>(ws, L.xd) + (size_t)t0 * (H / 32);
-  ra.logits = at<float>(ws, L.logits) + (size_t)t0 * E;
-  ra.idx = at<int32_t>(ws, L.idx) + (size_t)t0 * K;
-  ra.w = at<float>(ws, L.w) + (size_t)t0 * K;
+  ra.xq = p.xq;
+  ra.xd = p.xd;
+  ra.logits = p.logits;
+  ra.idx = p.idx;
+  ra.w = p.w;
   ra.route_counts = counts;
-  ra.cnt = at<int32_t>(ws, L.cnt);
-  ra.off = at<int32_t>(ws, L.off);
-  ra.uni = at<int32_t>(ws, L.uni);
-  ra.n_uni = at<int32_t>(ws, L.n_uni);
-  ra.perm = at<int32_t>(ws, L.perm);
-  ra.pos = at<int32_t>(ws, L.pos);
-  ra.pair_tok = at<int32_t>(ws, L.pair_tok);
-  ra.done = at<unsigned int>(ws, L.ctrl);
-  ra.status = status;
+  ra.cnt = p.cnt;
+  ra.off = p.off;
+  ra.uni = p.uni;
+  ra.n_uni = p.n_uni;
+  ra.perm = p.perm;
+  ra.pos = p.pos;
+  ra.pair_tok = p.pair_tok;
+  ra.done = p.done;
+  ra.status = p.status;
   ra.do_quant = 1;
   ra.do_bucket = 1;
   ra.epc = 2;
@@ -97,7 +125,14 @@ int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const flo
   cudaError_t err = launch_route_decode(ra, s);
   if (err != cudaSuccess) return cuda_status(err);
   prof_record(1, s);
+  return MOE_OK;
+}
 
+int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const void *const *table,
+                  float *out, void *ws, cudaStream_t s) {
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
   GateUpArgs ga{};
   ga.H = d.H;
   ga.I = d.I;
@@ -105,20 +140,21 @@ int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const flo
   ga.k = d.k;
   ga.T = Tc;
   ga.table = table;
-  ga.uni = ra.uni;
-  ga.n_uni = ra.n_uni;
-  ga.off = ra.off;
-  ga.pair_tok = ra.pair_tok;
-  ga.xq = ra.xq;
-  ga.xd = ra.xd;
-  ga.hq = at<int8_t>(ws, L.hq);
-  ga.hqs = at<int32_t>(ws, L.hqs);
-  ga.hd = at<float>(ws, L.hd);
-  ga.status = status;
-  ga.nstage = gateup_max_stages(d.H, Tc);
+  ga.uni = p.uni;
+  ga.n_uni = p.n_uni;
+  ga.off = p.off;
+  ga.pair_tok = p.pair_tok;
+  ga.xq = p.xq;
+  ga.xd = p.xd;
+  ga.hq = p.hq;
+  ga.hqs = p.hqs;
+  ga.hd = p.hd;
+  ga.status = p.status;
+  gateup_plan(d.H, Tc, &ga.rpm, &ga.nstage);
   ga.use_pdl = 0;
   if (ga.nstage < 2) return MOE_ERR_SHAPE;
-  err = launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.nstage), s);
+  cudaError_t err =
+      launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.rpm, ga.nstage), s);
   if (err != cudaSuccess) return cuda_status(err);
   prof_record(2, s);
 
@@ -129,26 +165,22 @@ int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const flo
   da.k = d.k;
   da.T = Tc;
   da.table = table;
-  da.uni = ra.uni;
-  da.n_uni = ra.n_uni;
-  da.off = ra.off;
-  da.pos = ra.pos;
-  da.w = ra.w;
-  da.hq = ga.hq;
-  da.hqs = ga.hqs;
-  da.hd = ga.hd;
-  da.out = out + (size_t)t0 * H;
-  da.status = status;
-  const int sb = d.I / 32;  // scale bytes per down row
-  int g = 16;
-  {
-    int a = sb, b = 16;
-    while (b) {
-      const int t = a % b;
-      a = b;
-      b = t;
-    }
-    g = a;
+  da.uni = p.uni;
+  da.n_uni = p.n_uni;
+  da.off = p.off;
+  da.pos = p.pos;
+  da.w = p.w;
+  da.hq = p.hq;
+  da.hqs = p.hqs;
+  da.hd = p.hd;
+  da.out = out + (size_t)t0 * d.H;
+  da.status = p.status;
+  // row groups: the fp16 scales of rg rows span a multiple of 16 bytes
+  int g = d.I / 32, b = 16;
+  while (b) {
+    const int t = g % b;
+    g = b;
+    b = t;
   }
   da.rg = 16 / g;
   const int nrg = d.H / da.rg;
@@ -160,6 +192,7 @@ int decode_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const flo
     da.rs = ((da.rs / 2 + da.rg - 1) / da.rg) * da.rg;
   da.nstage = down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs);
   da.use_pdl = 0;
+  da.preload = down_preload(d.I, d.k, Tc);
   if (da.nstage < 2) return MOE_ERR_SHAPE;
   err = launch_down_decode(
       da, grid, down_smem_bytes(d.H, d.I, d.k, Tc, da.rows_max, da.rs, da.nstage), s);
@@ -331,11 +364,64 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   if (err != cudaSuccess) return cuda_status(err);
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
     const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
-    rc = decode_chunk(*dims, t0, Tc, T <= kDecodeTMax ? L : ws_layout(*dims, T), x, Wr,
-                      expert_table, out, ws, route_counts_opt, s);
+    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, s);
+    if (rc != MOE_OK) return rc;
+    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, s);
     if (rc != MOE_OK) return rc;
   }
   return MOE_OK;
+}
+
+int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws,
+                    size_t ws_bytes, int32_t *route_counts_opt, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || T > kDecodeTMax) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, s);
+}
+
+int moe_read_union(const moe_dims *dims, int32_t T, void *ws, int32_t *host_uni, int32_t *host_n,
+                   void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || !ws || !host_uni || !host_n) return MOE_ERR_BAD_ARG;
+  const WsLayout L = ws_layout(*dims, T);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t st[2] = {0, 0};
+  cudaError_t err = cudaMemcpyAsync(host_n, at<int32_t>(ws, L.n_uni), 4, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess)
+    err = cudaMemcpyAsync(host_uni, at<int32_t>(ws, L.uni), (size_t)dims->E * 4,
+                          cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess)
+    err = cudaMemcpyAsync(st, at<int32_t>(ws, L.status), 8, cudaMemcpyDeviceToHost, s);
+  if (err == cudaSuccess) err = cudaStreamSynchronize(s);
+  if (err != cudaSuccess) return cuda_status(err);
+  if (st[0] != 0) return st[0];
+  if (*host_n < 0 || *host_n > dims->E) return MOE_ERR_DEVICE;
+  return MOE_OK;
+}
+
+int moe_layer_experts(const moe_dims *dims, int32_t T, const void *const *expert_table, float *out,
+                      void *ws, size_t ws_bytes, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || T > kDecodeTMax) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!expert_table || !out || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(out, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  return experts_chunk(*dims, 0, T, L, expert_table, out, ws, static_cast<cudaStream_t>(stream));
 }
 
 int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host, const float *Wr,

@@ -1,0 +1,750 @@
+// moe_decode.cu -- decode (GEMV) expert kernels of the routed-expert MoE layer.
+//
+//   k_gateup_decode: h = SiLU(W_gate x) * (W_up x) for every (union expert,
+//                    token) pair, requantised to Q8_0 per 32 rows of I.
+//   k_down_decode:   y = W_down Q8_0(h) per pair, then the combine
+//                    out[t] = y_shared, out = fmaf(w_s, y_s, out) in slot order.
+//
+// int4 gs64 weights (colibri, tantan.ink, 我看到的几个坑) against Q8_0-style int8
+// activations (Colibri, alphamatch.ai, 優化整數核心); the expert union of the
+// batch is read once per call (tantan.ink, 几个关键工程动作, Batch union).
+//
+// B200 design.  Both kernels are persistent, one CTA of 8 consumer warps +
+// 1 producer warp per SM.  The producer streams weight rows through a ring of
+// shared-memory stages with TMA bulk copies (cp.async.bulk, completion counted
+// on an mbarrier per stage, L2 evict-first), so the bytes in flight per SM
+// (3-4 stages of 45-52 KB) cover the HBM latency.  Consumers copy a stage's
+// rows to registers, release the stage at once, then unpack nibbles with one
+// LOP3 per word (low nibbles masked as values 0..15, high nibbles masked in
+// place as 16x their value) and run dp4a (unsigned x signed bytes) per
+// 32-block; the offset-binary bias and the 16x are folded into the integer
+// accumulator's start value, so each block sum is exact.
+//
+// Fixed order of the fp32 part (the layer's definition, shared with any CPU
+// restatement): per 64-group a = S0*d0, b = fma(S1, d1, a), chunk acc =
+// fma(s_g, b, acc); lane c owns the chunk of CSZ consecutive groups; the 32
+// chunk sums are added left to right (one lane per row after a transpose in
+// shared memory).  The h codes that feed the down projection are therefore
+// identical to the oracle's bit for bit.
+#include "moe_device.cuh"
+
+namespace moe {
+
+__host__ __device__ inline size_t al128d(size_t v) { return (v + 127) / 128 * 128; }
+
+// ---------------------------------------------------------------------------
+// Integer + fp32 dot of one lane's chunk of a weight row with one activation
+// vector.  w: packed words of the chunk's groups, act: 16 words per group
+// (elements 64g .. 64g+63), d: the two block scales per group, z: the integer
+// start values per group, -8 * (code sum of block 2g) and -128 * (code sum of
+// block 2g+1), which turn the unsigned nibble sums into exact signed sums.
+// ---------------------------------------------------------------------------
+template <int CSZ>
+__device__ __forceinline__ float chunk_dot(const uint32_t (&w)[CSZ][8], const float (&sc)[CSZ],
+                                           const uint32_t (&act)[CSZ][16], const float (&d)[CSZ][2],
+                                           const int (&z)[CSZ][2], int c0, int G) {
+  float acc = 0.0f;
+#pragma unroll
+  for (int gi = 0; gi < CSZ; ++gi) {
+    if (c0 + gi < G) {
+      int s0 = z[gi][0], s1 = z[gi][1], t0 = 0, t1 = 0;   // two chains per block
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        s0 = dp4a_us(w[gi][j] & 0x0F0F0F0Fu, act[gi][j], s0);
+        t0 = dp4a_us(w[gi][4 + j] & 0x0F0F0F0Fu, act[gi][4 + j], t0);
+        s1 = dp4a_us(w[gi][j] & 0xF0F0F0F0u, act[gi][8 + j], s1);
+        t1 = dp4a_us(w[gi][4 + j] & 0xF0F0F0F0u, act[gi][12 + j], t1);
+      }
+      s0 += t0;   // sum (u - 8) q over the low nibbles (block 2g)
+      s1 += t1;   // 16 * sum (u - 8) q over the high nibbles (block 2g+1)
+      const float fa = fmul((float)s0, d[gi][0]);
+      const float fb = ffma(fmul((float)s1, 0.0625f), d[gi][1], fa);  // (float)s1/16 is exact
+      acc = ffma(sc[gi], fb, acc);
+    }
+  }
+  return acc;
+}
+
+// Sum of the first nch of 32 chunk values, left to right (fixed order).
+__device__ __forceinline__ float chunk_sum(const float *rr, int nch) {
+  float v[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) v[c] = (c < nch) ? rr[c] : 0.0f;
+  float tot = v[0];
+#pragma unroll
+  for (int c = 1; c < 32; ++c)
+    if (c < nch) tot = fadd(tot, v[c]);
+  return tot;
+}
+
+// ===========================================================================
+// gate/up
+// ===========================================================================
+struct GuPlan {
+  size_t red, gu, xd, qs, xq, stg, total;
+  uint32_t sb;
+  int chp;
+};
+
+__host__ __device__ inline GuPlan gu_plan(int H, int T, int R, int ns, int csz) {
+  GuPlan p;
+  p.chp = csz * 64 + 16;
+  p.sb = (uint32_t)((size_t)R * H + (size_t)R * H / 16);
+  size_t o = al128d((size_t)16 * ns);
+  p.red = o;
+  o += al128d((size_t)8 * (2 * T > 8 ? 2 * T : 8) * 33 * 4);
+  p.gu = o;
+  o += al128d((size_t)T * 64 * 4);
+  p.xd = o;
+  o += al128d((size_t)T * (H / 32) * 4);
+  p.qs = o;
+  o += al128d((size_t)T * (H / 32) * 4);
+  p.xq = o;
+  o += al128d((size_t)T * 32 * p.chp);
+  p.stg = o;
+  o += (size_t)ns * p.sb;
+  p.total = o;
+  return p;
+}
+
+template <int CSZ, bool ONE>
+__global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int H = a.H, I = a.I, T = a.T, NS = a.nstage, R = a.rpm;
+  const int G = H / 64, HB = H / 32;
+  const int nch = (G + CSZ - 1) / CSZ;
+  const int SPU = 32 / R;  // stages per 32-row unit
+  const GuPlan pl = gu_plan(H, T, R, NS, CSZ);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + NS;
+  float *red = reinterpret_cast<float *>(smem + pl.red);
+  float *gu = reinterpret_cast<float *>(smem + pl.gu);
+  float *xd_s = reinterpret_cast<float *>(smem + pl.xd);
+  int *qs_s = reinterpret_cast<int *>(smem + pl.qs);
+  unsigned char *xq_s = smem + pl.xq;
+  unsigned char *stg = smem + pl.stg;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    s_abort = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 8);
+    }
+    fence_barrier_init();
+  }
+  if (a.use_pdl) pdl_wait();
+  // an earlier kernel of this call failed: leave everything untouched
+  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  const int n_uni = min(max(*a.n_uni, 0), a.E);
+  const int rbs = I / 32;  // 32-row units per expert
+  const int n_units = (n_uni + 1) * rbs;
+  const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
+  const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
+  const int n_stages = (u_end - u_begin) * SPU;
+  const size_t mg = (size_t)I * H / 2 + (size_t)I * H / 32;
+
+  // blobs this CTA reads must be 16-byte aligned (TMA bulk copies)
+  {
+    bool bad = false;
+    const int sl0 = u_begin / rbs, sl1 = (u_end - 1) / rbs;
+    for (int sl = sl0 + tid; sl <= sl1 && u_end > u_begin; sl += blockDim.x) {
+      const int e = sl == 0 ? a.E : a.uni[sl - 1];
+      bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
+    }
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) set_status(a.status, MOE_ERR_DEVICE, kDetGuAlign);
+      return;
+    }
+  }
+
+  // activations: xq in per-lane chunks (padded rows), block scales, code sums
+  {
+    const int pieces = CSZ * 4;
+    for (int i = tid; i < T * 32 * pieces; i += blockDim.x) {
+      const int t = i / (32 * pieces), r = i % (32 * pieces), c = r / pieces, j = r % pieces;
+      const int col = c * CSZ * 64 + 16 * j;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (col < H) v = *reinterpret_cast<const uint4 *>(a.xq + (size_t)t * H + col);
+      *reinterpret_cast<uint4 *>(xq_s + (size_t)(t * 32 + c) * pl.chp + 16 * j) = v;
+    }
+    for (int i = tid; i < T * HB; i += blockDim.x) {
+      xd_s[i] = a.xd[i];
+      const uint4 *q4 = reinterpret_cast<const uint4 *>(a.xq + (size_t)i * 32);
+      int s = 0;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const uint4 v = q4[j];
+        s = __dp4a((int)v.x, 0x01010101, s);
+        s = __dp4a((int)v.y, 0x01010101, s);
+        s = __dp4a((int)v.z, 0x01010101, s);
+        s = __dp4a((int)v.w, 0x01010101, s);
+      }
+      qs_s[i] = s;
+    }
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      const uint32_t pk = (uint32_t)R * (H / 2), sk = (uint32_t)R * (H / 32);
+      int issued = 0;
+      for (int j = 0; j < n_stages; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetGuEmpty)) {
+          s_abort = 1;
+          break;
+        }
+        if (*reinterpret_cast<volatile int *>(&s_abort)) break;
+        const int unit = u_begin + j / SPU, st = j % SPU;
+        const int slot = unit / rbs, rb = unit % rbs;
+        const int e = slot == 0 ? a.E : a.uni[slot - 1];
+        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
+        const size_t n0 = (size_t)rb * 32 + (size_t)st * R;
+        unsigned char *dst = stg + (size_t)s * pl.sb;
+        mbar_arrive_expect_tx(full + s, 2 * (pk + sk));
+        bulk_g2s_hint(dst, blob + n0 * (H / 2), pk, full + s, pol);
+        bulk_g2s_hint(dst + pk, blob + mg + n0 * (H / 2), pk, full + s, pol);
+        bulk_g2s_hint(dst + 2 * pk, blob + (size_t)I * (H / 2) + n0 * (H / 32), sk, full + s, pol);
+        bulk_g2s_hint(dst + 2 * pk + sk, blob + mg + (size_t)I * (H / 2) + n0 * (H / 32), sk,
+                      full + s, pol);
+        issued = j + 1;
+      }
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetGuDrain);
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- consumers
+  const int c0 = lane * CSZ;
+  const int RPW = R / 4;  // rows per warp per stage: 1 (R = 4) or 2 (R = 8)
+  // single token: this lane's activation chunk stays in registers
+  uint32_t act1[CSZ][16];
+  float d1[CSZ][2];
+  int q1[CSZ][2];
+  if (ONE) {
+#pragma unroll
+    for (int gi = 0; gi < CSZ; ++gi) {
+      const int g = c0 + gi;
+      const uint4 *src = reinterpret_cast<const uint4 *>(xq_s + (size_t)lane * pl.chp + 64 * gi);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 v = src[q];
+        act1[gi][4 * q] = v.x;
+        act1[gi][4 * q + 1] = v.y;
+        act1[gi][4 * q + 2] = v.z;
+        act1[gi][4 * q + 3] = v.w;
+      }
+      d1[gi][0] = g < G ? xd_s[2 * g] : 0.0f;
+      d1[gi][1] = g < G ? xd_s[2 * g + 1] : 0.0f;
+      q1[gi][0] = g < G ? -8 * qs_s[2 * g] : 0;
+      q1[gi][1] = g < G ? -128 * qs_s[2 * g + 1] : 0;
+    }
+  }
+
+  int cur_unit = -1, n_tok = 0, pos_base = 0, my_tok = 0;
+  bool bad = false;
+  for (int j = 0; j < n_stages; ++j) {
+    const int s = j % NS;
+    const int unit = u_begin + j / SPU, st = j % SPU;
+    const int slot = unit / rbs, rb = unit % rbs;
+    if (unit != cur_unit) {
+      cur_unit = unit;
+      if (slot == 0) {
+        n_tok = T;
+        pos_base = T * a.k;
+        my_tok = lane;
+      } else {
+        const int e = a.uni[slot - 1];
+        pos_base = a.off[e];
+        n_tok = a.off[e + 1] - pos_base;
+        my_tok = lane < n_tok ? a.pair_tok[pos_base + lane] : 0;
+      }
+    }
+    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
+    if (!bad) {
+      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetGuFull);
+      bad = __any_sync(0xffffffffu, bad);
+      if (bad && lane == 0) s_abort = 1;
+    }
+    if (!bad) {
+      const unsigned char *sb = stg + (size_t)s * pl.sb;
+      uint32_t wv[2][CSZ][8];
+      float sc[2][CSZ];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        if (q < RPW) {
+          const int jr = warp + 8 * q;
+          const int m = jr / R, r = jr % R;
+          const unsigned char *rowp = sb + (size_t)m * R * (H / 2) + (size_t)r * (H / 2);
+          const __half *scp = reinterpret_cast<const __half *>(
+              sb + (size_t)R * H + (size_t)m * R * (H / 32) + (size_t)r * (H / 32));
+#pragma unroll
+          for (int gi = 0; gi < CSZ; ++gi) {
+            const int g = c0 + gi;
+            if (g < G) {
+              const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
+              const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
+              wv[q][gi][0] = w0.x;
+              wv[q][gi][1] = w0.y;
+              wv[q][gi][2] = w0.z;
+              wv[q][gi][3] = w0.w;
+              wv[q][gi][4] = w1.x;
+              wv[q][gi][5] = w1.y;
+              wv[q][gi][6] = w1.z;
+              wv[q][gi][7] = w1.w;
+              sc[q][gi] = __half2float(scp[g]);
+            } else {
+#pragma unroll
+              for (int z = 0; z < 8; ++z) wv[q][gi][z] = 0u;
+              sc[q][gi] = 0.0f;
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
+      if (ONE) {
+        // chunk values of the warp's 8 rows of the unit are summed once per unit
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          if (q < RPW)
+            red[(warp * 8 + st * RPW + q) * 33 + lane] =
+                chunk_dot<CSZ>(wv[q], sc[q], act1, d1, q1, c0, G);
+        if (st == SPU - 1) {
+          __syncwarp();
+          if (lane < 8) {
+            const int sq = lane / RPW, q = lane % RPW;
+            const int jr = warp + 8 * q;
+            const int m = jr / R, r = jr % R;
+            gu[m * 32 + sq * R + r] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
+          }
+          __syncwarp();
+        }
+      } else {
+        for (int i = 0; i < n_tok; ++i) {
+          const int t = __shfl_sync(0xffffffffu, my_tok, i);
+          uint32_t act[CSZ][16];
+          float dd[CSZ][2];
+          int qq[CSZ][2];
+#pragma unroll
+          for (int gi = 0; gi < CSZ; ++gi) {
+            const int g = c0 + gi;
+            const uint4 *src =
+                reinterpret_cast<const uint4 *>(xq_s + (size_t)(t * 32 + lane) * pl.chp + 64 * gi);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = src[q];
+              act[gi][4 * q] = v.x;
+              act[gi][4 * q + 1] = v.y;
+              act[gi][4 * q + 2] = v.z;
+              act[gi][4 * q + 3] = v.w;
+            }
+            dd[gi][0] = g < G ? xd_s[t * HB + 2 * g] : 0.0f;
+            dd[gi][1] = g < G ? xd_s[t * HB + 2 * g + 1] : 0.0f;
+            qq[gi][0] = g < G ? -8 * qs_s[t * HB + 2 * g] : 0;
+            qq[gi][1] = g < G ? -128 * qs_s[t * HB + 2 * g + 1] : 0;
+          }
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+            if (q < RPW)
+              red[((warp * 2 + q) * T + i) * 33 + lane] =
+                  chunk_dot<CSZ>(wv[q], sc[q], act, dd, qq, c0, G);
+        }
+        __syncwarp();
+        if (lane < RPW * n_tok) {
+          const int q = lane / n_tok, i = lane % n_tok;
+          const int jr = warp + 8 * q;
+          const int m = jr / R, r = jr % R;
+          const float tot = chunk_sum(red + ((warp * 2 + q) * T + i) * 33, nch);
+          gu[(i * 2 + m) * 32 + st * R + r] = tot;
+        }
+        __syncwarp();
+      }
+    }
+    if (st == SPU - 1) {
+      // unit complete: h = SiLU(g) * u for its 32 rows, Q8_0 per token
+      named_sync(1, 256);
+      if (!bad) {
+        for (int i = warp; i < n_tok; i += 8) {
+          const float g = gu[(i * 2 + 0) * 32 + lane];
+          const float u = gu[(i * 2 + 1) * 32 + lane];
+          const float h = swiglu(g, u);
+          const float d = fdiv(warp_max(fabsf(h)), 127.0f);
+          const int q = q8_code(h, d);
+          const int pos = pos_base + i;
+          a.hq[(size_t)pos * I + rb * 32 + lane] = (int8_t)q;
+          int qsum = q;
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
+          if (lane == 0) {
+            a.hd[(size_t)pos * (I / 32) + rb] = d;
+            a.hqs[(size_t)pos * (I / 32) + rb] = qsum;
+          }
+        }
+      }
+      named_sync(1, 256);
+    }
+  }
+  if (a.use_pdl) pdl_launch_dependents();
+}
+
+static int gu_csz(int H) { return (H / 64 + 31) / 32; }
+
+size_t gateup_smem_bytes(int H, int T, int R, int nstage) {
+  return gu_plan(H, T, R, nstage, gu_csz(H)).total;
+}
+
+// Rows per matrix per stage and stage count: 8 rows (two per warp) when three
+// or more stages of that size fit, else 4.
+void gateup_plan(int H, int T, int *R, int *nstage) {
+  for (int r = 8; r >= 4; r -= 4) {
+    int ns = 8;
+    while (ns >= 2 && gateup_smem_bytes(H, T, r, ns) > (size_t)kMaxSmem) --ns;
+    if (ns >= 3 || r == 4) {
+      *R = r;
+      *nstage = ns > 6 ? 6 : ns;
+      return;
+    }
+  }
+}
+
+template <int CSZ, bool ONE>
+static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(k_gateup_decode<CSZ, ONE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(288);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.use_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ, ONE>, a);
+}
+
+cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
+  const bool one = a.T == 1;
+  switch (gu_csz(a.H)) {
+    case 1: return one ? launch_gu<1, true>(a, grid, smem, s) : launch_gu<1, false>(a, grid, smem, s);
+    case 2: return one ? launch_gu<2, true>(a, grid, smem, s) : launch_gu<2, false>(a, grid, smem, s);
+    case 3: return one ? launch_gu<3, true>(a, grid, smem, s) : launch_gu<3, false>(a, grid, smem, s);
+    case 4: return one ? launch_gu<4, true>(a, grid, smem, s) : launch_gu<4, false>(a, grid, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ===========================================================================
+// down + combine
+// ===========================================================================
+constexpr int kDnTokBatch = 4;
+
+struct DnPlan {
+  size_t red, ysm, act, stg, total;
+  uint32_t sb;
+};
+
+// Bytes of the per-position activations (codes, scales, code sums) when they
+// are small enough to keep in shared memory for the whole kernel, else 0.
+__host__ __device__ inline size_t dn_act_bytes(int I, int k, int T) {
+  const size_t P = (size_t)T * (k + 1);
+  const size_t b = P * I + 2 * P * (I / 32) * 4;
+  return b <= 48 * 1024 ? b : 0;
+}
+
+__host__ __device__ inline DnPlan dn_plan(int I, int k, int T, int rows_max, int rs, int ns) {
+  DnPlan p;
+  p.sb = (uint32_t)al128d((size_t)rs * (I / 2) + (size_t)rs * (I / 32));
+  size_t o = al128d((size_t)16 * ns + 16);
+  p.red = o;
+  o += al128d((size_t)8 * 32 * 33 * 4);
+  p.ysm = o;
+  o += al128d((size_t)T * (k + 1) * rows_max * 4);
+  p.act = o;
+  o += al128d(dn_act_bytes(I, k, T));
+  p.stg = o;
+  o += (size_t)ns * p.sb;
+  p.total = o;
+  return p;
+}
+
+template <int CSZ>
+__global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int H = a.H, I = a.I, T = a.T, K = a.k, NS = a.nstage, RS = a.rs;
+  const int G = I / 64, IB = I / 32;
+  const int nch = (G + CSZ - 1) / CSZ;
+  const DnPlan pl = dn_plan(I, K, T, a.rows_max, RS, NS);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+  uint64_t *empty = full + NS;
+  uint64_t *actbar = empty + NS;
+  float *red = reinterpret_cast<float *>(smem + pl.red);
+  float *ysm = reinterpret_cast<float *>(smem + pl.ysm);
+  unsigned char *stg = smem + pl.stg;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nrg = H / a.rg;
+  const int m0 = (int)((long long)blockIdx.x * nrg / gridDim.x) * a.rg;
+  const int m1 = (int)((long long)(blockIdx.x + 1) * nrg / gridDim.x) * a.rg;
+  const int nrows = m1 - m0;
+  const size_t mg = (size_t)I * H / 2 + (size_t)I * H / 32;
+  const size_t pk_off = 2 * mg, sc_off = 2 * mg + (size_t)H * (I / 2);
+  const int nsub = (nrows + RS - 1) / RS;  // row sub-ranges per union slot
+  const size_t sc_in_stage = (size_t)RS * (I / 2);
+
+  if (tid == 0) {
+    s_abort = 0;
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 8);
+    }
+    mbar_init(actbar, 1);
+    fence_barrier_init();
+  }
+  if (a.use_pdl) pdl_wait();
+  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  const int n_uni = min(max(*a.n_uni, 0), a.E);
+  const int nslot = n_uni + 1;
+  {
+    bool bad = false;
+    for (int sl = tid; sl < nslot; sl += blockDim.x) {
+      const int e = sl == 0 ? a.E : a.uni[sl - 1];
+      bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
+    }
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) set_status(a.status, MOE_ERR_DEVICE, kDetDnAlign);
+      return;
+    }
+  }
+  if (nrows <= 0) return;
+
+  // small batches: the h codes, scales and code sums of every position come
+  // into shared memory once (one TMA transaction) instead of per stage
+  const int P = T * (K + 1);
+  unsigned char *act_s = smem + pl.act;
+  const unsigned char *hq_b = a.preload ? act_s : reinterpret_cast<const unsigned char *>(a.hq);
+  const float *hd_b = a.preload ? reinterpret_cast<const float *>(act_s + (size_t)P * I) : a.hd;
+  const int *hqs_b =
+      a.preload ? reinterpret_cast<const int *>(act_s + (size_t)P * I + (size_t)P * IB * 4) : a.hqs;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      if (a.preload) {
+        const uint32_t bq = (uint32_t)P * I, bd = (uint32_t)P * IB * 4;
+        mbar_arrive_expect_tx(actbar, bq + 2 * bd);
+        bulk_g2s(act_s, a.hq, bq, actbar);
+        bulk_g2s(act_s + bq, a.hd, bd, actbar);
+        bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
+      }
+      int issued = 0;
+      for (int j = 0; j < nslot * nsub; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetDnEmpty)) {
+          s_abort = 1;
+          break;
+        }
+        if (*reinterpret_cast<volatile int *>(&s_abort)) break;
+        const int slot = j / nsub, r0 = (j % nsub) * RS;
+        const int nr = min(RS, nrows - r0);
+        const uint32_t bytes_pk = (uint32_t)nr * (I / 2), bytes_sc = (uint32_t)nr * (I / 32);
+        const int e = slot == 0 ? a.E : a.uni[slot - 1];
+        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
+        unsigned char *dst = stg + (size_t)s * pl.sb;
+        mbar_arrive_expect_tx(full + s, bytes_pk + bytes_sc);
+        bulk_g2s_hint(dst, blob + pk_off + (size_t)(m0 + r0) * (I / 2), bytes_pk, full + s, pol);
+        bulk_g2s_hint(dst + sc_in_stage, blob + sc_off + (size_t)(m0 + r0) * (I / 32), bytes_sc,
+                      full + s, pol);
+        issued = j + 1;
+      }
+      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
+        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
+      if (a.preload) mbar_wait(actbar, 0, a.status, kDetDnDrain);
+    }
+    return;
+  }
+
+  const int c0 = lane * CSZ;
+  float *redw = red + warp * 32 * 33;
+  bool bad = false;
+  if (a.preload) {
+    bad = !mbar_wait(actbar, 0, a.status, kDetDnFull);
+    bad = __any_sync(0xffffffffu, bad);
+    if (bad && lane == 0) s_abort = 1;
+  }
+  for (int j = 0; j < nslot * nsub; ++j) {
+    const int s = j % NS;
+    const int slot = j / nsub, r0 = (j % nsub) * RS;
+    const int nr = min(RS, nrows - r0);
+    int n_tok, pos_base;
+    if (slot == 0) {
+      n_tok = T;
+      pos_base = T * K;
+    } else {
+      const int e = a.uni[slot - 1];
+      pos_base = a.off[e];
+      n_tok = a.off[e + 1] - pos_base;
+    }
+    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
+    if (!bad) {
+      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetDnFull);
+      bad = __any_sync(0xffffffffu, bad);
+      if (bad && lane == 0) s_abort = 1;
+    }
+    if (bad) continue;
+    const unsigned char *sb = stg + (size_t)s * pl.sb;
+    // this warp's rows of the stage: a contiguous block
+    const int rpw = (nr + 7) / 8;
+    const int ra = min(nr, warp * rpw), rz = min(nr, ra + rpw);
+    for (int i0 = 0; i0 < n_tok; i0 += kDnTokBatch) {
+      const int nb = min(kDnTokBatch, n_tok - i0);
+      uint32_t av[kDnTokBatch][CSZ][16];
+      float dv[kDnTokBatch][CSZ][2];
+      int qv[kDnTokBatch][CSZ][2];
+#pragma unroll
+      for (int b = 0; b < kDnTokBatch; ++b) {
+        const int pos = pos_base + (b < nb ? i0 + b : i0);
+#pragma unroll
+        for (int gi = 0; gi < CSZ; ++gi) {
+          const int g = c0 + gi;
+          if (b < nb && g < G) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(hq_b + (size_t)pos * I + 64 * g);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 v = src[q];
+              av[b][gi][4 * q + 0] = v.x;
+              av[b][gi][4 * q + 1] = v.y;
+              av[b][gi][4 * q + 2] = v.z;
+              av[b][gi][4 * q + 3] = v.w;
+            }
+            dv[b][gi][0] = hd_b[(size_t)pos * IB + 2 * g];
+            dv[b][gi][1] = hd_b[(size_t)pos * IB + 2 * g + 1];
+            qv[b][gi][0] = -8 * hqs_b[(size_t)pos * IB + 2 * g];
+            qv[b][gi][1] = -128 * hqs_b[(size_t)pos * IB + 2 * g + 1];
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) av[b][gi][q] = 0u;
+            dv[b][gi][0] = dv[b][gi][1] = 0.0f;
+            qv[b][gi][0] = qv[b][gi][1] = 0;
+          }
+        }
+      }
+      const bool last_batch = i0 + kDnTokBatch >= n_tok;
+      // rows in passes so that (row, token) pairs fit the 32 lanes of the sum
+      const int ppass = 32 / nb;
+      for (int p0 = ra; p0 < rz; p0 += ppass) {
+        const int p1 = min(rz, p0 + ppass);
+        for (int ml = p0; ml < p1; ++ml) {
+          const unsigned char *rowp = sb + (size_t)ml * (I / 2);
+          const __half *scp = reinterpret_cast<const __half *>(sb + sc_in_stage + (size_t)ml * (I / 32));
+          uint32_t wv[CSZ][8];
+          float sc[CSZ];
+#pragma unroll
+          for (int gi = 0; gi < CSZ; ++gi) {
+            const int g = c0 + gi;
+            if (g < G) {
+              const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
+              const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
+              wv[gi][0] = w0.x;
+              wv[gi][1] = w0.y;
+              wv[gi][2] = w0.z;
+              wv[gi][3] = w0.w;
+              wv[gi][4] = w1.x;
+              wv[gi][5] = w1.y;
+              wv[gi][6] = w1.z;
+              wv[gi][7] = w1.w;
+              sc[gi] = __half2float(scp[g]);
+            } else {
+#pragma unroll
+              for (int z = 0; z < 8; ++z) wv[gi][z] = 0u;
+              sc[gi] = 0.0f;
+            }
+          }
+#pragma unroll
+          for (int b = 0; b < kDnTokBatch; ++b)
+            if (b < nb)
+              redw[((ml - p0) * nb + b) * 33 + lane] =
+                  chunk_dot<CSZ>(wv, sc, av[b], dv[b], qv[b], c0, G);
+        }
+        if (last_batch && p1 == rz) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(empty + s);  // every row of this warp is read
+        }
+        __syncwarp();
+        if (lane < (p1 - p0) * nb) {
+          const int ml = p0 + lane / nb, b = lane % nb;
+          const float tot = chunk_sum(redw + lane * 33, nch);
+          ysm[(size_t)(pos_base + i0 + b) * a.rows_max + r0 + ml] = tot;
+        }
+        __syncwarp();
+      }
+      if (last_batch && ra >= rz) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);  // this warp had no rows
+      }
+    }
+  }
+  named_sync(1, 256);
+  if (*reinterpret_cast<volatile int *>(&s_abort)) return;
+  for (int i = tid; i < T * nrows; i += 256) {
+    const int t = i / nrows, m = i % nrows;
+    float o = ysm[(size_t)(T * K + t) * a.rows_max + m];
+    for (int s = 0; s < K; ++s) {
+      const int p = a.pos[t * K + s];
+      o = ffma(a.w[t * K + s], ysm[(size_t)p * a.rows_max + m], o);
+    }
+    a.out[(size_t)t * H + m0 + m] = o;
+  }
+  if (a.use_pdl) pdl_launch_dependents();
+}
+
+size_t down_smem_bytes(int H, int I, int k, int T, int rows_max, int rs, int nstage) {
+  (void)H;
+  return dn_plan(I, k, T, rows_max, rs, nstage).total;
+}
+
+int down_preload(int I, int k, int T) { return dn_act_bytes(I, k, T) > 0 ? 1 : 0; }
+
+int down_max_stages(int H, int I, int k, int T, int rows_max, int rs) {
+  int ns = 6;
+  while (ns >= 2 && down_smem_bytes(H, I, k, T, rows_max, rs, ns) > (size_t)kMaxSmem) --ns;
+  return ns;
+}
+
+template <int CSZ>
+static cudaError_t launch_dn(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
+  cudaError_t err = cudaFuncSetAttribute(k_down_decode<CSZ>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(288);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.use_pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, k_down_decode<CSZ>, a);
+}
+
+cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
+  const int csz = (a.I / 64 + 31) / 32;
+  switch (csz) {
+    case 1: return launch_dn<1>(a, grid, smem, s);
+    case 2: return launch_dn<2>(a, grid, smem, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace moe

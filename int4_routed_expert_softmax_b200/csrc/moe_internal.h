@@ -115,6 +115,7 @@ struct GateUpArgs {
   float *hd;
   int32_t *status;
   int nstage;
+  int rpm;  // weight rows per matrix per stage (4 or 8)
   int use_pdl;
 };
 
@@ -132,6 +133,7 @@ struct DownArgs {
   int rg;        // row granularity (scale bytes of a row group are a multiple of 16)
   int rows_max;  // most output rows any CTA owns
   int rs;        // rows per stage (a multiple of rg)
+  int preload;   // per-position activations kept in shared memory (small batches)
   int use_pdl;
 };
 
@@ -146,9 +148,10 @@ cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStr
 
 // Shared-memory plans (host side, moe_kernels.cu).
 size_t route_smem_bytes(int H, int epc, int tt);
-size_t gateup_smem_bytes(int H, int T, int nstage);
+size_t gateup_smem_bytes(int H, int T, int R, int nstage);
+void gateup_plan(int H, int T, int *R, int *nstage);
 size_t down_smem_bytes(int H, int I, int k, int T, int rows_max, int rs, int nstage);
-int gateup_max_stages(int H, int T);
 int down_max_stages(int H, int I, int k, int T, int rows_max, int rs);
+int down_preload(int I, int k, int T);
 
 }  // namespace moe

@@ -23,10 +23,6 @@
 
 namespace moe {
 
-namespace {
-inline size_t al128(size_t v) { return align_up(v, 128); }
-}  // namespace
-
 // =====================================================================
 // Q8_0 quantisation: one warp per 32-block (lane = element).
 // =====================================================================
@@ -157,6 +153,77 @@ __device__ void bucket_block(int E, int k, int T, const int32_t *idx, int *s_wor
 }
 
 // =====================================================================
+// The same stable counting sort by a single warp (no block barriers): for
+// the decode batch (P = T*k <= 512 pairs).  s_work: >= 2E ints of shared
+// memory; idx may live in shared memory.
+// =====================================================================
+__device__ void bucket_warp(int E, int k, int T, const int32_t *idx, int *s_work, int32_t *cnt,
+                            int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm,
+                            int32_t *pos, int32_t *pair_tok) {
+  const int lane = threadIdx.x & 31;
+  const int P = T * k;
+  int *s_cnt = s_work;      // [E]
+  int *s_cur = s_work + E;  // [E]
+  for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
+  __syncwarp();
+  for (int p = lane; p < P; p += 32) atomicAdd(&s_cnt[idx[p]], 1);
+  __syncwarp();
+  // exclusive scans of the counts and of the union flags; lane owns a range
+  const int per = (E + 31) / 32;
+  const int b0 = min(E, lane * per), b1 = min(E, b0 + per);
+  int lc = 0, lf = 0;
+  for (int e = b0; e < b1; ++e) {
+    lc += s_cnt[e];
+    lf += s_cnt[e] > 0 ? 1 : 0;
+  }
+  int ic = lc, jf = lf;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int vc = __shfl_up_sync(0xffffffffu, ic, o);
+    const int vf = __shfl_up_sync(0xffffffffu, jf, o);
+    if (lane >= o) {
+      ic += vc;
+      jf += vf;
+    }
+  }
+  int run = ic - lc, runf = jf - lf;
+  for (int e = b0; e < b1; ++e) {
+    const int c = s_cnt[e];
+    cnt[e] = c;
+    off[e] = run;
+    s_cur[e] = run;
+    run += c;
+    if (c > 0) uni[runf++] = e;
+  }
+  const int nu = __shfl_sync(0xffffffffu, jf, 31);
+  if (lane == 0) {
+    off[E] = P;
+    *n_uni = nu;
+    uni[nu] = E;  // the shared expert follows the union
+  }
+  __syncwarp();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c0 = 0; c0 < P; c0 += 32) {
+    const int p = c0 + lane;
+    const bool has = p < P;
+    const int e = has ? idx[p] : -1 - lane;  // distinct dummies never match
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    const int base = has ? s_cur[e] : 0;
+    __syncwarp();
+    if (has && lane == __ffs(peers) - 1) s_cur[e] = base + __popc(peers);
+    if (has) {
+      const int q = base + __popc(peers & lt);
+      perm[q] = p;
+      if (pos) pos[p] = q;
+      if (pair_tok) pair_tok[q] = p / k;
+    }
+    __syncwarp();
+  }
+  if (pair_tok)
+    for (int t = lane; t < T; t += 32) pair_tok[P + t] = t;
+}
+
+// =====================================================================
 // Top-k of one token's logits by one warp (E <= 1024, k <= 32): lane s ends
 // holding slot s (expert, logit).  Ties go to the lower expert index.
 // =====================================================================
@@ -234,6 +301,22 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = a.H;
 
+  const int e0 = blockIdx.x * a.epc;
+  const int ne = min(a.epc, a.E - e0);
+  // start the copies of the first tile before the quantisation work below
+  auto issue = [&](int t0) {
+    const int nt = min(a.tt, a.T - t0);
+    const uint32_t xb = (uint32_t)nt * H * 4u;
+    const uint32_t wb = (t0 == 0) ? (uint32_t)ne * H * 4u : 0u;
+    mbar_arrive_expect_tx(bar, xb + wb);
+    if (wb) bulk_g2s(sW, a.Wr + (size_t)e0 * H, wb, bar);
+    bulk_g2s(sX, a.x + (size_t)t0 * H, xb, bar);
+  };
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_barrier_init();
+    issue(0);
+  }
   if (a.do_quant) {
     const int64_t nblk = (int64_t)a.T * (H / 32);
     for (int64_t b = (int64_t)blockIdx.x * 4 + warp; b < nblk; b += (int64_t)gridDim.x * 4) {
@@ -243,24 +326,11 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
       if (lane == 0) a.xd[b] = d;
     }
   }
-
-  const int e0 = blockIdx.x * a.epc;
-  const int ne = min(a.epc, a.E - e0);
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    fence_barrier_init();
-  }
   __syncthreads();
   int phase = 0;
   for (int t0 = 0; t0 < a.T; t0 += a.tt, ++phase) {
     const int nt = min(a.tt, a.T - t0);
-    if (tid == 0) {
-      const uint32_t xb = (uint32_t)nt * H * 4u;
-      const uint32_t wb = (t0 == 0) ? (uint32_t)ne * H * 4u : 0u;
-      mbar_arrive_expect_tx(bar, xb + wb);
-      if (wb) bulk_g2s(sW, a.Wr + (size_t)e0 * H, wb, bar);
-      bulk_g2s(sX, a.x + (size_t)t0 * H, xb, bar);
-    }
+    if (tid == 0 && t0 > 0) issue(t0);
     const bool ok = __syncthreads_and(mbar_wait(bar, phase & 1, a.status, kDetRouteBar));
     if (!ok) return;
     for (int p = warp; p < ne * nt; p += 4) {
@@ -294,10 +364,11 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
     warp_softmax_store(t, a.k, lane, e_sel, l_sel, a.idx, a.w, a.route_counts, s_idx);
   }
   __syncthreads();
+  if (warp != 0) return;
   if (a.do_bucket)
-    bucket_block(a.E, a.k, a.T, s_idx, s_work, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos,
-                 a.pair_tok);
-  if (tid == 0) *a.done = 0u;
+    bucket_warp(a.E, a.k, a.T, s_idx, s_work, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos,
+                a.pair_tok);
+  if (lane == 0) *a.done = 0u;
 }
 
 size_t route_smem_bytes(int H, int epc, int tt) {
@@ -347,599 +418,6 @@ cudaError_t launch_bucket(const BucketArgs &a, cudaStream_t s) {
   const size_t smem = (size_t)(3 * a.E + 64) * 4;
   k_bucket<<<1, 1024, smem, s>>>(a);
   return cudaGetLastError();
-}
-
-// =====================================================================
-// Decode gate/up: h = SiLU(Wg x) * (Wu x), requantised to Q8_0 per 32 rows.
-//
-// Work unit = (union slot, 32-row block of I); slot 0 is the shared expert,
-// slot u >= 1 is uni[u-1].  Units are split evenly over the persistent CTAs.
-// A unit is 8 stages of 4 gate rows + 4 up rows (packed nibbles + fp16
-// scales, 4H + H/4 bytes at H=6144: 26,112 B), each stage one TMA
-// transaction group.  Consumer warp w takes row (w & 3) of matrix (w >> 2);
-// lane c owns the chunk of CSZ consecutive 64-groups [c*CSZ, c*CSZ+CSZ) --
-// the chunk split of the fixed dot order -- and the 32 chunk sums are added
-// left to right by one lane per token.
-// =====================================================================
-struct GuPlan {
-  size_t red, gu, xd, qs, xq, stg, total;
-  uint32_t sb;
-  int chp;
-};
-
-__host__ __device__ inline size_t al128d(size_t v) { return (v + 127) / 128 * 128; }
-
-__host__ __device__ inline GuPlan gu_plan(int H, int T, int ns, int csz) {
-  GuPlan p;
-  p.chp = csz * 64 + 16;
-  p.sb = 4u * (uint32_t)H + (uint32_t)H / 4u;
-  size_t o = al128d((size_t)16 * ns);
-  p.red = o;
-  o += al128d((size_t)8 * T * 33 * 4);
-  p.gu = o;
-  o += al128d((size_t)T * 64 * 4);
-  p.xd = o;
-  o += al128d((size_t)T * (H / 32) * 4);
-  p.qs = o;
-  o += al128d((size_t)T * (H / 32) * 4);
-  p.xq = o;
-  o += al128d((size_t)T * 32 * p.chp);
-  p.stg = o;
-  o += (size_t)ns * p.sb;
-  p.total = o;
-  return p;
-}
-
-template <int CSZ>
-__global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int H = a.H, I = a.I, T = a.T, NS = a.nstage;
-  const int G = H / 64, HB = H / 32;
-  const int nch = (G + CSZ - 1) / CSZ;
-  const GuPlan pl = gu_plan(H, T, NS, CSZ);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *empty = full + NS;
-  float *red = reinterpret_cast<float *>(smem + pl.red);
-  float *gu = reinterpret_cast<float *>(smem + pl.gu);
-  float *xd_s = reinterpret_cast<float *>(smem + pl.xd);
-  int *qs_s = reinterpret_cast<int *>(smem + pl.qs);
-  unsigned char *xq_s = smem + pl.xq;
-  unsigned char *stg = smem + pl.stg;
-  __shared__ int s_abort;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid == 0) {
-    s_abort = 0;
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 8);
-    }
-    fence_barrier_init();
-  }
-  if (a.use_pdl) pdl_wait();
-
-  // an earlier kernel of this call failed: leave everything untouched
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
-  const int n_uni = min(max(*a.n_uni, 0), a.E);
-  const int rbs = I / 32;  // 32-row blocks per expert
-  const int n_units = (n_uni + 1) * rbs;
-  const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
-  const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
-  const int n_stages = (u_end - u_begin) * 8;
-  const size_t mg = (size_t)I * H / 2 + (size_t)I * H / 32;
-
-  // blobs this CTA reads must be 16-byte aligned (TMA bulk copies)
-  {
-    bool bad = false;
-    const int sl0 = u_begin / rbs, sl1 = (u_end - 1) / rbs;
-    for (int sl = sl0 + tid; sl <= sl1 && u_end > u_begin; sl += blockDim.x) {
-      const int e = sl == 0 ? a.E : a.uni[sl - 1];
-      bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
-    }
-    if (__syncthreads_or(bad)) {
-      if (tid == 0) set_status(a.status, MOE_ERR_DEVICE, kDetGuAlign);
-      return;
-    }
-  }
-
-  // stage this CTA's copy of the activations: xq in per-lane chunks
-  // (padded rows, conflict-free 16-byte reads), block scales and code sums.
-  {
-    const int pieces = CSZ * 4;  // 16-byte pieces per lane chunk
-    for (int i = tid; i < T * 32 * pieces; i += blockDim.x) {
-      const int t = i / (32 * pieces), r = i % (32 * pieces), c = r / pieces, j = r % pieces;
-      const int col = c * CSZ * 64 + 16 * j;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (col < H) v = *reinterpret_cast<const uint4 *>(a.xq + (size_t)t * H + col);
-      *reinterpret_cast<uint4 *>(xq_s + (size_t)(t * 32 + c) * pl.chp + 16 * j) = v;
-    }
-    for (int i = tid; i < T * HB; i += blockDim.x) {
-      xd_s[i] = a.xd[i];
-      const uint4 *q4 = reinterpret_cast<const uint4 *>(a.xq + (size_t)i * 32);
-      int s = 0;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const uint4 v = q4[j];
-        s = __dp4a((int)v.x, 0x01010101, s);
-        s = __dp4a((int)v.y, 0x01010101, s);
-        s = __dp4a((int)v.z, 0x01010101, s);
-        s = __dp4a((int)v.w, 0x01010101, s);
-      }
-      qs_s[i] = s;
-    }
-  }
-  __syncthreads();
-
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int j = 0; j < n_stages; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetGuEmpty)) {
-          s_abort = 1;
-          break;
-        }
-        if (*reinterpret_cast<volatile int *>(&s_abort)) break;
-        const int unit = u_begin + j / 8, st = j % 8;
-        const int slot = unit / rbs, rb = unit % rbs;
-        const int e = slot == 0 ? a.E : a.uni[slot - 1];
-        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
-        const size_t n0 = (size_t)rb * 32 + (size_t)st * 4;
-        unsigned char *dst = stg + (size_t)s * pl.sb;
-        mbar_arrive_expect_tx(full + s, pl.sb);
-        bulk_g2s_hint(dst, blob + n0 * (H / 2), 2u * H, full + s, pol);
-        bulk_g2s_hint(dst + 2 * H, blob + mg + n0 * (H / 2), 2u * H, full + s, pol);
-        bulk_g2s_hint(dst + 4 * H, blob + (size_t)I * (H / 2) + n0 * (H / 32), H / 8, full + s, pol);
-        bulk_g2s_hint(dst + 4 * H + H / 8, blob + mg + (size_t)I * (H / 2) + n0 * (H / 32), H / 8,
-                      full + s, pol);
-        issued = j + 1;
-      }
-      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetGuDrain);
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
-  const int r = warp & 3, mat = warp >> 2;
-  const int c0 = lane * CSZ;
-  int cur_unit = -1, n_tok = 0, pos_base = 0, my_tok = 0;
-  bool bad = false;
-  for (int j = 0; j < n_stages; ++j) {
-    const int s = j % NS;
-    const int unit = u_begin + j / 8, st = j % 8;
-    const int slot = unit / rbs, rb = unit % rbs;
-    if (unit != cur_unit) {
-      cur_unit = unit;
-      if (slot == 0) {
-        n_tok = T;
-        pos_base = T * a.k;
-        my_tok = lane;
-      } else {
-        const int e = a.uni[slot - 1];
-        pos_base = a.off[e];
-        n_tok = a.off[e + 1] - pos_base;
-        my_tok = lane < n_tok ? a.pair_tok[pos_base + lane] : 0;
-      }
-    }
-    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
-    if (!bad) {
-      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetGuFull);
-      bad = __any_sync(0xffffffffu, bad);
-      if (bad && lane == 0) s_abort = 1;
-    }
-    if (!bad) {
-      const unsigned char *sb = stg + (size_t)s * pl.sb;
-      const unsigned char *rowp = sb + (size_t)mat * 2 * H + (size_t)r * (H / 2);
-      const __half *scp = reinterpret_cast<const __half *>(sb + 4 * H + mat * (H / 8) + r * (H / 32));
-      uint32_t lo[CSZ][8], hi[CSZ][8];
-      float sc[CSZ];
-#pragma unroll
-      for (int gi = 0; gi < CSZ; ++gi) {
-        const int g = c0 + gi;
-        if (g < G) {
-          const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
-          const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
-          const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            lo[gi][q] = wv[q] & 0x0F0F0F0Fu;
-            hi[gi][q] = (wv[q] >> 4) & 0x0F0F0F0Fu;
-          }
-          sc[gi] = __half2float(scp[g]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) lo[gi][q] = hi[gi][q] = 0u;
-          sc[gi] = 0.0f;
-        }
-      }
-      for (int i = 0; i < n_tok; ++i) {
-        const int t = __shfl_sync(0xffffffffu, my_tok, i);
-        const unsigned char *xa = xq_s + (size_t)(t * 32 + lane) * pl.chp;
-        const float *xdt = xd_s + t * HB;
-        const int *qst = qs_s + t * HB;
-        float acc = 0.0f;
-#pragma unroll
-        for (int gi = 0; gi < CSZ; ++gi) {
-          const int g = c0 + gi;
-          if (g < G) {
-            const uint4 a0 = *reinterpret_cast<const uint4 *>(xa + 64 * gi);
-            const uint4 a1 = *reinterpret_cast<const uint4 *>(xa + 64 * gi + 16);
-            const uint4 a2 = *reinterpret_cast<const uint4 *>(xa + 64 * gi + 32);
-            const uint4 a3 = *reinterpret_cast<const uint4 *>(xa + 64 * gi + 48);
-            int s0 = -8 * qst[2 * g], s1 = -8 * qst[2 * g + 1];
-            s0 = dp4a_us(lo[gi][0], a0.x, s0);
-            s0 = dp4a_us(lo[gi][1], a0.y, s0);
-            s0 = dp4a_us(lo[gi][2], a0.z, s0);
-            s0 = dp4a_us(lo[gi][3], a0.w, s0);
-            s0 = dp4a_us(lo[gi][4], a1.x, s0);
-            s0 = dp4a_us(lo[gi][5], a1.y, s0);
-            s0 = dp4a_us(lo[gi][6], a1.z, s0);
-            s0 = dp4a_us(lo[gi][7], a1.w, s0);
-            s1 = dp4a_us(hi[gi][0], a2.x, s1);
-            s1 = dp4a_us(hi[gi][1], a2.y, s1);
-            s1 = dp4a_us(hi[gi][2], a2.z, s1);
-            s1 = dp4a_us(hi[gi][3], a2.w, s1);
-            s1 = dp4a_us(hi[gi][4], a3.x, s1);
-            s1 = dp4a_us(hi[gi][5], a3.y, s1);
-            s1 = dp4a_us(hi[gi][6], a3.z, s1);
-            s1 = dp4a_us(hi[gi][7], a3.w, s1);
-            const float fa = fmul((float)s0, xdt[2 * g]);
-            const float fb = ffma((float)s1, xdt[2 * g + 1], fa);
-            acc = ffma(sc[gi], fb, acc);
-          }
-        }
-        red[(warp * T + i) * 33 + lane] = acc;
-      }
-      __syncwarp();
-      for (int i = lane; i < n_tok; i += 32) {
-        const float *rr = red + (warp * T + i) * 33;
-        float tot = rr[0];
-        for (int c = 1; c < nch; ++c) tot = fadd(tot, rr[c]);
-        gu[(i * 2 + mat) * 32 + st * 4 + r] = tot;
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty + s);
-    }
-    if (st == 7) {
-      // unit complete: h = SiLU(g) * u for its 32 rows, Q8_0 per token
-      named_sync(1, 256);
-      if (!bad) {
-        for (int i = warp; i < n_tok; i += 8) {
-          const float g = gu[(i * 2 + 0) * 32 + lane];
-          const float u = gu[(i * 2 + 1) * 32 + lane];
-          const float h = swiglu(g, u);
-          const float d = fdiv(warp_max(fabsf(h)), 127.0f);
-          const int q = q8_code(h, d);
-          const int pos = pos_base + i;
-          a.hq[(size_t)pos * I + rb * 32 + lane] = (int8_t)q;
-          int qsum = q;
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
-          if (lane == 0) {
-            a.hd[(size_t)pos * (I / 32) + rb] = d;
-            a.hqs[(size_t)pos * (I / 32) + rb] = qsum;
-          }
-        }
-      }
-      named_sync(1, 256);
-    }
-  }
-  if (a.use_pdl) pdl_launch_dependents();
-}
-
-size_t gateup_smem_bytes(int H, int T, int nstage) {
-  const int csz = (H / 64 + 31) / 32;
-  return gu_plan(H, T, nstage, csz).total;
-}
-
-int gateup_max_stages(int H, int T) {
-  int ns = 8;
-  while (ns >= 2 && gateup_smem_bytes(H, T, ns) > (size_t)kMaxSmem) --ns;
-  return ns;
-}
-
-template <int CSZ>
-static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_gateup_decode<CSZ>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(288);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = a.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ>, a);
-}
-
-cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
-  const int csz = (a.H / 64 + 31) / 32;
-  switch (csz) {
-    case 1: return launch_gu<1>(a, grid, smem, s);
-    case 2: return launch_gu<2>(a, grid, smem, s);
-    case 3: return launch_gu<3>(a, grid, smem, s);
-    case 4: return launch_gu<4>(a, grid, smem, s);
-    default: return cudaErrorInvalidValue;
-  }
-}
-
-// =====================================================================
-// Decode down projection + combine.
-//
-// CTA c owns output rows [m0, m1) (balanced, in row groups of rg rows so
-// every scale copy is a multiple of 16 bytes) and loops over the union
-// slots; one stage = that slot's rows (packed + scales, ~42 x 1088 B at
-// H=6144, I=2048).  y per (position, row) stays in shared memory; the
-// combine out = y_shared, then fmaf(w_s, y_s, out) in slot order, runs in
-// the same CTA at the end (deterministic, no atomics).
-// =====================================================================
-struct DnPlan {
-  size_t red, ysm, stg, total;
-  uint32_t sb;
-};
-
-__host__ __device__ inline DnPlan dn_plan(int I, int k, int T, int rows_max, int rs, int ns) {
-  DnPlan p;
-  p.sb = (uint32_t)al128d((size_t)rs * (I / 2) + (size_t)rs * (I / 32));
-  size_t o = al128d((size_t)16 * ns);
-  p.red = o;
-  o += al128d((size_t)8 * T * 33 * 4);
-  p.ysm = o;
-  o += al128d((size_t)T * (k + 1) * rows_max * 4);
-  p.stg = o;
-  o += (size_t)ns * p.sb;
-  p.total = o;
-  return p;
-}
-
-constexpr int kDnTokBatch = 4;
-
-template <int CSZ>
-__global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int H = a.H, I = a.I, T = a.T, K = a.k, NS = a.nstage;
-  const int G = I / 64, IB = I / 32;
-  const int nch = (G + CSZ - 1) / CSZ;
-  const DnPlan pl = dn_plan(I, K, T, a.rows_max, a.rs, NS);
-  const int RS = a.rs;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-  uint64_t *empty = full + NS;
-  float *red = reinterpret_cast<float *>(smem + pl.red);
-  float *ysm = reinterpret_cast<float *>(smem + pl.ysm);
-  unsigned char *stg = smem + pl.stg;
-  __shared__ int s_abort;
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nrg = H / a.rg;
-  const int m0 = (int)((long long)blockIdx.x * nrg / gridDim.x) * a.rg;
-  const int m1 = (int)((long long)(blockIdx.x + 1) * nrg / gridDim.x) * a.rg;
-  const int nrows = m1 - m0;
-  const size_t mg = (size_t)I * H / 2 + (size_t)I * H / 32;
-  const size_t pk_off = 2 * mg, sc_off = 2 * mg + (size_t)H * (I / 2);
-  const int nsub = (nrows + RS - 1) / RS;  // row sub-ranges per union slot
-  const size_t sc_in_stage = (size_t)RS * (I / 2);
-
-  if (tid == 0) {
-    s_abort = 0;
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 8);
-    }
-    fence_barrier_init();
-  }
-  if (a.use_pdl) pdl_wait();
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
-  const int n_uni = min(max(*a.n_uni, 0), a.E);
-  const int nslot = n_uni + 1;
-  {
-    bool bad = false;
-    for (int sl = tid; sl < nslot; sl += blockDim.x) {
-      const int e = sl == 0 ? a.E : a.uni[sl - 1];
-      bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
-    }
-    if (__syncthreads_or(bad)) {
-      if (tid == 0) set_status(a.status, MOE_ERR_DEVICE, kDetDnAlign);
-      return;
-    }
-  }
-  if (nrows <= 0) return;
-
-  if (warp == 8) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_first();
-      int issued = 0;
-      for (int j = 0; j < nslot * nsub; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetDnEmpty)) {
-          s_abort = 1;
-          break;
-        }
-        if (*reinterpret_cast<volatile int *>(&s_abort)) break;
-        const int slot = j / nsub, r0 = (j % nsub) * RS;
-        const int nr = min(RS, nrows - r0);
-        const uint32_t bytes_pk = (uint32_t)nr * (I / 2), bytes_sc = (uint32_t)nr * (I / 32);
-        const int e = slot == 0 ? a.E : a.uni[slot - 1];
-        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
-        unsigned char *dst = stg + (size_t)s * pl.sb;
-        mbar_arrive_expect_tx(full + s, bytes_pk + bytes_sc);
-        bulk_g2s_hint(dst, blob + pk_off + (size_t)(m0 + r0) * (I / 2), bytes_pk, full + s, pol);
-        bulk_g2s_hint(dst + sc_in_stage, blob + sc_off + (size_t)(m0 + r0) * (I / 32), bytes_sc,
-                      full + s, pol);
-        issued = j + 1;
-      }
-      for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
-    }
-    return;
-  }
-
-  const int c0 = lane * CSZ;
-  bool bad = false;
-  for (int j = 0; j < nslot * nsub; ++j) {
-    const int s = j % NS;
-    const int slot = j / nsub, r0 = (j % nsub) * RS;
-    const int nr = min(RS, nrows - r0);
-    int n_tok, pos_base;
-    if (slot == 0) {
-      n_tok = T;
-      pos_base = T * K;
-    } else {
-      const int e = a.uni[slot - 1];
-      pos_base = a.off[e];
-      n_tok = a.off[e + 1] - pos_base;
-    }
-    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
-    if (!bad) {
-      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetDnFull);
-      bad = __any_sync(0xffffffffu, bad);
-      if (bad && lane == 0) s_abort = 1;
-    }
-    if (bad) continue;
-    const unsigned char *sb = stg + (size_t)s * pl.sb;
-    for (int i0 = 0; i0 < n_tok; i0 += kDnTokBatch) {
-      const int nb = min(kDnTokBatch, n_tok - i0);
-      // this lane's activation chunk for up to kDnTokBatch positions
-      uint32_t av[kDnTokBatch][CSZ][16];
-      float dv[kDnTokBatch][CSZ][2];
-      int qv[kDnTokBatch][CSZ][2];
-#pragma unroll
-      for (int b = 0; b < kDnTokBatch; ++b) {
-        const int pos = pos_base + (b < nb ? i0 + b : i0);
-#pragma unroll
-        for (int gi = 0; gi < CSZ; ++gi) {
-          const int g = c0 + gi;
-          if (b < nb && g < G) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(a.hq + (size_t)pos * I + 64 * g);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 v = __ldg(src + q);
-              av[b][gi][4 * q + 0] = v.x;
-              av[b][gi][4 * q + 1] = v.y;
-              av[b][gi][4 * q + 2] = v.z;
-              av[b][gi][4 * q + 3] = v.w;
-            }
-            dv[b][gi][0] = __ldg(a.hd + (size_t)pos * IB + 2 * g);
-            dv[b][gi][1] = __ldg(a.hd + (size_t)pos * IB + 2 * g + 1);
-            qv[b][gi][0] = __ldg(a.hqs + (size_t)pos * IB + 2 * g);
-            qv[b][gi][1] = __ldg(a.hqs + (size_t)pos * IB + 2 * g + 1);
-          } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) av[b][gi][q] = 0u;
-            dv[b][gi][0] = dv[b][gi][1] = 0.0f;
-            qv[b][gi][0] = qv[b][gi][1] = 0;
-          }
-        }
-      }
-      for (int ml = warp; ml < nr; ml += 8) {
-        const int m = r0 + ml;  // row of this CTA (stage row ml)
-        const unsigned char *rowp = sb + (size_t)ml * (I / 2);
-        const __half *scp = reinterpret_cast<const __half *>(sb + sc_in_stage + (size_t)ml * (I / 32));
-        float acc[kDnTokBatch];
-#pragma unroll
-        for (int b = 0; b < kDnTokBatch; ++b) acc[b] = 0.0f;
-#pragma unroll
-        for (int gi = 0; gi < CSZ; ++gi) {
-          const int g = c0 + gi;
-          if (g < G) {
-            const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
-            const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
-            const uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            uint32_t lo[8], hi[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              lo[q] = wv[q] & 0x0F0F0F0Fu;
-              hi[q] = (wv[q] >> 4) & 0x0F0F0F0Fu;
-            }
-            const float sc = __half2float(scp[g]);
-#pragma unroll
-            for (int b = 0; b < kDnTokBatch; ++b) {
-              if (b < nb) {
-                int s0 = -8 * qv[b][gi][0], s1 = -8 * qv[b][gi][1];
-#pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                  s0 = dp4a_us(lo[q], av[b][gi][q], s0);
-                  s1 = dp4a_us(hi[q], av[b][gi][8 + q], s1);
-                }
-                const float fa = fmul((float)s0, dv[b][gi][0]);
-                const float fb = ffma((float)s1, dv[b][gi][1], fa);
-                acc[b] = ffma(sc, fb, acc[b]);
-              }
-            }
-          }
-        }
-#pragma unroll
-        for (int b = 0; b < kDnTokBatch; ++b)
-          if (b < nb) red[(warp * T + b) * 33 + lane] = acc[b];
-        __syncwarp();
-        if (lane < nb) {
-          const float *rr = red + (warp * T + lane) * 33;
-          float tot = rr[0];
-          for (int c = 1; c < nch; ++c) tot = fadd(tot, rr[c]);
-          ysm[(size_t)(pos_base + i0 + lane) * a.rows_max + m] = tot;
-        }
-        __syncwarp();
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty + s);
-  }
-  named_sync(1, 256);
-  if (*reinterpret_cast<volatile int *>(&s_abort)) return;
-  for (int i = tid; i < T * nrows; i += 256) {
-    const int t = i / nrows, m = i % nrows;
-    float o = ysm[(size_t)(T * K + t) * a.rows_max + m];
-    for (int s = 0; s < K; ++s) {
-      const int p = a.pos[t * K + s];
-      o = ffma(a.w[t * K + s], ysm[(size_t)p * a.rows_max + m], o);
-    }
-    a.out[(size_t)t * H + m0 + m] = o;
-  }
-  if (a.use_pdl) pdl_launch_dependents();
-}
-
-size_t down_smem_bytes(int H, int I, int k, int T, int rows_max, int rs, int nstage) {
-  (void)H;
-  return dn_plan(I, k, T, rows_max, rs, nstage).total;
-}
-
-int down_max_stages(int H, int I, int k, int T, int rows_max, int rs) {
-  int ns = 6;
-  while (ns >= 2 && down_smem_bytes(H, I, k, T, rows_max, rs, ns) > (size_t)kMaxSmem) --ns;
-  return ns;
-}
-
-template <int CSZ>
-static cudaError_t launch_dn(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_down_decode<CSZ>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (err != cudaSuccess) return err;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(288);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = a.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_down_decode<CSZ>, a);
-}
-
-cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
-  const int csz = (a.I / 64 + 31) / 32;
-  switch (csz) {
-    case 1: return launch_dn<1>(a, grid, smem, s);
-    case 2: return launch_dn<2>(a, grid, smem, s);
-    default: return cudaErrorInvalidValue;
-  }
 }
 
 }  // namespace moe

@@ -160,6 +160,24 @@ def make_layer(w: Workload, layer: int = 0, device="cpu", T: int | None = None):
     return x, wr, blobs
 
 
+def chain_next(x, out, gamma: float = 0.5, zipf: bool = False):
+    """Input of the next stacked layer (workload glue between layers, not part
+    of the MoE layer): v = x + gamma * out / rms(out); x_next = v / rms(v); the
+    constant bias feature of the Zipf workloads is kept at 1.  NumPy float32 on
+    the host, so every consumer of a stacked workload derives the same inputs."""
+    import numpy as np
+    x = np.asarray(x, np.float32)
+    out = np.asarray(out, np.float32)
+    ro = np.sqrt(np.mean(out.astype(np.float64) ** 2, axis=-1, keepdims=True)).astype(np.float32)
+    ro = np.where(ro > 0, ro, np.float32(1.0))
+    v = (x + np.float32(gamma) * out / ro).astype(np.float32)
+    rv = np.sqrt(np.mean(v.astype(np.float64) ** 2, axis=-1, keepdims=True) + 1e-12).astype(np.float32)
+    nx = (v / rv).astype(np.float32)
+    if zipf:
+        nx[..., 0] = 1.0
+    return nx
+
+
 def shrink(w: Workload, **kw) -> Workload:
     """Same workload with some fields replaced (smaller parity cases)."""
     d = {f: getattr(w, f) for f in w.__dataclass_fields__}
