@@ -18,7 +18,9 @@
 // LOP3 per word (low nibbles masked as values 0..15, high nibbles masked in
 // place as 16x their value) and run dp4a (unsigned x signed bytes) per
 // 32-block; the offset-binary bias and the 16x are folded into the integer
-// accumulator's start value, so each block sum is exact.
+// accumulator's start value, so each block sum is exact.  Tile shapes are
+// compile-time and every ring / unit index advances incrementally: the
+// per-stage bookkeeping is a handful of instructions.
 //
 // Fixed order of the fp32 part (the layer's definition, shared with any CPU
 // restatement): per 64-group a = S0*d0, b = fma(S1, d1, a), chunk acc =
@@ -47,7 +49,7 @@ __device__ __forceinline__ float chunk_dot(const uint32_t (&w)[CSZ][8], const fl
 #pragma unroll
   for (int gi = 0; gi < CSZ; ++gi) {
     if (c0 + gi < G) {
-      int s0 = z[gi][0], s1 = z[gi][1], t0 = 0, t1 = 0;   // two chains per block
+      int s0 = z[gi][0], s1 = z[gi][1], t0 = 0, t1 = 0;  // two chains per block
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         s0 = dp4a_us(w[gi][j] & 0x0F0F0F0Fu, act[gi][j], s0);
@@ -55,8 +57,8 @@ __device__ __forceinline__ float chunk_dot(const uint32_t (&w)[CSZ][8], const fl
         s1 = dp4a_us(w[gi][j] & 0xF0F0F0F0u, act[gi][8 + j], s1);
         t1 = dp4a_us(w[gi][4 + j] & 0xF0F0F0F0u, act[gi][12 + j], t1);
       }
-      s0 += t0;   // sum (u - 8) q over the low nibbles (block 2g)
-      s1 += t1;   // 16 * sum (u - 8) q over the high nibbles (block 2g+1)
+      s0 += t0;  // sum (u - 8) q over the low nibbles (block 2g)
+      s1 += t1;  // 16 * sum (u - 8) q over the high nibbles (block 2g+1)
       const float fa = fmul((float)s0, d[gi][0]);
       const float fb = ffma(fmul((float)s1, 0.0625f), d[gi][1], fa);  // (float)s1/16 is exact
       acc = ffma(sc[gi], fb, acc);
@@ -75,6 +77,58 @@ __device__ __forceinline__ float chunk_sum(const float *rr, int nch) {
   for (int c = 1; c < 32; ++c)
     if (c < nch) tot = fadd(tot, v[c]);
   return tot;
+}
+
+// Weight words and scales of one row's chunk (CSZ groups) from shared memory.
+template <int CSZ>
+__device__ __forceinline__ void load_row(const unsigned char *rowp, const __half *scp, int c0, int G,
+                                         uint32_t (&w)[CSZ][8], float (&sc)[CSZ]) {
+#pragma unroll
+  for (int gi = 0; gi < CSZ; ++gi) {
+    const int g = c0 + gi;
+    if (g < G) {
+      const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
+      const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
+      w[gi][0] = w0.x;
+      w[gi][1] = w0.y;
+      w[gi][2] = w0.z;
+      w[gi][3] = w0.w;
+      w[gi][4] = w1.x;
+      w[gi][5] = w1.y;
+      w[gi][6] = w1.z;
+      w[gi][7] = w1.w;
+      sc[gi] = __half2float(scp[g]);
+    } else {
+#pragma unroll
+      for (int z = 0; z < 8; ++z) w[gi][z] = 0u;
+      sc[gi] = 0.0f;
+    }
+  }
+}
+
+// Activation chunk (CSZ groups) of one token: 16 words, 2 scales and the two
+// integer start values per group.
+template <int CSZ>
+__device__ __forceinline__ void load_act(const unsigned char *xa, const float *xd, const int *qs,
+                                         int c0, int G, uint32_t (&act)[CSZ][16], float (&d)[CSZ][2],
+                                         int (&z)[CSZ][2]) {
+#pragma unroll
+  for (int gi = 0; gi < CSZ; ++gi) {
+    const int g = c0 + gi;
+    const uint4 *src = reinterpret_cast<const uint4 *>(xa + 64 * gi);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint4 v = src[q];
+      act[gi][4 * q] = v.x;
+      act[gi][4 * q + 1] = v.y;
+      act[gi][4 * q + 2] = v.z;
+      act[gi][4 * q + 3] = v.w;
+    }
+    d[gi][0] = g < G ? xd[2 * g] : 0.0f;
+    d[gi][1] = g < G ? xd[2 * g + 1] : 0.0f;
+    z[gi][0] = g < G ? -8 * qs[2 * g] : 0;
+    z[gi][1] = g < G ? -128 * qs[2 * g + 1] : 0;
+  }
 }
 
 // ===========================================================================
@@ -107,13 +161,19 @@ __host__ __device__ inline GuPlan gu_plan(int H, int T, int R, int ns, int csz) 
   return p;
 }
 
-template <int CSZ, bool ONE>
+// Work unit = (union slot, 32-row block of I); slot 0 is the shared expert,
+// slot u >= 1 is uni[u-1]; units are split evenly over the CTAs.  A stage is
+// R gate rows + R up rows (packed nibbles + fp16 scales).  Consumer warp w
+// owns rows w and w+8 of the stage (R = 8: gate row w and up row w) or row w
+// (R = 4).
+template <int CSZ, bool ONE, int R>
 __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
+  constexpr int SPU = 32 / R;  // stages per 32-row unit
+  constexpr int RPW = R / 4;   // rows per warp per stage
   extern __shared__ __align__(128) unsigned char smem[];
-  const int H = a.H, I = a.I, T = a.T, NS = a.nstage, R = a.rpm;
+  const int H = a.H, I = a.I, T = a.T, NS = a.nstage;
   const int G = H / 64, HB = H / 32;
   const int nch = (G + CSZ - 1) / CSZ;
-  const int SPU = 32 / R;  // stages per 32-row unit
   const GuPlan pl = gu_plan(H, T, R, NS, CSZ);
   uint64_t *full = reinterpret_cast<uint64_t *>(smem);
   uint64_t *empty = full + NS;
@@ -191,18 +251,21 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const uint32_t pk = (uint32_t)R * (H / 2), sk = (uint32_t)R * (H / 32);
-      int issued = 0;
+      int s = 0, issued = 0;
+      uint32_t ph = 0;
+      int slot = u_begin / rbs, rb = u_begin % rbs, st = 0;
+      const unsigned char *blob = nullptr;
+      int blob_slot = -1;
       for (int j = 0; j < n_stages; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetGuEmpty)) {
+        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetGuEmpty)) {
           s_abort = 1;
           break;
         }
         if (*reinterpret_cast<volatile int *>(&s_abort)) break;
-        const int unit = u_begin + j / SPU, st = j % SPU;
-        const int slot = unit / rbs, rb = unit % rbs;
-        const int e = slot == 0 ? a.E : a.uni[slot - 1];
-        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
+        if (slot != blob_slot) {
+          blob_slot = slot;
+          blob = reinterpret_cast<const unsigned char *>(a.table[slot == 0 ? a.E : a.uni[slot - 1]]);
+        }
         const size_t n0 = (size_t)rb * 32 + (size_t)st * R;
         unsigned char *dst = stg + (size_t)s * pl.sb;
         mbar_arrive_expect_tx(full + s, 2 * (pk + sk));
@@ -212,6 +275,17 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
         bulk_g2s_hint(dst + 2 * pk + sk, blob + mg + (size_t)I * (H / 2) + n0 * (H / 32), sk,
                       full + s, pol);
         issued = j + 1;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++st == SPU) {
+          st = 0;
+          if (++rb == rbs) {
+            rb = 0;
+            ++slot;
+          }
+        }
       }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
         mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetGuDrain);
@@ -221,39 +295,26 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
 
   // ---------------------------------------------------------------- consumers
   const int c0 = lane * CSZ;
-  const int RPW = R / 4;  // rows per warp per stage: 1 (R = 4) or 2 (R = 8)
   // single token: this lane's activation chunk stays in registers
   uint32_t act1[CSZ][16];
   float d1[CSZ][2];
-  int q1[CSZ][2];
-  if (ONE) {
+  int z1[CSZ][2];
+  if (ONE) load_act<CSZ>(xq_s + (size_t)lane * pl.chp, xd_s, qs_s, c0, G, act1, d1, z1);
+  // this warp's rows of a stage
+  int row_m[RPW], row_r[RPW];
 #pragma unroll
-    for (int gi = 0; gi < CSZ; ++gi) {
-      const int g = c0 + gi;
-      const uint4 *src = reinterpret_cast<const uint4 *>(xq_s + (size_t)lane * pl.chp + 64 * gi);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 v = src[q];
-        act1[gi][4 * q] = v.x;
-        act1[gi][4 * q + 1] = v.y;
-        act1[gi][4 * q + 2] = v.z;
-        act1[gi][4 * q + 3] = v.w;
-      }
-      d1[gi][0] = g < G ? xd_s[2 * g] : 0.0f;
-      d1[gi][1] = g < G ? xd_s[2 * g + 1] : 0.0f;
-      q1[gi][0] = g < G ? -8 * qs_s[2 * g] : 0;
-      q1[gi][1] = g < G ? -128 * qs_s[2 * g + 1] : 0;
-    }
+  for (int q = 0; q < RPW; ++q) {
+    const int jr = warp + 8 * q;
+    row_m[q] = jr / R;
+    row_r[q] = jr % R;
   }
 
-  int cur_unit = -1, n_tok = 0, pos_base = 0, my_tok = 0;
+  int n_tok = 0, pos_base = 0, my_tok = 0;
+  int slot = u_begin / rbs, rb = u_begin % rbs, st = 0, s = 0;
+  uint32_t ph = 0;
   bool bad = false;
   for (int j = 0; j < n_stages; ++j) {
-    const int s = j % NS;
-    const int unit = u_begin + j / SPU, st = j % SPU;
-    const int slot = unit / rbs, rb = unit % rbs;
-    if (unit != cur_unit) {
-      cur_unit = unit;
+    if (st == 0) {  // a new unit: its expert's token list
       if (slot == 0) {
         n_tok = T;
         pos_base = T * a.k;
@@ -267,61 +328,33 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     }
     if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
     if (!bad) {
-      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetGuFull);
+      bad = !mbar_wait(full + s, ph, a.status, kDetGuFull);
       bad = __any_sync(0xffffffffu, bad);
       if (bad && lane == 0) s_abort = 1;
     }
     if (!bad) {
       const unsigned char *sb = stg + (size_t)s * pl.sb;
-      uint32_t wv[2][CSZ][8];
-      float sc[2][CSZ];
+      uint32_t wv[RPW][CSZ][8];
+      float sc[RPW][CSZ];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        if (q < RPW) {
-          const int jr = warp + 8 * q;
-          const int m = jr / R, r = jr % R;
-          const unsigned char *rowp = sb + (size_t)m * R * (H / 2) + (size_t)r * (H / 2);
-          const __half *scp = reinterpret_cast<const __half *>(
-              sb + (size_t)R * H + (size_t)m * R * (H / 32) + (size_t)r * (H / 32));
-#pragma unroll
-          for (int gi = 0; gi < CSZ; ++gi) {
-            const int g = c0 + gi;
-            if (g < G) {
-              const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
-              const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
-              wv[q][gi][0] = w0.x;
-              wv[q][gi][1] = w0.y;
-              wv[q][gi][2] = w0.z;
-              wv[q][gi][3] = w0.w;
-              wv[q][gi][4] = w1.x;
-              wv[q][gi][5] = w1.y;
-              wv[q][gi][6] = w1.z;
-              wv[q][gi][7] = w1.w;
-              sc[q][gi] = __half2float(scp[g]);
-            } else {
-#pragma unroll
-              for (int z = 0; z < 8; ++z) wv[q][gi][z] = 0u;
-              sc[q][gi] = 0.0f;
-            }
-          }
-        }
-      }
+      for (int q = 0; q < RPW; ++q)
+        load_row<CSZ>(sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2),
+                      reinterpret_cast<const __half *>(sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) +
+                                                       (size_t)row_r[q] * (H / 32)),
+                      c0, G, wv[q], sc[q]);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
       if (ONE) {
-        // chunk values of the warp's 8 rows of the unit are summed once per unit
+        // chunk values of the warp's 8 rows of the unit, summed once per unit
 #pragma unroll
-        for (int q = 0; q < 2; ++q)
-          if (q < RPW)
-            red[(warp * 8 + st * RPW + q) * 33 + lane] =
-                chunk_dot<CSZ>(wv[q], sc[q], act1, d1, q1, c0, G);
+        for (int q = 0; q < RPW; ++q)
+          red[(warp * 8 + st * RPW + q) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act1, d1, z1, c0, G);
         if (st == SPU - 1) {
           __syncwarp();
           if (lane < 8) {
             const int sq = lane / RPW, q = lane % RPW;
             const int jr = warp + 8 * q;
-            const int m = jr / R, r = jr % R;
-            gu[m * 32 + sq * R + r] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
+            gu[(jr / R) * 32 + sq * R + jr % R] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
           }
           __syncwarp();
         }
@@ -330,38 +363,18 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
           const int t = __shfl_sync(0xffffffffu, my_tok, i);
           uint32_t act[CSZ][16];
           float dd[CSZ][2];
-          int qq[CSZ][2];
+          int zz[CSZ][2];
+          load_act<CSZ>(xq_s + (size_t)(t * 32 + lane) * pl.chp, xd_s + t * HB, qs_s + t * HB, c0, G,
+                        act, dd, zz);
 #pragma unroll
-          for (int gi = 0; gi < CSZ; ++gi) {
-            const int g = c0 + gi;
-            const uint4 *src =
-                reinterpret_cast<const uint4 *>(xq_s + (size_t)(t * 32 + lane) * pl.chp + 64 * gi);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 v = src[q];
-              act[gi][4 * q] = v.x;
-              act[gi][4 * q + 1] = v.y;
-              act[gi][4 * q + 2] = v.z;
-              act[gi][4 * q + 3] = v.w;
-            }
-            dd[gi][0] = g < G ? xd_s[t * HB + 2 * g] : 0.0f;
-            dd[gi][1] = g < G ? xd_s[t * HB + 2 * g + 1] : 0.0f;
-            qq[gi][0] = g < G ? -8 * qs_s[t * HB + 2 * g] : 0;
-            qq[gi][1] = g < G ? -128 * qs_s[t * HB + 2 * g + 1] : 0;
-          }
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-            if (q < RPW)
-              red[((warp * 2 + q) * T + i) * 33 + lane] =
-                  chunk_dot<CSZ>(wv[q], sc[q], act, dd, qq, c0, G);
+          for (int q = 0; q < RPW; ++q)
+            red[((warp * 2 + q) * T + i) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act, dd, zz, c0, G);
         }
         __syncwarp();
         if (lane < RPW * n_tok) {
           const int q = lane / n_tok, i = lane % n_tok;
           const int jr = warp + 8 * q;
-          const int m = jr / R, r = jr % R;
-          const float tot = chunk_sum(red + ((warp * 2 + q) * T + i) * 33, nch);
-          gu[(i * 2 + m) * 32 + st * R + r] = tot;
+          gu[(i * 2 + jr / R) * 32 + st * R + jr % R] = chunk_sum(red + ((warp * 2 + q) * T + i) * 33, nch);
         }
         __syncwarp();
       }
@@ -389,6 +402,17 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
       named_sync(1, 256);
     }
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+    if (++st == SPU) {
+      st = 0;
+      if (++rb == rbs) {
+        rb = 0;
+        ++slot;
+      }
+    }
   }
   if (a.use_pdl) pdl_launch_dependents();
 }
@@ -413,9 +437,9 @@ void gateup_plan(int H, int T, int *R, int *nstage) {
   }
 }
 
-template <int CSZ, bool ONE>
+template <int CSZ, bool ONE, int R>
 static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_gateup_decode<CSZ, ONE>,
+  cudaError_t err = cudaFuncSetAttribute(k_gateup_decode<CSZ, ONE, R>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -428,22 +452,37 @@ static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStr
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ, ONE>, a);
+  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ, ONE, R>, a);
+}
+
+template <int CSZ>
+static cudaError_t launch_gu_csz(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
+  const bool one = a.T == 1;
+  if (a.rpm == 8)
+    return one ? launch_gu<CSZ, true, 8>(a, grid, smem, s) : launch_gu<CSZ, false, 8>(a, grid, smem, s);
+  return one ? launch_gu<CSZ, true, 4>(a, grid, smem, s) : launch_gu<CSZ, false, 4>(a, grid, smem, s);
 }
 
 cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
-  const bool one = a.T == 1;
+  if (a.rpm != 4 && a.rpm != 8) return cudaErrorInvalidValue;
   switch (gu_csz(a.H)) {
-    case 1: return one ? launch_gu<1, true>(a, grid, smem, s) : launch_gu<1, false>(a, grid, smem, s);
-    case 2: return one ? launch_gu<2, true>(a, grid, smem, s) : launch_gu<2, false>(a, grid, smem, s);
-    case 3: return one ? launch_gu<3, true>(a, grid, smem, s) : launch_gu<3, false>(a, grid, smem, s);
-    case 4: return one ? launch_gu<4, true>(a, grid, smem, s) : launch_gu<4, false>(a, grid, smem, s);
+    case 1: return launch_gu_csz<1>(a, grid, smem, s);
+    case 2: return launch_gu_csz<2>(a, grid, smem, s);
+    case 3: return launch_gu_csz<3>(a, grid, smem, s);
+    case 4: return launch_gu_csz<4>(a, grid, smem, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
 // ===========================================================================
 // down + combine
+//
+// CTA c owns output rows [m0, m1) (balanced, in row groups of rg rows so every
+// scale copy is a multiple of 16 bytes) and loops over the union slots; one
+// stage = that slot's rows (or a sub-range of RS rows when the whole range
+// does not fit three stages).  y per (position, row) stays in shared memory;
+// the combine out = y_shared, then fmaf(w_s, y_s, out) in slot order, runs in
+// the same CTA at the end (deterministic, no atomics).
 // ===========================================================================
 constexpr int kDnTokBatch = 4;
 
@@ -476,7 +515,7 @@ __host__ __device__ inline DnPlan dn_plan(int I, int k, int T, int rows_max, int
   return p;
 }
 
-template <int CSZ>
+template <int CSZ, bool ONE>
 __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   extern __shared__ __align__(128) unsigned char smem[];
   const int H = a.H, I = a.I, T = a.T, K = a.k, NS = a.nstage, RS = a.rs;
@@ -535,6 +574,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   const float *hd_b = a.preload ? reinterpret_cast<const float *>(act_s + (size_t)P * I) : a.hd;
   const int *hqs_b =
       a.preload ? reinterpret_cast<const int *>(act_s + (size_t)P * I + (size_t)P * IB * 4) : a.hqs;
+  const int n_st = nslot * nsub;
 
   if (warp == 8) {
     if (lane == 0) {
@@ -546,25 +586,33 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
         bulk_g2s(act_s + bq, a.hd, bd, actbar);
         bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
       }
-      int issued = 0;
-      for (int j = 0; j < nslot * nsub; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(empty + s, ((j / NS) - 1) & 1, a.status, kDetDnEmpty)) {
+      int s = 0, issued = 0, slot = 0, sub = 0;
+      uint32_t ph = 0;
+      for (int j = 0; j < n_st; ++j) {
+        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetDnEmpty)) {
           s_abort = 1;
           break;
         }
         if (*reinterpret_cast<volatile int *>(&s_abort)) break;
-        const int slot = j / nsub, r0 = (j % nsub) * RS;
+        const int r0 = sub * RS;
         const int nr = min(RS, nrows - r0);
         const uint32_t bytes_pk = (uint32_t)nr * (I / 2), bytes_sc = (uint32_t)nr * (I / 32);
-        const int e = slot == 0 ? a.E : a.uni[slot - 1];
-        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[e]);
+        const unsigned char *blob =
+            reinterpret_cast<const unsigned char *>(a.table[slot == 0 ? a.E : a.uni[slot - 1]]);
         unsigned char *dst = stg + (size_t)s * pl.sb;
         mbar_arrive_expect_tx(full + s, bytes_pk + bytes_sc);
         bulk_g2s_hint(dst, blob + pk_off + (size_t)(m0 + r0) * (I / 2), bytes_pk, full + s, pol);
         bulk_g2s_hint(dst + sc_in_stage, blob + sc_off + (size_t)(m0 + r0) * (I / 32), bytes_sc,
                       full + s, pol);
         issued = j + 1;
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1u;
+        }
+        if (++sub == nsub) {
+          sub = 0;
+          ++slot;
+        }
       }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
         mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
@@ -581,9 +629,10 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     bad = __any_sync(0xffffffffu, bad);
     if (bad && lane == 0) s_abort = 1;
   }
-  for (int j = 0; j < nslot * nsub; ++j) {
-    const int s = j % NS;
-    const int slot = j / nsub, r0 = (j % nsub) * RS;
+  int s = 0, slot = 0, sub = 0;
+  uint32_t ph = 0;
+  for (int j = 0; j < n_st; ++j) {
+    const int r0 = sub * RS;
     const int nr = min(RS, nrows - r0);
     int n_tok, pos_base;
     if (slot == 0) {
@@ -596,101 +645,88 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     }
     if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
     if (!bad) {
-      bad = !mbar_wait(full + s, (j / NS) & 1, a.status, kDetDnFull);
+      bad = !mbar_wait(full + s, ph, a.status, kDetDnFull);
       bad = __any_sync(0xffffffffu, bad);
       if (bad && lane == 0) s_abort = 1;
     }
-    if (bad) continue;
-    const unsigned char *sb = stg + (size_t)s * pl.sb;
-    // this warp's rows of the stage: a contiguous block
-    const int rpw = (nr + 7) / 8;
-    const int ra = min(nr, warp * rpw), rz = min(nr, ra + rpw);
-    for (int i0 = 0; i0 < n_tok; i0 += kDnTokBatch) {
-      const int nb = min(kDnTokBatch, n_tok - i0);
-      uint32_t av[kDnTokBatch][CSZ][16];
-      float dv[kDnTokBatch][CSZ][2];
-      int qv[kDnTokBatch][CSZ][2];
-#pragma unroll
-      for (int b = 0; b < kDnTokBatch; ++b) {
-        const int pos = pos_base + (b < nb ? i0 + b : i0);
-#pragma unroll
-        for (int gi = 0; gi < CSZ; ++gi) {
-          const int g = c0 + gi;
-          if (b < nb && g < G) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(hq_b + (size_t)pos * I + 64 * g);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 v = src[q];
-              av[b][gi][4 * q + 0] = v.x;
-              av[b][gi][4 * q + 1] = v.y;
-              av[b][gi][4 * q + 2] = v.z;
-              av[b][gi][4 * q + 3] = v.w;
-            }
-            dv[b][gi][0] = hd_b[(size_t)pos * IB + 2 * g];
-            dv[b][gi][1] = hd_b[(size_t)pos * IB + 2 * g + 1];
-            qv[b][gi][0] = -8 * hqs_b[(size_t)pos * IB + 2 * g];
-            qv[b][gi][1] = -128 * hqs_b[(size_t)pos * IB + 2 * g + 1];
-          } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) av[b][gi][q] = 0u;
-            dv[b][gi][0] = dv[b][gi][1] = 0.0f;
-            qv[b][gi][0] = qv[b][gi][1] = 0;
-          }
-        }
-      }
-      const bool last_batch = i0 + kDnTokBatch >= n_tok;
-      // rows in passes so that (row, token) pairs fit the 32 lanes of the sum
-      const int ppass = 32 / nb;
-      for (int p0 = ra; p0 < rz; p0 += ppass) {
-        const int p1 = min(rz, p0 + ppass);
-        for (int ml = p0; ml < p1; ++ml) {
-          const unsigned char *rowp = sb + (size_t)ml * (I / 2);
-          const __half *scp = reinterpret_cast<const __half *>(sb + sc_in_stage + (size_t)ml * (I / 32));
+    if (!bad) {
+      const unsigned char *sb = stg + (size_t)s * pl.sb;
+      // this warp's rows of the stage: a contiguous block
+      const int rpw = (nr + 7) >> 3;
+      const int ra = min(nr, warp * rpw), rz = min(nr, ra + rpw);
+      if (ONE) {
+        // one pair per slot: activation chunk in registers for the stage
+        uint32_t av[CSZ][16];
+        float dv[CSZ][2];
+        int zv[CSZ][2];
+        load_act<CSZ>(hq_b + (size_t)pos_base * I + 64 * c0, hd_b + (size_t)pos_base * IB,
+                      hqs_b + (size_t)pos_base * IB, c0, G, av, dv, zv);
+        for (int ml = ra; ml < rz; ++ml) {
           uint32_t wv[CSZ][8];
           float sc[CSZ];
+          load_row<CSZ>(sb + (size_t)ml * (I / 2),
+                        reinterpret_cast<const __half *>(sb + sc_in_stage + (size_t)ml * (I / 32)), c0,
+                        G, wv, sc);
+          redw[(ml - ra) * 33 + lane] = chunk_dot<CSZ>(wv, sc, av, dv, zv, c0, G);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);
+        if (lane < rz - ra)
+          ysm[(size_t)pos_base * a.rows_max + r0 + ra + lane] = chunk_sum(redw + lane * 33, nch);
+        __syncwarp();
+      } else {
+        for (int i0 = 0; i0 < n_tok; i0 += kDnTokBatch) {
+          const int nb = min(kDnTokBatch, n_tok - i0);
+          uint32_t av[kDnTokBatch][CSZ][16];
+          float dv[kDnTokBatch][CSZ][2];
+          int zv[kDnTokBatch][CSZ][2];
 #pragma unroll
-          for (int gi = 0; gi < CSZ; ++gi) {
-            const int g = c0 + gi;
-            if (g < G) {
-              const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
-              const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
-              wv[gi][0] = w0.x;
-              wv[gi][1] = w0.y;
-              wv[gi][2] = w0.z;
-              wv[gi][3] = w0.w;
-              wv[gi][4] = w1.x;
-              wv[gi][5] = w1.y;
-              wv[gi][6] = w1.z;
-              wv[gi][7] = w1.w;
-              sc[gi] = __half2float(scp[g]);
-            } else {
-#pragma unroll
-              for (int z = 0; z < 8; ++z) wv[gi][z] = 0u;
-              sc[gi] = 0.0f;
-            }
+          for (int b = 0; b < kDnTokBatch; ++b) {
+            const int pos = pos_base + (b < nb ? i0 + b : i0);
+            load_act<CSZ>(hq_b + (size_t)pos * I + 64 * c0, hd_b + (size_t)pos * IB,
+                          hqs_b + (size_t)pos * IB, c0, G, av[b], dv[b], zv[b]);
           }
+          const bool last_batch = i0 + kDnTokBatch >= n_tok;
+          // rows in passes so that (row, token) pairs fit the 32 lanes of the sum
+          const int ppass = 32 / nb;
+          for (int p0 = ra; p0 < rz; p0 += ppass) {
+            const int p1 = min(rz, p0 + ppass);
+            for (int ml = p0; ml < p1; ++ml) {
+              uint32_t wv[CSZ][8];
+              float sc[CSZ];
+              load_row<CSZ>(sb + (size_t)ml * (I / 2),
+                            reinterpret_cast<const __half *>(sb + sc_in_stage + (size_t)ml * (I / 32)),
+                            c0, G, wv, sc);
 #pragma unroll
-          for (int b = 0; b < kDnTokBatch; ++b)
-            if (b < nb)
-              redw[((ml - p0) * nb + b) * 33 + lane] =
-                  chunk_dot<CSZ>(wv, sc, av[b], dv[b], qv[b], c0, G);
+              for (int b = 0; b < kDnTokBatch; ++b)
+                if (b < nb)
+                  redw[((ml - p0) * nb + b) * 33 + lane] = chunk_dot<CSZ>(wv, sc, av[b], dv[b], zv[b], c0, G);
+            }
+            if (last_batch && p1 == rz) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(empty + s);  // every row of this warp is read
+            }
+            __syncwarp();
+            if (lane < (p1 - p0) * nb) {
+              const int ml = p0 + lane / nb, b = lane % nb;
+              ysm[(size_t)(pos_base + i0 + b) * a.rows_max + r0 + ml] = chunk_sum(redw + lane * 33, nch);
+            }
+            __syncwarp();
+          }
+          if (last_batch && ra >= rz) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);  // this warp had no rows
+          }
         }
-        if (last_batch && p1 == rz) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(empty + s);  // every row of this warp is read
-        }
-        __syncwarp();
-        if (lane < (p1 - p0) * nb) {
-          const int ml = p0 + lane / nb, b = lane % nb;
-          const float tot = chunk_sum(redw + lane * 33, nch);
-          ysm[(size_t)(pos_base + i0 + b) * a.rows_max + r0 + ml] = tot;
-        }
-        __syncwarp();
       }
-      if (last_batch && ra >= rz) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty + s);  // this warp had no rows
-      }
+    }
+    if (++s == NS) {
+      s = 0;
+      ph ^= 1u;
+    }
+    if (++sub == nsub) {
+      sub = 0;
+      ++slot;
     }
   }
   named_sync(1, 256);
@@ -698,9 +734,9 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   for (int i = tid; i < T * nrows; i += 256) {
     const int t = i / nrows, m = i % nrows;
     float o = ysm[(size_t)(T * K + t) * a.rows_max + m];
-    for (int s = 0; s < K; ++s) {
-      const int p = a.pos[t * K + s];
-      o = ffma(a.w[t * K + s], ysm[(size_t)p * a.rows_max + m], o);
+    for (int q = 0; q < K; ++q) {
+      const int p = a.pos[t * K + q];
+      o = ffma(a.w[t * K + q], ysm[(size_t)p * a.rows_max + m], o);
     }
     a.out[(size_t)t * H + m0 + m] = o;
   }
@@ -720,9 +756,9 @@ int down_max_stages(int H, int I, int k, int T, int rows_max, int rs) {
   return ns;
 }
 
-template <int CSZ>
+template <int CSZ, bool ONE>
 static cudaError_t launch_dn(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_down_decode<CSZ>,
+  cudaError_t err = cudaFuncSetAttribute(k_down_decode<CSZ, ONE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -735,14 +771,15 @@ static cudaError_t launch_dn(const DownArgs &a, int grid, size_t smem, cudaStrea
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_down_decode<CSZ>, a);
+  return cudaLaunchKernelEx(&cfg, k_down_decode<CSZ, ONE>, a);
 }
 
 cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
   const int csz = (a.I / 64 + 31) / 32;
+  const bool one = a.T == 1;
   switch (csz) {
-    case 1: return launch_dn<1>(a, grid, smem, s);
-    case 2: return launch_dn<2>(a, grid, smem, s);
+    case 1: return one ? launch_dn<1, true>(a, grid, smem, s) : launch_dn<1, false>(a, grid, smem, s);
+    case 2: return one ? launch_dn<2, true>(a, grid, smem, s) : launch_dn<2, false>(a, grid, smem, s);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -224,49 +224,148 @@ __device__ void bucket_warp(int E, int k, int T, const int32_t *idx, int *s_work
 }
 
 // =====================================================================
-// Top-k of one token's logits by one warp (E <= 1024, k <= 32): lane s ends
-// holding slot s (expert, logit).  Ties go to the lower expert index.
+// The same counting sort for P = T*k <= 32 pairs, in registers: lane p holds
+// pair p; its position is the number of pairs before it in (expert, pair id)
+// order; counts, offsets and the union follow from comparisons.
 // =====================================================================
-__device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &e_sel,
-                                          float &l_sel) {
-  float v[32];
-  const int nper = (E + 31) >> 5;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (j < nper && e < E) ? __ldcg(lg + e) : 0.0f;
+__device__ void bucket_small(int E, int k, int T, const int32_t *idx, int32_t *cnt, int32_t *off,
+                             int32_t *uni, int32_t *n_uni, int32_t *perm, int32_t *pos,
+                             int32_t *pair_tok) {
+  const int lane = threadIdx.x & 31;
+  const int P = T * k;
+  const int ep = lane < P ? idx[lane] : INT_MAX;
+  int rank = 0, first = 1, below = 0;  // below: distinct experts smaller than ep
+  for (int q = 0; q < P; ++q) {
+    const int eq = __shfl_sync(0xffffffffu, ep, q);
+    rank += (eq < ep || (eq == ep && q < lane)) ? 1 : 0;
+    if (eq == ep && q < lane) first = 0;
   }
-  unsigned taken = 0u;
+  // distinct experts below ep: pairs q that are the first of their expert
+  const int fl = (lane < P) ? first : 0;
+  for (int q = 0; q < P; ++q) {
+    const int eq = __shfl_sync(0xffffffffu, ep, q);
+    const int fq = __shfl_sync(0xffffffffu, fl, q);
+    below += (fq && eq < ep) ? 1 : 0;
+  }
+  const int nu = __reduce_add_sync(0xffffffffu, (unsigned)fl);
+  if (lane < P) {
+    perm[rank] = lane;
+    if (pos) pos[lane] = rank;
+    if (pair_tok) pair_tok[rank] = lane / k;
+    if (first) uni[below] = ep;
+  }
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int e = e0 + lane;
+    int c = 0, o = 0;
+    for (int q = 0; q < P; ++q) {
+      const int eq = __shfl_sync(0xffffffffu, ep, q);
+      c += eq == e ? 1 : 0;
+      o += eq < e ? 1 : 0;
+    }
+    if (e < E) {
+      cnt[e] = c;
+      off[e] = o;
+    }
+  }
+  if (lane == 0) {
+    off[E] = P;
+    *n_uni = nu;
+    uni[nu] = E;
+  }
+  if (pair_tok)
+    for (int t = lane; t < T; t += 32) pair_tok[P + t] = t;
+}
+
+// =====================================================================
+// Top-k of one token's logits by one warp (E <= 1024, k <= 32): lane s ends
+// holding slot s (expert, logit); ties go to the lower expert index.
+// Selection by a bitwise radix search for the k-th largest logit: logits map
+// to order-preserving unsigned keys (-0 taken as +0 so that equal values tie);
+// 32 halving steps with a warp-wide count (redux) find the k-th largest key;
+// every key above it is kept, and keys equal to it are taken in ascending
+// expert index until k are kept; the kept k are then ranked by (logit
+// descending, index ascending).  scratch: 96 words of shared memory per warp.
+// =====================================================================
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v == 0.0f) v = 0.0f;  // -0 == +0
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+template <int NPER>
+__device__ __forceinline__ void warp_topk_radix(const float *lg, int E, int k, int lane, int &e_sel,
+                                                float &l_sel, uint32_t *scratch) {
+  float v[NPER];
+  uint32_t key[NPER];
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = e < E ? __ldcg(lg + e) : 0.0f;
+    key[j] = e < E ? order_key(v[j]) : 0u;  // absent entries never reach the top k (k <= E)
+  }
+  uint32_t pre = 0u;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = pre | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int j = 0; j < NPER; ++j) c += (lane + 32 * j < E && key[j] >= cand) ? 1 : 0;
+    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) pre = cand;
+  }
+  // pre = k-th largest key: keep > pre, then == pre by ascending index
+  int gt = 0;
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) gt += (lane + 32 * j < E && key[j] > pre) ? 1 : 0;
+  const int need = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+  const unsigned lt = (1u << lane) - 1u;
+  int eq_before = 0, sel_before = 0;
+  uint32_t *s_key = scratch, *s_e = scratch + 32;
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) {
+    const int e = lane + 32 * j;
+    const bool valid = e < E;
+    const bool eq = valid && key[j] == pre;
+    const unsigned beq = __ballot_sync(0xffffffffu, eq);
+    const bool keep = valid && (key[j] > pre || (eq && eq_before + __popc(beq & lt) < need));
+    eq_before += __popc(beq);
+    const unsigned bk = __ballot_sync(0xffffffffu, keep);
+    if (keep) {
+      const int at = sel_before + __popc(bk & lt);  // compaction in index order
+      s_key[at] = key[j];
+      s_e[at] = (uint32_t)e;
+    }
+    sel_before += __popc(bk);
+  }
+  __syncwarp();
   e_sel = 0;
   l_sel = 0.0f;
-  for (int s = 0; s < k; ++s) {
-    float bv = 0.0f;
-    int be = INT_MAX;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int e = lane + 32 * j;
-      if (j < nper && e < E && !((taken >> j) & 1u)) {
-        if (be == INT_MAX || v[j] > bv) {
-          bv = v[j];
-          be = e;
-        }
-      }
+  if (lane < k) {
+    const uint32_t mk = s_key[lane];
+    const int me = (int)s_e[lane];
+    int rank = 0;
+    for (int i = 0; i < k; ++i) {
+      const uint32_t ok = s_key[i];
+      const int oe = (int)s_e[i];
+      rank += (ok > mk || (ok == mk && oe < me)) ? 1 : 0;
     }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-      if (oe != INT_MAX && (be == INT_MAX || ov > bv || (ov == bv && oe < be))) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (lane == s) {
-      e_sel = be;
-      l_sel = bv;
-    }
+    scratch[64 + rank] = (uint32_t)me;
   }
+  __syncwarp();
+  if (lane < k) {
+    e_sel = (int)scratch[64 + lane];
+    l_sel = __ldcg(lg + e_sel);
+  }
+  __syncwarp();
+}
+
+__device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &e_sel,
+                                          float &l_sel, uint32_t *scratch) {
+  const int nper = (E + 31) >> 5;
+  if (nper <= 1) warp_topk_radix<1>(lg, E, k, lane, e_sel, l_sel, scratch);
+  else if (nper <= 2) warp_topk_radix<2>(lg, E, k, lane, e_sel, l_sel, scratch);
+  else if (nper <= 4) warp_topk_radix<4>(lg, E, k, lane, e_sel, l_sel, scratch);
+  else if (nper <= 8) warp_topk_radix<8>(lg, E, k, lane, e_sel, l_sel, scratch);
+  else if (nper <= 16) warp_topk_radix<16>(lg, E, k, lane, e_sel, l_sel, scratch);
+  else warp_topk_radix<32>(lg, E, k, lane, e_sel, l_sel, scratch);
 }
 
 // softmax over the k kept logits held one per lane; writes idx / w of token t.
@@ -317,23 +416,16 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
     fence_barrier_init();
     issue(0);
   }
-  if (a.do_quant) {
-    const int64_t nblk = (int64_t)a.T * (H / 32);
-    for (int64_t b = (int64_t)blockIdx.x * 4 + warp; b < nblk; b += (int64_t)gridDim.x * 4) {
-      const float v = a.x[b * 32 + lane];
-      const float d = fdiv(warp_max(fabsf(v)), 127.0f);
-      a.xq[b * 32 + lane] = (int8_t)q8_code(v, d);
-      if (lane == 0) a.xd[b] = d;
-    }
-  }
   __syncthreads();
+  const int HB = H / 32;
   int phase = 0;
   for (int t0 = 0; t0 < a.T; t0 += a.tt, ++phase) {
     const int nt = min(a.tt, a.T - t0);
     if (tid == 0 && t0 > 0) issue(t0);
     const bool ok = __syncthreads_and(mbar_wait(bar, phase & 1, a.status, kDetRouteBar));
     if (!ok) return;
-    for (int p = warp; p < ne * nt; p += 4) {
+    const int npair = ne * nt;
+    for (int p = warp; p < npair; p += 4) {
       const int ei = p / nt, ti = p % nt;
       const float *wv = sW + (size_t)ei * H;
       const float *xv = sX + (size_t)ti * H;
@@ -343,6 +435,19 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
 #pragma unroll
       for (int off = 16; off >= 1; off >>= 1) acc = fadd(acc, __shfl_xor_sync(0xffffffffu, acc, off));
       if (lane == 0) a.logits[(size_t)(t0 + ti) * a.E + e0 + ei] = acc;
+    }
+    if (a.do_quant) {
+      // Q8_0 of this tile's x from the staged copy: block b of the tile goes
+      // to CTA b mod grid, on the warps after the logit work
+      const int nblk = nt * HB;
+      int q = (warp - npair % 4 + 4) % 4;  // spread: idle warps first
+      for (int b = blockIdx.x + (int)gridDim.x * q; b < nblk; b += (int)gridDim.x * 4) {
+        const float v = sX[(size_t)b * 32 + lane];
+        const float d = fdiv(warp_max(fabsf(v)), 127.0f);
+        const size_t gb = (size_t)t0 * HB + b;
+        a.xq[gb * 32 + lane] = (int8_t)q8_code(v, d);
+        if (lane == 0) a.xd[gb] = d;
+      }
     }
     __syncthreads();
   }
@@ -357,23 +462,28 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   __threadfence();
   int *s_idx = reinterpret_cast<int *>(sW);               // [T*k]
   int *s_work = s_idx + kDecodeTMax * kMaxK;              // bucket scratch
+  uint32_t *s_tk = reinterpret_cast<uint32_t *>(s_work + 3 * MOE_MAX_E + 64);  // [4][96]
   for (int t = warp; t < a.T; t += 4) {
     int e_sel;
     float l_sel;
-    warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, lane, e_sel, l_sel);
+    warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, lane, e_sel, l_sel, s_tk + warp * 96);
     warp_softmax_store(t, a.k, lane, e_sel, l_sel, a.idx, a.w, a.route_counts, s_idx);
   }
   __syncthreads();
   if (warp != 0) return;
-  if (a.do_bucket)
-    bucket_warp(a.E, a.k, a.T, s_idx, s_work, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos,
-                a.pair_tok);
+  if (a.do_bucket) {
+    if (a.T * a.k <= 32)
+      bucket_small(a.E, a.k, a.T, s_idx, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos, a.pair_tok);
+    else
+      bucket_warp(a.E, a.k, a.T, s_idx, s_work, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos,
+                  a.pair_tok);
+  }
   if (lane == 0) *a.done = 0u;
 }
 
 size_t route_smem_bytes(int H, int epc, int tt) {
   size_t fl = (size_t)(epc + tt) * H * 4;
-  size_t need_tail = (size_t)(kDecodeTMax * kMaxK + 3 * MOE_MAX_E + 64) * 4;
+  size_t need_tail = (size_t)(kDecodeTMax * kMaxK + 3 * MOE_MAX_E + 64 + 4 * 96) * 4;
   return 128 + (fl > need_tail ? fl : need_tail);
 }
 
@@ -392,12 +502,13 @@ cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s) {
 // =====================================================================
 __global__ void __launch_bounds__(256) k_topk(const float *logits, int T, int E, int k, int32_t *idx,
                                              float *w, int32_t *counts) {
+  __shared__ uint32_t s_tk[8][96];
   const int lane = threadIdx.x & 31;
   const int t = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if (t >= T) return;
   int e_sel;
   float l_sel;
-  warp_topk(logits + (size_t)t * E, E, k, lane, e_sel, l_sel);
+  warp_topk(logits + (size_t)t * E, E, k, lane, e_sel, l_sel, s_tk[threadIdx.x >> 5]);
   warp_softmax_store(t, k, lane, e_sel, l_sel, idx, w, counts, nullptr);
 }
 
