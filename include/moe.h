@@ -152,6 +152,28 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
                            void *ws, size_t ws_bytes, int32_t *route_counts_opt, int32_t path,
                            void *stream);
 
+/* moe_layer_forward without a caller workspace.  (No counterpart in the
+ * source pages: this is an interface convenience of this library.)
+ * For callers that cannot call cudaMalloc -- code that runs inside a host
+ * which owns and budgets all device memory, or latency-critical paths that
+ * must not allocate once they are running -- the workspace lives in the
+ * library itself: one statically allocated device array of
+ * MOE_STATIC_WS_BYTES (4 MiB) per GPU that loads the library, held until the
+ * process exits.  Arguments as moe_layer_forward.  The call allocates
+ * nothing.  Its first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before capturing any stream into a graph.  Batches whose workspace
+ * (moe_workspace_bytes) exceeds MOE_STATIC_WS_BYTES are refused with
+ * MOE_ERR_WORKSPACE and a message on stderr (for H=6144, I=2048, E=256,
+ * k=8 every T <= 16 fits).  All calls share the one array and each call
+ * leaves its intermediates there (the call resets what must start at zero);
+ * calls whose work overlaps on the GPU, e.g. on two streams at once, race on
+ * it and give wrong results. */
+#define MOE_STATIC_WS_BYTES (4u << 20)
+int moe_layer_forward_static(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                             const void *const *expert_table, float *out, int32_t *route_counts_opt,
+                             int32_t path, void *stream);
+
 /* The layer in two halves, for callers that must place the experts between
  * routing and the FFN (the tiered cache below):
  *   moe_layer_route:   Q8_0 of x, router + top-k + softmax, batch union into ws

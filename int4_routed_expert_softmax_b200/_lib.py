@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "moe_bucket": (ctypes.c_int, [D, i32, P, P, P, P, P, P, P]),
             "moe_layer_forward": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
             "moe_layer_forward_host": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
+            "moe_layer_forward_static": (ctypes.c_int, [D, i32, P, P, P, P, P, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -155,6 +156,14 @@ def moe_layer_forward_host(d: MoeDims, x_host, Wr, table, out_host, ws, route_co
     _check("moe_layer_forward_host", lib().moe_layer_forward_host(
         ctypes.byref(d), x_host.shape[0], _ptr(x_host), _ptr(Wr), _ptr(table), _ptr(out_host),
         _ptr(ws), ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
+
+
+def moe_layer_forward_static(d: MoeDims, x, Wr, table, out, route_counts=None,
+                             path: int = MOE_PATH_AUTO, stream=None):
+    """moe_layer_forward on the library's static device workspace (no allocation)."""
+    _check("moe_layer_forward_static", lib().moe_layer_forward_static(
+        ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(route_counts),
+        path, _stream(stream)))
 
 
 def moe_workspace_view(d: MoeDims, T: int, ws: torch.Tensor) -> MoeWsView:
