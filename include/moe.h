@@ -95,8 +95,14 @@ int moe_check_dims(const moe_dims *dims);
 size_t moe_expert_bytes(const moe_dims *dims);
 
 /* Device workspace needed by moe_layer_forward for batches of up to T_max
- * tokens (256-byte aligned segments).  0 if the dims are not accepted. */
+ * tokens on the path MOE_PATH_AUTO picks for T_max (256-byte aligned
+ * segments).  0 if the dims are not accepted. */
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max);
+
+/* Same for an explicit path: MOE_PATH_PREFILL needs the prefill segments (the
+ * fp16 activation codes and the per-pair down rows, about T*(k+1)*H*4 bytes)
+ * for any T; MOE_PATH_DECODE never does. */
+size_t moe_workspace_bytes_path(const moe_dims *dims, int32_t T_max, int32_t path);
 
 /* Q8_0 quantisation of rows x T x cols fp32 (cols % 32 == 0):
  * q [rows][cols] int8, d [rows][cols/32] fp32.  Bit-exact definition above.
@@ -127,18 +133,31 @@ int moe_router_topk(const moe_dims *dims, int32_t T, const float *x, const float
 int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt,
                int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm, void *stream);
 
-/* The whole layer on T tokens:
+/* The whole layer on T tokens.
+ * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): GEMV kernels that
+ * stream each union expert's bytes once per 16 tokens, every fp32 step in the
+ * layer's fixed order -- bit-identical to the CPU definition.
+ * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
+ * union on the tensor cores (exact 32-block integer sums, scales applied in
+ * fp32 in another order) and the combine; within the layer's float tolerance
+ * of the definition, the routing (idx, w, cnt, off, uni, perm) and the Q8_0
+ * codes of x still bit-exact.  (Batched expert unions: colibri deep review
+ * page, technology table, row I/O 即引擎; prefill GEMM order: tantan.ink
+ * page, section 我看到的几个坑.)
+ * Arguments:
  *   x [T][H] fp32 (the normalised hidden state; no residual, no norm here),
  *   Wr [E][H] fp32,
  *   expert_table: DEVICE array of E+1 device pointers to expert blobs;
  *                 entry E is the shared expert (weight 1),
  *   out [T][H] fp32 = shared(x) + sum_s w[t,s] * expert_{idx[t,s]}(x),
- *   ws / ws_bytes: device workspace of at least moe_workspace_bytes(dims, T),
+ *   ws / ws_bytes: device workspace of at least moe_workspace_bytes_path(dims,
+ *                  T, path),
  *                  256-byte aligned; holds every intermediate (see view),
  *   route_counts_opt [E] int32 or NULL (incremented per selection),
  *   path: enum moe_path.
  * Every step runs in the library's kernels; nothing is synchronised with the
- * host.  Results do not depend on the path. */
+ * host.  Device-side failures (a bounded wait that ran out, a misaligned
+ * blob) are written to the workspace status word (see moe_ws_view). */
 int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
                       const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
                       int32_t *route_counts_opt, int32_t path, void *stream);

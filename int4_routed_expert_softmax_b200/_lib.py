@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
             "moe_check_dims": (ctypes.c_int, [D]),
             "moe_expert_bytes": (sz, [D]),
             "moe_workspace_bytes": (sz, [D, i32]),
+            "moe_workspace_bytes_path": (sz, [D, i32, i32]),
             "moe_workspace_view": (ctypes.c_int, [D, i32, P, ctypes.POINTER(MoeWsView)]),
             "moe_device_sms": (ctypes.c_int, []),
             "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -108,6 +109,10 @@ def moe_expert_bytes(d: MoeDims) -> int:
 
 def moe_workspace_bytes(d: MoeDims, T_max: int) -> int:
     return int(lib().moe_workspace_bytes(ctypes.byref(d), T_max))
+
+
+def moe_workspace_bytes_path(d: MoeDims, T_max: int, path: int) -> int:
+    return int(lib().moe_workspace_bytes_path(ctypes.byref(d), T_max, path))
 
 
 def moe_device_sms() -> int:
@@ -173,9 +178,9 @@ def moe_workspace_view(d: MoeDims, T: int, ws: torch.Tensor) -> MoeWsView:
 
 
 # ----------------------------------------------------------------- helpers
-def alloc_workspace(d: MoeDims, T_max: int, device="cuda") -> torch.Tensor:
-    """Device workspace for batches of up to T_max tokens (256-byte aligned)."""
-    n = moe_workspace_bytes(d, T_max)
+def alloc_workspace(d: MoeDims, T_max: int, device="cuda", path: int = MOE_PATH_AUTO) -> torch.Tensor:
+    """Device workspace for batches of up to T_max tokens on `path` (256-byte aligned)."""
+    n = moe_workspace_bytes_path(d, T_max, path)
     if n == 0:
         raise MoeError("moe_workspace_bytes", -2)
     ws = torch.empty(n + 256, dtype=torch.uint8, device=device)

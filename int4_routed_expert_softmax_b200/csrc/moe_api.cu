@@ -201,6 +201,83 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   return MOE_OK;
 }
 
+bool use_prefill(int T, int path) {
+  return path == MOE_PATH_PREFILL || (path == MOE_PATH_AUTO && T > kDecodeTMax);
+}
+
+// The prefill path on all T tokens at once: Q8_0 of x (int8 and fp16 codes),
+// router logits, top-k + softmax, bucketing, grouped GEMM gate/up, grouped GEMM
+// down, combine.
+int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
+                    const void *const *table, float *out, void *ws, const WsLayout &L,
+                    int32_t *counts, cudaStream_t s) {
+  const int sms = device_sms();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  int8_t *xq = at<int8_t>(ws, L.xq);
+  float *xd = at<float>(ws, L.xd);
+  float *logits = at<float>(ws, L.logits);
+  int32_t *idx = at<int32_t>(ws, L.idx);
+  float *w = at<float>(ws, L.w);
+  int32_t *status = at<int32_t>(ws, L.status);
+  prof_record(0, s);
+  QuantArgs qa{x, xq, xd, at<void>(ws, L.xh), (int64_t)T * (d.H / 32)};
+  cudaError_t err = launch_quant(qa, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  RouterTiledArgs ra{d.H, d.E, T, x, Wr, logits};
+  err = launch_router_tiled(ra, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  err = launch_topk(logits, T, d.E, d.k, idx, w, counts, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  BucketArgs ba{};
+  ba.E = d.E;
+  ba.k = d.k;
+  ba.T = T;
+  ba.idx = idx;
+  ba.cnt = at<int32_t>(ws, L.cnt);
+  ba.off = at<int32_t>(ws, L.off);
+  ba.uni = at<int32_t>(ws, L.uni);
+  ba.n_uni = at<int32_t>(ws, L.n_uni);
+  ba.perm = at<int32_t>(ws, L.perm);
+  ba.pos = at<int32_t>(ws, L.pos);
+  ba.pair_tok = at<int32_t>(ws, L.pair_tok);
+  err = launch_bucket(ba, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(1, s);
+
+  PfArgs pa{};
+  pa.mode = 0;
+  pa.H = d.H;
+  pa.I = d.I;
+  pa.E = d.E;
+  pa.k = d.k;
+  pa.T = T;
+  pa.table = table;
+  pa.uni = ba.uni;
+  pa.n_uni = ba.n_uni;
+  pa.off = ba.off;
+  pa.pair_tok = ba.pair_tok;
+  pa.bsrc = at<void>(ws, L.xh);
+  pa.bscale = xd;
+  pa.hq = at<int8_t>(ws, L.hq);
+  pa.hh = at<void>(ws, L.hh);
+  pa.hd = at<float>(ws, L.hd);
+  pa.y = at<float>(ws, L.y);
+  pa.status = status;
+  err = launch_gemm_pf(pa, sms, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(2, s);
+  pa.mode = 1;
+  pa.bsrc = pa.hh;
+  pa.bscale = pa.hd;
+  err = launch_gemm_pf(pa, sms, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  CombineArgs ca{d.H, d.k, T, pa.y, w, ba.pos, out};
+  err = launch_combine(ca, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  prof_record(3, s);
+  return MOE_OK;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -235,8 +312,13 @@ size_t moe_expert_bytes(const moe_dims *dims) {
 }
 
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max) {
+  return moe_workspace_bytes_path(dims, T_max, MOE_PATH_AUTO);
+}
+
+size_t moe_workspace_bytes_path(const moe_dims *dims, int32_t T_max, int32_t path) {
   if (moe_check_dims(dims) != MOE_OK || T_max < 0) return 0;
-  return ws_layout(*dims, T_max).total;
+  if (path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return 0;
+  return ws_layout(*dims, T_max, use_prefill(T_max, path)).total;
 }
 
 int moe_workspace_view(const moe_dims *dims, int32_t T, void *ws, moe_ws_view *v) {
@@ -295,7 +377,7 @@ int moe_quant_q8_0(const float *x, int64_t rows, int32_t cols, int8_t *q, float 
   if (rows < 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_SHAPE;
   if (rows == 0) return MOE_OK;
   if (!x || !q || !d) return MOE_ERR_BAD_ARG;
-  QuantArgs a{x, q, d, rows * (int64_t)(cols / 32)};
+  QuantArgs a{x, q, d, nullptr, rows * (int64_t)(cols / 32)};
   return cuda_status(launch_quant(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -356,12 +438,14 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   if (!x || !Wr || !expert_table || !out || !ws) return MOE_ERR_BAD_ARG;
   if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(out, 16)) return MOE_ERR_BAD_ARG;
   if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(*dims, T);
+  const bool pf = use_prefill(T, path);
+  const WsLayout L = ws_layout(*dims, T, pf);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // status word and the router's arrival counter start at zero on every call
   cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
   if (err != cudaSuccess) return cuda_status(err);
+  if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
     const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
     rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, s);
@@ -433,7 +517,8 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
   if (T == 0) return MOE_OK;
   if (!x_host || !out_host || !ws) return MOE_ERR_BAD_ARG;
   if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
-  const WsLayout L = ws_layout(*dims, T);
+  if (path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
+  const WsLayout L = ws_layout(*dims, T, use_prefill(T, path));
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float *xd = at<float>(ws, L.xin);

@@ -28,7 +28,11 @@ enum Detail : int32_t {
   kDetDnDrain = 22,
   kDetDnAlign = 23,
   kDetPfAlign = 30,
-  kDetPfWait = 31,
+  kDetPfFull = 31,
+  kDetPfEmpty = 32,
+  kDetPfAccFull = 33,
+  kDetPfAccFree = 34,
+  kDetPfDrain = 35,
 };
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -38,13 +42,14 @@ inline size_t matrix_bytes(int N, int K) {
 }
 inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matrix_bytes(H, I); }
 
-// Byte offsets of the workspace segments for batches of up to T tokens.
+// Byte offsets of the workspace segments for batches of up to T tokens.  The
+// prefill segments (xh, hh, y) are sized only when `prefill` is set.
 struct WsLayout {
   size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
-      pair_tok, hq, hqs, hd, total;
+      pair_tok, hq, hqs, hd, xh, hh, y, total;
 };
 
-inline WsLayout ws_layout(const moe_dims &d, int T) {
+inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
   WsLayout L{};
   const size_t P = (size_t)T * (size_t)(d.k + 1);
   size_t o = 0;
@@ -72,6 +77,10 @@ inline WsLayout ws_layout(const moe_dims &d, int T) {
   L.hq = seg(P * d.I);
   L.hqs = seg(P * (d.I / 32) * 4);
   L.hd = seg(P * (d.I / 32) * 4);
+  const size_t Tp = prefill ? (size_t)T : 0, Pp = prefill ? P : 0;
+  L.xh = seg(Tp * d.H * 2);
+  L.hh = seg(Pp * d.I * 2);
+  L.y = seg(Pp * d.H * 4);
   L.total = o;
   return L;
 }
@@ -80,6 +89,7 @@ struct QuantArgs {
   const float *x;
   int8_t *q;
   float *d;
+  void *qh;  // optional: the codes again as fp16 (exact small integers)
   int64_t nblk;
 };
 
@@ -137,6 +147,34 @@ struct DownArgs {
   int use_pdl;
 };
 
+// Prefill grouped GEMM over the expert union (moe_prefill.cu).  mode 0: gate/up
+// of every (slot, token) pair with SwiGLU and Q8_0 of h; mode 1: down into y.
+struct PfArgs {
+  int mode, H, I, E, k, T;
+  const void *const *table;
+  const int32_t *uni, *n_uni, *off, *pair_tok;
+  const void *bsrc;     // fp16 codes of the activations: mode 0 [T][H] (xh), mode 1 [P][I] (hh)
+  const float *bscale;  // their Q8_0 block scales: mode 0 [T][H/32], mode 1 [P][I/32]
+  int8_t *hq;           // mode 0 outputs, in pair order
+  void *hh;
+  float *hd;
+  float *y;             // mode 1 output [P][H]
+  int32_t *status;
+};
+
+struct RouterTiledArgs {
+  int H, E, T;
+  const float *x, *Wr;
+  float *logits;
+};
+
+struct CombineArgs {
+  int H, k, T;
+  const float *y, *w;
+  const int32_t *pos;
+  float *out;
+};
+
 // Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s);
 cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s);
@@ -145,6 +183,11 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
                         int32_t *counts, cudaStream_t s);
 cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s);
 cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s);
+
+cudaError_t launch_gemm_pf(const PfArgs &a, int grid, cudaStream_t s);
+cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+size_t pf_smem_bytes(int E);
 
 // Shared-memory plans (host side, moe_kernels.cu).
 size_t route_smem_bytes(int H, int epc, int tt);

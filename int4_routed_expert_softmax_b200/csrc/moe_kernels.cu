@@ -33,7 +33,9 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
   for (int64_t b = gw; b < a.nblk; b += nw) {
     const float v = a.x[b * 32 + lane];
     const float d = fdiv(warp_max(fabsf(v)), 127.0f);
-    a.q[b * 32 + lane] = (int8_t)q8_code(v, d);
+    const int c = q8_code(v, d);
+    a.q[b * 32 + lane] = (int8_t)c;
+    if (a.qh != nullptr) static_cast<__half *>(a.qh)[b * 32 + lane] = __int2half_rn(c);
     if (lane == 0) a.d[b] = d;
   }
 }

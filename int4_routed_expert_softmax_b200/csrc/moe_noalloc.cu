@@ -32,8 +32,8 @@ extern "C" int moe_layer_forward_static(const moe_dims *dims, int32_t T, const f
                                         void *stream) {
   const int rc = moe_check_dims(dims);
   if (rc != MOE_OK) return rc;
-  if (T < 0) return MOE_ERR_BAD_ARG;
-  const size_t need = moe_workspace_bytes(dims, T);
+  if (T < 0 || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
+  const size_t need = moe_workspace_bytes_path(dims, T, path);
   if (need > kStaticWsBytes) {
     std::fprintf(stderr,
                  "libmoe: moe_layer_forward_static needs %zu workspace bytes for T=%d, more than "

@@ -50,7 +50,7 @@ def gpu_layer(w: mi.Workload, x, Wr, blobs, path=0, ws=None):
     d = moe.dims(w.H, w.I, w.E, w.k)
     T = x.shape[0]
     if ws is None:
-        ws = moe.alloc_workspace(d, T)
+        ws = moe.alloc_workspace(d, T, path=path)
     table = moe.expert_table(blobs)
     out = torch.full((T, w.H), float("nan"), dtype=torch.float32, device=x.device)
     moe.moe_layer_forward(d, x, Wr, table, out, ws, path=path)
