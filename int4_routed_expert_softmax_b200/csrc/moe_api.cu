@@ -242,6 +242,12 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   ba.pair_tok = at<int32_t>(ws, L.pair_tok);
   err = launch_bucket(ba, s);
   if (err != cudaSuccess) return cuda_status(err);
+  GatherScaleArgs ga{d.H / 32, T, d.k, xd, ba.pair_tok, at<float>(ws, L.xdp)};
+  err = launch_gather_scales(ga, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  GatherRowsArgs gr{d.H, T, d.k, at<void>(ws, L.xh), ba.pair_tok, at<void>(ws, L.xg)};
+  err = launch_gather_rows(gr, s);
+  if (err != cudaSuccess) return cuda_status(err);
   prof_record(1, s);
 
   PfArgs pa{};
@@ -256,20 +262,32 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   pa.n_uni = ba.n_uni;
   pa.off = ba.off;
   pa.pair_tok = ba.pair_tok;
-  pa.bsrc = at<void>(ws, L.xh);
-  pa.bscale = xd;
+  pa.bsrc = gr.xg;
+  pa.bscale = ga.xdp;
   pa.hq = at<int8_t>(ws, L.hq);
   pa.hh = at<void>(ws, L.hh);
   pa.hd = at<float>(ws, L.hd);
+  pa.hdT = at<float>(ws, L.hdt);
   pa.y = at<float>(ws, L.y);
   pa.status = status;
-  err = launch_gemm_pf(pa, sms, s);
+  const size_t P = (size_t)T * (size_t)(d.k + 1);
+  pa.maps = at<CUtensorMap>(ws, L.maps);
+  CUtensorMap map_x, map_h, tmpl_gu, tmpl_dn;
+  err = make_f16_map(&map_x, pa.bsrc, (uint64_t)P, (uint64_t)d.H, kPfBoxRows);
+  if (err == cudaSuccess) err = make_f16_map(&map_h, pa.hh, (uint64_t)P, (uint64_t)d.I, kPfBoxRows);
+  // the templates' address is replaced per expert on the device
+  if (err == cudaSuccess) err = make_u8_map(&tmpl_gu, pa.maps, (uint64_t)d.I, (uint64_t)d.H / 2, 64);
+  if (err == cudaSuccess) err = make_u8_map(&tmpl_dn, pa.maps, (uint64_t)d.H, (uint64_t)d.I / 2, 128);
+  if (err != cudaSuccess) return cuda_status(err);
+  err = launch_make_maps(pa, tmpl_gu, tmpl_dn, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  err = launch_gemm_pf(pa, map_x, sms, s);
   if (err != cudaSuccess) return cuda_status(err);
   prof_record(2, s);
   pa.mode = 1;
   pa.bsrc = pa.hh;
-  pa.bscale = pa.hd;
-  err = launch_gemm_pf(pa, sms, s);
+  pa.bscale = pa.hdT;
+  err = launch_gemm_pf(pa, map_h, sms, s);
   if (err != cudaSuccess) return cuda_status(err);
   CombineArgs ca{d.H, d.k, T, pa.y, w, ba.pos, out};
   err = launch_combine(ca, s);

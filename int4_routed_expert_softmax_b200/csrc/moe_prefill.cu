@@ -116,7 +116,29 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
   d |= (uint64_t)1u << 46;
   return d;
 }
-// Byte offset of byte kb (0..31) of row `row` in such a 32-byte-wide slice.
+// Descriptor of a K-major operand with 128-byte swizzle (rows of 128 bytes,
+// 8-row atoms 1024 bytes apart) as a 2D TMA copy with SWIZZLE_128B writes it;
+// a K slice of 32 bytes starts 32 bytes further into the row.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// TMA: one box of a 2D tensor (64 fp16 from column x, rows y ..) into shared
+// memory; completion counted on `bar`.  x * 2 bytes is a multiple of 16.
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Byte offset of byte kb (0..31) of row `row` in a no-swizzle 32-byte-wide slice.
 __host__ __device__ __forceinline__ uint32_t il_off(int row, int kb) {
   return (uint32_t)((row >> 3) * 256 + (kb >> 4) * 128 + (row & 7) * 16 + (kb & 15));
 }
@@ -138,40 +160,47 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
   hi = *reinterpret_cast<const uint32_t *>(&hb);
 }
 
-// Bounded wait by every lane of a warp; the verdict is made warp-uniform.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t detail,
-                                          volatile int *abort_flag) {
-  const bool ok = mbar_wait(bar, parity, status, detail) && !*abort_flag;
-  return __all_sync(0xffffffffu, ok);
-}
 
 // ===========================================================================
 // grouped GEMM
+//
+// 9 warps per CTA, one CTA per SM, persistent over the CTA's stages (stage =
+// one 64-group of one tile; tiles blockIdx.x, + gridDim.x, ...).
+//   control warp (lane 0): TMA copies of the packed weights (kPfLR stages
+//     ahead, tensor maps built per expert on the device) and of the activation
+//     rows (kPfLB stages ahead); the 4 MMAs of each stage.
+//   8 worker warps, in step (one reducing barrier per stage): expand stage i's
+//     nibbles to fp16 (A buffer i & 1); cp.async the scales of stage i+kPfLD;
+//     apply the scales of stage i-1 from TMEM; write a tile's outputs after its
+//     last group.
+// Hand-offs between the two go through mbarriers; every wait is bounded.
 // ===========================================================================
-constexpr int kPfNS = 5;          // pipeline stages (one 64-group each)
-constexpr int kPfLag = 3;         // stages of copies in flight ahead of the nibble expansion
-constexpr int kPfWarps = 13;
-constexpr int kPfThreads = kPfWarps * 32;
-constexpr int kPfMmaWarp = 4;
-constexpr int kPfEpi0 = 5;
-constexpr uint32_t kPfTmemCols = 512;  // 2 buffers x 2 blocks x 128 columns
-constexpr int kUxPitch = 129;          // up-projection exchange rows (floats), odd: no bank conflicts
+constexpr int kPfWorkers = 256;
+constexpr int kPfThreads = kPfWorkers + 32;
+constexpr int kPfCtl = 8;                // control warp
+constexpr int kPfLR = 8, kPfRR = kPfLR + 1;  // packed-weight TMA: stages ahead, ring slots
+constexpr int kPfLB = 4, kPfRB = kPfLB + 2;  // activation TMA: stages ahead, ring slots
+constexpr int kPfLD = 4, kPfRD = kPfLD + 3;  // scale cp.async: stages ahead, ring slots
+constexpr uint32_t kPfTmemCols = 512;    // 2 buffers x 2 blocks x 128 columns
+constexpr int kUxPitch = 129;            // up-projection exchange rows (floats), odd: no bank conflicts
 
-// stage slot layout (bytes)
-constexpr uint32_t kSlotA = 0;         // 4 K-slices x [128 rows x 32 B] fp16 weights
-constexpr uint32_t kSlotB = 16384;     // 4 K-slices x [N rows x 32 B] fp16 activations (N <= 128)
-constexpr uint32_t kSlotRaw = 32768;   // [128 rows][32 B] packed weights of the group
-constexpr uint32_t kSlotD = 36864;     // [2 blocks][128] fp32 activation block scales
-constexpr uint32_t kSlotW = 37888;     // [128] u32: the fp16 weight scales of groups g & ~1, g | 1
-constexpr uint32_t kSlotBytes = 38400;
+constexpr uint32_t kABytes = 16384;      // 4 K-slices x [128 rows x 32 B] fp16 weights, no swizzle
+constexpr uint32_t kBBytes = 16384;      // [N rows][128 B] fp16 activations, 128-byte swizzle (N <= 128)
+constexpr uint32_t kRawBytes = 4096;     // [128 rows][32 B] packed weights of a group
+constexpr uint32_t kSclD = 512;          // scale slot: [128] u32 weight scales (groups g & ~1, g | 1),
+constexpr uint32_t kSclBytes = 1536;     //   then [2 blocks][128] fp32 activation block scales
 
 struct PfLayout {
-  uint32_t stage, ux, total;
+  uint32_t tile_pre, a, b, raw, scl, ux, total;
 };
 __host__ __device__ inline PfLayout pf_layout(int E) {
   PfLayout L;
-  L.stage = (uint32_t)((256 + 4 * (E + 2) + 1023) / 1024 * 1024);
-  L.ux = L.stage + (uint32_t)kPfNS * kSlotBytes;
+  L.tile_pre = 576;
+  L.a = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
+  L.b = L.a + 2 * kABytes;
+  L.raw = L.b + (uint32_t)kPfRB * kBBytes;
+  L.scl = L.raw + (uint32_t)kPfRR * kRawBytes;
+  L.ux = L.scl + (uint32_t)kPfRD * kSclBytes;
   L.total = L.ux + 64u * kUxPitch * 4u;
   return L;
 }
@@ -215,27 +244,55 @@ __device__ __forceinline__ PfTile pf_tile(int t, const int *tile_pre, int nslot,
   return r;
 }
 
+// A position in the CTA's stage sequence.
+struct PfCur {
+  int t, g;
+  PfTile tl;
+};
+
+// Named barrier over the 256 worker threads that also ANDs a predicate.
+__device__ __forceinline__ bool workers_sync_and(bool v) {
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.and.pred po, 1, 256, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(out)
+      : "r"((uint32_t)v)
+      : "memory");
+  return out != 0;
+}
+
+__device__ __forceinline__ void tmap_acquire(const CUtensorMap *m) {
+  asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(m) : "memory");
+}
+
 template <int MODE>
-__global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a) {
+__global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
+  // 9 warps: one SM sub-partition holds 3 of them, so at most 16K / 96 = 170 registers.
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I;
   const int K = MODE == 0 ? H : I;
   const int G = K / 64;
   const int NWT = MODE == 0 ? I / 64 : H / 128;
+  const size_t P = (size_t)a.T * (size_t)(a.k + 1);
   const PfLayout L = pf_layout(a.E);
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [NS] producers: stage written (128 arrivals)
-  uint64_t *empty = full + kPfNS;                       // [NS] MMA commit + 8 epilogue warps
-  uint64_t *accf = empty + kPfNS;                       // [2]  accumulator buffer written (MMA commit)
-  uint64_t *acce = accf + 2;                            // [2]  accumulator buffer read (8 epilogue warps)
-  uint64_t *drain = acce + 2;                           // MMA drain before teardown
-  uint64_t *uxw = drain + 1;                            // up rows handed over (8 epilogue warps)
-  uint64_t *uxr = uxw + 1;                              // up rows consumed (8 epilogue warps)
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 192);
-  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 196);
-  int *s_ntiles = reinterpret_cast<int *>(smem + 200);
-  int *tile_pre = reinterpret_cast<int *>(smem + 256);
-  unsigned char *stage = smem + L.stage;
+  uint64_t *rawfull = reinterpret_cast<uint64_t *>(smem);  // [RR] packed weights landed (TMA bytes)
+  uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (8 worker warps)
+  uint64_t *bfull = rawfree + kPfRR;                        // [RB] activation rows landed (TMA bytes)
+  uint64_t *bfree = bfull + kPfRB;                          // [RB] read by the MMAs (commit)
+  uint64_t *aready = bfree + kPfRB;                         // [2]  A buffer written (8 worker warps)
+  uint64_t *accf = aready + 2;                              // [2]  accumulators written (commit)
+  uint64_t *tfree = accf + 2;                               // [2]  accumulators read (8 worker warps)
+  uint64_t *drain = tfree + 2;                              // teardown
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
+  int *s_ntiles = reinterpret_cast<int *>(smem + 520);
+  int *tile_pre = reinterpret_cast<int *>(smem + L.tile_pre);
+  unsigned char *abuf = smem + L.a;
+  unsigned char *bbuf = smem + L.b;
+  unsigned char *raw = smem + L.raw;
+  unsigned char *scl = smem + L.scl;
   float *ux = reinterpret_cast<float *>(smem + L.ux);
 
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
@@ -244,17 +301,20 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a) {
 
   if (tid == 0) {
     *abort_flag = 0;
-    for (int s = 0; s < kPfNS; ++s) {
-      mbar_init(full + s, 128);
-      mbar_init(empty + s, 9);
+    for (int s = 0; s < kPfRR; ++s) {
+      mbar_init(rawfull + s, 1);
+      mbar_init(rawfree + s, 8);
+    }
+    for (int s = 0; s < kPfRB; ++s) {
+      mbar_init(bfull + s, 1);
+      mbar_init(bfree + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
+      mbar_init(aready + b, 8);
       mbar_init(accf + b, 1);
-      mbar_init(acce + b, 8);
+      mbar_init(tfree + b, 8);
     }
     mbar_init(drain, 1);
-    mbar_init(uxw, 8);
-    mbar_init(uxr, 8);
     fence_barrier_init();
   }
   if (warp == 0) {
@@ -286,8 +346,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a) {
       tile_pre[nslot] = run;
       *s_ntiles = run;
     }
-  }
-  if (warp == kPfMmaWarp) {
     tmem_alloc(tmem_slot, kPfTmemCols);
     tmem_relinquish();
   }
@@ -296,287 +354,378 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_tiles = *s_ntiles;
-  const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
+  const int my_tiles = blockIdx.x < (unsigned)n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int S = my_tiles * G;  // stages of this CTA
 
-  if (warp < kPfMmaWarp) {
-    // ---------------------------------------------------------------- producers
-    const int pt = tid;  // weight row of the tile this thread copies and expands
-    int st = 0, cv = 0;
-    bool bad = false;
-    auto expand = [&](int cs) {
-      unsigned char *sl = stage + (size_t)(cs % kPfNS) * kSlotBytes;
-      const uint4 q0 = *reinterpret_cast<const uint4 *>(sl + kSlotRaw + pt * 32);
-      const uint4 q1 = *reinterpret_cast<const uint4 *>(sl + kSlotRaw + pt * 32 + 16);
-#pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        // K-slice k4 holds group elements 16*k4 .. 16*k4+15: low nibbles of
-        // bytes 0..15 / 16..31, then high nibbles of the same bytes.
-        const uint4 src = (k4 & 1) ? q1 : q0;
-        const int sh = (k4 >> 1) * 4;
-        uint32_t h[8];
-        nib4_to_f16((src.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
-        nib4_to_f16((src.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
-        nib4_to_f16((src.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
-        nib4_to_f16((src.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
-        unsigned char *dst = sl + kSlotA + k4 * 4096;
-        *reinterpret_cast<uint4 *>(dst + il_off(pt, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4 *>(dst + il_off(pt, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
-      }
-      fence_proxy_async();
-      mbar_arrive(full + cs % kPfNS);
-    };
-    for (int t = blockIdx.x; t < n_tiles && !bad; t += gridDim.x) {
-      const PfTile tl = pf_tile(t, tile_pre, nslot, a);
-      const unsigned char *blob = static_cast<const unsigned char *>(a.table[tl.e]);
-      if ((reinterpret_cast<uintptr_t>(blob) & 15) != 0) {
-        set_status(a.status, MOE_ERR_DEVICE, kDetPfAlign);
-        *abort_flag = 1;
-        bad = true;
-        break;
-      }
-      const unsigned char *wrow, *srow;
-      if (MODE == 0) {
-        const size_t base = pt < 64 ? 0 : mg;
-        const size_t row = (size_t)tl.wt * 64 + (pt & 63);
-        wrow = blob + base + row * (size_t)(H / 2);
-        srow = blob + base + (size_t)I * (size_t)(H / 2) + row * (size_t)(H / 64) * 2;
-      } else {
-        const size_t base = 2 * mg;
-        const size_t row = (size_t)tl.wt * 128 + pt;
-        wrow = blob + base + row * (size_t)(I / 2);
-        srow = blob + base + (size_t)H * (size_t)(I / 2) + row * (size_t)(I / 64) * 2;
-      }
-      const __half *bsrc = static_cast<const __half *>(a.bsrc);
-      for (int g = 0; g < G; ++g) {
-        const int s = st % kPfNS;
-        const uint32_t u = (uint32_t)(st / kPfNS);
-        if (u > 0 && !mbar_wait(empty + s, (u - 1) & 1u, a.status, kDetPfEmpty)) bad = true;
-        if (bad || *abort_flag) {
-          *abort_flag = 1;
-          bad = true;
-          break;
-        }
-        unsigned char *sl = stage + (size_t)s * kSlotBytes;
-        cp_async16(sl + kSlotRaw + pt * 32, wrow + g * 32, 16);
-        cp_async16(sl + kSlotRaw + pt * 32 + 16, wrow + g * 32 + 16, 16);
-        cp_async4(sl + kSlotW + pt * 4, srow + (g & ~1) * 2, 4);
-        for (int ch = pt; ch < tl.n * 8; ch += 128) {
-          const int r = ch >> 3, cc = ch & 7;
-          const bool ok = r < tl.nval;
-          const size_t brow = ok ? (MODE == 0 ? (size_t)a.pair_tok[tl.p0 + r] : (size_t)(tl.p0 + r)) : 0;
-          cp_async16(sl + kSlotB + (cc >> 1) * (tl.n * 32) + il_off(r, (cc & 1) * 16),
-                     bsrc + brow * (size_t)K + g * 64 + cc * 8, ok ? 16u : 0u);
-        }
-        for (int r = pt; r < tl.n; r += 128) {
-          const bool ok = r < tl.nval;
-          const size_t brow = ok ? (MODE == 0 ? (size_t)a.pair_tok[tl.p0 + r] : (size_t)(tl.p0 + r)) : 0;
-          const float *src = a.bscale + brow * (size_t)(K / 32) + 2 * g;
-          float *dd = reinterpret_cast<float *>(sl + kSlotD);
-          cp_async4(dd + r, src, ok ? 4u : 0u);
-          cp_async4(dd + 128 + r, src + 1, ok ? 4u : 0u);
-        }
-        cp_async_commit();
-        ++st;
-        if (st - cv > kPfLag) {
-          cp_async_wait<kPfLag>();
-          expand(cv++);
-        }
-      }
+  auto cur_begin = [&](PfCur &c) {
+    c.t = blockIdx.x;
+    c.g = 0;
+    if (c.t < n_tiles) c.tl = pf_tile(c.t, tile_pre, nslot, a);
+  };
+  auto cur_next = [&](PfCur &c) {
+    if (++c.g == G) {
+      c.g = 0;
+      c.t += gridDim.x;
+      if (c.t < n_tiles) c.tl = pf_tile(c.t, tile_pre, nslot, a);
     }
-    cp_async_wait_all();
-    while (!bad && cv < st) expand(cv++);
-  } else if (warp == kPfMmaWarp) {
-    // ---------------------------------------------------------------- MMA issuer
+  };
+
+  if (warp == kPfCtl) {
+    // ================================================================ control
     if (lane == 0) {
-      int st = 0;
       bool bad = false;
-      for (int t = blockIdx.x; t < n_tiles && !bad; t += gridDim.x) {
-        const PfTile tl = pf_tile(t, tile_pre, nslot, a);
-        const uint32_t idesc = pf_idesc(tl.n);
-        for (int g = 0; g < G; ++g, ++st) {
-          const int s = st % kPfNS, buf = st & 1;
-          const uint32_t u = (uint32_t)(st / kPfNS), nu = (uint32_t)(st >> 1);
-          if (!mbar_wait(full + s, u & 1u, a.status, kDetPfFull) ||
-              !mbar_wait(acce + buf, (nu & 1u) ^ 1u, a.status, kDetPfAccFree) || *abort_flag) {
-            *abort_flag = 1;
-            bad = true;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(stage + (size_t)s * kSlotBytes + kSlotA);
-          const uint32_t sb = smem_u32(stage + (size_t)s * kSlotBytes + kSlotB);
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-#pragma unroll
-            for (int ks = 0; ks < 2; ++ks) {
-              const int k4 = 2 * b + ks;
-              umma_f16(tmem + (uint32_t)(buf * 256 + b * 128), umma_desc(sa + k4 * 4096),
-                       umma_desc(sb + (uint32_t)(k4 * tl.n * 32)), idesc, (uint32_t)ks);
-            }
-          umma_commit(accf + buf);
-          umma_commit(empty + s);
+      PfCur cr, cb, cm;
+      cur_begin(cr);
+      cur_begin(cb);
+      cur_begin(cm);
+      int raw_next = 0, b_next = 0, mma_next = 0, rtile = -1;
+      const CUtensorMap *m0 = nullptr, *m1 = nullptr;
+      auto issue_raw = [&]() -> bool {  // stage raw_next == cr
+        const int j = raw_next, s = j % kPfRR;
+        if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty)) return false;
+        if (cr.t != rtile) {
+          rtile = cr.t;
+          const CUtensorMap *em = a.maps + (size_t)cr.tl.e * 3;
+          m0 = MODE == 0 ? em : em + 2;
+          m1 = em + 1;
+          tmap_acquire(m0);
+          if (MODE == 0) tmap_acquire(m1);
         }
+        unsigned char *dst = raw + (size_t)s * kRawBytes;
+        mbar_arrive_expect_tx(rawfull + s, kRawBytes);
+        if (MODE == 0) {
+          tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 64, rawfull + s);
+          tma_load_2d(dst + 64 * 32, m1, cr.g * 32, cr.tl.wt * 64, rawfull + s);
+        } else {
+          tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 128, rawfull + s);
+        }
+        ++raw_next;
+        cur_next(cr);
+        return true;
+      };
+      auto issue_b = [&]() -> bool {  // stage b_next == cb
+        const int j = b_next, s = j % kPfRB;
+        if (j >= kPfRB && !mbar_wait(bfree + s, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) return false;
+        unsigned char *dst = bbuf + (size_t)s * kBBytes;
+        mbar_arrive_expect_tx(bfull + s, (uint32_t)cb.tl.n * 128u);
+        for (int i = 0; i < cb.tl.n / (int)kPfBoxRows; ++i)
+          tma_load_2d(dst + i * (int)kPfBoxRows * 128, &bmap, cb.g * 64, cb.tl.p0 + i * (int)kPfBoxRows, bfull + s);
+        ++b_next;
+        cur_next(cb);
+        return true;
+      };
+      auto issue_mma = [&]() -> bool {  // stage mma_next == cm
+        const int j = mma_next, buf = j & 1;
+        if (!mbar_wait(aready + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfFull)) return false;
+        if (!mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull)) return false;
+        if (j >= 2 && !mbar_wait(tfree + buf, (uint32_t)((j >> 1) - 1) & 1u, a.status, kDetPfAccFree)) return false;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(abuf + (size_t)buf * kABytes);
+        const uint32_t sb = smem_u32(bbuf + (size_t)(j % kPfRB) * kBBytes);
+        const uint32_t idesc = pf_idesc(cm.tl.n);
+        const uint32_t d = tmem + (uint32_t)(buf * 256);
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const int k4 = 2 * b + ks;
+            umma_f16(d + (uint32_t)(b * 128), umma_desc(sa + k4 * 4096), umma_desc_sw128(sb + (uint32_t)(k4 * 32)),
+                     idesc, (uint32_t)ks);
+          }
+        umma_commit(accf + buf);
+        umma_commit(bfree + j % kPfRB);
+        ++mma_next;
+        cur_next(cm);
+        return true;
+      };
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
+      while (!bad && raw_next < S && raw_next < kPfLR) bad = !issue_raw();
+      while (!bad && b_next < S && b_next < kPfLB) bad = !issue_b();
+      while (!bad && mma_next < S) {
+        if (raw_next < S && !issue_raw()) bad = true;
+        if (!bad && b_next < S && !issue_b()) bad = true;
+        if (!bad && !issue_mma()) bad = true;
+        if (*abort_flag) bad = true;
       }
-      if (st > 0) {  // wait for the MMAs still in flight before TMEM is released
+      if (bad) *abort_flag = 1;
+      // teardown: copies issued but not yet landed, MMAs not yet finished
+      for (int j = max(0, raw_next - kPfRR); j < raw_next; ++j)
+        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
+      for (int j = max(mma_next, b_next - kPfRB); j < b_next; ++j)
+        mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
+      if (mma_next > 0) {
         umma_commit(drain);
         mbar_wait(drain, 0, a.status, kDetPfDrain);
       }
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue
-    const int ew = warp - kPfEpi0;
-    const int q = warp & 3;      // TMEM lane quarter this warp may access
-    const int half = ew >> 2;    // its 16-column chunks: half, half + 2, ...
+    // ================================================================ workers
+    bool ok = true;
+    const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
+    // scale copies: weight scales of row tid (tid < 128), block scales of column tid & 127
+    PfCur cs;
+    cur_begin(cs);
+    const int crow = tid & 127, chalf = tid >> 7;
+    const unsigned char *srow = nullptr;
+    int stile = -1;
+    auto issue_scl = [&](int j) {  // stage j == cs
+      if (j < S) {
+        if (cs.t != stile) {
+          stile = cs.t;
+          const unsigned char *blob = static_cast<const unsigned char *>(a.table[cs.tl.e]);
+          if (MODE == 0) {
+            const size_t base = crow < 64 ? 0 : mg;
+            const size_t row = (size_t)cs.tl.wt * 64 + (crow & 63);
+            srow = blob + base + (size_t)I * (size_t)(H / 2) + row * (size_t)(H / 64) * 2;
+          } else {
+            const size_t row = (size_t)cs.tl.wt * 128 + crow;
+            srow = blob + 2 * mg + (size_t)H * (size_t)(I / 2) + row * (size_t)(I / 64) * 2;
+          }
+        }
+        unsigned char *ss = scl + (size_t)(j % kPfRD) * kSclBytes;
+        if (chalf == 0) cp_async4(ss + crow * 4, srow + (cs.g & ~1) * 2, 4);
+        if (crow < cs.tl.n) {
+          const bool v = crow < cs.tl.nval;
+          const float *src = a.bscale + (size_t)(2 * cs.g + chalf) * P + (v ? cs.tl.p0 + crow : 0);
+          cp_async4(reinterpret_cast<float *>(ss + kSclD) + chalf * 128 + crow, src, v ? 4u : 0u);
+        }
+        cur_next(cs);
+      }
+      cp_async_commit();
+    };
+    // epilogue state: TMEM lane quarter q, 16-column chunks half, half + 2, ...
+    const int q = warp & 3, half = warp >> 2;
     const int row = q * 32 + lane;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-    int st = 0, tcount = 0;
-    bool bad = false;
-    for (int t = blockIdx.x; t < n_tiles && !bad; t += gridDim.x, ++tcount) {
-      const PfTile tl = pf_tile(t, tile_pre, nslot, a);
-      const int nch = tl.n >> 4;
-      float2 acc[4][8];
+    PfCur ce;
+    cur_begin(ce);
+    float2 acc[4][8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
-      for (int g = 0; g < G; ++g, ++st) {
-        const int s = st % kPfNS, buf = st & 1;
-        const uint32_t u = (uint32_t)(st / kPfNS), nu = (uint32_t)(st >> 1);
-        if (!warp_wait(full + s, u & 1u, a.status, kDetPfFull, abort_flag) ||
-            !warp_wait(accf + buf, nu & 1u, a.status, kDetPfAccFull, abort_flag)) {
-          if (lane == 0) *abort_flag = 1;
-          bad = true;
-          break;
+      for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+
+    for (int j = 0; j < kPfLD; ++j) issue_scl(j);
+    for (int i = 0; i <= S; ++i) {
+      // a. expand stage i: row crow, bytes 16 chalf ..: K-slices chalf (low
+      //    nibbles) and 2 + chalf (high nibbles)
+      if (i < S) {
+        const bool got = __all_sync(0xffffffffu, mbar_wait(rawfull + i % kPfRR, (uint32_t)(i / kPfRR) & 1u, a.status,
+                                                            kDetPfFull));
+        if (!got) ok = false;
+        if (got) {
+          const uint4 src = *reinterpret_cast<const uint4 *>(raw + (size_t)(i % kPfRR) * kRawBytes + crow * 32 + chalf * 16);
+          unsigned char *ab = abuf + (size_t)(i & 1) * kABytes;
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int sh = hi * 4;
+            uint32_t h[8];
+            nib4_to_f16((src.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
+            nib4_to_f16((src.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
+            nib4_to_f16((src.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
+            nib4_to_f16((src.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
+            unsigned char *dst = ab + (2 * hi + chalf) * 4096;
+            *reinterpret_cast<uint4 *>(dst + il_off(crow, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4 *>(dst + il_off(crow, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+          fence_proxy_async();
         }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(aready + (i & 1));
+          mbar_arrive(rawfree + i % kPfRR);
+        }
+      }
+      // b. scale copies of stage i+kPfLD; this thread's copies of stage i-1 done
+      issue_scl(i + kPfLD);
+      cp_async_wait<kPfLD + 1>();
+      // c.
+      if (!workers_sync_and(ok && !*abort_flag)) break;
+      if (i == 0) continue;
+      // d. scales of stage i-1
+      const int j = i - 1, buf = j & 1;
+      const bool got = __all_sync(0xffffffffu, mbar_wait(accf + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfAccFull));
+      if (!got) ok = false;
+      const int nch = ce.tl.n >> 4;
+      if (got) {
         tc_fence_after();
-        const unsigned char *sl = stage + (size_t)s * kSlotBytes;
-        const uint32_t wsv = *reinterpret_cast<const uint32_t *>(sl + kSlotW + row * 4);
-        const float sg = __half2float(__ushort_as_half((unsigned short)((g & 1) ? (wsv >> 16) : (wsv & 0xFFFFu))));
+        const unsigned char *ss = scl + (size_t)(j % kPfRD) * kSclBytes;
+        const uint32_t wsv = *reinterpret_cast<const uint32_t *>(ss + row * 4);
+        const float sg = __half2float(__ushort_as_half((unsigned short)((ce.g & 1) ? (wsv >> 16) : (wsv & 0xFFFFu))));
         const float2 sg2 = make_float2(sg, sg);
-        const float *d0p = reinterpret_cast<const float *>(sl + kSlotD);
+        const float *d0p = reinterpret_cast<const float *>(ss + kSclD);
         const float *d1p = d0p + 128;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = half + 2 * i;
+        for (int ci = 0; ci < 4; ++ci) {
+          const int c = half + 2 * ci;
           if (c < nch) {
+            float4 da[4], db[4];
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              da[j4] = *reinterpret_cast<const float4 *>(d0p + c * 16 + 4 * j4);
+              db[j4] = *reinterpret_cast<const float4 *>(d1p + c * 16 + 4 * j4);
+            }
             uint32_t v0[16], v1[16];
             tmem_ld16(tq + (uint32_t)(buf * 256 + c * 16), v0);
             tmem_ld16(tq + (uint32_t)(buf * 256 + 128 + c * 16), v1);
             tmem_ld_wait();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float2 da = *reinterpret_cast<const float2 *>(d0p + c * 16 + 2 * j);
-              const float2 db = *reinterpret_cast<const float2 *>(d1p + c * 16 + 2 * j);
-              const float2 s0 = make_float2(__uint_as_float(v0[2 * j]), __uint_as_float(v0[2 * j + 1]));
-              const float2 s1 = make_float2(__uint_as_float(v1[2 * j]), __uint_as_float(v1[2 * j + 1]));
-              const float2 fb = __ffma2_rn(s1, db, __fmul2_rn(s0, da));
-              acc[i][j] = __ffma2_rn(sg2, fb, acc[i][j]);
+            for (int jj = 0; jj < 8; ++jj) {
+              const float4 &a4 = da[jj >> 1];
+              const float4 &b4 = db[jj >> 1];
+              const float2 dap = (jj & 1) ? make_float2(a4.z, a4.w) : make_float2(a4.x, a4.y);
+              const float2 dbp = (jj & 1) ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
+              const float2 s0 = make_float2(__uint_as_float(v0[2 * jj]), __uint_as_float(v0[2 * jj + 1]));
+              const float2 s1 = make_float2(__uint_as_float(v1[2 * jj]), __uint_as_float(v1[2 * jj + 1]));
+              const float2 fb = __ffma2_rn(s1, dbp, __fmul2_rn(s0, dap));
+              acc[ci][jj] = __ffma2_rn(sg2, fb, acc[ci][jj]);
             }
           }
         }
         tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(acce + buf);
-          mbar_arrive(empty + s);
-        }
       }
-      if (bad) break;
-      if (MODE == 1) {
-        float *yc = a.y + (size_t)tl.p0 * H + (size_t)tl.wt * 128 + row;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tfree + buf);
+      if (ce.g == G - 1) {
+        // the tile's outputs
+        const PfTile tl = ce.tl;
+        if (MODE == 1) {
+          float *yc = a.y + (size_t)tl.p0 * H + (size_t)tl.wt * 128 + row;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int c = half + 2 * i;
-          if (c < nch) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int col = c * 16 + 2 * j;
-              if (col < tl.nval) yc[(size_t)col * H] = acc[i][j].x;
-              if (col + 1 < tl.nval) yc[(size_t)(col + 1) * H] = acc[i][j].y;
-            }
-          }
-        }
-      } else {
-        // Rows 64..127 hold u of rows 0..63 (g): hand u over, then SwiGLU and
-        // Q8_0 of h along I (one 32-block = one warp's lanes), per token.
-        if (q >= 2) {
-          if (tcount > 0 && !warp_wait(uxr, (uint32_t)(tcount - 1) & 1u, a.status, kDetPfFull, abort_flag)) {
-            if (lane == 0) *abort_flag = 1;
-            bad = true;
-            break;
-          }
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = half + 2 * i;
+          for (int ci = 0; ci < 4; ++ci) {
+            const int c = half + 2 * ci;
             if (c < nch) {
 #pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                ux[(row - 64) * kUxPitch + c * 16 + 2 * j] = acc[i][j].x;
-                ux[(row - 64) * kUxPitch + c * 16 + 2 * j + 1] = acc[i][j].y;
+              for (int jj = 0; jj < 8; ++jj) {
+                const int col = c * 16 + 2 * jj;
+                if (col < tl.nval) yc[(size_t)col * H] = acc[ci][jj].x;
+                if (col + 1 < tl.nval) yc[(size_t)(col + 1) * H] = acc[ci][jj].y;
               }
             }
           }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(uxw);
-        if (!warp_wait(uxw, (uint32_t)tcount & 1u, a.status, kDetPfFull, abort_flag)) {
-          if (lane == 0) *abort_flag = 1;
-          bad = true;
-          break;
-        }
-        if (q < 2) {
-          const int ii = tl.wt * 64 + row;  // row of I
-          __half *hh = static_cast<__half *>(a.hh);
+        } else {
+          // Rows 64..127 hold u of rows 0..63 (g): hand u over, then SwiGLU and
+          // Q8_0 of h along I (one 32-block = one warp's lanes), per token.
+          if (q >= 2) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int c = half + 2 * i;
-            if (c < nch) {
+            for (int ci = 0; ci < 4; ++ci) {
+              const int c = half + 2 * ci;
+              if (c < nch) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int col = c * 16 + j;
-                const float gv = (j & 1) ? acc[i][j >> 1].y : acc[i][j >> 1].x;
-                const float h = swiglu(gv, ux[row * kUxPitch + col]);
-                const float d = fdiv(warp_max(fabsf(h)), 127.0f);
-                const int qv = q8_code(h, d);
-                if (col < tl.nval) {
-                  const size_t p = (size_t)(tl.p0 + col);
-                  a.hq[p * I + ii] = (int8_t)qv;
-                  hh[p * I + ii] = __int2half_rn(qv);
-                  if (lane == 0) a.hd[p * (I / 32) + ii / 32] = d;
+                for (int jj = 0; jj < 8; ++jj) {
+                  ux[(row - 64) * kUxPitch + c * 16 + 2 * jj] = acc[ci][jj].x;
+                  ux[(row - 64) * kUxPitch + c * 16 + 2 * jj + 1] = acc[ci][jj].y;
                 }
               }
             }
           }
+          workers_sync_and(true);
+          if (q < 2) {
+            // h = SiLU(g) * u and its Q8_0 codes in fast fp32 (this path is held
+            // to the layer's tolerance, not to the fixed-order bits)
+            const int ii = tl.wt * 64 + row;  // row of I
+            __half *hh = static_cast<__half *>(a.hh);
+#pragma unroll
+            for (int ci = 0; ci < 4; ++ci) {
+              const int c = half + 2 * ci;
+              if (c < nch) {
+#pragma unroll
+                for (int jj = 0; jj < 16; ++jj) {
+                  const int col = c * 16 + jj;
+                  const float gv = (jj & 1) ? acc[ci][jj >> 1].y : acc[ci][jj >> 1].x;
+                  const float h = __fdividef(gv, 1.0f + __expf(-gv)) * ux[row * kUxPitch + col];
+                  const float amax = warp_max(fabsf(h));
+                  const float d = amax * (1.0f / 127.0f);
+                  const float inv = amax > 0.0f ? __fdividef(127.0f, amax) : 0.0f;
+                  const int qv = (int)fminf(fmaxf(rintf(h * inv), -127.0f), 127.0f);
+                  if (col < tl.nval) {
+                    const size_t p = (size_t)(tl.p0 + col);
+                    a.hq[p * I + ii] = (int8_t)qv;
+                    hh[p * I + ii] = __int2half_rn(qv);
+                    if (lane == 0) {
+                      a.hd[p * (I / 32) + ii / 32] = d;
+                      a.hdT[(size_t)(ii / 32) * P + p] = d;
+                    }
+                  }
+                }
+              }
+            }
+          }
+          // the next tile's hand-over comes after at least one more worker barrier
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(uxr);
+#pragma unroll
+        for (int ci = 0; ci < 4; ++ci)
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) acc[ci][jj] = make_float2(0.0f, 0.0f);
       }
+      cur_next(ce);
     }
+    if (!ok) *abort_flag = 1;
+    cp_async_wait_all();
   }
-  // every role has left its loop; every wait above is bounded
+  // teardown: every copy and MMA of this CTA has completed (see the control warp)
   tc_fence_before();
   __syncthreads();
-  if (warp == kPfMmaWarp) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kPfTmemCols);
   }
 }
 
+// Tensor maps of the packed weights of the union's experts and the shared
+// expert, [E+1][gate, up, down], from host-encoded templates (the global
+// address patched per expert).  A blob that is not 16-byte aligned sets
+// MOE_ERR_DEVICE and gets no maps.
+__global__ void __launch_bounds__(32) k_make_maps(const PfArgs a, const __grid_constant__ CUtensorMap tgu,
+                                                 const __grid_constant__ CUtensorMap tdn, CUtensorMap *maps) {
+  const int e = blockIdx.x;
+  if (e < a.E && a.off[e + 1] == a.off[e]) return;  // not in the union
+  const unsigned char *blob = static_cast<const unsigned char *>(a.table[e]);
+  if ((reinterpret_cast<uintptr_t>(blob) & 15) != 0) {
+    if (threadIdx.x == 0) set_status(a.status, MOE_ERR_DEVICE, kDetPfAlign);
+    return;
+  }
+  const size_t mg = (size_t)a.I * (size_t)(a.H / 2) + (size_t)a.I * (size_t)(a.H / 64) * 2;
+  CUtensorMap *em = maps + (size_t)e * 3;
+  const uint32_t *sgu = reinterpret_cast<const uint32_t *>(&tgu);
+  const uint32_t *sdn = reinterpret_cast<const uint32_t *>(&tdn);
+  const int m = threadIdx.x >> 5;  // one warp: 32 words per map, three maps in turn
+  (void)m;
+  for (int mi = 0; mi < 3; ++mi) {
+    uint32_t *dst = reinterpret_cast<uint32_t *>(em + mi);
+    dst[threadIdx.x] = (mi == 2 ? sdn : sgu)[threadIdx.x];
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) {
+    for (int mi = 0; mi < 3; ++mi) {
+      const unsigned char *base = blob + (size_t)mi * mg;
+      asm volatile("tensormap.replace.tile.global_address.global.b1024.b64 [%0], %1;" ::"l"(em + mi), "l"(base)
+                   : "memory");
+    }
+    asm volatile("fence.proxy.tensormap::generic.release.gpu;" ::: "memory");
+  }
+}
+
 size_t pf_smem_bytes(int E) { return pf_layout(E).total; }
 
-cudaError_t launch_gemm_pf(const PfArgs &a, int grid, cudaStream_t s) {
+cudaError_t launch_make_maps(const PfArgs &a, const CUtensorMap &tgu, const CUtensorMap &tdn, cudaStream_t s) {
+  k_make_maps<<<a.E + 1, 32, 0, s>>>(a, tgu, tdn, const_cast<CUtensorMap *>(a.maps));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s) {
   const size_t smem = pf_layout(a.E).total;
   if (smem > (size_t)kMaxSmem) return cudaErrorInvalidConfiguration;
   cudaError_t err;
   if (a.mode == 0) {
     err = cudaFuncSetAttribute(k_gemm_pf<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a);
+    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap);
   } else {
     err = cudaFuncSetAttribute(k_gemm_pf<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a);
+    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap);
   }
   return cudaGetLastError();
 }
@@ -651,6 +800,53 @@ cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s) {
   if (err != cudaSuccess) return err;
   const dim3 grid((unsigned)((a.T + kRtTok - 1) / kRtTok), (unsigned)((a.E + kRtExp - 1) / kRtExp));
   k_router_tiled<<<grid, 256, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// x's fp16 codes in pair order: xg[p] = xh[pair_tok[p]] (the gate/up GEMM's
+// activation rows, copied by TMA boxes of consecutive rows).
+// ===========================================================================
+__global__ void __launch_bounds__(256) k_gather_rows(const GatherRowsArgs a) {
+  const int64_t P = (int64_t)a.T * (a.k + 1);
+  const int w = a.H / 8;  // 16-byte units per row
+  const int64_t n = P * w;
+  const uint4 *src = static_cast<const uint4 *>(a.xh);
+  uint4 *dst = static_cast<uint4 *>(a.xg);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t p = i / w, c = i - p * w;
+    dst[i] = src[(int64_t)a.pair_tok[p] * w + c];
+  }
+}
+
+cudaError_t launch_gather_rows(const GatherRowsArgs &a, cudaStream_t s) {
+  const int64_t n = (int64_t)a.T * (a.k + 1) * (a.H / 8);
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_gather_rows<<<(unsigned)blocks, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+// ===========================================================================
+// x's Q8_0 block scales in pair order, block-major (the gate/up GEMM copies a
+// tile's scales of one block as one contiguous run).
+// ===========================================================================
+__global__ void __launch_bounds__(256) k_gather_scales(const GatherScaleArgs a) {
+  const int64_t P = (int64_t)a.T * (a.k + 1);
+  const int64_t n = P * a.nb;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t b = i / P, p = i - b * P;
+    a.xdp[i] = a.xd[(int64_t)a.pair_tok[p] * a.nb + b];
+  }
+}
+
+cudaError_t launch_gather_scales(const GatherScaleArgs &a, cudaStream_t s) {
+  const int64_t n = (int64_t)a.T * (a.k + 1) * a.nb;
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  k_gather_scales<<<(unsigned)blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
