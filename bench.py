@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="decode", choices=["decode"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -64,6 +64,18 @@ def peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s (burst) of this machine's B200s: the prefill
+    GEMM issues tcgen05.mma kind::f16, so this is its own dtype's peak."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        for k in ("bf16_tflops", "bf16_tflops_burst"):
+            if k in d:
+                return float(d[k]), "measured"
+    return 1590.0, "fallback"
 
 
 # ----------------------------------------------------------------- clocks
@@ -337,6 +349,148 @@ def run_native(args, ws_n, rank, local):
         gpu_launches=3 * K, wall_s=round(wall, 3))
 
 
+# ----------------------------------------------------------------- prefill
+def prefill_ops(w: mi.Workload, T: int) -> float:
+    """Algorithmic int8 multiply-adds x 2 of one prefill layer: every (token,
+    slot) pair, routed and shared, through gate, up and down."""
+    return 2.0 * T * (w.k + 1) * 3 * w.H * w.I
+
+
+def run_prefill(args, ws_n, rank, local):
+    import int4_routed_expert_softmax_b200 as moe
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = mi.WORKLOADS["prefill"]
+    seed = w.seed + 1000 * rank
+    T = w.T
+    x = mi.make_x(T, w.H, mi.sub_seed(seed, 0, 1), dev, zipf=True)
+    Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), dev, zipf_s=w.zipf_s)
+    blobs = mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, 0, 3), dev)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    ws = moe.alloc_workspace(d, T, dev, path=moe.MOE_PATH_PREFILL)
+    table = moe.expert_table(blobs)
+    out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    view = moe.moe_workspace_view(d, T, ws)
+    nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
+    status_t = moe.ws_slice(ws, view.status, (4,), torch.int32)
+    stream = torch.cuda.current_stream()
+    PF = moe.MOE_PATH_PREFILL
+
+    def step():
+        moe.moe_layer_forward(d, x, Wr, table, out, ws, path=PF)
+
+    moe.moe_profile_enable(True)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if int(status_t[0].item()) != 0:
+        raise RuntimeError(f"device status {status_t.tolist()}")
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    prof = []
+    barrier(ws_n)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.zero_()
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+            prof.append(moe.moe_profile_last())
+        torch.cuda.synchronize()
+    barrier(ws_n)
+    moe.moe_profile_enable(False)
+    if int(status_t[0].item()) != 0:
+        raise RuntimeError(f"device status {status_t.tolist()}")
+    my_ms = sum(a.elapsed_time(b) for a, b in ev)
+    max_ms = allreduce_max(my_ms, ws_n)
+    ops = prefill_ops(w, T)
+    value = ops * K * ws_n / (max_ms * 1e-3) / 1e12
+    rt_ms = sum(p[0] for p in prof) / K
+    gu_ms = sum(p[1] for p in prof) / K
+    dn_ms = sum(p[2] for p in prof) / K
+    peak, src = tensor_peak()
+    gu_ops = 2.0 * T * (w.k + 1) * 2 * w.H * w.I
+    gu_tflops = gu_ops / (gu_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "k_gemm_pf<0> (gate/up)", "achieved": round(gu_tflops, 2),
+                "peak": peak, "unit": "TFLOP/s", "frac": round(gu_tflops / peak, 4), "peak_source": src,
+                "peak_dtype": "fp16/bf16 dense (the kernel's tcgen05 kind::f16)",
+                "frac_of_int8_peak": round(gu_tflops / (2 * peak), 4), "traffic": None,
+                "ops_per_launch": gu_ops, "us_per_launch": round(gu_ms * 1e3, 1)}
+    kernels = {"route+bucket+gathers": {"us": round(rt_ms * 1e3, 1)},
+               "k_gemm_pf<0> gate/up": {"us": round(gu_ms * 1e3, 1), "TFLOP/s": round(gu_tflops, 2)},
+               "k_gemm_pf<1> down + combine": {"us": round(dn_ms * 1e3, 1),
+                                               "TFLOP/s": round(2.0 * T * (w.k + 1) * w.H * w.I / (dn_ms * 1e-3) / 1e12, 2)}}
+    e2e = None
+    if not args.no_e2e:
+        xh = x.cpu().pin_memory()
+        oh = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
+        for _ in range(min(2, args.warmup)):
+            moe.moe_layer_forward_host(d, xh, Wr, table, oh, ws, path=PF)
+        torch.cuda.synchronize()
+        e_ms = 0.0
+        barrier(ws_n)
+        for _ in range(K):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            moe.moe_layer_forward_host(d, xh, Wr, table, oh, ws, path=PF)
+            b.record(stream)
+            b.synchronize()
+            e_ms += a.elapsed_time(b)
+        e_max = allreduce_max(e_ms, ws_n)
+        e2e = {"value": round(ops * K * ws_n / (e_max * 1e-3) / 1e12, 2), "unit": "TOPS",
+               "h2d_bytes_per_step": T * w.H * 4, "d2h_bytes_per_step": T * w.H * 4}
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu:
+        cpu = oracle_prefill_sample(w, x.cpu().numpy(), Wr.cpu().numpy(), lambda e: blobs[e].cpu().numpy(),
+                                    args.cpu_seconds)
+    return dict(
+        metric=METRIC, value=round(value, 2), unit="TOPS", n_gpus=ws_n, steps=K, warmup=args.warmup,
+        ms_per_step=round(max_ms / K, 4), higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="int4xint8->fp32 (exact fp16 integer operands)", data="synthetic",
+        config={"workload": "prefill: one GLM-5.2-shaped MoE layer, 2048 tokens, router biased to Zipf(1.1) "
+                            "expert popularity, grouped GEMM over the union",
+                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": T, "global_batch": T * ws_n,
+                "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step; "
+                "weights 5.2 GB > L2"},
+        union=int(nuni_t.item()), us_per_token_layer=round(max_ms / K / T * 1e3, 3),
+        roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clk.summary(),
+        gpu_launches=10 * K)
+
+
+def oracle_prefill_sample(w, x_h, Wr_h, blob_fn, budget_s: float, tokens_max: int = 64):
+    """The oracle on sampled tokens of the prefill batch, until the budget is
+    spent; returns the cpu_baseline record in TOPS (same op count per token)."""
+    import numpy as np
+
+    import oracle as orc
+    lg = orc.router_logits(x_h[:tokens_max], Wr_h)
+    idx, _ = orc.topk_softmax(lg, w.k)
+    cache = {}
+    spent, n = 0.0, 0
+    for t in range(tokens_max):
+        need = sorted(set(idx[t].tolist()) | {w.E})
+        for e in need:
+            if e not in cache:
+                cache[e] = blob_fn(e)
+        dummy = np.zeros(16, np.uint8)
+        blist = [cache.get(e, dummy) for e in range(w.E + 1)]
+        t0 = time.perf_counter()
+        orc.moe_layer_tokens(x_h, Wr_h, blist, w.H, w.I, w.E, w.k, [t])
+        spent += time.perf_counter() - t0
+        n += 1
+        if spent >= budget_s:
+            break
+    return {"value": round(prefill_ops(w, n) / spent / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+            "sample": f"{n} tokens of the prefill batch (tokens 0..{n - 1}), single-threaded C oracle, "
+                      f"{spent:.1f} s"}
+
+
 # ----------------------------------------------------------------- reference arm
 def run_reference(args, ws_n, rank):
     """The CPU oracle on a bounded sample of the same workload (rank 0 only)."""
@@ -345,6 +499,8 @@ def run_reference(args, ws_n, rank):
     import numpy as np  # noqa: F401
 
     import oracle as orc  # noqa: F401
+    if args.workload == "prefill":
+        return run_reference_prefill(args, ws_n)
     w = mi.WORKLOADS[args.workload]
     seed = w.seed
     Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), "cpu").numpy()
@@ -382,6 +538,36 @@ def run_reference(args, ws_n, rank):
         e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 
 
+def run_reference_prefill(args, ws_n):
+    w = mi.WORKLOADS["prefill"]
+    x = mi.make_x(w.T, w.H, mi.sub_seed(w.seed, 0, 1), "cpu", zipf=True).numpy()
+    Wr = mi.make_router(w.E, w.H, mi.sub_seed(w.seed, 0, 2), "cpu", zipf_s=w.zipf_s).numpy()
+    cache = {}
+
+    def blob_fn(e):
+        if e not in cache:
+            b = torch.empty(w.blob_bytes, dtype=torch.uint8)
+            mi.fill_blob(b, w.H, w.I, mi.blob_seed(mi.sub_seed(w.seed, 0, 3), e))
+            cache[e] = b.numpy()
+        return cache[e]
+
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    oracle_prefill_sample(w, x, Wr, blob_fn, 0.0, 1)  # warm-up: one token
+    recs = [oracle_prefill_sample(w, x, Wr, blob_fn, per_step, 16) for _ in range(args.steps)]
+    value = sum(r["value"] for r in recs) / len(recs)
+    cpu = {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+           "sample": recs[0]["sample"] + f"; {len(recs)} steps"}
+    return dict(
+        impl="reference", metric=METRIC, value=round(value, 6), unit="TOPS", n_gpus=ws_n, steps=args.steps,
+        warmup=args.warmup, higher_is_better=True, scaling="weak", vs_baseline=None,
+        dtype="int4xint8->fp32", data="synthetic",
+        config={"workload": "prefill: one GLM-5.2-shaped MoE layer, 2048 tokens, router biased to Zipf(1.1) "
+                            "expert popularity, grouped GEMM over the union",
+                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T},
+        cpu_baseline=cpu,
+        e2e={"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -393,7 +579,7 @@ def main():
         return
     ws_n, rank, local = dist_setup()
     try:
-        res = run_native(args, ws_n, rank, local)
+        res = run_prefill(args, ws_n, rank, local) if args.workload == "prefill" else run_native(args, ws_n, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

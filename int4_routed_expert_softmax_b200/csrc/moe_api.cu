@@ -267,27 +267,28 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   pa.hq = at<int8_t>(ws, L.hq);
   pa.hh = at<void>(ws, L.hh);
   pa.hd = at<float>(ws, L.hd);
-  pa.hdT = at<float>(ws, L.hdt);
   pa.y = at<float>(ws, L.y);
   pa.status = status;
   const size_t P = (size_t)T * (size_t)(d.k + 1);
   pa.maps = at<CUtensorMap>(ws, L.maps);
-  CUtensorMap map_x, map_h, tmpl_gu, tmpl_dn;
+  CUtensorMap map_x, map_h, map_dx, map_dh, tmpl_gu, tmpl_dn;
   err = make_f16_map(&map_x, pa.bsrc, (uint64_t)P, (uint64_t)d.H, kPfBoxRows);
   if (err == cudaSuccess) err = make_f16_map(&map_h, pa.hh, (uint64_t)P, (uint64_t)d.I, kPfBoxRows);
+  if (err == cudaSuccess) err = make_f32x4_map(&map_dx, ga.xdp, (uint64_t)P, (uint64_t)d.H / 32, kPfBoxRows);
+  if (err == cudaSuccess) err = make_f32x4_map(&map_dh, pa.hd, (uint64_t)P, (uint64_t)d.I / 32, kPfBoxRows);
   // the templates' address is replaced per expert on the device
   if (err == cudaSuccess) err = make_u8_map(&tmpl_gu, pa.maps, (uint64_t)d.I, (uint64_t)d.H / 2, 64);
   if (err == cudaSuccess) err = make_u8_map(&tmpl_dn, pa.maps, (uint64_t)d.H, (uint64_t)d.I / 2, 128);
   if (err != cudaSuccess) return cuda_status(err);
   err = launch_make_maps(pa, tmpl_gu, tmpl_dn, s);
   if (err != cudaSuccess) return cuda_status(err);
-  err = launch_gemm_pf(pa, map_x, sms, s);
+  err = launch_gemm_pf(pa, map_x, map_dx, sms, s);
   if (err != cudaSuccess) return cuda_status(err);
   prof_record(2, s);
   pa.mode = 1;
   pa.bsrc = pa.hh;
-  pa.bscale = pa.hdT;
-  err = launch_gemm_pf(pa, map_h, sms, s);
+  pa.bscale = pa.hd;
+  err = launch_gemm_pf(pa, map_h, map_dh, sms, s);
   if (err != cudaSuccess) return cuda_status(err);
   CombineArgs ca{d.H, d.k, T, pa.y, w, ba.pos, out};
   err = launch_combine(ca, s);

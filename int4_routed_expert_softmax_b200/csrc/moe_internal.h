@@ -47,7 +47,7 @@ inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matri
 // prefill segments (xh, hh, y) are sized only when `prefill` is set.
 struct WsLayout {
   size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
-      pair_tok, hq, hqs, hd, xh, xg, xdp, hh, hdt, y, maps, total;
+      pair_tok, hq, hqs, hd, xh, xg, xdp, hh, y, maps, total;
 };
 
 inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
@@ -83,7 +83,6 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
   L.xg = seg(Pp * d.H * 2);
   L.xdp = seg(Pp * (d.H / 32) * 4);
   L.hh = seg(Pp * d.I * 2);
-  L.hdt = seg(Pp * (d.I / 32) * 4);
   L.y = seg(Pp * d.H * 4);
   L.maps = seg(prefill ? (size_t)(d.E + 1) * 3 * 128 : 0);
   L.total = o;
@@ -159,17 +158,16 @@ struct PfArgs {
   const void *const *table;
   const int32_t *uni, *n_uni, *off, *pair_tok;
   const void *bsrc;     // fp16 codes of the activations: mode 0 [T][H] (xh), mode 1 [P][I] (hh)
-  const float *bscale;  // their Q8_0 block scales, block-major in pair order: mode 0 [H/32][P], mode 1 [I/32][P]
+  const float *bscale;  // their Q8_0 block scales in pair order: mode 0 [P][H/32] (xdp), mode 1 [P][I/32] (hd)
   int8_t *hq;           // mode 0 outputs, in pair order
   void *hh;
   float *hd;            // [P][I/32]
-  float *hdT;           // [I/32][P] (the down GEMM's scales)
   float *y;             // mode 1 output [P][H]
   const CUtensorMap *maps;  // [E+1][gate, up, down] tensor maps of the packed weights (device)
   int32_t *status;
 };
 
-// x's block scales gathered into pair order, block-major: xdp[b][p] = xd[pair_tok[p]][b].
+// x's block scales gathered into pair order: xdp[p][b] = xd[pair_tok[p]][b].
 struct GatherScaleArgs {
   int nb, T, k;
   const float *xd;
@@ -207,10 +205,13 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
 cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s);
 cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s);
 
-cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s);
+cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUtensorMap &dmap, int grid, cudaStream_t s);
 // 2D tensor map over a row-major fp16 matrix [rows][cols] for TMA copies of
 // boxes of 64 columns x box_rows rows with 128-byte swizzle (moe_tma.cpp).
 cudaError_t make_f16_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+// 2D tensor map over a row-major fp32 matrix [rows][cols] for boxes of 4 columns x
+// box_rows rows, no swizzle (moe_tma.cpp).
+cudaError_t make_f32x4_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // Template for the packed-weight maps: a uint8 matrix [rows][cols] (cols = K/2),
 // boxes of 32 bytes x box_rows rows, no swizzle (moe_tma.cpp).
 cudaError_t make_u8_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);

@@ -165,33 +165,34 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
 // grouped GEMM
 //
 // 9 warps per CTA, one CTA per SM, persistent over the CTA's stages (stage =
-// one 64-group of one tile; tiles blockIdx.x, + gridDim.x, ...).
-//   control warp (lane 0): TMA copies of the packed weights (kPfLR stages
-//     ahead, tensor maps built per expert on the device) and of the activation
-//     rows (kPfLB stages ahead); the 4 MMAs of each stage.
-//   8 worker warps, in step (one reducing barrier per stage): expand stage i's
-//     nibbles to fp16 (A buffer i & 1); cp.async the scales of stage i+kPfLD;
-//     apply the scales of stage i-1 from TMEM; write a tile's outputs after its
-//     last group.
-// Hand-offs between the two go through mbarriers; every wait is bounded.
+// one 64-group of one tile; tiles blockIdx.x, + gridDim.x, ...; a tile has an
+// even number of stages).
+//   copy warp (lane 0): TMA copies of the packed weights (tensor maps built
+//     per expert on the device), of the activation rows and of their block
+//     scales, as far ahead as the rings allow;
+//   MMA warp (lane 0): the 4 MMAs of each stage.
+//   8 worker warps, each at its own pace: expand stage i's nibbles to fp16
+//     (A buffer i & 1), then apply the scales of stage i-1 to the TMEM block
+//     sums and write a tile's outputs after its last group.
+// Every hand-off is an mbarrier; every wait is bounded.
 // ===========================================================================
 constexpr int kPfWorkers = 256;
-constexpr int kPfThreads = kPfWorkers + 32;
-constexpr int kPfCtl = 8;                // control warp
+constexpr int kPfThreads = kPfWorkers + 64;
+constexpr int kPfTmaWarp = 8;                // issues the TMA copies
+constexpr int kPfMmaWarp = 9;                // issues the MMAs
 constexpr int kPfLR = 8, kPfRR = kPfLR + 1;  // packed-weight TMA: stages ahead, ring slots
 constexpr int kPfLB = 4, kPfRB = kPfLB + 2;  // activation TMA: stages ahead, ring slots
-constexpr int kPfLD = 4, kPfRD = kPfLD + 3;  // scale cp.async: stages ahead, ring slots
-constexpr uint32_t kPfTmemCols = 512;    // 2 buffers x 2 blocks x 128 columns
-constexpr int kUxPitch = 129;            // up-projection exchange rows (floats), odd: no bank conflicts
+constexpr int kPfRD = 4;                     // block-scale ring slots (one per stage pair)
+constexpr uint32_t kPfTmemCols = 512;        // 2 buffers x 2 blocks x 128 columns
+constexpr int kUxPitch = 129;                // up-projection exchange rows (floats), odd: no bank conflicts
 
-constexpr uint32_t kABytes = 16384;      // 4 K-slices x [128 rows x 32 B] fp16 weights, no swizzle
-constexpr uint32_t kBBytes = 16384;      // [N rows][128 B] fp16 activations, 128-byte swizzle (N <= 128)
-constexpr uint32_t kRawBytes = 4096;     // [128 rows][32 B] packed weights of a group
-constexpr uint32_t kSclD = 512;          // scale slot: [128] u32 weight scales (groups g & ~1, g | 1),
-constexpr uint32_t kSclBytes = 1536;     //   then [2 blocks][128] fp32 activation block scales
+constexpr uint32_t kABytes = 16384;   // 4 K-slices x [128 rows x 32 B] fp16 weights, no swizzle
+constexpr uint32_t kBBytes = 16384;   // [N rows][128 B] fp16 activations, 128-byte swizzle (N <= 128)
+constexpr uint32_t kRawBytes = 4096;  // [128 rows][32 B] packed weights of a group
+constexpr uint32_t kDBytes = 2048;    // [N rows][4] fp32 block scales of a stage pair
 
 struct PfLayout {
-  uint32_t tile_pre, a, b, raw, scl, ux, total;
+  uint32_t tile_pre, a, b, raw, d, ux, total;
 };
 __host__ __device__ inline PfLayout pf_layout(int E) {
   PfLayout L;
@@ -199,8 +200,8 @@ __host__ __device__ inline PfLayout pf_layout(int E) {
   L.a = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
   L.b = L.a + 2 * kABytes;
   L.raw = L.b + (uint32_t)kPfRB * kBBytes;
-  L.scl = L.raw + (uint32_t)kPfRR * kRawBytes;
-  L.ux = L.scl + (uint32_t)kPfRD * kSclBytes;
+  L.d = L.raw + (uint32_t)kPfRR * kRawBytes;
+  L.ux = L.d + (uint32_t)kPfRD * kDBytes;
   L.total = L.ux + 64u * kUxPitch * 4u;
   return L;
 }
@@ -250,32 +251,20 @@ struct PfCur {
   PfTile tl;
 };
 
-// Named barrier over the 256 worker threads that also ANDs a predicate.
-__device__ __forceinline__ bool workers_sync_and(bool v) {
-  uint32_t out;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\tbar.red.and.pred po, 1, 256, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(out)
-      : "r"((uint32_t)v)
-      : "memory");
-  return out != 0;
-}
-
 __device__ __forceinline__ void tmap_acquire(const CUtensorMap *m) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(m) : "memory");
 }
 
 template <int MODE>
-__global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
-  // 9 warps: one SM sub-partition holds 3 of them, so at most 16K / 96 = 170 registers.
+__global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap,
+                                           const __grid_constant__ CUtensorMap dmap) {
+  // 10 warps: one SM sub-partition holds 3 of them, so at most 16K / 96 = 170 registers.
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I;
   const int K = MODE == 0 ? H : I;
   const int G = K / 64;
   const int NWT = MODE == 0 ? I / 64 : H / 128;
-  const size_t P = (size_t)a.T * (size_t)(a.k + 1);
   const PfLayout L = pf_layout(a.E);
   uint64_t *rawfull = reinterpret_cast<uint64_t *>(smem);  // [RR] packed weights landed (TMA bytes)
   uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (8 worker warps)
@@ -284,7 +273,11 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
   uint64_t *aready = bfree + kPfRB;                         // [2]  A buffer written (8 worker warps)
   uint64_t *accf = aready + 2;                              // [2]  accumulators written (commit)
   uint64_t *tfree = accf + 2;                               // [2]  accumulators read (8 worker warps)
-  uint64_t *drain = tfree + 2;                              // teardown
+  uint64_t *dfull = tfree + 2;                              // [RD] block scales landed (TMA bytes)
+  uint64_t *dfree = dfull + kPfRD;                          // [RD] read (8 worker warps)
+  uint64_t *uxw = dfree + kPfRD;                            // up rows handed over (8 worker warps)
+  uint64_t *uxr = uxw + 1;                                  // up rows consumed (8 worker warps)
+  uint64_t *drain = uxr + 1;                                // teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
   int *s_ntiles = reinterpret_cast<int *>(smem + 520);
@@ -292,7 +285,7 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
   unsigned char *abuf = smem + L.a;
   unsigned char *bbuf = smem + L.b;
   unsigned char *raw = smem + L.raw;
-  unsigned char *scl = smem + L.scl;
+  unsigned char *dsm = smem + L.d;
   float *ux = reinterpret_cast<float *>(smem + L.ux);
 
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
@@ -314,6 +307,12 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
       mbar_init(accf + b, 1);
       mbar_init(tfree + b, 8);
     }
+    for (int s = 0; s < kPfRD; ++s) {
+      mbar_init(dfull + s, 1);
+      mbar_init(dfree + s, 8);
+    }
+    mbar_init(uxw, 8);
+    mbar_init(uxr, 8);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -370,19 +369,23 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
     }
   };
 
-  if (warp == kPfCtl) {
-    // ================================================================ control
+  if (warp == kPfTmaWarp) {
+    // ================================================================ copies
     if (lane == 0) {
       bool bad = false;
-      PfCur cr, cb, cm;
+      PfCur cr;
       cur_begin(cr);
-      cur_begin(cb);
-      cur_begin(cm);
-      int raw_next = 0, b_next = 0, mma_next = 0, rtile = -1;
+      int rtile = -1, issued = 0;
       const CUtensorMap *m0 = nullptr, *m1 = nullptr;
-      auto issue_raw = [&]() -> bool {  // stage raw_next == cr
-        const int j = raw_next, s = j % kPfRR;
-        if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty)) return false;
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&dmap) : "memory");
+      for (int j = 0; j < S && !bad; ++j, cur_next(cr)) {
+        // packed weights of stage j
+        const int s = j % kPfRR;
+        if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty)) {
+          bad = true;
+          break;
+        }
         if (cr.t != rtile) {
           rtile = cr.t;
           const CUtensorMap *em = a.maps + (size_t)cr.tl.e * 3;
@@ -399,61 +402,90 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
         } else {
           tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 128, rawfull + s);
         }
-        ++raw_next;
-        cur_next(cr);
-        return true;
-      };
-      auto issue_b = [&]() -> bool {  // stage b_next == cb
-        const int j = b_next, s = j % kPfRB;
-        if (j >= kPfRB && !mbar_wait(bfree + s, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) return false;
-        unsigned char *dst = bbuf + (size_t)s * kBBytes;
-        mbar_arrive_expect_tx(bfull + s, (uint32_t)cb.tl.n * 128u);
-        for (int i = 0; i < cb.tl.n / (int)kPfBoxRows; ++i)
-          tma_load_2d(dst + i * (int)kPfBoxRows * 128, &bmap, cb.g * 64, cb.tl.p0 + i * (int)kPfBoxRows, bfull + s);
-        ++b_next;
-        cur_next(cb);
-        return true;
-      };
-      auto issue_mma = [&]() -> bool {  // stage mma_next == cm
-        const int j = mma_next, buf = j & 1;
-        if (!mbar_wait(aready + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfFull)) return false;
-        if (!mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull)) return false;
-        if (j >= 2 && !mbar_wait(tfree + buf, (uint32_t)((j >> 1) - 1) & 1u, a.status, kDetPfAccFree)) return false;
+        // activation rows of stage j
+        const int sb = j % kPfRB;
+        if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) {
+          bad = true;
+          break;
+        }
+        unsigned char *db = bbuf + (size_t)sb * kBBytes;
+        mbar_arrive_expect_tx(bfull + sb, (uint32_t)cr.tl.n * 128u);
+        for (int i = 0; i < cr.tl.n / (int)kPfBoxRows; ++i)
+          tma_load_2d(db + i * (int)kPfBoxRows * 128, &bmap, cr.g * 64, cr.tl.p0 + i * (int)kPfBoxRows, bfull + sb);
+        if ((j & 1) == 0) {
+          // block scales of groups g, g+1: [N rows][4 floats], 4-float boxes from column 2g
+          const int jp = j >> 1, ds = jp % kPfRD;
+          if (jp >= kPfRD && !mbar_wait(dfree + ds, (uint32_t)(jp / kPfRD - 1) & 1u, a.status, kDetPfEmpty)) {
+            bad = true;
+            break;
+          }
+          unsigned char *dd = dsm + (size_t)ds * kDBytes;
+          mbar_arrive_expect_tx(dfull + ds, (uint32_t)cr.tl.n * 16u);
+          for (int i = 0; i < cr.tl.n / (int)kPfBoxRows; ++i)
+            tma_load_2d(dd + i * (int)kPfBoxRows * 16, &dmap, cr.g * 2, cr.tl.p0 + i * (int)kPfBoxRows, dfull + ds);
+        }
+        issued = j + 1;
+        if (*abort_flag) bad = true;
+      }
+      if (bad) *abort_flag = 1;
+      // teardown: copies issued but not yet landed (only after a failure can
+      // some never have been waited for)
+      for (int j = max(0, issued - kPfRR); j < issued; ++j)
+        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
+      for (int j = max(0, issued - kPfRB); j < issued; ++j)
+        mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
+      for (int jp = max(0, (issued + 1) / 2 - kPfRD); jp < (issued + 1) / 2; ++jp)
+        mbar_wait(dfull + jp % kPfRD, (uint32_t)(jp / kPfRD) & 1u, a.status, kDetPfDrain);
+    }
+    __syncwarp();
+  } else if (warp == kPfMmaWarp) {
+    // ================================================================ MMAs
+    if (lane == 0) {
+      bool bad = false;
+      PfCur cm;
+      cur_begin(cm);
+      uint64_t adesc[2][4], bdesc[kPfRB][4];
+#pragma unroll
+      for (int b = 0; b < 2; ++b)
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) adesc[b][k4] = umma_desc(smem_u32(abuf + (size_t)b * kABytes) + k4 * 4096);
+#pragma unroll
+      for (int r = 0; r < kPfRB; ++r)
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4)
+          bdesc[r][k4] = umma_desc_sw128(smem_u32(bbuf + (size_t)r * kBBytes) + (uint32_t)(k4 * 32));
+      int done = 0;
+      for (int j = 0; j < S && !bad; ++j, cur_next(cm)) {
+        const int buf = j & 1, sb = j % kPfRB;
+        if (!mbar_wait(aready + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfFull) ||
+            !mbar_wait(bfull + sb, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull) ||
+            (j >= 2 && !mbar_wait(tfree + buf, (uint32_t)((j >> 1) - 1) & 1u, a.status, kDetPfAccFree)) ||
+            *abort_flag) {
+          bad = true;
+          break;
+        }
         tc_fence_after();
-        const uint32_t sa = smem_u32(abuf + (size_t)buf * kABytes);
-        const uint32_t sb = smem_u32(bbuf + (size_t)(j % kPfRB) * kBBytes);
         const uint32_t idesc = pf_idesc(cm.tl.n);
         const uint32_t d = tmem + (uint32_t)(buf * 256);
+        uint64_t bd[4];
+#pragma unroll
+        for (int r = 0; r < kPfRB; ++r)
+          if (r == sb)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4) bd[k4] = bdesc[r][k4];
 #pragma unroll
         for (int b = 0; b < 2; ++b)
 #pragma unroll
           for (int ks = 0; ks < 2; ++ks) {
             const int k4 = 2 * b + ks;
-            umma_f16(d + (uint32_t)(b * 128), umma_desc(sa + k4 * 4096), umma_desc_sw128(sb + (uint32_t)(k4 * 32)),
-                     idesc, (uint32_t)ks);
+            umma_f16(d + (uint32_t)(b * 128), buf ? adesc[1][k4] : adesc[0][k4], bd[k4], idesc, (uint32_t)ks);
           }
         umma_commit(accf + buf);
-        umma_commit(bfree + j % kPfRB);
-        ++mma_next;
-        cur_next(cm);
-        return true;
-      };
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
-      while (!bad && raw_next < S && raw_next < kPfLR) bad = !issue_raw();
-      while (!bad && b_next < S && b_next < kPfLB) bad = !issue_b();
-      while (!bad && mma_next < S) {
-        if (raw_next < S && !issue_raw()) bad = true;
-        if (!bad && b_next < S && !issue_b()) bad = true;
-        if (!bad && !issue_mma()) bad = true;
-        if (*abort_flag) bad = true;
+        umma_commit(bfree + sb);
+        done = j + 1;
       }
       if (bad) *abort_flag = 1;
-      // teardown: copies issued but not yet landed, MMAs not yet finished
-      for (int j = max(0, raw_next - kPfRR); j < raw_next; ++j)
-        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
-      for (int j = max(mma_next, b_next - kPfRB); j < b_next; ++j)
-        mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
-      if (mma_next > 0) {
+      if (done > 0) {
         umma_commit(drain);
         mbar_wait(drain, 0, a.status, kDetPfDrain);
       }
@@ -461,43 +493,28 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
     __syncwarp();
   } else {
     // ================================================================ workers
-    bool ok = true;
+    bool bad = false;
     const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
-    // scale copies: weight scales of row tid (tid < 128), block scales of column tid & 127
-    PfCur cs;
-    cur_begin(cs);
-    const int crow = tid & 127, chalf = tid >> 7;
-    const unsigned char *srow = nullptr;
-    int stile = -1;
-    auto issue_scl = [&](int j) {  // stage j == cs
-      if (j < S) {
-        if (cs.t != stile) {
-          stile = cs.t;
-          const unsigned char *blob = static_cast<const unsigned char *>(a.table[cs.tl.e]);
-          if (MODE == 0) {
-            const size_t base = crow < 64 ? 0 : mg;
-            const size_t row = (size_t)cs.tl.wt * 64 + (crow & 63);
-            srow = blob + base + (size_t)I * (size_t)(H / 2) + row * (size_t)(H / 64) * 2;
-          } else {
-            const size_t row = (size_t)cs.tl.wt * 128 + crow;
-            srow = blob + 2 * mg + (size_t)H * (size_t)(I / 2) + row * (size_t)(I / 64) * 2;
-          }
-        }
-        unsigned char *ss = scl + (size_t)(j % kPfRD) * kSclBytes;
-        if (chalf == 0) cp_async4(ss + crow * 4, srow + (cs.g & ~1) * 2, 4);
-        if (crow < cs.tl.n) {
-          const bool v = crow < cs.tl.nval;
-          const float *src = a.bscale + (size_t)(2 * cs.g + chalf) * P + (v ? cs.tl.p0 + crow : 0);
-          cp_async4(reinterpret_cast<float *>(ss + kSclD) + chalf * 128 + crow, src, v ? 4u : 0u);
-        }
-        cur_next(cs);
-      }
-      cp_async_commit();
-    };
-    // epilogue state: TMEM lane quarter q, 16-column chunks half, half + 2, ...
-    const int q = warp & 3, half = warp >> 2;
+    const int crow = tid & 127, chalf = tid >> 7;  // expansion: row, 16-byte half of its 32 packed bytes
+    const int q = warp & 3, half = warp >> 2;      // epilogue: TMEM lane quarter, 16-column chunks half, +2, ..
     const int row = q * 32 + lane;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    // weight scales of this thread's row: 4 bytes (groups g, g+1) per stage
+    // pair, loaded one pair ahead
+    auto scale_row = [&](const PfTile &tl) -> const uint32_t * {
+      const unsigned char *blob = static_cast<const unsigned char *>(a.table[tl.e]);
+      if (MODE == 0) {
+        const size_t base = row < 64 ? 0 : mg;
+        const size_t r = (size_t)tl.wt * 64 + (row & 63);
+        return reinterpret_cast<const uint32_t *>(blob + base + (size_t)I * (size_t)(H / 2) + r * (size_t)(H / 64) * 2);
+      }
+      const size_t r = (size_t)tl.wt * 128 + row;
+      return reinterpret_cast<const uint32_t *>(blob + 2 * mg + (size_t)H * (size_t)(I / 2) + r * (size_t)(I / 64) * 2);
+    };
+    PfCur cw;
+    cur_begin(cw);
+    uint32_t w_next = 0, w_cur = 0;
+    if (S > 0) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
     PfCur ce;
     cur_begin(ce);
     float2 acc[4][8];
@@ -505,88 +522,84 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+    int tcount = 0;
 
-    for (int j = 0; j < kPfLD; ++j) issue_scl(j);
-    for (int i = 0; i <= S; ++i) {
-      // a. expand stage i: row crow, bytes 16 chalf ..: K-slices chalf (low
-      //    nibbles) and 2 + chalf (high nibbles)
+    for (int i = 0; i <= S && !bad; ++i) {
+      // expansion of stage i: row crow, bytes 16 chalf ..: K-slices chalf (low
+      // nibbles) and 2 + chalf (high nibbles)
       if (i < S) {
-        const bool got = __all_sync(0xffffffffu, mbar_wait(rawfull + i % kPfRR, (uint32_t)(i / kPfRR) & 1u, a.status,
-                                                            kDetPfFull));
-        if (!got) ok = false;
-        if (got) {
-          const uint4 src = *reinterpret_cast<const uint4 *>(raw + (size_t)(i % kPfRR) * kRawBytes + crow * 32 + chalf * 16);
-          unsigned char *ab = abuf + (size_t)(i & 1) * kABytes;
-#pragma unroll
-          for (int hi = 0; hi < 2; ++hi) {
-            const int sh = hi * 4;
-            uint32_t h[8];
-            nib4_to_f16((src.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
-            nib4_to_f16((src.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
-            nib4_to_f16((src.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
-            nib4_to_f16((src.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
-            unsigned char *dst = ab + (2 * hi + chalf) * 4096;
-            *reinterpret_cast<uint4 *>(dst + il_off(crow, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4 *>(dst + il_off(crow, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
-          }
-          fence_proxy_async();
+        if (!__all_sync(0xffffffffu, mbar_wait(rawfull + i % kPfRR, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull))) {
+          bad = true;
+          break;
         }
+        const uint4 src = *reinterpret_cast<const uint4 *>(raw + (size_t)(i % kPfRR) * kRawBytes + crow * 32 + chalf * 16);
+        unsigned char *ab = abuf + (size_t)(i & 1) * kABytes;
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int sh = hi * 4;
+          uint32_t h[8];
+          nib4_to_f16((src.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
+          nib4_to_f16((src.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
+          nib4_to_f16((src.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
+          nib4_to_f16((src.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
+          unsigned char *dst = ab + (2 * hi + chalf) * 4096;
+          *reinterpret_cast<uint4 *>(dst + il_off(crow, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4 *>(dst + il_off(crow, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+        fence_proxy_async();
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(aready + (i & 1));
           mbar_arrive(rawfree + i % kPfRR);
         }
       }
-      // b. scale copies of stage i+kPfLD; this thread's copies of stage i-1 done
-      issue_scl(i + kPfLD);
-      cp_async_wait<kPfLD + 1>();
-      // c.
-      if (!workers_sync_and(ok && !*abort_flag)) break;
       if (i == 0) continue;
-      // d. scales of stage i-1
-      const int j = i - 1, buf = j & 1;
-      const bool got = __all_sync(0xffffffffu, mbar_wait(accf + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfAccFull));
-      if (!got) ok = false;
+      // scales of stage j = i-1
+      const int j = i - 1, buf = j & 1, jp = j >> 1, ds = jp % kPfRD;
+      if ((j & 1) == 0) {
+        w_cur = w_next;
+        cur_next(cw);
+        cur_next(cw);
+        if (cw.t < n_tiles) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
+      }
+      if (!__all_sync(0xffffffffu, mbar_wait(accf + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfAccFull) &&
+                                       mbar_wait(dfull + ds, (uint32_t)(jp / kPfRD) & 1u, a.status, kDetPfFull))) {
+        bad = true;
+        break;
+      }
+      tc_fence_after();
       const int nch = ce.tl.n >> 4;
-      if (got) {
-        tc_fence_after();
-        const unsigned char *ss = scl + (size_t)(j % kPfRD) * kSclBytes;
-        const uint32_t wsv = *reinterpret_cast<const uint32_t *>(ss + row * 4);
-        const float sg = __half2float(__ushort_as_half((unsigned short)((ce.g & 1) ? (wsv >> 16) : (wsv & 0xFFFFu))));
-        const float2 sg2 = make_float2(sg, sg);
-        const float *d0p = reinterpret_cast<const float *>(ss + kSclD);
-        const float *d1p = d0p + 128;
+      const float sg = __half2float(__ushort_as_half((unsigned short)((ce.g & 1) ? (w_cur >> 16) : (w_cur & 0xFFFFu))));
+      const float2 sg2 = make_float2(sg, sg);
+      const float *dp = reinterpret_cast<const float *>(dsm + (size_t)ds * kDBytes) + 2 * (ce.g & 1);  // [col][4]
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci) {
-          const int c = half + 2 * ci;
-          if (c < nch) {
-            float4 da[4], db[4];
+      for (int ci = 0; ci < 4; ++ci) {
+        const int c = half + 2 * ci;
+        if (c < nch) {
+          float2 dv[16];
 #pragma unroll
-            for (int j4 = 0; j4 < 4; ++j4) {
-              da[j4] = *reinterpret_cast<const float4 *>(d0p + c * 16 + 4 * j4);
-              db[j4] = *reinterpret_cast<const float4 *>(d1p + c * 16 + 4 * j4);
-            }
-            uint32_t v0[16], v1[16];
-            tmem_ld16(tq + (uint32_t)(buf * 256 + c * 16), v0);
-            tmem_ld16(tq + (uint32_t)(buf * 256 + 128 + c * 16), v1);
-            tmem_ld_wait();
+          for (int k = 0; k < 16; ++k) dv[k] = *reinterpret_cast<const float2 *>(dp + (c * 16 + k) * 4);
+          uint32_t v0[16], v1[16];
+          tmem_ld16(tq + (uint32_t)(buf * 256 + c * 16), v0);
+          tmem_ld16(tq + (uint32_t)(buf * 256 + 128 + c * 16), v1);
+          tmem_ld_wait();
 #pragma unroll
-            for (int jj = 0; jj < 8; ++jj) {
-              const float4 &a4 = da[jj >> 1];
-              const float4 &b4 = db[jj >> 1];
-              const float2 dap = (jj & 1) ? make_float2(a4.z, a4.w) : make_float2(a4.x, a4.y);
-              const float2 dbp = (jj & 1) ? make_float2(b4.z, b4.w) : make_float2(b4.x, b4.y);
-              const float2 s0 = make_float2(__uint_as_float(v0[2 * jj]), __uint_as_float(v0[2 * jj + 1]));
-              const float2 s1 = make_float2(__uint_as_float(v1[2 * jj]), __uint_as_float(v1[2 * jj + 1]));
-              const float2 fb = __ffma2_rn(s1, dbp, __fmul2_rn(s0, dap));
-              acc[ci][jj] = __ffma2_rn(sg2, fb, acc[ci][jj]);
-            }
+          for (int jj = 0; jj < 8; ++jj) {
+            const float2 dap = make_float2(dv[2 * jj].x, dv[2 * jj + 1].x);
+            const float2 dbp = make_float2(dv[2 * jj].y, dv[2 * jj + 1].y);
+            const float2 s0 = make_float2(__uint_as_float(v0[2 * jj]), __uint_as_float(v0[2 * jj + 1]));
+            const float2 s1 = make_float2(__uint_as_float(v1[2 * jj]), __uint_as_float(v1[2 * jj + 1]));
+            const float2 fb = __ffma2_rn(s1, dbp, __fmul2_rn(s0, dap));
+            acc[ci][jj] = __ffma2_rn(sg2, fb, acc[ci][jj]);
           }
         }
-        tc_fence_before();
       }
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(tfree + buf);
+      if (lane == 0) {
+        mbar_arrive(tfree + buf);
+        if (j & 1) mbar_arrive(dfree + ds);
+      }
       if (ce.g == G - 1) {
         // the tile's outputs
         const PfTile tl = ce.tl;
@@ -608,6 +621,11 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
           // Rows 64..127 hold u of rows 0..63 (g): hand u over, then SwiGLU and
           // Q8_0 of h along I (one 32-block = one warp's lanes), per token.
           if (q >= 2) {
+            if (tcount > 0 &&
+                !__all_sync(0xffffffffu, mbar_wait(uxr, (uint32_t)(tcount - 1) & 1u, a.status, kDetPfFull))) {
+              bad = true;
+              break;
+            }
 #pragma unroll
             for (int ci = 0; ci < 4; ++ci) {
               const int c = half + 2 * ci;
@@ -620,7 +638,12 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
               }
             }
           }
-          workers_sync_and(true);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(uxw);
+          if (!__all_sync(0xffffffffu, mbar_wait(uxw, (uint32_t)tcount & 1u, a.status, kDetPfFull))) {
+            bad = true;
+            break;
+          }
           if (q < 2) {
             // h = SiLU(g) * u and its Q8_0 codes in fast fp32 (this path is held
             // to the layer's tolerance, not to the fixed-order bits)
@@ -643,16 +666,15 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
                     const size_t p = (size_t)(tl.p0 + col);
                     a.hq[p * I + ii] = (int8_t)qv;
                     hh[p * I + ii] = __int2half_rn(qv);
-                    if (lane == 0) {
-                      a.hd[p * (I / 32) + ii / 32] = d;
-                      a.hdT[(size_t)(ii / 32) * P + p] = d;
-                    }
+                    if (lane == 0) a.hd[p * (I / 32) + ii / 32] = d;
                   }
                 }
               }
             }
           }
-          // the next tile's hand-over comes after at least one more worker barrier
+          __syncwarp();
+          if (lane == 0) mbar_arrive(uxr);
+          ++tcount;
         }
 #pragma unroll
         for (int ci = 0; ci < 4; ++ci)
@@ -660,9 +682,9 @@ __global__ void __maxnreg__(168) k_gemm_pf(const PfArgs a, const __grid_constant
           for (int jj = 0; jj < 8; ++jj) acc[ci][jj] = make_float2(0.0f, 0.0f);
       }
       cur_next(ce);
+      if (*abort_flag) bad = true;
     }
-    if (!ok) *abort_flag = 1;
-    cp_async_wait_all();
+    if (bad) *abort_flag = 1;
   }
   // teardown: every copy and MMA of this CTA has completed (see the control warp)
   tc_fence_before();
@@ -714,18 +736,18 @@ cudaError_t launch_make_maps(const PfArgs &a, const CUtensorMap &tgu, const CUte
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s) {
+cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUtensorMap &dmap, int grid, cudaStream_t s) {
   const size_t smem = pf_layout(a.E).total;
   if (smem > (size_t)kMaxSmem) return cudaErrorInvalidConfiguration;
   cudaError_t err;
   if (a.mode == 0) {
     err = cudaFuncSetAttribute(k_gemm_pf<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap);
+    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
   } else {
     err = cudaFuncSetAttribute(k_gemm_pf<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap);
+    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
   }
   return cudaGetLastError();
 }
@@ -829,14 +851,14 @@ cudaError_t launch_gather_rows(const GatherRowsArgs &a, cudaStream_t s) {
 }
 
 // ===========================================================================
-// x's Q8_0 block scales in pair order, block-major (the gate/up GEMM copies a
-// tile's scales of one block as one contiguous run).
+// x's Q8_0 block scales in pair order (rows of H/32): the gate/up GEMM copies
+// a tile's scales of two groups as 4-float boxes.
 // ===========================================================================
 __global__ void __launch_bounds__(256) k_gather_scales(const GatherScaleArgs a) {
   const int64_t P = (int64_t)a.T * (a.k + 1);
   const int64_t n = P * a.nb;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t b = i / P, p = i - b * P;
+    const int64_t p = i / a.nb, b = i - p * a.nb;
     a.xdp[i] = a.xd[(int64_t)a.pair_tok[p] * a.nb + b];
   }
 }
