@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--experts", type=int, default=None,
                     help="routed experts per layer (profiling: a small pool, same per-step work)")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="prefill batch size (profiling a small case; default: the workload's 2048)")
     return ap.parse_args()
 
 
@@ -64,6 +66,23 @@ def peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def profiled_traffic(name: str, source: str):
+    """DRAM bytes per launch of a kernel from its committed ncu summary
+    (profiles/<name>.md), or None once the kernel's source has changed since."""
+    import hashlib
+    p = os.path.join(ROOT, "profiles", name + ".md")
+    if not os.path.exists(p):
+        return None
+    traffic, sha = None, None
+    for line in open(p):
+        if line.startswith("traffic_bytes_per_launch:"):
+            traffic = int(line.split(":")[1])
+        if line.startswith("source:") and "sha256[:16]" in line:
+            sha = line.split()[-1]
+    cur = hashlib.sha256(open(os.path.join(ROOT, source), "rb").read()).hexdigest()[:16]
+    return traffic if sha == cur else None
 
 
 def tensor_peak():
@@ -283,7 +302,9 @@ def run_native(args, ws_n, rank, local):
     gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "kernel": "k_gateup_decode", "achieved": round(gu_gbs, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(gu_gbs / peak, 4),
-                "peak_source": peak_src, "traffic": None,
+                "peak_source": peak_src,
+                "traffic": profiled_traffic("k_gateup_decode_glm_T1",
+                                            "int4_routed_expert_softmax_b200/csrc/moe_decode.cu"),
                 "bytes_per_launch": round(gu_bytes / K), "us_per_launch": round(gu_ms / K * 1e3, 2)}
     kernels = {
         "k_route_decode": {"us": round(rt_ms / K * 1e3, 2),
@@ -362,8 +383,10 @@ def run_prefill(args, ws_n, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = mi.WORKLOADS["prefill"]
+    if args.experts:
+        w = mi.shrink(w, E=args.experts)
     seed = w.seed + 1000 * rank
-    T = w.T
+    T = args.tokens or w.T
     x = mi.make_x(T, w.H, mi.sub_seed(seed, 0, 1), dev, zipf=True)
     Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), dev, zipf_s=w.zipf_s)
     blobs = mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, 0, 3), dev)

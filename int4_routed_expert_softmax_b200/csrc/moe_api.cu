@@ -151,7 +151,7 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   ga.hd = p.hd;
   ga.status = p.status;
   gateup_plan(d.H, Tc, &ga.rpm, &ga.nstage);
-  ga.use_pdl = 0;
+  ga.use_pdl = 1;
   if (ga.nstage < 2) return MOE_ERR_SHAPE;
   cudaError_t err =
       launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.rpm, ga.nstage), s);
@@ -191,7 +191,7 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   while (da.rs > da.rg && down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs) < 3)
     da.rs = ((da.rs / 2 + da.rg - 1) / da.rg) * da.rg;
   da.nstage = down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs);
-  da.use_pdl = 0;
+  da.use_pdl = 1;
   da.preload = down_preload(d.I, d.k, Tc);
   if (da.nstage < 2) return MOE_ERR_SHAPE;
   err = launch_down_decode(

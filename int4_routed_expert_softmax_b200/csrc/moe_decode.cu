@@ -439,8 +439,8 @@ void gateup_plan(int H, int T, int *R, int *nstage) {
 
 template <int CSZ, bool ONE, int R>
 static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_gateup_decode<CSZ, ONE, R>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int smem_set[64] = {0};
+  cudaError_t err = ensure_smem(k_gateup_decode<CSZ, ONE, R>, smem, smem_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -758,8 +758,8 @@ int down_max_stages(int H, int I, int k, int T, int rows_max, int rs) {
 
 template <int CSZ, bool ONE>
 static cudaError_t launch_dn(const DownArgs &a, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t err = cudaFuncSetAttribute(k_down_decode<CSZ, ONE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int smem_set[64] = {0};
+  cudaError_t err = ensure_smem(k_down_decode<CSZ, ONE>, smem, smem_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);

@@ -38,6 +38,21 @@ enum Detail : int32_t {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the call
+// costs host time on every launch otherwise).  `cache` is the kernel's own
+// per-device record; concurrent first calls both set the same value.
+template <typename K>
+inline cudaError_t ensure_smem(K kernel, size_t smem, int (&cache)[64]) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if ((int)smem <= cache[dev]) return cudaSuccess;
+  err = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (err == cudaSuccess) cache[dev] = (int)smem;
+  return err;
+}
+
 inline size_t matrix_bytes(int N, int K) {
   return (size_t)N * (size_t)(K / 2) + (size_t)N * (size_t)(K / 64) * 2;
 }

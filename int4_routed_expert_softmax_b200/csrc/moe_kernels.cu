@@ -402,6 +402,9 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int H = a.H;
 
+  // the experts kernel that follows may be scheduled now; it waits for this
+  // grid's completion (griddepcontrol.wait) before it reads anything
+  pdl_launch_dependents();
   const int e0 = blockIdx.x * a.epc;
   const int ne = min(a.epc, a.E - e0);
   // start the copies of the first tile before the quantisation work below
@@ -491,8 +494,8 @@ size_t route_smem_bytes(int H, int epc, int tt) {
 
 cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s) {
   const size_t smem = route_smem_bytes(a.H, a.epc, a.tt);
-  cudaError_t err = cudaFuncSetAttribute(k_route_decode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  static int smem_set[64] = {0};
+  cudaError_t err = ensure_smem(k_route_decode, smem, smem_set);
   if (err != cudaSuccess) return err;
   const int grid = (a.E + a.epc - 1) / a.epc;
   k_route_decode<<<grid, 128, smem, s>>>(a);

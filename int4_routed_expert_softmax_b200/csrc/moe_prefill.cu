@@ -741,11 +741,13 @@ cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUten
   if (smem > (size_t)kMaxSmem) return cudaErrorInvalidConfiguration;
   cudaError_t err;
   if (a.mode == 0) {
-    err = cudaFuncSetAttribute(k_gemm_pf<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_set0[64] = {0};
+    err = ensure_smem(k_gemm_pf<0>, smem, smem_set0);
     if (err != cudaSuccess) return err;
     k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
   } else {
-    err = cudaFuncSetAttribute(k_gemm_pf<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    static int smem_set1[64] = {0};
+    err = ensure_smem(k_gemm_pf<1>, smem, smem_set1);
     if (err != cudaSuccess) return err;
     k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
   }
@@ -818,7 +820,8 @@ __global__ void __launch_bounds__(256) k_router_tiled(const RouterTiledArgs a) {
 cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
   const size_t smem = (size_t)(kRtTok + kRtExp) * kRtKC * 4;
-  cudaError_t err = cudaFuncSetAttribute(k_router_tiled, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  static int smem_set[64] = {0};
+  cudaError_t err = ensure_smem(k_router_tiled, smem, smem_set);
   if (err != cudaSuccess) return err;
   const dim3 grid((unsigned)((a.T + kRtTok - 1) / kRtTok), (unsigned)((a.E + kRtExp - 1) / kRtExp));
   k_router_tiled<<<grid, 256, smem, s>>>(a);

@@ -18,7 +18,9 @@
  *  - router = softmax over the experts, top-k kept and renormalised; the pages
  *    do not name the router function, this is the layer's definition as stated
  *    for this library.
- * Every reading taken where the pages are silent is listed in the design doc.
+ * Where the pages are silent (rounding mode, tie-breaks, scale types, the
+ * order of every fp32 sum, the nibble layout), the choice is stated at the
+ * function that makes it.
  *
  * Arithmetic is IEEE binary32 with explicit fmaf() where a fused multiply-add
  * is meant; the file is compiled with -ffp-contract=off so no other
