@@ -228,8 +228,24 @@ __device__ void bucket_warp(int E, int k, int T, const int32_t *idx, int *s_work
 // =====================================================================
 // The same counting sort for P = T*k <= 32 pairs, in registers: lane p holds
 // pair p; its position is the number of pairs before it in (expert, pair id)
-// order; counts, offsets and the union follow from comparisons.
+// order; the union follows from comparisons.  Counts and offsets of all E
+// experts: bucket_small_counts (any number of warps).
 // =====================================================================
+__device__ void bucket_small_counts(int E, int P, const int *s_pairs, int32_t *cnt, int32_t *off, int warp,
+                                    int nwarps) {
+  const int lane = threadIdx.x & 31;
+  for (int e = warp * 32 + lane; e < E; e += nwarps * 32) {
+    int c = 0, o = 0;
+    for (int q = 0; q < P; ++q) {
+      const int eq = s_pairs[q];  // every lane reads the same word
+      c += eq == e ? 1 : 0;
+      o += eq < e ? 1 : 0;
+    }
+    cnt[e] = c;
+    off[e] = o;
+  }
+}
+
 __device__ void bucket_small(int E, int k, int T, const int32_t *idx, int32_t *cnt, int32_t *off,
                              int32_t *uni, int32_t *n_uni, int32_t *perm, int32_t *pos,
                              int32_t *pair_tok) {
@@ -244,30 +260,17 @@ __device__ void bucket_small(int E, int k, int T, const int32_t *idx, int32_t *c
   }
   // distinct experts below ep: pairs q that are the first of their expert
   const int fl = (lane < P) ? first : 0;
+  const unsigned firsts = __ballot_sync(0xffffffffu, fl);
   for (int q = 0; q < P; ++q) {
     const int eq = __shfl_sync(0xffffffffu, ep, q);
-    const int fq = __shfl_sync(0xffffffffu, fl, q);
-    below += (fq && eq < ep) ? 1 : 0;
+    below += (((firsts >> q) & 1u) && eq < ep) ? 1 : 0;
   }
-  const int nu = __reduce_add_sync(0xffffffffu, (unsigned)fl);
+  const int nu = __popc(firsts);
   if (lane < P) {
     perm[rank] = lane;
     if (pos) pos[lane] = rank;
     if (pair_tok) pair_tok[rank] = lane / k;
     if (first) uni[below] = ep;
-  }
-  for (int e0 = 0; e0 < E; e0 += 32) {
-    const int e = e0 + lane;
-    int c = 0, o = 0;
-    for (int q = 0; q < P; ++q) {
-      const int eq = __shfl_sync(0xffffffffu, ep, q);
-      c += eq == e ? 1 : 0;
-      o += eq < e ? 1 : 0;
-    }
-    if (e < E) {
-      cnt[e] = c;
-      off[e] = o;
-    }
   }
   if (lane == 0) {
     off[E] = P;
@@ -286,12 +289,16 @@ __device__ void bucket_small(int E, int k, int T, const int32_t *idx, int32_t *c
 // 32 halving steps with a warp-wide count (redux) find the k-th largest key;
 // every key above it is kept, and keys equal to it are taken in ascending
 // expert index until k are kept; the kept k are then ranked by (logit
-// descending, index ascending).  scratch: 96 words of shared memory per warp.
+// descending, index ascending).  scratch: 128 words of shared memory per warp.
 // =====================================================================
 __device__ __forceinline__ uint32_t order_key(float v) {
   if (v == 0.0f) v = 0.0f;  // -0 == +0
   const uint32_t u = __float_as_uint(v);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// The logit of a key (-0 comes back as +0, equal in every later use).
+__device__ __forceinline__ float key_value(uint32_t kk) {
+  return __uint_as_float((kk & 0x80000000u) ? (kk & 0x7FFFFFFFu) : ~kk);
 }
 
 template <int NPER>
@@ -308,10 +315,10 @@ __device__ __forceinline__ void warp_topk_radix(const float *lg, int E, int k, i
   uint32_t pre = 0u;
   for (int bit = 31; bit >= 0; --bit) {
     const uint32_t cand = pre | (1u << bit);
-    int c = 0;
+    int c = 0;  // keys >= cand over the warp: one vote per held key (absent keys are 0 < cand)
 #pragma unroll
-    for (int j = 0; j < NPER; ++j) c += (lane + 32 * j < E && key[j] >= cand) ? 1 : 0;
-    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) pre = cand;
+    for (int j = 0; j < NPER; ++j) c += __popc(__ballot_sync(0xffffffffu, key[j] >= cand));
+    if (c >= k) pre = cand;
   }
   // pre = k-th largest key: keep > pre, then == pre by ascending index
   int gt = 0;
@@ -350,11 +357,12 @@ __device__ __forceinline__ void warp_topk_radix(const float *lg, int E, int k, i
       rank += (ok > mk || (ok == mk && oe < me)) ? 1 : 0;
     }
     scratch[64 + rank] = (uint32_t)me;
+    scratch[96 + rank] = mk;
   }
   __syncwarp();
   if (lane < k) {
     e_sel = (int)scratch[64 + lane];
-    l_sel = __ldcg(lg + e_sel);
+    l_sel = key_value(scratch[96 + lane]);
   }
   __syncwarp();
 }
@@ -458,23 +466,28 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   }
   if (a.done == nullptr) return;
 
-  // ---- the last CTA to arrive does top-k and the batch union
-  __threadfence();
+  // ---- the last CTA to arrive does top-k and the batch union.  The ticket is
+  // an acquire-release add at GPU scope: after the barrier it publishes this
+  // CTA's logits and codes, and the last CTA's add sees everyone's.
   __syncthreads();
-  if (tid == 0) *s_flag = (atomicAdd(a.done, 1u) == gridDim.x - 1) ? 1 : 0;
+  if (tid == 0) {
+    unsigned int old;
+    asm volatile("atom.acq_rel.gpu.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(a.done) : "memory");
+    *s_flag = (old == gridDim.x - 1) ? 1 : 0;
+  }
   __syncthreads();
   if (!*s_flag) return;
-  __threadfence();
   int *s_idx = reinterpret_cast<int *>(sW);               // [T*k]
   int *s_work = s_idx + kDecodeTMax * kMaxK;              // bucket scratch
-  uint32_t *s_tk = reinterpret_cast<uint32_t *>(s_work + 3 * MOE_MAX_E + 64);  // [4][96]
+  uint32_t *s_tk = reinterpret_cast<uint32_t *>(s_work + 3 * MOE_MAX_E + 64);  // [4][128]
   for (int t = warp; t < a.T; t += 4) {
     int e_sel;
     float l_sel;
-    warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, lane, e_sel, l_sel, s_tk + warp * 96);
+    warp_topk(a.logits + (size_t)t * a.E, a.E, a.k, lane, e_sel, l_sel, s_tk + warp * 128);
     warp_softmax_store(t, a.k, lane, e_sel, l_sel, a.idx, a.w, a.route_counts, s_idx);
   }
   __syncthreads();
+  if (a.do_bucket && a.T * a.k <= 32) bucket_small_counts(a.E, a.T * a.k, s_idx, a.cnt, a.off, warp, 4);
   if (warp != 0) return;
   if (a.do_bucket) {
     if (a.T * a.k <= 32)
@@ -488,7 +501,7 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
 
 size_t route_smem_bytes(int H, int epc, int tt) {
   size_t fl = (size_t)(epc + tt) * H * 4;
-  size_t need_tail = (size_t)(kDecodeTMax * kMaxK + 3 * MOE_MAX_E + 64 + 4 * 96) * 4;
+  size_t need_tail = (size_t)(kDecodeTMax * kMaxK + 3 * MOE_MAX_E + 64 + 4 * 128) * 4;
   return 128 + (fl > need_tail ? fl : need_tail);
 }
 
@@ -507,7 +520,7 @@ cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s) {
 // =====================================================================
 __global__ void __launch_bounds__(256) k_topk(const float *logits, int T, int E, int k, int32_t *idx,
                                              float *w, int32_t *counts) {
-  __shared__ uint32_t s_tk[8][96];
+  __shared__ uint32_t s_tk[8][128];
   const int lane = threadIdx.x & 31;
   const int t = (int)(((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   if (t >= T) return;
