@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "stacked", "tiered"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -514,6 +514,158 @@ def oracle_prefill_sample(w, x_h, Wr_h, blob_fn, budget_s: float, tokens_max: in
                       f"{spent:.1f} s"}
 
 
+# ----------------------------------------------------------------- stacked and tiered
+def chain_next_dev(x: torch.Tensor, out: torch.Tensor, gamma: float = 0.5, zipf: bool = False) -> torch.Tensor:
+    """Input of the next layer (workload glue between layers, outside every
+    timed region): v = x + gamma * out / rms(out); x' = v / rms(v)."""
+    ro = out.double().pow(2).mean(-1, keepdim=True).sqrt().float()
+    ro = torch.where(ro > 0, ro, torch.ones_like(ro))
+    v = x + gamma * out / ro
+    nx = v / (v.double().pow(2).mean(-1, keepdim=True) + 1e-12).sqrt().float()
+    if zipf:
+        nx[..., 0] = 1.0
+    return nx.contiguous()
+
+
+def run_stacked(args, ws_n, rank, local):
+    """8 stacked GLM-5.2-shaped layers resident in HBM; batches of 1, 4 and 16
+    tokens with independently drawn hidden states; per-layer us and
+    union-weighted expert GB/s."""
+    import int4_routed_expert_softmax_b200 as moe
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = mi.WORKLOADS["stacked"]
+    seed = w.seed + 1000 * rank
+    L = w.layers
+    routers = [mi.make_router(w.E, w.H, mi.sub_seed(seed, l, 2), dev) for l in range(L)]
+    blobs = [mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, l, 3), dev) for l in range(L)]
+    tables = [moe.expert_table(b) for b in blobs]
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    stream = torch.cuda.current_stream()
+    res, tot_b, tot_ms = {}, 0.0, 0.0
+    with ClockSampler(local) as clk:
+        for T in w.T_list:
+            ws = moe.alloc_workspace(d, T, dev)
+            view = moe.moe_workspace_view(d, T, ws)
+            nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
+            out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+            layer_ms, layer_b = [], []
+            for it in range(args.warmup + args.steps):
+                x = mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1), dev)
+                for l in range(L):
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record(stream)
+                    moe.moe_layer_forward(d, x, routers[l], tables[l], out, ws)
+                    b.record(stream)
+                    b.synchronize()
+                    if it >= args.warmup:
+                        layer_ms.append(a.elapsed_time(b))
+                        layer_b.append((int(nuni_t.item()) + 1) * w.blob_bytes)
+                    x = chain_next_dev(x, out)
+            ms = allreduce_max(sum(layer_ms), ws_n)
+            bts = allreduce_sum(float(sum(layer_b)), ws_n)
+            res[f"T={T}"] = {"us_per_layer": round(ms / len(layer_ms) * 1e3, 2),
+                             "us_per_token_layer": round(ms / len(layer_ms) / T * 1e3, 2),
+                             "union_mean": round(sum(layer_b) / len(layer_b) / w.blob_bytes - 1, 1),
+                             "GB/s": round(bts / (ms * 1e-3) / 1e9, 1)}
+            tot_b += bts
+            tot_ms += ms
+    value = tot_b / (tot_ms * 1e-3) / 1e9
+    return dict(metric=METRIC, value=round(value, 1), unit="GB/s", n_gpus=ws_n, steps=args.steps,
+                warmup=args.warmup, ms_per_step=round(tot_ms / args.steps, 4), higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="int4xint8->fp32", data="synthetic",
+                config={"workload": "stacked: 8 GLM-5.2-shaped layers resident in HBM (41.2 GB), batches of "
+                                    "1, 4, 16 tokens, layers chained", "layers": L, "T_list": list(w.T_list),
+                        "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)"},
+                by_batch=res, clocks=clk.summary(), gpu_launches=None)
+
+
+def run_tiered(args, ws_n, rank, local):
+    """16 GLM-5.2-shaped layers in pinned host memory, 20 GB HBM expert cache
+    (LRU + pins learned from route counts + one-layer-ahead prefetch), 512
+    decode tokens with Zipf(1.1) routing persisting token to token."""
+    import numpy as np  # noqa: F401
+
+    import int4_routed_expert_softmax_b200 as moe
+    from int4_routed_expert_softmax_b200 import _cache as C
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    w = mi.WORKLOADS["tiered"]
+    seed = w.seed + 1000 * rank
+    L, E1 = w.layers, w.E + 1
+    n_tok = args.steps
+    host = torch.empty((L, E1, w.blob_bytes), dtype=torch.uint8, pin_memory=True)
+    for l in range(L):
+        host[l].copy_(mi.make_blobs(w.H, w.I, E1, mi.sub_seed(seed, l, 3), dev), non_blocking=False)
+    routers = [mi.make_router(w.E, w.H, mi.sub_seed(seed, l, 2), dev, zipf_s=w.zipf_s) for l in range(L)]
+    torch.cuda.synchronize()
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    cache = C.ExpertCache(d, L, [[host[l, e] for e in range(E1)] for l in range(L)], w.cache_bytes)
+    ws = moe.alloc_workspace(d, 1, dev)
+    ws_pred = moe.alloc_workspace(d, 1, dev)
+    out = torch.empty((1, w.H), dtype=torch.float32, device=dev)
+    counts = [torch.zeros(w.E, dtype=torch.int32, device=dev) for _ in range(L)]
+    side = torch.cuda.Stream(device=dev)
+    stream = torch.cuda.current_stream()
+    xs = mi.make_x(args.warmup + n_tok, w.H, mi.sub_seed(seed, 0, 1), dev, zipf=True, rho=w.rho)
+
+    def token(t):
+        x = xs[t:t + 1].contiguous()
+        for l in range(L):
+            cache.tiered_layer_forward(l, x, routers[l], out, ws, ws_pred=ws_pred,
+                                       Wr_next=routers[l + 1] if l + 1 < L else None,
+                                       route_counts=counts[l], side_stream=side)
+            x = chain_next_dev(x, out, zipf=True)
+
+    for t in range(args.warmup):
+        token(t)
+    # pins learned from the warm-up's route counts
+    n_pin = max(0, min(cache.stats()["slots_per_layer"] - (w.k + 1) - 8, w.E // 4))
+    for l in range(L):
+        cache.learn_pins(l, counts[l].cpu().tolist(), n_pin)
+    torch.cuda.synchronize()
+    s0 = cache.stats()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(ws_n)
+    with ClockSampler(local) as clk:
+        a.record(stream)
+        for t in range(args.warmup, args.warmup + n_tok):
+            token(t)
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = allreduce_max(a.elapsed_time(b), ws_n)
+    s1 = cache.stats()
+    dd = {k: s1[k] - s0[k] for k in ("hits", "misses", "prefetches", "prefetch_hits", "bytes_h2d", "evictions")}
+    # host link alone: one 20 MB blob copy, pinned host -> HBM
+    blob_dev = torch.empty(w.blob_bytes, dtype=torch.uint8, device=dev)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(20):
+        blob_dev.copy_(host[0, 0], non_blocking=True)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    link = 20 * w.blob_bytes / (c0.elapsed_time(c1) * 1e-3) / 1e9
+    tok_s = n_tok * ws_n / (ms * 1e-3)
+    lookups = dd["hits"] + dd["misses"]
+    cache.close()
+    return dict(metric=METRIC, value=round(tok_s, 2), unit="tok/s", n_gpus=ws_n, steps=n_tok,
+                warmup=args.warmup, ms_per_step=round(ms / n_tok, 3), higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="int4xint8->fp32", data="synthetic",
+                config={"workload": "tiered: 16 GLM-5.2-shaped layers (82.5 GB) in pinned host memory, HBM cache "
+                                    "20 GB, LRU + learned pins + one-layer-ahead prefetch, decode tokens with "
+                                    "Zipf(1.1) routing persisting token to token (rho 0.9)",
+                        "layers": L, "cache_bytes": w.cache_bytes, "tokens_timed": n_tok,
+                        "pins_per_layer": n_pin, "parallelism": f"replicas x{ws_n}"},
+                hit_rate=round(dd["hits"] / max(1, lookups), 4),
+                prefetch_accuracy=round(dd["prefetch_hits"] / max(1, dd["prefetches"]), 4),
+                host_link_GBps={"during_run": round(dd["bytes_h2d"] / (ms * 1e-3) / 1e9, 2),
+                                "single_copy": round(link, 2)},
+                cache_delta=dd, us_per_token_layer=round(ms / n_tok / L * 1e3, 2), clocks=clk.summary(),
+                gpu_launches=None)
+
+
 # ----------------------------------------------------------------- reference arm
 def run_reference(args, ws_n, rank):
     """The CPU oracle on a bounded sample of the same workload (rank 0 only)."""
@@ -602,7 +754,8 @@ def main():
         return
     ws_n, rank, local = dist_setup()
     try:
-        res = run_prefill(args, ws_n, rank, local) if args.workload == "prefill" else run_native(args, ws_n, rank, local)
+        fn = {"prefill": run_prefill, "stacked": run_stacked, "tiered": run_tiered}.get(args.workload, run_native)
+        res = fn(args, ws_n, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
