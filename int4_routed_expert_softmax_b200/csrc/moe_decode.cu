@@ -194,7 +194,12 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     }
     fence_barrier_init();
   }
-  if (a.use_pdl) pdl_wait();
+  if (a.use_pdl) {
+    pdl_wait();
+    // the down kernel may be scheduled from here on (as SMs free up); this
+    // grid's own routing inputs are complete, which is all it reads early
+    pdl_launch_dependents();
+  }
   // an earlier kernel of this call failed: leave everything untouched
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
@@ -414,7 +419,6 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
     }
   }
-  if (a.use_pdl) pdl_launch_dependents();
 }
 
 static int gu_csz(int H) { return (H / 64 + 31) / 32; }
@@ -549,7 +553,12 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     mbar_init(actbar, 1);
     fence_barrier_init();
   }
-  if (a.use_pdl) pdl_wait();
+  // The union comes from the routing kernel, which completed before the gate/up
+  // kernel passed its own dependency wait; this grid is scheduled only after
+  // that point, so the union and the expert table are read before this grid's
+  // wait, and the first ring of weight copies overlaps the gate/up kernel's
+  // tail.  The h codes (the gate/up kernel's output) are read after it.
+  __syncthreads();
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int nslot = n_uni + 1;
@@ -579,16 +588,27 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   if (warp == 8) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      if (a.preload) {
-        const uint32_t bq = (uint32_t)P * I, bd = (uint32_t)P * IB * 4;
-        mbar_arrive_expect_tx(actbar, bq + 2 * bd);
-        bulk_g2s(act_s, a.hq, bq, actbar);
-        bulk_g2s(act_s + bq, a.hd, bd, actbar);
-        bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
-      }
       int s = 0, issued = 0, slot = 0, sub = 0;
       uint32_t ph = 0;
+      bool waited = !a.use_pdl, failed = false;
       for (int j = 0; j < n_st; ++j) {
+        if (j == NS && !waited) {
+          // the ring is full: wait for the gate/up kernel, then its outputs
+          pdl_wait();
+          waited = true;
+          if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) {
+            failed = true;
+            s_abort = 1;
+            break;
+          }
+          if (a.preload) {
+            const uint32_t bq = (uint32_t)P * I, bd = (uint32_t)P * IB * 4;
+            mbar_arrive_expect_tx(actbar, bq + 2 * bd);
+            bulk_g2s(act_s, a.hq, bq, actbar);
+            bulk_g2s(act_s + bq, a.hd, bd, actbar);
+            bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
+          }
+        }
         if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetDnEmpty)) {
           s_abort = 1;
           break;
@@ -614,10 +634,31 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
           ++slot;
         }
       }
+      if (!waited && !failed) {
+        // fewer stages than ring slots
+        pdl_wait();
+        waited = true;
+        if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) {
+          failed = true;
+          s_abort = 1;
+        } else if (a.preload) {
+          const uint32_t bq = (uint32_t)P * I, bd = (uint32_t)P * IB * 4;
+          mbar_arrive_expect_tx(actbar, bq + 2 * bd);
+          bulk_g2s(act_s, a.hq, bq, actbar);
+          bulk_g2s(act_s + bq, a.hd, bd, actbar);
+          bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
+        }
+      }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
         mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
-      if (a.preload) mbar_wait(actbar, 0, a.status, kDetDnDrain);
+      if (a.preload && waited && !failed) mbar_wait(actbar, 0, a.status, kDetDnDrain);
     }
+    return;
+  }
+  // consumers: the gate/up kernel's outputs are read only after its completion
+  if (a.use_pdl) pdl_wait();
+  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) {
+    s_abort = 1;
     return;
   }
 
