@@ -264,7 +264,11 @@ def run_native(args, ws_n, rank, local):
     K = args.steps
     ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    layer_ms, prof, nuni = [], [], []
+    # each step's union size is copied on the device after the step's end
+    # event; the host never waits inside the loop
+    nuni_hist = torch.zeros(K, dtype=torch.int32, device=dev)
+    layer_ms = []
+    moe.moe_profile_enable(True)                      # fresh per-call history
     barrier(ws_n)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
@@ -274,15 +278,18 @@ def run_native(args, ws_n, rank, local):
             ev0[i].record(stream)
             step(args.warmup + i)
             ev1[i].record(stream)
-            prof.append(moe.moe_profile_last())       # waits for this step
-            nuni.append(int(nuni_t.item()))
+            nuni_hist[i:i + 1].copy_(nuni_t)
         torch.cuda.synchronize()
     barrier(ws_n)
     torch.cuda.synchronize()
     wall = time.perf_counter() - wall0
     for i in range(K):
         layer_ms.append(ev0[i].elapsed_time(ev1[i]))
+    prof = moe.moe_profile_read(K)
     moe.moe_profile_enable(False)
+    nuni = [int(u) for u in nuni_hist.tolist()]
+    if len(prof) != K:
+        raise RuntimeError(f"profiled {len(prof)} of {K} calls")
     if int(status_t[0].item()) != 0:
         raise RuntimeError(f"device status {status_t.tolist()}")
 
@@ -312,6 +319,9 @@ def run_native(args, ws_n, rank, local):
         "k_gateup_decode": {"us": round(gu_ms / K * 1e3, 2), "GB/s": round(gu_gbs, 1)},
         "k_down_decode": {"us": round(dn_ms / K * 1e3, 2),
                           "GB/s": round(dn_bytes / (dn_ms * 1e-3) / 1e9, 1)},
+        "call_span": {"us": round(sum(p[3] for p in prof) / K * 1e3, 2)},
+        "timing": "device %globaltimer stamps per kernel phase (first CTA start, last CTA end); "
+                  "gate/up from its dependency wait, down from its first CTA (overlaps gate/up's tail)",
     }
 
     # ---- end to end: host buffers through moe_layer_forward_host
@@ -413,7 +423,7 @@ def run_prefill(args, ws_n, rank, local):
         raise RuntimeError(f"device status {status_t.tolist()}")
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    prof = []
+    moe.moe_profile_enable(True)                      # fresh per-call history
     barrier(ws_n)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
@@ -422,10 +432,12 @@ def run_prefill(args, ws_n, rank, local):
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
-            prof.append(moe.moe_profile_last())
         torch.cuda.synchronize()
     barrier(ws_n)
+    prof = moe.moe_profile_read(K)
     moe.moe_profile_enable(False)
+    if len(prof) != K:
+        raise RuntimeError(f"profiled {len(prof)} of {K} calls")
     if int(status_t[0].item()) != 0:
         raise RuntimeError(f"device status {status_t.tolist()}")
     my_ms = sum(a.elapsed_time(b) for a, b in ev)

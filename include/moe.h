@@ -100,8 +100,8 @@ size_t moe_expert_bytes(const moe_dims *dims);
 size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max);
 
 /* Same for an explicit path: MOE_PATH_PREFILL needs the prefill segments (the
- * fp16 activation codes and the per-pair down rows, about T*(k+1)*H*4 bytes)
- * for any T; MOE_PATH_DECODE never does. */
+ * fp16 hi/lo activation rows and the per-pair down rows, about
+ * T*(k+1)*(2H+I)*4 bytes, plus 8 MB) for any T; MOE_PATH_DECODE never does. */
 size_t moe_workspace_bytes_path(const moe_dims *dims, int32_t T_max, int32_t path);
 
 /* Q8_0 quantisation of rows x T x cols fp32 (cols % 32 == 0):
@@ -138,10 +138,11 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
  * stream each union expert's bytes once per 16 tokens, every fp32 step in the
  * layer's fixed order -- bit-identical to the CPU definition.
  * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
- * union on the tensor cores (exact 32-block integer sums, scales applied in
- * fp32 in another order) and the combine; within the layer's float tolerance
- * of the definition, the routing (idx, w, cnt, off, uni, perm) and the Q8_0
- * codes of x still bit-exact.  (Batched expert unions: colibri deep review
+ * union on the tensor cores (the int4 weights, exact in fp16, times an fp16
+ * hi + lo split of the dequantised Q8_0 activations, 22 significant bits;
+ * fp32 accumulation; weight scales applied per group) and the combine; within
+ * the layer's float tolerance of the definition, the routing (idx, w, cnt, off,
+ * uni, perm) and the Q8_0 codes of x still bit-exact.  (Batched expert unions: colibri deep review
  * page, technology table, row I/O 即引擎; prefill GEMM order: tantan.ink
  * page, section 我看到的几个坑.)
  * Arguments:
@@ -332,16 +333,29 @@ int moe_workspace_view(const moe_dims *dims, int32_t T_max, void *ws, moe_ws_vie
  * (device of the current context), or a negative status. */
 int moe_device_sms(void);
 
-/* Per-kernel timing.  moe_profile_enable(1) makes every following
- * moe_layer_forward record CUDA events on its stream around each of its
- * kernels (library-owned events of the current device); moe_profile_enable(0)
- * stops it.  moe_profile_last(ms, n) waits for the events of the most recent
- * forward call and writes up to n durations in milliseconds:
- *   ms[0] router + top-k + bucket, ms[1] gate/up (+ SwiGLU + requant),
- *   ms[2] down + combine.
- * Returns the number of durations written, or a negative status. */
+/* Per-call kernel timing on the device.  moe_profile_enable(1) allocates (once)
+ * and zeroes a library-owned ring of 1024 records on the current device; from
+ * then on every moe_layer_forward, and every moe_layer_route with the
+ * moe_layer_experts that follows it, takes the next record, and its kernels
+ * stamp each phase's first start and last end there with the GPU's global
+ * nanosecond timer (thread 0 of every CTA, atomics; no stream events, so the
+ * launch sequence and its programmatic dependent launches are unchanged).
+ * Calls after the ring is full go unrecorded.  moe_profile_enable(0) stops
+ * recording.
+ * moe_profile_read(ms, max_calls) synchronizes the device, writes 4 floats
+ * (milliseconds) per recorded call, oldest first, into ms[4 * max_calls]:
+ *   [0] routing: decode = the routing kernel (Q8_0, logits, top-k, union);
+ *       prefill = quantisation through the tensor-map build,
+ *   [1] gate/up: decode = from the gate/up kernel's dependency wait to its
+ *       last CTA's end; prefill = the gate/up grouped GEMM,
+ *   [2] down: decode = the down kernel including its combine, from its first
+ *       CTA's start (weight copies overlap the gate/up kernel's tail);
+ *       prefill = the down grouped GEMM and the combine kernel,
+ *   [3] the call: first start to last end over the three phases,
+ * (0 for a phase that was not stamped), then zeroes the ring and starts a new
+ * history.  Returns the number of calls written, or a negative status. */
 int moe_profile_enable(int on);
-int moe_profile_last(float *ms, int n);
+int moe_profile_read(float *ms, int max_calls);
 
 #ifdef __cplusplus
 }

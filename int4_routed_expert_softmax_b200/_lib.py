@@ -57,7 +57,7 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_view": (ctypes.c_int, [D, i32, P, ctypes.POINTER(MoeWsView)]),
             "moe_device_sms": (ctypes.c_int, []),
             "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
-            "moe_profile_last": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
+            "moe_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
             "moe_quant_q8_0": (ctypes.c_int, [P, i64, i32, P, P, P]),
             "moe_router_topk": (ctypes.c_int, [D, i32, P, P, P, P, P, P, P]),
             "moe_bucket": (ctypes.c_int, [D, i32, P, P, P, P, P, P, P]),
@@ -120,16 +120,17 @@ def moe_device_sms() -> int:
 
 
 def moe_profile_enable(on: bool) -> None:
-    lib().moe_profile_enable(1 if on else 0)
+    _check("moe_profile_enable", lib().moe_profile_enable(1 if on else 0))
 
 
-def moe_profile_last() -> list:
-    """Per-kernel ms of the last forward: [router+bucket, gate/up, down]."""
-    buf = (ctypes.c_float * 3)()
-    n = lib().moe_profile_last(buf, 3)
+def moe_profile_read(max_calls: int = 1024) -> list:
+    """Device-stamped ms per recorded call since the last read, oldest first:
+    [routing, gate/up, down, whole call] each; clears the history."""
+    buf = (ctypes.c_float * (4 * max_calls))()
+    n = lib().moe_profile_read(buf, max_calls)
     if n < 0:
-        raise MoeError("moe_profile_last", n)
-    return [float(buf[i]) for i in range(n)]
+        raise MoeError("moe_profile_read", n)
+    return [[float(buf[4 * c + j]) for j in range(4)] for c in range(n)]
 
 
 def moe_quant_q8_0(x: torch.Tensor, q: torch.Tensor, d: torch.Tensor, stream=None):

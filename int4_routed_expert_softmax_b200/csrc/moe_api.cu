@@ -30,18 +30,36 @@ bool dims_shape_ok(const moe_dims &d) {
          d.E >= 1 && d.E <= MOE_MAX_E && d.k >= 1 && d.k <= d.E && d.k <= kMaxK;
 }
 
-// ---- optional per-kernel events (moe_profile_enable)
+// ---- optional per-call kernel timing (moe_profile_enable).  Each profiled
+// call owns one zeroed record of a per-device ring; its kernels stamp their
+// phases there with %globaltimer, so nothing is added to the stream between
+// them.  The ring is zeroed at enable and after every read.
 bool g_prof = false;
-cudaEvent_t g_ev[kMaxDevices][4] = {};
-int g_ev_dev = -1;
+unsigned long long *g_prof_buf[kMaxDevices] = {};
+int g_prof_n[kMaxDevices] = {};
+unsigned long long *g_prof_cur[kMaxDevices] = {};
 
-void prof_record(int i, cudaStream_t s) {
-  if (!g_prof) return;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return;
-  if (g_ev[dev][i] == nullptr && cudaEventCreate(&g_ev[dev][i]) != cudaSuccess) return;
-  cudaEventRecord(g_ev[dev][i], s);
-  g_ev_dev = dev;
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
+// A fresh record for the next call on the current device, or null when
+// profiling is off or the ring is full (the call then goes unrecorded).
+unsigned long long *prof_next() {
+  if (!g_prof) return nullptr;
+  const int dev = current_device();
+  if (dev < 0 || g_prof_buf[dev] == nullptr || g_prof_n[dev] >= kProfSlots) return nullptr;
+  g_prof_cur[dev] = g_prof_buf[dev] + (size_t)(g_prof_n[dev]++) * kProfWords;
+  return g_prof_cur[dev];
+}
+
+// The record of the most recent routing call (the experts half of a split layer).
+unsigned long long *prof_current() {
+  if (!g_prof) return nullptr;
+  const int dev = current_device();
+  return dev < 0 ? nullptr : g_prof_cur[dev];
 }
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -93,7 +111,8 @@ ChunkPtrs chunk_ptrs(const moe_dims &d, int t0, const WsLayout &L, void *ws) {
 }
 
 int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
-                const float *Wr, void *ws, int32_t *counts, cudaStream_t s) {
+                const float *Wr, void *ws, int32_t *counts, unsigned long long *prof,
+                cudaStream_t s) {
   const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
   RouteArgs ra{};
   ra.H = d.H;
@@ -121,15 +140,14 @@ int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const floa
   ra.do_bucket = 1;
   ra.epc = 2;
   ra.tt = Tc < 2 ? Tc : 2;
-  prof_record(0, s);
+  ra.prof = prof;
   cudaError_t err = launch_route_decode(ra, s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(1, s);
   return MOE_OK;
 }
 
 int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const void *const *table,
-                  float *out, void *ws, cudaStream_t s) {
+                  float *out, void *ws, unsigned long long *prof, cudaStream_t s) {
   const int sms = device_sms();
   if (sms <= 0) return MOE_ERR_CUDA;
   const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
@@ -152,11 +170,11 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   ga.status = p.status;
   gateup_plan(d.H, Tc, &ga.rpm, &ga.nstage);
   ga.use_pdl = 1;
+  ga.prof = prof;
   if (ga.nstage < 2) return MOE_ERR_SHAPE;
   cudaError_t err =
       launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.rpm, ga.nstage), s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(2, s);
 
   DownArgs da{};
   da.H = d.H;
@@ -192,12 +210,12 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
     da.rs = ((da.rs / 2 + da.rg - 1) / da.rg) * da.rg;
   da.nstage = down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs);
   da.use_pdl = 1;
+  da.prof = prof;
   da.preload = down_preload(d.I, d.k, Tc);
   if (da.nstage < 2) return MOE_ERR_SHAPE;
   err = launch_down_decode(
       da, grid, down_smem_bytes(d.H, d.I, d.k, Tc, da.rows_max, da.rs, da.nstage), s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(3, s);
   return MOE_OK;
 }
 
@@ -219,8 +237,8 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   int32_t *idx = at<int32_t>(ws, L.idx);
   float *w = at<float>(ws, L.w);
   int32_t *status = at<int32_t>(ws, L.status);
-  prof_record(0, s);
-  QuantArgs qa{x, xq, xd, at<void>(ws, L.xh), (int64_t)T * (d.H / 32)};
+  unsigned long long *prof = prof_next();
+  QuantArgs qa{x, xq, xd, (int64_t)T * (d.H / 32), prof};
   cudaError_t err = launch_quant(qa, s);
   if (err != cudaSuccess) return cuda_status(err);
   RouterTiledArgs ra{d.H, d.E, T, x, Wr, logits};
@@ -242,13 +260,9 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   ba.pair_tok = at<int32_t>(ws, L.pair_tok);
   err = launch_bucket(ba, s);
   if (err != cudaSuccess) return cuda_status(err);
-  GatherScaleArgs ga{d.H / 32, T, d.k, xd, ba.pair_tok, at<float>(ws, L.xdp)};
-  err = launch_gather_scales(ga, s);
-  if (err != cudaSuccess) return cuda_status(err);
-  GatherRowsArgs gr{d.H, T, d.k, at<void>(ws, L.xh), ba.pair_tok, at<void>(ws, L.xg)};
+  GatherRowsArgs gr{d.H, T, d.k, xq, xd, ba.pair_tok, at<void>(ws, L.xg)};
   err = launch_gather_rows(gr, s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(1, s);
 
   PfArgs pa{};
   pa.mode = 0;
@@ -262,38 +276,33 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   pa.n_uni = ba.n_uni;
   pa.off = ba.off;
   pa.pair_tok = ba.pair_tok;
-  pa.bsrc = gr.xg;
-  pa.bscale = ga.xdp;
   pa.hq = at<int8_t>(ws, L.hq);
-  pa.hh = at<void>(ws, L.hh);
   pa.hd = at<float>(ws, L.hd);
+  pa.hs = at<void>(ws, L.hs);
   pa.y = at<float>(ws, L.y);
+  pa.ux = at<float>(ws, L.ux);
   pa.status = status;
+  pa.prof = prof;
   const size_t P = (size_t)T * (size_t)(d.k + 1);
   pa.maps = at<CUtensorMap>(ws, L.maps);
-  CUtensorMap map_x, map_h, map_dx, map_dh, tmpl_gu, tmpl_dn;
-  err = make_f16_map(&map_x, pa.bsrc, (uint64_t)P, (uint64_t)d.H, kPfBoxRows);
-  if (err == cudaSuccess) err = make_f16_map(&map_h, pa.hh, (uint64_t)P, (uint64_t)d.I, kPfBoxRows);
-  if (err == cudaSuccess) err = make_f32x4_map(&map_dx, ga.xdp, (uint64_t)P, (uint64_t)d.H / 32, kPfBoxRows);
-  if (err == cudaSuccess) err = make_f32x4_map(&map_dh, pa.hd, (uint64_t)P, (uint64_t)d.I / 32, kPfBoxRows);
+  CUtensorMap map_x, map_h, tmpl_gu, tmpl_dn;
+  err = make_f16_map(&map_x, gr.xg, (uint64_t)P, 2 * (uint64_t)d.H, kPfBoxRows);
+  if (err == cudaSuccess) err = make_f16_map(&map_h, pa.hs, (uint64_t)P, 2 * (uint64_t)d.I, kPfBoxRows);
   // the templates' address is replaced per expert on the device
   if (err == cudaSuccess) err = make_u8_map(&tmpl_gu, pa.maps, (uint64_t)d.I, (uint64_t)d.H / 2, 64);
   if (err == cudaSuccess) err = make_u8_map(&tmpl_dn, pa.maps, (uint64_t)d.H, (uint64_t)d.I / 2, 128);
   if (err != cudaSuccess) return cuda_status(err);
   err = launch_make_maps(pa, tmpl_gu, tmpl_dn, s);
   if (err != cudaSuccess) return cuda_status(err);
-  err = launch_gemm_pf(pa, map_x, map_dx, sms, s);
+  const int grid = sms < kPfMaxCtas ? sms : kPfMaxCtas;
+  err = launch_gemm_pf(pa, map_x, grid, s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(2, s);
   pa.mode = 1;
-  pa.bsrc = pa.hh;
-  pa.bscale = pa.hd;
-  err = launch_gemm_pf(pa, map_h, map_dh, sms, s);
+  err = launch_gemm_pf(pa, map_h, grid, s);
   if (err != cudaSuccess) return cuda_status(err);
-  CombineArgs ca{d.H, d.k, T, pa.y, w, ba.pos, out};
+  CombineArgs ca{d.H, d.k, T, pa.y, w, ba.pos, out, prof};
   err = launch_combine(ca, s);
   if (err != cudaSuccess) return cuda_status(err);
-  prof_record(3, s);
   return MOE_OK;
 }
 
@@ -370,24 +379,59 @@ int moe_device_sms(void) {
 }
 
 int moe_profile_enable(int on) {
+  if (on) {
+    const int dev = current_device();
+    if (dev < 0) return MOE_ERR_CUDA;
+    const size_t bytes = (size_t)kProfSlots * kProfWords * sizeof(unsigned long long);
+    if (g_prof_buf[dev] == nullptr) {
+      cudaError_t e = cudaMalloc(&g_prof_buf[dev], bytes);
+      if (e != cudaSuccess) {
+        g_prof_buf[dev] = nullptr;
+        return cuda_status(e);
+      }
+    }
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemset(g_prof_buf[dev], 0, bytes);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_status(e);
+    g_prof_n[dev] = 0;
+    g_prof_cur[dev] = nullptr;
+  }
   g_prof = on != 0;
   return MOE_OK;
 }
 
-int moe_profile_last(float *ms, int n) {
-  if (ms == nullptr || n < 0) return MOE_ERR_BAD_ARG;
-  const int dev = g_ev_dev;
-  if (dev < 0) return 0;
-  for (int i = 0; i < 4; ++i)
-    if (g_ev[dev][i] == nullptr) return 0;
-  cudaError_t e = cudaEventSynchronize(g_ev[dev][3]);
+int moe_profile_read(float *ms, int max_calls) {
+  if (ms == nullptr || max_calls < 0) return MOE_ERR_BAD_ARG;
+  const int dev = current_device();
+  if (dev < 0) return MOE_ERR_CUDA;
+  if (g_prof_buf[dev] == nullptr) return 0;
+  const int n = g_prof_n[dev];
+  const size_t bytes = (size_t)kProfSlots * kProfWords * sizeof(unsigned long long);
+  static thread_local unsigned long long rec[kProfSlots * kProfWords];
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess && n > 0)
+    e = cudaMemcpy(rec, g_prof_buf[dev], (size_t)n * kProfWords * sizeof(unsigned long long),
+                   cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(g_prof_buf[dev], 0, bytes);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e);
-  int w = 0;
-  for (int i = 0; i < 3 && w < n; ++i) {
-    float t = 0.0f;
-    e = cudaEventElapsedTime(&t, g_ev[dev][i], g_ev[dev][i + 1]);
-    if (e != cudaSuccess) return cuda_status(e);
-    ms[w++] = t;
+  g_prof_n[dev] = 0;
+  g_prof_cur[dev] = nullptr;
+  const int w = n < max_calls ? n : max_calls;
+  for (int c = 0; c < w; ++c) {
+    const unsigned long long *r = rec + (size_t)c * kProfWords;
+    unsigned long long first = ~0ull, last = 0;
+    for (int k = 0; k < 3; ++k) {
+      const unsigned long long st = ~r[2 * k], en = r[2 * k + 1];
+      const bool ok = r[2 * k] != 0 && en != 0 && en >= st;
+      ms[(size_t)c * 4 + k] = ok ? (float)((double)(en - st) * 1e-6) : 0.0f;
+      if (ok) {
+        first = st < first ? st : first;
+        last = en > last ? en : last;
+      }
+    }
+    ms[(size_t)c * 4 + 3] = last > 0 ? (float)((double)(last - first) * 1e-6) : 0.0f;
   }
   return w;
 }
@@ -396,7 +440,7 @@ int moe_quant_q8_0(const float *x, int64_t rows, int32_t cols, int8_t *q, float 
   if (rows < 0 || cols <= 0 || cols % 32 != 0) return MOE_ERR_SHAPE;
   if (rows == 0) return MOE_OK;
   if (!x || !q || !d) return MOE_ERR_BAD_ARG;
-  QuantArgs a{x, q, d, nullptr, rows * (int64_t)(cols / 32)};
+  QuantArgs a{x, q, d, rows * (int64_t)(cols / 32), nullptr};
   return cuda_status(launch_quant(a, static_cast<cudaStream_t>(stream)));
 }
 
@@ -465,11 +509,12 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
   if (err != cudaSuccess) return cuda_status(err);
   if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
+  unsigned long long *prof = prof_next();
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
     const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
-    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, s);
+    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, s);
     if (rc != MOE_OK) return rc;
-    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, s);
+    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, prof, s);
     if (rc != MOE_OK) return rc;
   }
   return MOE_OK;
@@ -489,7 +534,7 @@ int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
   if (err != cudaSuccess) return cuda_status(err);
-  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, s);
+  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, prof_next(), s);
 }
 
 int moe_read_union(const moe_dims *dims, int32_t T, void *ws, int32_t *host_uni, int32_t *host_n,
@@ -524,7 +569,8 @@ int moe_layer_experts(const moe_dims *dims, int32_t T, const void *const *expert
   if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   const WsLayout L = ws_layout(*dims, T);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  return experts_chunk(*dims, 0, T, L, expert_table, out, ws, static_cast<cudaStream_t>(stream));
+  return experts_chunk(*dims, 0, T, L, expert_table, out, ws, prof_current(),
+                       static_cast<cudaStream_t>(stream));
 }
 
 int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host, const float *Wr,

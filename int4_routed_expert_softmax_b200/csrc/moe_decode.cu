@@ -202,6 +202,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
   }
   // an earlier kernel of this call failed: leave everything untouched
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  prof_start(a.prof, 1);
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int rbs = I / 32;  // 32-row units per expert
   const int n_units = (n_uni + 1) * rbs;
@@ -419,6 +420,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
     }
   }
+  prof_end(a.prof, 1);
 }
 
 static int gu_csz(int H) { return (H / 64 + 31) / 32; }
@@ -558,6 +560,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   // that point, so the union and the expert table are read before this grid's
   // wait, and the first ring of weight copies overlaps the gate/up kernel's
   // tail.  The h codes (the gate/up kernel's output) are read after it.
+  prof_start(a.prof, 2);
   __syncthreads();
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
@@ -781,6 +784,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     }
     a.out[(size_t)t * H + m0 + m] = o;
   }
+  prof_end(a.prof, 2);
   if (a.use_pdl) pdl_launch_dependents();
 }
 

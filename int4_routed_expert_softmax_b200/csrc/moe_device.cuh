@@ -172,6 +172,22 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// ------------------------------------------------------------------ profiling
+// Per-call profiling record (moe_profile_enable): for phase k, word 2k holds
+// ~(earliest start) and word 2k+1 the latest end in ns of %globaltimer, both
+// kept with atomicMax from a zeroed record, stamped by thread 0 of every CTA.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void prof_start(unsigned long long *p, int k) {
+  if (p != nullptr && threadIdx.x == 0) atomicMax(p + 2 * k, ~global_ns());
+}
+__device__ __forceinline__ void prof_end(unsigned long long *p, int k) {
+  if (p != nullptr && threadIdx.x == 0) atomicMax(p + 2 * k + 1, global_ns());
+}
+
 // Named barrier among `nthreads` threads (warp multiples) with id `id` (1..15).
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

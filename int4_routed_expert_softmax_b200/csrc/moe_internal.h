@@ -16,6 +16,9 @@ constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
 constexpr int kMaxK = 32;                              // kernels keep <= 32 slots per token
 constexpr int kDecodeTMax = MOE_DECODE_T_MAX;
 constexpr int kMaxSmem = 227 * 1024 - 1024;            // dynamic shared memory per CTA (sm_100 opt-in limit, minus static)
+constexpr int kPfMaxCtas = 256;                        // prefill GEMM grid bound (one CTA per SM)
+constexpr int kProfSlots = 1024;                       // per-call profiling records kept per device
+constexpr int kProfWords = 8;                          // per record: 4 phases x (~first start, last end) in ns
 
 // Device-side error details (status[1]) -- which wait or check failed.
 enum Detail : int32_t {
@@ -59,10 +62,10 @@ inline size_t matrix_bytes(int N, int K) {
 inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matrix_bytes(H, I); }
 
 // Byte offsets of the workspace segments for batches of up to T tokens.  The
-// prefill segments (xh, hh, y) are sized only when `prefill` is set.
+// prefill segments (xg, hs, y, ux, maps) are sized only when `prefill` is set.
 struct WsLayout {
   size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
-      pair_tok, hq, hqs, hd, xh, xg, xdp, hh, y, maps, total;
+      pair_tok, hq, hqs, hd, xg, hs, y, ux, maps, total;
 };
 
 inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
@@ -93,12 +96,11 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
   L.hq = seg(P * d.I);
   L.hqs = seg(P * (d.I / 32) * 4);
   L.hd = seg(P * (d.I / 32) * 4);
-  const size_t Tp = prefill ? (size_t)T : 0, Pp = prefill ? P : 0;
-  L.xh = seg(Tp * d.H * 2);
-  L.xg = seg(Pp * d.H * 2);
-  L.xdp = seg(Pp * (d.H / 32) * 4);
-  L.hh = seg(Pp * d.I * 2);
+  const size_t Pp = prefill ? P : 0;
+  L.xg = seg(Pp * d.H * 4);  // fp16 hi/lo split of x^, [P][2H]
+  L.hs = seg(Pp * d.I * 4);  // fp16 hi/lo split of h^, [P][2I]
   L.y = seg(Pp * d.H * 4);
+  L.ux = seg(prefill ? (size_t)kPfMaxCtas * 64 * 128 * 4 : 0);
   L.maps = seg(prefill ? (size_t)(d.E + 1) * 3 * 128 : 0);
   L.total = o;
   return L;
@@ -108,8 +110,8 @@ struct QuantArgs {
   const float *x;
   int8_t *q;
   float *d;
-  void *qh;  // optional: the codes again as fp16 (exact small integers)
   int64_t nblk;
+  unsigned long long *prof;  // profiling record or null (phase 0 start)
 };
 
 struct RouteArgs {
@@ -125,6 +127,7 @@ struct RouteArgs {
   int do_bucket;
   int epc;  // experts per CTA
   int tt;   // tokens per x tile
+  unsigned long long *prof;  // profiling record or null (phase 0)
 };
 
 struct BucketArgs {
@@ -146,6 +149,7 @@ struct GateUpArgs {
   int nstage;
   int rpm;  // weight rows per matrix per stage (4 or 8)
   int use_pdl;
+  unsigned long long *prof;  // profiling record or null (phase 1)
 };
 
 struct DownArgs {
@@ -164,6 +168,7 @@ struct DownArgs {
   int rs;        // rows per stage (a multiple of rg)
   int preload;   // per-position activations kept in shared memory (small batches)
   int use_pdl;
+  unsigned long long *prof;  // profiling record or null (phase 2)
 };
 
 // Prefill grouped GEMM over the expert union (moe_prefill.cu).  mode 0: gate/up
@@ -172,28 +177,23 @@ struct PfArgs {
   int mode, H, I, E, k, T;
   const void *const *table;
   const int32_t *uni, *n_uni, *off, *pair_tok;
-  const void *bsrc;     // fp16 codes of the activations: mode 0 [T][H] (xh), mode 1 [P][I] (hh)
-  const float *bscale;  // their Q8_0 block scales in pair order: mode 0 [P][H/32] (xdp), mode 1 [P][I/32] (hd)
-  int8_t *hq;           // mode 0 outputs, in pair order
-  void *hh;
-  float *hd;            // [P][I/32]
+  int8_t *hq;           // mode 0 outputs in pair order: Q8_0 codes of h [P][I],
+  float *hd;            //   their block scales [P][I/32],
+  void *hs;             //   and the fp16 hi/lo split of h^ = q d [P][2I] (mode 1's B rows)
   float *y;             // mode 1 output [P][H]
+  float *ux;            // mode 0 up-row exchange, [CTA][64][128] fp32
   const CUtensorMap *maps;  // [E+1][gate, up, down] tensor maps of the packed weights (device)
   int32_t *status;
+  unsigned long long *prof;  // profiling record or null (phase mode + 1; k_make_maps ends phase 0)
 };
 
-// x's block scales gathered into pair order: xdp[p][b] = xd[pair_tok[p]][b].
-struct GatherScaleArgs {
-  int nb, T, k;
-  const float *xd;
-  const int32_t *pair_tok;
-  float *xdp;
-};
-
-// x's fp16 codes gathered into pair order: xg[p] = xh[pair_tok[p]] (rows of H).
+// The gate/up GEMM's activation rows in pair order: xg[p] = fp16 hi/lo split of
+// the dequantised Q8_0 codes of token pair_tok[p] ([P][2H], per 64-group 64 hi
+// then 64 lo).
 struct GatherRowsArgs {
   int H, T, k;
-  const void *xh;
+  const int8_t *xq;
+  const float *xd;
   const int32_t *pair_tok;
   void *xg;
 };
@@ -209,6 +209,7 @@ struct CombineArgs {
   const float *y, *w;
   const int32_t *pos;
   float *out;
+  unsigned long long *prof;  // profiling record or null (phase 2 end)
 };
 
 // Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
@@ -220,21 +221,17 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
 cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s);
 cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s);
 
-cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUtensorMap &dmap, int grid, cudaStream_t s);
+cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s);
 // 2D tensor map over a row-major fp16 matrix [rows][cols] for TMA copies of
 // boxes of 64 columns x box_rows rows with 128-byte swizzle (moe_tma.cpp).
 cudaError_t make_f16_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
-// 2D tensor map over a row-major fp32 matrix [rows][cols] for boxes of 4 columns x
-// box_rows rows, no swizzle (moe_tma.cpp).
-cudaError_t make_f32x4_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 // Template for the packed-weight maps: a uint8 matrix [rows][cols] (cols = K/2),
 // boxes of 32 bytes x box_rows rows, no swizzle (moe_tma.cpp).
 cudaError_t make_u8_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 cudaError_t launch_make_maps(const PfArgs &a, const CUtensorMap &tgu, const CUtensorMap &tdn, cudaStream_t s);
-constexpr uint32_t kPfBoxRows = 16;  // rows per activation TMA box of the prefill GEMM
+constexpr uint32_t kPfBoxRows = 32;  // rows per activation TMA box of the prefill GEMM
 cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
-cudaError_t launch_gather_scales(const GatherScaleArgs &a, cudaStream_t s);
 cudaError_t launch_gather_rows(const GatherRowsArgs &a, cudaStream_t s);
 size_t pf_smem_bytes(int E);
 

@@ -27,6 +27,7 @@ namespace moe {
 // Q8_0 quantisation: one warp per 32-block (lane = element).
 // =====================================================================
 __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
+  prof_start(a.prof, 0);
   const int lane = threadIdx.x & 31;
   const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -35,7 +36,6 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
     const float d = fdiv(warp_max(fabsf(v)), 127.0f);
     const int c = q8_code(v, d);
     a.q[b * 32 + lane] = (int8_t)c;
-    if (a.qh != nullptr) static_cast<__half *>(a.qh)[b * 32 + lane] = __int2half_rn(c);
     if (lane == 0) a.d[b] = d;
   }
 }
@@ -413,6 +413,7 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   // the experts kernel that follows may be scheduled now; it waits for this
   // grid's completion (griddepcontrol.wait) before it reads anything
   pdl_launch_dependents();
+  prof_start(a.prof, 0);
   const int e0 = blockIdx.x * a.epc;
   const int ne = min(a.epc, a.E - e0);
   // start the copies of the first tile before the quantisation work below
@@ -464,7 +465,10 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
     }
     __syncthreads();
   }
-  if (a.done == nullptr) return;
+  if (a.done == nullptr) {
+    prof_end(a.prof, 0);
+    return;
+  }
 
   // ---- the last CTA to arrive does top-k and the batch union.  The ticket is
   // an acquire-release add at GPU scope: after the barrier it publishes this
@@ -497,6 +501,7 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
                   a.pair_tok);
   }
   if (lane == 0) *a.done = 0u;
+  prof_end(a.prof, 0);
 }
 
 size_t route_smem_bytes(int H, int epc, int tt) {

@@ -13,28 +13,26 @@
 //                    mode 1 = down into per-pair rows y.
 //   k_combine      : out = y_shared + sum_s w_s * y_s, slot order.
 //
-// The GEMM tile is 128 weight rows (MMA M) by up to 128 token rows of one
-// expert (MMA N, a multiple of 16), so an expert with few tokens wastes at most
-// 15 columns.  K advances one 64-group per pipeline stage.
+// The GEMM tile is 128 weight rows (MMA M; for gate/up 64 gate rows and the 64
+// up rows of the same intermediate rows) by up to 128 token rows of one expert
+// (MMA N, a multiple of 16), so an expert with few tokens wastes at most 15
+// columns.  K advances one 64-group per pipeline stage.
 //
-// Exact block sums on fp16 tensor cores.  The int4 weights (-8..7) and the
-// Q8_0 activation codes (-127..127) are small integers, exact in fp16, and
-// every product and every 32-element block sum (|sum| <= 32512) is exact in
-// the fp32 accumulator.  So tcgen05.mma kind::f16 yields, per 32-block b, the
-// exact integer S_b as an fp32 value in TMEM.  The epilogue then applies the
-// scales, three fp32 operations per output and 64-group:
-//     acc += s_g * (S_0 * d_0 + S_1 * d_1)
-// (kind::i8 would return int32 sums and need two more fp32 operations per
-// output to convert them; the epilogue's fp32 rate, not the MMA rate, bounds
-// this kernel.)  The weights are expanded nibble -> fp16 in shared memory by
-// the producer warps: bytes 0x64 0x0u form the half 1024 + u, one packed fp16
-// subtraction of 1032 gives u - 8.
+// Operands.  The int4 weights (-8..7) are exact in fp16; the expansion warps
+// turn nibbles into fp16 in shared memory (bytes 0x64 0x0u form the half
+// 1024 + u, one packed fp16 subtraction of 1032 gives u - 8).  The activations
+// enter as the dequantised Q8_0 values x^ = q d split into two fp16 numbers,
+// hi = fp16(x^) and lo = fp16(x^ - hi), together 22 significant bits.  Per
+// K16 slice two tcgen05.mma kind::f16 (hi, then lo) accumulate into one fp32
+// TMEM accumulator, so the activation block scales never reach the epilogue:
+// per output and 64-group it does one fp32 FMA with the weight scale,
+//     acc += s_g * C_g.
+// (The exact alternative -- integer codes, one accumulator per 32-block,
+// acc += s_g * (S_0 d_0 + S_1 d_1) -- costs three fp32 operations and two TMEM
+// reads per output and group, more than the tensor cores' time for the same
+// group.)  The down GEMM takes h the same way: the gate/up epilogue writes
+// h's Q8_0 codes and scales and the hi/lo split of their product.
 //
-// Warp roles (13 warps): 0-3 producers (cp.async of packed weights, activation
-// rows gathered by token, scales; nibble expansion), 4 MMA issuer (one thread)
-// and TMEM owner, 5-12 epilogue (two warps per TMEM lane quarter).  Every wait
-// is bounded; a wait that runs out records MOE_ERR_TIMEOUT in the status word
-// and every role leaves its loop.
 #include <cuda_fp16.h>
 
 #include "moe_device.cuh"
@@ -88,22 +86,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "r"(taddr));
 }
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// cp.async with zero fill: src_bytes = 0 writes zeros and reads nothing.
-__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Shared-memory operand descriptor, K-major without swizzle: core matrices of
 // 8 rows x 16 bytes; the two 16-byte K halves of a 32-byte row slice are 128
@@ -164,45 +146,44 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
 // ===========================================================================
 // grouped GEMM
 //
-// 9 warps per CTA, one CTA per SM, persistent over the CTA's stages (stage =
-// one 64-group of one tile; tiles blockIdx.x, + gridDim.x, ...; a tile has an
-// even number of stages).
-//   copy warp (lane 0): TMA copies of the packed weights (tensor maps built
-//     per expert on the device), of the activation rows and of their block
-//     scales, as far ahead as the rings allow;
-//   MMA warp (lane 0): the 4 MMAs of each stage.
-//   8 worker warps, each at its own pace: expand stage i's nibbles to fp16
-//     (A buffer i & 1), then apply the scales of stage i-1 to the TMEM block
-//     sums and write a tile's outputs after its last group.
+// One CTA per SM, persistent over its tiles (blockIdx.x, + gridDim.x, ...);
+// a tile is G pipeline stages, one 64-group of K each.  14 warps:
+//   0-7   epilogue: TMEM lane quarter warp & 3, columns 64 * (warp >> 2) ..;
+//         per stage acc += s_g * C_g, a tile's outputs after its last group;
+//   8-11  expansion: packed nibbles of stage i -> fp16 A buffer i % kPfNA
+//         (thread = A row);
+//   12    copies (lane 0): TMA of the packed weights (tensor maps built per
+//         expert on the device) and of the activation hi/lo rows;
+//   13    MMAs (lane 0): 8 per stage, hi then lo of each K16 slice, into TMEM
+//         buffer i % kPfNT.
 // Every hand-off is an mbarrier; every wait is bounded.
 // ===========================================================================
-constexpr int kPfWorkers = 256;
-constexpr int kPfThreads = kPfWorkers + 64;
-constexpr int kPfTmaWarp = 8;                // issues the TMA copies
-constexpr int kPfMmaWarp = 9;                // issues the MMAs
-constexpr int kPfLR = 8, kPfRR = kPfLR + 1;  // packed-weight TMA: stages ahead, ring slots
-constexpr int kPfLB = 4, kPfRB = kPfLB + 2;  // activation TMA: stages ahead, ring slots
-constexpr int kPfRD = 4;                     // block-scale ring slots (one per stage pair)
-constexpr uint32_t kPfTmemCols = 512;        // 2 buffers x 2 blocks x 128 columns
-constexpr int kUxPitch = 129;                // up-projection exchange rows (floats), odd: no bank conflicts
+constexpr int kPfEpiWarps = 8;
+constexpr int kPfExpWarp0 = 8;               // expansion warps 8..11
+constexpr int kPfTmaWarp = 12;
+constexpr int kPfMmaWarp = 13;
+constexpr int kPfThreads = 14 * 32;
+constexpr int kPfNA = 3;                     // expanded-weight buffers
+constexpr int kPfNT = 4;                     // TMEM accumulator buffers (128 columns each)
+constexpr int kPfRB = 4;                     // activation ring slots
+constexpr int kPfRR = 8;                     // packed-weight ring slots
+constexpr uint32_t kPfTmemCols = 512;
 
-constexpr uint32_t kABytes = 16384;   // 4 K-slices x [128 rows x 32 B] fp16 weights, no swizzle
-constexpr uint32_t kBBytes = 16384;   // [N rows][128 B] fp16 activations, 128-byte swizzle (N <= 128)
+constexpr uint32_t kABytes = 16384;   // 4 K16 slices x [128 rows x 32 B] fp16 weights, no swizzle
+constexpr uint32_t kBHalf = 16384;    // [128 rows][128 B] fp16, 128-byte swizzle (hi or lo)
+constexpr uint32_t kBBytes = 2 * kBHalf;
 constexpr uint32_t kRawBytes = 4096;  // [128 rows][32 B] packed weights of a group
-constexpr uint32_t kDBytes = 2048;    // [N rows][4] fp32 block scales of a stage pair
 
 struct PfLayout {
-  uint32_t tile_pre, a, b, raw, d, ux, total;
+  uint32_t tile_pre, a, b, raw, total;
 };
 __host__ __device__ inline PfLayout pf_layout(int E) {
   PfLayout L;
-  L.tile_pre = 576;
+  L.tile_pre = 1024;
   L.a = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
-  L.b = L.a + 2 * kABytes;
+  L.b = L.a + (uint32_t)kPfNA * kABytes;
   L.raw = L.b + (uint32_t)kPfRB * kBBytes;
-  L.d = L.raw + (uint32_t)kPfRR * kRawBytes;
-  L.ux = L.d + (uint32_t)kPfRD * kDBytes;
-  L.total = L.ux + 64u * kUxPitch * 4u;
+  L.total = L.raw + (uint32_t)kPfRR * kRawBytes;
   return L;
 }
 
@@ -255,10 +236,13 @@ __device__ __forceinline__ void tmap_acquire(const CUtensorMap *m) {
   asm volatile("fence.proxy.tensormap::generic.acquire.gpu [%0], 128;" ::"l"(m) : "memory");
 }
 
+// All lanes of the warp wait on `bar` (bounded); false when it ran out.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t det) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, det));
+}
+
 template <int MODE>
-__global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap,
-                                           const __grid_constant__ CUtensorMap dmap) {
-  // 10 warps: one SM sub-partition holds 3 of them, so at most 16K / 96 = 170 registers.
+__global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I;
@@ -267,16 +251,15 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
   const int NWT = MODE == 0 ? I / 64 : H / 128;
   const PfLayout L = pf_layout(a.E);
   uint64_t *rawfull = reinterpret_cast<uint64_t *>(smem);  // [RR] packed weights landed (TMA bytes)
-  uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (8 worker warps)
+  uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (4 expansion warps)
   uint64_t *bfull = rawfree + kPfRR;                        // [RB] activation rows landed (TMA bytes)
   uint64_t *bfree = bfull + kPfRB;                          // [RB] read by the MMAs (commit)
-  uint64_t *aready = bfree + kPfRB;                         // [2]  A buffer written (8 worker warps)
-  uint64_t *accf = aready + 2;                              // [2]  accumulators written (commit)
-  uint64_t *tfree = accf + 2;                               // [2]  accumulators read (8 worker warps)
-  uint64_t *dfull = tfree + 2;                              // [RD] block scales landed (TMA bytes)
-  uint64_t *dfree = dfull + kPfRD;                          // [RD] read (8 worker warps)
-  uint64_t *uxw = dfree + kPfRD;                            // up rows handed over (8 worker warps)
-  uint64_t *uxr = uxw + 1;                                  // up rows consumed (8 worker warps)
+  uint64_t *aready = bfree + kPfRB;                         // [NA] A buffer written (4 expansion warps)
+  uint64_t *afree = aready + kPfNA;                         // [NA] A buffer read by the MMAs (commit)
+  uint64_t *accf = afree + kPfNA;                           // [NT] accumulators written (commit)
+  uint64_t *tfree = accf + kPfNT;                           // [NT] accumulators read (8 epilogue warps)
+  uint64_t *uxw = tfree + kPfNT;                            // up rows handed over (4 warps)
+  uint64_t *uxr = uxw + 1;                                  // up rows consumed (4 warps)
   uint64_t *drain = uxr + 1;                                // teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
@@ -285,9 +268,8 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
   unsigned char *abuf = smem + L.a;
   unsigned char *bbuf = smem + L.b;
   unsigned char *raw = smem + L.raw;
-  unsigned char *dsm = smem + L.d;
-  float *ux = reinterpret_cast<float *>(smem + L.ux);
 
+  prof_start(a.prof, MODE + 1);
   if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int nslot = n_uni + 1;
@@ -296,23 +278,22 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
     *abort_flag = 0;
     for (int s = 0; s < kPfRR; ++s) {
       mbar_init(rawfull + s, 1);
-      mbar_init(rawfree + s, 8);
+      mbar_init(rawfree + s, 4);
     }
     for (int s = 0; s < kPfRB; ++s) {
       mbar_init(bfull + s, 1);
       mbar_init(bfree + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(aready + b, 8);
-      mbar_init(accf + b, 1);
-      mbar_init(tfree + b, 8);
+    for (int s = 0; s < kPfNA; ++s) {
+      mbar_init(aready + s, 4);
+      mbar_init(afree + s, 1);
     }
-    for (int s = 0; s < kPfRD; ++s) {
-      mbar_init(dfull + s, 1);
-      mbar_init(dfree + s, 8);
+    for (int s = 0; s < kPfNT; ++s) {
+      mbar_init(accf + s, 1);
+      mbar_init(tfree + s, kPfEpiWarps);
     }
-    mbar_init(uxw, 8);
-    mbar_init(uxr, 8);
+    mbar_init(uxw, 4);
+    mbar_init(uxr, 4);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -378,7 +359,6 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
       int rtile = -1, issued = 0;
       const CUtensorMap *m0 = nullptr, *m1 = nullptr;
       asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&dmap) : "memory");
       for (int j = 0; j < S && !bad; ++j, cur_next(cr)) {
         // packed weights of stage j
         const int s = j % kPfRR;
@@ -402,27 +382,20 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
         } else {
           tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 128, rawfull + s);
         }
-        // activation rows of stage j
+        // activation hi/lo rows of stage j: boxes of kPfBoxRows rows; rows past
+        // the tile's own land in unused B rows, rows past the array read zero
         const int sb = j % kPfRB;
         if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) {
           bad = true;
           break;
         }
         unsigned char *db = bbuf + (size_t)sb * kBBytes;
-        mbar_arrive_expect_tx(bfull + sb, (uint32_t)cr.tl.n * 128u);
-        for (int i = 0; i < cr.tl.n / (int)kPfBoxRows; ++i)
-          tma_load_2d(db + i * (int)kPfBoxRows * 128, &bmap, cr.g * 64, cr.tl.p0 + i * (int)kPfBoxRows, bfull + sb);
-        if ((j & 1) == 0) {
-          // block scales of groups g, g+1: [N rows][4 floats], 4-float boxes from column 2g
-          const int jp = j >> 1, ds = jp % kPfRD;
-          if (jp >= kPfRD && !mbar_wait(dfree + ds, (uint32_t)(jp / kPfRD - 1) & 1u, a.status, kDetPfEmpty)) {
-            bad = true;
-            break;
-          }
-          unsigned char *dd = dsm + (size_t)ds * kDBytes;
-          mbar_arrive_expect_tx(dfull + ds, (uint32_t)cr.tl.n * 16u);
-          for (int i = 0; i < cr.tl.n / (int)kPfBoxRows; ++i)
-            tma_load_2d(dd + i * (int)kPfBoxRows * 16, &dmap, cr.g * 2, cr.tl.p0 + i * (int)kPfBoxRows, dfull + ds);
+        const int nbox = (cr.tl.n + (int)kPfBoxRows - 1) / (int)kPfBoxRows;
+        mbar_arrive_expect_tx(bfull + sb, (uint32_t)nbox * kPfBoxRows * 256u);
+        for (int i = 0; i < nbox; ++i) {
+          const int y = cr.tl.p0 + i * (int)kPfBoxRows;
+          tma_load_2d(db + i * (int)kPfBoxRows * 128, &bmap, cr.g * 128, y, bfull + sb);
+          tma_load_2d(db + kBHalf + i * (int)kPfBoxRows * 128, &bmap, cr.g * 128 + 64, y, bfull + sb);
         }
         issued = j + 1;
         if (*abort_flag) bad = true;
@@ -434,8 +407,6 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
         mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
       for (int j = max(0, issued - kPfRB); j < issued; ++j)
         mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
-      for (int jp = max(0, (issued + 1) / 2 - kPfRD); jp < (issued + 1) / 2; ++jp)
-        mbar_wait(dfull + jp % kPfRD, (uint32_t)(jp / kPfRD) & 1u, a.status, kDetPfDrain);
     }
     __syncwarp();
   } else if (warp == kPfMmaWarp) {
@@ -444,44 +415,33 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
       bool bad = false;
       PfCur cm;
       cur_begin(cm);
-      uint64_t adesc[2][4], bdesc[kPfRB][4];
-#pragma unroll
-      for (int b = 0; b < 2; ++b)
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) adesc[b][k4] = umma_desc(smem_u32(abuf + (size_t)b * kABytes) + k4 * 4096);
-#pragma unroll
-      for (int r = 0; r < kPfRB; ++r)
-#pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4)
-          bdesc[r][k4] = umma_desc_sw128(smem_u32(bbuf + (size_t)r * kBBytes) + (uint32_t)(k4 * 32));
+      // descriptors advance by (byte offset >> 4) in their start-address field
+      const uint64_t a0 = umma_desc(smem_u32(abuf));
+      const uint64_t b0 = umma_desc_sw128(smem_u32(bbuf));
       int done = 0;
       for (int j = 0; j < S && !bad; ++j, cur_next(cm)) {
-        const int buf = j & 1, sb = j % kPfRB;
-        if (!mbar_wait(aready + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfFull) ||
+        const int na = j % kPfNA, sb = j % kPfRB, tb = j % kPfNT;
+        if (!mbar_wait(aready + na, (uint32_t)(j / kPfNA) & 1u, a.status, kDetPfFull) ||
             !mbar_wait(bfull + sb, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull) ||
-            (j >= 2 && !mbar_wait(tfree + buf, (uint32_t)((j >> 1) - 1) & 1u, a.status, kDetPfAccFree)) ||
+            (j >= kPfNT && !mbar_wait(tfree + tb, (uint32_t)(j / kPfNT - 1) & 1u, a.status, kDetPfAccFree)) ||
             *abort_flag) {
           bad = true;
           break;
         }
         tc_fence_after();
         const uint32_t idesc = pf_idesc(cm.tl.n);
-        const uint32_t d = tmem + (uint32_t)(buf * 256);
-        uint64_t bd[4];
+        const uint32_t d = tmem + (uint32_t)(tb * 128);
+        const uint64_t ad = a0 + (uint64_t)((na * kABytes) >> 4);
+        const uint64_t bd = b0 + (uint64_t)((sb * kBBytes) >> 4);
 #pragma unroll
-        for (int r = 0; r < kPfRB; ++r)
-          if (r == sb)
-#pragma unroll
-            for (int k4 = 0; k4 < 4; ++k4) bd[k4] = bdesc[r][k4];
-#pragma unroll
-        for (int b = 0; b < 2; ++b)
-#pragma unroll
-          for (int ks = 0; ks < 2; ++ks) {
-            const int k4 = 2 * b + ks;
-            umma_f16(d + (uint32_t)(b * 128), buf ? adesc[1][k4] : adesc[0][k4], bd[k4], idesc, (uint32_t)ks);
-          }
-        umma_commit(accf + buf);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const uint64_t ak = ad + (uint64_t)((k4 * 4096) >> 4);
+          umma_f16(d, ak, bd + (uint64_t)((k4 * 32) >> 4), idesc, (uint32_t)(k4 > 0));
+          umma_f16(d, ak, bd + (uint64_t)((kBHalf + k4 * 32) >> 4), idesc, 1u);
+        }
+        umma_commit(accf + tb);
         umma_commit(bfree + sb);
+        umma_commit(afree + na);
         done = j + 1;
       }
       if (bad) *abort_flag = 1;
@@ -491,208 +451,191 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
       }
     }
     __syncwarp();
+  } else if (warp >= kPfExpWarp0) {
+    // ================================================================ expansion
+    bool bad = false;
+    const int r = tid - kPfExpWarp0 * 32;  // A row
+    for (int i = 0; i < S && !bad; ++i) {
+      const int ra = i % kPfRR, na = i % kPfNA;
+      if (!warp_wait(rawfull + ra, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull) ||
+          (i >= kPfNA && !warp_wait(afree + na, (uint32_t)(i / kPfNA - 1) & 1u, a.status, kDetPfFull))) {
+        bad = true;
+        break;
+      }
+      const uint4 *src = reinterpret_cast<const uint4 *>(raw + (size_t)ra * kRawBytes + r * 32);
+      const uint4 s0 = src[0], s1 = src[1];
+      unsigned char *ab = abuf + (size_t)na * kABytes;
+      // byte j: low nibble = element j, high nibble = element j + 32; slice k4
+      // = elements 16 k4 .. 16 k4 + 15
+#pragma unroll
+      for (int k4 = 0; k4 < 4; ++k4) {
+        const uint4 v = (k4 & 1) ? s1 : s0;
+        const int sh = (k4 >> 1) * 4;
+        uint32_t h[8];
+        nib4_to_f16((v.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
+        nib4_to_f16((v.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
+        nib4_to_f16((v.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
+        nib4_to_f16((v.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
+        unsigned char *dst = ab + k4 * 4096;
+        *reinterpret_cast<uint4 *>(dst + il_off(r, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(dst + il_off(r, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(aready + na);
+        mbar_arrive(rawfree + ra);
+      }
+      if (*abort_flag) bad = true;
+    }
+    if (bad) *abort_flag = 1;
   } else {
-    // ================================================================ workers
+    // ================================================================ epilogue
     bool bad = false;
     const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
-    const int crow = tid & 127, chalf = tid >> 7;  // expansion: row, 16-byte half of its 32 packed bytes
-    const int q = warp & 3, half = warp >> 2;      // epilogue: TMEM lane quarter, 16-column chunks half, +2, ..
+    const int q = warp & 3, half = warp >> 2;  // TMEM lane quarter, 64-column half
     const int row = q * 32 + lane;
-    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 64);
     // weight scales of this thread's row: 4 bytes (groups g, g+1) per stage
     // pair, loaded one pair ahead
     auto scale_row = [&](const PfTile &tl) -> const uint32_t * {
       const unsigned char *blob = static_cast<const unsigned char *>(a.table[tl.e]);
       if (MODE == 0) {
         const size_t base = row < 64 ? 0 : mg;
-        const size_t r = (size_t)tl.wt * 64 + (row & 63);
-        return reinterpret_cast<const uint32_t *>(blob + base + (size_t)I * (size_t)(H / 2) + r * (size_t)(H / 64) * 2);
+        const size_t rr = (size_t)tl.wt * 64 + (row & 63);
+        return reinterpret_cast<const uint32_t *>(blob + base + (size_t)I * (size_t)(H / 2) + rr * (size_t)(H / 64) * 2);
       }
-      const size_t r = (size_t)tl.wt * 128 + row;
-      return reinterpret_cast<const uint32_t *>(blob + 2 * mg + (size_t)H * (size_t)(I / 2) + r * (size_t)(I / 64) * 2);
+      const size_t rr = (size_t)tl.wt * 128 + row;
+      return reinterpret_cast<const uint32_t *>(blob + 2 * mg + (size_t)H * (size_t)(I / 2) + rr * (size_t)(I / 64) * 2);
     };
-    PfCur cw;
+    PfCur cw;  // scale prefetch cursor, one stage pair ahead
     cur_begin(cw);
     uint32_t w_next = 0, w_cur = 0;
     if (S > 0) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
     PfCur ce;
     cur_begin(ce);
-    float2 acc[4][8];
+    float acc[64];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = make_float2(0.0f, 0.0f);
+    for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
     int tcount = 0;
+    float *ux = a.ux + (size_t)blockIdx.x * 64 * 128;  // this CTA's up-row exchange [64 rows][128 cols]
 
-    for (int i = 0; i <= S && !bad; ++i) {
-      // expansion of stage i: row crow, bytes 16 chalf ..: K-slices chalf (low
-      // nibbles) and 2 + chalf (high nibbles)
-      if (i < S) {
-        if (!__all_sync(0xffffffffu, mbar_wait(rawfull + i % kPfRR, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull))) {
-          bad = true;
-          break;
-        }
-        const uint4 src = *reinterpret_cast<const uint4 *>(raw + (size_t)(i % kPfRR) * kRawBytes + crow * 32 + chalf * 16);
-        unsigned char *ab = abuf + (size_t)(i & 1) * kABytes;
-#pragma unroll
-        for (int hi = 0; hi < 2; ++hi) {
-          const int sh = hi * 4;
-          uint32_t h[8];
-          nib4_to_f16((src.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
-          nib4_to_f16((src.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
-          nib4_to_f16((src.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
-          nib4_to_f16((src.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
-          unsigned char *dst = ab + (2 * hi + chalf) * 4096;
-          *reinterpret_cast<uint4 *>(dst + il_off(crow, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4 *>(dst + il_off(crow, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(aready + (i & 1));
-          mbar_arrive(rawfree + i % kPfRR);
-        }
-      }
-      if (i == 0) continue;
-      // scales of stage j = i-1
-      const int j = i - 1, buf = j & 1, jp = j >> 1, ds = jp % kPfRD;
+    for (int j = 0; j < S && !bad; ++j) {
+      const int tb = j % kPfNT;
       if ((j & 1) == 0) {
         w_cur = w_next;
         cur_next(cw);
         cur_next(cw);
         if (cw.t < n_tiles) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
       }
-      if (!__all_sync(0xffffffffu, mbar_wait(accf + buf, (uint32_t)(j >> 1) & 1u, a.status, kDetPfAccFull) &&
-                                       mbar_wait(dfull + ds, (uint32_t)(jp / kPfRD) & 1u, a.status, kDetPfFull))) {
+      if (!warp_wait(accf + tb, (uint32_t)(j / kPfNT) & 1u, a.status, kDetPfAccFull)) {
         bad = true;
         break;
       }
       tc_fence_after();
-      const int nch = ce.tl.n >> 4;
+      const int nch = ce.tl.n >> 4;  // 16-column chunks of the tile
       const float sg = __half2float(__ushort_as_half((unsigned short)((ce.g & 1) ? (w_cur >> 16) : (w_cur & 0xFFFFu))));
-      const float2 sg2 = make_float2(sg, sg);
-      const float *dp = reinterpret_cast<const float *>(dsm + (size_t)ds * kDBytes) + 2 * (ce.g & 1);  // [col][4]
 #pragma unroll
-      for (int ci = 0; ci < 4; ++ci) {
-        const int c = half + 2 * ci;
+      for (int c2 = 0; c2 < 2; ++c2) {
+        const int c = half * 4 + c2 * 2;  // chunks c, c + 1
         if (c < nch) {
-          float2 dv[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) dv[k] = *reinterpret_cast<const float2 *>(dp + (c * 16 + k) * 4);
           uint32_t v0[16], v1[16];
-          tmem_ld16(tq + (uint32_t)(buf * 256 + c * 16), v0);
-          tmem_ld16(tq + (uint32_t)(buf * 256 + 128 + c * 16), v1);
+          tmem_ld16(tq + (uint32_t)(tb * 128 + c2 * 32), v0);
+          tmem_ld16(tq + (uint32_t)(tb * 128 + c2 * 32 + 16), v1);
           tmem_ld_wait();
 #pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const float2 dap = make_float2(dv[2 * jj].x, dv[2 * jj + 1].x);
-            const float2 dbp = make_float2(dv[2 * jj].y, dv[2 * jj + 1].y);
-            const float2 s0 = make_float2(__uint_as_float(v0[2 * jj]), __uint_as_float(v0[2 * jj + 1]));
-            const float2 s1 = make_float2(__uint_as_float(v1[2 * jj]), __uint_as_float(v1[2 * jj + 1]));
-            const float2 fb = __ffma2_rn(s1, dbp, __fmul2_rn(s0, dap));
-            acc[ci][jj] = __ffma2_rn(sg2, fb, acc[ci][jj]);
+          for (int k = 0; k < 16; ++k) {
+            acc[c2 * 32 + k] = ffma(sg, __uint_as_float(v0[k]), acc[c2 * 32 + k]);
+            acc[c2 * 32 + 16 + k] = ffma(sg, __uint_as_float(v1[k]), acc[c2 * 32 + 16 + k]);
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(tfree + buf);
-        if (j & 1) mbar_arrive(dfree + ds);
-      }
+      if (lane == 0) mbar_arrive(tfree + tb);
       if (ce.g == G - 1) {
-        // the tile's outputs
+        // the tile's outputs; this thread holds columns 64 half + 0..63
         const PfTile tl = ce.tl;
+        const int col0 = half * 64;
         if (MODE == 1) {
           float *yc = a.y + (size_t)tl.p0 * H + (size_t)tl.wt * 128 + row;
 #pragma unroll
-          for (int ci = 0; ci < 4; ++ci) {
-            const int c = half + 2 * ci;
-            if (c < nch) {
-#pragma unroll
-              for (int jj = 0; jj < 8; ++jj) {
-                const int col = c * 16 + 2 * jj;
-                if (col < tl.nval) yc[(size_t)col * H] = acc[ci][jj].x;
-                if (col + 1 < tl.nval) yc[(size_t)(col + 1) * H] = acc[ci][jj].y;
-              }
-            }
-          }
+          for (int k = 0; k < 64; ++k)
+            if (col0 + k < tl.nval) yc[(size_t)(col0 + k) * H] = acc[k];
         } else {
-          // Rows 64..127 hold u of rows 0..63 (g): hand u over, then SwiGLU and
-          // Q8_0 of h along I (one 32-block = one warp's lanes), per token.
+          // Rows 64..127 hold u of rows 0..63 (g): hand u over through this
+          // CTA's exchange rows in global memory, then SwiGLU and Q8_0 of h
+          // along I (one 32-block = one warp's lanes), per token.
           if (q >= 2) {
-            if (tcount > 0 &&
-                !__all_sync(0xffffffffu, mbar_wait(uxr, (uint32_t)(tcount - 1) & 1u, a.status, kDetPfFull))) {
+            if (tcount > 0 && !warp_wait(uxr, (uint32_t)(tcount - 1) & 1u, a.status, kDetPfFull)) {
               bad = true;
               break;
             }
+            float *uw = ux + (size_t)(row - 64) * 128 + col0;
 #pragma unroll
-            for (int ci = 0; ci < 4; ++ci) {
-              const int c = half + 2 * ci;
-              if (c < nch) {
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                  ux[(row - 64) * kUxPitch + c * 16 + 2 * jj] = acc[ci][jj].x;
-                  ux[(row - 64) * kUxPitch + c * 16 + 2 * jj + 1] = acc[ci][jj].y;
-                }
-              }
+            for (int k = 0; k < 64; k += 4)
+              if (col0 + k < tl.n) *reinterpret_cast<float4 *>(uw + k) = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(uxw);
+          } else {
+            if (!warp_wait(uxw, (uint32_t)tcount & 1u, a.status, kDetPfFull)) {
+              bad = true;
+              break;
             }
-          }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(uxw);
-          if (!__all_sync(0xffffffffu, mbar_wait(uxw, (uint32_t)tcount & 1u, a.status, kDetPfFull))) {
-            bad = true;
-            break;
-          }
-          if (q < 2) {
-            // h = SiLU(g) * u and its Q8_0 codes in fast fp32 (this path is held
-            // to the layer's tolerance, not to the fixed-order bits)
             const int ii = tl.wt * 64 + row;  // row of I
-            __half *hh = static_cast<__half *>(a.hh);
+            const float *ur = ux + (size_t)row * 128 + col0;
+            __half *hs = static_cast<__half *>(a.hs);
+            const size_t hcol = (size_t)(ii >> 6) * 128 + (ii & 63);
 #pragma unroll
-            for (int ci = 0; ci < 4; ++ci) {
-              const int c = half + 2 * ci;
-              if (c < nch) {
+            for (int k = 0; k < 64; k += 4) {
+              if (col0 + k < tl.n) {
+                const float4 u4 = *reinterpret_cast<const float4 *>(ur + k);
+                const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
-                for (int jj = 0; jj < 16; ++jj) {
-                  const int col = c * 16 + jj;
-                  const float gv = (jj & 1) ? acc[ci][jj >> 1].y : acc[ci][jj >> 1].x;
-                  const float h = __fdividef(gv, 1.0f + __expf(-gv)) * ux[row * kUxPitch + col];
+                for (int m = 0; m < 4; ++m) {
+                  // h = SiLU(g) * u and its Q8_0 codes in fast fp32 (this path is
+                  // held to the layer's tolerance, not to the fixed-order bits)
+                  const float gv = acc[k + m];
+                  const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv[m];
                   const float amax = warp_max(fabsf(h));
                   const float d = amax * (1.0f / 127.0f);
                   const float inv = amax > 0.0f ? __fdividef(127.0f, amax) : 0.0f;
                   const int qv = (int)fminf(fmaxf(rintf(h * inv), -127.0f), 127.0f);
+                  const int col = col0 + k + m;
                   if (col < tl.nval) {
                     const size_t p = (size_t)(tl.p0 + col);
                     a.hq[p * I + ii] = (int8_t)qv;
-                    hh[p * I + ii] = __int2half_rn(qv);
                     if (lane == 0) a.hd[p * (I / 32) + ii / 32] = d;
+                    const float hv = (float)qv * d;  // dequantised h, split hi + lo
+                    const __half hi = __float2half_rn(hv);
+                    const __half lo = __float2half_rn(hv - __half2float(hi));
+                    hs[p * (size_t)(2 * I) + hcol] = hi;
+                    hs[p * (size_t)(2 * I) + hcol + 64] = lo;
                   }
                 }
               }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(uxr);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(uxr);
           ++tcount;
         }
 #pragma unroll
-        for (int ci = 0; ci < 4; ++ci)
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) acc[ci][jj] = make_float2(0.0f, 0.0f);
+        for (int k = 0; k < 64; ++k) acc[k] = 0.0f;
       }
       cur_next(ce);
       if (*abort_flag) bad = true;
     }
     if (bad) *abort_flag = 1;
   }
-  // teardown: every copy and MMA of this CTA has completed (see the control warp)
+  // teardown: every copy and MMA of this CTA has completed (see the MMA warp)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kPfTmemCols);
   }
+  prof_end(a.prof, MODE + 1);
 }
 
 // Tensor maps of the packed weights of the union's experts and the shared
@@ -702,6 +645,7 @@ __global__ void __maxnreg__(160) k_gemm_pf(const PfArgs a, const __grid_constant
 __global__ void __launch_bounds__(32) k_make_maps(const PfArgs a, const __grid_constant__ CUtensorMap tgu,
                                                  const __grid_constant__ CUtensorMap tdn, CUtensorMap *maps) {
   const int e = blockIdx.x;
+  prof_end(a.prof, 0);
   if (e < a.E && a.off[e + 1] == a.off[e]) return;  // not in the union
   const unsigned char *blob = static_cast<const unsigned char *>(a.table[e]);
   if ((reinterpret_cast<uintptr_t>(blob) & 15) != 0) {
@@ -736,7 +680,7 @@ cudaError_t launch_make_maps(const PfArgs &a, const CUtensorMap &tgu, const CUte
   return cudaGetLastError();
 }
 
-cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUtensorMap &dmap, int grid, cudaStream_t s) {
+cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s) {
   const size_t smem = pf_layout(a.E).total;
   if (smem > (size_t)kMaxSmem) return cudaErrorInvalidConfiguration;
   cudaError_t err;
@@ -744,12 +688,12 @@ cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, const CUten
     static int smem_set0[64] = {0};
     err = ensure_smem(k_gemm_pf<0>, smem, smem_set0);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
+    k_gemm_pf<0><<<grid, kPfThreads, smem, s>>>(a, bmap);
   } else {
     static int smem_set1[64] = {0};
     err = ensure_smem(k_gemm_pf<1>, smem, smem_set1);
     if (err != cudaSuccess) return err;
-    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap, dmap);
+    k_gemm_pf<1><<<grid, kPfThreads, smem, s>>>(a, bmap);
   }
   return cudaGetLastError();
 }
@@ -829,18 +773,35 @@ cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s) {
 }
 
 // ===========================================================================
-// x's fp16 codes in pair order: xg[p] = xh[pair_tok[p]] (the gate/up GEMM's
-// activation rows, copied by TMA boxes of consecutive rows).
+// The gate/up GEMM's activation rows in pair order, as an fp16 hi/lo split of
+// the Q8_0-dequantised x: for p and h, x^ = q[t][h] * d[t][h / 32] (t =
+// pair_tok[p]), hi = fp16(x^), lo = fp16(x^ - hi); row p of xg holds, per
+// 64-group g, hi of the group's 64 elements at 128 g and lo at 128 g + 64.
+// A thread writes 8 elements (16 bytes of hi, 16 of lo).
 // ===========================================================================
 __global__ void __launch_bounds__(256) k_gather_rows(const GatherRowsArgs a) {
   const int64_t P = (int64_t)a.T * (a.k + 1);
-  const int w = a.H / 8;  // 16-byte units per row
+  const int w = a.H / 8;  // 8-element units per row
   const int64_t n = P * w;
-  const uint4 *src = static_cast<const uint4 *>(a.xh);
-  uint4 *dst = static_cast<uint4 *>(a.xg);
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t p = i / w, c = i - p * w;
-    dst[i] = src[(int64_t)a.pair_tok[p] * w + c];
+    const int64_t p = i / w;
+    const int h = (int)(i - p * w) * 8;
+    const int64_t t = a.pair_tok[p];
+    const uint2 qv = *reinterpret_cast<const uint2 *>(a.xq + t * a.H + h);
+    const float d = a.xd[t * (a.H / 32) + h / 32];
+    const int8_t *qb = reinterpret_cast<const int8_t *>(&qv);
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const float x0 = (float)qb[2 * m] * d, x1 = (float)qb[2 * m + 1] * d;
+      const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
+      const __half l0 = __float2half_rn(x0 - __half2float(h0)), l1 = __float2half_rn(x1 - __half2float(h1));
+      hi[m] = (uint32_t)__half_as_ushort(h0) | ((uint32_t)__half_as_ushort(h1) << 16);
+      lo[m] = (uint32_t)__half_as_ushort(l0) | ((uint32_t)__half_as_ushort(l1) << 16);
+    }
+    __half *row = static_cast<__half *>(a.xg) + p * (2 * (int64_t)a.H) + (h >> 6) * 128 + (h & 63);
+    *reinterpret_cast<uint4 *>(row) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4 *>(row + 64) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -850,28 +811,6 @@ cudaError_t launch_gather_rows(const GatherRowsArgs &a, cudaStream_t s) {
   int64_t blocks = (n + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
   k_gather_rows<<<(unsigned)blocks, 256, 0, s>>>(a);
-  return cudaGetLastError();
-}
-
-// ===========================================================================
-// x's Q8_0 block scales in pair order (rows of H/32): the gate/up GEMM copies
-// a tile's scales of two groups as 4-float boxes.
-// ===========================================================================
-__global__ void __launch_bounds__(256) k_gather_scales(const GatherScaleArgs a) {
-  const int64_t P = (int64_t)a.T * (a.k + 1);
-  const int64_t n = P * a.nb;
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t p = i / a.nb, b = i - p * a.nb;
-    a.xdp[i] = a.xd[(int64_t)a.pair_tok[p] * a.nb + b];
-  }
-}
-
-cudaError_t launch_gather_scales(const GatherScaleArgs &a, cudaStream_t s) {
-  const int64_t n = (int64_t)a.T * (a.k + 1) * a.nb;
-  if (n == 0) return cudaSuccess;
-  int64_t blocks = (n + 255) / 256;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  k_gather_scales<<<(unsigned)blocks, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 
@@ -895,6 +834,7 @@ __global__ void __launch_bounds__(256) k_combine(const CombineArgs a) {
     }
     reinterpret_cast<float4 *>(a.out + (size_t)t * a.H)[c] = o;
   }
+  prof_end(a.prof, 2);
 }
 
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {

@@ -43,22 +43,6 @@ cudaError_t make_f16_map(CUtensorMap *map, const void *base, uint64_t rows, uint
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t make_f32x4_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-  EncodeTiledFn enc = encoder();
-  if (enc == nullptr) return cudaErrorNotSupported;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (cols * 4) % 16 != 0 || rows == 0 || box_rows == 0 ||
-      box_rows > 256)
-    return cudaErrorInvalidValue;
-  const cuuint64_t dims[2] = {cols, rows};
-  const cuuint64_t strides[1] = {cols * 4};
-  const cuuint32_t box[2] = {4, box_rows};
-  const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
-                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
-}
-
 cudaError_t make_u8_map(CUtensorMap *map, const void *base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
   EncodeTiledFn enc = encoder();
   if (enc == nullptr) return cudaErrorNotSupported;

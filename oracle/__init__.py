@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "or_block_dot": (ctypes.c_int32, [P, i32, i32, i32, i32, P]),
             "or_expert_dot": (f32, [P, i32, i32, i32, P, P]),
             "or_expert_ffn": (None, [P, i32, i32, P, P, P, P, P, P, P, P]),
+            "or_expert_down": (None, [P, i32, i32, P, P, P]),
             "or_moe_layer": (i32, [i32, i32, i32, i32, i32, P, P, P, P, P]),
             "or_moe_layer_tokens": (i32, [i32, i32, i32, i32, P, P, P, P, i32, P]),
         }
@@ -196,6 +197,16 @@ def expert_ffn(blob: np.ndarray, H: int, I: int, xq: np.ndarray, xd: np.ndarray)
     y = np.zeros(H, np.float32)
     lib().or_expert_ffn(_p(blob), H, I, _p(xq), _p(xd), _p(g), _p(u), _p(h), _p(hq), _p(hd), _p(y))
     return dict(g=g, u=u, h=h, hq=hq, hd=hd, y=y)
+
+
+def expert_down(blob: np.ndarray, H: int, I: int, hq: np.ndarray, hd: np.ndarray) -> np.ndarray:
+    """y [H] of one expert from given codes hq [I] and scales hd [I/32]."""
+    blob = _c(blob, np.uint8)
+    hq = _c(hq, np.int8)
+    hd = _c(hd, np.float32)
+    y = np.zeros(H, np.float32)
+    lib().or_expert_down(_p(blob), H, I, _p(hq), _p(hd), _p(y))
+    return y
 
 
 class _Trace(ctypes.Structure):

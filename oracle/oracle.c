@@ -294,11 +294,15 @@ float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, co
   return total;
 }
 
+void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y) {
+  const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
+  for (int m = 0; m < H; ++m) y[m] = or_expert_dot(down, H, I, m, hq, hd);
+}
+
 void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
                    float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
   const uint8_t *gate = blob;
   const uint8_t *up = blob + or_matrix_bytes(I, H);
-  const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
   float *hh = (float *)malloc(sizeof(float) * (size_t)I);
   int8_t *q = (int8_t *)malloc((size_t)I);
   float *dd = (float *)malloc(sizeof(float) * (size_t)(I / 32));
@@ -313,8 +317,7 @@ void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const fl
   if (h) memcpy(h, hh, sizeof(float) * (size_t)I);
   if (hq) memcpy(hq, q, (size_t)I);
   if (hd) memcpy(hd, dd, sizeof(float) * (size_t)(I / 32));
-  if (y)
-    for (int m = 0; m < H; ++m) y[m] = or_expert_dot(down, H, I, m, q, dd);
+  if (y) or_expert_down(blob, H, I, q, dd, y);
   free(dd);
   free(q);
   free(hh);

@@ -81,6 +81,10 @@ int32_t or_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_
 /* Row n of the matrix against the Q8_0 vector (q, d), in the fixed order. */
 float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d);
 
+/* The down projection of one expert from given Q8_0 codes of h:
+ * y[m] = row m of the down matrix against (hq[I], hd[I/32]), m < H. */
+void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y);
+
 /* One SwiGLU expert on one token.  Any of the intermediate outputs may be NULL.
  * g[I], u[I], h[I], hq[I], hd[I/32], y[H]. */
 void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,

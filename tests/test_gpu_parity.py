@@ -249,3 +249,28 @@ def test_misaligned_blob_reports_device_error():
     torch.cuda.synchronize()
     st = moe.ws_slice(ws, moe.moe_workspace_view(d, x.shape[0], ws).status, (4,), torch.int32).cpu()
     assert int(st[0]) == -8   # MOE_ERR_DEVICE
+
+
+@pytest.mark.parametrize("path", [1, 2])
+def test_profile_records_each_call_and_leaves_output_unchanged(path):
+    """Device-stamped per-call timing: one record per call with positive phase
+    durations no longer than the call span, and bitwise the same output."""
+    moe = _moe()
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    out0, ws, d = gpu_layer(w, x, Wr, blobs, path=path)
+    moe.moe_profile_enable(True)
+    try:
+        out = torch.empty_like(out0)
+        for _ in range(3):
+            moe.moe_layer_forward(d, x, Wr, moe.expert_table(blobs), out, ws, path=path)
+        rec = moe.moe_profile_read(16)
+        again = moe.moe_profile_read(16)
+    finally:
+        moe.moe_profile_enable(False)
+    assert torch.equal(out, out0)
+    assert len(rec) == 3 and again == []
+    for r in rec:
+        assert all(v > 0 for v in r), r
+        assert max(r[:3]) <= r[3] * (1 + 1e-6), r
+        assert r[3] < 1000.0, r       # milliseconds

@@ -5,10 +5,12 @@ C ABI with path = MOE_PATH_PREFILL.
 Bit-exact: the Q8_0 codes and scales of x, the router logits, the top-k
 indices and weights, the bucket counts / offsets / union / permutation.
 Final outputs: within rel-L2 <= 1e-4 and max-abs <= 2e-3 * rms(ref).  The
-grouped GEMM adds the exact 32-block sums in another fp32 order than the
-oracle, so a Q8_0 code of SiLU(g)*u may differ by one where h lies within
-rounding of a half-integer multiple of its block scale; those flips are
-counted and bounded (at most 1 in 1000 codes, never by more than one)."""
+grouped GEMM multiplies the weights by an fp16 hi/lo split of the dequantised
+activations (22 significant bits) and accumulates in fp32 in another order
+than the oracle, so its sums differ from the oracle's by about 1e-6 relative
+and a Q8_0 code of SiLU(g)*u may differ by one where h lies within that of a
+half-integer multiple of its block scale; those flips are counted and bounded
+(at most 1 in 1000 codes, never by more than one)."""
 import numpy as np
 import pytest
 import torch
@@ -52,17 +54,45 @@ def _check_hq(g, tr, T, k):
     ref = tr["hd"].astype(np.float64)
     got = hd.astype(np.float64)
     assert np.all(np.abs(got - ref) <= 1e-5 * np.abs(ref) + 1e-30)
+    return int(diff.astype(bool).sum())
+
+
+def _out_from_codes(g, tr, blobs, w, T):
+    """The oracle's down projections of the path's own h codes, combined in
+    the layer's order (float64 sums of float32 terms)."""
+    hq, hd = hq_by_slot(g, T, w.k)
+    bl = blobs.cpu().numpy()
+    out = np.zeros((T, w.H), np.float64)
+    for t in range(T):
+        out[t] = orc.expert_down(bl[w.E], w.H, w.I, hq[t, w.k], hd[t, w.k])
+        for s in range(w.k):
+            e = int(tr["idx"][t, s])
+            out[t] += np.float64(tr["w"][t, s]) * orc.expert_down(bl[e], w.H, w.I, hq[t, s], hd[t, s])
+    return out
 
 
 def _check_full(w, x, Wr, blobs):
+    """Routing bit-exact; h codes within the flip bound; outputs within 1e-5 of
+    the oracle's down projection of the path's own codes; and within the layer's
+    tolerance of the oracle itself wherever that tolerance covers a flip: a
+    flipped code moves every output of its token by up to 8 * s * d, which at
+    I = 128 can reach 5e-3 rms (beyond the 2e-3 max-abs bound), at I >= 1024
+    less than half of it."""
     T = x.shape[0]
     out, ws, d = gpu_layer(w, x, Wr, blobs, path=PREFILL)
     ref, tr = oracle_layer_from_device(x, Wr, blobs, w.H, w.I, w.E, w.k)
     g = ws_trace(ws, d, T)
     _check_routing(g, tr)
-    _check_hq(g, tr, T, w.k)
-    ok, rel, mrel = within_tolerance(out.cpu().numpy(), ref)
-    assert ok, (rel, mrel)
+    flips = _check_hq(g, tr, T, w.k)
+    got = out.cpu().numpy()
+    oc = _out_from_codes(g, tr, blobs, w, T)
+    nr = np.linalg.norm(oc)
+    rms = np.sqrt(np.mean(oc * oc))
+    assert np.linalg.norm(got - oc) <= 1e-5 * nr, np.linalg.norm(got - oc) / nr
+    assert np.abs(got - oc).max() <= 1e-4 * rms, np.abs(got - oc).max() / rms
+    if flips == 0 or w.I >= 1024:
+        ok, rel, mrel = within_tolerance(got, ref)
+        assert ok, (rel, mrel, flips)
     return out, ref
 
 

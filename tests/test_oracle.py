@@ -285,6 +285,23 @@ def test_expert_ffn_vs_float64():
     assert np.allclose(r["y"], y, rtol=1e-5, atol=1e-5 * np.abs(y).max())
 
 
+def test_expert_down_from_codes_vs_float64():
+    """The down projection from given codes: the dequantised matrix times the
+    dequantised codes in float64; and the FFN's own y from its own codes."""
+    H, I = 256, 128
+    blob = orc_blob(H, I)
+    _, _, Wd = dequant_blob(blob, H, I)
+    hq, hd = orc.quant_q8_0((rng.normal(size=I) * 3).astype(np.float32))
+    y = orc.expert_down(blob, H, I, hq, hd)
+    ref = Wd @ (hq.astype(np.float64) * np.repeat(hd.astype(np.float64), 32))
+    mag = np.abs(Wd) @ np.abs(hq.astype(np.float64) * np.repeat(hd.astype(np.float64), 32))
+    assert np.all(np.abs(y - ref) <= (I // 64 + 8) * 2.0**-23 * mag)
+    x = rng.normal(size=H).astype(np.float32)
+    xq, xd = orc.quant_q8_0(x)
+    r = orc.expert_ffn(blob, H, I, xq, xd)
+    assert np.array_equal(orc.expert_down(blob, H, I, r["hq"], r["hd"]).view(np.uint32), r["y"].view(np.uint32))
+
+
 # ----------------------------------------------------------------- layer
 def orc_blob(H, I, seed=None):
     parts = []
