@@ -101,7 +101,7 @@ size_t moe_workspace_bytes(const moe_dims *dims, int32_t T_max);
 
 /* Same for an explicit path: MOE_PATH_PREFILL needs the prefill segments (the
  * fp16 hi/lo activation rows and the per-pair down rows, about
- * T*(k+1)*(2H+I)*4 bytes, plus 8 MB) for any T; MOE_PATH_DECODE never does. */
+ * T*(k+1)*(2H+I)*4 bytes) for any T; MOE_PATH_DECODE never does. */
 size_t moe_workspace_bytes_path(const moe_dims *dims, int32_t T_max, int32_t path);
 
 /* Q8_0 quantisation of rows x T x cols fp32 (cols % 32 == 0):

@@ -280,7 +280,6 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   pa.hd = at<float>(ws, L.hd);
   pa.hs = at<void>(ws, L.hs);
   pa.y = at<float>(ws, L.y);
-  pa.ux = at<float>(ws, L.ux);
   pa.status = status;
   pa.prof = prof;
   const size_t P = (size_t)T * (size_t)(d.k + 1);
@@ -289,7 +288,7 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   err = make_f16_map(&map_x, gr.xg, (uint64_t)P, 2 * (uint64_t)d.H, kPfBoxRows);
   if (err == cudaSuccess) err = make_f16_map(&map_h, pa.hs, (uint64_t)P, 2 * (uint64_t)d.I, kPfBoxRows);
   // the templates' address is replaced per expert on the device
-  if (err == cudaSuccess) err = make_u8_map(&tmpl_gu, pa.maps, (uint64_t)d.I, (uint64_t)d.H / 2, 64);
+  if (err == cudaSuccess) err = make_u8_map(&tmpl_gu, pa.maps, (uint64_t)d.I, (uint64_t)d.H / 2, 128);
   if (err == cudaSuccess) err = make_u8_map(&tmpl_dn, pa.maps, (uint64_t)d.H, (uint64_t)d.I / 2, 128);
   if (err != cudaSuccess) return cuda_status(err);
   err = launch_make_maps(pa, tmpl_gu, tmpl_dn, s);

@@ -62,10 +62,10 @@ inline size_t matrix_bytes(int N, int K) {
 inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matrix_bytes(H, I); }
 
 // Byte offsets of the workspace segments for batches of up to T tokens.  The
-// prefill segments (xg, hs, y, ux, maps) are sized only when `prefill` is set.
+// prefill segments (xg, hs, y, maps) are sized only when `prefill` is set.
 struct WsLayout {
   size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
-      pair_tok, hq, hqs, hd, xg, hs, y, ux, maps, total;
+      pair_tok, hq, hqs, hd, xg, hs, y, maps, total;
 };
 
 inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
@@ -100,7 +100,6 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
   L.xg = seg(Pp * d.H * 4);  // fp16 hi/lo split of x^, [P][2H]
   L.hs = seg(Pp * d.I * 4);  // fp16 hi/lo split of h^, [P][2I]
   L.y = seg(Pp * d.H * 4);
-  L.ux = seg(prefill ? (size_t)kPfMaxCtas * 64 * 128 * 4 : 0);
   L.maps = seg(prefill ? (size_t)(d.E + 1) * 3 * 128 : 0);
   L.total = o;
   return L;
@@ -181,7 +180,6 @@ struct PfArgs {
   float *hd;            //   their block scales [P][I/32],
   void *hs;             //   and the fp16 hi/lo split of h^ = q d [P][2I] (mode 1's B rows)
   float *y;             // mode 1 output [P][H]
-  float *ux;            // mode 0 up-row exchange, [CTA][64][128] fp32
   const CUtensorMap *maps;  // [E+1][gate, up, down] tensor maps of the packed weights (device)
   int32_t *status;
   unsigned long long *prof;  // profiling record or null (phase mode + 1; k_make_maps ends phase 0)

@@ -13,13 +13,14 @@
 //                    mode 1 = down into per-pair rows y.
 //   k_combine      : out = y_shared + sum_s w_s * y_s, slot order.
 //
-// The GEMM tile is 128 weight rows (MMA M; for gate/up 64 gate rows and the 64
-// up rows of the same intermediate rows) by up to 128 token rows of one expert
-// (MMA N, a multiple of 16), so an expert with few tokens wastes at most 15
-// columns.  K advances one 64-group per pipeline stage.
+// The GEMM tile is two blocks of 128 weight rows (MMA M = 128 each; for
+// gate/up the gate and the up rows of the same 128 intermediate rows) by up to
+// 64 token rows of one expert (MMA N, a multiple of 16), so an expert with few
+// tokens wastes at most 15 columns.  K advances one 64-group per pipeline
+// stage.
 //
 // Operands.  The int4 weights (-8..7) are exact in fp16; the expansion warps
-// turn nibbles into fp16 in shared memory (bytes 0x64 0x0u form the half
+// turn nibbles into fp16 in tensor memory (bytes 0x64 0x0u form the half
 // 1024 + u, one packed fp16 subtraction of 1032 gives u - 8).  The activations
 // enter as the dequantised Q8_0 values x^ = q d split into two fp16 numbers,
 // hi = fp16(x^) and lo = fp16(x^ - hi), together 22 significant bits.  Per
@@ -85,6 +86,11 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
         "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
       : "r"(taddr));
 }
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory operand descriptor, K-major without swizzle: core matrices of
@@ -147,49 +153,64 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
 // grouped GEMM
 //
 // One CTA per SM, persistent over its tiles (blockIdx.x, + gridDim.x, ...);
-// a tile is G pipeline stages, one 64-group of K each.  14 warps:
-//   0-7   epilogue: TMEM lane quarter warp & 3, columns 64 * (warp >> 2) ..;
-//         per stage acc += s_g * C_g, a tile's outputs after its last group;
-//   8-11  expansion: packed nibbles of stage i -> fp16 A buffer i % kPfNA
-//         (thread = A row);
-//   12    copies (lane 0): TMA of the packed weights (tensor maps built per
-//         expert on the device) and of the activation hi/lo rows;
-//   13    MMAs (lane 0): 8 per stage, hi then lo of each K16 slice, into TMEM
-//         buffer i % kPfNT.
-// Every hand-off is an mbarrier; every wait is bounded.
+// a tile is G pipeline stages, one 64-group of K each.  A tile is two blocks
+// of 128 weight rows (gate/up: the gate rows and the up rows of the same 128
+// intermediate rows; down: 256 consecutive output rows) against up to 64
+// token rows of one expert.  23 warps (80 registers per thread, so that
+// nothing spills: with shared memory nearly full, L1 has little room for
+// local memory):
+//   0-15  epilogue: TMEM lane quarter warp & 3, columns 16 * (warp >> 2) ..
+//         of both blocks; per stage acc += s_g * C_g, after a tile's last
+//         group its outputs (gate/up: SwiGLU and Q8_0 of h in the thread that
+//         holds g and u);
+//   16-19 expansion: packed nibbles of stage i -> fp16 A operands in tensor
+//         memory (thread = weight row = TMEM lane, both blocks);
+//   20    weight copies (lane 0): TMA of the packed weights (tensor maps built
+//         per expert on the device), as far ahead as the ring allows;
+//   21    activation copies (lane 0): TMA of the hi/lo token rows;
+//   22    MMAs (lane 0): per block and K16 slice hi then lo, A from tensor
+//         memory, B from shared memory.
+// Shared memory then carries only the activation rows and the packed weights,
+// which keeps its bandwidth below the tensor cores' need.  Every hand-off is
+// an mbarrier; every wait is bounded.
 // ===========================================================================
-constexpr int kPfEpiWarps = 8;
-constexpr int kPfExpWarp0 = 8;               // expansion warps 8..11
-constexpr int kPfTmaWarp = 12;
-constexpr int kPfMmaWarp = 13;
-constexpr int kPfThreads = 14 * 32;
-constexpr int kPfNA = 3;                     // expanded-weight buffers
-constexpr int kPfNT = 4;                     // TMEM accumulator buffers (128 columns each)
-constexpr int kPfRB = 4;                     // activation ring slots
-constexpr int kPfRR = 8;                     // packed-weight ring slots
+constexpr int kPfEpiWarps = 16;              // epilogue warps 0..15
+constexpr int kPfExpWarp0 = 16;              // expansion warps 16..19
+constexpr int kPfRawWarp = 20;
+constexpr int kPfActWarp = 21;
+constexpr int kPfMmaWarp = 22;
+constexpr int kPfThreads = 23 * 32;
+constexpr int kPfTileN = 64;                 // token rows per tile (MMA N <= 64)
+constexpr int kPfNA = 2;                     // A operand buffers (tensor memory, 64 columns each)
+constexpr int kPfNT = 3;                     // accumulator buffers (tensor memory, 128 columns each)
+constexpr int kPfRB = 6;                     // activation ring slots
+constexpr int kPfRR = 7;                     // packed-weight ring slots
 constexpr uint32_t kPfTmemCols = 512;
+constexpr uint32_t kPfAccCols = 128;         // per buffer: block 0 at +0, block 1 at +64
+constexpr uint32_t kPfACol0 = kPfNT * kPfAccCols;  // A buffers from column 384: block b, slice k at +32 b + 8 k
 
-constexpr uint32_t kABytes = 16384;   // 4 K16 slices x [128 rows x 32 B] fp16 weights, no swizzle
-constexpr uint32_t kBHalf = 16384;    // [128 rows][128 B] fp16, 128-byte swizzle (hi or lo)
+constexpr uint32_t kBHalf = 8192;     // [64 rows][128 B] fp16, 128-byte swizzle (hi or lo)
 constexpr uint32_t kBBytes = 2 * kBHalf;
-constexpr uint32_t kRawBytes = 4096;  // [128 rows][32 B] packed weights of a group
+constexpr uint32_t kRawBlk = 4096;    // [128 rows][32 B] packed weights of a group, one block
+constexpr uint32_t kRawBytes = 2 * kRawBlk;
 
 struct PfLayout {
-  uint32_t tile_pre, a, b, raw, total;
+  uint32_t tile_pre, b, raw, hst, total;
 };
 __host__ __device__ inline PfLayout pf_layout(int E) {
   PfLayout L;
   L.tile_pre = 1024;
-  L.a = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
-  L.b = L.a + (uint32_t)kPfNA * kABytes;
+  L.b = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
   L.raw = L.b + (uint32_t)kPfRB * kBBytes;
-  L.total = L.raw + (uint32_t)kPfRR * kRawBytes;
+  L.hst = L.raw + (uint32_t)kPfRR * kRawBytes;
+  L.total = L.hst + (uint32_t)kPfEpiWarps * 32 * 32 * 4;  // g, u staging: [32][512 epilogue threads]
   return L;
 }
 
 struct PfTile {
   int e;     // table index (E = the shared expert)
   int wt;    // weight tile
+  int nblk;  // 128-row weight blocks in the tile (down: 1 for the last tile when H % 256 = 128)
   int p0;    // first pair position of the token tile
   int nval;  // valid token rows
   int n;     // MMA N (nval rounded up to 16)
@@ -199,6 +220,7 @@ struct PfTile {
 // (positions T*k ..), slot u >= 1 the union's expert uni[u-1]; inside a slot the
 // token tile runs fastest, so CTAs working on neighbouring tiles read the same
 // weight rows (one HBM read, the rest from L2).
+template <int MODE>
 __device__ __forceinline__ PfTile pf_tile(int t, const int *tile_pre, int nslot, const PfArgs &a) {
   int lo = 0, hi = nslot - 1;
   while (lo < hi) {
@@ -216,17 +238,19 @@ __device__ __forceinline__ PfTile pf_tile(int t, const int *tile_pre, int nslot,
     p0 = a.off[r.e];
     n = a.off[r.e + 1] - p0;
   }
-  const int ntt = (n + 127) >> 7;
+  const int ntt = (n + kPfTileN - 1) / kPfTileN;
   const int q = t - tile_pre[lo];
   r.wt = q / ntt;
   const int tt = q - r.wt * ntt;
-  r.p0 = p0 + tt * 128;
-  r.nval = min(128, n - tt * 128);
+  r.nblk = (MODE == 1 && 256 * r.wt + 128 >= a.H) ? 1 : 2;
+  r.p0 = p0 + tt * kPfTileN;
+  r.nval = min(kPfTileN, n - tt * kPfTileN);
   r.n = (r.nval + 15) & ~15;
   return r;
 }
 
 // A position in the CTA's stage sequence.
+template <int MODE>
 struct PfCur {
   int t, g;
   PfTile tl;
@@ -241,31 +265,48 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, det));
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 x fp16 -> fp32, issued by one thread.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// 16 consecutive TMEM columns of this warp's 32 lanes from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+      "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 template <int MODE>
-__global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
+__global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I;
   const int K = MODE == 0 ? H : I;
   const int G = K / 64;
-  const int NWT = MODE == 0 ? I / 64 : H / 128;
+  const int NWT = MODE == 0 ? I / 128 : (H + 255) / 256;
   const PfLayout L = pf_layout(a.E);
   uint64_t *rawfull = reinterpret_cast<uint64_t *>(smem);  // [RR] packed weights landed (TMA bytes)
   uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (4 expansion warps)
   uint64_t *bfull = rawfree + kPfRR;                        // [RB] activation rows landed (TMA bytes)
   uint64_t *bfree = bfull + kPfRB;                          // [RB] read by the MMAs (commit)
-  uint64_t *aready = bfree + kPfRB;                         // [NA] A buffer written (4 expansion warps)
-  uint64_t *afree = aready + kPfNA;                         // [NA] A buffer read by the MMAs (commit)
+  uint64_t *aready = bfree + kPfRB;                         // [NA] A operands written (4 expansion warps)
+  uint64_t *afree = aready + kPfNA;                         // [NA] A operands read by the MMAs (commit)
   uint64_t *accf = afree + kPfNA;                           // [NT] accumulators written (commit)
   uint64_t *tfree = accf + kPfNT;                           // [NT] accumulators read (8 epilogue warps)
-  uint64_t *uxw = tfree + kPfNT;                            // up rows handed over (4 warps)
-  uint64_t *uxr = uxw + 1;                                  // up rows consumed (4 warps)
-  uint64_t *drain = uxr + 1;                                // teardown
+  uint64_t *drain = tfree + kPfNT;                          // teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
   int *s_ntiles = reinterpret_cast<int *>(smem + 520);
   int *tile_pre = reinterpret_cast<int *>(smem + L.tile_pre);
-  unsigned char *abuf = smem + L.a;
   unsigned char *bbuf = smem + L.b;
   unsigned char *raw = smem + L.raw;
 
@@ -292,8 +333,6 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
       mbar_init(accf + s, 1);
       mbar_init(tfree + s, kPfEpiWarps);
     }
-    mbar_init(uxw, 4);
-    mbar_init(uxr, 4);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -311,7 +350,7 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
           const int e = a.uni[s - 1];
           n = a.off[e + 1] - a.off[e];
         }
-        nt = ((max(n, 0) + 127) >> 7) * NWT;
+        nt = ((max(n, 0) + kPfTileN - 1) / kPfTileN) * NWT;
       }
       int incl = nt;
 #pragma unroll
@@ -337,30 +376,28 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
   const int my_tiles = blockIdx.x < (unsigned)n_tiles ? (n_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int S = my_tiles * G;  // stages of this CTA
 
-  auto cur_begin = [&](PfCur &c) {
+  auto cur_begin = [&](PfCur<MODE> &c) {
     c.t = blockIdx.x;
     c.g = 0;
-    if (c.t < n_tiles) c.tl = pf_tile(c.t, tile_pre, nslot, a);
+    if (c.t < n_tiles) c.tl = pf_tile<MODE>(c.t, tile_pre, nslot, a);
   };
-  auto cur_next = [&](PfCur &c) {
+  auto cur_next = [&](PfCur<MODE> &c) {
     if (++c.g == G) {
       c.g = 0;
       c.t += gridDim.x;
-      if (c.t < n_tiles) c.tl = pf_tile(c.t, tile_pre, nslot, a);
+      if (c.t < n_tiles) c.tl = pf_tile<MODE>(c.t, tile_pre, nslot, a);
     }
   };
 
-  if (warp == kPfTmaWarp) {
-    // ================================================================ copies
+  if (warp == kPfRawWarp) {
+    // ======================================================= weight copies
     if (lane == 0) {
       bool bad = false;
-      PfCur cr;
+      PfCur<MODE> cr;
       cur_begin(cr);
       int rtile = -1, issued = 0;
       const CUtensorMap *m0 = nullptr, *m1 = nullptr;
-      asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
       for (int j = 0; j < S && !bad; ++j, cur_next(cr)) {
-        // packed weights of stage j
         const int s = j % kPfRR;
         if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty)) {
           bad = true;
@@ -370,41 +407,57 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
           rtile = cr.t;
           const CUtensorMap *em = a.maps + (size_t)cr.tl.e * 3;
           m0 = MODE == 0 ? em : em + 2;
-          m1 = em + 1;
+          m1 = MODE == 0 ? em + 1 : em + 2;
           tmap_acquire(m0);
           if (MODE == 0) tmap_acquire(m1);
         }
         unsigned char *dst = raw + (size_t)s * kRawBytes;
-        mbar_arrive_expect_tx(rawfull + s, kRawBytes);
+        const int nb = cr.tl.nblk;
+        mbar_arrive_expect_tx(rawfull + s, (uint32_t)nb * kRawBlk);
         if (MODE == 0) {
-          tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 64, rawfull + s);
-          tma_load_2d(dst + 64 * 32, m1, cr.g * 32, cr.tl.wt * 64, rawfull + s);
-        } else {
           tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 128, rawfull + s);
+          tma_load_2d(dst + kRawBlk, m1, cr.g * 32, cr.tl.wt * 128, rawfull + s);
+        } else {
+          tma_load_2d(dst, m0, cr.g * 32, cr.tl.wt * 256, rawfull + s);
+          if (nb == 2) tma_load_2d(dst + kRawBlk, m1, cr.g * 32, cr.tl.wt * 256 + 128, rawfull + s);
         }
-        // activation hi/lo rows of stage j: boxes of kPfBoxRows rows; rows past
-        // the tile's own land in unused B rows, rows past the array read zero
+        issued = j + 1;
+        if (*abort_flag) bad = true;
+      }
+      if (bad) *abort_flag = 1;
+      // teardown: copies issued but not yet landed
+      for (int j = max(0, issued - kPfRR); j < issued; ++j)
+        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
+    }
+    __syncwarp();
+  } else if (warp == kPfActWarp) {
+    // =================================================== activation copies
+    if (lane == 0) {
+      bool bad = false;
+      PfCur<MODE> cb;
+      cur_begin(cb);
+      int issued = 0;
+      asm volatile("prefetch.tensormap [%0];" ::"l"(&bmap) : "memory");
+      for (int j = 0; j < S && !bad; ++j, cur_next(cb)) {
+        // hi/lo rows of stage j: boxes of kPfBoxRows rows; rows past the
+        // tile's own land in unused B rows, rows past the array read zero
         const int sb = j % kPfRB;
         if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) {
           bad = true;
           break;
         }
         unsigned char *db = bbuf + (size_t)sb * kBBytes;
-        const int nbox = (cr.tl.n + (int)kPfBoxRows - 1) / (int)kPfBoxRows;
+        const int nbox = (cb.tl.n + (int)kPfBoxRows - 1) / (int)kPfBoxRows;
         mbar_arrive_expect_tx(bfull + sb, (uint32_t)nbox * kPfBoxRows * 256u);
         for (int i = 0; i < nbox; ++i) {
-          const int y = cr.tl.p0 + i * (int)kPfBoxRows;
-          tma_load_2d(db + i * (int)kPfBoxRows * 128, &bmap, cr.g * 128, y, bfull + sb);
-          tma_load_2d(db + kBHalf + i * (int)kPfBoxRows * 128, &bmap, cr.g * 128 + 64, y, bfull + sb);
+          const int y = cb.tl.p0 + i * (int)kPfBoxRows;
+          tma_load_2d(db + i * (int)kPfBoxRows * 128, &bmap, cb.g * 128, y, bfull + sb);
+          tma_load_2d(db + kBHalf + i * (int)kPfBoxRows * 128, &bmap, cb.g * 128 + 64, y, bfull + sb);
         }
         issued = j + 1;
         if (*abort_flag) bad = true;
       }
       if (bad) *abort_flag = 1;
-      // teardown: copies issued but not yet landed (only after a failure can
-      // some never have been waited for)
-      for (int j = max(0, issued - kPfRR); j < issued; ++j)
-        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
       for (int j = max(0, issued - kPfRB); j < issued; ++j)
         mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
     }
@@ -413,10 +466,9 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
     // ================================================================ MMAs
     if (lane == 0) {
       bool bad = false;
-      PfCur cm;
+      PfCur<MODE> cm;
       cur_begin(cm);
       // descriptors advance by (byte offset >> 4) in their start-address field
-      const uint64_t a0 = umma_desc(smem_u32(abuf));
       const uint64_t b0 = umma_desc_sw128(smem_u32(bbuf));
       int done = 0;
       for (int j = 0; j < S && !bad; ++j, cur_next(cm)) {
@@ -430,14 +482,15 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
         }
         tc_fence_after();
         const uint32_t idesc = pf_idesc(cm.tl.n);
-        const uint32_t d = tmem + (uint32_t)(tb * 128);
-        const uint64_t ad = a0 + (uint64_t)((na * kABytes) >> 4);
         const uint64_t bd = b0 + (uint64_t)((sb * kBBytes) >> 4);
+        for (int blk = 0; blk < cm.tl.nblk; ++blk) {
+          const uint32_t d = tmem + (uint32_t)(tb * kPfAccCols + 64 * blk);
+          const uint32_t at = tmem + kPfACol0 + (uint32_t)(na * 64 + 32 * blk);
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          const uint64_t ak = ad + (uint64_t)((k4 * 4096) >> 4);
-          umma_f16(d, ak, bd + (uint64_t)((k4 * 32) >> 4), idesc, (uint32_t)(k4 > 0));
-          umma_f16(d, ak, bd + (uint64_t)((kBHalf + k4 * 32) >> 4), idesc, 1u);
+          for (int k4 = 0; k4 < 4; ++k4) {
+            umma_f16_ts(d, at + 8 * k4, bd + (uint64_t)((k4 * 32) >> 4), idesc, (uint32_t)(k4 > 0));
+            umma_f16_ts(d, at + 8 * k4, bd + (uint64_t)((kBHalf + k4 * 32) >> 4), idesc, 1u);
+          }
         }
         umma_commit(accf + tb);
         umma_commit(bfree + sb);
@@ -454,33 +507,41 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
   } else if (warp >= kPfExpWarp0) {
     // ================================================================ expansion
     bool bad = false;
-    const int r = tid - kPfExpWarp0 * 32;  // A row
-    for (int i = 0; i < S && !bad; ++i) {
+    const int q = warp - kPfExpWarp0;   // TMEM lane quarter
+    const int r = q * 32 + lane;        // weight row of both blocks = TMEM lane
+    const uint32_t tl_a = tmem + ((uint32_t)(q * 32) << 16) + kPfACol0;
+    PfCur<MODE> cx;
+    cur_begin(cx);
+    for (int i = 0; i < S && !bad; ++i, cur_next(cx)) {
       const int ra = i % kPfRR, na = i % kPfNA;
       if (!warp_wait(rawfull + ra, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull) ||
           (i >= kPfNA && !warp_wait(afree + na, (uint32_t)(i / kPfNA - 1) & 1u, a.status, kDetPfFull))) {
         bad = true;
         break;
       }
-      const uint4 *src = reinterpret_cast<const uint4 *>(raw + (size_t)ra * kRawBytes + r * 32);
-      const uint4 s0 = src[0], s1 = src[1];
-      unsigned char *ab = abuf + (size_t)na * kABytes;
-      // byte j: low nibble = element j, high nibble = element j + 32; slice k4
-      // = elements 16 k4 .. 16 k4 + 15
+      tc_fence_after();
+      for (int blk = 0; blk < cx.tl.nblk; ++blk) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(raw + (size_t)ra * kRawBytes + blk * kRawBlk + r * 32);
+        const uint4 s0 = src[0], s1 = src[1];
+        // byte j: low nibble = element j, high nibble = element j + 32; column
+        // 8 k + c of the block holds elements 16 k + 2 c (low half), + 1
 #pragma unroll
-      for (int k4 = 0; k4 < 4; ++k4) {
-        const uint4 v = (k4 & 1) ? s1 : s0;
-        const int sh = (k4 >> 1) * 4;
-        uint32_t h[8];
-        nib4_to_f16((v.x >> sh) & 0x0F0F0F0Fu, h[0], h[1]);
-        nib4_to_f16((v.y >> sh) & 0x0F0F0F0Fu, h[2], h[3]);
-        nib4_to_f16((v.z >> sh) & 0x0F0F0F0Fu, h[4], h[5]);
-        nib4_to_f16((v.w >> sh) & 0x0F0F0F0Fu, h[6], h[7]);
-        unsigned char *dst = ab + k4 * 4096;
-        *reinterpret_cast<uint4 *>(dst + il_off(r, 0)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4 *>(dst + il_off(r, 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+        for (int hk = 0; hk < 2; ++hk) {  // K16 slices 2 hk, 2 hk + 1: the low / high nibbles
+          uint32_t v[16];
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const uint4 w = k2 ? s1 : s0;
+            const int sh = hk * 4;
+            nib4_to_f16((w.x >> sh) & 0x0F0F0F0Fu, v[8 * k2 + 0], v[8 * k2 + 1]);
+            nib4_to_f16((w.y >> sh) & 0x0F0F0F0Fu, v[8 * k2 + 2], v[8 * k2 + 3]);
+            nib4_to_f16((w.z >> sh) & 0x0F0F0F0Fu, v[8 * k2 + 4], v[8 * k2 + 5]);
+            nib4_to_f16((w.w >> sh) & 0x0F0F0F0Fu, v[8 * k2 + 6], v[8 * k2 + 7]);
+          }
+          tmem_st16(tl_a + (uint32_t)(na * 64 + 32 * blk + 16 * hk), v);
+        }
       }
-      fence_proxy_async();
+      tmem_st_wait();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(aready + na);
@@ -493,135 +554,125 @@ __global__ void __maxnreg__(128) k_gemm_pf(const PfArgs a, const __grid_constant
     // ================================================================ epilogue
     bool bad = false;
     const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
-    const int q = warp & 3, half = warp >> 2;  // TMEM lane quarter, 64-column half
+    const int q = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 16-column quarter
     const int row = q * 32 + lane;
-    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * 64);
-    // weight scales of this thread's row: 4 bytes (groups g, g+1) per stage
-    // pair, loaded one pair ahead
-    auto scale_row = [&](const PfTile &tl) -> const uint32_t * {
+    const int col0 = cq * 16;
+    const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
+    // weight scales of this thread's rows of both blocks: 4 bytes (groups g,
+    // g+1) each per stage pair, loaded one pair ahead
+    auto scale_at = [&](const PfTile &tl, int blk, int g) -> uint32_t {
       const unsigned char *blob = static_cast<const unsigned char *>(a.table[tl.e]);
+      const unsigned char *p;
       if (MODE == 0) {
-        const size_t base = row < 64 ? 0 : mg;
-        const size_t rr = (size_t)tl.wt * 64 + (row & 63);
-        return reinterpret_cast<const uint32_t *>(blob + base + (size_t)I * (size_t)(H / 2) + rr * (size_t)(H / 64) * 2);
+        const size_t rr = (size_t)tl.wt * 128 + row;
+        p = blob + (size_t)blk * mg + (size_t)I * (size_t)(H / 2) + rr * (size_t)(H / 64) * 2;
+      } else {
+        const size_t rr = (size_t)tl.wt * 256 + (size_t)blk * 128 + row;
+        p = blob + 2 * mg + (size_t)H * (size_t)(I / 2) + rr * (size_t)(I / 64) * 2;
       }
-      const size_t rr = (size_t)tl.wt * 128 + row;
-      return reinterpret_cast<const uint32_t *>(blob + 2 * mg + (size_t)H * (size_t)(I / 2) + rr * (size_t)(I / 64) * 2);
+      return __ldg(reinterpret_cast<const uint32_t *>(p) + (g >> 1));
     };
-    PfCur cw;  // scale prefetch cursor, one stage pair ahead
-    cur_begin(cw);
-    uint32_t w_next = 0, w_cur = 0;
-    if (S > 0) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
-    PfCur ce;
+    PfCur<MODE> ce;
     cur_begin(ce);
-    float acc[64];
+    uint32_t w0n = 0, w1n = 0;  // scales of the next stage pair
+    if (S > 0) {
+      w0n = scale_at(ce.tl, 0, 0);
+      if (ce.tl.nblk == 2) w1n = scale_at(ce.tl, 1, 0);
+    }
+    uint32_t w0c = 0, w1c = 0;
+    float acc0[16], acc1[16];
 #pragma unroll
-    for (int i = 0; i < 64; ++i) acc[i] = 0.0f;
-    int tcount = 0;
-    float *ux = a.ux + (size_t)blockIdx.x * 64 * 128;  // this CTA's up-row exchange [64 rows][128 cols]
+    for (int i = 0; i < 16; ++i) acc0[i] = acc1[i] = 0.0f;
 
     for (int j = 0; j < S && !bad; ++j) {
       const int tb = j % kPfNT;
-      if ((j & 1) == 0) {
-        w_cur = w_next;
-        cur_next(cw);
-        cur_next(cw);
-        if (cw.t < n_tiles) w_next = __ldg(scale_row(cw.tl) + (cw.g >> 1));
+      if ((ce.g & 1) == 0) {
+        w0c = w0n;
+        w1c = w1n;
+        // the pair after this one: in this tile, or the first of the next
+        if (ce.g + 2 < G) {
+          w0n = scale_at(ce.tl, 0, ce.g + 2);
+          if (ce.tl.nblk == 2) w1n = scale_at(ce.tl, 1, ce.g + 2);
+        } else if (ce.t + (int)gridDim.x < n_tiles) {
+          const PfTile nt = pf_tile<MODE>(ce.t + (int)gridDim.x, tile_pre, nslot, a);
+          w0n = scale_at(nt, 0, 0);
+          if (nt.nblk == 2) w1n = scale_at(nt, 1, 0);
+        }
       }
       if (!warp_wait(accf + tb, (uint32_t)(j / kPfNT) & 1u, a.status, kDetPfAccFull)) {
         bad = true;
         break;
       }
       tc_fence_after();
-      const int nch = ce.tl.n >> 4;  // 16-column chunks of the tile
-      const float sg = __half2float(__ushort_as_half((unsigned short)((ce.g & 1) ? (w_cur >> 16) : (w_cur & 0xFFFFu))));
+      if (col0 < ce.tl.n) {
+        const int sh = (ce.g & 1) * 16;
+        const float s0 = __half2float(__ushort_as_half((unsigned short)(w0c >> sh)));
+        const float s1 = __half2float(__ushort_as_half((unsigned short)(w1c >> sh)));
+        uint32_t v[16];
+        tmem_ld16(tq + (uint32_t)(tb * kPfAccCols), v);
+        tmem_ld_wait();
 #pragma unroll
-      for (int c2 = 0; c2 < 2; ++c2) {
-        const int c = half * 4 + c2 * 2;  // chunks c, c + 1
-        if (c < nch) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(tq + (uint32_t)(tb * 128 + c2 * 32), v0);
-          tmem_ld16(tq + (uint32_t)(tb * 128 + c2 * 32 + 16), v1);
-          tmem_ld_wait();
+        for (int k = 0; k < 16; ++k) acc0[k] = ffma(s0, __uint_as_float(v[k]), acc0[k]);
+        tmem_ld16(tq + (uint32_t)(tb * kPfAccCols + 64), v);
+        tmem_ld_wait();
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            acc[c2 * 32 + k] = ffma(sg, __uint_as_float(v0[k]), acc[c2 * 32 + k]);
-            acc[c2 * 32 + 16 + k] = ffma(sg, __uint_as_float(v1[k]), acc[c2 * 32 + 16 + k]);
-          }
-        }
+        for (int k = 0; k < 16; ++k) acc1[k] = ffma(s1, __uint_as_float(v[k]), acc1[k]);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tfree + tb);
-      if (ce.g == G - 1) {
-        // the tile's outputs; this thread holds columns 64 half + 0..63
+      if (ce.g == G - 1 && col0 < ce.tl.nval) {
+        // the tile's outputs; this thread holds columns col0 .. col0 + 15 of both blocks
         const PfTile tl = ce.tl;
-        const int col0 = half * 64;
+        const int ncol = min(16, tl.nval - col0);
         if (MODE == 1) {
-          float *yc = a.y + (size_t)tl.p0 * H + (size_t)tl.wt * 128 + row;
+          float *yc = a.y + (size_t)(tl.p0 + col0) * H + (size_t)tl.wt * 256 + row;
 #pragma unroll
-          for (int k = 0; k < 64; ++k)
-            if (col0 + k < tl.nval) yc[(size_t)(col0 + k) * H] = acc[k];
-        } else {
-          // Rows 64..127 hold u of rows 0..63 (g): hand u over through this
-          // CTA's exchange rows in global memory, then SwiGLU and Q8_0 of h
-          // along I (one 32-block = one warp's lanes), per token.
-          if (q >= 2) {
-            if (tcount > 0 && !warp_wait(uxr, (uint32_t)(tcount - 1) & 1u, a.status, kDetPfFull)) {
-              bad = true;
-              break;
+          for (int k = 0; k < 16; ++k) {
+            if (k < ncol) {
+              yc[(size_t)k * H] = acc0[k];
+              if (tl.nblk == 2) yc[(size_t)k * H + 128] = acc1[k];
             }
-            float *uw = ux + (size_t)(row - 64) * 128 + col0;
-#pragma unroll
-            for (int k = 0; k < 64; k += 4)
-              if (col0 + k < tl.n) *reinterpret_cast<float4 *>(uw + k) = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(uxw);
-          } else {
-            if (!warp_wait(uxw, (uint32_t)tcount & 1u, a.status, kDetPfFull)) {
-              bad = true;
-              break;
-            }
-            const int ii = tl.wt * 64 + row;  // row of I
-            const float *ur = ux + (size_t)row * 128 + col0;
-            __half *hs = static_cast<__half *>(a.hs);
-            const size_t hcol = (size_t)(ii >> 6) * 128 + (ii & 63);
-#pragma unroll
-            for (int k = 0; k < 64; k += 4) {
-              if (col0 + k < tl.n) {
-                const float4 u4 = *reinterpret_cast<const float4 *>(ur + k);
-                const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
-#pragma unroll
-                for (int m = 0; m < 4; ++m) {
-                  // h = SiLU(g) * u and its Q8_0 codes in fast fp32 (this path is
-                  // held to the layer's tolerance, not to the fixed-order bits)
-                  const float gv = acc[k + m];
-                  const float h = __fdividef(gv, 1.0f + __expf(-gv)) * uv[m];
-                  const float amax = warp_max(fabsf(h));
-                  const float d = amax * (1.0f / 127.0f);
-                  const float inv = amax > 0.0f ? __fdividef(127.0f, amax) : 0.0f;
-                  const int qv = (int)fminf(fmaxf(rintf(h * inv), -127.0f), 127.0f);
-                  const int col = col0 + k + m;
-                  if (col < tl.nval) {
-                    const size_t p = (size_t)(tl.p0 + col);
-                    a.hq[p * I + ii] = (int8_t)qv;
-                    if (lane == 0) a.hd[p * (I / 32) + ii / 32] = d;
-                    const float hv = (float)qv * d;  // dequantised h, split hi + lo
-                    const __half hi = __float2half_rn(hv);
-                    const __half lo = __float2half_rn(hv - __half2float(hi));
-                    hs[p * (size_t)(2 * I) + hcol] = hi;
-                    hs[p * (size_t)(2 * I) + hcol + 64] = lo;
-                  }
-                }
-              }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(uxr);
           }
-          ++tcount;
-        }
+        } else {
+          // h = SiLU(g) * u, its Q8_0 codes along I (one 32-block of I = one
+          // warp's lanes) and the hi/lo split of the dequantised h for the down
+          // GEMM, in fast fp32 (this path is held to the layer's tolerance, not
+          // to the fixed-order bits).  g and u go through shared memory (own
+          // values only) so that the per-column loop stays rolled.
+          float *hst = reinterpret_cast<float *>(smem + L.hst) + tid;
 #pragma unroll
-        for (int k = 0; k < 64; ++k) acc[k] = 0.0f;
+          for (int k = 0; k < 16; ++k) {
+            hst[k * kPfEpiWarps * 32] = acc0[k];
+            hst[(16 + k) * kPfEpiWarps * 32] = acc1[k];
+          }
+          const int ii = tl.wt * 128 + row;  // row of I
+          __half *hs = static_cast<__half *>(a.hs);
+          const size_t hcol = (size_t)(ii >> 6) * 128 + (ii & 63);
+#pragma unroll 1
+          for (int k = 0; k < 16; ++k) {
+            const float gv = hst[k * kPfEpiWarps * 32];
+            const float h = __fdividef(gv, 1.0f + __expf(-gv)) * hst[(16 + k) * kPfEpiWarps * 32];
+            const float amax = warp_max(fabsf(h));
+            const float d = amax * (1.0f / 127.0f);
+            const float inv = amax > 0.0f ? __fdividef(127.0f, amax) : 0.0f;
+            const int qv = (int)fminf(fmaxf(rintf(h * inv), -127.0f), 127.0f);
+            if (k < ncol) {
+              const size_t p = (size_t)(tl.p0 + col0 + k);
+              a.hq[p * I + ii] = (int8_t)qv;
+              if (lane == 0) a.hd[p * (I / 32) + ii / 32] = d;
+              const float hv = (float)qv * d;
+              const __half hi = __float2half_rn(hv);
+              const __half lo = __float2half_rn(hv - __half2float(hi));
+              hs[p * (size_t)(2 * I) + hcol] = hi;
+              hs[p * (size_t)(2 * I) + hcol + 64] = lo;
+            }
+          }
+        }
+      }
+      if (ce.g == G - 1) {
+#pragma unroll
+        for (int k = 0; k < 16; ++k) acc0[k] = acc1[k] = 0.0f;
       }
       cur_next(ce);
       if (*abort_flag) bad = true;
