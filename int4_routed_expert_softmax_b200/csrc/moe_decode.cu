@@ -225,17 +225,18 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     }
   }
 
-  // activations: xq in per-lane chunks (padded rows), block scales, code sums
-  {
+  // activations (consumer warps only; the producer starts streaming weights
+  // at once): xq in per-lane chunks (padded rows), block scales, code sums
+  if (warp != 8) {
     const int pieces = CSZ * 4;
-    for (int i = tid; i < T * 32 * pieces; i += blockDim.x) {
+    for (int i = tid; i < T * 32 * pieces; i += 256) {
       const int t = i / (32 * pieces), r = i % (32 * pieces), c = r / pieces, j = r % pieces;
       const int col = c * CSZ * 64 + 16 * j;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (col < H) v = *reinterpret_cast<const uint4 *>(a.xq + (size_t)t * H + col);
       *reinterpret_cast<uint4 *>(xq_s + (size_t)(t * 32 + c) * pl.chp + 16 * j) = v;
     }
-    for (int i = tid; i < T * HB; i += blockDim.x) {
+    for (int i = tid; i < T * HB; i += 256) {
       xd_s[i] = a.xd[i];
       const uint4 *q4 = reinterpret_cast<const uint4 *>(a.xq + (size_t)i * 32);
       int s = 0;
@@ -249,8 +250,8 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
       qs_s[i] = s;
     }
+    named_sync(1, 256);
   }
-  __syncthreads();
 
   if (warp == 8) {
     // -------------------------------------------------------------- producer
