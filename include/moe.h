@@ -164,9 +164,14 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
                       int32_t *route_counts_opt, int32_t path, void *stream);
 
 /* Same as moe_layer_forward with x_host [T][H] and out_host [T][H] in HOST
- * memory (pinned for overlap; pageable works but serialises).  The copies in
- * and out are enqueued on `stream` around the layer; the call returns after
- * enqueueing (synchronise the stream before reading out_host). */
+ * memory.  Pinned memory the device can address (cudaHostAlloc /
+ * cudaMallocHost, or registered and mapped) moves without separate copies: a
+ * staging kernel reads x across the link into the workspace while it zeroes
+ * the control words, and on the decode path the down kernel stores out
+ * straight into out_host.  Other memory (pageable) goes through
+ * cudaMemcpyAsync before and after the layer; so does out on the prefill path.
+ * Everything is enqueued on `stream`; the call returns after enqueueing
+ * (synchronise the stream before reading out_host). */
 int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
                            const float *Wr, const void *const *expert_table, float *out_host,
                            void *ws, size_t ws_bytes, int32_t *route_counts_opt, int32_t path,

@@ -305,6 +305,18 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   return MOE_OK;
 }
 
+// The device address of pinned host memory the current device can use, or
+// null (pageable or unknown memory, or no mapping).
+const void *host_device_view(const void *p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+    return nullptr;
+  }
+  if (at.type != cudaMemoryTypeHost || at.devicePointer == nullptr) return nullptr;
+  return at.devicePointer;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -490,6 +502,30 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
   return cuda_status(launch_bucket(a, static_cast<cudaStream_t>(stream)));
 }
 
+// The layer after argument checks; `zeroed`: the caller has already zeroed the
+// status word and the router's arrival counter for this call.
+static int forward_checked(const moe_dims &d, int32_t T, const float *x, const float *Wr, const void *const *expert_table,
+                    float *out, void *ws, int32_t *route_counts_opt, bool pf, const WsLayout &L, bool zeroed,
+                    cudaStream_t s) {
+  int rc = MOE_OK;
+  if (!zeroed) {
+    // status word and the router's arrival counter start at zero on every call
+    cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
+    if (err != cudaSuccess) return cuda_status(err);
+  }
+  const moe_dims *dims = &d;
+  if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
+  unsigned long long *prof = prof_next();
+  for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
+    const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
+    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, s);
+    if (rc != MOE_OK) return rc;
+    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, prof, s);
+    if (rc != MOE_OK) return rc;
+  }
+  return MOE_OK;
+}
+
 int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
                       const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
                       int32_t *route_counts_opt, int32_t path, void *stream) {
@@ -503,20 +539,8 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   const bool pf = use_prefill(T, path);
   const WsLayout L = ws_layout(*dims, T, pf);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // status word and the router's arrival counter start at zero on every call
-  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
-  if (err != cudaSuccess) return cuda_status(err);
-  if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
-  unsigned long long *prof = prof_next();
-  for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
-    const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
-    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, s);
-    if (rc != MOE_OK) return rc;
-    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, prof, s);
-    if (rc != MOE_OK) return rc;
-  }
-  return MOE_OK;
+  return forward_checked(*dims, T, x, Wr, expert_table, out, ws, route_counts_opt, pf, L, false,
+                         static_cast<cudaStream_t>(stream));
 }
 
 int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws,
@@ -584,15 +608,30 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
   if (path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
   const WsLayout L = ws_layout(*dims, T, use_prefill(T, path));
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (!Wr || !expert_table || !aligned(Wr, 16)) return MOE_ERR_BAD_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   float *xd = at<float>(ws, L.xin);
   float *yd = at<float>(ws, L.yout);
+  const bool pf = use_prefill(T, path);
   const size_t bytes = (size_t)T * dims->H * sizeof(float);
-  cudaError_t err = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+  // Pinned host buffers the device can address: x comes across in the kernel
+  // that also zeroes the control words, and the decode path's down kernel
+  // writes out straight into host memory -- no separate copies.  Anything else
+  // (pageable memory, the prefill path's out) goes through cudaMemcpyAsync.
+  const float *x_dev_view = static_cast<const float *>(host_device_view(x_host));
+  float *out_dev_view = pf ? nullptr : static_cast<float *>(const_cast<void *>(host_device_view(out_host)));
+  cudaError_t err;
+  if (x_dev_view != nullptr && aligned(x_dev_view, 16)) {
+    err = launch_stage_in(x_dev_view, xd, (int64_t)T * dims->H, ws, L.xin, s);
+  } else {
+    err = cudaMemcpyAsync(xd, x_host, bytes, cudaMemcpyHostToDevice, s);
+    if (err == cudaSuccess) err = cudaMemsetAsync(ws, 0, L.xin, s);
+  }
   if (err != cudaSuccess) return cuda_status(err);
-  rc = moe_layer_forward(dims, T, xd, Wr, expert_table, yd, ws, ws_bytes, route_counts_opt, path,
-                         stream);
+  float *out_target = (out_dev_view != nullptr && aligned(out_dev_view, 16)) ? out_dev_view : yd;
+  rc = forward_checked(*dims, T, xd, Wr, expert_table, out_target, ws, route_counts_opt, pf, L, true, s);
   if (rc != MOE_OK) return rc;
+  if (out_target == out_dev_view) return MOE_OK;
   return cuda_status(cudaMemcpyAsync(out_host, yd, bytes, cudaMemcpyDeviceToHost, s));
 }
 

@@ -212,6 +212,10 @@ struct CombineArgs {
 
 // Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s);
+// Zero ctrl_bytes (a multiple of 16) at ctrl and copy n floats (a multiple of 4)
+// from device-accessible host memory to x_dev.
+cudaError_t launch_stage_in(const float *x_host, float *x_dev, int64_t n, void *ctrl, size_t ctrl_bytes,
+                            cudaStream_t s);
 cudaError_t launch_route_decode(const RouteArgs &a, cudaStream_t s);
 cudaError_t launch_bucket(const BucketArgs &a, cudaStream_t s);
 cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, float *w,

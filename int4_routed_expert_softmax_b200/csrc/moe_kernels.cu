@@ -40,6 +40,30 @@ __global__ void __launch_bounds__(256) k_quant(QuantArgs a) {
   }
 }
 
+// =====================================================================
+// Host-buffer entry: zero the workspace's control words and copy x from
+// device-accessible pinned host memory into the workspace (one pass of 16-byte
+// loads across the link), in place of a memset and a separate copy.
+// =====================================================================
+__global__ void __launch_bounds__(256) k_stage_in(const float4 *x_host, float4 *x_dev, int64_t n4, uint4 *ctrl,
+                                                  int ctrl16) {
+  if (blockIdx.x == 0)
+    for (int i = threadIdx.x; i < ctrl16; i += blockDim.x) ctrl[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x)
+    x_dev[i] = x_host[i];
+}
+
+cudaError_t launch_stage_in(const float *x_host, float *x_dev, int64_t n, void *ctrl, size_t ctrl_bytes,
+                            cudaStream_t s) {
+  const int64_t n4 = n / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 148) blocks = 148;
+  k_stage_in<<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float4 *>(x_host), reinterpret_cast<float4 *>(x_dev),
+                                              n4, static_cast<uint4 *>(ctrl), (int)(ctrl_bytes / 16));
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s) {
   if (a.nblk == 0) return cudaSuccess;
   int64_t blocks = (a.nblk + 7) / 8;
@@ -88,67 +112,81 @@ __device__ int block_exclusive_scan(const int *in, int *out, int n, int *scratch
 }
 
 // =====================================================================
-// Stable counting sort of P = T*k pairs by expert, one CTA.
-// s_idx: the pairs' experts in shared memory (or global), s_work: >= 3E+40
-// ints of shared memory.  Writes cnt, off, uni (+ shared slot E), n_uni,
-// perm, pos and pair_tok (routed positions, then T shared positions).
+// Stable counting sort of the P = T*k (token, slot) pairs by expert, one CTA.
+// Writes cnt, off, uni (+ shared slot E), n_uni, perm, pos and pair_tok
+// (routed positions, then T shared positions).
+// Each warp owns a contiguous segment of pairs.  Pass 1 counts per (warp,
+// expert); an exclusive scan over the warps (per expert) and over the experts
+// gives every warp its start inside every expert's range; pass 2 places the
+// pairs, lanes with equal experts ranked by lane -- pair order is kept inside
+// every expert, with no block-wide barrier in either pass.
+// s_work: 3E + 64 + (blockDim.x / 32) * E ints of shared memory.
 // =====================================================================
 __device__ void bucket_block(int E, int k, int T, const int32_t *idx, int *s_work, int32_t *cnt,
                              int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm,
                              int32_t *pos, int32_t *pair_tok) {
   const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = nt >> 5;
   const int P = T * k;
-  int *s_cnt = s_work;           // [E]
-  int *s_off = s_work + E;       // [E]  (exclusive)
-  int *s_cur = s_work + 2 * E;   // [E]  running cursors
-  int *scratch = s_work + 3 * E; // [40]
-  for (int e = tid; e < E; e += nt) s_cnt[e] = 0;
+  int *s_cnt = s_work;            // [E]
+  int *s_off = s_work + E;        // [E]  (exclusive)
+  int *s_flag = s_work + 2 * E;   // [E]  union flags, then union ranks
+  int *scratch = s_work + 3 * E;  // [64]
+  int *s_wc = scratch + 64;       // [nw][E]: per-warp counts, then per-warp cursors
+  for (int i = tid; i < nw * E; i += nt) s_wc[i] = 0;
   __syncthreads();
-  for (int p = tid; p < P; p += nt) atomicAdd(&s_cnt[idx[p]], 1);
+  const int seg = ((P + nw - 1) / nw + 31) & ~31;
+  const int p0 = min(P, warp * seg), p1 = min(P, p0 + seg);
+  int *wc = s_wc + (size_t)warp * E;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int c = p0; c < p1; c += 32) {
+    const int p = c + lane;
+    const bool has = p < p1;
+    const int e = has ? idx[p] : -1 - lane;  // distinct dummies never match
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (has && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += nt) {
+    int run = 0;
+    for (int w = 0; w < nw; ++w) {
+      const int c = s_wc[(size_t)w * E + e];
+      s_wc[(size_t)w * E + e] = run;
+      run += c;
+    }
+    s_cnt[e] = run;
+  }
   __syncthreads();
   block_exclusive_scan(s_cnt, s_off, E, scratch);
   for (int e = tid; e < E; e += nt) {
     cnt[e] = s_cnt[e];
     off[e] = s_off[e];
-    s_cur[e] = (s_cnt[e] > 0) ? 1 : 0;  // flags for the union scan
+    s_flag[e] = (s_cnt[e] > 0) ? 1 : 0;  // flags for the union scan
   }
   if (tid == 0) off[E] = P;
   __syncthreads();
-  const int nu = block_exclusive_scan(s_cur, s_cur, E, scratch);
+  const int nu = block_exclusive_scan(s_flag, s_flag, E, scratch);
   for (int e = tid; e < E; e += nt)
-    if (s_cnt[e] > 0) uni[s_cur[e]] = e;
+    if (s_cnt[e] > 0) uni[s_flag[e]] = e;
   if (tid == 0) {
     *n_uni = nu;
     uni[nu] = E;  // the shared expert follows the union
   }
-  __syncthreads();
-  for (int e = tid; e < E; e += nt) s_cur[e] = s_off[e];
-  __syncthreads();
-  // stable placement: chunks of nt pairs in order; inside a chunk, warps take
-  // turns; inside a warp, lanes with equal experts are ranked by lane.
-  const int nwarps = (nt + 31) / 32;
-  for (int c0 = 0; c0 < P; c0 += nt) {
-    const int p = c0 + tid;
-    const bool has = p < P;
-    const int e = has ? idx[p] : -1 - lane;  // distinct dummies never match
-    for (int w = 0; w < nwarps; ++w) {
-      if (warp == w) {
-        const unsigned peers = __match_any_sync(0xffffffffu, e);
-        const unsigned lt = (1u << lane) - 1u;
-        const int leader = __ffs(peers) - 1;
-        int base = 0;
-        if (has) base = s_cur[e];
-        __syncwarp();
-        if (has && lane == leader) s_cur[e] = base + __popc(peers);
-        if (has) {
-          const int q = base + __popc(peers & lt);
-          perm[q] = p;
-          if (pos) pos[p] = q;
-          if (pair_tok) pair_tok[q] = p / k;
-        }
-      }
-      __syncthreads();
+  for (int c = p0; c < p1; c += 32) {
+    const int p = c + lane;
+    const bool has = p < p1;
+    const int e = has ? idx[p] : -1 - lane;
+    const unsigned peers = __match_any_sync(0xffffffffu, e);
+    if (has) {
+      const int q = s_off[e] + wc[e] + __popc(peers & lt);
+      perm[q] = p;
+      if (pos) pos[p] = q;
+      if (pair_tok) pair_tok[q] = p / k;
     }
+    __syncwarp();
+    if (has && lane == __ffs(peers) - 1) wc[e] += __popc(peers);
+    __syncwarp();
   }
   if (pair_tok)
     for (int t = tid; t < T; t += nt) pair_tok[P + t] = t;
@@ -549,7 +587,10 @@ __global__ void __launch_bounds__(1024) k_bucket(BucketArgs a) {
 }
 
 cudaError_t launch_bucket(const BucketArgs &a, cudaStream_t s) {
-  const size_t smem = (size_t)(3 * a.E + 64) * 4;
+  const size_t smem = (size_t)(3 * a.E + 64 + 32 * a.E) * 4;
+  static int smem_set[64] = {0};
+  cudaError_t err = ensure_smem(k_bucket, smem, smem_set);
+  if (err != cudaSuccess) return err;
   k_bucket<<<1, 1024, smem, s>>>(a);
   return cudaGetLastError();
 }

@@ -218,6 +218,26 @@ def test_layer_forward_host_matches_device():
     assert torch.equal(oh, out_dev.cpu())
 
 
+@pytest.mark.parametrize("pinned", [True, False])
+def test_layer_forward_host_decode_T3(pinned):
+    """The host-buffer entry on the decode path: pinned buffers go across in
+    the staging kernel and the down kernel's own stores; pageable buffers
+    through copies.  Both equal the device-buffer call bit for bit."""
+    moe = _moe()
+    w = mi.shrink(mi.WORKLOADS["decode"], seed=91)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV, T=3)
+    out_dev, ws, d = gpu_layer(w, x, Wr, blobs)
+    xh = x.cpu()
+    oh = torch.full((3, w.H), float("nan"), dtype=torch.float32)
+    if pinned:
+        xh, oh = xh.pin_memory(), oh.pin_memory()
+    for _ in range(2):
+        moe.moe_layer_forward_host(d, xh, Wr, moe.expert_table(blobs), oh, ws)
+        torch.cuda.synchronize()
+        assert torch.equal(oh, out_dev.cpu())
+        oh.fill_(float("nan"))
+
+
 def test_route_counts_accumulate():
     moe = _moe()
     w = mi.WORKLOADS["tiny"]
