@@ -754,40 +754,56 @@ cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, c
 // the xor-tree sum over 32 chains, chain l = fmaf over h = 32 i + l with i
 // ascending.  A CTA holds 16 tokens x 32 experts; a warp keeps 8 x 8 logits,
 // lane l owning chain l of each.  x and Wr come through shared memory in K
-// chunks of 512.
+// chunks of 256, copied asynchronously one chunk ahead (two buffers).
 // ===========================================================================
-constexpr int kRtTok = 16, kRtExp = 32, kRtKC = 512;
+constexpr int kRtTok = 16, kRtExp = 32, kRtKC = 256;
+constexpr int kRtBuf = (kRtTok + kRtExp) * kRtKC;  // floats per K-chunk buffer
+
+// 16-byte asynchronous global -> shared copy; src_bytes = 0 writes zeros.
+__device__ __forceinline__ void cp_async16z(void *dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
 
 __global__ void __launch_bounds__(256) k_router_tiled(const RouterTiledArgs a) {
-  extern __shared__ __align__(16) float rsm[];
-  float *xs = rsm;                    // [kRtTok][kRtKC]
-  float *wsm = rsm + kRtTok * kRtKC;  // [kRtExp][kRtKC]
+  extern __shared__ __align__(16) float rsm[];  // 2 x {x [kRtTok][kRtKC], Wr [kRtExp][kRtKC]}
   const int H = a.H, E = a.E, T = a.T;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int t0 = blockIdx.x * kRtTok, e0 = blockIdx.y * kRtExp;
   const int tw = (warp & 1) * 8, ew = (warp >> 1) * 8;
+  // K-chunk copies run one chunk ahead of the arithmetic (two buffers)
+  auto load = [&](int k0, int b) {
+    const int kc4 = min(kRtKC, H - k0) / 4;
+    float *xs = rsm + b * kRtBuf, *wsm = xs + kRtTok * kRtKC;
+    for (int i = tid; i < kRtTok * kc4; i += 256) {
+      const int r = i / kc4, c = i - r * kc4;
+      const bool ok = t0 + r < T;
+      cp_async16z(xs + r * kRtKC + 4 * c, ok ? a.x + (size_t)(t0 + r) * H + k0 + 4 * c : a.x, ok ? 16u : 0u);
+    }
+    for (int i = tid; i < kRtExp * kc4; i += 256) {
+      const int r = i / kc4, c = i - r * kc4;
+      const bool ok = e0 + r < E;
+      cp_async16z(wsm + r * kRtKC + 4 * c, ok ? a.Wr + (size_t)(e0 + r) * H + k0 + 4 * c : a.Wr, ok ? 16u : 0u);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
   float acc[8][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
-  for (int k0 = 0; k0 < H; k0 += kRtKC) {
-    const int kc = min(kRtKC, H - k0);  // a multiple of 128
-    const int kc4 = kc / 4;
-    __syncthreads();
-    for (int i = threadIdx.x; i < kRtTok * kc4; i += 256) {
-      const int r = i / kc4, c = i - r * kc4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (t0 + r < T) v = __ldg(reinterpret_cast<const float4 *>(a.x + (size_t)(t0 + r) * H + k0) + c);
-      reinterpret_cast<float4 *>(xs + r * kRtKC)[c] = v;
-    }
-    for (int i = threadIdx.x; i < kRtExp * kc4; i += 256) {
-      const int r = i / kc4, c = i - r * kc4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e0 + r < E) v = __ldg(reinterpret_cast<const float4 *>(a.Wr + (size_t)(e0 + r) * H + k0) + c);
-      reinterpret_cast<float4 *>(wsm + r * kRtKC)[c] = v;
+  const int nch = (H + kRtKC - 1) / kRtKC;
+  load(0, 0);
+  for (int ci = 0; ci < nch; ++ci) {
+    if (ci + 1 < nch) {
+      load((ci + 1) * kRtKC, (ci + 1) & 1);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
     }
     __syncthreads();
+    const int kc = min(kRtKC, H - ci * kRtKC);  // a multiple of 128
+    const float *xs = rsm + (ci & 1) * kRtBuf, *wsm = xs + kRtTok * kRtKC;
     for (int k = lane; k < kc; k += 32) {
       float xv[8], wv[8];
 #pragma unroll
@@ -799,6 +815,7 @@ __global__ void __launch_bounds__(256) k_router_tiled(const RouterTiledArgs a) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = ffma(xv[i], wv[j], acc[i][j]);
     }
+    __syncthreads();  // the buffer is refilled by the next iteration's copies
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i)
@@ -814,7 +831,7 @@ __global__ void __launch_bounds__(256) k_router_tiled(const RouterTiledArgs a) {
 
 cudaError_t launch_router_tiled(const RouterTiledArgs &a, cudaStream_t s) {
   if (a.T == 0) return cudaSuccess;
-  const size_t smem = (size_t)(kRtTok + kRtExp) * kRtKC * 4;
+  const size_t smem = (size_t)2 * kRtBuf * 4;
   static int smem_set[64] = {0};
   cudaError_t err = ensure_smem(k_router_tiled, smem, smem_set);
   if (err != cudaSuccess) return err;
