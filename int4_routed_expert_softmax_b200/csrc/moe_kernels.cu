@@ -405,9 +405,52 @@ __device__ __forceinline__ void warp_topk_radix(const float *lg, int E, int k, i
   __syncwarp();
 }
 
+// The same selection for small k by k rounds of a warp argmax: each lane keeps
+// its NPER keys in registers; a round takes each lane's best live key (the
+// lowest index among equal keys), the warp's largest key, and among the lanes
+// holding it the lowest expert index -- so round r yields the r-th largest
+// logit, ties to the lower index, as the radix selection does.
+template <int NPER>
+__device__ __forceinline__ void warp_topk_rounds(const float *lg, int E, int k, int lane, int &e_sel,
+                                                 float &l_sel) {
+  uint32_t key[NPER];
+  uint32_t live = 0u;  // bit j: entry lane + 32 j present and not yet taken
+#pragma unroll
+  for (int j = 0; j < NPER; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? order_key(__ldcg(lg + e)) : 0u;
+    if (e < E) live |= 1u << j;
+  }
+  e_sel = 0;
+  l_sel = 0.0f;
+  for (int r = 0; r < k; ++r) {
+    uint32_t bk = 0u;
+    int bj = -1;
+#pragma unroll
+    for (int j = 0; j < NPER; ++j)
+      if (((live >> j) & 1u) && (bj < 0 || key[j] > bk)) {
+        bk = key[j];
+        bj = j;
+      }
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bj >= 0 ? bk : 0u);
+    const uint32_t cand = (bj >= 0 && bk == m) ? (uint32_t)(lane + 32 * bj) : 0xFFFFFFFFu;
+    const uint32_t win = __reduce_min_sync(0xffffffffu, cand);
+    if (win != 0xFFFFFFFFu && lane == (int)(win & 31u)) live &= ~(1u << (win >> 5));
+    if (lane == r) {
+      e_sel = (int)win;
+      l_sel = key_value(m);
+    }
+  }
+}
+
 __device__ __forceinline__ void warp_topk(const float *lg, int E, int k, int lane, int &e_sel,
                                           float &l_sel, uint32_t *scratch) {
   const int nper = (E + 31) >> 5;
+  if (k <= 12 && nper <= 8) {
+    if (nper <= 4) warp_topk_rounds<4>(lg, E, k, lane, e_sel, l_sel);
+    else warp_topk_rounds<8>(lg, E, k, lane, e_sel, l_sel);
+    return;
+  }
   if (nper <= 1) warp_topk_radix<1>(lg, E, k, lane, e_sel, l_sel, scratch);
   else if (nper <= 2) warp_topk_radix<2>(lg, E, k, lane, e_sel, l_sel, scratch);
   else if (nper <= 4) warp_topk_radix<4>(lg, E, k, lane, e_sel, l_sel, scratch);

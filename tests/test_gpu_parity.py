@@ -63,6 +63,24 @@ def test_router_topk_bit_exact(name, T):
     assert np.array_equal(cnt.cpu().numpy(), np.bincount(io.reshape(-1), minlength=w.E))
 
 
+@pytest.mark.parametrize("E,k,T", [(512, 8, 5), (256, 16, 3), (1024, 32, 2), (40, 12, 7)])
+def test_router_topk_selection_paths(E, k, T):
+    # k <= 12 with E <= 256 takes the argmax-rounds selection, the rest the radix selection
+    moe = _moe()
+    H = 256
+    x = mi.make_x(T, H, 21 + E, DEV)
+    Wr = mi.make_router(E, H, 22 + k, DEV)
+    d = moe.dims(H, 128, E, k)
+    idx = torch.empty((T, k), dtype=torch.int32, device=DEV)
+    wt = torch.empty((T, k), dtype=torch.float32, device=DEV)
+    lg = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    moe.moe_router_topk(d, x, Wr, idx, wt, lg)
+    torch.cuda.synchronize()
+    io, wo = orc.topk_softmax(orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy()), k)
+    assert np.array_equal(idx.cpu().numpy(), io)
+    assert np.array_equal(wt.cpu().numpy().view(np.uint32), wo.view(np.uint32))
+
+
 def test_router_ties_lower_index_first():
     moe = _moe()
     H, E, k, T = 256, 16, 4, 3
