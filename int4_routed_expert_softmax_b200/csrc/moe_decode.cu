@@ -148,7 +148,7 @@ __host__ __device__ inline GuPlan gu_plan(int H, int T, int R, int ns, int csz) 
   p.red = o;
   o += al128d((size_t)8 * (2 * T > 8 ? 2 * T : 8) * 33 * 4);
   p.gu = o;
-  o += al128d((size_t)T * 64 * 4);
+  o += al128d((size_t)(T == 1 ? 2 : T) * 64 * 4);  // one token: two buffers (unit parity)
   p.xd = o;
   o += al128d((size_t)T * (H / 32) * 4);
   p.qs = o;
@@ -318,6 +318,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
 
   int n_tok = 0, pos_base = 0, my_tok = 0;
   int slot = u_begin / rbs, rb = u_begin % rbs, st = 0, s = 0;
+  int cu = 0;  // units this CTA has completed
   uint32_t ph = 0;
   bool bad = false;
   for (int j = 0; j < n_stages; ++j) {
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
           if (lane < 8) {
             const int sq = lane / RPW, q = lane % RPW;
             const int jr = warp + 8 * q;
-            gu[(jr / R) * 32 + sq * R + jr % R] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
+            gu[(cu & 1) * 64 + (jr / R) * 32 + sq * R + jr % R] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
           }
           __syncwarp();
         }
@@ -386,7 +387,36 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
         __syncwarp();
       }
     }
-    if (st == SPU - 1) {
+    if (ONE && st == SPU - 1) {
+      // unit complete: one warp (rotating with the unit) waits for the
+      // others' g and u sums and forms h = SiLU(g) * u and its Q8_0 block;
+      // the rest arrive and go on to the next unit.  The sums sit in one of
+      // two buffers and barriers by unit parity: the ring of NS < 2 units of
+      // stages keeps every warp within one unit of the slowest, so a buffer
+      // is rewritten only after its reader is done with it.
+      const int par = cu & 1;
+      __threadfence_block();
+      if ((cu & 7) == warp) {
+        named_sync(2 + par, 256);
+        if (!bad) {
+          const float *gb = gu + par * 64;
+          const float h = swiglu(gb[lane], gb[32 + lane]);
+          const float d = fdiv(warp_max(fabsf(h)), 127.0f);
+          const int q = q8_code(h, d);
+          a.hq[(size_t)pos_base * I + rb * 32 + lane] = (int8_t)q;
+          int qsum = q;
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
+          if (lane == 0) {
+            a.hd[(size_t)pos_base * (I / 32) + rb] = d;
+            a.hqs[(size_t)pos_base * (I / 32) + rb] = qsum;
+          }
+        }
+      } else {
+        named_arrive(2 + par, 256);
+      }
+      ++cu;
+    } else if (st == SPU - 1) {
       // unit complete: h = SiLU(g) * u for its 32 rows, Q8_0 per token
       named_sync(1, 256);
       if (!bad) {
@@ -421,6 +451,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
     }
   }
+  if (ONE) named_sync(1, 256);  // the end stamp follows the last unit's epilogue
   prof_end(a.prof, 1);
 }
 
@@ -431,7 +462,9 @@ size_t gateup_smem_bytes(int H, int T, int R, int nstage) {
 }
 
 // Rows per matrix per stage and stage count: 8 rows (two per warp) when three
-// or more stages of that size fit, else 4.
+// or more stages of that size fit, else 4.  At most 6 stages: fewer than the
+// 2 x 32 / R stages of two units, which the single-token epilogue hand-off
+// relies on.
 void gateup_plan(int H, int T, int *R, int *nstage) {
   for (int r = 8; r >= 4; r -= 4) {
     int ns = 8;

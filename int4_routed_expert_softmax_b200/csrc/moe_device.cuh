@@ -193,6 +193,13 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Arrival at named barrier `id` without waiting (the waiting side uses
+// named_sync with the same thread count); prior shared-memory writes of the
+// arriving threads are visible to the waiting threads once it completes.
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Programmatic dependent launch: wait for the preceding kernel's results /
 // let the following kernel start its prologue.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
