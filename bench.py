@@ -152,7 +152,9 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- distributed
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """One process per GPU (RANK / LOCAL_RANK / WORLD_SIZE from the launcher).
+    The bench uses NCCL; the CPU tests of this plumbing use gloo."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -160,10 +162,19 @@ def dist_setup():
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     return ws, rank, local
+
+
+def rank_seed(w: mi.Workload, rank: int) -> int:
+    """Seed of a rank's replica: every rank draws its own router, experts and tokens
+    (independent problems; no data-path collective)."""
+    return w.seed + 1000 * rank
 
 
 def barrier(ws):
@@ -172,22 +183,28 @@ def barrier(ws):
         dist.barrier()
 
 
-def allreduce_max(v: float, ws: int) -> float:
+def _reduce(v: float, ws: int, op: str) -> float:
     if ws == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def allreduce_max(v: float, ws: int) -> float:
+    return _reduce(v, ws, "max")
 
 
 def allreduce_sum(v: float, ws: int) -> float:
-    if ws == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce(v, ws, "sum")
+
+
+def aggregate(my_units: float, my_ms: float, ws: int):
+    """Whole-job totals: the units all ranks processed and the slowest rank's
+    device time (ms); the job's throughput is their ratio."""
+    return allreduce_sum(float(my_units), ws), allreduce_max(float(my_ms), ws)
 
 
 # ----------------------------------------------------------------- oracle timing
@@ -230,7 +247,7 @@ def run_native(args, ws_n, rank, local):
     w = mi.WORKLOADS[args.workload]
     if args.experts:
         w = mi.shrink(w, E=args.experts)
-    seed = w.seed + 1000 * rank
+    seed = rank_seed(w, rank)
     wl = mi.shrink(w, seed=seed)
     T = w.T
     Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), dev)
@@ -295,8 +312,7 @@ def run_native(args, ws_n, rank, local):
 
     my_bytes = sum((u + 1) * blob_b for u in nuni)
     my_ms = sum(layer_ms)
-    max_ms = allreduce_max(my_ms, ws_n)
-    all_bytes = allreduce_sum(float(my_bytes), ws_n)
+    all_bytes, max_ms = aggregate(my_bytes, my_ms, ws_n)
     value = all_bytes / (max_ms * 1e-3) / 1e9
     ms_per_step = max_ms / K
 
@@ -395,7 +411,7 @@ def run_prefill(args, ws_n, rank, local):
     w = mi.WORKLOADS["prefill"]
     if args.experts:
         w = mi.shrink(w, E=args.experts)
-    seed = w.seed + 1000 * rank
+    seed = rank_seed(w, rank)
     T = args.tokens or w.T
     x = mi.make_x(T, w.H, mi.sub_seed(seed, 0, 1), dev, zipf=True)
     Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), dev, zipf_s=w.zipf_s)
@@ -547,7 +563,7 @@ def run_stacked(args, ws_n, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = mi.WORKLOADS["stacked"]
-    seed = w.seed + 1000 * rank
+    seed = rank_seed(w, rank)
     L = w.layers
     routers = [mi.make_router(w.E, w.H, mi.sub_seed(seed, l, 2), dev) for l in range(L)]
     blobs = [mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, l, 3), dev) for l in range(L)]
@@ -604,7 +620,7 @@ def run_tiered(args, ws_n, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     w = mi.WORKLOADS["tiered"]
-    seed = w.seed + 1000 * rank
+    seed = rank_seed(w, rank)
     L, E1 = w.layers, w.E + 1
     n_tok = args.steps
     host = torch.empty((L, E1, w.blob_bytes), dtype=torch.uint8, pin_memory=True)
