@@ -163,13 +163,16 @@ __host__ __device__ inline GuPlan gu_plan(int H, int T, int R, int ns, int csz) 
 
 // Work unit = (union slot, 32-row block of I); slot 0 is the shared expert,
 // slot u >= 1 is uni[u-1]; units are split evenly over the CTAs.  A stage is
-// R gate rows + R up rows (packed nibbles + fp16 scales).  Consumer warp w
-// owns rows w and w+8 of the stage (R = 8: gate row w and up row w) or row w
-// (R = 4).
-template <int CSZ, bool ONE, int R>
-__global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
-  constexpr int SPU = 32 / R;  // stages per 32-row unit
-  constexpr int RPW = R / 4;   // rows per warp per stage
+// R gate rows + R up rows (packed nibbles + fp16 scales).  NW consumer warps
+// (warp NW is the producer); consumer warp w owns rows w, w + NW, ... of the
+// stage's 2R rows (NW = 8, R = 8: gate row w and up row w; NW = 16: one row).
+template <int CSZ, bool ONE, int R, int NW>
+__global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a) {
+  static_assert(NW == 8 || (ONE && NW == 16 && R == 8), "16 consumer warps: one token, 8-row stages");
+  constexpr int SPU = 32 / R;         // stages per 32-row unit
+  constexpr int RPW = 2 * R / NW;     // rows per warp per stage
+  constexpr int PWR = SPU * RPW;      // rows per warp per unit
+  constexpr int NCT = NW * 32;        // consumer threads
   extern __shared__ __align__(128) unsigned char smem[];
   const int H = a.H, I = a.I, T = a.T, NS = a.nstage;
   const int G = H / 64, HB = H / 32;
@@ -190,7 +193,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     s_abort = 0;
     for (int s = 0; s < NS; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, 8);
+      mbar_init(empty + s, NW);
     }
     fence_barrier_init();
   }
@@ -200,8 +203,9 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
     // grid's own routing inputs are complete, which is all it reads early
     pdl_launch_dependents();
   }
-  // an earlier kernel of this call failed: leave everything untouched
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  // an earlier kernel of this call failed: leave everything untouched (one
+  // decision for the whole CTA, so that no named barrier below misses a warp)
+  if (__syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   prof_start(a.prof, 1);
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int rbs = I / 32;  // 32-row units per expert
@@ -227,16 +231,16 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
 
   // activations (consumer warps only; the producer starts streaming weights
   // at once): xq in per-lane chunks (padded rows), block scales, code sums
-  if (warp != 8) {
+  if (warp != NW) {
     const int pieces = CSZ * 4;
-    for (int i = tid; i < T * 32 * pieces; i += 256) {
+    for (int i = tid; i < T * 32 * pieces; i += NCT) {
       const int t = i / (32 * pieces), r = i % (32 * pieces), c = r / pieces, j = r % pieces;
       const int col = c * CSZ * 64 + 16 * j;
       uint4 v = make_uint4(0, 0, 0, 0);
       if (col < H) v = *reinterpret_cast<const uint4 *>(a.xq + (size_t)t * H + col);
       *reinterpret_cast<uint4 *>(xq_s + (size_t)(t * 32 + c) * pl.chp + 16 * j) = v;
     }
-    for (int i = tid; i < T * HB; i += 256) {
+    for (int i = tid; i < T * HB; i += NCT) {
       xd_s[i] = a.xd[i];
       const uint4 *q4 = reinterpret_cast<const uint4 *>(a.xq + (size_t)i * 32);
       int s = 0;
@@ -250,10 +254,10 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
       qs_s[i] = s;
     }
-    named_sync(1, 256);
+    named_sync(1, NCT);
   }
 
-  if (warp == 8) {
+  if (warp == NW) {
     // -------------------------------------------------------------- producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
@@ -311,7 +315,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
   int row_m[RPW], row_r[RPW];
 #pragma unroll
   for (int q = 0; q < RPW; ++q) {
-    const int jr = warp + 8 * q;
+    const int jr = warp + NW * q;
     row_m[q] = jr / R;
     row_r[q] = jr % R;
   }
@@ -353,16 +357,16 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
       if (ONE) {
-        // chunk values of the warp's 8 rows of the unit, summed once per unit
+        // chunk values of the warp's PWR rows of the unit, summed once per unit
 #pragma unroll
         for (int q = 0; q < RPW; ++q)
-          red[(warp * 8 + st * RPW + q) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act1, d1, z1, c0, G);
+          red[(warp * PWR + st * RPW + q) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act1, d1, z1, c0, G);
         if (st == SPU - 1) {
           __syncwarp();
-          if (lane < 8) {
+          if (lane < PWR) {
             const int sq = lane / RPW, q = lane % RPW;
-            const int jr = warp + 8 * q;
-            gu[(cu & 1) * 64 + (jr / R) * 32 + sq * R + jr % R] = chunk_sum(red + (warp * 8 + lane) * 33, nch);
+            const int jr = warp + NW * q;
+            gu[(cu & 1) * 64 + (jr / R) * 32 + sq * R + jr % R] = chunk_sum(red + (warp * PWR + lane) * 33, nch);
           }
           __syncwarp();
         }
@@ -396,8 +400,8 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       // is rewritten only after its reader is done with it.
       const int par = cu & 1;
       __threadfence_block();
-      if ((cu & 7) == warp) {
-        named_sync(2 + par, 256);
+      if (cu % NW == warp) {
+        named_sync(2 + par, NCT);
         if (!bad) {
           const float *gb = gu + par * 64;
           const float h = swiglu(gb[lane], gb[32 + lane]);
@@ -413,7 +417,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
           }
         }
       } else {
-        named_arrive(2 + par, 256);
+        named_arrive(2 + par, NCT);
       }
       ++cu;
     } else if (st == SPU - 1) {
@@ -451,7 +455,7 @@ __global__ void __launch_bounds__(288, 1) k_gateup_decode(GateUpArgs a) {
       }
     }
   }
-  if (ONE) named_sync(1, 256);  // the end stamp follows the last unit's epilogue
+  if (ONE) named_sync(1, NCT);  // the end stamp follows the last unit's epilogue
   prof_end(a.prof, 1);
 }
 
@@ -477,14 +481,14 @@ void gateup_plan(int H, int T, int *R, int *nstage) {
   }
 }
 
-template <int CSZ, bool ONE, int R>
+template <int CSZ, bool ONE, int R, int NW = 8>
 static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
   static int smem_set[64] = {0};
-  cudaError_t err = ensure_smem(k_gateup_decode<CSZ, ONE, R>, smem, smem_set);
+  cudaError_t err = ensure_smem(k_gateup_decode<CSZ, ONE, R, NW>, smem, smem_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(288);
+  cfg.blockDim = dim3(NW * 32 + 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -492,12 +496,16 @@ static cudaError_t launch_gu(const GateUpArgs &a, int grid, size_t smem, cudaStr
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = a.use_pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ, ONE, R>, a);
+  return cudaLaunchKernelEx(&cfg, k_gateup_decode<CSZ, ONE, R, NW>, a);
 }
 
 template <int CSZ>
 static cudaError_t launch_gu_csz(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s) {
   const bool one = a.T == 1;
+  // 8 consumer warps.  The consumers, not the copies, bound this kernel (the
+  // producer waits for a free stage over half its time), but 16 consumer
+  // warps (NW = 16) measured slower: 17 warps per CTA cap the registers at 96
+  // and the hot loop spills (36.8 us against 27.5 us per launch).
   if (a.rpm == 8)
     return one ? launch_gu<CSZ, true, 8>(a, grid, smem, s) : launch_gu<CSZ, false, 8>(a, grid, smem, s);
   return one ? launch_gu<CSZ, true, 4>(a, grid, smem, s) : launch_gu<CSZ, false, 4>(a, grid, smem, s);
@@ -595,8 +603,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   // wait, and the first ring of weight copies overlaps the gate/up kernel's
   // tail.  The h codes (the gate/up kernel's output) are read after it.
   prof_start(a.prof, 2);
-  __syncthreads();
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  if (__syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int nslot = n_uni + 1;
   {
@@ -692,17 +699,15 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     }
     return;
   }
-  // consumers: the gate/up kernel's outputs are read only after its completion
+  // consumers: the gate/up kernel's outputs are read only after its completion.
+  // A failure seen here skips the work but not the final named barrier.
   if (a.use_pdl) pdl_wait();
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) {
-    s_abort = 1;
-    return;
-  }
+  bool bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int32_t *>(a.status) != 0);
+  if (bad && lane == 0) s_abort = 1;
 
   const int c0 = lane * CSZ;
   float *redw = red + warp * 32 * 33;
-  bool bad = false;
-  if (a.preload) {
+  if (a.preload && !bad) {
     bad = !mbar_wait(actbar, 0, a.status, kDetDnFull);
     bad = __any_sync(0xffffffffu, bad);
     if (bad && lane == 0) s_abort = 1;
