@@ -158,7 +158,8 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
  *   path: enum moe_path.
  * Every step runs in the library's kernels; nothing is synchronised with the
  * host.  Device-side failures (a bounded wait that ran out, a misaligned
- * blob) are written to the workspace status word (see moe_ws_view). */
+ * blob) are written to the workspace status word (see moe_ws_view), which
+ * every call resets first: read it after a call and before the next. */
 int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
                       const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
                       int32_t *route_counts_opt, int32_t path, void *stream);
@@ -358,7 +359,9 @@ int moe_device_sms(void);
  *       prefill = the down grouped GEMM and the combine kernel,
  *   [3] the call: first start to last end over the three phases,
  * (0 for a phase that was not stamped), then zeroes the ring and starts a new
- * history.  Returns the number of calls written, or a negative status. */
+ * history.  Returns the number of calls written, or a negative status.
+ * The profiling state is process-wide; a lock serialises these calls and the
+ * record hand-out of concurrent layer calls. */
 int moe_profile_enable(int on);
 int moe_profile_read(float *ms, int max_calls);
 

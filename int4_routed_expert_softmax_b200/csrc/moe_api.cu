@@ -33,7 +33,9 @@ bool dims_shape_ok(const moe_dims &d) {
 // ---- optional per-call kernel timing (moe_profile_enable).  Each profiled
 // call owns one zeroed record of a per-device ring; its kernels stamp their
 // phases there with %globaltimer, so nothing is added to the stream between
-// them.  The ring is zeroed at enable and after every read.
+// them.  The ring is zeroed at enable and after every read.  The state is
+// process-wide; g_prof_mu serialises every access to it across host threads.
+std::mutex g_prof_mu;
 bool g_prof = false;
 unsigned long long *g_prof_buf[kMaxDevices] = {};
 int g_prof_n[kMaxDevices] = {};
@@ -48,6 +50,7 @@ int current_device() {
 // A fresh record for the next call on the current device, or null when
 // profiling is off or the ring is full (the call then goes unrecorded).
 unsigned long long *prof_next() {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof) return nullptr;
   const int dev = current_device();
   if (dev < 0 || g_prof_buf[dev] == nullptr || g_prof_n[dev] >= kProfSlots) return nullptr;
@@ -57,6 +60,7 @@ unsigned long long *prof_next() {
 
 // The record of the most recent routing call (the experts half of a split layer).
 unsigned long long *prof_current() {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof) return nullptr;
   const int dev = current_device();
   return dev < 0 ? nullptr : g_prof_cur[dev];
@@ -390,6 +394,7 @@ int moe_device_sms(void) {
 }
 
 int moe_profile_enable(int on) {
+  std::lock_guard<std::mutex> lock(g_prof_mu);
   if (on) {
     const int dev = current_device();
     if (dev < 0) return MOE_ERR_CUDA;
@@ -414,6 +419,7 @@ int moe_profile_enable(int on) {
 
 int moe_profile_read(float *ms, int max_calls) {
   if (ms == nullptr || max_calls < 0) return MOE_ERR_BAD_ARG;
+  std::lock_guard<std::mutex> lock(g_prof_mu);
   const int dev = current_device();
   if (dev < 0) return MOE_ERR_CUDA;
   if (g_prof_buf[dev] == nullptr) return 0;
