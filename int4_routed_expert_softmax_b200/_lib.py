@@ -76,8 +76,38 @@ def lib() -> ctypes.CDLL:
 def _ptr(t: torch.Tensor | None):
     if t is None:
         return None
-    assert t.is_contiguous(), "tensors passed to libmoe must be contiguous"
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _arg(t, name: str, dtype, numel: int = 0, cuda: bool = True, optional: bool = False):
+    """Checks a tensor before its address crosses the C ABI, which sees only
+    pointers: device (or host) memory, dtype, contiguity, and at least `numel`
+    elements -- so that a wrong tensor is refused here instead of being read
+    or written out of bounds by a kernel."""
+    if t is None:
+        if optional:
+            return
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.is_cuda != cuda:
+        raise ValueError(f"{name} must be in {'device' if cuda else 'host'} memory")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < numel:
+        raise ValueError(f"{name} has {t.numel()} elements, needs at least {numel}")
+
+
+def _rows(x, name: str, cols: int, cuda: bool = True) -> int:
+    """x [T][cols] float32: returns T."""
+    _arg(x, name, torch.float32, cuda=cuda)
+    if x.dim() != 2 or x.shape[1] != cols:
+        raise ValueError(f"{name} must be [T][{cols}], got {tuple(x.shape)}")
+    return x.shape[0]
 
 
 def _stream(stream=None):
@@ -134,24 +164,54 @@ def moe_profile_read(max_calls: int = 1024) -> list:
 
 
 def moe_quant_q8_0(x: torch.Tensor, q: torch.Tensor, d: torch.Tensor, stream=None):
+    _arg(x, "x", torch.float32)
+    if x.dim() != 2:
+        raise ValueError("x must be [rows][cols]")
     rows, cols = x.shape
+    _arg(q, "q", torch.int8, rows * cols)
+    _arg(d, "d", torch.float32, rows * (cols // 32))
     _check("moe_quant_q8_0", lib().moe_quant_q8_0(_ptr(x), rows, cols, _ptr(q), _ptr(d), _stream(stream)))
 
 
 def moe_router_topk(d: MoeDims, x, Wr, idx, w, logits, route_counts=None, stream=None):
+    T = _rows(x, "x", d.H)
+    _arg(Wr, "Wr", torch.float32, d.E * d.H)
+    _arg(idx, "idx", torch.int32, T * d.k)
+    _arg(w, "w", torch.float32, T * d.k)
+    _arg(logits, "logits", torch.float32, T * d.E)
+    _arg(route_counts, "route_counts", torch.int32, d.E, optional=True)
     _check("moe_router_topk", lib().moe_router_topk(
         ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(idx), _ptr(w), _ptr(logits),
         _ptr(route_counts), _stream(stream)))
 
 
 def moe_bucket(d: MoeDims, idx, cnt, off, uni, n_uni, perm, stream=None):
+    _arg(idx, "idx", torch.int32)
+    if idx.dim() != 2 or idx.shape[1] != d.k:
+        raise ValueError(f"idx must be [T][{d.k}], got {tuple(idx.shape)}")
+    T = idx.shape[0]
+    _arg(cnt, "cnt", torch.int32, d.E)
+    _arg(off, "off", torch.int32, d.E + 1)
+    _arg(uni, "uni", torch.int32, d.E)
+    _arg(n_uni, "n_uni", torch.int32, 1)
+    _arg(perm, "perm", torch.int32, T * d.k)
     _check("moe_bucket", lib().moe_bucket(
         ctypes.byref(d), idx.shape[0], _ptr(idx), _ptr(cnt), _ptr(off), _ptr(uni), _ptr(n_uni),
         _ptr(perm), _stream(stream)))
 
 
+def _layer_args(d: MoeDims, x, Wr, table, out, route_counts, host: bool):
+    T = _rows(x, "x", d.H, cuda=not host)
+    _arg(out, "out", torch.float32, T * d.H, cuda=not host)
+    _arg(Wr, "Wr", torch.float32, d.E * d.H)
+    _arg(table, "table", torch.int64, d.E + 1)
+    _arg(route_counts, "route_counts", torch.int32, d.E, optional=True)
+
+
 def moe_layer_forward(d: MoeDims, x, Wr, table, out, ws, route_counts=None,
                       path: int = MOE_PATH_AUTO, stream=None):
+    _layer_args(d, x, Wr, table, out, route_counts, host=False)
+    _arg(ws, "ws", torch.uint8)
     _check("moe_layer_forward", lib().moe_layer_forward(
         ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
@@ -159,6 +219,8 @@ def moe_layer_forward(d: MoeDims, x, Wr, table, out, ws, route_counts=None,
 
 def moe_layer_forward_host(d: MoeDims, x_host, Wr, table, out_host, ws, route_counts=None,
                            path: int = MOE_PATH_AUTO, stream=None):
+    _layer_args(d, x_host, Wr, table, out_host, route_counts, host=True)
+    _arg(ws, "ws", torch.uint8)
     _check("moe_layer_forward_host", lib().moe_layer_forward_host(
         ctypes.byref(d), x_host.shape[0], _ptr(x_host), _ptr(Wr), _ptr(table), _ptr(out_host),
         _ptr(ws), ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
@@ -167,12 +229,14 @@ def moe_layer_forward_host(d: MoeDims, x_host, Wr, table, out_host, ws, route_co
 def moe_layer_forward_static(d: MoeDims, x, Wr, table, out, route_counts=None,
                              path: int = MOE_PATH_AUTO, stream=None):
     """moe_layer_forward on the library's static device workspace (no allocation)."""
+    _layer_args(d, x, Wr, table, out, route_counts, host=False)
     _check("moe_layer_forward_static", lib().moe_layer_forward_static(
         ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(route_counts),
         path, _stream(stream)))
 
 
 def moe_workspace_view(d: MoeDims, T: int, ws: torch.Tensor) -> MoeWsView:
+    _arg(ws, "ws", torch.uint8)
     v = MoeWsView()
     _check("moe_workspace_view", lib().moe_workspace_view(ctypes.byref(d), T, _ptr(ws), ctypes.byref(v)))
     return v
