@@ -7,7 +7,7 @@ import ctypes
 
 import torch
 
-from ._lib import MoeDims, MoeError, _ptr, _stream, lib
+from ._lib import MoeDims, MoeError, _arg, _ptr, _rows, _stream, lib
 
 MOE_CACHE_DEVICE, MOE_CACHE_HOST = 0, 1
 MOE_FAULT_NONE, MOE_FAULT_COPY, MOE_FAULT_ALLOC = 0, 1, 2
@@ -161,6 +161,14 @@ class ExpertCache:
     def tiered_layer_forward(self, layer, x, Wr, out, ws, ws_pred=None, Wr_next=None,
                              route_counts=None, compute_stream=None, side_stream=None):
         """One tiered decode layer; returns (prefetches started, predicted union size)."""
+        d = self.d
+        T = _rows(x, "x", d.H)
+        _arg(Wr, "Wr", torch.float32, d.E * d.H)
+        _arg(Wr_next, "Wr_next", torch.float32, d.E * d.H, optional=True)
+        _arg(out, "out", torch.float32, T * d.H)
+        _arg(ws, "ws", torch.uint8)
+        _arg(ws_pred, "ws_pred", torch.uint8, optional=True)
+        _arg(route_counts, "route_counts", torch.int32, d.E, optional=True)
         po = (ctypes.c_int32 * 2)()
         _chk("moe_tiered_layer_forward", _sigs().moe_tiered_layer_forward(
             self.handle, layer, ctypes.byref(self.d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(Wr_next),
@@ -178,12 +186,17 @@ def _cstream(stream):
 
 
 def moe_layer_route(d: MoeDims, x, Wr, ws, route_counts=None, stream=None):
+    _rows(x, "x", d.H)
+    _arg(Wr, "Wr", torch.float32, d.E * d.H)
+    _arg(ws, "ws", torch.uint8)
+    _arg(route_counts, "route_counts", torch.int32, d.E, optional=True)
     _chk("moe_layer_route", _sigs().moe_layer_route(
         ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(ws), _nbytes(ws), _ptr(route_counts),
         _stream(stream)))
 
 
 def moe_read_union(d: MoeDims, T: int, ws, stream=None):
+    _arg(ws, "ws", torch.uint8)
     buf = (ctypes.c_int32 * d.E)()
     n = ctypes.c_int32()
     _chk("moe_read_union", _sigs().moe_read_union(ctypes.byref(d), T, _ptr(ws), buf, ctypes.byref(n),
@@ -192,6 +205,10 @@ def moe_read_union(d: MoeDims, T: int, ws, stream=None):
 
 
 def moe_layer_experts(d: MoeDims, T: int, table, out, ws, stream=None):
+    if not isinstance(table, int):
+        _arg(table, "table", torch.int64, d.E + 1)
+    _arg(out, "out", torch.float32, T * d.H)
+    _arg(ws, "ws", torch.uint8)
     tp = table if isinstance(table, int) else table.data_ptr()
     _chk("moe_layer_experts", _sigs().moe_layer_experts(
         ctypes.byref(d), T, ctypes.c_void_p(tp), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)))
