@@ -68,7 +68,8 @@ enum moe_status {
   MOE_ERR_NOT_RESIDENT = -6,/* expert not in the cache */
   MOE_ERR_TIMEOUT = -7,     /* a device-side bounded wait ran out */
   MOE_ERR_DEVICE = -8,      /* device-side check failed (see status word) */
-  MOE_ERR_ALLOC = -9        /* host or device allocation failed */
+  MOE_ERR_ALLOC = -9,       /* host or device allocation failed */
+  MOE_ERR_IO = -10          /* a file is missing, unreadable or corrupt */
 };
 
 typedef struct moe_dims {
@@ -296,6 +297,22 @@ int expert_cache_stats(const moe_cache *cache, moe_cache_stats *stats);
 /* Host-side fault injection for failure tests (see enum moe_cache_fault);
  * cache may be NULL for MOE_FAULT_ALLOC. */
 int expert_cache_inject_fault(moe_cache *cache, int32_t kind, int32_t count);
+
+/* Route-usage record on disk (the learned cache's history across sessions:
+ * the engine writes the experts each turn routes to into a usage file and
+ * pins the hottest -- tantan.ink page, section 几个关键工程动作; "colibri deep
+ * review", 学习缓存 row).  counts: HOST array [n_layers][E] of selection
+ * counts (the per-layer route_counts of the layer calls, widened to 64 bits).
+ * moe_usage_save writes <path>.tmp and renames it over <path> (a reader never
+ * sees a partial record); the file holds a magic tag, the version, n_layers,
+ * E, the counts and an FNV-1a 64 hash of them.  moe_usage_load replaces
+ * counts (accumulate = 0) or adds the file's counts to them (accumulate = 1);
+ * MOE_ERR_SHAPE if the file was written for other n_layers / E, MOE_ERR_IO if
+ * it is missing, truncated, longer than its record or fails its hash --
+ * counts are left untouched on every error.  Host only; no GPU needed. */
+int moe_usage_save(const char *path, int32_t n_layers, int32_t E, const uint64_t *counts);
+int moe_usage_load(const char *path, int32_t n_layers, int32_t E, uint64_t *counts,
+                   int32_t accumulate);
 
 /* One tiered decode layer (native runtime of the cache):
  * route(x) -> read union -> acquire (misses copied on side_stream, compute

@@ -4,13 +4,16 @@ every kernel live in libmoe.so."""
 from __future__ import annotations
 
 import ctypes
+import os
 
+import numpy as np
 import torch
 
 from ._lib import MoeDims, MoeError, _arg, _ptr, _rows, _stream, lib
 
 MOE_CACHE_DEVICE, MOE_CACHE_HOST = 0, 1
 MOE_FAULT_NONE, MOE_FAULT_COPY, MOE_FAULT_ALLOC = 0, 1, 2
+MOE_ERR_IO = -10
 
 
 class CacheStats(ctypes.Structure):
@@ -52,6 +55,8 @@ def _sigs():
         "moe_layer_experts": (ctypes.c_int, [D, i32, P, P, P, sz, P]),
         "moe_tiered_layer_forward": (ctypes.c_int, [P, i32, D, i32, P, P, P, P, P, sz, P, sz, P, P, P,
                                                     I32P]),
+        "moe_usage_save": (ctypes.c_int, [ctypes.c_char_p, i32, i32, ctypes.POINTER(ctypes.c_uint64)]),
+        "moe_usage_load": (ctypes.c_int, [ctypes.c_char_p, i32, i32, ctypes.POINTER(ctypes.c_uint64), i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -143,7 +148,8 @@ class ExpertCache:
                     _sigs().expert_cache_release(self.handle, layer, _cstream(compute_stream)))
 
     def learn_pins(self, layer, counts, n_pin, stream=None):
-        a, _ = _ilist(counts)
+        # 64-bit usage counts saturate at the 32-bit range the call takes
+        a, _ = _ilist(min(int(v), 2**31 - 1) for v in counts)
         return _chk("expert_cache_learn_pins",
                     _sigs().expert_cache_learn_pins(self.handle, layer, a, n_pin, _cstream(stream)))
 
@@ -212,3 +218,32 @@ def moe_layer_experts(d: MoeDims, T: int, table, out, ws, stream=None):
     tp = table if isinstance(table, int) else table.data_ptr()
     _chk("moe_layer_experts", _sigs().moe_layer_experts(
         ctypes.byref(d), T, ctypes.c_void_p(tp), _ptr(out), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+# ----------------------------------------------------------------- route usage on disk
+def usage_save(path, counts) -> None:
+    """Writes the route-usage record: counts [n_layers][E] of non-negative
+    selection counts (the layers' route_counts), atomically (temp + rename)."""
+    a = np.asarray(counts)
+    if a.ndim != 2 or (a.size and a.min() < 0):
+        raise ValueError("counts must be [n_layers][E] non-negative integers")
+    a = np.ascontiguousarray(a, dtype=np.uint64)
+    _chk("moe_usage_save", _sigs().moe_usage_save(
+        os.fsencode(path), a.shape[0], a.shape[1], a.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64))))
+
+
+def usage_load(path, n_layers: int, E: int, counts=None) -> np.ndarray:
+    """Reads a route-usage record [n_layers][E] (uint64).  With `counts` given
+    (a uint64 array of that shape) the file's counts are added to it in place
+    and it is returned; on any error it is left unchanged."""
+    if counts is None:
+        out = np.zeros((n_layers, E), dtype=np.uint64)
+        acc = 0
+    else:
+        out = counts
+        if out.dtype != np.uint64 or out.shape != (n_layers, E) or not out.flags.c_contiguous:
+            raise ValueError("counts must be a contiguous uint64 array [n_layers][E]")
+        acc = 1
+    _chk("moe_usage_load", _sigs().moe_usage_load(
+        os.fsencode(path), n_layers, E, out.ctypes.data_as(ctypes.POINTER(ctypes.c_uint64)), acc))
+    return out

@@ -340,6 +340,7 @@ const char *moe_status_string(int status) {
     case MOE_ERR_TIMEOUT: return "device wait timed out";
     case MOE_ERR_DEVICE: return "device-side check failed";
     case MOE_ERR_ALLOC: return "allocation failed";
+    case MOE_ERR_IO: return "file missing, unreadable or corrupt";
     default: return "unknown status";
   }
 }
