@@ -556,9 +556,9 @@ def chain_next_dev(x: torch.Tensor, out: torch.Tensor, gamma: float = 0.5, zipf:
 
 
 def run_stacked(args, ws_n, rank, local):
-    """8 stacked GLM-5.2-shaped layers resident in HBM; batches of 1, 4 and 16
-    tokens with independently drawn hidden states; per-layer us and
-    union-weighted expert GB/s."""
+    """8 stacked GLM-5.2-shaped layers resident in HBM; batches of 1, 2, 3, 4 and
+    16 tokens (2-3: draft-verification sizes) with independently drawn hidden
+    states; per-layer us and union-weighted expert GB/s."""
     import int4_routed_expert_softmax_b200 as moe
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -604,9 +604,11 @@ def run_stacked(args, ws_n, rank, local):
                 warmup=args.warmup, ms_per_step=round(tot_ms / args.steps, 4), higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="int4xint8->fp32", data="synthetic",
                 config={"workload": "stacked: 8 GLM-5.2-shaped layers resident in HBM (41.2 GB), batches of "
-                                    "1, 4, 16 tokens, layers chained", "layers": L, "T_list": list(w.T_list),
+                                    + ", ".join(str(t) for t in w.T_list) + " tokens, layers chained",
+                        "layers": L, "T_list": list(w.T_list),
                         "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)"},
-                by_batch=res, clocks=clk.summary(), gpu_launches=None)
+                by_batch=res, clocks=clk.summary(),
+                gpu_launches=3 * L * args.steps * len(w.T_list))  # decode path: 3 kernels per layer call
 
 
 def run_tiered(args, ws_n, rank, local):

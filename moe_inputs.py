@@ -69,7 +69,7 @@ WORKLOADS = {
     # one GLM-5.2-shaped layer, batch 1, all experts resident
     "decode": Workload("decode", **GLM, T=1, seed=2),
     # 8 stacked GLM-5.2-shaped layers, batch 1 / 4 / 16
-    "stacked": Workload("stacked", **GLM, T=16, layers=8, seed=3, T_list=(1, 4, 16)),
+    "stacked": Workload("stacked", **GLM, T=16, layers=8, seed=3, T_list=(1, 2, 3, 4, 16)),
     # prefill, 2048 tokens, Zipf(1.1) expert popularity
     "prefill": Workload("prefill", **GLM, T=2048, zipf_s=1.1, seed=4),
     # tiered decode: 16 layers in pinned host memory, 20 GiB HBM cache, 512 tokens

@@ -172,7 +172,7 @@ def test_layer_decode_glm_T1(seed):
     _check_layer(w, x, Wr, blobs)
 
 
-@pytest.mark.parametrize("T", [4, 16])
+@pytest.mark.parametrize("T", [2, 3, 4, 16])   # 2-3: draft-verification batch sizes
 def test_layer_stacked_batches(T):
     w = mi.WORKLOADS["stacked"]
     x, Wr, blobs = mi.make_layer(w, 3, DEV, T=T)
