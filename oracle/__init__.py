@@ -64,6 +64,15 @@ def lib() -> ctypes.CDLL:
             "or_expert_down": (None, [P, i32, i32, P, P, P]),
             "or_moe_layer": (i32, [i32, i32, i32, i32, i32, P, P, P, P, P]),
             "or_moe_layer_tokens": (i32, [i32, i32, i32, i32, P, P, P, P, i32, P]),
+            "or_e2m1_value": (f32, [i32]),
+            "or_mx_code": (i32, [P, i32, i32, i32, i32]),
+            "or_mx_scale_exp": (i32, [P, i32, i32, i32, i32]),
+            "or_mx_weight": (f32, [P, i32, i32, i32, i32]),
+            "or_mx_pack_matrix": (None, [P, P, i32, i32, P]),
+            "or_mx_block_dot": (ctypes.c_int32, [P, i32, i32, i32, i32, P]),
+            "or_mx_expert_dot": (f32, [P, i32, i32, i32, P, P]),
+            "or_mx_expert_ffn": (None, [P, i32, i32, P, P, P, P, P, P, P, P]),
+            "or_moe_layer_mx": (i32, [i32, i32, i32, i32, i32, P, P, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -184,8 +193,9 @@ def expert_dot(mat, N, K, n, q, d) -> float:
     return float(lib().or_expert_dot(_p(mat), N, K, n, _p(q), _p(d)))
 
 
-def expert_ffn(blob: np.ndarray, H: int, I: int, xq: np.ndarray, xd: np.ndarray):
-    """Returns dict g, u, h, hq, hd, y for one token."""
+def expert_ffn(blob: np.ndarray, H: int, I: int, xq: np.ndarray, xd: np.ndarray, fmt: str = "int4"):
+    """Returns dict g, u, h, hq, hd, y for one token (fmt "int4": int4 gs64
+    blob; "mxfp4": MXFP4 blob)."""
     blob = _c(blob, np.uint8)
     xq = _c(xq, np.int8)
     xd = _c(xd, np.float32)
@@ -195,7 +205,8 @@ def expert_ffn(blob: np.ndarray, H: int, I: int, xq: np.ndarray, xd: np.ndarray)
     hq = np.zeros(I, np.int8)
     hd = np.zeros(I // 32, np.float32)
     y = np.zeros(H, np.float32)
-    lib().or_expert_ffn(_p(blob), H, I, _p(xq), _p(xd), _p(g), _p(u), _p(h), _p(hq), _p(hd), _p(y))
+    fn = lib().or_mx_expert_ffn if fmt == "mxfp4" else lib().or_expert_ffn
+    fn(_p(blob), H, I, _p(xq), _p(xd), _p(g), _p(u), _p(h), _p(hq), _p(hd), _p(y))
     return dict(g=g, u=u, h=h, hq=hq, hd=hd, y=y)
 
 
@@ -207,6 +218,44 @@ def expert_down(blob: np.ndarray, H: int, I: int, hq: np.ndarray, hd: np.ndarray
     y = np.zeros(H, np.float32)
     lib().or_expert_down(_p(blob), H, I, _p(hq), _p(hd), _p(y))
     return y
+
+
+# ---------------------------------------------------------------- MXFP4 experts
+def e2m1_value(code: int) -> float:
+    return float(lib().or_e2m1_value(code))
+
+
+def mx_pack_matrix(codes: np.ndarray, exps: np.ndarray) -> np.ndarray:
+    """codes uint8 [N][K] in 0..15 (E2M1), exps uint8 [N][K/32] (E8M0)."""
+    codes = _c(codes, np.uint8)
+    exps = _c(exps, np.uint8)
+    N, K = codes.shape
+    out = np.zeros(matrix_bytes(N, K), np.uint8)
+    lib().or_mx_pack_matrix(_p(codes), _p(exps), N, K, _p(out))
+    return out
+
+
+def mx_code(mat, N, K, n, k) -> int:
+    return int(lib().or_mx_code(_p(mat), N, K, n, k))
+
+
+def mx_scale_exp(mat, N, K, n, b) -> int:
+    return int(lib().or_mx_scale_exp(_p(mat), N, K, n, b))
+
+
+def mx_weight(mat, N, K, n, k) -> float:
+    return float(lib().or_mx_weight(_p(mat), N, K, n, k))
+
+
+def mx_block_dot(mat, N, K, n, b, q) -> int:
+    q = _c(q, np.int8)
+    return int(lib().or_mx_block_dot(_p(mat), N, K, n, b, _p(q)))
+
+
+def mx_expert_dot(mat, N, K, n, q, d) -> float:
+    q = _c(q, np.int8)
+    d = _c(d, np.float32)
+    return float(lib().or_mx_expert_dot(_p(mat), N, K, n, _p(q), _p(d)))
 
 
 class _Trace(ctypes.Structure):
@@ -226,8 +275,9 @@ def _blob_ptrs(blobs):
 
 
 def moe_layer(x: np.ndarray, Wr: np.ndarray, blobs, H: int, I: int, E: int, k: int,
-              trace: bool = False):
-    """Full layer on every token.  Returns out [T][H] (and the trace dict)."""
+              trace: bool = False, fmt: str = "int4"):
+    """Full layer on every token.  Returns out [T][H] (and the trace dict).
+    fmt: "int4" (int4 gs64 blobs) or "mxfp4" (MXFP4 blobs)."""
     x = _c(x, np.float32)
     Wr = _c(Wr, np.float32)
     T = x.shape[0]
@@ -245,8 +295,8 @@ def moe_layer(x: np.ndarray, Wr: np.ndarray, blobs, H: int, I: int, E: int, k: i
             hq=np.zeros((T, k + 1, I), np.int8), hd=np.zeros((T, k + 1, I // 32), np.float32),
             y=np.zeros((T, k + 1, H), np.float32))
         tr = _Trace(**{n: a.ctypes.data for n, a in arrays.items()})
-    rc = lib().or_moe_layer(H, I, E, k, T, _p(x), _p(Wr), ptrs, _p(out),
-                            ctypes.byref(tr) if tr is not None else None)
+    fn = lib().or_moe_layer_mx if fmt == "mxfp4" else lib().or_moe_layer
+    rc = fn(H, I, E, k, T, _p(x), _p(Wr), ptrs, _p(out), ctypes.byref(tr) if tr is not None else None)
     if rc != 0:
         raise ValueError("oracle rejected the shape")
     del keep

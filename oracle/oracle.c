@@ -294,21 +294,107 @@ float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, co
   return total;
 }
 
+/* ------------------------------------------------------------------------ */
+/* MXFP4 experts (microscaled FP4): the native expert format that the        */
+/* Kimi K3 row of the tantan.ink model table streams without conversion      */
+/* ("QAT-trained MXFP4 experts").  The pages give no finer detail; the       */
+/* format is the OCP Microscaling one: blocks of 32 E2M1 elements sharing an */
+/* E8M0 scale.  Readings stated here:                                        */
+/*  - element value = e2m1(code) * 2^(E - 127); E = 255 (NaN) is outside the */
+/*    contract;                                                              */
+/*  - [N][K] matrix = N*K/2 packed bytes (two consecutive elements per byte, */
+/*    the lower-indexed one in the low nibble), then N*K/32 E8M0 bytes, one  */
+/*    per 32-block of a row -- the same byte count as the int4 gs64 layout,  */
+/*    and the same blob order gate | up | down;                              */
+/*  - activations stay Q8_0, so a block's products 2*e2m1 * q are integers   */
+/*    and its sum S_b is exact; the block term is (S_b * d_b) * 2^(E_b-128)  */
+/*    (the second factor a power of two), and the terms are summed in the    */
+/*    chunk order of the int4 layout: lane chunks of ceil(K/64/32) 64-groups,*/
+/*    two blocks per group, chunk sums left to right.                        */
+/* ------------------------------------------------------------------------ */
+float or_e2m1_value(int code) {
+  int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
+  /* subnormal when the exponent field is 0: m * 2^-1; else (1 + m/2) * 2^(e-1) */
+  float mag = (e == 0) ? 0.5f * (float)m : (1.0f + 0.5f * (float)m) * pow2i(e - 1);
+  return sign ? -mag : mag;
+}
+
+int or_mx_code(const uint8_t *mat, int N, int K, int n, int k) {
+  (void)N;
+  uint8_t byte = mat[(size_t)n * (size_t)(K / 2) + (size_t)(k / 2)];
+  return (k & 1) ? (byte >> 4) : (byte & 15);
+}
+
+int or_mx_scale_exp(const uint8_t *mat, int N, int K, int n, int b) {
+  return mat[(size_t)N * (size_t)(K / 2) + (size_t)n * (size_t)(K / 32) + (size_t)b];
+}
+
+/* 2^k for any k in [-149, 127], exact (a subnormal power of two below -126). */
+static float pow2_any(int k) { return ldexpf(1.0f, k); }
+
+float or_mx_weight(const uint8_t *mat, int N, int K, int n, int k) {
+  return or_e2m1_value(or_mx_code(mat, N, K, n, k)) * pow2_any(or_mx_scale_exp(mat, N, K, n, k / 32) - 127);
+}
+
+void or_mx_pack_matrix(const uint8_t *codes, const uint8_t *exps, int N, int K, uint8_t *mat) {
+  for (int n = 0; n < N; ++n)
+    for (int j = 0; j < K / 2; ++j) {
+      uint8_t lo = codes[(size_t)n * K + 2 * j] & 15, hi = codes[(size_t)n * K + 2 * j + 1] & 15;
+      mat[(size_t)n * (K / 2) + j] = (uint8_t)(lo | (hi << 4));
+    }
+  memcpy(mat + (size_t)N * (K / 2), exps, (size_t)N * (size_t)(K / 32));
+}
+
+int32_t or_mx_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q) {
+  int32_t s = 0;
+  for (int i = 0; i < 32; ++i) {
+    int k = 32 * b + i;
+    /* 2 * e2m1 is an integer in [-12, 12] */
+    int32_t c2 = (int32_t)(2.0f * or_e2m1_value(or_mx_code(mat, N, K, n, k)));
+    s += c2 * (int32_t)q[k];
+  }
+  return s;
+}
+
+float or_mx_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {
+  int G = K / 64;
+  int csz = (G + 31) / 32;
+  int nch = (G + csz - 1) / csz;
+  float total = 0.0f;
+  for (int c = 0; c < nch; ++c) {
+    float acc = 0.0f;
+    int g1 = (c + 1) * csz < G ? (c + 1) * csz : G;
+    for (int b = 2 * c * csz; b < 2 * g1; ++b) {
+      int32_t sb = or_mx_block_dot(mat, N, K, n, b, q);
+      float t = ((float)sb * d[b]) * pow2_any(or_mx_scale_exp(mat, N, K, n, b) - 128);
+      acc = acc + t;
+    }
+    total = (c == 0) ? acc : total + acc;
+  }
+  return total;
+}
+
 void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y) {
   const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
   for (int m = 0; m < H; ++m) y[m] = or_expert_dot(down, H, I, m, hq, hd);
 }
 
-void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
-                   float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
+/* Row n of an [N][K] matrix of weight format fmt (OR_FMT_INT4_GS64 or
+ * OR_FMT_MXFP4) against the Q8_0 vector (q, d). */
+static float fmt_dot(int fmt, const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {
+  return fmt == OR_FMT_MXFP4 ? or_mx_expert_dot(mat, N, K, n, q, d) : or_expert_dot(mat, N, K, n, q, d);
+}
+
+static void expert_ffn_fmt(int fmt, const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
+                           float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
   const uint8_t *gate = blob;
-  const uint8_t *up = blob + or_matrix_bytes(I, H);
+  const uint8_t *up = blob + or_matrix_bytes(I, H);  /* both formats: N*K/2 + N*K/32 bytes */
   float *hh = (float *)malloc(sizeof(float) * (size_t)I);
   int8_t *q = (int8_t *)malloc((size_t)I);
   float *dd = (float *)malloc(sizeof(float) * (size_t)(I / 32));
   for (int n = 0; n < I; ++n) {
-    float gv = or_expert_dot(gate, I, H, n, xq, xd);
-    float uv = or_expert_dot(up, I, H, n, xq, xd);
+    float gv = fmt_dot(fmt, gate, I, H, n, xq, xd);
+    float uv = fmt_dot(fmt, up, I, H, n, xq, xd);
     if (g) g[n] = gv;
     if (u) u[n] = uv;
     hh[n] = or_silu(gv) * uv;
@@ -317,10 +403,23 @@ void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const fl
   if (h) memcpy(h, hh, sizeof(float) * (size_t)I);
   if (hq) memcpy(hq, q, (size_t)I);
   if (hd) memcpy(hd, dd, sizeof(float) * (size_t)(I / 32));
-  if (y) or_expert_down(blob, H, I, q, dd, y);
+  if (y) {
+    const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
+    for (int m = 0; m < H; ++m) y[m] = fmt_dot(fmt, down, H, I, m, q, dd);
+  }
   free(dd);
   free(q);
   free(hh);
+}
+
+void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
+                   float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
+  expert_ffn_fmt(OR_FMT_INT4_GS64, blob, H, I, xq, xd, g, u, h, hq, hd, y);
+}
+
+void or_mx_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
+                      float *g, float *u, float *h, int8_t *hq, float *hd, float *y) {
+  expert_ffn_fmt(OR_FMT_MXFP4, blob, H, I, xq, xd, g, u, h, hq, hd, y);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -335,7 +434,7 @@ static int dims_ok(int H, int I, int E, int k) {
   return H > 0 && I > 0 && H % 128 == 0 && I % 128 == 0 && E >= 1 && k >= 1 && k <= E;
 }
 
-static void token_forward(int H, int I, int E, int k, const float *xt, const float *Wr,
+static void token_forward(int fmt, int H, int I, int E, int k, const float *xt, const float *Wr,
                           const uint8_t *const *blobs, float *out, int8_t *xq_o, float *xd_o,
                           float *logit_o, int32_t *idx_o, float *w_o, int8_t *hq_o,
                           float *hd_o, float *y_o) {
@@ -349,13 +448,13 @@ static void token_forward(int H, int I, int E, int k, const float *xt, const flo
   or_router_logits(xt, Wr, 1, H, E, lg);
   or_topk_softmax(lg, 1, E, k, idx, w);
   /* shared expert first (slot k in the trace) */
-  or_expert_ffn(blobs[E], H, I, xq, xd, NULL, NULL, NULL, hq_o ? hq_o + (size_t)k * I : NULL,
-                hd_o ? hd_o + (size_t)k * (I / 32) : NULL, y);
+  expert_ffn_fmt(fmt, blobs[E], H, I, xq, xd, NULL, NULL, NULL, hq_o ? hq_o + (size_t)k * I : NULL,
+                 hd_o ? hd_o + (size_t)k * (I / 32) : NULL, y);
   if (y_o) memcpy(y_o + (size_t)k * H, y, sizeof(float) * (size_t)H);
   memcpy(out, y, sizeof(float) * (size_t)H);
   for (int s = 0; s < k; ++s) {
-    or_expert_ffn(blobs[idx[s]], H, I, xq, xd, NULL, NULL, NULL, hq_o ? hq_o + (size_t)s * I : NULL,
-                  hd_o ? hd_o + (size_t)s * (I / 32) : NULL, y);
+    expert_ffn_fmt(fmt, blobs[idx[s]], H, I, xq, xd, NULL, NULL, NULL,
+                   hq_o ? hq_o + (size_t)s * I : NULL, hd_o ? hd_o + (size_t)s * (I / 32) : NULL, y);
     if (y_o) memcpy(y_o + (size_t)s * H, y, sizeof(float) * (size_t)H);
     for (int m = 0; m < H; ++m) out[m] = fmaf(w[s], y[m], out[m]);
   }
@@ -372,13 +471,13 @@ static void token_forward(int H, int I, int E, int k, const float *xt, const flo
   free(xq);
 }
 
-int or_moe_layer(int H, int I, int E, int k, int T, const float *x, const float *Wr,
-                 const uint8_t *const *blobs, float *out, or_layer_trace *tr) {
+static int layer_fmt(int fmt, int H, int I, int E, int k, int T, const float *x, const float *Wr,
+                     const uint8_t *const *blobs, float *out, or_layer_trace *tr) {
   if (!dims_ok(H, I, E, k) || T < 0) return -1;
   int32_t *idx_all = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T * k : 1));
   for (int t = 0; t < T; ++t) {
     size_t tk = (size_t)t * (size_t)(k + 1);
-    token_forward(H, I, E, k, x + (size_t)t * H, Wr, blobs, out + (size_t)t * H,
+    token_forward(fmt, H, I, E, k, x + (size_t)t * H, Wr, blobs, out + (size_t)t * H,
                   tr && tr->xq ? tr->xq + (size_t)t * H : NULL,
                   tr && tr->xd ? tr->xd + (size_t)t * (H / 32) : NULL,
                   tr && tr->logits ? tr->logits + (size_t)t * E : NULL, idx_all + (size_t)t * k,
@@ -394,12 +493,22 @@ int or_moe_layer(int H, int I, int E, int k, int T, const float *x, const float 
   return 0;
 }
 
+int or_moe_layer(int H, int I, int E, int k, int T, const float *x, const float *Wr,
+                 const uint8_t *const *blobs, float *out, or_layer_trace *tr) {
+  return layer_fmt(OR_FMT_INT4_GS64, H, I, E, k, T, x, Wr, blobs, out, tr);
+}
+
+int or_moe_layer_mx(int H, int I, int E, int k, int T, const float *x, const float *Wr,
+                    const uint8_t *const *blobs, float *out, or_layer_trace *tr) {
+  return layer_fmt(OR_FMT_MXFP4, H, I, E, k, T, x, Wr, blobs, out, tr);
+}
+
 int or_moe_layer_tokens(int H, int I, int E, int k, const float *x, const float *Wr,
                         const uint8_t *const *blobs, const int32_t *tok, int n_tok,
                         float *out) {
   if (!dims_ok(H, I, E, k) || n_tok < 0) return -1;
   for (int i = 0; i < n_tok; ++i)
-    token_forward(H, I, E, k, x + (size_t)tok[i] * H, Wr, blobs, out + (size_t)i * H, NULL,
+    token_forward(OR_FMT_INT4_GS64, H, I, E, k, x + (size_t)tok[i] * H, Wr, blobs, out + (size_t)i * H, NULL,
                   NULL, NULL, NULL, NULL, NULL, NULL, NULL);
   return 0;
 }

@@ -90,6 +90,27 @@ void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const f
 void or_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
                    float *g, float *u, float *h, int8_t *hq, float *hd, float *y);
 
+/* ---- MXFP4 experts (microscaled FP4: 32 E2M1 elements per E8M0 scale).
+ * Matrix [N][K]: N*K/2 bytes, two consecutive elements per byte (lower index
+ * in the low nibble), then N*K/32 E8M0 exponent bytes; value = e2m1(code) *
+ * 2^(E-127).  Blob = gate | up | down as for int4 gs64, same byte count. */
+#define OR_FMT_INT4_GS64 0
+#define OR_FMT_MXFP4 1
+/* E2M1 value of a 4-bit code (sign, 2 exponent bits with bias 1, 1 mantissa bit). */
+float or_e2m1_value(int code);
+int or_mx_code(const uint8_t *mat, int N, int K, int n, int k);
+int or_mx_scale_exp(const uint8_t *mat, int N, int K, int n, int b);
+float or_mx_weight(const uint8_t *mat, int N, int K, int n, int k);
+/* codes[N][K] (0..15), exps[N][K/32] -> packed matrix. */
+void or_mx_pack_matrix(const uint8_t *codes, const uint8_t *exps, int N, int K, uint8_t *mat);
+/* Exact int32 sum over block b of row n: sum 2*e2m1(code) * q. */
+int32_t or_mx_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q);
+/* Row n against the Q8_0 vector: block terms (S_b * d_b) * 2^(E_b - 128) summed
+ * in the chunk order of or_expert_dot. */
+float or_mx_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d);
+void or_mx_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
+                      float *g, float *u, float *h, int8_t *hq, float *hd, float *y);
+
 /* Intermediates of a full layer call (all optional, NULL to skip). */
 typedef struct or_layer_trace {
   int8_t *xq;      /* [T][H]      */
@@ -111,6 +132,11 @@ typedef struct or_layer_trace {
  * shared expert.  Returns 0, or -1 on a shape it does not accept. */
 int or_moe_layer(int H, int I, int E, int k, int T, const float *x, const float *Wr,
                  const uint8_t *const *blobs, float *out, or_layer_trace *trace);
+
+/* The whole layer with MXFP4 expert blobs (routing, SwiGLU, Q8_0 of h and the
+ * combine exactly as or_moe_layer). */
+int or_moe_layer_mx(int H, int I, int E, int k, int T, const float *x, const float *Wr,
+                    const uint8_t *const *blobs, float *out, or_layer_trace *trace);
 
 /* Token subset variant: only rows tok[0..n_tok) of x are evaluated; out is
  * [n_tok][H].  Used to time and check a bounded sample of a large batch
