@@ -105,6 +105,35 @@ def fill_blob(out: torch.Tensor, H: int, I: int, seed: int) -> torch.Tensor:
     return out
 
 
+def fill_blob_mx(out: torch.Tensor, H: int, I: int, seed: int) -> torch.Tensor:
+    """Fill one MXFP4 expert blob in place from its own seed: random bytes for the
+    packed E2M1 codes (every 4-bit code is a valid value), and per 32-block an
+    E8M0 exponent E = 127 + round(log2(8 s / 6)) with s drawn like the int4
+    scales (exp(N(ln 0.02, 0.3))), so the largest weight 6 * 2^(E-127) is near
+    the int4 workload's 8 s."""
+    assert out.numel() == expert_bytes(H, I) and out.dtype == torch.uint8
+    dev = out.device
+    g = _gen(seed, dev)
+    out.random_(0, 256, generator=g)
+    mg = matrix_bytes(I, H)
+    for base, N, K in ((0, I, H), (mg, I, H), (2 * mg, H, I)):
+        e0 = base + N * (K // 2)
+        cnt = N * (K // 32)
+        z = torch.randn(cnt, generator=g, device=dev, dtype=torch.float32)
+        s = torch.exp(z * 0.3 + math.log(0.02))
+        e = 127 + torch.round(torch.log2(s * (8.0 / 6.0)))
+        out[e0:e0 + cnt] = e.clamp(0, 254).to(torch.uint8)
+    return out
+
+
+def make_blobs_mx(H: int, I: int, n: int, seed: int, device="cpu") -> torch.Tensor:
+    """MXFP4 expert blobs [n][expert_bytes], blob e from its own seed."""
+    out = torch.zeros((n, expert_bytes(H, I)), dtype=torch.uint8, device=device)
+    for e in range(n):
+        fill_blob_mx(out[e], H, I, blob_seed(seed, e))
+    return out
+
+
 def blob_seed(seed: int, e: int) -> int:
     return (seed * 7919 + e * 104_729 + 13) & 0x7FFF_FFFF
 

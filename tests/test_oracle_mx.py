@@ -172,3 +172,19 @@ def test_layer_vs_float64_and_int4_routing():
             return Wd @ (hq.astype(np.float64) * np.repeat(hd.astype(np.float64), 32))
         ref[t] = ffn(E) + sum(float(tr["w"][t, s]) * ffn(int(tr["idx"][t, s])) for s in range(k))
     assert np.linalg.norm(out - ref) / np.linalg.norm(ref) < 1e-3
+
+
+def test_seeded_mx_blobs_feed_the_layer():
+    """The seeded MXFP4 workload blobs: exponents in range, weights of the int4
+    workload's magnitude, and a finite layer output."""
+    import moe_inputs as mi
+    H, I, E, k, T = 256, 128, 4, 2, 2
+    blobs = mi.make_blobs_mx(H, I, E + 1, 11).numpy()
+    assert np.array_equal(blobs, mi.make_blobs_mx(H, I, E + 1, 11).numpy())     # seeded
+    N, K = I, H
+    ex = np.array([orc.mx_scale_exp(blobs[0], N, K, n, b) for n in range(N) for b in range(K // 32)])
+    assert ex.min() >= 115 and ex.max() <= 127
+    x = rng.normal(size=(T, H)).astype(np.float32)
+    Wr = (rng.normal(size=(E, H)) * 0.02).astype(np.float32)
+    out = orc.moe_layer(x, Wr, blobs, H, I, E, k, fmt="mxfp4")
+    assert np.all(np.isfinite(out)) and np.abs(out).max() > 0
