@@ -311,7 +311,8 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
   unsigned char *raw = smem + L.raw;
 
   prof_start(a.prof, MODE + 1);
-  if (*reinterpret_cast<volatile int32_t *>(a.status) != 0) return;
+  // one decision for the whole CTA: no barrier below may miss a thread
+  if (__syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   const int n_uni = min(max(*a.n_uni, 0), a.E);
   const int nslot = n_uni + 1;
 
