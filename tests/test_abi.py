@@ -22,7 +22,8 @@ def lib():
 def declared_functions():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\**\s*(moe_\w+)\s*\(", src, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\s*\**\s*((?:moe|expert_cache)_\w+)\s*\(",
+                                 src, flags=re.M)))
 
 
 def test_header_declares_the_entry_points():
@@ -93,3 +94,37 @@ def test_oracle_is_separate_from_the_product():
             if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
                 txt = open(os.path.join(dirpath, f), encoding="utf-8").read()
                 assert "import oracle" not in txt and "oracle.h" not in txt and "liboracle" not in txt, f
+
+
+def test_header_is_c99_and_host_calls_work_from_c(lib, tmp_path):
+    """The boundary is a C ABI: a C99 program (-Wall -Wextra -Werror -pedantic)
+    includes moe.h, links libmoe.so and runs the host-only calls (status names,
+    shape checks, sizes, the route-usage record) without a GPU."""
+    src = tmp_path / "abi.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+int main(void) {
+  moe_dims d = {6144, 2048, 256, 8};
+  uint64_t c[2 * 4] = {1, 2, 3, 4, 5, 6, 7, (uint64_t)1 << 40}, r[2 * 4];
+  if (moe_check_dims(&d) != MOE_OK) return 1;
+  if (moe_expert_bytes(&d) != (size_t)20054016) return 2;
+  if (strcmp(moe_status_string(MOE_ERR_IO), "unknown status") == 0) return 3;
+  if (moe_usage_save(USAGE_PATH, 2, 4, c) != MOE_OK) return 4;
+  memset(r, 0, sizeof r);
+  if (moe_usage_load(USAGE_PATH, 2, 4, r, 0) != MOE_OK) return 5;
+  if (memcmp(c, r, sizeof c) != 0) return 6;
+  if (moe_usage_load(USAGE_PATH, 4, 2, r, 0) != MOE_ERR_SHAPE) return 7;
+  printf("ok\n");
+  return 0;
+}
+""")
+    exe = tmp_path / "abi"
+    libdir = os.path.dirname(lib._name)
+    cc = ["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", f"-I{os.path.join(ROOT, 'include')}",
+          f'-DUSAGE_PATH="{tmp_path / "u.bin"}"', str(src), f"-L{libdir}", "-lmoe",
+          f"-Wl,-rpath,{libdir}", "-o", str(exe)]
+    subprocess.run(cc, check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
