@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "or_mx_expert_dot": (f32, [P, i32, i32, i32, P, P]),
             "or_mx_expert_ffn": (None, [P, i32, i32, P, P, P, P, P, P, P, P]),
             "or_moe_layer_mx": (i32, [i32, i32, i32, i32, i32, P, P, P, P, P]),
+            "or_moe_layer_tokens_mx": (i32, [i32, i32, i32, i32, P, P, P, P, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -309,14 +310,17 @@ def moe_layer(x: np.ndarray, Wr: np.ndarray, blobs, H: int, I: int, E: int, k: i
     return out
 
 
-def moe_layer_tokens(x: np.ndarray, Wr: np.ndarray, blobs, H, I, E, k, tokens) -> np.ndarray:
-    """Layer output for the listed token rows only (routing is per token)."""
+def moe_layer_tokens(x: np.ndarray, Wr: np.ndarray, blobs, H, I, E, k, tokens,
+                     fmt: str = "int4") -> np.ndarray:
+    """Layer output for the listed token rows only (routing is per token);
+    fmt "int4" or "mxfp4" as in moe_layer."""
     x = _c(x, np.float32)
     Wr = _c(Wr, np.float32)
     tok = _c(tokens, np.int32)
     out = np.zeros((tok.size, H), np.float32)
     keep, ptrs = _blob_ptrs(blobs)
-    rc = lib().or_moe_layer_tokens(H, I, E, k, _p(x), _p(Wr), ptrs, _p(tok), tok.size, _p(out))
+    fn = lib().or_moe_layer_tokens_mx if fmt == "mxfp4" else lib().or_moe_layer_tokens
+    rc = fn(H, I, E, k, _p(x), _p(Wr), ptrs, _p(tok), tok.size, _p(out))
     del keep
     if rc != 0:
         raise ValueError("oracle rejected the shape")

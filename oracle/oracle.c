@@ -503,12 +503,23 @@ int or_moe_layer_mx(int H, int I, int E, int k, int T, const float *x, const flo
   return layer_fmt(OR_FMT_MXFP4, H, I, E, k, T, x, Wr, blobs, out, tr);
 }
 
+static int layer_tokens_fmt(int fmt, int H, int I, int E, int k, const float *x, const float *Wr,
+                            const uint8_t *const *blobs, const int32_t *tok, int n_tok, float *out) {
+  if (!dims_ok(H, I, E, k) || n_tok < 0) return -1;
+  for (int i = 0; i < n_tok; ++i)
+    token_forward(fmt, H, I, E, k, x + (size_t)tok[i] * H, Wr, blobs, out + (size_t)i * H, NULL,
+                  NULL, NULL, NULL, NULL, NULL, NULL, NULL);
+  return 0;
+}
+
 int or_moe_layer_tokens(int H, int I, int E, int k, const float *x, const float *Wr,
                         const uint8_t *const *blobs, const int32_t *tok, int n_tok,
                         float *out) {
-  if (!dims_ok(H, I, E, k) || n_tok < 0) return -1;
-  for (int i = 0; i < n_tok; ++i)
-    token_forward(OR_FMT_INT4_GS64, H, I, E, k, x + (size_t)tok[i] * H, Wr, blobs, out + (size_t)i * H, NULL,
-                  NULL, NULL, NULL, NULL, NULL, NULL, NULL);
-  return 0;
+  return layer_tokens_fmt(OR_FMT_INT4_GS64, H, I, E, k, x, Wr, blobs, tok, n_tok, out);
+}
+
+int or_moe_layer_tokens_mx(int H, int I, int E, int k, const float *x, const float *Wr,
+                           const uint8_t *const *blobs, const int32_t *tok, int n_tok,
+                           float *out) {
+  return layer_tokens_fmt(OR_FMT_MXFP4, H, I, E, k, x, Wr, blobs, tok, n_tok, out);
 }

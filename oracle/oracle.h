@@ -144,6 +144,10 @@ int or_moe_layer_mx(int H, int I, int E, int k, int T, const float *x, const flo
 int or_moe_layer_tokens(int H, int I, int E, int k, const float *x, const float *Wr,
                         const uint8_t *const *blobs, const int32_t *tok, int n_tok,
                         float *out);
+/* The same with MXFP4 expert blobs. */
+int or_moe_layer_tokens_mx(int H, int I, int E, int k, const float *x, const float *Wr,
+                           const uint8_t *const *blobs, const int32_t *tok, int n_tok,
+                           float *out);
 
 #ifdef __cplusplus
 }

@@ -188,3 +188,15 @@ def test_seeded_mx_blobs_feed_the_layer():
     Wr = (rng.normal(size=(E, H)) * 0.02).astype(np.float32)
     out = orc.moe_layer(x, Wr, blobs, H, I, E, k, fmt="mxfp4")
     assert np.all(np.isfinite(out)) and np.abs(out).max() > 0
+
+
+def test_token_subset_equals_full_layer_rows():
+    import moe_inputs as mi
+    H, I, E, k, T = 256, 128, 4, 2, 5
+    blobs = mi.make_blobs_mx(H, I, E + 1, 12).numpy()
+    x = rng.normal(size=(T, H)).astype(np.float32)
+    Wr = (rng.normal(size=(E, H)) * 0.02).astype(np.float32)
+    full = orc.moe_layer(x, Wr, blobs, H, I, E, k, fmt="mxfp4")
+    sub = orc.moe_layer_tokens(x, Wr, blobs, H, I, E, k, [4, 0, 2], fmt="mxfp4")
+    assert np.array_equal(sub.view(np.uint32), full[[4, 0, 2]].view(np.uint32))
+    assert not np.array_equal(full, orc.moe_layer(x, Wr, blobs, H, I, E, k))   # the format matters
