@@ -403,6 +403,19 @@ def prefill_ops(w: mi.Workload, T: int) -> float:
     return 2.0 * T * (w.k + 1) * 3 * w.H * w.I
 
 
+def attainable(ops: float, n_union: int, blob_bytes: int, hbm_gbs: float, fp16_tflops: float,
+               ms_per_layer: float) -> dict:
+    """The prefill layer's attainable floor: the slower of its expert bytes (the
+    union plus the shared expert, each read once) at the HBM copy peak and its
+    int8 operations at the int8 peak, taken as twice the fp16/bf16 peak (the
+    nominal dense ratio); and the measured layer time as a fraction of it."""
+    hbm_us = (n_union + 1) * blob_bytes / (hbm_gbs * 1e9) * 1e6
+    int8_us = ops / (2.0 * fp16_tflops * 1e12) * 1e6
+    floor = max(hbm_us, int8_us)
+    return {"floor_us": round(floor, 1), "hbm_floor_us": round(hbm_us, 1), "int8_floor_us": round(int8_us, 1),
+            "bound": "hbm" if hbm_us >= int8_us else "tensor", "frac": round(floor / (ms_per_layer * 1e3), 4)}
+
+
 def run_prefill(args, ws_n, rank, local):
     import int4_routed_expert_softmax_b200 as moe
 
@@ -500,6 +513,11 @@ def run_prefill(args, ws_n, rank, local):
     if rank == 0 and ws_n == 1 and not args.no_cpu:
         cpu = oracle_prefill_sample(w, x.cpu().numpy(), Wr.cpu().numpy(), lambda e: blobs[e].cpu().numpy(),
                                     args.cpu_seconds)
+    n_u = int(nuni_t.item())
+    cnt = moe.ws_slice(ws, view.cnt, (w.E,), torch.int32).cpu()
+    nz = cnt[cnt > 0]
+    counts = {"union": n_u, "top": int(nz.max()), "median": float(nz.float().median()), "min": int(nz.min()),
+              "rows": int(nz.sum()) + T}
     return dict(
         metric=METRIC, value=round(value, 2), unit="TOPS", n_gpus=ws_n, steps=K, warmup=args.warmup,
         ms_per_step=round(max_ms / K, 4), higher_is_better=True, scaling="weak", vs_baseline=None,
@@ -509,7 +527,8 @@ def run_prefill(args, ws_n, rank, local):
                 "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": T, "global_batch": T * ws_n,
                 "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step; "
                 "weights 5.2 GB > L2"},
-        union=int(nuni_t.item()), us_per_token_layer=round(max_ms / K / T * 1e3, 3),
+        union=n_u, routing_counts=counts, us_per_token_layer=round(max_ms / K / T * 1e3, 3),
+        attainable=attainable(ops, n_u, w.blob_bytes, peaks()[0], peak, max_ms / K),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clk.summary(),
         gpu_launches=10 * K)
 
