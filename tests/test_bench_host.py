@@ -32,3 +32,24 @@ def test_profiled_traffic_follows_the_source_hash(tmp_path, monkeypatch):
     assert bench.profiled_traffic("k_test", "k.cu") is None
     assert bench.profiled_traffic("missing", "k.cu") is None
     assert os.path.exists(str(src))
+
+
+def test_reference_arm_prints_one_line_per_workload():
+    """bench.py --impl reference (the oracle on the host cores, a bounded sample)
+    prints the contract's JSON line with the oracle as its cpu_baseline."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    for wl, unit in (("decode", "GB/s"), ("prefill", "TOPS")):
+        r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                            "--workload", wl, "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"],
+                           capture_output=True, text=True, timeout=600,
+                           env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+        assert r.returncode == 0, r.stderr[-2000:]
+        lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+        assert len(lines) == 1
+        d = json.loads(lines[0])
+        assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
+        assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+        assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
