@@ -50,9 +50,7 @@ def lib() -> ctypes.CDLL:
             "or_pack_matrix": (None, [P, P, i32, i32, P]),
             "or_half_to_float": (f32, [ctypes.c_uint16]),
             "or_quant_q8_0": (None, [P, i64, P, P]),
-            "or_expf": (f32, [f32]),
             "or_silu": (f32, [f32]),
-            "or_expf_n": (None, [P, P, i64]),
             "or_silu_n": (None, [P, P, i64]),
             "or_router_logit": (f32, [P, P, i32]),
             "or_router_logits": (None, [P, P, i32, i32, i32, P]),
@@ -133,13 +131,6 @@ def quant_q8_0(x: np.ndarray):
     d = np.zeros(x.shape[:-1] + (x.shape[-1] // 32,), np.float32)
     lib().or_quant_q8_0(_p(x), n, _p(q), _p(d))
     return q, d
-
-
-def expf(x: np.ndarray) -> np.ndarray:
-    x = _c(x, np.float32)
-    y = np.empty_like(x)
-    lib().or_expf_n(_p(x), _p(y), x.size)
-    return y
 
 
 def silu(x: np.ndarray) -> np.ndarray:

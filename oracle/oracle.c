@@ -116,52 +116,17 @@ void or_quant_q8_0(const float *x, int64_t n, int8_t *q, float *d) {
 }
 
 /* ------------------------------------------------------------------------ */
-/* exp and SiLU.                                                             */
-/* exp by the Cody-Waite method: x = k ln2 + r with k = rint(x log2 e), ln2   */
-/* split into a 16-bit head (so k*head is exact) and a tail, |r| <= ln2/2;    */
-/* exp(r) by its Taylor series to degree 7 in Horner form; then exp(x) =      */
-/* exp(r) * 2^k with one rounding.  Truncation error r^8/8! < 1e-8 relative.  */
-/* The constants are the mathematical values rounded to binary32.             */
+/* SiLU, the gate of the SwiGLU expert FFN: SiLU(g) = g / (1 + e^-g).        */
+/* e^x is the C library's expf (a library primitive; the pages fix no        */
+/* approximation of their own).                                               */
 /* ------------------------------------------------------------------------ */
-
-static float pow2i(int k) { /* 2^k for -126 <= k <= 127, exact */
-  return ldexpf(1.0f, k);
-}
-
-float or_expf(float x) {
-  if (x != x) return x;
-  if (x > 100.0f) return INFINITY;
-  if (x < -104.0f) return 0.0f;
-  const float log2e = 1.44269502162933349609375f;   /* binary32(1/ln 2) */
-  const float ln2_hi = 0.693145751953125f;          /* ln 2, 16 significant bits */
-  const float ln2_lo = 1.428606765330187045037746e-06f; /* binary32(ln 2 - ln2_hi) */
-  float kf = rintf(x * log2e);
-  int k = (int)kf;
-  float r = fmaf(-kf, ln2_hi, x);
-  r = fmaf(-kf, ln2_lo, r);
-  float p = 1.0f / 5040.0f;
-  p = fmaf(p, r, 1.0f / 720.0f);
-  p = fmaf(p, r, 1.0f / 120.0f);
-  p = fmaf(p, r, 1.0f / 24.0f);
-  p = fmaf(p, r, 1.0f / 6.0f);
-  p = fmaf(p, r, 0.5f);
-  p = fmaf(p, r, 1.0f);
-  p = fmaf(p, r, 1.0f);
-  if (k > 126) return (p * pow2i(126)) * pow2i(k - 126);
-  if (k < -126) return (p * pow2i(k + 126)) * pow2i(-126);
-  return p * pow2i(k);
-}
 
 /* SwiGLU expert FFN, SiLU(gate) * up: the experts of the models the pages run
  * (GLM-5.2 MoE layers; colibri (tantan.ink), "它的核心判断"). */
 float or_silu(float g) {
-  float e = or_expf(-g);
+  float e = expf(-g);
   float den = 1.0f + e;
   return g / den;
-}
-
-void or_expf_n(const float *x, float *y, int64_t n) {
-  for (int64_t i = 0; i < n; ++i) y[i] = or_expf(x[i]);
 }
 
 void or_silu_n(const float *x, float *y, int64_t n) {
@@ -202,7 +167,8 @@ void or_router_logits(const float *x, const float *Wr, int T, int H, int E, floa
 /* Top-k: the k largest logits, a tie going to the lower expert index, listed
  * by descending logit.  Weights: softmax over the k kept logits, i.e. the full
  * softmax renormalised over the selection:
- *   m = l[idx0]; e_s = exp(l_s - m); Z = ((e_0 + e_1) + e_2) + ...; w_s = e_s / Z. */
+ *   m = l[idx0]; e_s = expf(l_s - m) (C library); Z = ((e_0 + e_1) + e_2) + ...;
+ *   w_s = e_s / Z. */
 void or_topk_softmax(const float *logits, int T, int E, int k, int32_t *idx, float *w) {
   unsigned char *taken = (unsigned char *)malloc((size_t)E);
   float *ev = (float *)malloc(sizeof(float) * (size_t)k);
@@ -219,7 +185,7 @@ void or_topk_softmax(const float *logits, int T, int E, int k, int32_t *idx, flo
     float m = l[idx[(size_t)t * k]];
     float z = 0.0f;
     for (int s = 0; s < k; ++s) {
-      ev[s] = or_expf(l[idx[(size_t)t * k + s]] - m);
+      ev[s] = expf(l[idx[(size_t)t * k + s]] - m);
       z = (s == 0) ? ev[0] : z + ev[s];
     }
     for (int s = 0; s < k; ++s) w[(size_t)t * k + s] = ev[s] / z;
@@ -257,15 +223,12 @@ void or_bucket(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *o
 /* ------------------------------------------------------------------------ */
 /* int4 x int8 dot products (the integer kernels of the engine: Colibri       */
 /* article (alphamatch.ai), "優化整數核心").                                  */
-/* Row n of a [N][K] matrix against a Q8_0 vector (q, d):                     */
+/* Row n of a [N][K] matrix against a Q8_0 vector (q, d), the definition      */
+/* written out:                                                               */
 /*   S_b = sum over the 32 elements of block b of w*q          (exact int32) */
-/*   group g (blocks 2g, 2g+1, scale s_g):                                    */
-/*     a = float(S_2g) * d_2g;  b = fmaf(float(S_2g+1), d_2g+1, a)            */
-/*   the G = K/64 groups are cut into chunks of csz = ceil(G/32) consecutive  */
-/*   groups; inside a chunk acc = fmaf(s_g, b, acc) from 0, g ascending;      */
-/*   the chunk sums are added left to right.  (Fixed order, this library's    */
-/*   reading: the hidden state h feeds a second quantisation, so both sides   */
-/*   must produce it bit for bit.)                                            */
+/*   row value = sum over the groups g = 0 .. K/64-1, in ascending order, of  */
+/*               s_g * (S_2g * d_2g + S_2g+1 * d_2g+1)                        */
+/* in binary32 with one accumulator, each product and sum rounded once.       */
 /* ------------------------------------------------------------------------ */
 
 int32_t or_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q) {
@@ -275,31 +238,22 @@ int32_t or_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_
 }
 
 float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {
-  int G = K / 64;
-  int csz = (G + 31) / 32;
-  int nch = (G + csz - 1) / csz;
-  float total = 0.0f;
-  for (int c = 0; c < nch; ++c) {
-    float acc = 0.0f;
-    int g1 = (c + 1) * csz < G ? (c + 1) * csz : G;
-    for (int g = c * csz; g < g1; ++g) {
-      int32_t s0 = or_block_dot(mat, N, K, n, 2 * g, q);
-      int32_t s1 = or_block_dot(mat, N, K, n, 2 * g + 1, q);
-      float a = (float)s0 * d[2 * g];
-      float b = fmaf((float)s1, d[2 * g + 1], a);
-      acc = fmaf(or_scale(mat, N, K, n, g), b, acc);
-    }
-    total = (c == 0) ? acc : total + acc;
+  float acc = 0.0f;
+  for (int g = 0; g < K / 64; ++g) {
+    float s0 = (float)or_block_dot(mat, N, K, n, 2 * g, q);
+    float s1 = (float)or_block_dot(mat, N, K, n, 2 * g + 1, q);
+    float grp = s0 * d[2 * g] + s1 * d[2 * g + 1];
+    acc = acc + or_scale(mat, N, K, n, g) * grp;
   }
-  return total;
+  return acc;
 }
 
 /* ------------------------------------------------------------------------ */
-/* MXFP4 experts (microscaled FP4): the native expert format that the        */
-/* Kimi K3 row of the tantan.ink model table streams without conversion      */
-/* ("QAT-trained MXFP4 experts").  The pages give no finer detail; the       */
-/* format is the OCP Microscaling one: blocks of 32 E2M1 elements sharing an */
-/* E8M0 scale.  Readings stated here:                                        */
+/* MXFP4 experts (microscaled FP4): in the model-family table of the colibri */
+/* deep review (ai-tools-nav), the Kimi K3 row says that family's experts    */
+/* come QAT-trained in MXFP4 and are streamed as shipped, with no conversion. */
+/* The pages give no finer detail; the format is the OCP Microscaling one:   */
+/* blocks of 32 E2M1 elements sharing an E8M0 scale.  Readings stated here:  */
 /*  - element value = e2m1(code) * 2^(E - 127); E = 255 (NaN) is outside the */
 /*    contract;                                                              */
 /*  - [N][K] matrix = N*K/2 packed bytes (two consecutive elements per byte, */
@@ -308,14 +262,14 @@ float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, co
 /*    and the same blob order gate | up | down;                              */
 /*  - activations stay Q8_0, so a block's products 2*e2m1 * q are integers   */
 /*    and its sum S_b is exact; the block term is (S_b * d_b) * 2^(E_b-128)  */
-/*    (the second factor a power of two), and the terms are summed in the    */
-/*    chunk order of the int4 layout: lane chunks of ceil(K/64/32) 64-groups,*/
-/*    two blocks per group, chunk sums left to right.                        */
+/*    (the second factor a power of two), and the row value is the sum of    */
+/*    the block terms over b = 0 .. K/32-1 in ascending order, one binary32  */
+/*    accumulator.                                                           */
 /* ------------------------------------------------------------------------ */
 float or_e2m1_value(int code) {
   int sign = (code >> 3) & 1, e = (code >> 1) & 3, m = code & 1;
   /* subnormal when the exponent field is 0: m * 2^-1; else (1 + m/2) * 2^(e-1) */
-  float mag = (e == 0) ? 0.5f * (float)m : (1.0f + 0.5f * (float)m) * pow2i(e - 1);
+  float mag = (e == 0) ? 0.5f * (float)m : (1.0f + 0.5f * (float)m) * ldexpf(1.0f, e - 1);
   return sign ? -mag : mag;
 }
 
@@ -357,21 +311,13 @@ int32_t or_mx_block_dot(const uint8_t *mat, int N, int K, int n, int b, const in
 }
 
 float or_mx_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {
-  int G = K / 64;
-  int csz = (G + 31) / 32;
-  int nch = (G + csz - 1) / csz;
-  float total = 0.0f;
-  for (int c = 0; c < nch; ++c) {
-    float acc = 0.0f;
-    int g1 = (c + 1) * csz < G ? (c + 1) * csz : G;
-    for (int b = 2 * c * csz; b < 2 * g1; ++b) {
-      int32_t sb = or_mx_block_dot(mat, N, K, n, b, q);
-      float t = ((float)sb * d[b]) * pow2_any(or_mx_scale_exp(mat, N, K, n, b) - 128);
-      acc = acc + t;
-    }
-    total = (c == 0) ? acc : total + acc;
+  float acc = 0.0f;
+  for (int b = 0; b < K / 32; ++b) {
+    int32_t sb = or_mx_block_dot(mat, N, K, n, b, q);
+    float t = ((float)sb * d[b]) * pow2_any(or_mx_scale_exp(mat, N, K, n, b) - 128);
+    acc = acc + t;
   }
-  return total;
+  return acc;
 }
 
 void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y) {
@@ -425,7 +371,8 @@ void or_mx_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const
 /* ------------------------------------------------------------------------ */
 /* The layer: shared expert (part of the resident dense weights, colibri      */
 /* (tantan.ink), "它的核心判断") plus the router-weighted routed experts.      */
-/* out[t] = y_shared; then for s = 0..k-1: out = fmaf(w[t,s], y_s, out).      */
+/* out[t] = y_shared; then for s = 0..k-1: out = out + w[t,s] * y_s, each     */
+/* product and sum rounded once (the sum in slot order, shared term first).   */
 /* No residual add, no norm: the input is the already normalised hidden       */
 /* state (reading).  The shared expert has weight 1 (reading).               */
 /* ------------------------------------------------------------------------ */
@@ -456,7 +403,7 @@ static void token_forward(int fmt, int H, int I, int E, int k, const float *xt, 
     expert_ffn_fmt(fmt, blobs[idx[s]], H, I, xq, xd, NULL, NULL, NULL,
                    hq_o ? hq_o + (size_t)s * I : NULL, hd_o ? hd_o + (size_t)s * (I / 32) : NULL, y);
     if (y_o) memcpy(y_o + (size_t)s * H, y, sizeof(float) * (size_t)H);
-    for (int m = 0; m < H; ++m) out[m] = fmaf(w[s], y[m], out[m]);
+    for (int m = 0; m < H; ++m) out[m] = out[m] + w[s] * y[m];
   }
   if (xq_o) memcpy(xq_o, xq, (size_t)H);
   if (xd_o) memcpy(xd_o, xd, sizeof(float) * (size_t)(H / 32));

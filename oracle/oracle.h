@@ -22,9 +22,12 @@
  * order of every fp32 sum, the nibble layout), the choice is stated at the
  * function that makes it.
  *
- * Arithmetic is IEEE binary32 with explicit fmaf() where a fused multiply-add
- * is meant; the file is compiled with -ffp-contract=off so no other
- * contraction happens.  Integer dot products are exact (int32).
+ * Arithmetic is IEEE binary32, each operation rounded once; the file is
+ * compiled with -ffp-contract=off, so the only fused multiply-adds are the
+ * explicit fmaf() of the router's fixed order.  Sums run in the plain order of
+ * the definition (index ascending, one accumulator), not in any order a
+ * kernel chooses.  e^x is the C library's expf.  Integer dot products are
+ * exact (int32).
  *
  * Parity status: every function here is pinned by tests/test_oracle.py
  * (brute force, closed forms, exact-integer special cases, invariants, and a
@@ -58,12 +61,9 @@ float or_half_to_float(uint16_t h);
 /* Q8_0: x[n] (n % 32 == 0) -> q[n], d[n/32]. */
 void or_quant_q8_0(const float *x, int64_t n, int8_t *q, float *d);
 
-/* exp(x) by Cody-Waite reduction and a degree-7 Taylor polynomial. */
-float or_expf(float x);
-/* SiLU(g) = g / (1 + exp(-g)). */
+/* SiLU(g) = g / (1 + expf(-g)), expf from the C library. */
 float or_silu(float g);
-/* Element-wise array forms of the two above (for sweeps in the tests). */
-void or_expf_n(const float *x, float *y, int64_t n);
+/* Element-wise array form of the above (for sweeps in the tests). */
 void or_silu_n(const float *x, float *y, int64_t n);
 
 /* Router logits in the fixed order (32 strided fmaf chains, xor tree). */
@@ -78,7 +78,8 @@ void or_bucket(const int32_t *idx, int T, int k, int E, int32_t *cnt, int32_t *o
 
 /* Exact int32 dot of 32-element block b of row n with q[32b .. 32b+32). */
 int32_t or_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q);
-/* Row n of the matrix against the Q8_0 vector (q, d), in the fixed order. */
+/* Row n of the matrix against the Q8_0 vector (q, d): the sum over the groups
+ * g ascending of s_g * (S_2g d_2g + S_2g+1 d_2g+1), one binary32 accumulator. */
 float or_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d);
 
 /* The down projection of one expert from given Q8_0 codes of h:
@@ -106,7 +107,7 @@ void or_mx_pack_matrix(const uint8_t *codes, const uint8_t *exps, int N, int K, 
 /* Exact int32 sum over block b of row n: sum 2*e2m1(code) * q. */
 int32_t or_mx_block_dot(const uint8_t *mat, int N, int K, int n, int b, const int8_t *q);
 /* Row n against the Q8_0 vector: block terms (S_b * d_b) * 2^(E_b - 128) summed
- * in the chunk order of or_expert_dot. */
+ * over b ascending, one binary32 accumulator. */
 float or_mx_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d);
 void or_mx_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
                       float *g, float *u, float *h, int8_t *hq, float *hd, float *y);

@@ -1,6 +1,6 @@
 """Pins of the oracle's MXFP4 expert format (32 E2M1 codes per E8M0 exponent; the
-native expert format of the Kimi K3 row of the model table on the colibri page,
-tantan.ink) against facts that do not come from the oracle: the FP4 (E2M1) value
+expert format of the Kimi K3 row of the model-family table on the colibri deep
+review page, ai-tools-nav) against facts that do not come from the oracle: the FP4 (E2M1) value
 set, a hand-worked row (tests/golden/mxfp4_row.txt), exact-integer special
 cases, a cross-format case where int4 gs64 and MXFP4 hold the same weights, and
 float64 evaluations within a stated bound.  CPU only."""
