@@ -208,6 +208,35 @@ def aggregate(my_units: float, my_ms: float, ws: int):
 
 
 # ----------------------------------------------------------------- oracle timing
+def host_cpu() -> dict:
+    """The host the oracle baseline ran on: CPU model and logical CPU count."""
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
+def decode_config(w: mi.Workload, ws_n: int) -> dict:
+    """The decode workload's config record (the native and the reference arm print the same)."""
+    return {"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
+                        "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
+            "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T, "global_batch": w.T * ws_n,
+            "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
+            "x_pool": POOL}
+
+
+def prefill_config(w: mi.Workload, ws_n: int) -> dict:
+    return {"workload": "prefill: one GLM-5.2-shaped MoE layer, 2048 tokens, router biased to Zipf(1.1) "
+                        "expert popularity, grouped GEMM over the union",
+            "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T, "global_batch": w.T * ws_n,
+            "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step"}
+
+
 def oracle_sample(w: mi.Workload, x_pool, Wr_h, blob_fn, budget_s: float, max_tokens: int):
     """Times the CPU oracle token-layer by token-layer until the budget is spent.
     Returns (bytes, seconds, tokens)."""
@@ -375,7 +404,7 @@ def run_native(args, ws_n, rank, local):
         Wr_h = Wr.cpu().numpy()
         nb, ns, nt = oracle_sample(w, xh.reshape(POOL * T, w.H), Wr_h,
                                    lambda e: blobs[e].cpu().numpy(), args.cpu_seconds, 64)
-        cpu = {"value": round(nb / ns / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+        cpu = {"value": round(nb / ns / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", **host_cpu(),
                "us_per_token_layer": round(ns / nt * 1e6, 1),
                "sample": f"{nt} token-layers of the decode workload (pool draws 0..{nt - 1}), "
                          f"single-threaded C oracle"}
@@ -385,11 +414,7 @@ def run_native(args, ws_n, rank, local):
         metric=METRIC, value=round(value, 1), unit="GB/s", n_gpus=ws_n, steps=K, warmup=args.warmup,
         ms_per_step=round(ms_per_step, 5), higher_is_better=True, scaling="weak", vs_baseline=None,
         dtype="int4xint8->fp32", data="synthetic",
-        config={"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
-                            "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
-                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": T, "global_batch": T * ws_n,
-                "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
-                "x_pool": POOL},
+        config=decode_config(w, ws_n),
         us_per_token_layer=round(ms_per_step / T * 1e3, 2),
         union_mean=round(sum(nuni) / len(nuni), 2),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clocks,
@@ -521,12 +546,9 @@ def run_prefill(args, ws_n, rank, local):
     return dict(
         metric=METRIC, value=round(value, 2), unit="TOPS", n_gpus=ws_n, steps=K, warmup=args.warmup,
         ms_per_step=round(max_ms / K, 4), higher_is_better=True, scaling="weak", vs_baseline=None,
-        dtype="int4xint8->fp32 (exact fp16 integer operands)", data="synthetic",
-        config={"workload": "prefill: one GLM-5.2-shaped MoE layer, 2048 tokens, router biased to Zipf(1.1) "
-                            "expert popularity, grouped GEMM over the union",
-                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": T, "global_batch": T * ws_n,
-                "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step; "
-                "weights 5.2 GB > L2"},
+        dtype="int4xint8->fp32 (tensor cores: int4 weights exact in fp16 x an fp16 hi/lo split of the "
+              "dequantised int8 activations, fp32 accumulation)", data="synthetic",
+        config=prefill_config(w, ws_n),
         union=n_u, routing_counts=counts, us_per_token_layer=round(max_ms / K / T * 1e3, 3),
         attainable=attainable(ops, n_u, w.blob_bytes, peaks()[0], peak, max_ms / K),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clk.summary(),
@@ -557,7 +579,7 @@ def oracle_prefill_sample(w, x_h, Wr_h, blob_fn, budget_s: float, tokens_max: in
         if spent >= budget_s:
             break
     return {"value": round(prefill_ops(w, n) / spent / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
-            "sample": f"{n} tokens of the prefill batch (tokens 0..{n - 1}), single-threaded C oracle, "
+            **host_cpu(), "sample": f"{n} tokens of the prefill batch (tokens 0..{n - 1}), single-threaded C oracle, "
                       f"{spent:.1f} s"}
 
 
@@ -748,16 +770,14 @@ def run_reference(args, ws_n, rank):
         b, s, n = oracle_sample(w, xpool[(mi_ + i) % POOL:(mi_ + i) % POOL + 1], Wr, blob_fn, per_step, 1)
         tb, ts, tn = tb + b, ts + s, tn + n
     value = tb / ts / 1e9
-    cpu = {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+    cpu = {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle", **host_cpu(),
            "sample": f"{tn} token-layers of the decode workload, single-threaded C oracle"}
     return dict(
         impl="reference", metric=METRIC, value=round(value, 4), unit="GB/s", n_gpus=ws_n,
         steps=args.steps, warmup=args.warmup, ms_per_step=round(ts / max(1, tn) * 1e3, 3),
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="int4xint8->fp32",
         data="synthetic",
-        config={"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
-                            "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
-                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T},
+        config=decode_config(w, ws_n),
         us_per_token_layer=round(ts / max(1, tn) * 1e6, 1), cpu_baseline=cpu,
         e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 
@@ -779,15 +799,13 @@ def run_reference_prefill(args, ws_n):
     oracle_prefill_sample(w, x, Wr, blob_fn, 0.0, 1)  # warm-up: one token
     recs = [oracle_prefill_sample(w, x, Wr, blob_fn, per_step, 16) for _ in range(args.steps)]
     value = sum(r["value"] for r in recs) / len(recs)
-    cpu = {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+    cpu = {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle", **host_cpu(),
            "sample": recs[0]["sample"] + f"; {len(recs)} steps"}
     return dict(
         impl="reference", metric=METRIC, value=round(value, 6), unit="TOPS", n_gpus=ws_n, steps=args.steps,
         warmup=args.warmup, higher_is_better=True, scaling="weak", vs_baseline=None,
         dtype="int4xint8->fp32", data="synthetic",
-        config={"workload": "prefill: one GLM-5.2-shaped MoE layer, 2048 tokens, router biased to Zipf(1.1) "
-                            "expert popularity, grouped GEMM over the union",
-                "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T},
+        config=prefill_config(w, ws_n),
         cpu_baseline=cpu,
         e2e={"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 

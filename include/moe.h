@@ -135,15 +135,21 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
                int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm, void *stream);
 
 /* The whole layer on T tokens.
+ * Both paths: the Q8_0 codes of x, the router logits (canonical fixed fp32
+ * order), the top-k indices and the union (cnt, off, uni, perm) are bit-exact;
+ * the softmax weights agree with the definition within a few units in the
+ * last place (CUDA's expf); the outputs are within the layer's float
+ * tolerance of the definition (relative L2 <= 1e-4, max-abs <= 2e-3 rms), a
+ * Q8_0 code of SiLU(g)*u differing by one where h lies within rounding of a
+ * code boundary.  Each path is deterministic: the same call gives the same
+ * bits.
  * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): GEMV kernels that
- * stream each union expert's bytes once per 16 tokens, every fp32 step in the
- * layer's fixed order -- bit-identical to the CPU definition.
+ * stream each union expert's bytes once per 16 tokens, the expert sums in the
+ * kernels' own fixed fp32 order.
  * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
  * union on the tensor cores (the int4 weights, exact in fp16, times an fp16
  * hi + lo split of the dequantised Q8_0 activations, 22 significant bits;
- * fp32 accumulation; weight scales applied per group) and the combine; within
- * the layer's float tolerance of the definition, the routing (idx, w, cnt, off,
- * uni, perm) and the Q8_0 codes of x still bit-exact.  (Batched expert unions: colibri deep review
+ * fp32 accumulation; weight scales applied per group) and the combine.  (Batched expert unions: colibri deep review
  * page, technology table, row I/O 即引擎; prefill GEMM order: tantan.ink
  * page, section 我看到的几个坑.)
  * Arguments:
@@ -188,8 +194,10 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
  * MOE_STATIC_WS_BYTES (4 MiB) per GPU that loads the library, held until the
  * process exits.  Arguments as moe_layer_forward.  The call allocates
  * nothing.  Its first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current; make that first call
- * before capturing any stream into a graph.  Batches whose workspace
+ * (cudaGetSymbolAddress) with that device current and keeps it for later
+ * calls; make that first call before capturing any stream into a graph, and
+ * do not reset the device's context (cudaDeviceReset) between calls, which
+ * would leave the kept address stale.  Batches whose workspace
  * (moe_workspace_bytes) exceeds MOE_STATIC_WS_BYTES are refused with
  * MOE_ERR_WORKSPACE and a message on stderr (for H=6144, I=2048, E=256,
  * k=8 every T <= 16 fits).  All calls share the one array and each call
@@ -351,6 +359,24 @@ typedef struct moe_ws_view {
 } moe_ws_view;
 
 int moe_workspace_view(const moe_dims *dims, int32_t T_max, void *ws, moe_ws_view *view);
+
+/* Wait limit of the kernels' bounded waits, in SM clock cycles, for layer
+ * calls enqueued after this call (process-wide); cycles <= 0 restores the
+ * default (2e9, about a second).  Returns the previous limit.  Every wait of
+ * a kernel for data (an mbarrier phase: a copy landed, a stage freed, an MMA
+ * done) gives up after the limit, writes MOE_ERR_TIMEOUT and the wait's
+ * detail code to the workspace status word, and ends its role; the copies and
+ * MMAs its CTA already issued are still awaited (with the default limit)
+ * before the CTA exits, and the kernels after it in the call skip their work.
+ * The workspace, the device and later calls stay usable.  A short limit is
+ * for failure tests: it makes the waits of a healthy call run out.  (The
+ * pages' engine degrades with a warning instead of crashing when a source
+ * fails: tantan.ink page, section 我看到的几个坑.) */
+int64_t moe_set_wait_limit(int64_t cycles);
+
+/* Binary version (major * 10 + minor, e.g. 100 for sm_100a) of the kernels
+ * the current device loaded from this library, or a negative status. */
+int moe_device_binary_version(void);
 
 /* Number of streaming multiprocessors the kernels size their grids for
  * (device of the current context), or a negative status. */

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_bytes_path": (sz, [D, i32, i32]),
             "moe_workspace_view": (ctypes.c_int, [D, i32, P, ctypes.POINTER(MoeWsView)]),
             "moe_device_sms": (ctypes.c_int, []),
+            "moe_set_wait_limit": (i64, [i64]),
+            "moe_device_binary_version": (ctypes.c_int, []),
             "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
             "moe_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
             "moe_quant_q8_0": (ctypes.c_int, [P, i64, i32, P, P, P]),
@@ -147,6 +149,18 @@ def moe_workspace_bytes_path(d: MoeDims, T_max: int, path: int) -> int:
 
 def moe_device_sms() -> int:
     return int(lib().moe_device_sms())
+
+
+def moe_set_wait_limit(cycles: int) -> int:
+    """Wait limit (SM clocks) of the kernels' bounded waits for later calls;
+    cycles <= 0 restores the default.  Returns the previous limit."""
+    return int(lib().moe_set_wait_limit(int(cycles)))
+
+
+def moe_device_binary_version() -> int:
+    """SM version the current device's copy of the library's kernels was built
+    for (100 = sm_100a), or a negative status."""
+    return int(lib().moe_device_binary_version())
 
 
 def moe_profile_enable(on: bool) -> None:

@@ -1,5 +1,6 @@
 // moe_api.cu -- the C ABI of libmoe (declared in include/moe.h): argument
 // checks, workspace carving and the launch sequence of the layer.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -7,6 +8,11 @@
 #include "moe_internal.h"
 
 namespace moe {
+
+// Wait limit of the kernels' work waits (moe_set_wait_limit), process-wide.
+static std::atomic<long long> g_wait_limit{kWaitLimitCycles};
+long long wait_limit_cycles() { return g_wait_limit.load(std::memory_order_relaxed); }
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -145,6 +151,7 @@ int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const floa
   ra.epc = 2;
   ra.tt = Tc < 2 ? Tc : 2;
   ra.prof = prof;
+  ra.wait_limit = wait_limit_cycles();
   cudaError_t err = launch_route_decode(ra, s);
   if (err != cudaSuccess) return cuda_status(err);
   return MOE_OK;
@@ -175,6 +182,7 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   gateup_plan(d.H, Tc, &ga.rpm, &ga.nstage);
   ga.use_pdl = 1;
   ga.prof = prof;
+  ga.wait_limit = wait_limit_cycles();
   if (ga.nstage < 2) return MOE_ERR_SHAPE;
   cudaError_t err =
       launch_gateup_decode(ga, sms, gateup_smem_bytes(d.H, Tc, ga.rpm, ga.nstage), s);
@@ -215,6 +223,7 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   da.nstage = down_max_stages(d.H, d.I, d.k, Tc, da.rows_max, da.rs);
   da.use_pdl = 1;
   da.prof = prof;
+  da.wait_limit = wait_limit_cycles();
   da.preload = down_preload(d.I, d.k, Tc);
   if (da.nstage < 2) return MOE_ERR_SHAPE;
   err = launch_down_decode(
@@ -286,6 +295,7 @@ int prefill_forward(const moe_dims &d, int T, const float *x, const float *Wr,
   pa.y = at<float>(ws, L.y);
   pa.status = status;
   pa.prof = prof;
+  pa.wait_limit = wait_limit_cycles();
   const size_t P = (size_t)T * (size_t)(d.k + 1);
   pa.maps = at<CUtensorMap>(ws, L.maps);
   CUtensorMap map_x, map_h, tmpl_gu, tmpl_dn;
@@ -368,8 +378,9 @@ size_t moe_workspace_bytes_path(const moe_dims *dims, int32_t T_max, int32_t pat
 int moe_workspace_view(const moe_dims *dims, int32_t T, void *ws, moe_ws_view *v) {
   if (moe_check_dims(dims) != MOE_OK) return MOE_ERR_SHAPE;
   if (ws == nullptr || v == nullptr || T < 0) return MOE_ERR_BAD_ARG;
-  const int Tl = T > kDecodeTMax ? T : T;
-  const WsLayout L = ws_layout(*dims, Tl);
+  // every field of the view lies before the prefill-only segments of the
+  // layout, so the decode layout gives the same offsets on either path
+  const WsLayout L = ws_layout(*dims, T);
   v->status = at<int32_t>(ws, L.status);
   v->xq = at<int8_t>(ws, L.xq);
   v->xd = at<float>(ws, L.xd);
@@ -387,6 +398,18 @@ int moe_workspace_view(const moe_dims *dims, int32_t T, void *ws, moe_ws_view *v
   v->hd = at<float>(ws, L.hd);
   v->T_max = T;
   return MOE_OK;
+}
+
+int64_t moe_set_wait_limit(int64_t cycles) {
+  const long long v = cycles > 0 ? (long long)cycles : kWaitLimitCycles;
+  return (int64_t)g_wait_limit.exchange(v);
+}
+
+int moe_device_binary_version(void) {
+  cudaFuncAttributes fa{};
+  const cudaError_t e = func_attributes(&fa);
+  if (e != cudaSuccess) return cuda_status(e);
+  return fa.binaryVersion;
 }
 
 int moe_device_sms(void) {
@@ -483,6 +506,7 @@ int moe_router_topk(const moe_dims *dims, int32_t T, const float *x, const float
   ra.tt = T < 2 ? T : 2;
   ra.done = nullptr;
   ra.status = nullptr;
+  ra.wait_limit = wait_limit_cycles();
   cudaError_t err = launch_route_decode(ra, s);
   if (err != cudaSuccess) return cuda_status(err);
   return cuda_status(launch_topk(logits, T, dims->E, dims->k, idx, w, route_counts_opt, s));

@@ -22,12 +22,14 @@
 // compile-time and every ring / unit index advances incrementally: the
 // per-stage bookkeeping is a handful of instructions.
 //
-// Fixed order of the fp32 part (the layer's definition, shared with any CPU
-// restatement): per 64-group a = S0*d0, b = fma(S1, d1, a), chunk acc =
+// Fixed order of the fp32 part (this kernel's own, so every call gives the
+// same bits): per 64-group a = S0*d0, b = fma(S1, d1, a), chunk acc =
 // fma(s_g, b, acc); lane c owns the chunk of CSZ consecutive groups; the 32
 // chunk sums are added left to right (one lane per row after a transpose in
-// shared memory).  The h codes that feed the down projection are therefore
-// identical to the oracle's bit for bit.
+// shared memory).  The definition sums the groups in plain ascending order;
+// the two orders differ by a few units in the last place of each sum, so a
+// Q8_0 code of h can differ by one where h lies that close to a rounding
+// boundary, and the outputs agree within the layer's float tolerance.
 #include "moe_device.cuh"
 
 namespace moe {
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
       const unsigned char *blob = nullptr;
       int blob_slot = -1;
       for (int j = 0; j < n_stages; ++j) {
-        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetGuEmpty)) {
+        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetGuEmpty, a.wait_limit)) {
           s_abort = 1;
           break;
         }
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
         }
       }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetGuDrain);
+        mbar_drain(full + j % NS, (j / NS) & 1, a.status, kDetGuDrain);
     }
     return;
   }
@@ -340,7 +342,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
     }
     if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
     if (!bad) {
-      bad = !mbar_wait(full + s, ph, a.status, kDetGuFull);
+      bad = !mbar_wait(full + s, ph, a.status, kDetGuFull, a.wait_limit);
       bad = __any_sync(0xffffffffu, bad);
       if (bad && lane == 0) s_abort = 1;
     }
@@ -653,7 +655,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
             bulk_g2s(act_s + bq + bd, a.hqs, bd, actbar);
           }
         }
-        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetDnEmpty)) {
+        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetDnEmpty, a.wait_limit)) {
           s_abort = 1;
           break;
         }
@@ -694,8 +696,8 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
         }
       }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
-        mbar_wait(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
-      if (a.preload && waited && !failed) mbar_wait(actbar, 0, a.status, kDetDnDrain);
+        mbar_drain(full + j % NS, (j / NS) & 1, a.status, kDetDnDrain);
+      if (a.preload && waited && !failed) mbar_drain(actbar, 0, a.status, kDetDnDrain);
     }
     return;
   }
@@ -708,7 +710,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   const int c0 = lane * CSZ;
   float *redw = red + warp * 32 * 33;
   if (a.preload && !bad) {
-    bad = !mbar_wait(actbar, 0, a.status, kDetDnFull);
+    bad = !mbar_wait(actbar, 0, a.status, kDetDnFull, a.wait_limit);
     bad = __any_sync(0xffffffffu, bad);
     if (bad && lane == 0) s_abort = 1;
   }
@@ -728,7 +730,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     }
     if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
     if (!bad) {
-      bad = !mbar_wait(full + s, ph, a.status, kDetDnFull);
+      bad = !mbar_wait(full + s, ph, a.status, kDetDnFull, a.wait_limit);
       bad = __any_sync(0xffffffffu, bad);
       if (bad && lane == 0) s_abort = 1;
     }

@@ -3,9 +3,11 @@
 // * Fixed-order fp32 arithmetic: every step whose result feeds an integer
 //   decision (router top-k, Q8_0 codes of x and of SiLU(g)*u) is written with
 //   explicit round-to-nearest intrinsics (__fmul_rn, __fadd_rn, __fmaf_rn,
-//   __fdiv_rn) so the compiler cannot contract or reorder it; the same step
-//   sequence is the layer's definition, so these values are reproducible bit
-//   for bit on any device and by a CPU restatement.
+//   __fdiv_rn) so the compiler cannot contract or reorder it.  The router's
+//   logits and the Q8_0 codes of x follow the layer's canonical order and are
+//   reproducible bit for bit by a CPU restatement; the expert sums follow the
+//   kernels' own fixed order (deterministic run to run) and agree with the
+//   plain definition within the layer's float tolerance.  e^x is CUDA's expf.
 // * TMA bulk copies (cp.async.bulk, global -> shared, completion counted on
 //   an mbarrier) and bounded mbarrier waits: a wait that runs out records an
 //   error code in the workspace status word and returns false; no kernel
@@ -31,41 +33,9 @@ __device__ __forceinline__ float fadd(float a, float b) { return __fadd_rn(a, b)
 __device__ __forceinline__ float ffma(float a, float b, float c) { return __fmaf_rn(a, b, c); }
 __device__ __forceinline__ float fdiv(float a, float b) { return __fdiv_rn(a, b); }
 
-// 2^k as a float for -126 <= k <= 127 (exact: exponent field only).
-__device__ __forceinline__ float pow2_exact(int k) { return __int_as_float((k + 127) << 23); }
-
-// exp(x): Cody-Waite argument reduction x = k*ln2 + r (ln2 split into a
-// 16-significant-bit head, so k*head is exact for |k| < 256, and a tail),
-// Taylor series of exp(r) to degree 7 evaluated by Horner's rule with fused
-// multiply-adds, then one rounding when scaling by 2^k.  Coefficients are the
-// binary32 roundings of 1/n!.  Max error about one ulp over the normal range.
-__device__ __forceinline__ float exp_cw(float x) {
-  if (x != x) return x;
-  if (x > 100.0f) return __int_as_float(0x7f800000);
-  if (x < -104.0f) return 0.0f;
-  const float kLog2e = 1.44269502162933349609375f;
-  const float kLn2Hi = 0.693145751953125f;
-  const float kLn2Lo = 1.428606765330187045037746e-06f;
-  const float kf = rintf(fmul(x, kLog2e));
-  const int k = (int)kf;
-  float r = ffma(-kf, kLn2Hi, x);
-  r = ffma(-kf, kLn2Lo, r);
-  float p = 1.0f / 5040.0f;
-  p = ffma(p, r, 1.0f / 720.0f);
-  p = ffma(p, r, 1.0f / 120.0f);
-  p = ffma(p, r, 1.0f / 24.0f);
-  p = ffma(p, r, 1.0f / 6.0f);
-  p = ffma(p, r, 0.5f);
-  p = ffma(p, r, 1.0f);
-  p = ffma(p, r, 1.0f);
-  if (k > 126) return fmul(fmul(p, pow2_exact(126)), pow2_exact(k - 126));
-  if (k < -126) return fmul(fmul(p, pow2_exact(k + 126)), pow2_exact(-126));
-  return fmul(p, pow2_exact(k));
-}
-
 // SwiGLU activation: SiLU(g) * u with SiLU(g) = g / (1 + exp(-g)).
 __device__ __forceinline__ float swiglu(float g, float u) {
-  const float e = exp_cw(-g);
+  const float e = expf(-g);
   const float den = fadd(1.0f, e);
   return fmul(fdiv(g, den), u);
 }
@@ -130,19 +100,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Bounded wait for the phase of `parity` to complete.  Gives up after
-// kWaitLimitCycles SM clocks (about a second), records `code` and returns false.
+// Bounded wait for the phase of `parity` to complete.  Gives up after `limit`
+// SM clocks (the launch's wait limit: about a second by default, shorter when
+// a caller sets one with moe_set_wait_limit), records `detail` with
+// MOE_ERR_TIMEOUT in the status word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
-                                          int32_t detail) {
+                                          int32_t detail, long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       set_status(status, MOE_ERR_TIMEOUT, detail);
       return false;
     }
   }
   return true;
+}
+
+// The same wait for the teardown of a role: the completion of copies or MMAs
+// this CTA issued itself, which must land before the CTA exits.  Always the
+// full limit (kWaitLimitCycles), whatever the launch's wait limit.
+__device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity, int32_t *status,
+                                           int32_t detail) {
+  return mbar_wait(bar, parity, status, detail, kWaitLimitCycles);
 }
 
 // 1-D bulk copy global -> shared (this CTA), completion on `bar`.

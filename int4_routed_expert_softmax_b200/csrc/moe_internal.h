@@ -12,7 +12,7 @@
 
 namespace moe {
 
-constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at 1.9 GHz
+constexpr long long kWaitLimitCycles = 2000000000LL;  // ~1 s at 1.9 GHz: default wait limit, and every drain's
 constexpr int kMaxK = 32;                              // kernels keep <= 32 slots per token
 constexpr int kDecodeTMax = MOE_DECODE_T_MAX;
 constexpr int kMaxSmem = 227 * 1024 - 1024;            // dynamic shared memory per CTA (sm_100 opt-in limit, minus static)
@@ -23,6 +23,7 @@ constexpr int kProfWords = 8;                          // per record: 4 phases x
 // Device-side error details (status[1]) -- which wait or check failed.
 enum Detail : int32_t {
   kDetRouteBar = 1,
+  kDetRouteDrain = 2,
   kDetGuFull = 10,
   kDetGuEmpty = 11,
   kDetGuDrain = 12,
@@ -38,6 +39,10 @@ enum Detail : int32_t {
   kDetPfAccFree = 34,
   kDetPfDrain = 35,
 };
+
+// The wait limit kernels launched now take for their work waits (set by
+// moe_set_wait_limit; kWaitLimitCycles by default).
+long long wait_limit_cycles();
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -127,6 +132,7 @@ struct RouteArgs {
   int epc;  // experts per CTA
   int tt;   // tokens per x tile
   unsigned long long *prof;  // profiling record or null (phase 0)
+  long long wait_limit;  // SM clocks a work wait may take (wait_limit_cycles())
 };
 
 struct BucketArgs {
@@ -149,6 +155,7 @@ struct GateUpArgs {
   int rpm;  // weight rows per matrix per stage (4 or 8)
   int use_pdl;
   unsigned long long *prof;  // profiling record or null (phase 1)
+  long long wait_limit;  // SM clocks a work wait may take (wait_limit_cycles())
 };
 
 struct DownArgs {
@@ -168,6 +175,7 @@ struct DownArgs {
   int preload;   // per-position activations kept in shared memory (small batches)
   int use_pdl;
   unsigned long long *prof;  // profiling record or null (phase 2)
+  long long wait_limit;  // SM clocks a work wait may take (wait_limit_cycles())
 };
 
 // Prefill grouped GEMM over the expert union (moe_prefill.cu).  mode 0: gate/up
@@ -183,6 +191,7 @@ struct PfArgs {
   const CUtensorMap *maps;  // [E+1][gate, up, down] tensor maps of the packed weights (device)
   int32_t *status;
   unsigned long long *prof;  // profiling record or null (phase mode + 1; k_make_maps ends phase 0)
+  long long wait_limit;  // SM clocks a work wait may take (wait_limit_cycles())
 };
 
 // The gate/up GEMM's activation rows in pair order: xg[p] = fp16 hi/lo split of
@@ -212,6 +221,9 @@ struct CombineArgs {
 
 // Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s);
+// Attributes of one of the library's kernels (binaryVersion: the SM the
+// loaded code was built for).
+cudaError_t func_attributes(cudaFuncAttributes *fa);
 // Zero ctrl_bytes (a multiple of 16) at ctrl and copy n floats (a multiple of 4)
 // from device-accessible host memory to x_dev.
 cudaError_t launch_stage_in(const float *x_host, float *x_dev, int64_t n, void *ctrl, size_t ctrl_bytes,

@@ -64,6 +64,8 @@ cudaError_t launch_stage_in(const float *x_host, float *x_dev, int64_t n, void *
   return cudaGetLastError();
 }
 
+cudaError_t func_attributes(cudaFuncAttributes *fa) { return cudaFuncGetAttributes(fa, k_quant); }
+
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s) {
   if (a.nblk == 0) return cudaSuccess;
   int64_t blocks = (a.nblk + 7) / 8;
@@ -464,7 +466,7 @@ __device__ __forceinline__ void warp_softmax_store(int t, int k, int lane, int e
                                                    int32_t *idx, float *w, int32_t *counts,
                                                    int *s_idx) {
   const float m = __shfl_sync(0xffffffffu, l_sel, 0);
-  const float ev = (lane < k) ? exp_cw(__fsub_rn(l_sel, m)) : 0.0f;
+  const float ev = (lane < k) ? expf(__fsub_rn(l_sel, m)) : 0.0f;
   float z = __shfl_sync(0xffffffffu, ev, 0);
   for (int s = 1; s < k; ++s) z = fadd(z, __shfl_sync(0xffffffffu, ev, s));
   if (lane < k) {
@@ -517,8 +519,13 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
   for (int t0 = 0; t0 < a.T; t0 += a.tt, ++phase) {
     const int nt = min(a.tt, a.T - t0);
     if (tid == 0 && t0 > 0) issue(t0);
-    const bool ok = __syncthreads_and(mbar_wait(bar, phase & 1, a.status, kDetRouteBar));
-    if (!ok) return;
+    const bool ok = __syncthreads_and(mbar_wait(bar, phase & 1, a.status, kDetRouteBar, a.wait_limit));
+    if (!ok) {
+      // the copies of this tile may still be in flight: they land in this
+      // CTA's shared memory before it exits
+      if (tid == 0) mbar_drain(bar, phase & 1, a.status, kDetRouteDrain);
+      return;
+    }
     const int npair = ne * nt;
     for (int p = warp; p < npair; p += 4) {
       const int ei = p / nt, ti = p % nt;

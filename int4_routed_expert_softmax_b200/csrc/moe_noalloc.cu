@@ -6,9 +6,10 @@
 // GPU that loads the library holds it until the process exits).  Host code
 // cannot use the array's name as a device address, so the first call on each
 // device asks the runtime for the address (cudaGetSymbolAddress) with that
-// device current and caches it; later calls reuse it.  The call itself
-// allocates nothing: it runs the same launch sequence as moe_layer_forward
-// on that workspace.
+// device current and caches it; later calls reuse it (a reset of the
+// device's context between calls would leave the cached address stale, which
+// the header tells callers not to do).  The call itself allocates nothing: it
+// runs the same launch sequence as moe_layer_forward on that workspace.
 #include <cstdio>
 #include <mutex>
 

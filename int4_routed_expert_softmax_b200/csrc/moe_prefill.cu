@@ -261,8 +261,9 @@ __device__ __forceinline__ void tmap_acquire(const CUtensorMap *m) {
 }
 
 // All lanes of the warp wait on `bar` (bounded); false when it ran out.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t det) {
-  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, det));
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, int32_t *status, int32_t det,
+                                          long long limit) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, status, det, limit));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem]^T, fp16 x fp16 -> fp32, issued by one thread.
@@ -400,7 +401,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       const CUtensorMap *m0 = nullptr, *m1 = nullptr;
       for (int j = 0; j < S && !bad; ++j, cur_next(cr)) {
         const int s = j % kPfRR;
-        if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty)) {
+        if (j >= kPfRR && !mbar_wait(rawfree + s, (uint32_t)(j / kPfRR - 1) & 1u, a.status, kDetPfEmpty, a.wait_limit)) {
           bad = true;
           break;
         }
@@ -428,7 +429,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       if (bad) *abort_flag = 1;
       // teardown: copies issued but not yet landed
       for (int j = max(0, issued - kPfRR); j < issued; ++j)
-        mbar_wait(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
+        mbar_drain(rawfull + j % kPfRR, (uint32_t)(j / kPfRR) & 1u, a.status, kDetPfDrain);
     }
     __syncwarp();
   } else if (warp == kPfActWarp) {
@@ -443,7 +444,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
         // hi/lo rows of stage j: boxes of kPfBoxRows rows; rows past the
         // tile's own land in unused B rows, rows past the array read zero
         const int sb = j % kPfRB;
-        if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty)) {
+        if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty, a.wait_limit)) {
           bad = true;
           break;
         }
@@ -460,7 +461,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       }
       if (bad) *abort_flag = 1;
       for (int j = max(0, issued - kPfRB); j < issued; ++j)
-        mbar_wait(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
+        mbar_drain(bfull + j % kPfRB, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfDrain);
     }
     __syncwarp();
   } else if (warp == kPfMmaWarp) {
@@ -474,9 +475,9 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       int done = 0;
       for (int j = 0; j < S && !bad; ++j, cur_next(cm)) {
         const int na = j % kPfNA, sb = j % kPfRB, tb = j % kPfNT;
-        if (!mbar_wait(aready + na, (uint32_t)(j / kPfNA) & 1u, a.status, kDetPfFull) ||
-            !mbar_wait(bfull + sb, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull) ||
-            (j >= kPfNT && !mbar_wait(tfree + tb, (uint32_t)(j / kPfNT - 1) & 1u, a.status, kDetPfAccFree)) ||
+        if (!mbar_wait(aready + na, (uint32_t)(j / kPfNA) & 1u, a.status, kDetPfFull, a.wait_limit) ||
+            !mbar_wait(bfull + sb, (uint32_t)(j / kPfRB) & 1u, a.status, kDetPfFull, a.wait_limit) ||
+            (j >= kPfNT && !mbar_wait(tfree + tb, (uint32_t)(j / kPfNT - 1) & 1u, a.status, kDetPfAccFree, a.wait_limit)) ||
             *abort_flag) {
           bad = true;
           break;
@@ -501,7 +502,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       if (bad) *abort_flag = 1;
       if (done > 0) {
         umma_commit(drain);
-        mbar_wait(drain, 0, a.status, kDetPfDrain);
+        mbar_drain(drain, 0, a.status, kDetPfDrain);
       }
     }
     __syncwarp();
@@ -515,8 +516,8 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
     cur_begin(cx);
     for (int i = 0; i < S && !bad; ++i, cur_next(cx)) {
       const int ra = i % kPfRR, na = i % kPfNA;
-      if (!warp_wait(rawfull + ra, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull) ||
-          (i >= kPfNA && !warp_wait(afree + na, (uint32_t)(i / kPfNA - 1) & 1u, a.status, kDetPfFull))) {
+      if (!warp_wait(rawfull + ra, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull, a.wait_limit) ||
+          (i >= kPfNA && !warp_wait(afree + na, (uint32_t)(i / kPfNA - 1) & 1u, a.status, kDetPfFull, a.wait_limit))) {
         bad = true;
         break;
       }
@@ -600,7 +601,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
           if (nt.nblk == 2) w1n = scale_at(nt, 1, 0);
         }
       }
-      if (!warp_wait(accf + tb, (uint32_t)(j / kPfNT) & 1u, a.status, kDetPfAccFull)) {
+      if (!warp_wait(accf + tb, (uint32_t)(j / kPfNT) & 1u, a.status, kDetPfAccFull, a.wait_limit)) {
         bad = true;
         break;
       }

@@ -90,3 +90,92 @@ def hq_by_slot(tr_gpu, T, k):
         hq[t, k] = tr_gpu["hq"][P + t]
         hd[t, k] = tr_gpu["hd"][P + t]
     return hq, hd
+
+
+# ----------------------------------------------------------------- layer checks
+FLIP_RATE = 1e-3   # h codes that may differ by one from the oracle's (fraction)
+W_RTOL = 1e-6      # softmax weights: CUDA's expf against the C library's
+
+
+def check_routing(g, tr):
+    """Routing against the oracle's trace: Q8_0 codes and scales of x, logits,
+    top-k indices and the union bit for bit; softmax weights within W_RTOL."""
+    assert g["status"][0] == 0, g["status"]
+    assert np.array_equal(g["xq"], tr["xq"])
+    assert np.array_equal(g["xd"].view(np.uint32), tr["xd"].view(np.uint32))
+    assert np.array_equal(g["logits"].view(np.uint32), tr["logits"].view(np.uint32))
+    assert np.array_equal(g["idx"], tr["idx"])
+    wg = g["w"].astype(np.float64)
+    wo = tr["w"].astype(np.float64)
+    assert np.all(np.abs(wg - wo) <= W_RTOL * np.abs(wo)), np.abs(wg - wo).max()
+    assert np.array_equal(g["cnt"], tr["cnt"])
+    assert np.array_equal(g["off"], tr["off"])
+    assert g["n_uni"] == tr["n_uni"] and np.array_equal(g["uni"], tr["uni"])
+    assert np.array_equal(g["perm"], tr["perm"])
+
+
+def check_hq(g, tr, T, k):
+    """h codes within one of the oracle's, at most FLIP_RATE of them differing;
+    block scales within 1e-5 relative.  Returns the number of differing codes."""
+    hq, hd = hq_by_slot(g, T, k)
+    diff = np.abs(hq.astype(np.int32) - tr["hq"].astype(np.int32))
+    assert diff.max() <= 1, diff.max()
+    assert diff.astype(bool).mean() <= FLIP_RATE, diff.astype(bool).mean()
+    ref = tr["hd"].astype(np.float64)
+    got = hd.astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 1e-5 * np.abs(ref) + 1e-30)
+    return int(diff.astype(bool).sum())
+
+
+def out_from_codes(g, tr, blobs, w, T):
+    """The oracle's down projections of the path's own h codes, combined in the
+    layer's order (float64 sums of float32 terms)."""
+    hq, hd = hq_by_slot(g, T, w.k)
+    bl = blobs.cpu().numpy() if isinstance(blobs, torch.Tensor) else np.asarray(blobs)
+    out = np.zeros((T, w.H), np.float64)
+    for t in range(T):
+        out[t] = orc.expert_down(bl[w.E], w.H, w.I, hq[t, w.k], hd[t, w.k])
+        for s in range(w.k):
+            e = int(tr["idx"][t, s])
+            out[t] += np.float64(tr["w"][t, s]) * orc.expert_down(bl[e], w.H, w.I, hq[t, s], hd[t, s])
+    return out
+
+
+def check_traced(got, ref, g, tr, blobs, w, T):
+    """A call's outputs `got` and workspace trace `g` against the oracle's
+    outputs `ref` and trace `tr` on the same inputs.  Routing bit-exact; h codes
+    within the flip bound; outputs within 1e-5 (rel-L2) of the oracle's down
+    projection of the path's own codes; and within the layer's tolerance of the
+    oracle itself wherever that tolerance covers a flip: a flipped code moves
+    every output of its token by up to 8 * s * d, which at I = 128 can reach
+    5e-3 rms (beyond the 2e-3 max-abs bound), at I >= 1024 less than half of it.
+    Returns the number of differing h codes."""
+    check_routing(g, tr)
+    flips = check_hq(g, tr, T, w.k)
+    oc = out_from_codes(g, tr, blobs, w, T)
+    nr = np.linalg.norm(oc)
+    rms = np.sqrt(np.mean(oc * oc))
+    assert np.linalg.norm(got - oc) <= 1e-5 * nr, np.linalg.norm(got - oc) / nr
+    assert np.abs(got - oc).max() <= 1e-4 * rms, np.abs(got - oc).max() / rms
+    if flips == 0 or w.I >= 1024:
+        ok, rel, mrel = within_tolerance(got, ref)
+        assert ok, (rel, mrel, flips)
+    return flips
+
+
+def check_layer(w, x, Wr, blobs, path=0):
+    """One layer call through the C ABI against the oracle (check_traced).
+    Batches over 16 tokens on the decode path keep only their last chunk in the
+    workspace: there the outputs are checked against the oracle directly.
+    Returns (out, ref, flips)."""
+    T = x.shape[0]
+    out, ws, d = gpu_layer(w, x, Wr, blobs, path=path)
+    ref, tr = oracle_layer_from_device(x, Wr, blobs, w.H, w.I, w.E, w.k)
+    got = out.cpu().numpy()
+    if T <= 16 or path == 2:
+        flips = check_traced(got, ref, ws_trace(ws, d, T), tr, blobs, w, T)
+    else:
+        flips = 0
+        ok, rel, mrel = within_tolerance(got, ref)
+        assert ok, (rel, mrel)
+    return out, ref, flips

@@ -42,11 +42,6 @@ def test_every_declared_symbol_is_exported(lib):
         getattr(lib, n)
 
 
-def test_library_is_built_for_sm100a(lib):
-    out = subprocess.run(["cuobjdump", "--list-elf", lib._name], capture_output=True, text=True).stdout
-    assert "sm_100a" in out
-
-
 def test_dims_and_sizes(lib):
     import int4_routed_expert_softmax_b200 as moe
     d = moe.dims(6144, 2048, 256, 8)

@@ -3,7 +3,8 @@ the expert union on the tensor cores, combine) with the CPU oracle, through the
 C ABI with path = MOE_PATH_PREFILL.
 
 Bit-exact: the Q8_0 codes and scales of x, the router logits, the top-k
-indices and weights, the bucket counts / offsets / union / permutation.
+indices, the bucket counts / offsets / union / permutation; the softmax weights
+within 1e-6 relative (CUDA's expf against the C library's).
 Final outputs: within rel-L2 <= 1e-4 and max-abs <= 2e-3 * rms(ref).  The
 grouped GEMM multiplies the weights by an fp16 hi/lo split of the dequantised
 activations (22 significant bits) and accumulates in fp32 in another order
@@ -17,14 +18,14 @@ import torch
 
 import moe_inputs as mi
 import oracle as orc
-from tests._common import gpu_layer, hq_by_slot, oracle_layer_from_device, within_tolerance, ws_trace
+from tests._common import (check_hq, check_layer, check_routing, gpu_layer, hq_by_slot, oracle_layer_from_device,
+                           out_from_codes, W_RTOL, within_tolerance, ws_trace)
 
 pytestmark = pytest.mark.gpu
 
 DEV = "cuda"
 PREFILL = 2
 DECODE = 1
-FLIP_RATE = 1e-3
 
 
 def _moe():
@@ -32,67 +33,8 @@ def _moe():
     return moe
 
 
-def _check_routing(g, tr):
-    assert g["status"][0] == 0, g["status"]
-    assert np.array_equal(g["xq"], tr["xq"])
-    assert np.array_equal(g["xd"].view(np.uint32), tr["xd"].view(np.uint32))
-    assert np.array_equal(g["logits"].view(np.uint32), tr["logits"].view(np.uint32))
-    assert np.array_equal(g["idx"], tr["idx"])
-    assert np.array_equal(g["w"].view(np.uint32), tr["w"].view(np.uint32))
-    assert np.array_equal(g["cnt"], tr["cnt"])
-    assert np.array_equal(g["off"], tr["off"])
-    assert g["n_uni"] == tr["n_uni"] and np.array_equal(g["uni"], tr["uni"])
-    assert np.array_equal(g["perm"], tr["perm"])
-
-
-def _check_hq(g, tr, T, k):
-    hq, hd = hq_by_slot(g, T, k)
-    diff = np.abs(hq.astype(np.int32) - tr["hq"].astype(np.int32))
-    assert diff.max() <= 1, diff.max()
-    assert diff.astype(bool).mean() <= FLIP_RATE, diff.astype(bool).mean()
-    # block scales: amax / 127 of nearly equal h
-    ref = tr["hd"].astype(np.float64)
-    got = hd.astype(np.float64)
-    assert np.all(np.abs(got - ref) <= 1e-5 * np.abs(ref) + 1e-30)
-    return int(diff.astype(bool).sum())
-
-
-def _out_from_codes(g, tr, blobs, w, T):
-    """The oracle's down projections of the path's own h codes, combined in
-    the layer's order (float64 sums of float32 terms)."""
-    hq, hd = hq_by_slot(g, T, w.k)
-    bl = blobs.cpu().numpy()
-    out = np.zeros((T, w.H), np.float64)
-    for t in range(T):
-        out[t] = orc.expert_down(bl[w.E], w.H, w.I, hq[t, w.k], hd[t, w.k])
-        for s in range(w.k):
-            e = int(tr["idx"][t, s])
-            out[t] += np.float64(tr["w"][t, s]) * orc.expert_down(bl[e], w.H, w.I, hq[t, s], hd[t, s])
-    return out
-
-
 def _check_full(w, x, Wr, blobs):
-    """Routing bit-exact; h codes within the flip bound; outputs within 1e-5 of
-    the oracle's down projection of the path's own codes; and within the layer's
-    tolerance of the oracle itself wherever that tolerance covers a flip: a
-    flipped code moves every output of its token by up to 8 * s * d, which at
-    I = 128 can reach 5e-3 rms (beyond the 2e-3 max-abs bound), at I >= 1024
-    less than half of it."""
-    T = x.shape[0]
-    out, ws, d = gpu_layer(w, x, Wr, blobs, path=PREFILL)
-    ref, tr = oracle_layer_from_device(x, Wr, blobs, w.H, w.I, w.E, w.k)
-    g = ws_trace(ws, d, T)
-    _check_routing(g, tr)
-    flips = _check_hq(g, tr, T, w.k)
-    got = out.cpu().numpy()
-    oc = _out_from_codes(g, tr, blobs, w, T)
-    nr = np.linalg.norm(oc)
-    rms = np.sqrt(np.mean(oc * oc))
-    assert np.linalg.norm(got - oc) <= 1e-5 * nr, np.linalg.norm(got - oc) / nr
-    assert np.abs(got - oc).max() <= 1e-4 * rms, np.abs(got - oc).max() / rms
-    if flips == 0 or w.I >= 1024:
-        ok, rel, mrel = within_tolerance(got, ref)
-        assert ok, (rel, mrel, flips)
+    out, ref, _ = check_layer(w, x, Wr, blobs, path=PREFILL)
     return out, ref
 
 
@@ -118,13 +60,12 @@ def test_prefill_shapes(H, I, E, k, T):
 
 
 def test_prefill_glm_T16_matches_decode_path():
-    """One 16-token batch of the GLM-shaped layer on both paths: the decode path
-    is bit-identical to the oracle, the prefill path within tolerance."""
+    """One 16-token batch of the GLM-shaped layer on both paths: each within
+    the layer's tolerance of the oracle, and of each other."""
     w = mi.WORKLOADS["stacked"]
     x, Wr, blobs = mi.make_layer(w, 1, DEV, T=16)
     out_pf, ref = _check_full(w, x, Wr, blobs)
-    out_dc, _, _ = gpu_layer(w, x, Wr, blobs, path=DECODE)
-    assert np.array_equal(out_dc.cpu().numpy().view(np.uint32), ref.view(np.uint32))
+    out_dc, _, _ = check_layer(w, x, Wr, blobs, path=DECODE)
     ok, rel, mrel = within_tolerance(out_pf.cpu().numpy(), out_dc.cpu().numpy())
     assert ok, (rel, mrel)
 
@@ -158,7 +99,7 @@ def test_prefill_glm_full_size_sampled():
     assert np.array_equal(g["logits"].view(np.uint32), lg.view(np.uint32))
     idx, wt = orc.topk_softmax(lg, w.k)
     assert np.array_equal(g["idx"], idx)
-    assert np.array_equal(g["w"].view(np.uint32), wt.view(np.uint32))
+    assert np.all(np.abs(g["w"].astype(np.float64) - wt) <= W_RTOL * np.abs(wt.astype(np.float64)))
     cnt, off, uni, n, perm = orc.bucket(idx, w.E)
     assert np.array_equal(g["cnt"], cnt) and np.array_equal(g["off"], off)
     assert g["n_uni"] == n and np.array_equal(g["uni"], uni)

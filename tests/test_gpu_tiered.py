@@ -8,7 +8,7 @@ import torch
 
 import moe_inputs as mi
 import oracle as orc
-from tests._common import within_tolerance
+from tests._common import check_traced, within_tolerance, ws_trace
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -60,8 +60,9 @@ def test_tiered_bitwise_equals_resident(per_layer):
 
 
 def test_tiered_chain_matches_oracle():
-    """Two tokens through 3 stacked layers: the oracle runs the same chain on
-    its own outputs."""
+    """Two tokens through 3 stacked layers: at every layer the oracle runs on
+    the tiered path's own input (the chain of the path's outputs), and the
+    call's routing, h codes and outputs are checked against it."""
     import int4_routed_expert_softmax_b200 as moe
     from int4_routed_expert_softmax_b200 import _cache as C
     H, I, E, k, L = 1024, 256, 64, 8, 3
@@ -76,17 +77,14 @@ def test_tiered_chain_matches_oracle():
     out = torch.empty((1, H), device=DEV)
     for t in range(2):
         xg = x0[t:t + 1]
-        xo = x0[t:t + 1]
         for l in range(L):
             cache.tiered_layer_forward(l, torch.from_numpy(xg).to(DEV), routers[l], out, ws,
                                        side_stream=side)
             torch.cuda.synchronize()
             got = out.cpu().numpy()
-            ref = orc.moe_layer(xo, Wh[l], hb[l], H, I, E, k)
-            ok, rel, mrel = within_tolerance(got, ref)
-            assert ok, (t, l, rel, mrel)
+            ref, tr = orc.moe_layer(xg, Wh[l], hb[l], H, I, E, k, trace=True)
+            check_traced(got, ref, ws_trace(ws, d, 1), tr, hb[l], w, 1)
             xg = mi.chain_next(xg, got, zipf=True)
-            xo = mi.chain_next(xo, ref, zipf=True)
     cache.close()
 
 

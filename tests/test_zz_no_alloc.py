@@ -2,9 +2,10 @@
 memory (hosts that own and budget all device memory, or paths that must not
 allocate once running).  Its workspace is a static device array inside the
 library; the test checks, through the C ABI, that two calls in a row give the
-output of moe_layer_forward with a caller workspace (within the float
-tolerance of the parity tests), and that batches too large for the static
-workspace are refused on the host.  Kept in its own file, collected last."""
+output of moe_layer_forward with a caller workspace bit for bit (both run the
+same kernels in the same order, and each kernel is deterministic), and that
+batches too large for the static workspace are refused on the host.  Kept in
+its own file, collected last."""
 import ctypes
 
 import numpy as np
@@ -33,8 +34,10 @@ def test_static_workspace_entry_matches_workspace_entry(name, T):
         out = torch.full((T, w.H), float("nan"), dtype=torch.float32, device=DEV)
         moe.moe_layer_forward_static(d, x, Wr, table, out)
         torch.cuda.synchronize()
-        ok, rel, mrel = within_tolerance(out.cpu().numpy(), ref_h)
+        got = out.cpu().numpy()
+        ok, rel, mrel = within_tolerance(got, ref_h)
         assert ok, (call, rel, mrel)
+        assert np.array_equal(got.view(np.uint32), ref_h.view(np.uint32)), call
 
 
 def test_static_workspace_refuses_oversized_batches():
