@@ -345,29 +345,57 @@ def run_native(args, ws_n, rank, local):
     value = all_bytes / (max_ms * 1e-3) / 1e9
     ms_per_step = max_ms / K
 
+    launches = moe.moe_layer_launches(d, T)
+    fused = launches == 1
+    rt_ms = sum(p[0] for p in prof)
     gu_ms = sum(p[1] for p in prof)
     dn_ms = sum(p[2] for p in prof)
-    rt_ms = sum(p[0] for p in prof)
+    call_ms = sum(p[3] for p in prof)
     gu_bytes = sum((u + 1) * gu_b for u in nuni)
     dn_bytes = sum((u + 1) * dn_b for u in nuni)
+    x_b = T * w.H * 4
     peak, peak_src = peaks()
-    gu_gbs = gu_bytes / (gu_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "k_gateup_decode", "achieved": round(gu_gbs, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(gu_gbs / peak, 4),
-                "peak_source": peak_src,
-                "traffic": profiled_traffic("k_gateup_decode_glm_T1",
-                                            "int4_routed_expert_softmax_b200/csrc/moe_decode.cu"),
-                "bytes_per_launch": round(gu_bytes / K), "us_per_launch": round(gu_ms / K * 1e3, 2)}
-    kernels = {
-        "k_route_decode": {"us": round(rt_ms / K * 1e3, 2),
-                           "GB/s": round(router_b * K / (rt_ms * 1e-3) / 1e9, 1)},
-        "k_gateup_decode": {"us": round(gu_ms / K * 1e3, 2), "GB/s": round(gu_gbs, 1)},
-        "k_down_decode": {"us": round(dn_ms / K * 1e3, 2),
-                          "GB/s": round(dn_bytes / (dn_ms * 1e-3) / 1e9, 1)},
-        "call_span": {"us": round(sum(p[3] for p in prof) / K * 1e3, 2)},
-        "timing": "device %globaltimer stamps per kernel phase (first CTA start, last CTA end); "
-                  "gate/up from its dependency wait, down from its first CTA (overlaps gate/up's tail)",
-    }
+    gbs = lambda b, ms: b / (ms * 1e-3) / 1e9
+    # the expert FFN span: from routing's end (the union known) to the last output
+    ffn_ms = call_ms - rt_ms
+    ffn = {"bytes_per_launch": round(my_bytes / K), "us": round(ffn_ms / K * 1e3, 2),
+           "achieved": round(gbs(my_bytes, ffn_ms), 1), "frac": round(gbs(my_bytes, ffn_ms) / peak, 4),
+           "what": "expert bytes ((|U|+1) blobs) / device time from the union known to the last output"}
+    if fused:
+        launch_b = my_bytes + K * (router_b + x_b)
+        roofline = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(gbs(launch_b, call_ms), 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(gbs(launch_b, call_ms) / peak, 4),
+                    "peak_source": peak_src,
+                    "traffic": profiled_traffic("k_decode_fused_glm_T1",
+                                                "int4_routed_expert_softmax_b200/csrc/moe_fused.cu"),
+                    "bytes_per_launch": round(launch_b / K), "us_per_launch": round(call_ms / K * 1e3, 2),
+                    "bytes_what": "(|U|+1) x 20,054,016 expert bytes + 6,291,456 router bytes + x",
+                    "ffn": ffn}
+        kernels = {
+            "k_decode_fused": {"us": round(call_ms / K * 1e3, 2), "GB/s": round(gbs(launch_b, call_ms), 1)},
+            "phases_us": {"routing": round(rt_ms / K * 1e3, 2), "gate_up": round(gu_ms / K * 1e3, 2),
+                          "down": round(dn_ms / K * 1e3, 2)},
+            "timing": "device %globaltimer stamps per phase of the one kernel (first CTA start, last CTA end): "
+                      "routing to the union known, gate/up stages, down stages and combine",
+        }
+    else:
+        roofline = {"bound": "hbm", "kernel": "k_gateup_decode", "achieved": round(gbs(gu_bytes, gu_ms), 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(gbs(gu_bytes, gu_ms) / peak, 4),
+                    "peak_source": peak_src,
+                    "traffic": profiled_traffic("k_gateup_decode_glm_T1",
+                                                "int4_routed_expert_softmax_b200/csrc/moe_decode.cu"),
+                    "bytes_per_launch": round(gu_bytes / K), "us_per_launch": round(gu_ms / K * 1e3, 2),
+                    "down": {"achieved": round(gbs(dn_bytes, dn_ms), 1),
+                             "frac": round(gbs(dn_bytes, dn_ms) / peak, 4)},
+                    "ffn": ffn}
+        kernels = {
+            "k_route_decode": {"us": round(rt_ms / K * 1e3, 2), "GB/s": round(gbs(router_b * K, rt_ms), 1)},
+            "k_gateup_decode": {"us": round(gu_ms / K * 1e3, 2), "GB/s": round(gbs(gu_bytes, gu_ms), 1)},
+            "k_down_decode": {"us": round(dn_ms / K * 1e3, 2), "GB/s": round(gbs(dn_bytes, dn_ms), 1)},
+            "call_span": {"us": round(call_ms / K * 1e3, 2)},
+            "timing": "device %globaltimer stamps per kernel phase (first CTA start, last CTA end); "
+                      "gate/up from its dependency wait, down from its first CTA (overlaps gate/up's tail)",
+        }
 
     # ---- end to end: host buffers through moe_layer_forward_host
     e2e = None
@@ -418,7 +446,7 @@ def run_native(args, ws_n, rank, local):
         us_per_token_layer=round(ms_per_step / T * 1e3, 2),
         union_mean=round(sum(nuni) / len(nuni), 2),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clocks,
-        gpu_launches=3 * K, wall_s=round(wall, 3))
+        gpu_launches=launches * K, wall_s=round(wall, 3))
 
 
 # ----------------------------------------------------------------- prefill

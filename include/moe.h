@@ -145,7 +145,10 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
  * bits.
  * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): GEMV kernels that
  * stream each union expert's bytes once per 16 tokens, the expert sums in the
- * kernels' own fixed fp32 order.
+ * kernels' own fixed fp32 order.  One token runs in a single cooperative
+ * kernel (routing, union, gate/up, down and combine, one CTA per SM) when the
+ * shape fits it; larger batches run three kernels per 16 tokens (routing,
+ * gate/up, down + combine).  Both give the same bits.
  * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
  * union on the tensor cores (the int4 weights, exact in fp16, times an fp16
  * hi + lo split of the dequantised Q8_0 activations, 22 significant bits;
@@ -208,6 +211,29 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
 int moe_layer_forward_static(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
                              const void *const *expert_table, float *out, int32_t *route_counts_opt,
                              int32_t path, void *stream);
+
+/* One rank's share of the layer under expert parallelism (GPU form of the
+ * pages' cluster mode, where the routed-expert FFNs run on workers: colibri
+ * deep review page, its local-cluster section).  Routing (Q8_0 of x, logits,
+ * top-k, softmax, union) covers every expert, as in moe_layer_forward, and
+ * writes the same workspace record; then only the union experts e with
+ * expert_lo <= e < expert_hi, and the shared expert if with_shared != 0, run
+ * their FFNs, and
+ *   out[t] = [with_shared: shared(x_t)] + sum over s with expert_lo <= idx[t,s] < expert_hi
+ *            of w[t,s] * expert_{idx[t,s]}(x_t),
+ * in the same order as moe_layer_forward (the terms of other ranks left out).
+ * Summing every rank's out over a partition of [0, E) with the shared expert
+ * on one rank (an all-reduce) gives the layer's output within its float
+ * tolerance.  expert_table entries outside the range (and entry E when
+ * !with_shared) are never read and may be NULL.  Always the decode path
+ * (chunks of MOE_DECODE_T_MAX tokens; one token in the fused kernel).
+ * MOE_ERR_BAD_ARG unless 0 <= expert_lo <= expert_hi <= E.  Other arguments
+ * as moe_layer_forward; workspace: moe_workspace_bytes_path(dims, T,
+ * MOE_PATH_DECODE). */
+int moe_layer_forward_ep(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                         const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                         int32_t *route_counts_opt, int32_t expert_lo, int32_t expert_hi,
+                         int32_t with_shared, void *stream);
 
 /* The layer in two halves, for callers that must place the experts between
  * routing and the FFN (the tiered cache below):
@@ -377,6 +403,12 @@ int64_t moe_set_wait_limit(int64_t cycles);
 /* Binary version (major * 10 + minor, e.g. 100 for sm_100a) of the kernels
  * the current device loaded from this library, or a negative status. */
 int moe_device_binary_version(void);
+
+/* Number of this library's kernels one moe_layer_forward call of T tokens on
+ * `path` enqueues on the current device (plus one workspace memset), or a
+ * negative status: 1 for a one-token decode call that the fused kernel runs,
+ * 3 per 16-token chunk on the three-kernel decode path, 9 on the prefill path. */
+int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path);
 
 /* Number of streaming multiprocessors the kernels size their grids for
  * (device of the current context), or a negative status. */

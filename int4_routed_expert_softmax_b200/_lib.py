@@ -57,6 +57,7 @@ def lib() -> ctypes.CDLL:
             "moe_workspace_view": (ctypes.c_int, [D, i32, P, ctypes.POINTER(MoeWsView)]),
             "moe_device_sms": (ctypes.c_int, []),
             "moe_set_wait_limit": (i64, [i64]),
+            "moe_layer_launches": (ctypes.c_int, [D, i32, i32]),
             "moe_device_binary_version": (ctypes.c_int, []),
             "moe_profile_enable": (ctypes.c_int, [ctypes.c_int]),
             "moe_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_float), ctypes.c_int]),
@@ -66,6 +67,7 @@ def lib() -> ctypes.CDLL:
             "moe_layer_forward": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
             "moe_layer_forward_host": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
             "moe_layer_forward_static": (ctypes.c_int, [D, i32, P, P, P, P, P, i32, P]),
+            "moe_layer_forward_ep": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, i32, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -155,6 +157,11 @@ def moe_set_wait_limit(cycles: int) -> int:
     """Wait limit (SM clocks) of the kernels' bounded waits for later calls;
     cycles <= 0 restores the default.  Returns the previous limit."""
     return int(lib().moe_set_wait_limit(int(cycles)))
+
+
+def moe_layer_launches(d: MoeDims, T: int, path: int = MOE_PATH_AUTO) -> int:
+    """Kernels one moe_layer_forward call of T tokens enqueues on the current device."""
+    return int(lib().moe_layer_launches(ctypes.byref(d), T, path))
 
 
 def moe_device_binary_version() -> int:

@@ -91,7 +91,7 @@ T *at(void *ws, size_t off) {
 struct ChunkPtrs {
   int8_t *xq;
   float *xd, *logits, *w;
-  int32_t *idx, *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok, *hqs, *status;
+  int32_t *idx, *cnt, *off, *uni, *n_uni, *own, *n_own, *perm, *pos, *pair_tok, *hqs, *status;
   int8_t *hq;
   float *hd;
   unsigned int *done;
@@ -109,6 +109,8 @@ ChunkPtrs chunk_ptrs(const moe_dims &d, int t0, const WsLayout &L, void *ws) {
   p.off = at<int32_t>(ws, L.off);
   p.uni = at<int32_t>(ws, L.uni);
   p.n_uni = at<int32_t>(ws, L.n_uni);
+  p.own = at<int32_t>(ws, L.own);
+  p.n_own = at<int32_t>(ws, L.n_own);
   p.perm = at<int32_t>(ws, L.perm);
   p.pos = at<int32_t>(ws, L.pos);
   p.pair_tok = at<int32_t>(ws, L.pair_tok);
@@ -120,9 +122,16 @@ ChunkPtrs chunk_ptrs(const moe_dims &d, int t0, const WsLayout &L, void *ws) {
   return p;
 }
 
+// The routed experts [lo, hi) and the shared expert (if shared) that a call
+// computes: all of them, except on one rank of an expert-parallel layer.
+struct Owned {
+  int lo, hi, shared;
+};
+Owned all_owned(const moe_dims &d) { return Owned{0, d.E, 1}; }
+
 int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
                 const float *Wr, void *ws, int32_t *counts, unsigned long long *prof,
-                cudaStream_t s) {
+                const Owned &ow, cudaStream_t s) {
   const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
   RouteArgs ra{};
   ra.H = d.H;
@@ -144,6 +153,11 @@ int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const floa
   ra.perm = p.perm;
   ra.pos = p.pos;
   ra.pair_tok = p.pair_tok;
+  ra.own = p.own;
+  ra.n_own = p.n_own;
+  ra.e_lo = ow.lo;
+  ra.e_hi = ow.hi;
+  ra.with_shared = ow.shared;
   ra.done = p.done;
   ra.status = p.status;
   ra.do_quant = 1;
@@ -158,7 +172,7 @@ int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const floa
 }
 
 int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const void *const *table,
-                  float *out, void *ws, unsigned long long *prof, cudaStream_t s) {
+                  float *out, void *ws, unsigned long long *prof, const Owned &ow, cudaStream_t s) {
   const int sms = device_sms();
   if (sms <= 0) return MOE_ERR_CUDA;
   const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
@@ -173,6 +187,8 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   ga.n_uni = p.n_uni;
   ga.off = p.off;
   ga.pair_tok = p.pair_tok;
+  ga.own = p.own;
+  ga.n_own = p.n_own;
   ga.xq = p.xq;
   ga.xd = p.xd;
   ga.hq = p.hq;
@@ -199,6 +215,12 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
   da.n_uni = p.n_uni;
   da.off = p.off;
   da.pos = p.pos;
+  da.own = p.own;
+  da.n_own = p.n_own;
+  da.idx = p.idx;
+  da.e_lo = ow.lo;
+  da.e_hi = ow.hi;
+  da.with_shared = ow.shared;
   da.w = p.w;
   da.hq = p.hq;
   da.hqs = p.hqs;
@@ -230,6 +252,80 @@ int experts_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const vo
       da, grid, down_smem_bytes(d.H, d.I, d.k, Tc, da.rows_max, da.rs, da.nstage), s);
   if (err != cudaSuccess) return cuda_status(err);
   return MOE_OK;
+}
+
+// The fused batch-1 kernel (moe_fused.cu) when the layer's shape fits it:
+// kFusedNA when it does not (the three-kernel path then runs), else a status.
+constexpr int kFusedNA = 1;
+
+// Whether the fused kernel runs this layer's one-token calls on the current
+// device (its shape fits one CTA per SM, cooperative launch available); fills
+// its plan.  Asked once per device and shape.
+bool fused_usable(const moe_dims &d, FusedArgs *fa, size_t *smem, int *grid) {
+  const int sms = device_sms();
+  if (sms <= 0) return false;
+  *fa = FusedArgs{};
+  if (!fused_plan(d.H, d.I, d.E, d.k, sms, fa, smem)) return false;
+  fa->H = d.H;
+  fa->I = d.I;
+  fa->E = d.E;
+  fa->k = d.k;
+  *grid = sms;
+  static std::mutex mu;
+  static int known[kMaxDevices] = {0};
+  static moe_dims key[kMaxDevices];
+  static bool fits[kMaxDevices] = {false};
+  const int dev = current_device();
+  if (dev < 0) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!known[dev] || key[dev].H != d.H || key[dev].I != d.I || key[dev].E != d.E || key[dev].k != d.k) {
+    int coop = 0;
+    if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
+    fits[dev] = coop && fused_ctas_per_sm(*fa, *smem) >= 1;
+    cudaGetLastError();
+    known[dev] = 1;
+    key[dev] = d;
+  }
+  return fits[dev];
+}
+
+int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
+                  const void *const *table, float *out, void *ws, int32_t *counts,
+                  unsigned long long *prof, const Owned &ow, cudaStream_t s) {
+  FusedArgs fa{};
+  size_t smem = 0;
+  int sms = 0;
+  if (!fused_usable(d, &fa, &smem, &sms)) return kFusedNA;
+  const ChunkPtrs p = chunk_ptrs(d, 0, L, ws);
+  fa.x = x;
+  fa.Wr = Wr;
+  fa.table = table;
+  fa.out = out;
+  fa.xq = p.xq;
+  fa.xd = p.xd;
+  fa.logits = p.logits;
+  fa.w = p.w;
+  fa.idx = p.idx;
+  fa.route_counts = counts;
+  fa.cnt = p.cnt;
+  fa.off = p.off;
+  fa.uni = p.uni;
+  fa.n_uni = p.n_uni;
+  fa.perm = p.perm;
+  fa.pos = p.pos;
+  fa.pair_tok = p.pair_tok;
+  fa.hq = p.hq;
+  fa.hqs = p.hqs;
+  fa.hd = p.hd;
+  fa.status = p.status;
+  fa.arrivals = at<unsigned int>(ws, L.ctrl) + 1;
+  fa.slot_done = at<int32_t>(ws, L.ctrl) + kCtrlSlot0;
+  fa.e_lo = ow.lo;
+  fa.e_hi = ow.hi;
+  fa.with_shared = ow.shared;
+  fa.wait_limit = wait_limit_cycles();
+  fa.prof = prof;
+  return cuda_status(launch_decode_fused(fa, sms, smem, s));
 }
 
 bool use_prefill(int T, int path) {
@@ -412,6 +508,21 @@ int moe_device_binary_version(void) {
   return fa.binaryVersion;
 }
 
+int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
+  if (T == 0) return 0;
+  if (use_prefill(T, path)) return 9;  // quant, router, top-k, bucket, gather, maps, 2 GEMMs, combine
+  if (T == 1) {
+    FusedArgs fa{};
+    size_t smem = 0;
+    int grid = 0;
+    if (fused_usable(*dims, &fa, &smem, &grid)) return 1;
+  }
+  return 3 * ((T + kDecodeTMax - 1) / kDecodeTMax);
+}
+
 int moe_device_sms(void) {
   const int n = device_sms();
   return n > 0 ? n : MOE_ERR_CUDA;
@@ -537,7 +648,7 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
 // status word and the router's arrival counter for this call.
 static int forward_checked(const moe_dims &d, int32_t T, const float *x, const float *Wr, const void *const *expert_table,
                     float *out, void *ws, int32_t *route_counts_opt, bool pf, const WsLayout &L, bool zeroed,
-                    cudaStream_t s) {
+                    cudaStream_t s, const Owned &ow) {
   int rc = MOE_OK;
   if (!zeroed) {
     // status word and the router's arrival counter start at zero on every call
@@ -547,11 +658,15 @@ static int forward_checked(const moe_dims &d, int32_t T, const float *x, const f
   const moe_dims *dims = &d;
   if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
   unsigned long long *prof = prof_next();
+  if (T == 1) {
+    rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
+    if (rc != kFusedNA) return rc;
+  }
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
     const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
-    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, s);
+    rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, ow, s);
     if (rc != MOE_OK) return rc;
-    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, prof, s);
+    rc = experts_chunk(*dims, t0, Tc, L, expert_table, out, ws, prof, ow, s);
     if (rc != MOE_OK) return rc;
   }
   return MOE_OK;
@@ -571,7 +686,25 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   const WsLayout L = ws_layout(*dims, T, pf);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   return forward_checked(*dims, T, x, Wr, expert_table, out, ws, route_counts_opt, pf, L, false,
-                         static_cast<cudaStream_t>(stream));
+                         static_cast<cudaStream_t>(stream), all_owned(*dims));
+}
+
+int moe_layer_forward_ep(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                         const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                         int32_t *route_counts_opt, int32_t expert_lo, int32_t expert_hi,
+                         int32_t with_shared, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0 || expert_lo < 0 || expert_hi < expert_lo || expert_hi > dims->E) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !expert_table || !out || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(out, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T, false);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  return forward_checked(*dims, T, x, Wr, expert_table, out, ws, route_counts_opt, false, L, false,
+                         static_cast<cudaStream_t>(stream),
+                         Owned{expert_lo, expert_hi, with_shared ? 1 : 0});
 }
 
 int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws,
@@ -588,7 +721,7 @@ int moe_layer_route(const moe_dims *dims, int32_t T, const float *x, const float
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
   if (err != cudaSuccess) return cuda_status(err);
-  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, prof_next(), s);
+  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, prof_next(), all_owned(*dims), s);
 }
 
 int moe_read_union(const moe_dims *dims, int32_t T, void *ws, int32_t *host_uni, int32_t *host_n,
@@ -623,7 +756,7 @@ int moe_layer_experts(const moe_dims *dims, int32_t T, const void *const *expert
   if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   const WsLayout L = ws_layout(*dims, T);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  return experts_chunk(*dims, 0, T, L, expert_table, out, ws, prof_current(),
+  return experts_chunk(*dims, 0, T, L, expert_table, out, ws, prof_current(), all_owned(*dims),
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -660,7 +793,8 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
   }
   if (err != cudaSuccess) return cuda_status(err);
   float *out_target = (out_dev_view != nullptr && aligned(out_dev_view, 16)) ? out_dev_view : yd;
-  rc = forward_checked(*dims, T, xd, Wr, expert_table, out_target, ws, route_counts_opt, pf, L, true, s);
+  rc = forward_checked(*dims, T, xd, Wr, expert_table, out_target, ws, route_counts_opt, pf, L, true, s,
+                       all_owned(*dims));
   if (rc != MOE_OK) return rc;
   if (out_target == out_dev_view) return MOE_OK;
   return cuda_status(cudaMemcpyAsync(out_host, yd, bytes, cudaMemcpyDeviceToHost, s));

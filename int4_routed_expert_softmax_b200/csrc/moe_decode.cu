@@ -30,108 +30,9 @@
 // the two orders differ by a few units in the last place of each sum, so a
 // Q8_0 code of h can differ by one where h lies that close to a rounding
 // boundary, and the outputs agree within the layer's float tolerance.
-#include "moe_device.cuh"
+#include "moe_decode.cuh"
 
 namespace moe {
-
-__host__ __device__ inline size_t al128d(size_t v) { return (v + 127) / 128 * 128; }
-
-// ---------------------------------------------------------------------------
-// Integer + fp32 dot of one lane's chunk of a weight row with one activation
-// vector.  w: packed words of the chunk's groups, act: 16 words per group
-// (elements 64g .. 64g+63), d: the two block scales per group, z: the integer
-// start values per group, -8 * (code sum of block 2g) and -128 * (code sum of
-// block 2g+1), which turn the unsigned nibble sums into exact signed sums.
-// ---------------------------------------------------------------------------
-template <int CSZ>
-__device__ __forceinline__ float chunk_dot(const uint32_t (&w)[CSZ][8], const float (&sc)[CSZ],
-                                           const uint32_t (&act)[CSZ][16], const float (&d)[CSZ][2],
-                                           const int (&z)[CSZ][2], int c0, int G) {
-  float acc = 0.0f;
-#pragma unroll
-  for (int gi = 0; gi < CSZ; ++gi) {
-    if (c0 + gi < G) {
-      int s0 = z[gi][0], s1 = z[gi][1], t0 = 0, t1 = 0;  // two chains per block
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        s0 = dp4a_us(w[gi][j] & 0x0F0F0F0Fu, act[gi][j], s0);
-        t0 = dp4a_us(w[gi][4 + j] & 0x0F0F0F0Fu, act[gi][4 + j], t0);
-        s1 = dp4a_us(w[gi][j] & 0xF0F0F0F0u, act[gi][8 + j], s1);
-        t1 = dp4a_us(w[gi][4 + j] & 0xF0F0F0F0u, act[gi][12 + j], t1);
-      }
-      s0 += t0;  // sum (u - 8) q over the low nibbles (block 2g)
-      s1 += t1;  // 16 * sum (u - 8) q over the high nibbles (block 2g+1)
-      const float fa = fmul((float)s0, d[gi][0]);
-      const float fb = ffma(fmul((float)s1, 0.0625f), d[gi][1], fa);  // (float)s1/16 is exact
-      acc = ffma(sc[gi], fb, acc);
-    }
-  }
-  return acc;
-}
-
-// Sum of the first nch of 32 chunk values, left to right (fixed order).
-__device__ __forceinline__ float chunk_sum(const float *rr, int nch) {
-  float v[32];
-#pragma unroll
-  for (int c = 0; c < 32; ++c) v[c] = (c < nch) ? rr[c] : 0.0f;
-  float tot = v[0];
-#pragma unroll
-  for (int c = 1; c < 32; ++c)
-    if (c < nch) tot = fadd(tot, v[c]);
-  return tot;
-}
-
-// Weight words and scales of one row's chunk (CSZ groups) from shared memory.
-template <int CSZ>
-__device__ __forceinline__ void load_row(const unsigned char *rowp, const __half *scp, int c0, int G,
-                                         uint32_t (&w)[CSZ][8], float (&sc)[CSZ]) {
-#pragma unroll
-  for (int gi = 0; gi < CSZ; ++gi) {
-    const int g = c0 + gi;
-    if (g < G) {
-      const uint4 w0 = *reinterpret_cast<const uint4 *>(rowp + 32 * g);
-      const uint4 w1 = *reinterpret_cast<const uint4 *>(rowp + 32 * g + 16);
-      w[gi][0] = w0.x;
-      w[gi][1] = w0.y;
-      w[gi][2] = w0.z;
-      w[gi][3] = w0.w;
-      w[gi][4] = w1.x;
-      w[gi][5] = w1.y;
-      w[gi][6] = w1.z;
-      w[gi][7] = w1.w;
-      sc[gi] = __half2float(scp[g]);
-    } else {
-#pragma unroll
-      for (int z = 0; z < 8; ++z) w[gi][z] = 0u;
-      sc[gi] = 0.0f;
-    }
-  }
-}
-
-// Activation chunk (CSZ groups) of one token: 16 words, 2 scales and the two
-// integer start values per group.
-template <int CSZ>
-__device__ __forceinline__ void load_act(const unsigned char *xa, const float *xd, const int *qs,
-                                         int c0, int G, uint32_t (&act)[CSZ][16], float (&d)[CSZ][2],
-                                         int (&z)[CSZ][2]) {
-#pragma unroll
-  for (int gi = 0; gi < CSZ; ++gi) {
-    const int g = c0 + gi;
-    const uint4 *src = reinterpret_cast<const uint4 *>(xa + 64 * gi);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint4 v = src[q];
-      act[gi][4 * q] = v.x;
-      act[gi][4 * q + 1] = v.y;
-      act[gi][4 * q + 2] = v.z;
-      act[gi][4 * q + 3] = v.w;
-    }
-    d[gi][0] = g < G ? xd[2 * g] : 0.0f;
-    d[gi][1] = g < G ? xd[2 * g + 1] : 0.0f;
-    z[gi][0] = g < G ? -8 * qs[2 * g] : 0;
-    z[gi][1] = g < G ? -128 * qs[2 * g + 1] : 0;
-  }
-}
 
 // ===========================================================================
 // gate/up
@@ -209,9 +110,9 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
   // decision for the whole CTA, so that no named barrier below misses a warp)
   if (__syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   prof_start(a.prof, 1);
-  const int n_uni = min(max(*a.n_uni, 0), a.E);
+  const int n_slots = min(max(*a.n_own, 0), a.E + 1);  // the union slots this call computes
   const int rbs = I / 32;  // 32-row units per expert
-  const int n_units = (n_uni + 1) * rbs;
+  const int n_units = n_slots * rbs;
   const int u_begin = (int)((long long)blockIdx.x * n_units / gridDim.x);
   const int u_end = (int)((long long)(blockIdx.x + 1) * n_units / gridDim.x);
   const int n_stages = (u_end - u_begin) * SPU;
@@ -222,7 +123,8 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
     bool bad = false;
     const int sl0 = u_begin / rbs, sl1 = (u_end - 1) / rbs;
     for (int sl = sl0 + tid; sl <= sl1 && u_end > u_begin; sl += blockDim.x) {
-      const int e = sl == 0 ? a.E : a.uni[sl - 1];
+      const int so = a.own[sl];
+      const int e = so == 0 ? a.E : a.uni[so - 1];
       bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
     }
     if (__syncthreads_or(bad)) {
@@ -277,7 +179,8 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
         if (*reinterpret_cast<volatile int *>(&s_abort)) break;
         if (slot != blob_slot) {
           blob_slot = slot;
-          blob = reinterpret_cast<const unsigned char *>(a.table[slot == 0 ? a.E : a.uni[slot - 1]]);
+          const int so = a.own[slot];
+          blob = reinterpret_cast<const unsigned char *>(a.table[so == 0 ? a.E : a.uni[so - 1]]);
         }
         const size_t n0 = (size_t)rb * 32 + (size_t)st * R;
         unsigned char *dst = stg + (size_t)s * pl.sb;
@@ -329,12 +232,13 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
   bool bad = false;
   for (int j = 0; j < n_stages; ++j) {
     if (st == 0) {  // a new unit: its expert's token list
-      if (slot == 0) {
+      const int so = a.own[slot];
+      if (so == 0) {
         n_tok = T;
         pos_base = T * a.k;
         my_tok = lane;
       } else {
-        const int e = a.uni[slot - 1];
+        const int e = a.uni[so - 1];
         pos_base = a.off[e];
         n_tok = a.off[e + 1] - pos_base;
         my_tok = lane < n_tok ? a.pair_tok[pos_base + lane] : 0;
@@ -606,12 +510,12 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   // tail.  The h codes (the gate/up kernel's output) are read after it.
   prof_start(a.prof, 2);
   if (__syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
-  const int n_uni = min(max(*a.n_uni, 0), a.E);
-  const int nslot = n_uni + 1;
+  const int nslot = min(max(*a.n_own, 0), a.E + 1);  // the union slots this call computes
   {
     bool bad = false;
     for (int sl = tid; sl < nslot; sl += blockDim.x) {
-      const int e = sl == 0 ? a.E : a.uni[sl - 1];
+      const int so = a.own[sl];
+      const int e = so == 0 ? a.E : a.uni[so - 1];
       bad |= (reinterpret_cast<uintptr_t>(a.table[e]) & 15u) != 0;
     }
     if (__syncthreads_or(bad)) {
@@ -663,8 +567,8 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
         const int r0 = sub * RS;
         const int nr = min(RS, nrows - r0);
         const uint32_t bytes_pk = (uint32_t)nr * (I / 2), bytes_sc = (uint32_t)nr * (I / 32);
-        const unsigned char *blob =
-            reinterpret_cast<const unsigned char *>(a.table[slot == 0 ? a.E : a.uni[slot - 1]]);
+        const int so = a.own[slot];
+        const unsigned char *blob = reinterpret_cast<const unsigned char *>(a.table[so == 0 ? a.E : a.uni[so - 1]]);
         unsigned char *dst = stg + (size_t)s * pl.sb;
         mbar_arrive_expect_tx(full + s, bytes_pk + bytes_sc);
         bulk_g2s_hint(dst, blob + pk_off + (size_t)(m0 + r0) * (I / 2), bytes_pk, full + s, pol);
@@ -720,11 +624,12 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
     const int r0 = sub * RS;
     const int nr = min(RS, nrows - r0);
     int n_tok, pos_base;
-    if (slot == 0) {
+    const int so = a.own[slot];
+    if (so == 0) {
       n_tok = T;
       pos_base = T * K;
     } else {
-      const int e = a.uni[slot - 1];
+      const int e = a.uni[so - 1];
       pos_base = a.off[e];
       n_tok = a.off[e + 1] - pos_base;
     }
@@ -818,8 +723,10 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
   if (*reinterpret_cast<volatile int *>(&s_abort)) return;
   for (int i = tid; i < T * nrows; i += 256) {
     const int t = i / nrows, m = i % nrows;
-    float o = ysm[(size_t)(T * K + t) * a.rows_max + m];
+    float o = a.with_shared ? ysm[(size_t)(T * K + t) * a.rows_max + m] : 0.0f;
     for (int q = 0; q < K; ++q) {
+      const int e = a.idx[t * K + q];
+      if (e < a.e_lo || e >= a.e_hi) continue;  // another rank's expert
       const int p = a.pos[t * K + q];
       o = ffma(a.w[t * K + q], ysm[(size_t)p * a.rows_max + m], o);
     }

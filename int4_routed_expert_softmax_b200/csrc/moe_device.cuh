@@ -100,15 +100,41 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the same phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for the phase of `parity` to complete.  Gives up after `limit`
 // SM clocks (the launch's wait limit: about a second by default, shorter when
 // a caller sets one with moe_set_wait_limit), records `detail` with
-// MOE_ERR_TIMEOUT in the status word and returns false.
+// MOE_ERR_TIMEOUT in the status word and returns false.  With the default
+// limit the wait uses try_wait, which may suspend the thread until the phase
+// completes; with a shorter one it polls with test_wait, so that the limit,
+// not the hardware's suspend time, bounds the wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *status,
                                           int32_t detail, long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (limit >= kWaitLimitCycles) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+      if (clock64() - t0 > limit) {
+        set_status(status, MOE_ERR_TIMEOUT, detail);
+        return false;
+      }
+    }
+    return true;
+  }
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_test_wait(bar, parity)) {
     if (clock64() - t0 > limit) {
       set_status(status, MOE_ERR_TIMEOUT, detail);
       return false;

@@ -19,6 +19,10 @@ constexpr int kMaxSmem = 227 * 1024 - 1024;            // dynamic shared memory 
 constexpr int kPfMaxCtas = 256;                        // prefill GEMM grid bound (one CTA per SM)
 constexpr int kProfSlots = 1024;                       // per-call profiling records kept per device
 constexpr int kProfWords = 8;                          // per record: 4 phases x (~first start, last end) in ns
+// Control words of the workspace (zeroed at the start of every call): [0] the
+// routing kernel's arrival ticket, [1] the fused kernel's routing arrivals,
+// [kCtrlSlot0 + s] gate/up units completed for union slot s (fused kernel).
+constexpr int kCtrlSlot0 = 4;
 
 // Device-side error details (status[1]) -- which wait or check failed.
 enum Detail : int32_t {
@@ -38,6 +42,14 @@ enum Detail : int32_t {
   kDetPfAccFull = 33,
   kDetPfAccFree = 34,
   kDetPfDrain = 35,
+  kDetFuRoute = 40,
+  kDetFuRouteDrain = 41,
+  kDetFuGrid = 42,
+  kDetFuFull = 43,
+  kDetFuEmpty = 44,
+  kDetFuDrain = 45,
+  kDetFuSlot = 46,
+  kDetFuAlign = 47,
 };
 
 // The wait limit kernels launched now take for their work waits (set by
@@ -69,7 +81,7 @@ inline size_t expert_bytes(int H, int I) { return 2 * matrix_bytes(I, H) + matri
 // Byte offsets of the workspace segments for batches of up to T tokens.  The
 // prefill segments (xg, hs, y, maps) are sized only when `prefill` is set.
 struct WsLayout {
-  size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, perm, pos,
+  size_t status, ctrl, xin, yout, xq, xd, logits, idx, w, cnt, off, uni, n_uni, own, n_own, perm, pos,
       pair_tok, hq, hqs, hd, xg, hs, y, maps, total;
 };
 
@@ -83,7 +95,7 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
     return at;
   };
   L.status = seg(16);
-  L.ctrl = seg(64);
+  L.ctrl = seg((size_t)(kCtrlSlot0 + kMaxK + 1) * 4);
   L.xin = seg((size_t)T * d.H * 4);
   L.yout = seg((size_t)T * d.H * 4);
   L.xq = seg((size_t)T * d.H);
@@ -95,6 +107,8 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
   L.off = seg((size_t)(d.E + 1) * 4);
   L.uni = seg((size_t)(d.E + 1) * 4);
   L.n_uni = seg(16);
+  L.own = seg((size_t)(d.E + 1) * 4);  // the union slots a call computes (expert parallelism)
+  L.n_own = seg(16);
   L.perm = seg((size_t)T * d.k * 4);
   L.pos = seg((size_t)T * d.k * 4);
   L.pair_tok = seg(P * 4);
@@ -125,6 +139,8 @@ struct RouteArgs {
   float *xd, *logits, *w;
   int32_t *idx, *route_counts;
   int32_t *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok;
+  int32_t *own, *n_own;     // owned slot list (null: not written)
+  int e_lo, e_hi, with_shared;
   unsigned int *done;
   int32_t *status;
   int do_quant;
@@ -145,6 +161,7 @@ struct GateUpArgs {
   int H, I, E, k, T;
   const void *const *table;
   const int32_t *uni, *n_uni, *off, *pair_tok;
+  const int32_t *own, *n_own;  // the slots to compute: 0 = shared expert, s >= 1 = uni[s - 1]
   const int8_t *xq;
   const float *xd;
   int8_t *hq;
@@ -162,6 +179,9 @@ struct DownArgs {
   int H, I, E, k, T;
   const void *const *table;
   const int32_t *uni, *n_uni, *off, *pos;
+  const int32_t *own, *n_own;  // the slots to compute: 0 = shared expert, s >= 1 = uni[s - 1]
+  const int32_t *idx;          // the combine adds the pairs whose expert is in [e_lo, e_hi)
+  int e_lo, e_hi, with_shared;
   const float *w;
   const int8_t *hq;
   const int32_t *hqs;
@@ -211,6 +231,32 @@ struct RouterTiledArgs {
   float *logits;
 };
 
+// The whole batch-1 decode layer in one cooperative kernel (moe_fused.cu).
+struct FusedArgs {
+  int H, I, E, k;
+  const float *x, *Wr;
+  const void *const *table;
+  float *out;
+  int8_t *xq;
+  float *xd, *logits, *w;
+  int32_t *idx, *route_counts;
+  int32_t *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok;
+  int8_t *hq;
+  int32_t *hqs;
+  float *hd;
+  int32_t *status;
+  unsigned int *arrivals;  // routing arrivals of the grid (zeroed per call)
+  int32_t *slot_done;      // [k + 1] gate/up units completed per union slot (zeroed per call)
+  int nstage;              // ring stages
+  int rows_max;            // down: most output rows a CTA owns
+  int rg;                  // down: row granularity (scale bytes of rg rows: a multiple of 16)
+  int rs;                  // down: rows per stage (a multiple of rg)
+  int e_lo, e_hi;          // routed experts this call computes (expert parallelism)
+  int with_shared;         // and the shared expert
+  long long wait_limit;
+  unsigned long long *prof;
+};
+
 struct CombineArgs {
   int H, k, T;
   const float *y, *w;
@@ -234,6 +280,13 @@ cudaError_t launch_topk(const float *logits, int T, int E, int k, int32_t *idx, 
                         int32_t *counts, cudaStream_t s);
 cudaError_t launch_gateup_decode(const GateUpArgs &a, int grid, size_t smem, cudaStream_t s);
 cudaError_t launch_down_decode(const DownArgs &a, int grid, size_t smem, cudaStream_t s);
+
+// Fused batch-1 decode (moe_fused.cu): plan (false if the shape does not fit
+// one CTA per SM) and launch (cooperative: every CTA resident at once).
+bool fused_plan(int H, int I, int E, int k, int grid, FusedArgs *a, size_t *smem);
+cudaError_t launch_decode_fused(const FusedArgs &a, int grid, size_t smem, cudaStream_t s);
+// CTAs of the fused kernel that fit on one SM with `smem` bytes (0 if none).
+int fused_ctas_per_sm(const FusedArgs &a, size_t smem);
 
 cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s);
 // 2D tensor map over a row-major fp16 matrix [rows][cols] for TMA copies of

@@ -297,3 +297,61 @@ def test_profile_records_each_call_and_leaves_output_unchanged(path):
         assert all(v > 0 for v in r), r
         assert max(r[:3]) <= r[3] * (1 + 1e-6), r
         assert r[3] < 1000.0, r       # milliseconds
+
+
+# ----------------------------------------------------------------- fused one-token kernel
+@pytest.mark.parametrize("H,I,E,k,seed", [
+    (256, 128, 16, 2, 1),        # tiny shape: most CTAs own no unit and no output row
+    (1024, 256, 64, 8, 2),
+    (384, 384, 5, 5, 3),         # k = E, ragged group count
+    (128, 128, 1, 1, 4),         # a single expert
+    (1024, 256, 1024, 32, 5),    # 7 router rows per CTA, k = 32
+    (8192, 4096, 8, 2, 6),       # widest shape: down rows in two stages per slot
+    (6144, 2048, 256, 8, 7),     # the GLM-5.2 decode layer
+])
+def test_fused_one_token_equals_three_kernel_path(H, I, E, k, seed):
+    """One token runs in the fused cooperative kernel; the same layer split into
+    moe_layer_route + moe_layer_experts runs the three-kernel path.  Both use the
+    same per-row order, so every output and every intermediate agrees bit for
+    bit; the fused call is also checked against the oracle."""
+    moe = _moe()
+    from int4_routed_expert_softmax_b200 import _cache as C
+    w = mi.Workload("fused", H=H, I=I, E=E, k=k, T=1, seed=900 + seed)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    d = moe.dims(H, I, E, k)
+    assert moe.moe_layer_launches(d, 1) == 1
+    assert moe.moe_layer_launches(d, 2) == 3
+    out_f, ws_f, _ = gpu_layer(w, x, Wr, blobs)
+    ws_s = moe.alloc_workspace(d, 1)
+    out_s = torch.full_like(out_f, float("nan"))
+    C.moe_layer_route(d, x, Wr, ws_s)
+    C.moe_layer_experts(d, 1, moe.expert_table(blobs), out_s, ws_s)
+    torch.cuda.synchronize()
+    assert torch.equal(out_f, out_s)
+    from tests._common import ws_trace
+    tf, ts = ws_trace(ws_f, d, 1), ws_trace(ws_s, d, 1)
+    for key in ("status", "xq", "xd", "logits", "idx", "w", "cnt", "off", "uni", "perm", "pos", "pair_tok", "hq",
+                "hd"):
+        assert np.array_equal(tf[key], ts[key]), key
+    assert tf["n_uni"] == ts["n_uni"]
+    if H * I <= 1024 * 256 or H == 6144:
+        _check_layer(w, x, Wr, blobs)
+
+
+def test_fused_route_counts_and_repeat():
+    moe = _moe()
+    w = mi.shrink(mi.WORKLOADS["decode"], seed=501)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    ws = moe.alloc_workspace(d, 1)
+    cnt = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    table = moe.expert_table(blobs)
+    outs = []
+    for _ in range(3):
+        out = torch.empty((1, w.H), device=DEV)
+        moe.moe_layer_forward(d, x, Wr, table, out, ws, route_counts=cnt)
+        outs.append(out)
+    torch.cuda.synchronize()
+    io, _ = orc.topk_softmax(orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy()), w.k)
+    assert np.array_equal(cnt.cpu().numpy(), 3 * np.bincount(io.reshape(-1), minlength=w.E))
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])

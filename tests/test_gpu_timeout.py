@@ -20,7 +20,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 SHORT = 200                       # SM clocks: shorter than any copy from HBM takes
 MOE_ERR_TIMEOUT = -7
-ROUTE_DETAILS = {1}               # the routing kernel's staging wait
+ROUTE_DETAILS = {1, 40, 42}       # the routing kernel's staging wait; the fused kernel's, its grid arrival
 EXPERT_DETAILS = {10, 11, 20, 21}  # gate/up and down: stage landed / stage freed
 PREFILL_DETAILS = {31, 32, 33, 34}  # grouped GEMM: operands landed / freed, accumulators
 
@@ -56,6 +56,8 @@ def test_wait_limit_setter_round_trip():
 
 @pytest.mark.parametrize("name", ["tiny", "medium"])
 def test_routing_wait_runs_out_then_recovers(name):
+    """tiny: four tokens, the three-kernel path; medium: one token, the fused
+    cooperative kernel."""
     moe = _moe()
     w = mi.WORKLOADS["tiny"] if name == "tiny" else _medium()
     x, Wr, blobs = mi.make_layer(w, 0, DEV)
