@@ -677,7 +677,7 @@ def run_stacked(args, ws_n, rank, local):
                         "layers": L, "T_list": list(w.T_list),
                         "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)"},
                 by_batch=res, clocks=clk.summary(),
-                gpu_launches=3 * L * args.steps * len(w.T_list))  # decode path: 3 kernels per layer call
+                gpu_launches=sum(moe.moe_layer_launches(d, T) for T in w.T_list) * L * args.steps)
 
 
 def run_tiered(args, ws_n, rank, local):
@@ -708,14 +708,30 @@ def run_tiered(args, ws_n, rank, local):
     side = torch.cuda.Stream(device=dev)
     stream = torch.cuda.current_stream()
     xs = mi.make_x(args.warmup + n_tok, w.H, mi.sub_seed(seed, 0, 1), dev, zipf=True, rho=w.rho)
+    # the glue between layers (x_{l+1} = RMS-normalised x_l + gamma out_l, not
+    # part of the MoE layer) as one CUDA graph on fixed buffers, so that its
+    # launches cost one replay per layer
+    x_buf = xs[0:1].clone()
+    for _ in range(2):
+        x_buf.copy_(chain_next_dev(x_buf, out, zipf=True))
+    torch.cuda.synchronize()
+    glue = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(glue):
+        x_buf.copy_(chain_next_dev(x_buf, out, zipf=True))
+    host_s = {"layer_call": 0.0, "glue": 0.0}
 
-    def token(t):
-        x = xs[t:t + 1].contiguous()
+    def token(t, timed=False):
+        x_buf.copy_(xs[t:t + 1])
         for l in range(L):
-            cache.tiered_layer_forward(l, x, routers[l], out, ws, ws_pred=ws_pred,
+            h0 = time.perf_counter()
+            cache.tiered_layer_forward(l, x_buf, routers[l], out, ws, ws_pred=ws_pred,
                                        Wr_next=routers[l + 1] if l + 1 < L else None,
                                        route_counts=counts[l], side_stream=side)
-            x = chain_next_dev(x, out, zipf=True)
+            h1 = time.perf_counter()
+            glue.replay()
+            if timed:
+                host_s["layer_call"] += h1 - h0
+                host_s["glue"] += time.perf_counter() - h1
 
     for t in range(args.warmup):
         token(t)
@@ -727,14 +743,19 @@ def run_tiered(args, ws_n, rank, local):
     s0 = cache.stats()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
+    moe.moe_profile_enable(True)   # per layer call: routing, gate/up, down, first start to last end
     barrier(ws_n)
     with ClockSampler(local) as clk:
         a.record(stream)
         for t in range(args.warmup, args.warmup + n_tok):
-            token(t)
+            token(t, timed=True)
         b.record(stream)
         torch.cuda.synchronize()
     ms = allreduce_max(a.elapsed_time(b), ws_n)
+    prof = moe.moe_profile_read(1024)
+    moe.moe_profile_enable(False)
+    device_us = {name: round(sum(p[i] for p in prof) / max(1, len(prof)) * 1e3, 2)
+                 for i, name in enumerate(("routing", "gate_up", "down", "call_span"))}
     s1 = cache.stats()
     dd = {k: s1[k] - s0[k] for k in ("hits", "misses", "prefetches", "prefetch_hits", "bytes_h2d", "evictions")}
     # host link alone: one 20 MB blob copy, pinned host -> HBM
@@ -761,8 +782,13 @@ def run_tiered(args, ws_n, rank, local):
                 prefetch_accuracy=round(dd["prefetch_hits"] / max(1, dd["prefetches"]), 4),
                 host_link_GBps={"during_run": round(dd["bytes_h2d"] / (ms * 1e-3) / 1e9, 2),
                                 "single_copy": round(link, 2)},
-                cache_delta=dd, us_per_token_layer=round(ms / n_tok / L * 1e3, 2), clocks=clk.summary(),
-                gpu_launches=None)
+                cache_delta=dd, us_per_token_layer=round(ms / n_tok / L * 1e3, 2),
+                host_us_per_layer={k: round(v / (n_tok * L) * 1e6, 1) for k, v in host_s.items()},
+                device_us_per_layer=dict(device_us, calls=len(prof),
+                                         what="device stamps: routing kernel, gate/up, down, and the "
+                                              "span from routing's first CTA to down's last (misses' "
+                                              "copies and the host's acquire fall inside it)"),
+                clocks=clk.summary(), gpu_launches=None)
 
 
 # ----------------------------------------------------------------- reference arm

@@ -212,6 +212,25 @@ int moe_layer_forward_static(const moe_dims *dims, int32_t T, const float *x, co
                              const void *const *expert_table, float *out, int32_t *route_counts_opt,
                              int32_t path, void *stream);
 
+/* The layer with MXFP4 expert blobs: the format in which the Kimi K3
+ * family's experts ship, QAT-trained and streamed without conversion (colibri
+ * deep review page, model-family table, Kimi K3 row).  Each blob is
+ * gate [I][H] | up [I][H] | down [H][I]; a matrix [N][K] is N*K/2 bytes of
+ * E2M1 codes (two consecutive elements per byte, the lower-indexed one in the
+ * low nibble; sign bit, two exponent bits of bias 1, one mantissa bit) then
+ * N*K/32 E8M0 exponent bytes, one per 32-block of a row (weight =
+ * e2m1 * 2^(E - 127), E = 255 outside the contract): the same byte count as
+ * int4 gs64.  Activations stay Q8_0, so every block sum is exact in integers
+ * (2 * e2m1 is an integer).  Decode path only, in the one-token fused kernel:
+ * a batch runs token by token, each token a full pass over its experts (the
+ * workspace's union record then holds the last token's).  MOE_ERR_SHAPE if
+ * the shape does not fit the fused kernel.  Other arguments as
+ * moe_layer_forward (workspace: moe_workspace_bytes_path(dims, T,
+ * MOE_PATH_DECODE)). */
+int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                            const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                            int32_t *route_counts_opt, void *stream);
+
 /* One rank's share of the layer under expert parallelism (GPU form of the
  * pages' cluster mode, where the routed-expert FFNs run on workers: colibri
  * deep review page, its local-cluster section).  Routing (Q8_0 of x, logits,

@@ -68,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "moe_layer_forward_host": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, P]),
             "moe_layer_forward_static": (ctypes.c_int, [D, i32, P, P, P, P, P, i32, P]),
             "moe_layer_forward_ep": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, i32, i32, i32, P]),
+            "moe_layer_forward_mxfp4": (ctypes.c_int, [D, i32, P, P, P, P, P, sz, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -236,6 +237,19 @@ def moe_layer_forward(d: MoeDims, x, Wr, table, out, ws, route_counts=None,
     _check("moe_layer_forward", lib().moe_layer_forward(
         ctypes.byref(d), x.shape[0], _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(route_counts), path, _stream(stream)))
+
+
+def moe_layer_forward_mxfp4(d: MoeDims, x, Wr, table, out, ws, route_counts=None, stream=None):
+    """The layer with MXFP4 expert blobs (decode path, token by token)."""
+    T = _rows(x, "x", d.H)
+    _arg(Wr, "Wr", torch.float32, d.E * d.H)
+    _arg(table, "table", torch.int64, d.E + 1)
+    _arg(out, "out", torch.float32, T * d.H)
+    _arg(ws, "ws", torch.uint8)
+    _arg(route_counts, "route_counts", torch.int32, d.E, optional=True)
+    _check("moe_layer_forward_mxfp4", lib().moe_layer_forward_mxfp4(
+        ctypes.byref(d), T, _ptr(x), _ptr(Wr), _ptr(table), _ptr(out), _ptr(ws), ws.numel(),
+        _ptr(route_counts), _stream(stream)))
 
 
 def moe_layer_forward_host(d: MoeDims, x_host, Wr, table, out_host, ws, route_counts=None,

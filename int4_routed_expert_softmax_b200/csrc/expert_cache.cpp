@@ -15,6 +15,8 @@
 // Backend MOE_CACHE_HOST keeps the policy identical but uses host memory and
 // memcpy, so the policy and its failure paths are testable without a GPU.
 #include <algorithm>
+#include <atomic>
+#include <chrono>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -42,6 +44,7 @@ struct Layer {
   const void **d_table = nullptr; // device table [E+1]
   cudaEvent_t table_done = nullptr;
   bool table_pending = false;
+  bool table_dirty = true;        // residency changed since the device table was uploaded
   cudaEvent_t released = nullptr; // last release of this layer
   bool released_valid = false;
   int n_pinned = 0;
@@ -62,6 +65,14 @@ struct moe_cache {
   std::vector<char> slot_ready_valid;
   moe_cache_stats st{};
   int fault_copy = 0;
+  // tiered layers: union mailboxes (mapped pinned host memory the routing
+  // kernel writes; [0] this layer's union, [1] the predicted one), their
+  // sequence counter, and the stream the one-layer-ahead prediction runs on
+  int32_t *mbox_host[2] = {nullptr, nullptr};
+  int32_t *mbox_dev[2] = {nullptr, nullptr};
+  int32_t seq = 0;
+  cudaStream_t pred_stream = nullptr;
+  cudaEvent_t x_ready = nullptr;
 };
 
 namespace {
@@ -84,6 +95,7 @@ void drop(moe_cache *c, Layer &ly, int e) {
   const int slot = ly.slot_of[e];
   ly.lru.erase(ly.where[e]);
   ly.slot_of[e] = -1;
+  ly.table_dirty = true;
   ly.prefetched[e] = 0;
   ly.free_slots.push_back(slot);
   c->st.evictions++;
@@ -149,6 +161,7 @@ int make_resident(moe_cache *c, int layer, int e, cudaStream_t s, const std::vec
     return rc;
   }
   ly.slot_of[e] = slot;
+  ly.table_dirty = true;
   ly.lru.push_front(e);
   ly.where[e] = ly.lru.begin();
   c->st.resident++;
@@ -181,6 +194,10 @@ void destroy_all(moe_cache *c) {
     for (auto ev : c->slot_ready)
       if (ev) cudaEventDestroy(ev);
     if (c->pool) cudaFree(c->pool);
+    for (int i = 0; i < 2; ++i)
+      if (c->mbox_host[i]) cudaFreeHost(c->mbox_host[i]);
+    if (c->x_ready) cudaEventDestroy(c->x_ready);
+    if (c->pred_stream) cudaStreamDestroy(c->pred_stream);
   } else {
     std::free(c->pool);
   }
@@ -256,6 +273,24 @@ int expert_cache_create(const moe_dims *dims, int32_t n_layers, const void *cons
         destroy_all(c);
         return MOE_ERR_CUDA;
       }
+    for (int i = 0; i < 2; ++i) {
+      void *p = nullptr, *pd = nullptr;
+      if (cudaHostAlloc(&p, sizeof(int32_t) * (size_t)(moe::kMailUni + dims->E), cudaHostAllocMapped) !=
+              cudaSuccess ||
+          cudaHostGetDevicePointer(&pd, p, 0) != cudaSuccess) {
+        if (p) cudaFreeHost(p);
+        destroy_all(c);
+        return MOE_ERR_ALLOC;
+      }
+      c->mbox_host[i] = static_cast<int32_t *>(p);
+      c->mbox_dev[i] = static_cast<int32_t *>(pd);
+      std::memset(p, 0, sizeof(int32_t) * (size_t)(moe::kMailUni + dims->E));
+    }
+    if (cudaStreamCreateWithFlags(&c->pred_stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&c->x_ready, cudaEventDisableTiming) != cudaSuccess) {
+      destroy_all(c);
+      return MOE_ERR_CUDA;
+    }
   } else {
     c->pool = static_cast<unsigned char *>(std::malloc(pool_bytes));
     if (!c->pool) {
@@ -415,26 +450,39 @@ int expert_cache_acquire(moe_cache *c, int32_t layer, const int32_t *experts, in
   ly.last_slots.clear();
   for (int e : want) ly.last_slots.push_back(ly.slot_of[e]);
   if (dev(c)) {
-    if (ly.table_pending) {
+    // the compute stream waits for the copies these slots still have in
+    // flight; a copy found complete is not waited on again
+    for (int s : ly.last_slots)
+      if (c->slot_ready_valid[s]) {
+        const cudaError_t q = cudaEventQuery(c->slot_ready[s]);
+        if (q == cudaSuccess) {
+          c->slot_ready_valid[s] = 0;
+        } else if (q == cudaErrorNotReady) {
+          rc = cuda_err(cudaStreamWaitEvent(ks, c->slot_ready[s], 0));
+          if (rc) return rc;
+        } else {
+          return cuda_err(q);
+        }
+      }
+  }
+  if (ly.table_dirty || !dev(c)) {
+    // the device table of the layer changes only with its residency
+    if (dev(c) && ly.table_pending) {
       rc = cuda_err(cudaEventSynchronize(ly.table_done));
       if (rc) return rc;
       ly.table_pending = false;
     }
-  }
-  for (int e = 0; e < c->E1; ++e)
-    ly.h_table[e] = ly.slot_of[e] >= 0 ? c->pool + (size_t)ly.slot_of[e] * c->blob : nullptr;
-  if (dev(c)) {
-    for (int s : ly.last_slots)
-      if (c->slot_ready_valid[s]) {
-        rc = cuda_err(cudaStreamWaitEvent(ks, c->slot_ready[s], 0));
-        if (rc) return rc;
-      }
-    rc = cuda_err(cudaMemcpyAsync(ly.d_table, ly.h_table, sizeof(void *) * (size_t)c->E1,
-                                  cudaMemcpyHostToDevice, ks));
-    if (rc) return rc;
-    rc = cuda_err(cudaEventRecord(ly.table_done, ks));
-    if (rc) return rc;
-    ly.table_pending = true;
+    for (int e = 0; e < c->E1; ++e)
+      ly.h_table[e] = ly.slot_of[e] >= 0 ? c->pool + (size_t)ly.slot_of[e] * c->blob : nullptr;
+    if (dev(c)) {
+      rc = cuda_err(cudaMemcpyAsync(ly.d_table, ly.h_table, sizeof(void *) * (size_t)c->E1,
+                                    cudaMemcpyHostToDevice, ks));
+      if (rc) return rc;
+      rc = cuda_err(cudaEventRecord(ly.table_done, ks));
+      if (rc) return rc;
+      ly.table_pending = true;
+    }
+    ly.table_dirty = false;
   }
   *d_table = ly.d_table;
   return MOE_OK;
@@ -490,6 +538,33 @@ int expert_cache_stats(const moe_cache *c, moe_cache_stats *stats) {
 
 }  // extern "C"
 
+namespace {
+
+// Waits (host, bounded) until the routing kernel has posted sequence `seq` to
+// the mailbox, then copies the union out.  If it never comes, the routing
+// failed on the device: the stream is synchronised and its status returned.
+int wait_mailbox(const int32_t *mb, int32_t seq, int E, int32_t *uni, int32_t *n, cudaStream_t s, void *ws,
+                 const moe_dims *dims, int T) {
+  const volatile int32_t *vm = mb;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (long spin = 0; vm[moe::kMailSeq] != seq; ++spin) {
+    if ((spin & 1023) == 0 && std::chrono::steady_clock::now() - t0 > std::chrono::seconds(2)) {
+      int32_t h[1];
+      int32_t hn = 0;
+      const int rc = moe_read_union(dims, T, ws, h, &hn, s);  // synchronises; returns the device status
+      return rc != MOE_OK ? rc : MOE_ERR_TIMEOUT;
+    }
+  }
+  std::atomic_thread_fence(std::memory_order_acquire);
+  const int nu = vm[moe::kMailN];
+  if (nu < 0 || nu > E) return MOE_ERR_DEVICE;
+  for (int i = 0; i < nu; ++i) uni[i] = vm[moe::kMailUni + i];
+  *n = nu;
+  return MOE_OK;
+}
+
+}  // namespace
+
 extern "C" int moe_tiered_layer_forward(moe_cache *c, int32_t layer, const moe_dims *dims, int32_t T,
                                         const float *x, const float *Wr, const float *Wr_next_opt,
                                         float *out, void *ws, size_t ws_bytes, void *ws_pred,
@@ -501,26 +576,38 @@ extern "C" int moe_tiered_layer_forward(moe_cache *c, int32_t layer, const moe_d
       dims->k != c->d.k)
     return MOE_ERR_SHAPE;
   if (prefetch_out_opt) prefetch_out_opt[0] = prefetch_out_opt[1] = 0;
-  int rc = moe_layer_route(dims, T, x, Wr, ws, ws_bytes, route_counts_opt, compute_stream);
+  cudaStream_t cs = static_cast<cudaStream_t>(compute_stream);
+  // routing; the kernel posts the union to the mailbox when it is done
+  const int32_t seq = ++c->seq;
+  int rc = moe::route_to_mailbox(dims, T, x, Wr, ws, ws_bytes, route_counts_opt, c->mbox_dev[0], seq, true, cs);
   if (rc != MOE_OK) return rc;
   const bool predict = Wr_next_opt != nullptr && ws_pred != nullptr && layer + 1 < c->L;
+  int32_t seq_pred = 0;
   if (predict) {
-    // one-layer-ahead: the next layer's router on this layer's input
-    rc = moe_layer_route(dims, T, x, Wr_next_opt, ws_pred, ws_pred_bytes, nullptr, compute_stream);
+    // one-layer-ahead: the next layer's router on this layer's input, on the
+    // cache's own stream (off the layer's critical path)
+    seq_pred = ++c->seq;
+    if (cudaEventRecord(c->x_ready, cs) != cudaSuccess || cudaStreamWaitEvent(c->pred_stream, c->x_ready, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    rc = moe::route_to_mailbox(dims, T, x, Wr_next_opt, ws_pred, ws_pred_bytes, nullptr, c->mbox_dev[1], seq_pred,
+                               false, c->pred_stream);
     if (rc != MOE_OK) return rc;
   }
   std::vector<int32_t> uni(dims->E), pred(dims->E);
   int32_t n = 0, np = 0;
-  rc = moe_read_union(dims, T, ws, uni.data(), &n, compute_stream);
+  rc = wait_mailbox(c->mbox_host[0], seq, dims->E, uni.data(), &n, cs, ws, dims, T);
   if (rc != MOE_OK) return rc;
-  if (predict) {
-    rc = moe_read_union(dims, T, ws_pred, pred.data(), &np, compute_stream);
-    if (rc != MOE_OK) return rc;
-  }
   const void *table = nullptr;
   rc = expert_cache_acquire(c, layer, uni.data(), n, side_stream, compute_stream, &table);
   if (rc != MOE_OK) return rc;
+  rc = moe_layer_experts(dims, T, static_cast<const void *const *>(table), out, ws, ws_bytes, compute_stream);
+  if (rc != MOE_OK) return rc;
+  rc = expert_cache_release(c, layer, compute_stream);
+  if (rc != MOE_OK) return rc;
   if (predict) {
+    // the prediction has long been posted: prefetch layer + 1's union
+    rc = wait_mailbox(c->mbox_host[1], seq_pred, dims->E, pred.data(), &np, c->pred_stream, ws_pred, dims, T);
+    if (rc != MOE_OK) return rc;
     const int started = expert_cache_prefetch(c, layer + 1, pred.data(), np, side_stream);
     if (started < 0) return started;
     if (prefetch_out_opt) {
@@ -528,8 +615,5 @@ extern "C" int moe_tiered_layer_forward(moe_cache *c, int32_t layer, const moe_d
       prefetch_out_opt[1] = np;
     }
   }
-  rc = moe_layer_experts(dims, T, static_cast<const void *const *>(table), out, ws, ws_bytes,
-                         compute_stream);
-  if (rc != MOE_OK) return rc;
-  return expert_cache_release(c, layer, compute_stream);
+  return MOE_OK;
 }

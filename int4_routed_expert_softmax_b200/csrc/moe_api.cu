@@ -131,7 +131,7 @@ Owned all_owned(const moe_dims &d) { return Owned{0, d.E, 1}; }
 
 int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const float *x,
                 const float *Wr, void *ws, int32_t *counts, unsigned long long *prof,
-                const Owned &ow, cudaStream_t s) {
+                const Owned &ow, cudaStream_t s, int32_t *mail = nullptr, int32_t mail_seq = 0) {
   const ChunkPtrs p = chunk_ptrs(d, t0, L, ws);
   RouteArgs ra{};
   ra.H = d.H;
@@ -155,6 +155,8 @@ int route_chunk(const moe_dims &d, int t0, int Tc, const WsLayout &L, const floa
   ra.pair_tok = p.pair_tok;
   ra.own = p.own;
   ra.n_own = p.n_own;
+  ra.mail = mail;
+  ra.mail_seq = mail_seq;
   ra.e_lo = ow.lo;
   ra.e_hi = ow.hi;
   ra.with_shared = ow.shared;
@@ -261,7 +263,7 @@ constexpr int kFusedNA = 1;
 // Whether the fused kernel runs this layer's one-token calls on the current
 // device (its shape fits one CTA per SM, cooperative launch available); fills
 // its plan.  Asked once per device and shape.
-bool fused_usable(const moe_dims &d, FusedArgs *fa, size_t *smem, int *grid) {
+bool fused_usable(const moe_dims &d, int fmt, FusedArgs *fa, size_t *smem, int *grid) {
   const int sms = device_sms();
   if (sms <= 0) return false;
   *fa = FusedArgs{};
@@ -270,32 +272,34 @@ bool fused_usable(const moe_dims &d, FusedArgs *fa, size_t *smem, int *grid) {
   fa->I = d.I;
   fa->E = d.E;
   fa->k = d.k;
+  fa->fmt = fmt;
   *grid = sms;
   static std::mutex mu;
-  static int known[kMaxDevices] = {0};
-  static moe_dims key[kMaxDevices];
-  static bool fits[kMaxDevices] = {false};
+  static int known[kMaxDevices][2] = {};
+  static moe_dims key[kMaxDevices][2];
+  static bool fits[kMaxDevices][2] = {};
   const int dev = current_device();
-  if (dev < 0) return false;
+  if (dev < 0 || fmt < 0 || fmt > 1) return false;
   std::lock_guard<std::mutex> lock(mu);
-  if (!known[dev] || key[dev].H != d.H || key[dev].I != d.I || key[dev].E != d.E || key[dev].k != d.k) {
+  moe_dims &kd = key[dev][fmt];
+  if (!known[dev][fmt] || kd.H != d.H || kd.I != d.I || kd.E != d.E || kd.k != d.k) {
     int coop = 0;
     if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) != cudaSuccess) coop = 0;
-    fits[dev] = coop && fused_ctas_per_sm(*fa, *smem) >= 1;
+    fits[dev][fmt] = coop && fused_ctas_per_sm(*fa, *smem) >= 1;
     cudaGetLastError();
-    known[dev] = 1;
-    key[dev] = d;
+    known[dev][fmt] = 1;
+    kd = d;
   }
-  return fits[dev];
+  return fits[dev][fmt];
 }
 
 int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
                   const void *const *table, float *out, void *ws, int32_t *counts,
-                  unsigned long long *prof, const Owned &ow, cudaStream_t s) {
+                  unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4) {
   FusedArgs fa{};
   size_t smem = 0;
   int sms = 0;
-  if (!fused_usable(d, &fa, &smem, &sms)) return kFusedNA;
+  if (!fused_usable(d, fmt, &fa, &smem, &sms)) return kFusedNA;
   const ChunkPtrs p = chunk_ptrs(d, 0, L, ws);
   fa.x = x;
   fa.Wr = Wr;
@@ -428,6 +432,22 @@ const void *host_device_view(const void *p) {
 }
 
 }  // namespace
+
+int route_to_mailbox(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws, size_t ws_bytes,
+                     int32_t *route_counts_opt, int32_t *mail, int32_t seq, bool profile, cudaStream_t s) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 1 || T > kDecodeTMax || !x || !Wr || !ws || !mail) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  return route_chunk(*dims, 0, T, L, x, Wr, ws, route_counts_opt, profile ? prof_next() : nullptr,
+                     all_owned(*dims), s, mail, seq);
+}
+
 }  // namespace moe
 
 using namespace moe;
@@ -518,7 +538,7 @@ int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path) {
     FusedArgs fa{};
     size_t smem = 0;
     int grid = 0;
-    if (fused_usable(*dims, &fa, &smem, &grid)) return 1;
+    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return 1;
   }
   return 3 * ((T + kDecodeTMax - 1) / kDecodeTMax);
 }
@@ -687,6 +707,48 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   return forward_checked(*dims, T, x, Wr, expert_table, out, ws, route_counts_opt, pf, L, false,
                          static_cast<cudaStream_t>(stream), all_owned(*dims));
+}
+
+int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
+                            const void *const *expert_table, float *out, void *ws, size_t ws_bytes,
+                            int32_t *route_counts_opt, void *stream) {
+  int rc = moe_check_dims(dims);
+  if (rc != MOE_OK) return rc;
+  if (T < 0) return MOE_ERR_BAD_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !Wr || !expert_table || !out || !ws) return MOE_ERR_BAD_ARG;
+  if (!aligned(x, 16) || !aligned(Wr, 16) || !aligned(out, 16)) return MOE_ERR_BAD_ARG;
+  if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const WsLayout L = ws_layout(*dims, T, false);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  {
+    FusedArgs fa{};
+    size_t smem = 0;
+    int grid = 0;
+    if (!fused_usable(*dims, kFmtMxfp4, &fa, &smem, &grid)) return MOE_ERR_SHAPE;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the status word once per call; the fused kernel's control words per token
+  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
+  if (err != cudaSuccess) return cuda_status(err);
+  unsigned long long *prof = prof_next();
+  for (int t = 0; t < T; ++t) {
+    if (t > 0) {
+      err = cudaMemsetAsync(at<unsigned char>(ws, L.ctrl), 0, L.xin - L.ctrl, s);
+      if (err != cudaSuccess) return cuda_status(err);
+    }
+    // token t in the per-token rows of the workspace; the pair rows are reused
+    WsLayout Lt = L;
+    Lt.xq += (size_t)t * dims->H;
+    Lt.xd += (size_t)t * (dims->H / 32) * 4;
+    Lt.logits += (size_t)t * dims->E * 4;
+    Lt.idx += (size_t)t * dims->k * 4;
+    Lt.w += (size_t)t * dims->k * 4;
+    rc = fused_forward(*dims, Lt, x + (size_t)t * dims->H, Wr, expert_table, out + (size_t)t * dims->H, ws,
+                       route_counts_opt, t == 0 ? prof : nullptr, all_owned(*dims), s, kFmtMxfp4);
+    if (rc != MOE_OK) return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
+  }
+  return MOE_OK;
 }
 
 int moe_layer_forward_ep(const moe_dims *dims, int32_t T, const float *x, const float *Wr,

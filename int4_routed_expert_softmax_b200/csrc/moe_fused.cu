@@ -130,7 +130,10 @@ __device__ __forceinline__ bool wait_count(const int32_t *p, int32_t target, lon
 
 }  // namespace
 
-template <int CSZG, int CSZD>
+// FMT: the expert weight format, kFmtInt4 (int4 gs64, fp16 group scales) or
+// kFmtMxfp4 (E2M1 codes, E8M0 exponent per 32-block); both hold K/2 code
+// bytes and K/32 scale bytes per row, so the stream is the same.
+template <int CSZG, int CSZD, int FMT>
 __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   constexpr int R = kFuR, NW = kFuNW, SPU = kFuSPU, RPW = kFuRPW, PWR = kFuPWR, NCT = kFuNCT;
   constexpr int PROD = NW, EPI = NW + 1;  // warp roles after routing
@@ -456,17 +459,25 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
         const unsigned char *sb = stg + (size_t)s * pl.sb;
         uint32_t wv[RPW][CSZG][8];
         float sc[RPW][CSZG];
+        uint32_t ex[RPW][CSZG];
 #pragma unroll
-        for (int q = 0; q < RPW; ++q)
-          load_row<CSZG>(sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2),
-                         reinterpret_cast<const __half *>(sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) +
-                                                          (size_t)row_r[q] * (H / 32)),
-                         c0, GG, wv[q], sc[q]);
+        for (int q = 0; q < RPW; ++q) {
+          const unsigned char *rowp = sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2);
+          const unsigned char *scp = sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) + (size_t)row_r[q] * (H / 32);
+          if constexpr (FMT == kFmtMxfp4)
+            load_row_mx<CSZG>(rowp, scp, c0, GG, wv[q], ex[q]);
+          else
+            load_row<CSZG>(rowp, reinterpret_cast<const __half *>(scp), c0, GG, wv[q], sc[q]);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
 #pragma unroll
-        for (int q = 0; q < RPW; ++q)
-          redw[(st * RPW + q) * 33 + lane] = chunk_dot<CSZG>(wv[q], sc[q], act1, d1, z1, c0, GG);
+        for (int q = 0; q < RPW; ++q) {
+          if constexpr (FMT == kFmtMxfp4)
+            redw[(st * RPW + q) * 33 + lane] = chunk_dot_mx<CSZG>(wv[q], ex[q], act1, d1, c0, GG);
+          else
+            redw[(st * RPW + q) * 33 + lane] = chunk_dot<CSZG>(wv[q], sc[q], act1, d1, z1, c0, GG);
+        }
       }
       if (st == SPU - 1) {
         // unit complete: this warp's g and u row sums into the unit's buffer
@@ -517,11 +528,17 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
         const int ra = warp * nr_ / NW, rz = (warp + 1) * nr_ / NW;  // this warp's rows of the stage
         for (int ml = ra; ml < rz; ++ml) {
           uint32_t wv[CSZD][8];
-          float sc[CSZD];
-          load_row<CSZD>(sb + (size_t)ml * (I / 2),
-                         reinterpret_cast<const __half *>(sb + (size_t)RS * (I / 2) + (size_t)ml * (I / 32)), c0, GD,
-                         wv, sc);
-          redw[(ml - ra) * 33 + lane] = chunk_dot<CSZD>(wv, sc, av, dv, zv, c0, GD);
+          const unsigned char *rowp = sb + (size_t)ml * (I / 2);
+          const unsigned char *scp = sb + (size_t)RS * (I / 2) + (size_t)ml * (I / 32);
+          if constexpr (FMT == kFmtMxfp4) {
+            uint32_t ex[CSZD];
+            load_row_mx<CSZD>(rowp, scp, c0, GD, wv, ex);
+            redw[(ml - ra) * 33 + lane] = chunk_dot_mx<CSZD>(wv, ex, av, dv, c0, GD);
+          } else {
+            float sc[CSZD];
+            load_row<CSZD>(rowp, reinterpret_cast<const __half *>(scp), c0, GD, wv, sc);
+            redw[(ml - ra) * 33 + lane] = chunk_dot<CSZD>(wv, sc, av, dv, zv, c0, GD);
+          }
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(empty + s);
@@ -591,10 +608,10 @@ bool fused_plan(int H, int I, int E, int k, int grid, FusedArgs *a, size_t *smem
   return false;
 }
 
-template <int CSZG, int CSZD>
+template <int CSZG, int CSZD, int FMT>
 static cudaError_t launch_fu(const FusedArgs &a, int grid, size_t smem, cudaStream_t s) {
   static int smem_set[64] = {0};
-  cudaError_t err = ensure_smem(k_decode_fused<CSZG, CSZD>, smem, smem_set);
+  cudaError_t err = ensure_smem(k_decode_fused<CSZG, CSZD, FMT>, smem, smem_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -606,31 +623,37 @@ static cudaError_t launch_fu(const FusedArgs &a, int grid, size_t smem, cudaStre
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_fused<CSZG, CSZD>, a);
+  return cudaLaunchKernelEx(&cfg, k_decode_fused<CSZG, CSZD, FMT>, a);
 }
 
-template <int CSZG, int CSZD>
+template <int CSZG, int CSZD, int FMT>
 static int ctas_fu(size_t smem) {
   static int smem_set[64] = {0};
-  if (ensure_smem(k_decode_fused<CSZG, CSZD>, smem, smem_set) != cudaSuccess) return 0;
+  if (ensure_smem(k_decode_fused<CSZG, CSZD, FMT>, smem, smem_set) != cudaSuccess) return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_fused<CSZG, CSZD>, kFuThreads, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_fused<CSZG, CSZD, FMT>, kFuThreads, smem) !=
       cudaSuccess)
     return 0;
   return n;
 }
 
+#define MOE_FU_CASES(FN, F, ...)                                           \
+  case 11: return FN<1, 1, F>(__VA_ARGS__);                                \
+  case 12: return FN<1, 2, F>(__VA_ARGS__);                                \
+  case 21: return FN<2, 1, F>(__VA_ARGS__);                                \
+  case 22: return FN<2, 2, F>(__VA_ARGS__);                                \
+  case 31: return FN<3, 1, F>(__VA_ARGS__);                                \
+  case 32: return FN<3, 2, F>(__VA_ARGS__);                                \
+  case 41: return FN<4, 1, F>(__VA_ARGS__);                                \
+  case 42: return FN<4, 2, F>(__VA_ARGS__);
 #define MOE_FU_DISPATCH(FN, ...)                                           \
-  switch ((a.H / 64 + 31) / 32 * 10 + (a.I / 64 + 31) / 32) {              \
-    case 11: return FN<1, 1>(__VA_ARGS__);                                 \
-    case 12: return FN<1, 2>(__VA_ARGS__);                                 \
-    case 21: return FN<2, 1>(__VA_ARGS__);                                 \
-    case 22: return FN<2, 2>(__VA_ARGS__);                                 \
-    case 31: return FN<3, 1>(__VA_ARGS__);                                 \
-    case 32: return FN<3, 2>(__VA_ARGS__);                                 \
-    case 41: return FN<4, 1>(__VA_ARGS__);                                 \
-    case 42: return FN<4, 2>(__VA_ARGS__);                                 \
-    default: break;                                                        \
+  {                                                                        \
+    const int key = (a.H / 64 + 31) / 32 * 10 + (a.I / 64 + 31) / 32;     \
+    if (a.fmt == kFmtMxfp4) {                                              \
+      switch (key) { MOE_FU_CASES(FN, kFmtMxfp4, __VA_ARGS__) default: break; } \
+    } else {                                                               \
+      switch (key) { MOE_FU_CASES(FN, kFmtInt4, __VA_ARGS__) default: break; }  \
+    }                                                                      \
   }
 
 cudaError_t launch_decode_fused(const FusedArgs &a, int grid, size_t smem, cudaStream_t s) {

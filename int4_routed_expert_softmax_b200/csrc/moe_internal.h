@@ -23,6 +23,9 @@ constexpr int kProfWords = 8;                          // per record: 4 phases x
 // routing kernel's arrival ticket, [1] the fused kernel's routing arrivals,
 // [kCtrlSlot0 + s] gate/up units completed for union slot s (fused kernel).
 constexpr int kCtrlSlot0 = 4;
+// Expert weight formats of the decode kernels.
+constexpr int kFmtInt4 = 0;   // int4 gs64, fp16 group scales
+constexpr int kFmtMxfp4 = 1;  // E2M1 codes, one E8M0 exponent per 32-block
 
 // Device-side error details (status[1]) -- which wait or check failed.
 enum Detail : int32_t {
@@ -141,6 +144,8 @@ struct RouteArgs {
   int32_t *cnt, *off, *uni, *n_uni, *perm, *pos, *pair_tok;
   int32_t *own, *n_own;     // owned slot list (null: not written)
   int e_lo, e_hi, with_shared;
+  int32_t *mail;            // mapped pinned host mailbox [2 + E] or null: [0] seq, [1] n_uni, [2..] union
+  int32_t mail_seq;
   unsigned int *done;
   int32_t *status;
   int do_quant;
@@ -253,6 +258,7 @@ struct FusedArgs {
   int rs;                  // down: rows per stage (a multiple of rg)
   int e_lo, e_hi;          // routed experts this call computes (expert parallelism)
   int with_shared;         // and the shared expert
+  int fmt;                 // kFmtInt4 or kFmtMxfp4
   long long wait_limit;
   unsigned long long *prof;
 };
@@ -264,6 +270,16 @@ struct CombineArgs {
   float *out;
   unsigned long long *prof;  // profiling record or null (phase 2 end)
 };
+
+// Offsets of the union mailbox (mapped pinned host memory the routing kernel
+// writes for the tiered cache): sequence number, union size, union.
+constexpr int kMailSeq = 0, kMailN = 1, kMailUni = 2;
+
+// moe_layer_route that also posts the union to a mailbox (moe_api.cu):
+// mail = device address of mapped pinned host memory [2 + E], seq = the value
+// the host waits for in mail[kMailSeq]; profile = take a profiling record.
+int route_to_mailbox(const moe_dims *dims, int32_t T, const float *x, const float *Wr, void *ws, size_t ws_bytes,
+                     int32_t *route_counts_opt, int32_t *mail, int32_t seq, bool profile, cudaStream_t s);
 
 // Launchers (moe_kernels.cu).  Return cudaSuccess or the launch error.
 cudaError_t launch_quant(const QuantArgs &a, cudaStream_t s);

@@ -398,6 +398,17 @@ __global__ void __launch_bounds__(128) k_route_decode(RouteArgs a) {
       }
       if (lane == 0) *a.n_own = base;
     }
+    if (a.mail != nullptr) {
+      // post the union to the host's mailbox (mapped pinned memory): the
+      // entries and the size first, then the sequence number the host waits on
+      __syncwarp();
+      const int nu = *a.n_uni;
+      for (int i = lane; i < nu; i += 32) a.mail[kMailUni + i] = a.uni[i];
+      if (lane == 0) a.mail[kMailN] = nu;
+      __threadfence_system();
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<volatile int32_t *>(a.mail + kMailSeq) = a.mail_seq;
+    }
   }
   if (lane == 0) *a.done = 0u;
   prof_end(a.prof, 0);

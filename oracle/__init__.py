@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
             "or_mx_pack_matrix": (None, [P, P, i32, i32, P]),
             "or_mx_block_dot": (ctypes.c_int32, [P, i32, i32, i32, i32, P]),
             "or_mx_expert_dot": (f32, [P, i32, i32, i32, P, P]),
+            "or_mx_expert_down": (None, [P, i32, i32, P, P, P]),
             "or_mx_expert_ffn": (None, [P, i32, i32, P, P, P, P, P, P, P, P]),
             "or_moe_layer_mx": (i32, [i32, i32, i32, i32, i32, P, P, P, P, P]),
             "or_moe_layer_tokens_mx": (i32, [i32, i32, i32, i32, P, P, P, P, i32, P]),
@@ -202,13 +203,16 @@ def expert_ffn(blob: np.ndarray, H: int, I: int, xq: np.ndarray, xd: np.ndarray,
     return dict(g=g, u=u, h=h, hq=hq, hd=hd, y=y)
 
 
-def expert_down(blob: np.ndarray, H: int, I: int, hq: np.ndarray, hd: np.ndarray) -> np.ndarray:
-    """y [H] of one expert from given codes hq [I] and scales hd [I/32]."""
+def expert_down(blob: np.ndarray, H: int, I: int, hq: np.ndarray, hd: np.ndarray,
+                fmt: str = "int4") -> np.ndarray:
+    """y [H] of one expert from given codes hq [I] and scales hd [I/32];
+    fmt "int4" (int4 gs64 blob) or "mxfp4" (MXFP4 blob)."""
     blob = _c(blob, np.uint8)
     hq = _c(hq, np.int8)
     hd = _c(hd, np.float32)
     y = np.zeros(H, np.float32)
-    lib().or_expert_down(_p(blob), H, I, _p(hq), _p(hd), _p(y))
+    fn = lib().or_mx_expert_down if fmt == "mxfp4" else lib().or_expert_down
+    fn(_p(blob), H, I, _p(hq), _p(hd), _p(y))
     return y
 
 

@@ -325,6 +325,12 @@ void or_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const f
   for (int m = 0; m < H; ++m) y[m] = or_expert_dot(down, H, I, m, hq, hd);
 }
 
+/* The same down projection for an MXFP4 blob (same byte offsets). */
+void or_mx_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y) {
+  const uint8_t *down = blob + 2 * or_matrix_bytes(I, H);
+  for (int m = 0; m < H; ++m) y[m] = or_mx_expert_dot(down, H, I, m, hq, hd);
+}
+
 /* Row n of an [N][K] matrix of weight format fmt (OR_FMT_INT4_GS64 or
  * OR_FMT_MXFP4) against the Q8_0 vector (q, d). */
 static float fmt_dot(int fmt, const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d) {

@@ -109,6 +109,8 @@ int32_t or_mx_block_dot(const uint8_t *mat, int N, int K, int n, int b, const in
 /* Row n against the Q8_0 vector: block terms (S_b * d_b) * 2^(E_b - 128) summed
  * over b ascending, one binary32 accumulator. */
 float or_mx_expert_dot(const uint8_t *mat, int N, int K, int n, const int8_t *q, const float *d);
+/* The down projection of an MXFP4 expert from given Q8_0 codes of h. */
+void or_mx_expert_down(const uint8_t *blob, int H, int I, const int8_t *hq, const float *hd, float *y);
 void or_mx_expert_ffn(const uint8_t *blob, int H, int I, const int8_t *xq, const float *xd,
                       float *g, float *u, float *h, int8_t *hq, float *hd, float *y);
 

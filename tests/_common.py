@@ -24,7 +24,7 @@ def within_tolerance(got: np.ndarray, ref: np.ndarray):
 
 
 def oracle_layer_from_device(x: torch.Tensor, Wr: torch.Tensor, blobs: torch.Tensor,
-                             H, I, E, k, trace=True, tokens=None):
+                             H, I, E, k, trace=True, tokens=None, fmt="int4"):
     """Runs the oracle on host copies of the device inputs.  Only the blobs of
     the experts the oracle's own routing selects (and the shared expert) are
     copied back; the oracle never reads the others."""
@@ -40,8 +40,8 @@ def oracle_layer_from_device(x: torch.Tensor, Wr: torch.Tensor, blobs: torch.Ten
     dummy = np.zeros(16, np.uint8)
     blist = [blobs[e].cpu().numpy() if e in need else dummy for e in range(E + 1)]
     if tokens is not None:
-        return orc.moe_layer_tokens(xh, wh, blist, H, I, E, k, tokens)
-    return orc.moe_layer(xh, wh, blist, H, I, E, k, trace=trace)
+        return orc.moe_layer_tokens(xh, wh, blist, H, I, E, k, tokens, fmt=fmt)
+    return orc.moe_layer(xh, wh, blist, H, I, E, k, trace=trace, fmt=fmt)
 
 
 def gpu_layer(w: mi.Workload, x, Wr, blobs, path=0, ws=None):
@@ -127,21 +127,21 @@ def check_hq(g, tr, T, k):
     return int(diff.astype(bool).sum())
 
 
-def out_from_codes(g, tr, blobs, w, T):
+def out_from_codes(g, tr, blobs, w, T, fmt="int4"):
     """The oracle's down projections of the path's own h codes, combined in the
     layer's order (float64 sums of float32 terms)."""
     hq, hd = hq_by_slot(g, T, w.k)
     bl = blobs.cpu().numpy() if isinstance(blobs, torch.Tensor) else np.asarray(blobs)
     out = np.zeros((T, w.H), np.float64)
     for t in range(T):
-        out[t] = orc.expert_down(bl[w.E], w.H, w.I, hq[t, w.k], hd[t, w.k])
+        out[t] = orc.expert_down(bl[w.E], w.H, w.I, hq[t, w.k], hd[t, w.k], fmt=fmt)
         for s in range(w.k):
             e = int(tr["idx"][t, s])
-            out[t] += np.float64(tr["w"][t, s]) * orc.expert_down(bl[e], w.H, w.I, hq[t, s], hd[t, s])
+            out[t] += np.float64(tr["w"][t, s]) * orc.expert_down(bl[e], w.H, w.I, hq[t, s], hd[t, s], fmt=fmt)
     return out
 
 
-def check_traced(got, ref, g, tr, blobs, w, T):
+def check_traced(got, ref, g, tr, blobs, w, T, fmt="int4"):
     """A call's outputs `got` and workspace trace `g` against the oracle's
     outputs `ref` and trace `tr` on the same inputs.  Routing bit-exact; h codes
     within the flip bound; outputs within 1e-5 (rel-L2) of the oracle's down
@@ -152,7 +152,7 @@ def check_traced(got, ref, g, tr, blobs, w, T):
     Returns the number of differing h codes."""
     check_routing(g, tr)
     flips = check_hq(g, tr, T, w.k)
-    oc = out_from_codes(g, tr, blobs, w, T)
+    oc = out_from_codes(g, tr, blobs, w, T, fmt=fmt)
     nr = np.linalg.norm(oc)
     rms = np.sqrt(np.mean(oc * oc))
     assert np.linalg.norm(got - oc) <= 1e-5 * nr, np.linalg.norm(got - oc) / nr

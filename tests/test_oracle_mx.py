@@ -149,6 +149,24 @@ def test_expert_ffn_vs_float64():
     assert np.allclose(r["y"], y, rtol=1e-5, atol=1e-5 * np.abs(y).max())
 
 
+def test_expert_down_from_codes():
+    """The down projection from given codes: the FFN's own y from its own codes
+    bit for bit, and the dequantised matrix times other codes within the float
+    bound of its sum."""
+    H, I = 256, 128
+    blob, (Wg, Wu, Wd) = _mx_blob(H, I)
+    x = rng.normal(size=H).astype(np.float32)
+    xq, xd = orc.quant_q8_0(x)
+    r = orc.expert_ffn(blob, H, I, xq, xd, fmt="mxfp4")
+    assert np.array_equal(orc.expert_down(blob, H, I, r["hq"], r["hd"], fmt="mxfp4").view(np.uint32),
+                          r["y"].view(np.uint32))
+    hq, hd = orc.quant_q8_0((rng.normal(size=I) * 3).astype(np.float32))
+    y = orc.expert_down(blob, H, I, hq, hd, fmt="mxfp4").astype(np.float64)
+    hh = hq.astype(np.float64) * np.repeat(hd.astype(np.float64), 32)
+    ref, mag = Wd @ hh, np.abs(Wd) @ np.abs(hh)
+    assert np.all(np.abs(y - ref) <= (I // 32 + 8) * 2.0**-23 * mag)
+
+
 def test_layer_vs_float64_and_int4_routing():
     """The MXFP4 layer: the same routing as the int4 layer on the same x and
     router (the experts' format does not enter routing), and its output within
