@@ -15,7 +15,7 @@
 //
 // The GEMM tile is two blocks of 128 weight rows (MMA M = 128 each; for
 // gate/up the gate and the up rows of the same 128 intermediate rows) by up to
-// 64 token rows of one expert (MMA N, a multiple of 16), so an expert with few
+// 96 token rows of one expert (MMA N, a multiple of 16), so an expert with few
 // tokens wastes at most 15 columns.  K advances one 64-group per pipeline
 // stage.
 //
@@ -155,12 +155,14 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
 // One CTA per SM, persistent over its tiles (blockIdx.x, + gridDim.x, ...);
 // a tile is G pipeline stages, one 64-group of K each.  A tile is two blocks
 // of 128 weight rows (gate/up: the gate rows and the up rows of the same 128
-// intermediate rows; down: 256 consecutive output rows) against up to 64
-// token rows of one expert.  23 warps (80 registers per thread, so that
-// nothing spills: with shared memory nearly full, L1 has little room for
-// local memory):
-//   0-15  epilogue: TMEM lane quarter warp & 3, columns 16 * (warp >> 2) ..
-//         of both blocks; per stage acc += s_g * C_g, after a tile's last
+// intermediate rows; down: 256 consecutive output rows) against up to 96
+// token rows of one expert.  23 warps (at most 88 registers per thread):
+//   0-15  epilogue: TMEM lane quarter warp & 3, columns 24 * (warp >> 2) ..
+//         of both blocks; per stage acc += s_g * C_g in fp32 registers --
+//         every group's accumulator is read out, so that no tensor-core
+//         accumulation runs longer than one group (the tensor cores' fp32
+//         sums lose about 2^-25 relative per accumulation step, which over a
+//         whole K of 6144 would flip Q8_0 codes of h); after a tile's last
 //         group its outputs (gate/up: SwiGLU and Q8_0 of h in the thread that
 //         holds g and u);
 //   16-19 expansion: packed nibbles of stage i -> fp16 A operands in tensor
@@ -180,30 +182,30 @@ constexpr int kPfRawWarp = 20;
 constexpr int kPfActWarp = 21;
 constexpr int kPfMmaWarp = 22;
 constexpr int kPfThreads = 23 * 32;
-constexpr int kPfTileN = 64;                 // token rows per tile (MMA N <= 64)
+constexpr int kPfTileN = 96;                 // token rows per tile (MMA N <= 96)
 constexpr int kPfNA = 2;                     // A operand buffers (tensor memory, 64 columns each)
-constexpr int kPfNT = 3;                     // accumulator buffers (tensor memory, 128 columns each)
-constexpr int kPfRB = 6;                     // activation ring slots
+constexpr int kPfNT = 2;                     // accumulator buffers (tensor memory, 192 columns each)
+constexpr int kPfRB = 4;                     // activation ring slots
 constexpr int kPfRR = 7;                     // packed-weight ring slots
 constexpr uint32_t kPfTmemCols = 512;
-constexpr uint32_t kPfAccCols = 128;         // per buffer: block 0 at +0, block 1 at +64
+constexpr uint32_t kPfAccCols = 192;         // per buffer: block 0 at +0, block 1 at +96
 constexpr uint32_t kPfACol0 = kPfNT * kPfAccCols;  // A buffers from column 384: block b, slice k at +32 b + 8 k
+constexpr int kPfEpiCols = 24;               // token columns per epilogue thread (4 column quarters)
 
-constexpr uint32_t kBHalf = 8192;     // [64 rows][128 B] fp16, 128-byte swizzle (hi or lo)
+constexpr uint32_t kBHalf = (uint32_t)kPfTileN * 128;  // [96 rows][128 B] fp16, 128-byte swizzle (hi or lo)
 constexpr uint32_t kBBytes = 2 * kBHalf;
 constexpr uint32_t kRawBlk = 4096;    // [128 rows][32 B] packed weights of a group, one block
 constexpr uint32_t kRawBytes = 2 * kRawBlk;
 
 struct PfLayout {
-  uint32_t tile_pre, b, raw, hst, total;
+  uint32_t tile_pre, b, raw, total;
 };
 __host__ __device__ inline PfLayout pf_layout(int E) {
   PfLayout L;
   L.tile_pre = 1024;
   L.b = (uint32_t)((L.tile_pre + 4 * (E + 2) + 1023) / 1024 * 1024);
   L.raw = L.b + (uint32_t)kPfRB * kBBytes;
-  L.hst = L.raw + (uint32_t)kPfRR * kRawBytes;
-  L.total = L.hst + (uint32_t)kPfEpiWarps * 32 * 32 * 4;  // g, u staging: [32][512 epilogue threads]
+  L.total = L.raw + (uint32_t)kPfRR * kRawBytes;
   return L;
 }
 
@@ -287,7 +289,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 template <int MODE>
-__global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
+__global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const __grid_constant__ CUtensorMap bmap) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int H = a.H, I = a.I;
@@ -486,7 +488,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
         const uint32_t idesc = pf_idesc(cm.tl.n);
         const uint64_t bd = b0 + (uint64_t)((sb * kBBytes) >> 4);
         for (int blk = 0; blk < cm.tl.nblk; ++blk) {
-          const uint32_t d = tmem + (uint32_t)(tb * kPfAccCols + 64 * blk);
+          const uint32_t d = tmem + (uint32_t)(tb * kPfAccCols + kPfTileN * blk);
           const uint32_t at = tmem + kPfACol0 + (uint32_t)(na * 64 + 32 * blk);
 #pragma unroll
           for (int k4 = 0; k4 < 4; ++k4) {
@@ -556,9 +558,9 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
     // ================================================================ epilogue
     bool bad = false;
     const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
-    const int q = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 16-column quarter
+    const int q = warp & 3, cq = warp >> 2;  // TMEM lane quarter, 24-column quarter
     const int row = q * 32 + lane;
-    const int col0 = cq * 16;
+    const int col0 = cq * kPfEpiCols;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
     // weight scales of this thread's rows of both blocks: 4 bytes (groups g,
     // g+1) each per stage pair, loaded one pair ahead
@@ -582,9 +584,9 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       if (ce.tl.nblk == 2) w1n = scale_at(ce.tl, 1, 0);
     }
     uint32_t w0c = 0, w1c = 0;
-    float acc0[16], acc1[16];
+    float acc0[kPfEpiCols], acc1[kPfEpiCols];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) acc0[i] = acc1[i] = 0.0f;
+    for (int i = 0; i < kPfEpiCols; ++i) acc0[i] = acc1[i] = 0.0f;
 
     for (int j = 0; j < S && !bad; ++j) {
       const int tb = j % kPfNT;
@@ -610,27 +612,35 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
         const int sh = (ce.g & 1) * 16;
         const float s0 = __half2float(__ushort_as_half((unsigned short)(w0c >> sh)));
         const float s1 = __half2float(__ushort_as_half((unsigned short)(w1c >> sh)));
-        uint32_t v[16];
-        tmem_ld16(tq + (uint32_t)(tb * kPfAccCols), v);
-        tmem_ld_wait();
+        // eight columns at a time (48 accumulators stay live in registers)
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc0[k] = ffma(s0, __uint_as_float(v[k]), acc0[k]);
-        tmem_ld16(tq + (uint32_t)(tb * kPfAccCols + 64), v);
-        tmem_ld_wait();
+        for (int c8 = 0; c8 < kPfEpiCols; c8 += 8) {
+          uint32_t v8[8];
+          tmem_ld8(tq + (uint32_t)(tb * kPfAccCols + c8), v8);
+          tmem_ld_wait();
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc1[k] = ffma(s1, __uint_as_float(v[k]), acc1[k]);
+          for (int k = 0; k < 8; ++k) acc0[c8 + k] = ffma(s0, __uint_as_float(v8[k]), acc0[c8 + k]);
+        }
+#pragma unroll
+        for (int c8 = 0; c8 < kPfEpiCols; c8 += 8) {
+          uint32_t v8[8];
+          tmem_ld8(tq + (uint32_t)(tb * kPfAccCols + kPfTileN + c8), v8);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc1[c8 + k] = ffma(s1, __uint_as_float(v8[k]), acc1[c8 + k]);
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tfree + tb);
       if (ce.g == G - 1 && col0 < ce.tl.nval) {
-        // the tile's outputs; this thread holds columns col0 .. col0 + 15 of both blocks
+        // the tile's outputs; this thread holds columns col0 .. col0 + 23 of both blocks
         const PfTile tl = ce.tl;
-        const int ncol = min(16, tl.nval - col0);
+        const int ncol = min(kPfEpiCols, tl.nval - col0);
         if (MODE == 1) {
           float *yc = a.y + (size_t)(tl.p0 + col0) * H + (size_t)tl.wt * 256 + row;
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < kPfEpiCols; ++k) {
             if (k < ncol) {
               yc[(size_t)k * H] = acc0[k];
               if (tl.nblk == 2) yc[(size_t)k * H + 128] = acc1[k];
@@ -640,21 +650,14 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
           // h = SiLU(g) * u, its Q8_0 codes along I (one 32-block of I = one
           // warp's lanes) and the hi/lo split of the dequantised h for the down
           // GEMM, in fast fp32 (this path is held to the layer's tolerance, not
-          // to the fixed-order bits).  g and u go through shared memory (own
-          // values only) so that the per-column loop stays rolled.
-          float *hst = reinterpret_cast<float *>(smem + L.hst) + tid;
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            hst[k * kPfEpiWarps * 32] = acc0[k];
-            hst[(16 + k) * kPfEpiWarps * 32] = acc1[k];
-          }
+          // to the fixed-order bits)
           const int ii = tl.wt * 128 + row;  // row of I
           __half *hs = static_cast<__half *>(a.hs);
           const size_t hcol = (size_t)(ii >> 6) * 128 + (ii & 63);
-#pragma unroll 1
-          for (int k = 0; k < 16; ++k) {
-            const float gv = hst[k * kPfEpiWarps * 32];
-            const float h = __fdividef(gv, 1.0f + __expf(-gv)) * hst[(16 + k) * kPfEpiWarps * 32];
+#pragma unroll
+          for (int k = 0; k < kPfEpiCols; ++k) {
+            const float gv = acc0[k];
+            const float h = __fdividef(gv, 1.0f + __expf(-gv)) * acc1[k];
             const float amax = warp_max(fabsf(h));
             const float d = amax * (1.0f / 127.0f);
             const float inv = amax > 0.0f ? __fdividef(127.0f, amax) : 0.0f;
@@ -674,7 +677,7 @@ __global__ void __maxnreg__(80) k_gemm_pf(const PfArgs a, const __grid_constant_
       }
       if (ce.g == G - 1) {
 #pragma unroll
-        for (int k = 0; k < 16; ++k) acc0[k] = acc1[k] = 0.0f;
+        for (int k = 0; k < kPfEpiCols; ++k) acc0[k] = acc1[k] = 0.0f;
       }
       cur_next(ce);
       if (*abort_flag) bad = true;
