@@ -244,7 +244,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
         my_tok = lane < n_tok ? a.pair_tok[pos_base + lane] : 0;
       }
     }
-    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
+    if (!bad) bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int *>(&s_abort) != 0);
     if (!bad) {
       bad = !mbar_wait(full + s, ph, a.status, kDetGuFull, a.wait_limit);
       bad = __any_sync(0xffffffffu, bad);
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
       pos_base = a.off[e];
       n_tok = a.off[e + 1] - pos_base;
     }
-    if (!bad) bad = *reinterpret_cast<volatile int *>(&s_abort) != 0;
+    if (!bad) bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int *>(&s_abort) != 0);
     if (!bad) {
       bad = !mbar_wait(full + s, ph, a.status, kDetDnFull, a.wait_limit);
       bad = __any_sync(0xffffffffu, bad);

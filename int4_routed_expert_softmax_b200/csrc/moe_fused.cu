@@ -408,7 +408,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       const float *gb = gu + par * 64;
       const float g = gb[lane], uv = gb[32 + lane];
       if (cu + 2 < my_units) named_arrive(kBarGuFree + par, NCT + 32);
-      if (*s_abort) continue;
+      if (__any_sync(0xffffffffu, *s_abort != 0)) continue;  // one decision per warp
       const int u = (int)blockIdx.x + G * cu;
       const int slot = s_own[u / rbs], rb = u % rbs;
       const int pos_base = slot == 0 ? K : slot - 1;
@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     }
     for (int j = 0; j < n_gu; ++j) {
       const int cu = j / SPU, st = j % SPU;
-      if (!bad) bad = *s_abort != 0;
+      if (!bad) bad = __any_sync(0xffffffffu, *s_abort != 0);  // one decision per warp
       if (!bad) {
         bad = !mbar_wait(full + s, ph, a.status, kDetFuFull, lim);
         bad = __any_sync(0xffffffffu, bad);
@@ -512,7 +512,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       const int slot = s_own[jd / nsub], sub = jd % nsub;
       const int r0 = sub * RS, nr_ = min(RS, nrows - r0);
       const int pos_base = slot == 0 ? K : slot - 1;
-      if (!bad) bad = *s_abort != 0;
+      if (!bad) bad = __any_sync(0xffffffffu, *s_abort != 0);  // one decision per warp
       if (!bad) {
         bad = !mbar_wait(full + s, ph, a.status, kDetFuFull, lim);
         bad = __any_sync(0xffffffffu, bad);

@@ -171,7 +171,12 @@ __device__ __forceinline__ void nib4_to_f16(uint32_t n, uint32_t &lo, uint32_t &
 //         per expert on the device), as far ahead as the ring allows;
 //   21    activation copies (lane 0): TMA of the hi/lo token rows;
 //   22    MMAs (lane 0): per block and K16 slice hi then lo, A from tensor
-//         memory, B from shared memory.
+//         memory, B from shared memory;
+//   23    idle (completes the last warpgroup for setmaxnreg).
+// Launched at 80 registers per thread and split with setmaxnreg: the four
+// epilogue warpgroups take 96, the other two give theirs down to 48
+// (4 x 128 x 96 + 2 x 128 x 48 = 61440 = 768 x 80; the host checks the
+// launch count).
 // Shared memory then carries only the activation rows and the packed weights,
 // which keeps its bandwidth below the tensor cores' need.  Every hand-off is
 // an mbarrier; every wait is bounded.
@@ -181,16 +186,28 @@ constexpr int kPfExpWarp0 = 16;              // expansion warps 16..19
 constexpr int kPfRawWarp = 20;
 constexpr int kPfActWarp = 21;
 constexpr int kPfMmaWarp = 22;
-constexpr int kPfThreads = 23 * 32;
+constexpr int kPfThreads = 24 * 32;
+constexpr int kPfRegsLaunch = 80;            // registers per thread at launch (checked on the host)
+constexpr int kPfRegsEpi = 96;               // epilogue warpgroups after setmaxnreg.inc
+constexpr int kPfRegsOther = 48;             // the other two after setmaxnreg.dec
+static_assert(4 * 128 * kPfRegsEpi + 2 * 128 * kPfRegsOther <= kPfThreads * kPfRegsLaunch,
+              "register split exceeds the launch's registers");
 constexpr int kPfTileN = 96;                 // token rows per tile (MMA N <= 96)
 constexpr int kPfNA = 2;                     // A operand buffers (tensor memory, 64 columns each)
 constexpr int kPfNT = 2;                     // accumulator buffers (tensor memory, 192 columns each)
 constexpr int kPfRB = 4;                     // activation ring slots
 constexpr int kPfRR = 7;                     // packed-weight ring slots
+// Stage j's MMAs complete on mdone[j % MD] (one commit per stage).  Its
+// waiters -- the epilogue for stage j, the activation copies for j - RB, the
+// expansion for j - NA -- each wait for a stage that the barrier cannot have
+// passed: its next completion, stage j + MD, needs work from that waiter first
+// (MD >= RB, NA and NT).
+constexpr int kPfMD = 4;
 constexpr uint32_t kPfTmemCols = 512;
 constexpr uint32_t kPfAccCols = 192;         // per buffer: block 0 at +0, block 1 at +96
 constexpr uint32_t kPfACol0 = kPfNT * kPfAccCols;  // A buffers from column 384: block b, slice k at +32 b + 8 k
-constexpr int kPfEpiCols = 24;               // token columns per epilogue thread (4 column quarters)
+constexpr int kPfEpiCols = 24;
+static_assert(kPfMD >= kPfRB && kPfMD >= kPfNA && kPfMD >= kPfNT, "stage-done ring too short");               // token columns per epilogue thread (4 column quarters)
 
 constexpr uint32_t kBHalf = (uint32_t)kPfTileN * 128;  // [96 rows][128 B] fp16, 128-byte swizzle (hi or lo)
 constexpr uint32_t kBBytes = 2 * kBHalf;
@@ -300,11 +317,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
   uint64_t *rawfull = reinterpret_cast<uint64_t *>(smem);  // [RR] packed weights landed (TMA bytes)
   uint64_t *rawfree = rawfull + kPfRR;                      // [RR] expanded (4 expansion warps)
   uint64_t *bfull = rawfree + kPfRR;                        // [RB] activation rows landed (TMA bytes)
-  uint64_t *bfree = bfull + kPfRB;                          // [RB] read by the MMAs (commit)
-  uint64_t *aready = bfree + kPfRB;                         // [NA] A operands written (4 expansion warps)
-  uint64_t *afree = aready + kPfNA;                         // [NA] A operands read by the MMAs (commit)
-  uint64_t *accf = afree + kPfNA;                           // [NT] accumulators written (commit)
-  uint64_t *tfree = accf + kPfNT;                           // [NT] accumulators read (8 epilogue warps)
+  uint64_t *aready = bfull + kPfRB;                         // [NA] A operands written (4 expansion warps)
+  uint64_t *mdone = aready + kPfNA;                         // [MD] the stage's MMAs complete (one commit)
+  uint64_t *tfree = mdone + kPfMD;                          // [NT] accumulators read (16 epilogue warps)
   uint64_t *drain = tfree + kPfNT;                          // teardown
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + 512);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + 516);
@@ -325,18 +340,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
       mbar_init(rawfull + s, 1);
       mbar_init(rawfree + s, 4);
     }
-    for (int s = 0; s < kPfRB; ++s) {
-      mbar_init(bfull + s, 1);
-      mbar_init(bfree + s, 1);
-    }
-    for (int s = 0; s < kPfNA; ++s) {
-      mbar_init(aready + s, 4);
-      mbar_init(afree + s, 1);
-    }
-    for (int s = 0; s < kPfNT; ++s) {
-      mbar_init(accf + s, 1);
-      mbar_init(tfree + s, kPfEpiWarps);
-    }
+    for (int s = 0; s < kPfRB; ++s) mbar_init(bfull + s, 1);
+    for (int s = 0; s < kPfNA; ++s) mbar_init(aready + s, 4);
+    for (int s = 0; s < kPfMD; ++s) mbar_init(mdone + s, 1);
+    for (int s = 0; s < kPfNT; ++s) mbar_init(tfree + s, kPfEpiWarps);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -393,6 +400,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
     }
   };
 
+  if (warp >= kPfRawWarp) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfRegsOther));
   if (warp == kPfRawWarp) {
     // ======================================================= weight copies
     if (lane == 0) {
@@ -445,8 +454,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
       for (int j = 0; j < S && !bad; ++j, cur_next(cb)) {
         // hi/lo rows of stage j: boxes of kPfBoxRows rows; rows past the
         // tile's own land in unused B rows, rows past the array read zero
-        const int sb = j % kPfRB;
-        if (j >= kPfRB && !mbar_wait(bfree + sb, (uint32_t)(j / kPfRB - 1) & 1u, a.status, kDetPfEmpty, a.wait_limit)) {
+        const int sb = j % kPfRB, jp = j - kPfRB;  // jp: the stage that used this slot last
+        if (j >= kPfRB &&
+            !mbar_wait(mdone + jp % kPfMD, (uint32_t)(jp / kPfMD) & 1u, a.status, kDetPfEmpty, a.wait_limit)) {
           bad = true;
           break;
         }
@@ -496,9 +506,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
             umma_f16_ts(d, at + 8 * k4, bd + (uint64_t)((kBHalf + k4 * 32) >> 4), idesc, 1u);
           }
         }
-        umma_commit(accf + tb);
-        umma_commit(bfree + sb);
-        umma_commit(afree + na);
+        umma_commit(mdone + j % kPfMD);
         done = j + 1;
       }
       if (bad) *abort_flag = 1;
@@ -508,7 +516,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
       }
     }
     __syncwarp();
+  }
   } else if (warp >= kPfExpWarp0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kPfRegsOther));
     // ================================================================ expansion
     bool bad = false;
     const int q = warp - kPfExpWarp0;   // TMEM lane quarter
@@ -519,7 +529,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
     for (int i = 0; i < S && !bad; ++i, cur_next(cx)) {
       const int ra = i % kPfRR, na = i % kPfNA;
       if (!warp_wait(rawfull + ra, (uint32_t)(i / kPfRR) & 1u, a.status, kDetPfFull, a.wait_limit) ||
-          (i >= kPfNA && !warp_wait(afree + na, (uint32_t)(i / kPfNA - 1) & 1u, a.status, kDetPfFull, a.wait_limit))) {
+          (i >= kPfNA && !warp_wait(mdone + (i - kPfNA) % kPfMD, (uint32_t)((i - kPfNA) / kPfMD) & 1u, a.status,
+                                    kDetPfFull, a.wait_limit))) {
         bad = true;
         break;
       }
@@ -551,10 +562,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
         mbar_arrive(aready + na);
         mbar_arrive(rawfree + ra);
       }
-      if (*abort_flag) bad = true;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) bad = true;  // one decision per warp
     }
     if (bad) *abort_flag = 1;
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kPfRegsEpi));
     // ================================================================ epilogue
     bool bad = false;
     const size_t mg = (size_t)I * (size_t)(H / 2) + (size_t)I * (size_t)(H / 64) * 2;  // bytes of gate (= up)
@@ -562,26 +574,42 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
     const int row = q * 32 + lane;
     const int col0 = cq * kPfEpiCols;
     const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)col0;
-    // weight scales of this thread's rows of both blocks: 4 bytes (groups g,
-    // g+1) each per stage pair, loaded one pair ahead
-    auto scale_at = [&](const PfTile &tl, int blk, int g) -> uint32_t {
+    // weight scales of this thread's rows of both blocks (fp16 per group), as
+    // a row pointer per tile taken one tile ahead (block 1's row lies a fixed
+    // distance after block 0's); 4 bytes (groups g, g + 1) each per stage
+    // pair, loaded one pair ahead
+    const size_t blk1 = MODE == 0 ? mg / 4 : (size_t)128 * (I / 64) / 2;  // in 4-byte words
+    auto scale_row = [&](const PfTile &tl) -> const uint32_t * {
       const unsigned char *blob = static_cast<const unsigned char *>(a.table[tl.e]);
       const unsigned char *p;
       if (MODE == 0) {
         const size_t rr = (size_t)tl.wt * 128 + row;
-        p = blob + (size_t)blk * mg + (size_t)I * (size_t)(H / 2) + rr * (size_t)(H / 64) * 2;
+        p = blob + (size_t)I * (size_t)(H / 2) + rr * (size_t)(H / 64) * 2;
       } else {
-        const size_t rr = (size_t)tl.wt * 256 + (size_t)blk * 128 + row;
+        const size_t rr = (size_t)tl.wt * 256 + row;
         p = blob + 2 * mg + (size_t)H * (size_t)(I / 2) + rr * (size_t)(I / 64) * 2;
       }
-      return __ldg(reinterpret_cast<const uint32_t *>(p) + (g >> 1));
+      return reinterpret_cast<const uint32_t *>(p);
     };
     PfCur<MODE> ce;
     cur_begin(ce);
+    // this tile's scale row and the next tile's, each with its block count
+    const uint32_t *sr = nullptr, *sn = nullptr;
+    int nbn = 0;
+    auto next_rows = [&](int t) {
+      sn = nullptr;
+      if (t < n_tiles) {
+        const PfTile nt = pf_tile<MODE>(t, tile_pre, nslot, a);
+        sn = scale_row(nt);
+        nbn = nt.nblk;
+      }
+    };
     uint32_t w0n = 0, w1n = 0;  // scales of the next stage pair
     if (S > 0) {
-      w0n = scale_at(ce.tl, 0, 0);
-      if (ce.tl.nblk == 2) w1n = scale_at(ce.tl, 1, 0);
+      sr = scale_row(ce.tl);
+      w0n = __ldg(sr);
+      if (ce.tl.nblk == 2) w1n = __ldg(sr + blk1);
+      next_rows(ce.t + (int)gridDim.x);
     }
     uint32_t w0c = 0, w1c = 0;
     float acc0[kPfEpiCols], acc1[kPfEpiCols];
@@ -595,15 +623,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
         w1c = w1n;
         // the pair after this one: in this tile, or the first of the next
         if (ce.g + 2 < G) {
-          w0n = scale_at(ce.tl, 0, ce.g + 2);
-          if (ce.tl.nblk == 2) w1n = scale_at(ce.tl, 1, ce.g + 2);
-        } else if (ce.t + (int)gridDim.x < n_tiles) {
-          const PfTile nt = pf_tile<MODE>(ce.t + (int)gridDim.x, tile_pre, nslot, a);
-          w0n = scale_at(nt, 0, 0);
-          if (nt.nblk == 2) w1n = scale_at(nt, 1, 0);
+          w0n = __ldg(sr + ((ce.g + 2) >> 1));
+          if (ce.tl.nblk == 2) w1n = __ldg(sr + blk1 + ((ce.g + 2) >> 1));
+        } else if (sn != nullptr) {
+          w0n = __ldg(sn);
+          if (nbn == 2) w1n = __ldg(sn + blk1);
         }
       }
-      if (!warp_wait(accf + tb, (uint32_t)(j / kPfNT) & 1u, a.status, kDetPfAccFull, a.wait_limit)) {
+      if (!warp_wait(mdone + j % kPfMD, (uint32_t)(j / kPfMD) & 1u, a.status, kDetPfAccFull, a.wait_limit)) {
         bad = true;
         break;
       }
@@ -678,9 +705,12 @@ __global__ void __launch_bounds__(kPfThreads, 1) k_gemm_pf(const PfArgs a, const
       if (ce.g == G - 1) {
 #pragma unroll
         for (int k = 0; k < kPfEpiCols; ++k) acc0[k] = acc1[k] = 0.0f;
+        // the next tile's scale rows become current; look up the one after
+        sr = sn;
+        next_rows(ce.t + 2 * (int)gridDim.x);
       }
       cur_next(ce);
-      if (*abort_flag) bad = true;
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) bad = true;  // one decision per warp
     }
     if (bad) *abort_flag = 1;
   }
@@ -736,10 +766,25 @@ cudaError_t launch_make_maps(const PfArgs &a, const CUtensorMap &tgu, const CUte
   return cudaGetLastError();
 }
 
+// The register split of k_gemm_pf assumes the launch's count: a build that
+// gave the kernel fewer registers would leave setmaxnreg.inc waiting.
+template <int MODE>
+cudaError_t pf_regs_ok() {
+  static int ok = 0;  // 1 checked, -1 refused
+  if (ok == 0) {
+    cudaFuncAttributes fa{};
+    const cudaError_t err = cudaFuncGetAttributes(&fa, k_gemm_pf<MODE>);
+    if (err != cudaSuccess) return err;
+    ok = fa.numRegs == kPfRegsLaunch ? 1 : -1;
+  }
+  return ok == 1 ? cudaSuccess : cudaErrorInvalidConfiguration;
+}
+
 cudaError_t launch_gemm_pf(const PfArgs &a, const CUtensorMap &bmap, int grid, cudaStream_t s) {
   const size_t smem = pf_layout(a.E).total;
   if (smem > (size_t)kMaxSmem) return cudaErrorInvalidConfiguration;
-  cudaError_t err;
+  cudaError_t err = a.mode == 0 ? pf_regs_ok<0>() : pf_regs_ok<1>();
+  if (err != cudaSuccess) return err;
   if (a.mode == 0) {
     static int smem_set0[64] = {0};
     err = ensure_smem(k_gemm_pf<0>, smem, smem_set0);
