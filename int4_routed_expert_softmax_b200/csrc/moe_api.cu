@@ -293,9 +293,13 @@ bool fused_usable(const moe_dims &d, int fmt, FusedArgs *fa, size_t *smem, int *
   return fits[dev][fmt];
 }
 
+// One launch of the fused kernel.  tok < 0: the whole layer for one token
+// (its own routing).  tok >= 0: token tok of a batch of T whose routing record
+// the routing kernel has written (routed mode); out is that token's row.
 int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
                   const void *const *table, float *out, void *ws, int32_t *counts,
-                  unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4) {
+                  unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4,
+                  int tok = -1, int T = 1) {
   FusedArgs fa{};
   size_t smem = 0;
   int sms = 0;
@@ -329,7 +333,44 @@ int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const fl
   fa.with_shared = ow.shared;
   fa.wait_limit = wait_limit_cycles();
   fa.prof = prof;
+  if (tok >= 0) {
+    const size_t t = (size_t)tok;
+    fa.routed = 1;
+    fa.xq = p.xq + t * d.H;
+    fa.xd = p.xd + t * (d.H / 32);
+    fa.idx = p.idx + t * d.k;
+    fa.w = p.w + t * d.k;
+    fa.pos_t = p.pos + t * d.k;
+    fa.shared_pos = T * d.k + tok;
+    fa.route_counts = nullptr;  // counted by the routing kernel
+    fa.slot_done = at<int32_t>(ws, L.ctrl) + t * kCtrlWords + kCtrlSlot0;
+  }
   return cuda_status(launch_decode_fused(fa, sms, smem, s));
+}
+
+// A decode batch of 2 <= T <= kDecodeTMax tokens through the fused kernel,
+// token by token: the routing kernel writes the batch's record (codes of x,
+// top-k, union, pair positions), then one fused launch per token streams that
+// token's experts and writes its h codes at the batch's pair positions.  At
+// these batch sizes the union of the batch is nearly the sum of the tokens'
+// selections, so the per-token stream costs few extra bytes and runs at the
+// fused kernel's rate.  kFusedNA if the fused kernel does not fit the shape.
+int fused_batch_forward(const moe_dims &d, int T, const WsLayout &L, const float *x, const float *Wr,
+                        const void *const *table, float *out, void *ws, int32_t *counts,
+                        unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4) {
+  {
+    FusedArgs fa{};
+    size_t smem = 0;
+    int sms = 0;
+    if (!fused_usable(d, fmt, &fa, &smem, &sms)) return kFusedNA;
+  }
+  int rc = route_chunk(d, 0, T, L, x, Wr, ws, counts, prof, ow, s);
+  if (rc != MOE_OK) return rc;
+  for (int t = 0; t < T; ++t) {
+    rc = fused_forward(d, L, x, Wr, table, out + (size_t)t * d.H, ws, nullptr, prof, ow, s, fmt, t, T);
+    if (rc != MOE_OK) return rc;
+  }
+  return MOE_OK;
 }
 
 bool use_prefill(int T, int path) {
@@ -534,11 +575,12 @@ int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path) {
   if (T < 0 || path < MOE_PATH_AUTO || path > MOE_PATH_PREFILL) return MOE_ERR_BAD_ARG;
   if (T == 0) return 0;
   if (use_prefill(T, path)) return 9;  // quant, router, top-k, bucket, gather, maps, 2 GEMMs, combine
-  if (T == 1) {
+  if (T == 1 || (path == MOE_PATH_AUTO && T <= kDecodeTMax)) {
     FusedArgs fa{};
     size_t smem = 0;
     int grid = 0;
-    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return 1;
+    // one fused launch; a batch: the routing kernel, then one per token
+    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return T == 1 ? 1 : 1 + T;
   }
   return 3 * ((T + kDecodeTMax - 1) / kDecodeTMax);
 }
@@ -668,7 +710,7 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
 // status word and the router's arrival counter for this call.
 static int forward_checked(const moe_dims &d, int32_t T, const float *x, const float *Wr, const void *const *expert_table,
                     float *out, void *ws, int32_t *route_counts_opt, bool pf, const WsLayout &L, bool zeroed,
-                    cudaStream_t s, const Owned &ow) {
+                    cudaStream_t s, const Owned &ow, bool auto_path = true) {
   int rc = MOE_OK;
   if (!zeroed) {
     // status word and the router's arrival counter start at zero on every call
@@ -680,6 +722,9 @@ static int forward_checked(const moe_dims &d, int32_t T, const float *x, const f
   unsigned long long *prof = prof_next();
   if (T == 1) {
     rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
+    if (rc != kFusedNA) return rc;
+  } else if (auto_path && T <= kDecodeTMax) {
+    rc = fused_batch_forward(d, T, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
     if (rc != kFusedNA) return rc;
   }
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
@@ -706,7 +751,7 @@ int moe_layer_forward(const moe_dims *dims, int32_t T, const float *x, const flo
   const WsLayout L = ws_layout(*dims, T, pf);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
   return forward_checked(*dims, T, x, Wr, expert_table, out, ws, route_counts_opt, pf, L, false,
-                         static_cast<cudaStream_t>(stream), all_owned(*dims));
+                         static_cast<cudaStream_t>(stream), all_owned(*dims), path == MOE_PATH_AUTO);
 }
 
 int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
@@ -728,27 +773,33 @@ int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, con
     if (!fused_usable(*dims, kFmtMxfp4, &fa, &smem, &grid)) return MOE_ERR_SHAPE;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // the status word once per call; the fused kernel's control words per token
   cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
   if (err != cudaSuccess) return cuda_status(err);
   unsigned long long *prof = prof_next();
-  for (int t = 0; t < T; ++t) {
-    if (t > 0) {
-      err = cudaMemsetAsync(at<unsigned char>(ws, L.ctrl), 0, L.xin - L.ctrl, s);
-      if (err != cudaSuccess) return cuda_status(err);
+  if (T == 1 || T > kDecodeTMax) {
+    // token by token with the kernel's own routing (every token's control
+    // words zeroed before its launch)
+    for (int t = 0; t < T; ++t) {
+      if (t > 0) {
+        err = cudaMemsetAsync(at<unsigned char>(ws, L.ctrl), 0, L.xin - L.ctrl, s);
+        if (err != cudaSuccess) return cuda_status(err);
+      }
+      // token t in the per-token rows of the workspace; the pair rows are reused
+      WsLayout Lt = L;
+      Lt.xq += (size_t)t * dims->H;
+      Lt.xd += (size_t)t * (dims->H / 32) * 4;
+      Lt.logits += (size_t)t * dims->E * 4;
+      Lt.idx += (size_t)t * dims->k * 4;
+      Lt.w += (size_t)t * dims->k * 4;
+      rc = fused_forward(*dims, Lt, x + (size_t)t * dims->H, Wr, expert_table, out + (size_t)t * dims->H, ws,
+                         route_counts_opt, t == 0 ? prof : nullptr, all_owned(*dims), s, kFmtMxfp4);
+      if (rc != MOE_OK) return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
     }
-    // token t in the per-token rows of the workspace; the pair rows are reused
-    WsLayout Lt = L;
-    Lt.xq += (size_t)t * dims->H;
-    Lt.xd += (size_t)t * (dims->H / 32) * 4;
-    Lt.logits += (size_t)t * dims->E * 4;
-    Lt.idx += (size_t)t * dims->k * 4;
-    Lt.w += (size_t)t * dims->k * 4;
-    rc = fused_forward(*dims, Lt, x + (size_t)t * dims->H, Wr, expert_table, out + (size_t)t * dims->H, ws,
-                       route_counts_opt, t == 0 ? prof : nullptr, all_owned(*dims), s, kFmtMxfp4);
-    if (rc != MOE_OK) return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
+    return MOE_OK;
   }
-  return MOE_OK;
+  rc = fused_batch_forward(*dims, T, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, all_owned(*dims), s,
+                           kFmtMxfp4);
+  return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
 }
 
 int moe_layer_forward_ep(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
@@ -856,7 +907,7 @@ int moe_layer_forward_host(const moe_dims *dims, int32_t T, const float *x_host,
   if (err != cudaSuccess) return cuda_status(err);
   float *out_target = (out_dev_view != nullptr && aligned(out_dev_view, 16)) ? out_dev_view : yd;
   rc = forward_checked(*dims, T, xd, Wr, expert_table, out_target, ws, route_counts_opt, pf, L, true, s,
-                       all_owned(*dims));
+                       all_owned(*dims), path == MOE_PATH_AUTO);
   if (rc != MOE_OK) return rc;
   if (out_target == out_dev_view) return MOE_OK;
   return cuda_status(cudaMemcpyAsync(out_host, yd, bytes, cudaMemcpyDeviceToHost, s));

@@ -209,29 +209,29 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
     return;
   }
 
-  // ---------------------------------------------------------------- consumers
-  const int c0 = lane * CSZ;
-  // single token: this lane's activation chunk stays in registers
-  uint32_t act1[CSZ][16];
-  float d1[CSZ][2];
-  int z1[CSZ][2];
-  if (ONE) load_act<CSZ>(xq_s + (size_t)lane * pl.chp, xd_s, qs_s, c0, G, act1, d1, z1);
-  // this warp's rows of a stage
-  int row_m[RPW], row_r[RPW];
+  if (!ONE) {
+    // ------------------------------------------------------ consumers, batch
+    // unit by unit: a slot with one token (most routed slots of a small
+    // batch) keeps that token's activation chunk in registers for the unit and
+    // sums each row's chunks once per unit, as the single-token kernel does;
+    // a slot with several tokens runs them per stage against the rows in
+    // registers.  Each unit ends with every consumer warp at a named barrier
+    // (h = SiLU(g) * u and its Q8_0 per token), so all warps work on the same
+    // unit and share the red and gu buffers by unit.
+    const int c0 = lane * CSZ;
+    int row_m[RPW], row_r[RPW];
 #pragma unroll
-  for (int q = 0; q < RPW; ++q) {
-    const int jr = warp + NW * q;
-    row_m[q] = jr / R;
-    row_r[q] = jr % R;
-  }
-
-  int n_tok = 0, pos_base = 0, my_tok = 0;
-  int slot = u_begin / rbs, rb = u_begin % rbs, st = 0, s = 0;
-  int cu = 0;  // units this CTA has completed
-  uint32_t ph = 0;
-  bool bad = false;
-  for (int j = 0; j < n_stages; ++j) {
-    if (st == 0) {  // a new unit: its expert's token list
+    for (int q = 0; q < RPW; ++q) {
+      const int jr = warp + NW * q;
+      row_m[q] = jr / R;
+      row_r[q] = jr % R;
+    }
+    float *redw = red + (size_t)warp * (2 * T > 8 ? 2 * T : 8) * 33;
+    int slot = u_begin / rbs, rb = u_begin % rbs, s = 0;
+    uint32_t ph = 0;
+    bool bad = false;
+    for (int u = u_begin; u < u_end; ++u) {
+      int n_tok, pos_base, my_tok;
       const int so = a.own[slot];
       if (so == 0) {
         n_tok = T;
@@ -243,6 +243,149 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
         n_tok = a.off[e + 1] - pos_base;
         my_tok = lane < n_tok ? a.pair_tok[pos_base + lane] : 0;
       }
+      if (n_tok == 1) {
+        const int t = __shfl_sync(0xffffffffu, my_tok, 0);
+        uint32_t act1[CSZ][16];
+        float d1[CSZ][2];
+        int z1[CSZ][2];
+        load_act<CSZ>(xq_s + (size_t)(t * 32 + lane) * pl.chp, xd_s + t * HB, qs_s + t * HB, c0, G, act1, d1, z1);
+        for (int st = 0; st < SPU; ++st) {
+          if (!bad) bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int *>(&s_abort) != 0);
+          if (!bad) {
+            bad = !mbar_wait(full + s, ph, a.status, kDetGuFull, a.wait_limit);
+            bad = __any_sync(0xffffffffu, bad);
+            if (bad && lane == 0) s_abort = 1;
+          }
+          if (!bad) {
+            const unsigned char *sb = stg + (size_t)s * pl.sb;
+            uint32_t wv[RPW][CSZ][8];
+            float sc[RPW][CSZ];
+#pragma unroll
+            for (int q = 0; q < RPW; ++q)
+              load_row<CSZ>(sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2),
+                            reinterpret_cast<const __half *>(sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) +
+                                                             (size_t)row_r[q] * (H / 32)),
+                            c0, G, wv[q], sc[q]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
+#pragma unroll
+            for (int q = 0; q < RPW; ++q)
+              redw[(st * RPW + q) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act1, d1, z1, c0, G);
+          }
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+        if (!bad) {
+          // the warp's PWR rows of the unit: one chunk sum each
+          __syncwarp();
+          if (lane < PWR) {
+            const int sq = lane / RPW, q = lane % RPW;
+            const int jr = warp + NW * q;
+            gu[(jr / R) * 32 + sq * R + jr % R] = chunk_sum(redw + lane * 33, nch);
+          }
+        }
+      } else {
+        for (int st = 0; st < SPU; ++st) {
+          if (!bad) bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int *>(&s_abort) != 0);
+          if (!bad) {
+            bad = !mbar_wait(full + s, ph, a.status, kDetGuFull, a.wait_limit);
+            bad = __any_sync(0xffffffffu, bad);
+            if (bad && lane == 0) s_abort = 1;
+          }
+          if (!bad) {
+            const unsigned char *sb = stg + (size_t)s * pl.sb;
+            uint32_t wv[RPW][CSZ][8];
+            float sc[RPW][CSZ];
+#pragma unroll
+            for (int q = 0; q < RPW; ++q)
+              load_row<CSZ>(sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2),
+                            reinterpret_cast<const __half *>(sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) +
+                                                             (size_t)row_r[q] * (H / 32)),
+                            c0, G, wv[q], sc[q]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
+            for (int i = 0; i < n_tok; ++i) {
+              const int t = __shfl_sync(0xffffffffu, my_tok, i);
+              uint32_t act[CSZ][16];
+              float dd[CSZ][2];
+              int zz[CSZ][2];
+              load_act<CSZ>(xq_s + (size_t)(t * 32 + lane) * pl.chp, xd_s + t * HB, qs_s + t * HB, c0, G,
+                            act, dd, zz);
+#pragma unroll
+              for (int q = 0; q < RPW; ++q)
+                redw[(q * T + i) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act, dd, zz, c0, G);
+            }
+            __syncwarp();
+            if (lane < RPW * n_tok) {
+              const int q = lane / n_tok, i = lane % n_tok;
+              const int jr = warp + NW * q;
+              gu[(i * 2 + jr / R) * 32 + st * R + jr % R] = chunk_sum(redw + (q * T + i) * 33, nch);
+            }
+            __syncwarp();
+          }
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      // unit complete: h = SiLU(g) * u for its 32 rows, Q8_0 per token
+      named_sync(1, NCT);
+      if (!bad) {
+        for (int i = warp; i < n_tok; i += NW) {
+          const float g = gu[(i * 2 + 0) * 32 + lane];
+          const float uv = gu[(i * 2 + 1) * 32 + lane];
+          const float h = swiglu(g, uv);
+          const float d = fdiv(warp_max(fabsf(h)), 127.0f);
+          const int q = q8_code(h, d);
+          const int pos = pos_base + i;
+          a.hq[(size_t)pos * I + rb * 32 + lane] = (int8_t)q;
+          int qsum = q;
+#pragma unroll
+          for (int off = 16; off >= 1; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
+          if (lane == 0) {
+            a.hd[(size_t)pos * (I / 32) + rb] = d;
+            a.hqs[(size_t)pos * (I / 32) + rb] = qsum;
+          }
+        }
+      }
+      named_sync(1, NCT);
+      if (++rb == rbs) {
+        rb = 0;
+        ++slot;
+      }
+    }
+    prof_end(a.prof, 1);
+    return;
+  }
+
+  // ------------------------------------------------------ consumers, one token
+  const int c0 = lane * CSZ;
+  // this lane's activation chunk stays in registers
+  uint32_t act1[CSZ][16];
+  float d1[CSZ][2];
+  int z1[CSZ][2];
+  load_act<CSZ>(xq_s + (size_t)lane * pl.chp, xd_s, qs_s, c0, G, act1, d1, z1);
+  // this warp's rows of a stage
+  int row_m[RPW], row_r[RPW];
+#pragma unroll
+  for (int q = 0; q < RPW; ++q) {
+    const int jr = warp + NW * q;
+    row_m[q] = jr / R;
+    row_r[q] = jr % R;
+  }
+
+  int pos_base = 0;
+  int slot = u_begin / rbs, rb = u_begin % rbs, st = 0, s = 0;
+  int cu = 0;  // units this CTA has completed
+  uint32_t ph = 0;
+  bool bad = false;
+  for (int j = 0; j < n_stages; ++j) {
+    if (st == 0) {  // a new unit: its expert's position
+      const int so = a.own[slot];
+      pos_base = so == 0 ? a.k : a.off[a.uni[so - 1]];
     }
     if (!bad) bad = __any_sync(0xffffffffu, *reinterpret_cast<volatile int *>(&s_abort) != 0);
     if (!bad) {
@@ -262,7 +405,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
                       c0, G, wv[q], sc[q]);
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
-      if (ONE) {
+      {
         // chunk values of the warp's PWR rows of the unit, summed once per unit
 #pragma unroll
         for (int q = 0; q < RPW; ++q)
@@ -276,28 +419,9 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
           }
           __syncwarp();
         }
-      } else {
-        for (int i = 0; i < n_tok; ++i) {
-          const int t = __shfl_sync(0xffffffffu, my_tok, i);
-          uint32_t act[CSZ][16];
-          float dd[CSZ][2];
-          int zz[CSZ][2];
-          load_act<CSZ>(xq_s + (size_t)(t * 32 + lane) * pl.chp, xd_s + t * HB, qs_s + t * HB, c0, G,
-                        act, dd, zz);
-#pragma unroll
-          for (int q = 0; q < RPW; ++q)
-            red[((warp * 2 + q) * T + i) * 33 + lane] = chunk_dot<CSZ>(wv[q], sc[q], act, dd, zz, c0, G);
-        }
-        __syncwarp();
-        if (lane < RPW * n_tok) {
-          const int q = lane / n_tok, i = lane % n_tok;
-          const int jr = warp + 8 * q;
-          gu[(i * 2 + jr / R) * 32 + st * R + jr % R] = chunk_sum(red + ((warp * 2 + q) * T + i) * 33, nch);
-        }
-        __syncwarp();
       }
     }
-    if (ONE && st == SPU - 1) {
+    if (st == SPU - 1) {
       // unit complete: one warp (rotating with the unit) waits for the
       // others' g and u sums and forms h = SiLU(g) * u and its Q8_0 block;
       // the rest arrive and go on to the next unit.  The sums sit in one of
@@ -326,28 +450,6 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
         named_arrive(2 + par, NCT);
       }
       ++cu;
-    } else if (st == SPU - 1) {
-      // unit complete: h = SiLU(g) * u for its 32 rows, Q8_0 per token
-      named_sync(1, 256);
-      if (!bad) {
-        for (int i = warp; i < n_tok; i += 8) {
-          const float g = gu[(i * 2 + 0) * 32 + lane];
-          const float u = gu[(i * 2 + 1) * 32 + lane];
-          const float h = swiglu(g, u);
-          const float d = fdiv(warp_max(fabsf(h)), 127.0f);
-          const int q = q8_code(h, d);
-          const int pos = pos_base + i;
-          a.hq[(size_t)pos * I + rb * 32 + lane] = (int8_t)q;
-          int qsum = q;
-#pragma unroll
-          for (int off = 16; off >= 1; off >>= 1) qsum += __shfl_xor_sync(0xffffffffu, qsum, off);
-          if (lane == 0) {
-            a.hd[(size_t)pos * (I / 32) + rb] = d;
-            a.hqs[(size_t)pos * (I / 32) + rb] = qsum;
-          }
-        }
-      }
-      named_sync(1, 256);
     }
     if (++s == NS) {
       s = 0;
@@ -361,7 +463,7 @@ __global__ void __launch_bounds__(NW * 32 + 32, 1) k_gateup_decode(GateUpArgs a)
       }
     }
   }
-  if (ONE) named_sync(1, NCT);  // the end stamp follows the last unit's epilogue
+  named_sync(1, NCT);  // the end stamp follows the last unit's epilogue
   prof_end(a.prof, 1);
 }
 
@@ -644,8 +746,8 @@ __global__ void __launch_bounds__(288, 1) k_down_decode(DownArgs a) {
       // this warp's rows of the stage: a contiguous block
       const int rpw = (nr + 7) >> 3;
       const int ra = min(nr, warp * rpw), rz = min(nr, ra + rpw);
-      if (ONE) {
-        // one pair per slot: activation chunk in registers for the stage
+      if (ONE || n_tok == 1) {
+        // one pair in the slot: activation chunk in registers for the stage
         uint32_t av[CSZ][16];
         float dv[CSZ][2];
         int zv[CSZ][2];

@@ -79,7 +79,7 @@ __host__ __device__ inline FuPlan fu_plan(int H, int I, int E, int k, int rows_m
   p.bars = o;
   o += al128d((size_t)16 * (2 * ns + 2));
   p.misc = o;
-  o += al128d((size_t)4 * (8 + 5 * (kMaxK + 1)));
+  o += al128d((size_t)4 * (8 + 6 * (kMaxK + 1)));
   p.tab = o;
   o += al128d((size_t)8 * (E + 1));
   p.red = o;
@@ -152,6 +152,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   int *s_idx = s_ppos + (kMaxK + 1);              // [k] selected experts in slot order
   float *s_w = reinterpret_cast<float *>(s_idx + (kMaxK + 1));  // [k] softmax weights
   int *s_own = s_idx + 2 * (kMaxK + 1);           // [k + 1] the slots this call computes
+  int *s_bpos = s_own + (kMaxK + 1);              // [k + 1] slot -> row of hq / hd / hqs
   const unsigned char **s_tab = reinterpret_cast<const unsigned char **>(smem + pl.tab);  // [E + 1]
   float *red = reinterpret_cast<float *>(smem + pl.red);
   float *gu = reinterpret_cast<float *>(smem + pl.gu);
@@ -174,26 +175,30 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     fence_barrier_init();
   }
   __syncthreads();
+  // routed mode: the routing kernel of this call failed -- leave everything
+  // untouched (one decision for the whole CTA)
+  if (a.routed && __syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   prof_start(a.prof, 0);
 
   // ---------------------------------------------------------------- routing
   // this CTA's router rows [e0, e1) and x, staged in the (still idle) ring
   const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
-  const int nr = e1 - e0;
+  const int nr = a.routed ? 0 : e1 - e0;
   float *rx = reinterpret_cast<float *>(stg);
   float *rw = rx + H;
-  if (tid == 0) {
+  if (tid == 0 && !a.routed) {
     mbar_arrive_expect_tx(rbar, (uint32_t)(1 + nr) * (uint32_t)H * 4u);
     bulk_g2s(rx, a.x, (uint32_t)H * 4u, rbar);
     if (nr > 0) bulk_g2s(rw, a.Wr + (size_t)e0 * H, (uint32_t)nr * (uint32_t)H * 4u, rbar);
   }
   // the expert table, for the stream that follows the union
   for (int e = tid; e <= E; e += kFuThreads) s_tab[e] = static_cast<const unsigned char *>(a.table[e]);
-  const bool ok = mbar_wait(rbar, 0, a.status, kDetFuRoute, lim);
+  const bool ok = a.routed || mbar_wait(rbar, 0, a.status, kDetFuRoute, lim);
   if (!__syncthreads_and(ok)) {
     if (tid == 0) mbar_drain(rbar, 0, a.status, kDetFuRouteDrain);  // the copies land before exit
     return;
   }
+  if (!a.routed) {
   if (warp == PROD && lane == 0 && a.with_shared) {
     // a slice of the shared expert's blob into L2 while the grid routes (after
     // this CTA's routing data, which it must not delay)
@@ -251,6 +256,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   }
   __syncthreads();
   if (*s_abort) return;  // nothing in flight: the staging copies have landed
+  }  // !a.routed: the routing record and the Q8_0 codes of x come from the workspace
 
   if (warp != 0) {
     // the Q8_0 codes of x (every CTA's share, from L2) into this CTA's
@@ -278,11 +284,19 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
 
   // top-k, softmax and the union -- the same in every CTA
   if (warp == 0) {
-    int e_sel;
-    float l_sel;
-    warp_topk(a.logits, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red));
-    warp_softmax_store(0, K, lane, e_sel, l_sel, s_idx, s_w, blockIdx.x == 0 ? a.route_counts : nullptr,
-                       nullptr);
+    int e_sel = 0;
+    if (a.routed) {
+      if (lane < K) {
+        e_sel = a.idx[lane];
+        s_idx[lane] = e_sel;
+        s_w[lane] = a.w[lane];
+      }
+    } else {
+      float l_sel;
+      warp_topk(a.logits, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red));
+      warp_softmax_store(0, K, lane, e_sel, l_sel, s_idx, s_w, blockIdx.x == 0 ? a.route_counts : nullptr,
+                         nullptr);
+    }
     __syncwarp();
     // one token: the union is the k selected experts in ascending order;
     // pair s sits at position rank(e_s), the shared expert's pair at k
@@ -291,8 +305,12 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       for (int q = 0; q < K; ++q) rank += s_idx[q] < e_sel ? 1 : 0;
       s_uni[1 + rank] = e_sel;
       s_ppos[lane] = rank;
+      s_bpos[1 + rank] = a.routed ? a.pos_t[lane] : rank;
     }
-    if (lane == 0) s_uni[0] = E;
+    if (lane == 0) {
+      s_uni[0] = E;
+      s_bpos[0] = a.routed ? a.shared_pos : K;
+    }
     __syncwarp();
     // the slots this call computes (expert parallelism: the shared expert on
     // one rank, the routed experts in [e_lo, e_hi); by default all of them)
@@ -375,14 +393,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
             asm volatile("fence.proxy.async.global;" ::: "memory");
             seen = slot;
           }
-          const int pos_base = slot == 0 ? K : slot - 1;
+          const int hrow = s_bpos[slot];
           mbar_arrive_expect_tx(full + s, bp + bs + hq_b + 2 * hd_b);
           bulk_g2s_hint(dst, blob + 2 * mg + (size_t)(m0 + r0) * (I / 2), bp, full + s, pol);
           bulk_g2s_hint(dst + (size_t)RS * (I / 2), blob + 2 * mg + (size_t)H * (I / 2) + (size_t)(m0 + r0) * (I / 32),
                         bs, full + s, pol);
-          bulk_g2s(dst + hoff, a.hq + (size_t)pos_base * I, hq_b, full + s);
-          bulk_g2s(dst + hoff + hq_b, a.hd + (size_t)pos_base * IB, hd_b, full + s);
-          bulk_g2s(dst + hoff + hq_b + hd_b, a.hqs + (size_t)pos_base * IB, hd_b, full + s);
+          bulk_g2s(dst + hoff, a.hq + (size_t)hrow * I, hq_b, full + s);
+          bulk_g2s(dst + hoff + hq_b, a.hd + (size_t)hrow * IB, hd_b, full + s);
+          bulk_g2s(dst + hoff + hq_b + hd_b, a.hqs + (size_t)hrow * IB, hd_b, full + s);
         }
         issued = j + 1;
         if (++s == NS) {
@@ -411,15 +429,15 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       if (__any_sync(0xffffffffu, *s_abort != 0)) continue;  // one decision per warp
       const int u = (int)blockIdx.x + G * cu;
       const int slot = s_own[u / rbs], rb = u % rbs;
-      const int pos_base = slot == 0 ? K : slot - 1;
+      const int hrow = s_bpos[slot];
       const float h = swiglu(g, uv);
       const float d = fdiv(warp_max(fabsf(h)), 127.0f);
       const int q = q8_code(h, d);
-      a.hq[(size_t)pos_base * I + rb * 32 + lane] = (int8_t)q;
+      a.hq[(size_t)hrow * I + rb * 32 + lane] = (int8_t)q;
       const int qsum = __reduce_add_sync(0xffffffffu, q);
       if (lane == 0) {
-        a.hd[(size_t)pos_base * IB + rb] = d;
-        a.hqs[(size_t)pos_base * IB + rb] = qsum;
+        a.hd[(size_t)hrow * IB + rb] = d;
+        a.hqs[(size_t)hrow * IB + rb] = qsum;
       }
       __syncwarp();
       if (lane == 0) red_release_add(a.slot_done + slot, 1);
@@ -560,7 +578,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       if (s_idx[q] >= a.e_lo && s_idx[q] < a.e_hi) o = ffma(s_w[q], ysm[(size_t)s_ppos[q] * a.rows_max + i], o);
     a.out[m0 + i] = o;
   }
-  if (blockIdx.x == 0 && warp == 0) {
+  if (blockIdx.x == 0 && warp == 0 && !a.routed) {
     // the routing record of the workspace, as the routing kernel writes it
     // (read by no one in this kernel: written last)
     if (lane < K) {

@@ -23,6 +23,9 @@ constexpr int kProfWords = 8;                          // per record: 4 phases x
 // routing kernel's arrival ticket, [1] the fused kernel's routing arrivals,
 // [kCtrlSlot0 + s] gate/up units completed for union slot s (fused kernel).
 constexpr int kCtrlSlot0 = 4;
+// Control words per token of a decode batch (token t's block at kCtrlWords t;
+// the fused kernel's per-token launches each use their own block).
+constexpr int kCtrlWords = kCtrlSlot0 + kMaxK + 1;
 // Expert weight formats of the decode kernels.
 constexpr int kFmtInt4 = 0;   // int4 gs64, fp16 group scales
 constexpr int kFmtMxfp4 = 1;  // E2M1 codes, one E8M0 exponent per 32-block
@@ -98,7 +101,7 @@ inline WsLayout ws_layout(const moe_dims &d, int T, bool prefill = false) {
     return at;
   };
   L.status = seg(16);
-  L.ctrl = seg((size_t)(kCtrlSlot0 + kMaxK + 1) * 4);
+  L.ctrl = seg((size_t)kCtrlWords * 4 * (size_t)(T < 1 ? 1 : (T < kDecodeTMax ? T : kDecodeTMax)));
   L.xin = seg((size_t)T * d.H * 4);
   L.yout = seg((size_t)T * d.H * 4);
   L.xq = seg((size_t)T * d.H);
@@ -259,6 +262,13 @@ struct FusedArgs {
   int e_lo, e_hi;          // routed experts this call computes (expert parallelism)
   int with_shared;         // and the shared expert
   int fmt;                 // kFmtInt4 or kFmtMxfp4
+  // routed mode (a batch, token by token): the routing kernel has written the
+  // batch's record; this launch takes token t's Q8_0 codes (xq, xd), its top-k
+  // (idx, w) and its pairs' batch positions (pos_t [k], shared_pos) from it,
+  // writes h at those positions and leaves the record as it is
+  int routed;
+  const int32_t *pos_t;
+  int shared_pos;
   long long wait_limit;
   unsigned long long *prof;
 };

@@ -320,7 +320,9 @@ def test_fused_one_token_equals_three_kernel_path(H, I, E, k, seed):
     x, Wr, blobs = mi.make_layer(w, 0, DEV)
     d = moe.dims(H, I, E, k)
     assert moe.moe_layer_launches(d, 1) == 1
-    assert moe.moe_layer_launches(d, 2) == 3
+    assert moe.moe_layer_launches(d, 2) == 3          # routing kernel + one fused launch per token
+    assert moe.moe_layer_launches(d, 5) == 6
+    assert moe.moe_layer_launches(d, 2, 1) == 3       # MOE_PATH_DECODE: routing, gate/up, down
     out_f, ws_f, _ = gpu_layer(w, x, Wr, blobs)
     ws_s = moe.alloc_workspace(d, 1)
     out_s = torch.full_like(out_f, float("nan"))
@@ -355,3 +357,40 @@ def test_fused_route_counts_and_repeat():
     io, _ = orc.topk_softmax(orc.router_logits(x.cpu().numpy(), Wr.cpu().numpy()), w.k)
     assert np.array_equal(cnt.cpu().numpy(), 3 * np.bincount(io.reshape(-1), minlength=w.E))
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+# ----------------------------------------------------------------- small batches, token by token
+@pytest.mark.parametrize("name,T", [("medium", 2), ("medium", 5), ("tiny", 7), ("glm", 4), ("glm", 16)])
+def test_batch_token_by_token_equals_union_kernels(name, T):
+    """2 <= T <= 16 on the auto path: the routing kernel writes the batch's
+    record, then the fused kernel runs once per token (routed mode) and writes
+    each pair's h codes at the batch position.  MOE_PATH_DECODE runs the same
+    batch through the union's gate/up and down kernels.  Both compute every
+    (token, slot) pair with the same per-row code and order, so the outputs,
+    the routing record and the h codes agree bit for bit."""
+    moe = _moe()
+    from tests._common import ws_trace
+    if name == "glm":
+        w = mi.shrink(mi.WORKLOADS["decode"], T=T, seed=950 + T)
+    elif name == "tiny":
+        w = mi.shrink(mi.WORKLOADS["tiny"], T=T, seed=960 + T)
+    else:
+        w = mi.Workload("tok", H=1024, I=256, E=64, k=8, T=T, seed=970 + T)
+    x, Wr, blobs = mi.make_layer(w, 0, DEV, T=T)
+    d = moe.dims(w.H, w.I, w.E, w.k)
+    counts = torch.zeros(w.E, dtype=torch.int32, device=DEV)
+    table = moe.expert_table(blobs)
+    out_a = torch.full((T, w.H), float("nan"), dtype=torch.float32, device=DEV)
+    ws_a = moe.alloc_workspace(d, T)
+    moe.moe_layer_forward(d, x, Wr, table, out_a, ws_a, route_counts=counts)
+    out_b, ws_b, _ = gpu_layer(w, x, Wr, blobs, path=1)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a, out_b)
+    ta, tb = ws_trace(ws_a, d, T), ws_trace(ws_b, d, T)
+    for key in ("status", "xq", "xd", "logits", "idx", "w", "cnt", "off", "uni", "perm", "pos", "pair_tok", "hq",
+                "hd"):
+        assert np.array_equal(ta[key], tb[key]), key
+    # the routing kernel counted each selection once
+    assert np.array_equal(counts.cpu().numpy(), np.bincount(ta["idx"].reshape(-1), minlength=w.E))
+    if name != "glm":
+        _check_layer(w, x, Wr, blobs)
