@@ -57,6 +57,8 @@ def parse():
                     help="routed experts per layer (profiling: a small pool, same per-step work)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="prefill batch size (profiling a small case; default: the workload's 2048)")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="default workload: leave out the prefill sub-object of the line")
     return ap.parse_args()
 
 
@@ -580,7 +582,25 @@ def run_prefill(args, ws_n, rank, local):
         union=n_u, routing_counts=counts, us_per_token_layer=round(max_ms / K / T * 1e3, 3),
         attainable=attainable(ops, n_u, w.blob_bytes, peaks()[0], peak, max_ms / K),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clk.summary(),
-        gpu_launches=10 * K)
+        gpu_launches=moe.moe_layer_launches(d, T, PF) * K)
+
+
+def prefill_summary(args, rank, local) -> dict:
+    """The prefill layer (2048 tokens, Zipf(1.1) routing) as a sub-object of the
+    default line: a short run of its own (3 warm-up, 5 timed steps), with the
+    oracle timed on sampled tokens."""
+    a = argparse.Namespace(**vars(args))
+    a.workload, a.steps, a.warmup, a.experts, a.tokens = "prefill", 5, 3, None, None
+    a.cpu_seconds = min(args.cpu_seconds, 10.0)
+    r = run_prefill(a, 1, rank, local)
+    peak, _ = tensor_peak()
+    return {"metric": "prefill layer int8-equivalent TOPS", "value": r["value"], "unit": "TOPS",
+            "ms_per_step": r["ms_per_step"], "steps": a.steps, "warmup": a.warmup,
+            "frac_of_fp16_peak": round(r["value"] / peak, 4), "frac_of_int8_peak": round(r["value"] / (2 * peak), 4),
+            "peak_tflops_fp16": peak, "attainable": r["attainable"], "roofline": r["roofline"],
+            "kernels": r["kernels"], "e2e": r["e2e"], "cpu_baseline": r["cpu_baseline"], "dtype": r["dtype"],
+            "config": r["config"], "union": r["union"], "routing_counts": r["routing_counts"],
+            "clocks": r["clocks"], "gpu_launches": r["gpu_launches"]}
 
 
 def oracle_prefill_sample(w, x_h, Wr_h, blob_fn, budget_s: float, tokens_max: int = 64):
@@ -877,6 +897,8 @@ def main():
     try:
         fn = {"prefill": run_prefill, "stacked": run_stacked, "tiered": run_tiered}.get(args.workload, run_native)
         res = fn(args, ws_n, rank, local)
+        if args.workload == "decode" and ws_n == 1 and not args.no_prefill:
+            res["prefill"] = prefill_summary(args, rank, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
