@@ -808,7 +808,10 @@ def run_tiered(args, ws_n, rank, local):
                                          what="device stamps: routing kernel, gate/up, down, and the "
                                               "span from routing's first CTA to down's last (misses' "
                                               "copies and the host's acquire fall inside it)"),
-                clocks=clk.summary(), gpu_launches=None)
+                clocks=clk.summary(),
+                # per token: every layer's routing, gate/up and down kernels, plus the
+                # next layer's prediction router for all but the last layer
+                gpu_launches=n_tok * (3 * L + (L - 1)))
 
 
 # ----------------------------------------------------------------- reference arm
