@@ -293,13 +293,14 @@ bool fused_usable(const moe_dims &d, int fmt, FusedArgs *fa, size_t *smem, int *
   return fits[dev][fmt];
 }
 
-// One launch of the fused kernel.  tok < 0: the whole layer for one token
-// (its own routing).  tok >= 0: token tok of a batch of T whose routing record
-// the routing kernel has written (routed mode); out is that token's row.
+// One launch of the fused kernel.  batch_T == 0: the whole layer for one
+// token (its own routing).  batch_T >= 1: the batch of batch_T tokens whose
+// routing record the routing kernel has written (routed mode), all tokens in
+// this one launch.
 int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
                   const void *const *table, float *out, void *ws, int32_t *counts,
                   unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4,
-                  int tok = -1, int T = 1) {
+                  int batch_T = 0) {
   FusedArgs fa{};
   size_t smem = 0;
   int sms = 0;
@@ -333,28 +334,24 @@ int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const fl
   fa.with_shared = ow.shared;
   fa.wait_limit = wait_limit_cycles();
   fa.prof = prof;
-  if (tok >= 0) {
-    const size_t t = (size_t)tok;
+  if (batch_T > 0) {
     fa.routed = 1;
-    fa.xq = p.xq + t * d.H;
-    fa.xd = p.xd + t * (d.H / 32);
-    fa.idx = p.idx + t * d.k;
-    fa.w = p.w + t * d.k;
-    fa.pos_t = p.pos + t * d.k;
-    fa.shared_pos = T * d.k + tok;
+    fa.ntok = batch_T;
+    fa.pos_t = p.pos;
+    fa.shared_pos = batch_T * d.k;
     fa.route_counts = nullptr;  // counted by the routing kernel
-    fa.slot_done = at<int32_t>(ws, L.ctrl) + t * kCtrlWords + kCtrlSlot0;
   }
   return cuda_status(launch_decode_fused(fa, sms, smem, s));
 }
 
-// A decode batch of 2 <= T <= kDecodeTMax tokens through the fused kernel,
-// token by token: the routing kernel writes the batch's record (codes of x,
-// top-k, union, pair positions), then one fused launch per token streams that
-// token's experts and writes its h codes at the batch's pair positions.  At
-// these batch sizes the union of the batch is nearly the sum of the tokens'
-// selections, so the per-token stream costs few extra bytes and runs at the
-// fused kernel's rate.  kFusedNA if the fused kernel does not fit the shape.
+// A decode batch of 2 <= T <= kDecodeTMax tokens through the fused kernel:
+// the routing kernel writes the batch's record (codes of x, top-k, union, pair
+// positions), then one fused launch streams the tokens' experts one token
+// after the other (the ring never drains between them) and writes each pair's
+// h codes at the batch's pair position.  At these batch sizes the union of the
+// batch is nearly the sum of the tokens' selections, so streaming per token
+// costs few extra bytes and runs at the fused kernel's rate.  kFusedNA if the
+// fused kernel does not fit the shape.
 int fused_batch_forward(const moe_dims &d, int T, const WsLayout &L, const float *x, const float *Wr,
                         const void *const *table, float *out, void *ws, int32_t *counts,
                         unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4) {
@@ -364,13 +361,9 @@ int fused_batch_forward(const moe_dims &d, int T, const WsLayout &L, const float
     int sms = 0;
     if (!fused_usable(d, fmt, &fa, &smem, &sms)) return kFusedNA;
   }
-  int rc = route_chunk(d, 0, T, L, x, Wr, ws, counts, prof, ow, s);
+  const int rc = route_chunk(d, 0, T, L, x, Wr, ws, counts, prof, ow, s);
   if (rc != MOE_OK) return rc;
-  for (int t = 0; t < T; ++t) {
-    rc = fused_forward(d, L, x, Wr, table, out + (size_t)t * d.H, ws, nullptr, prof, ow, s, fmt, t, T);
-    if (rc != MOE_OK) return rc;
-  }
-  return MOE_OK;
+  return fused_forward(d, L, x, Wr, table, out, ws, nullptr, prof, ow, s, fmt, T);
 }
 
 bool use_prefill(int T, int path) {
@@ -579,8 +572,8 @@ int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path) {
     FusedArgs fa{};
     size_t smem = 0;
     int grid = 0;
-    // one fused launch; a batch: the routing kernel, then one per token
-    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return T == 1 ? 1 : 1 + T;
+    // one fused launch; a batch: the routing kernel, then one fused launch
+    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return T == 1 ? 1 : 2;
   }
   return 3 * ((T + kDecodeTMax - 1) / kDecodeTMax);
 }

@@ -49,13 +49,14 @@ constexpr int kFuRPW = 2 * kFuR / kFuNW; // rows per warp per gate/up stage
 constexpr int kFuPWR = kFuSPU * kFuRPW;  // rows per warp per unit
 constexpr int kFuNCT = kFuNW * 32;       // consumer threads
 constexpr int kFuWarps = kFuNW + 2;      // + the producer warp and the epilogue warp
+constexpr int kFuTMax = kDecodeTMax;     // tokens of one routed launch
 constexpr int kFuThreads = kFuWarps * 32;
 // named barriers (0 is __syncthreads): the consumers' end, and per unit parity
 // the hand-off of the g and u sums to the epilogue warp and the buffer's return
 constexpr int kBarEnd = 1, kBarGuFull = 2, kBarGuFree = 4;
 
 struct FuPlan {
-  size_t bars, misc, tab, red, gu, ysm, xd, qs, xq, stg, total;
+  size_t bars, misc, red, gu, ysm, xd, qs, xq, stg, total;
   uint32_t sb;    // bytes of one ring stage
   int chp;        // bytes of one lane's activation chunk
   int rw;         // red rows per warp
@@ -79,9 +80,7 @@ __host__ __device__ inline FuPlan fu_plan(int H, int I, int E, int k, int rows_m
   p.bars = o;
   o += al128d((size_t)16 * (2 * ns + 2));
   p.misc = o;
-  o += al128d((size_t)4 * (8 + 6 * (kMaxK + 1)));
-  p.tab = o;
-  o += al128d((size_t)8 * (E + 1));
+  o += al128d((size_t)4 * (8 + kFuTMax + 6 * kFuTMax * (k + 1)));
   p.red = o;
   o += al128d((size_t)kFuNW * p.rw * 33 * 4);
   p.gu = o;
@@ -147,13 +146,16 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   uint64_t *rbar = empty + NS;
   int *misc = reinterpret_cast<int *>(smem + pl.misc);
   volatile int *s_abort = misc;
-  int *s_uni = misc + 8;                          // [k + 1] slot -> expert (slot 0 = shared)
-  int *s_ppos = s_uni + (kMaxK + 1);              // [k] pair s -> position
-  int *s_idx = s_ppos + (kMaxK + 1);              // [k] selected experts in slot order
-  float *s_w = reinterpret_cast<float *>(s_idx + (kMaxK + 1));  // [k] softmax weights
-  int *s_own = s_idx + 2 * (kMaxK + 1);           // [k + 1] the slots this call computes
-  int *s_bpos = s_own + (kMaxK + 1);              // [k + 1] slot -> row of hq / hd / hqs
-  const unsigned char **s_tab = reinterpret_cast<const unsigned char **>(smem + pl.tab);  // [E + 1]
+  // per token t of this launch (stride SW = k + 1):
+  const int NT = a.routed ? a.ntok : 1;
+  const int SW = K + 1;
+  int *t_nsl = misc + 8;                           // [NT] slots computed
+  int *t_uni = t_nsl + kFuTMax;                    // [NT][k + 1] slot -> expert (slot 0 = shared)
+  int *t_ppos = t_uni + kFuTMax * SW;              // [NT][k] pair s -> slot - 1
+  int *t_idx = t_ppos + kFuTMax * SW;              // [NT][k] selected experts in pair order
+  float *t_w = reinterpret_cast<float *>(t_idx + kFuTMax * SW);  // [NT][k] softmax weights
+  int *t_own = t_idx + 2 * kFuTMax * SW;           // [NT][k + 1] the slots computed, in order
+  int *t_bpos = t_own + kFuTMax * SW;              // [NT][k + 1] slot -> row of hq / hd / hqs
   float *red = reinterpret_cast<float *>(smem + pl.red);
   float *gu = reinterpret_cast<float *>(smem + pl.gu);
   float *ysm = reinterpret_cast<float *>(smem + pl.ysm);
@@ -191,8 +193,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     bulk_g2s(rx, a.x, (uint32_t)H * 4u, rbar);
     if (nr > 0) bulk_g2s(rw, a.Wr + (size_t)e0 * H, (uint32_t)nr * (uint32_t)H * 4u, rbar);
   }
-  // the expert table, for the stream that follows the union
-  for (int e = tid; e <= E; e += kFuThreads) s_tab[e] = static_cast<const unsigned char *>(a.table[e]);
   const bool ok = a.routed || mbar_wait(rbar, 0, a.status, kDetFuRoute, lim);
   if (!__syncthreads_and(ok)) {
     if (tid == 0) mbar_drain(rbar, 0, a.status, kDetFuRouteDrain);  // the copies land before exit
@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   if (warp == PROD && lane == 0 && a.with_shared) {
     // a slice of the shared expert's blob into L2 while the grid routes (after
     // this CTA's routing data, which it must not delay)
-    const unsigned char *sh = s_tab[E];
+    const unsigned char *sh = static_cast<const unsigned char *>(a.table[E]);
     const size_t bytes = 2 * ((size_t)I * (H / 2) + (size_t)I * (H / 64) * 2) +
                          ((size_t)H * (I / 2) + (size_t)H * (I / 64) * 2);
     const size_t slice = ((bytes + G - 1) / G + 15) / 16 * 16;
@@ -258,11 +258,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   if (*s_abort) return;  // nothing in flight: the staging copies have landed
   }  // !a.routed: the routing record and the Q8_0 codes of x come from the workspace
 
-  if (warp != 0) {
-    // the Q8_0 codes of x (every CTA's share, from L2) into this CTA's
-    // activation chunks, with the block scales and code sums
-    for (int b = tid - 32; b < HB; b += kFuThreads - 32) {
-      const uint4 *src = reinterpret_cast<const uint4 *>(a.xq + (size_t)b * 32);
+  // the Q8_0 codes of a token (every CTA's share, from L2) into this CTA's
+  // activation chunks, with the block scales and code sums; threads
+  // [first, first + nthr)
+  auto load_token = [&](int t, int first, int nthr) {
+    const int8_t *xq_t = a.xq + (size_t)t * H;
+    const float *xd_t = a.xd + (size_t)t * HB;
+    for (int b = tid - first; b < HB; b += nthr) {
+      const uint4 *src = reinterpret_cast<const uint4 *>(xq_t + (size_t)b * 32);
       const uint4 q0 = __ldcg(src), q1 = __ldcg(src + 1);
       int sum = 0;
       sum = __dp4a((int)q0.x, 0x01010101, sum);
@@ -277,75 +280,98 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       uint4 *dst = reinterpret_cast<uint4 *>(xq_s + (size_t)c * pl.chp + (size_t)(g - c * CSZG) * 64 + (h & 63));
       dst[0] = q0;
       dst[1] = q1;
-      xd_s[b] = __ldcg(a.xd + b);
+      xd_s[b] = __ldcg(xd_t + b);
       qs_s[b] = sum;
     }
-  }
+  };
+  if (warp != 0) load_token(0, 32, kFuThreads - 32);
 
-  // top-k, softmax and the union -- the same in every CTA
+  // top-k, softmax and the union of every token -- the same in every CTA
   if (warp == 0) {
-    int e_sel = 0;
-    if (a.routed) {
-      if (lane < K) {
-        e_sel = a.idx[lane];
-        s_idx[lane] = e_sel;
-        s_w[lane] = a.w[lane];
+    for (int t = 0; t < NT; ++t) {
+      int *su = t_uni + t * SW, *sp = t_ppos + t * SW, *si = t_idx + t * SW, *so = t_own + t * SW;
+      int *sbp = t_bpos + t * SW;
+      float *sw = t_w + t * SW;
+      int e_sel = 0;
+      if (a.routed) {
+        if (lane < K) {
+          e_sel = a.idx[(size_t)t * K + lane];
+          si[lane] = e_sel;
+          sw[lane] = a.w[(size_t)t * K + lane];
+        }
+      } else {
+        float l_sel;
+        warp_topk(a.logits, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red));
+        warp_softmax_store(0, K, lane, e_sel, l_sel, si, sw, blockIdx.x == 0 ? a.route_counts : nullptr,
+                           nullptr);
       }
-    } else {
-      float l_sel;
-      warp_topk(a.logits, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red));
-      warp_softmax_store(0, K, lane, e_sel, l_sel, s_idx, s_w, blockIdx.x == 0 ? a.route_counts : nullptr,
-                         nullptr);
-    }
-    __syncwarp();
-    // one token: the union is the k selected experts in ascending order;
-    // pair s sits at position rank(e_s), the shared expert's pair at k
-    if (lane < K) {
-      int rank = 0;
-      for (int q = 0; q < K; ++q) rank += s_idx[q] < e_sel ? 1 : 0;
-      s_uni[1 + rank] = e_sel;
-      s_ppos[lane] = rank;
-      s_bpos[1 + rank] = a.routed ? a.pos_t[lane] : rank;
-    }
-    if (lane == 0) {
-      s_uni[0] = E;
-      s_bpos[0] = a.routed ? a.shared_pos : K;
-    }
-    __syncwarp();
-    // the slots this call computes (expert parallelism: the shared expert on
-    // one rank, the routed experts in [e_lo, e_hi); by default all of them)
-    if (lane == 0) {
-      int n = 0;
-      if (a.with_shared) s_own[n++] = 0;
-      for (int i = 1; i <= K; ++i)
-        if (s_uni[i] >= a.e_lo && s_uni[i] < a.e_hi) s_own[n++] = i;
-      misc[1] = n;
+      __syncwarp();
+      // one token: the union is the k selected experts in ascending order;
+      // pair s sits at slot 1 + rank(e_s), the shared expert at slot 0
+      if (lane < K) {
+        int rank = 0;
+        for (int q = 0; q < K; ++q) rank += si[q] < e_sel ? 1 : 0;
+        su[1 + rank] = e_sel;
+        sp[lane] = rank;
+        sbp[1 + rank] = a.routed ? a.pos_t[(size_t)t * K + lane] : rank;
+      }
+      if (lane == 0) {
+        su[0] = E;
+        sbp[0] = a.routed ? a.shared_pos + t : K;
+      }
+      __syncwarp();
+      // the slots this call computes (expert parallelism: the shared expert on
+      // one rank, the routed experts in [e_lo, e_hi); by default all of them)
+      if (lane == 0) {
+        int n = 0;
+        if (a.with_shared) so[n++] = 0;
+        for (int i = 1; i <= K; ++i)
+          if (su[i] >= a.e_lo && su[i] < a.e_hi) so[n++] = i;
+        t_nsl[t] = n;
+      }
+      __syncwarp();
     }
   }
   __syncthreads();
   prof_end(a.prof, 0);
   prof_start(a.prof, 1);
 
-  const int nslot = misc[1];  // slots this call computes
   const int rbs = I / 32;     // 32-row units per expert
-  const int n_units = nslot * rbs;
-  const int my_units = (int)blockIdx.x < n_units ? (n_units - 1 - (int)blockIdx.x) / G + 1 : 0;
-  const int n_gu = my_units * SPU;
+  // token t's units (slot, 32-row block) are dealt round-robin from CTA r_t,
+  // r_t = the units of the tokens before it, mod G, so the CTAs stay balanced
+  // over the launch; this CTA's first unit of token t is u0, then u0 + G, ...
+  auto units_of = [&](int t, int r, int &u0) -> int {
+    const int nu = t_nsl[t] * rbs;
+    u0 = (int)blockIdx.x - r;
+    if (u0 < 0) u0 += G;
+    return u0 < nu ? (nu - 1 - u0) / G + 1 : 0;
+  };
+  int units_all = 0;  // this CTA's units over the launch
+  {
+    int r = 0;
+    for (int t = 0; t < NT; ++t) {
+      int u0;
+      units_all += units_of(t, r, u0);
+      r = (r + t_nsl[t] * rbs) % G;
+    }
+  }
   const int nrg = H / a.rg;
   const int m0 = (int)((long long)blockIdx.x * nrg / G) * a.rg;
   const int m1 = (int)((long long)(blockIdx.x + 1) * nrg / G) * a.rg;
   const int nrows = m1 - m0;
   const int RS = a.rs;
   const int nsub = (nrows + RS - 1) / RS;
-  const int n_dn = nrows > 0 ? nslot * nsub : 0;
-  const int n_st = n_gu + n_dn;
   const size_t mg = (size_t)I * H / 2 + (size_t)I * H / 32;  // bytes of the gate (= up) matrix
+  auto blob_of = [&](int e) { return static_cast<const unsigned char *>(a.table[e]); };
 
   // every blob this grid reads must be 16-byte aligned (TMA bulk copies)
   {
     bool bad = false;
-    for (int sl = tid; sl < nslot; sl += kFuThreads)
-      bad |= (reinterpret_cast<uintptr_t>(s_tab[s_uni[s_own[sl]]]) & 15u) != 0;
+    for (int i = tid; i < NT * SW; i += kFuThreads) {
+      const int t = i / SW, sl = i % SW;
+      if (sl < t_nsl[t])
+        bad |= (reinterpret_cast<uintptr_t>(blob_of(t_uni[t * SW + t_own[t * SW + sl]])) & 15u) != 0;
+    }
     if (__syncthreads_or(bad)) {
       if (tid == 0) set_status(a.status, MOE_ERR_DEVICE, kDetFuAlign);
       return;
@@ -358,54 +384,77 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
       const uint64_t pol = policy_evict_first();
       const uint32_t pk = (uint32_t)R * (H / 2), sk = (uint32_t)R * (H / 32);
       const uint32_t hoff = (uint32_t)RS * fu_dn_row(I), hq_b = (uint32_t)I, hd_b = (uint32_t)IB * 4u;
-      int s = 0, issued = 0, seen = -1;  // seen: the last slot found published
+      int s = 0, issued = 0, r = 0;
       uint32_t ph = 0;
-      for (int j = 0; j < n_st; ++j) {
-        if (j >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetFuEmpty, lim)) {
-          *s_abort = 1;
-          break;
-        }
-        if (*s_abort) break;
-        unsigned char *dst = stg + (size_t)s * pl.sb;
-        if (j < n_gu) {
-          const int u = (int)blockIdx.x + G * (j / SPU), st = j % SPU;
-          const int slot = s_own[u / rbs], rb = u % rbs;
-          const unsigned char *blob = s_tab[s_uni[slot]];
-          const size_t n0 = (size_t)rb * 32 + (size_t)st * R;
-          mbar_arrive_expect_tx(full + s, 2 * (pk + sk));
-          bulk_g2s_hint(dst, blob + n0 * (H / 2), pk, full + s, pol);
-          bulk_g2s_hint(dst + pk, blob + mg + n0 * (H / 2), pk, full + s, pol);
-          bulk_g2s_hint(dst + 2 * pk, blob + (size_t)I * (H / 2) + n0 * (H / 32), sk, full + s, pol);
-          bulk_g2s_hint(dst + 2 * pk + sk, blob + mg + (size_t)I * (H / 2) + n0 * (H / 32), sk, full + s, pol);
-        } else {
-          const int jd = j - n_gu, slot = s_own[jd / nsub], r0 = (jd % nsub) * RS;
-          const int nr_ = min(RS, nrows - r0);
-          const unsigned char *blob = s_tab[s_uni[slot]];
-          const uint32_t bp = (uint32_t)nr_ * (I / 2), bs = (uint32_t)nr_ * (I / 32);
-          if (slot != seen) {
-            // every gate/up unit of the slot published its h codes (acquire);
-            // then the copy engine may read them (proxy fence)
-            if (!wait_count(a.slot_done + slot, rbs, lim)) {
-              set_status(a.status, MOE_ERR_TIMEOUT, kDetFuSlot);
-              *s_abort = 1;
-              break;
-            }
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            seen = slot;
+      bool stop = false;
+      for (int t = 0; t < NT && !stop; ++t) {
+        const int *su = t_uni + t * SW, *so = t_own + t * SW, *sbp = t_bpos + t * SW;
+        const int32_t *sdone = a.slot_done + (size_t)t * kCtrlWords;
+        int u0;
+        const int mu = units_of(t, r, u0);
+        r = (r + t_nsl[t] * rbs) % G;
+        const int n_gu = mu * SPU, n_dn = nrows > 0 ? t_nsl[t] * nsub : 0;
+        int seen = -1;  // the last slot found published
+        int bslot = -1;
+        const unsigned char *blob = nullptr;
+        for (int j = 0; j < n_gu + n_dn; ++j) {
+          if (issued >= NS && !mbar_wait(empty + s, ph ^ 1u, a.status, kDetFuEmpty, lim)) {
+            *s_abort = 1;
+            stop = true;
+            break;
           }
-          const int hrow = s_bpos[slot];
-          mbar_arrive_expect_tx(full + s, bp + bs + hq_b + 2 * hd_b);
-          bulk_g2s_hint(dst, blob + 2 * mg + (size_t)(m0 + r0) * (I / 2), bp, full + s, pol);
-          bulk_g2s_hint(dst + (size_t)RS * (I / 2), blob + 2 * mg + (size_t)H * (I / 2) + (size_t)(m0 + r0) * (I / 32),
-                        bs, full + s, pol);
-          bulk_g2s(dst + hoff, a.hq + (size_t)hrow * I, hq_b, full + s);
-          bulk_g2s(dst + hoff + hq_b, a.hd + (size_t)hrow * IB, hd_b, full + s);
-          bulk_g2s(dst + hoff + hq_b + hd_b, a.hqs + (size_t)hrow * IB, hd_b, full + s);
-        }
-        issued = j + 1;
-        if (++s == NS) {
-          s = 0;
-          ph ^= 1u;
+          if (*s_abort) {
+            stop = true;
+            break;
+          }
+          unsigned char *dst = stg + (size_t)s * pl.sb;
+          if (j < n_gu) {
+            const int u = u0 + G * (j / SPU), st = j % SPU;
+            const int slot = so[u / rbs], rb = u % rbs;
+            if (slot != bslot) {
+              bslot = slot;
+              blob = blob_of(su[slot]);
+            }
+            const size_t n0 = (size_t)rb * 32 + (size_t)st * R;
+            mbar_arrive_expect_tx(full + s, 2 * (pk + sk));
+            bulk_g2s_hint(dst, blob + n0 * (H / 2), pk, full + s, pol);
+            bulk_g2s_hint(dst + pk, blob + mg + n0 * (H / 2), pk, full + s, pol);
+            bulk_g2s_hint(dst + 2 * pk, blob + (size_t)I * (H / 2) + n0 * (H / 32), sk, full + s, pol);
+            bulk_g2s_hint(dst + 2 * pk + sk, blob + mg + (size_t)I * (H / 2) + n0 * (H / 32), sk, full + s, pol);
+          } else {
+            const int jd = j - n_gu, slot = so[jd / nsub], r0 = (jd % nsub) * RS;
+            const int nr_ = min(RS, nrows - r0);
+            if (slot != bslot) {
+              bslot = slot;
+              blob = blob_of(su[slot]);
+            }
+            const uint32_t bp = (uint32_t)nr_ * (I / 2), bs = (uint32_t)nr_ * (I / 32);
+            if (slot != seen) {
+              // every gate/up unit of the slot published its h codes (acquire);
+              // then the copy engine may read them (proxy fence)
+              if (!wait_count(sdone + slot, rbs, lim)) {
+                set_status(a.status, MOE_ERR_TIMEOUT, kDetFuSlot);
+                *s_abort = 1;
+                stop = true;
+                break;
+              }
+              asm volatile("fence.proxy.async.global;" ::: "memory");
+              seen = slot;
+            }
+            const int hrow = sbp[slot];
+            mbar_arrive_expect_tx(full + s, bp + bs + hq_b + 2 * hd_b);
+            bulk_g2s_hint(dst, blob + 2 * mg + (size_t)(m0 + r0) * (I / 2), bp, full + s, pol);
+            bulk_g2s_hint(dst + (size_t)RS * (I / 2), blob + 2 * mg + (size_t)H * (I / 2) + (size_t)(m0 + r0) * (I / 32),
+                          bs, full + s, pol);
+            bulk_g2s(dst + hoff, a.hq + (size_t)hrow * I, hq_b, full + s);
+            bulk_g2s(dst + hoff + hq_b, a.hd + (size_t)hrow * IB, hd_b, full + s);
+            bulk_g2s(dst + hoff + hq_b + hd_b, a.hqs + (size_t)hrow * IB, hd_b, full + s);
+          }
+          ++issued;
+          if (++s == NS) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
       }
       for (int j = (issued > NS ? issued - NS : 0); j < issued; ++j)
@@ -416,118 +465,143 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
 
   if (warp == EPI) {
     // ---------------------------------------------------------------- epilogue
-    // per gate/up unit of this CTA: wait for the consumers' g and u sums (two
-    // buffers by unit parity), free the buffer, form h = SiLU(g) * u and its
-    // Q8_0 block, store them and count the unit on its slot (release), so that
-    // the consumers never wait on this work
-    for (int cu = 0; cu < my_units; ++cu) {
-      const int par = cu & 1;
-      named_sync(kBarGuFull + par, NCT + 32);
-      const float *gb = gu + par * 64;
-      const float g = gb[lane], uv = gb[32 + lane];
-      if (cu + 2 < my_units) named_arrive(kBarGuFree + par, NCT + 32);
-      if (__any_sync(0xffffffffu, *s_abort != 0)) continue;  // one decision per warp
-      const int u = (int)blockIdx.x + G * cu;
-      const int slot = s_own[u / rbs], rb = u % rbs;
-      const int hrow = s_bpos[slot];
-      const float h = swiglu(g, uv);
-      const float d = fdiv(warp_max(fabsf(h)), 127.0f);
-      const int q = q8_code(h, d);
-      a.hq[(size_t)hrow * I + rb * 32 + lane] = (int8_t)q;
-      const int qsum = __reduce_add_sync(0xffffffffu, q);
-      if (lane == 0) {
-        a.hd[(size_t)hrow * IB + rb] = d;
-        a.hqs[(size_t)hrow * IB + rb] = qsum;
+    // per gate/up unit of this CTA (tokens in order): wait for the consumers'
+    // g and u sums (two buffers by unit parity), free the buffer, form h =
+    // SiLU(g) * u and its Q8_0 block, store them and count the unit on its
+    // slot (release), so that the consumers never wait on this work
+    int cu = 0, r = 0;
+    for (int t = 0; t < NT; ++t) {
+      const int *so = t_own + t * SW, *sbp = t_bpos + t * SW;
+      int32_t *sdone = a.slot_done + (size_t)t * kCtrlWords;
+      int u0;
+      const int mu = units_of(t, r, u0);
+      r = (r + t_nsl[t] * rbs) % G;
+      for (int c = 0; c < mu; ++c, ++cu) {
+        const int par = cu & 1;
+        named_sync(kBarGuFull + par, NCT + 32);
+        const float *gb = gu + par * 64;
+        const float g = gb[lane], uv = gb[32 + lane];
+        if (cu + 2 < units_all) named_arrive(kBarGuFree + par, NCT + 32);
+        if (__any_sync(0xffffffffu, *s_abort != 0)) continue;  // one decision per warp
+        const int u = u0 + G * c;
+        const int slot = so[u / rbs], rb = u % rbs;
+        const int hrow = sbp[slot];
+        const float h = swiglu(g, uv);
+        const float d = fdiv(warp_max(fabsf(h)), 127.0f);
+        const int q = q8_code(h, d);
+        a.hq[(size_t)hrow * I + rb * 32 + lane] = (int8_t)q;
+        const int qsum = __reduce_add_sync(0xffffffffu, q);
+        if (lane == 0) {
+          a.hd[(size_t)hrow * IB + rb] = d;
+          a.hqs[(size_t)hrow * IB + rb] = qsum;
+        }
+        __syncwarp();
+        if (lane == 0) red_release_add(sdone + slot, 1);
       }
-      __syncwarp();
-      if (lane == 0) red_release_add(a.slot_done + slot, 1);
     }
     return;
   }
 
   // ------------------------------------------------------------------ consumers
+  // Tokens in order: gate/up units, down rows, then (after every consumer
+  // warp is done with the token) the combine of this CTA's output rows.  On an
+  // abort the warps run through the remaining hand-offs without waiting on
+  // stages, so the epilogue warp's named barriers always find them.
   float *redw = red + (size_t)warp * pl.rw * 33;
   bool bad = false;
-  int s = 0;
+  int s = 0, cu = 0, r = 0;
   uint32_t ph = 0;
-  {
-    // gate/up: this CTA's units in round-robin order; one token, so the
-    // lane's activation chunk stays in registers for the whole phase
-    const int c0 = lane * CSZG;
-    uint32_t act1[CSZG][16];
-    float d1[CSZG][2];
-    int z1[CSZG][2];
-    load_act<CSZG>(xq_s + (size_t)lane * pl.chp, xd_s, qs_s, c0, GG, act1, d1, z1);
-    int row_m[RPW], row_r[RPW];
+  int row_m[RPW], row_r[RPW];
 #pragma unroll
-    for (int q = 0; q < RPW; ++q) {
-      const int jr = warp + NW * q;
-      row_m[q] = jr / R;
-      row_r[q] = jr % R;
+  for (int q = 0; q < RPW; ++q) {
+    const int jr = warp + NW * q;
+    row_m[q] = jr / R;
+    row_r[q] = jr % R;
+  }
+  const int cg0 = lane * CSZG, cd0 = lane * CSZD;
+  const size_t hoff = (size_t)RS * fu_dn_row(I);
+  for (int t = 0; t < NT; ++t) {
+    const int *so = t_own + t * SW;
+    const int nsl = t_nsl[t];
+    int u0;
+    const int mu = units_of(t, r, u0);
+    r = (r + nsl * rbs) % G;
+    const int n_gu = mu * SPU, n_dn = nrows > 0 ? nsl * nsub : 0;
+    if (t > 0) {
+      // the next token's codes into the activation chunks, once every
+      // consumer is done with the last token (its combine included)
+      named_sync(kBarEnd, NCT);
+      load_token(t, 0, NCT);
+      named_sync(kBarEnd, NCT);
     }
-    for (int j = 0; j < n_gu; ++j) {
-      const int cu = j / SPU, st = j % SPU;
-      if (!bad) bad = __any_sync(0xffffffffu, *s_abort != 0);  // one decision per warp
-      if (!bad) {
-        bad = !mbar_wait(full + s, ph, a.status, kDetFuFull, lim);
-        bad = __any_sync(0xffffffffu, bad);
-        if (bad && lane == 0) *s_abort = 1;
-      }
-      if (!bad) {
-        const unsigned char *sb = stg + (size_t)s * pl.sb;
-        uint32_t wv[RPW][CSZG][8];
-        float sc[RPW][CSZG];
-        uint32_t ex[RPW][CSZG];
-#pragma unroll
-        for (int q = 0; q < RPW; ++q) {
-          const unsigned char *rowp = sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2);
-          const unsigned char *scp = sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) + (size_t)row_r[q] * (H / 32);
-          if constexpr (FMT == kFmtMxfp4)
-            load_row_mx<CSZG>(rowp, scp, c0, GG, wv[q], ex[q]);
-          else
-            load_row<CSZG>(rowp, reinterpret_cast<const __half *>(scp), c0, GG, wv[q], sc[q]);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
-#pragma unroll
-        for (int q = 0; q < RPW; ++q) {
-          if constexpr (FMT == kFmtMxfp4)
-            redw[(st * RPW + q) * 33 + lane] = chunk_dot_mx<CSZG>(wv[q], ex[q], act1, d1, c0, GG);
-          else
-            redw[(st * RPW + q) * 33 + lane] = chunk_dot<CSZG>(wv[q], sc[q], act1, d1, z1, c0, GG);
-        }
-      }
-      if (st == SPU - 1) {
-        // unit complete: this warp's g and u row sums into the unit's buffer
-        // (once the epilogue warp has read the unit two before), then handed on
-        const int par = cu & 1;
-        if (cu >= 2) named_sync(kBarGuFree + par, NCT + 32);
+    {
+      // gate/up: this CTA's units of the token; the lane's activation chunk
+      // stays in registers for the token's gate/up phase
+      uint32_t act1[CSZG][16];
+      float d1[CSZG][2];
+      int z1[CSZG][2];
+      load_act<CSZG>(xq_s + (size_t)lane * pl.chp, xd_s, qs_s, cg0, GG, act1, d1, z1);
+      for (int j = 0; j < n_gu; ++j) {
+        const int st = j % SPU;
+        if (!bad) bad = __any_sync(0xffffffffu, *s_abort != 0);  // one decision per warp
         if (!bad) {
+          bad = !mbar_wait(full + s, ph, a.status, kDetFuFull, lim);
+          bad = __any_sync(0xffffffffu, bad);
+          if (bad && lane == 0) *s_abort = 1;
+        }
+        if (!bad) {
+          const unsigned char *sb = stg + (size_t)s * pl.sb;
+          uint32_t wv[RPW][CSZG][8];
+          float sc[RPW][CSZG];
+          uint32_t ex[RPW][CSZG];
+#pragma unroll
+          for (int q = 0; q < RPW; ++q) {
+            const unsigned char *rowp = sb + (size_t)row_m[q] * R * (H / 2) + (size_t)row_r[q] * (H / 2);
+            const unsigned char *scp = sb + (size_t)R * H + (size_t)row_m[q] * R * (H / 32) + (size_t)row_r[q] * (H / 32);
+            if constexpr (FMT == kFmtMxfp4)
+              load_row_mx<CSZG>(rowp, scp, cg0, GG, wv[q], ex[q]);
+            else
+              load_row<CSZG>(rowp, reinterpret_cast<const __half *>(scp), cg0, GG, wv[q], sc[q]);
+          }
           __syncwarp();
-          if (lane < PWR) {
-            const int sq = lane / RPW, q = lane % RPW;
-            const int jr = warp + NW * q;
-            gu[par * 64 + (jr / R) * 32 + sq * R + jr % R] = chunk_sum(redw + lane * 33, nchg);
+          if (lane == 0) mbar_arrive(empty + s);  // the stage's rows are in registers
+#pragma unroll
+          for (int q = 0; q < RPW; ++q) {
+            if constexpr (FMT == kFmtMxfp4)
+              redw[(st * RPW + q) * 33 + lane] = chunk_dot_mx<CSZG>(wv[q], ex[q], act1, d1, cg0, GG);
+            else
+              redw[(st * RPW + q) * 33 + lane] = chunk_dot<CSZG>(wv[q], sc[q], act1, d1, z1, cg0, GG);
           }
         }
-        named_arrive(kBarGuFull + par, NCT + 32);
-      }
-      if (++s == NS) {
-        s = 0;
-        ph ^= 1u;
+        if (st == SPU - 1) {
+          // unit complete: this warp's g and u row sums into the unit's buffer
+          // (once the epilogue warp has read the unit two before), then handed on
+          const int par = cu & 1;
+          if (cu >= 2) named_sync(kBarGuFree + par, NCT + 32);
+          if (!bad) {
+            __syncwarp();
+            if (lane < PWR) {
+              const int sq = lane / RPW, q = lane % RPW;
+              const int jr = warp + NW * q;
+              gu[par * 64 + (jr / R) * 32 + sq * R + jr % R] = chunk_sum(redw + lane * 33, nchg);
+            }
+          }
+          named_arrive(kBarGuFull + par, NCT + 32);
+          ++cu;
+        }
+        if (++s == NS) {
+          s = 0;
+          ph ^= 1u;
+        }
       }
     }
-  }
-  if (n_gu > 0) prof_end(a.prof, 1);
-  if (n_dn > 0) prof_start(a.prof, 2);
-  {
-    // down: this CTA's output rows of every slot, shared expert first; each
-    // stage brings the slot's h codes with the weights (the producer issues it
-    // once the slot's units are all published)
-    const int c0 = lane * CSZD;
-    const size_t hoff = (size_t)RS * fu_dn_row(I);
+    if (t == NT - 1 && mu > 0) prof_end(a.prof, 1);
+    if (t == 0 && n_dn > 0) prof_start(a.prof, 2);
+    // down: this CTA's output rows of every slot of the token, shared expert
+    // first; each stage brings the slot's h codes with the weights (the
+    // producer issues it once the slot's units are all published)
     for (int jd = 0; jd < n_dn; ++jd) {
-      const int slot = s_own[jd / nsub], sub = jd % nsub;
+      const int slot = so[jd / nsub], sub = jd % nsub;
       const int r0 = sub * RS, nr_ = min(RS, nrows - r0);
       const int pos_base = slot == 0 ? K : slot - 1;
       if (!bad) bad = __any_sync(0xffffffffu, *s_abort != 0);  // one decision per warp
@@ -541,8 +615,8 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
         uint32_t av[CSZD][16];
         float dv[CSZD][2];
         int zv[CSZD][2];
-        load_act<CSZD>(sb + hoff + 64 * c0, reinterpret_cast<const float *>(sb + hoff + I),
-                       reinterpret_cast<const int *>(sb + hoff + I + (size_t)IB * 4), c0, GD, av, dv, zv);
+        load_act<CSZD>(sb + hoff + 64 * cd0, reinterpret_cast<const float *>(sb + hoff + I),
+                       reinterpret_cast<const int *>(sb + hoff + I + (size_t)IB * 4), cd0, GD, av, dv, zv);
         const int ra = warp * nr_ / NW, rz = (warp + 1) * nr_ / NW;  // this warp's rows of the stage
         for (int ml = ra; ml < rz; ++ml) {
           uint32_t wv[CSZD][8];
@@ -550,12 +624,12 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
           const unsigned char *scp = sb + (size_t)RS * (I / 2) + (size_t)ml * (I / 32);
           if constexpr (FMT == kFmtMxfp4) {
             uint32_t ex[CSZD];
-            load_row_mx<CSZD>(rowp, scp, c0, GD, wv, ex);
-            redw[(ml - ra) * 33 + lane] = chunk_dot_mx<CSZD>(wv, ex, av, dv, c0, GD);
+            load_row_mx<CSZD>(rowp, scp, cd0, GD, wv, ex);
+            redw[(ml - ra) * 33 + lane] = chunk_dot_mx<CSZD>(wv, ex, av, dv, cd0, GD);
           } else {
             float sc[CSZD];
-            load_row<CSZD>(rowp, reinterpret_cast<const __half *>(scp), c0, GD, wv, sc);
-            redw[(ml - ra) * 33 + lane] = chunk_dot<CSZD>(wv, sc, av, dv, zv, c0, GD);
+            load_row<CSZD>(rowp, reinterpret_cast<const __half *>(scp), cd0, GD, wv, sc);
+            redw[(ml - ra) * 33 + lane] = chunk_dot<CSZD>(wv, sc, av, dv, zv, cd0, GD);
           }
         }
         __syncwarp();
@@ -568,26 +642,30 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
         ph ^= 1u;
       }
     }
+    named_sync(kBarEnd, NCT);
+    if (!*s_abort) {
+      // combine, in the layer's order: shared expert, then the pairs by weight
+      const int *si = t_idx + t * SW, *sp = t_ppos + t * SW;
+      const float *sw = t_w + t * SW;
+      for (int i = tid; i < nrows; i += NCT) {
+        float o = a.with_shared ? ysm[(size_t)K * a.rows_max + i] : 0.0f;
+        for (int q = 0; q < K; ++q)
+          if (si[q] >= a.e_lo && si[q] < a.e_hi) o = ffma(sw[q], ysm[(size_t)sp[q] * a.rows_max + i], o);
+        a.out[(size_t)t * H + m0 + i] = o;
+      }
+    }
   }
-  named_sync(kBarEnd, NCT);
   if (*s_abort) return;
-  // combine, in the layer's order: shared expert, then the slots by weight
-  for (int i = tid; i < nrows; i += NCT) {
-    float o = a.with_shared ? ysm[(size_t)K * a.rows_max + i] : 0.0f;
-    for (int q = 0; q < K; ++q)
-      if (s_idx[q] >= a.e_lo && s_idx[q] < a.e_hi) o = ffma(s_w[q], ysm[(size_t)s_ppos[q] * a.rows_max + i], o);
-    a.out[m0 + i] = o;
-  }
-  if (blockIdx.x == 0 && warp == 0 && !a.routed) {
+  if (!a.routed && blockIdx.x == 0 && warp == 0) {
     // the routing record of the workspace, as the routing kernel writes it
     // (read by no one in this kernel: written last)
     if (lane < K) {
-      a.idx[lane] = s_idx[lane];
-      a.w[lane] = s_w[lane];
+      a.idx[lane] = t_idx[lane];
+      a.w[lane] = t_w[lane];
     }
     __syncwarp();
-    bucket_small_counts(E, K, s_idx, a.cnt, a.off, 0, 1);
-    bucket_small(E, K, 1, s_idx, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos, a.pair_tok);
+    bucket_small_counts(E, K, t_idx, a.cnt, a.off, 0, 1);
+    bucket_small(E, K, 1, t_idx, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos, a.pair_tok);
   }
   prof_end(a.prof, 2);
 }
