@@ -293,14 +293,13 @@ bool fused_usable(const moe_dims &d, int fmt, FusedArgs *fa, size_t *smem, int *
   return fits[dev][fmt];
 }
 
-// One launch of the fused kernel.  batch_T == 0: the whole layer for one
-// token (its own routing).  batch_T >= 1: the batch of batch_T tokens whose
-// routing record the routing kernel has written (routed mode), all tokens in
-// this one launch.
+// One launch of the fused kernel: the whole layer for T <= kDecodeTMax
+// tokens (their routing, the experts of each token streamed one token after
+// the other, the combine), in the workspace rows of layout L.
 int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
                   const void *const *table, float *out, void *ws, int32_t *counts,
                   unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4,
-                  int batch_T = 0) {
+                  int T = 1) {
   FusedArgs fa{};
   size_t smem = 0;
   int sms = 0;
@@ -334,36 +333,8 @@ int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const fl
   fa.with_shared = ow.shared;
   fa.wait_limit = wait_limit_cycles();
   fa.prof = prof;
-  if (batch_T > 0) {
-    fa.routed = 1;
-    fa.ntok = batch_T;
-    fa.pos_t = p.pos;
-    fa.shared_pos = batch_T * d.k;
-    fa.route_counts = nullptr;  // counted by the routing kernel
-  }
+  fa.ntok = T;
   return cuda_status(launch_decode_fused(fa, sms, smem, s));
-}
-
-// A decode batch of 2 <= T <= kDecodeTMax tokens through the fused kernel:
-// the routing kernel writes the batch's record (codes of x, top-k, union, pair
-// positions), then one fused launch streams the tokens' experts one token
-// after the other (the ring never drains between them) and writes each pair's
-// h codes at the batch's pair position.  At these batch sizes the union of the
-// batch is nearly the sum of the tokens' selections, so streaming per token
-// costs few extra bytes and runs at the fused kernel's rate.  kFusedNA if the
-// fused kernel does not fit the shape.
-int fused_batch_forward(const moe_dims &d, int T, const WsLayout &L, const float *x, const float *Wr,
-                        const void *const *table, float *out, void *ws, int32_t *counts,
-                        unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4) {
-  {
-    FusedArgs fa{};
-    size_t smem = 0;
-    int sms = 0;
-    if (!fused_usable(d, fmt, &fa, &smem, &sms)) return kFusedNA;
-  }
-  const int rc = route_chunk(d, 0, T, L, x, Wr, ws, counts, prof, ow, s);
-  if (rc != MOE_OK) return rc;
-  return fused_forward(d, L, x, Wr, table, out, ws, nullptr, prof, ow, s, fmt, T);
 }
 
 bool use_prefill(int T, int path) {
@@ -572,8 +543,8 @@ int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path) {
     FusedArgs fa{};
     size_t smem = 0;
     int grid = 0;
-    // one fused launch; a batch: the routing kernel, then one fused launch
-    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return T == 1 ? 1 : 2;
+    // one fused launch for the whole layer
+    if (fused_usable(*dims, kFmtInt4, &fa, &smem, &grid)) return 1;
   }
   return 3 * ((T + kDecodeTMax - 1) / kDecodeTMax);
 }
@@ -717,7 +688,11 @@ static int forward_checked(const moe_dims &d, int32_t T, const float *x, const f
     rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
     if (rc != kFusedNA) return rc;
   } else if (auto_path && T <= kDecodeTMax) {
-    rc = fused_batch_forward(d, T, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
+    // a small batch: one fused launch streams the tokens' experts one token
+    // after the other.  At these sizes the batch union is nearly the sum of
+    // the tokens' selections, so per-token streaming costs few extra bytes
+    // and runs at the fused kernel's rate.
+    rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s, kFmtInt4, T);
     if (rc != kFusedNA) return rc;
   }
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
@@ -790,8 +765,8 @@ int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, con
     }
     return MOE_OK;
   }
-  rc = fused_batch_forward(*dims, T, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, all_owned(*dims), s,
-                           kFmtMxfp4);
+  rc = fused_forward(*dims, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, all_owned(*dims), s, kFmtMxfp4,
+                     T);
   return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
 }
 

@@ -49,7 +49,10 @@ constexpr int kFuRPW = 2 * kFuR / kFuNW; // rows per warp per gate/up stage
 constexpr int kFuPWR = kFuSPU * kFuRPW;  // rows per warp per unit
 constexpr int kFuNCT = kFuNW * 32;       // consumer threads
 constexpr int kFuWarps = kFuNW + 2;      // + the producer warp and the epilogue warp
-constexpr int kFuTMax = kDecodeTMax;     // tokens of one routed launch
+constexpr int kFuTMax = kDecodeTMax;     // tokens of one launch
+// the red buffer (kFuNW x >= kFuPWR rows of 33 words) doubles as the batch
+// record's bucketing scratch (2 E words)
+static_assert(kFuNW * kFuPWR * 33 >= 2 * MOE_MAX_E, "bucketing scratch");
 constexpr int kFuThreads = kFuWarps * 32;
 // named barriers (0 is __syncthreads): the consumers' end, and per unit parity
 // the hand-off of the g and u sums to the epilogue warp and the buffer's return
@@ -132,7 +135,9 @@ __device__ __forceinline__ bool wait_count(const int32_t *p, int32_t target, lon
 // FMT: the expert weight format, kFmtInt4 (int4 gs64, fp16 group scales) or
 // kFmtMxfp4 (E2M1 codes, E8M0 exponent per 32-block); both hold K/2 code
 // bytes and K/32 scale bytes per row, so the stream is the same.
-template <int CSZG, int CSZD, int FMT>
+// MULTI: a batch of a.ntok tokens (> 1); the one-token instantiation has the
+// token loops compiled away (this kernel's instruction fetch is a bound).
+template <int CSZG, int CSZD, int FMT, bool MULTI>
 __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   constexpr int R = kFuR, NW = kFuNW, SPU = kFuSPU, RPW = kFuRPW, PWR = kFuPWR, NCT = kFuNCT;
   constexpr int PROD = NW, EPI = NW + 1;  // warp roles after routing
@@ -146,14 +151,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   uint64_t *rbar = empty + NS;
   int *misc = reinterpret_cast<int *>(smem + pl.misc);
   volatile int *s_abort = misc;
-  // per token t of this launch (stride SW = k + 1):
-  const int NT = a.routed ? a.ntok : 1;
+  // per token t of this launch (stride SW = k + 1, or k):
+  const int NT = MULTI ? a.ntok : 1;
   const int SW = K + 1;
   int *t_nsl = misc + 8;                           // [NT] slots computed
   int *t_uni = t_nsl + kFuTMax;                    // [NT][k + 1] slot -> expert (slot 0 = shared)
-  int *t_ppos = t_uni + kFuTMax * SW;              // [NT][k] pair s -> slot - 1
-  int *t_idx = t_ppos + kFuTMax * SW;              // [NT][k] selected experts in pair order
-  float *t_w = reinterpret_cast<float *>(t_idx + kFuTMax * SW);  // [NT][k] softmax weights
+  int *t_ppos = t_uni + kFuTMax * SW;              // [NT][k + 1] pair s -> slot - 1
+  int *t_idx = t_ppos + kFuTMax * SW;              // [NT * k] selected experts in pair order
+  float *t_w = reinterpret_cast<float *>(t_idx + kFuTMax * SW);  // [NT * k] softmax weights
   int *t_own = t_idx + 2 * kFuTMax * SW;           // [NT][k + 1] the slots computed, in order
   int *t_bpos = t_own + kFuTMax * SW;              // [NT][k + 1] slot -> row of hq / hd / hqs
   float *red = reinterpret_cast<float *>(smem + pl.red);
@@ -177,68 +182,88 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     fence_barrier_init();
   }
   __syncthreads();
-  // routed mode: the routing kernel of this call failed -- leave everything
-  // untouched (one decision for the whole CTA)
-  if (a.routed && __syncthreads_or(*reinterpret_cast<volatile int32_t *>(a.status) != 0)) return;
   prof_start(a.prof, 0);
 
   // ---------------------------------------------------------------- routing
-  // this CTA's router rows [e0, e1) and x, staged in the (still idle) ring
+  // this CTA's router rows [e0, e1) and the tokens' x rows, staged in the
+  // (still idle) ring: the x rows in chunks of as many tokens as the ring
+  // holds after the router rows (every token at once for small batches)
   const int e0 = (int)((long long)blockIdx.x * E / G), e1 = (int)((long long)(blockIdx.x + 1) * E / G);
-  const int nr = a.routed ? 0 : e1 - e0;
-  float *rx = reinterpret_cast<float *>(stg);
-  float *rw = rx + H;
-  if (tid == 0 && !a.routed) {
-    mbar_arrive_expect_tx(rbar, (uint32_t)(1 + nr) * (uint32_t)H * 4u);
-    bulk_g2s(rx, a.x, (uint32_t)H * 4u, rbar);
+  const int nr = e1 - e0;
+  float *rw = reinterpret_cast<float *>(stg);
+  float *rx = rw + (size_t)nr * H;
+  const int xcap = (int)(((size_t)NS * pl.sb - (size_t)nr * H * 4) / ((size_t)H * 4));  // >= 1 (fused_plan)
+  if (tid == 0) {
+    const int nx = NT < xcap ? NT : xcap;
+    mbar_arrive_expect_tx(rbar, (uint32_t)(nr + nx) * (uint32_t)H * 4u);
     if (nr > 0) bulk_g2s(rw, a.Wr + (size_t)e0 * H, (uint32_t)nr * (uint32_t)H * 4u, rbar);
+    bulk_g2s(rx, a.x, (uint32_t)nx * (uint32_t)H * 4u, rbar);
   }
-  const bool ok = a.routed || mbar_wait(rbar, 0, a.status, kDetFuRoute, lim);
-  if (!__syncthreads_and(ok)) {
-    if (tid == 0) mbar_drain(rbar, 0, a.status, kDetFuRouteDrain);  // the copies land before exit
-    return;
-  }
-  if (!a.routed) {
-  if (warp == PROD && lane == 0 && a.with_shared) {
-    // a slice of the shared expert's blob into L2 while the grid routes (after
-    // this CTA's routing data, which it must not delay)
-    const unsigned char *sh = static_cast<const unsigned char *>(a.table[E]);
-    const size_t bytes = 2 * ((size_t)I * (H / 2) + (size_t)I * (H / 64) * 2) +
-                         ((size_t)H * (I / 2) + (size_t)H * (I / 64) * 2);
-    const size_t slice = ((bytes + G - 1) / G + 15) / 16 * 16;
-    const size_t b0 = slice * blockIdx.x;
-    if ((reinterpret_cast<uintptr_t>(sh) & 15u) == 0 && b0 < bytes) {
-      const size_t n = bytes - b0 < slice ? bytes - b0 : slice;
-      asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sh + b0), "r"((uint32_t)n) : "memory");
+  const int nlp = nr * NT;  // (row, token) pairs of logits
+  for (int c0 = 0, ph = 0; c0 < NT; c0 += xcap, ph ^= 1) {
+    const int nx = NT - c0 < xcap ? NT - c0 : xcap;
+    const bool ok = mbar_wait(rbar, (uint32_t)ph, a.status, kDetFuRoute, lim);
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0) mbar_drain(rbar, (uint32_t)ph, a.status, kDetFuRouteDrain);  // the copies land before exit
+      return;
+    }
+    if (c0 == 0 && warp == PROD && lane == 0 && a.with_shared) {
+      // a slice of the shared expert's blob into L2 while the grid routes
+      // (after this CTA's routing data, which it must not delay)
+      const unsigned char *sh = static_cast<const unsigned char *>(a.table[E]);
+      const size_t bytes = 2 * ((size_t)I * (H / 2) + (size_t)I * (H / 64) * 2) +
+                           ((size_t)H * (I / 2) + (size_t)H * (I / 64) * 2);
+      const size_t slice = ((bytes + G - 1) / G + 15) / 16 * 16;
+      const size_t b0 = slice * blockIdx.x;
+      if ((reinterpret_cast<uintptr_t>(sh) & 15u) == 0 && b0 < bytes) {
+        const size_t n = bytes - b0 < slice ? bytes - b0 : slice;
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(sh + b0), "r"((uint32_t)n) : "memory");
+      }
+    }
+    // logits of this CTA's rows for the chunk's tokens, the router's fixed
+    // order: lane l sums h = l, l + 32, ... with fmaf, then an xor tree 16,
+    // 8, 4, 2, 1 (the producer and epilogue warps take rows too)
+    for (int p = warp; p < nr * nx; p += kFuWarps) {
+      const int r = p / nx, tc = p - r * nx;
+      const float *wv = rw + (size_t)r * H;
+      const float *xv = rx + (size_t)tc * H;
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int i = lane; i < H; i += 32) acc = ffma(xv[i], wv[i], acc);
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) acc = fadd(acc, __shfl_xor_sync(0xffffffffu, acc, off));
+      if (lane == 0) a.logits[(size_t)(c0 + tc) * E + e0 + r] = acc;
+    }
+    if (c0 + xcap < NT) {
+      // the next chunk of x rows, once every warp is done with this one
+      __syncthreads();
+      if (tid == 0) {
+        const int nn = NT - c0 - xcap < xcap ? NT - c0 - xcap : xcap;
+        mbar_arrive_expect_tx(rbar, (uint32_t)nn * (uint32_t)H * 4u);
+        bulk_g2s(rx, a.x + (size_t)(c0 + xcap) * H, (uint32_t)nn * (uint32_t)H * 4u, rbar);
+      }
     }
   }
-  // logits of this CTA's rows, the router's fixed order: lane l sums
-  // h = l, l + 32, ... with fmaf, then an xor tree 16, 8, 4, 2, 1 (the
-  // producer and epilogue warps take rows too)
-  for (int r = warp; r < nr; r += kFuWarps) {
-    const float *wv = rw + (size_t)r * H;
-    float acc = 0.0f;
-#pragma unroll 8
-    for (int i = lane; i < H; i += 32) acc = ffma(rx[i], wv[i], acc);
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) acc = fadd(acc, __shfl_xor_sync(0xffffffffu, acc, off));
-    if (lane == 0) a.logits[e0 + r] = acc;
-  }
-  // Q8_0 of x: this CTA's share of the blocks, into the workspace (every CTA
-  // reads all the codes back after the grid barrier); one warp per block
+  // Q8_0 of x: this CTA's share of the batch's blocks, into the workspace
+  // (every CTA reads the codes back after the grid barrier); one warp per block
   {
-    const int b0 = (int)((long long)blockIdx.x * HB / G), b1 = (int)((long long)(blockIdx.x + 1) * HB / G);
-    const int qw = (warp - nr % kFuWarps + kFuWarps) % kFuWarps;  // the warps after the logit rows first
+    const int NB = NT * HB;
+    const int c_last = ((NT - 1) / xcap) * xcap;  // first token of the staged chunk
+    const int b0 = (int)((long long)blockIdx.x * NB / G), b1 = (int)((long long)(blockIdx.x + 1) * NB / G);
+    const int qw = (warp - nlp % kFuWarps + kFuWarps) % kFuWarps;  // the warps after the logit rows first
     for (int b = b0 + qw; b < b1; b += kFuWarps) {
-      const float v = rx[b * 32 + lane];
+      const int t = b / HB, bb = b - t * HB;
+      // the last chunk's x rows are still staged; earlier ones come from L2
+      const float v = t >= c_last ? rx[(size_t)(t - c_last) * H + bb * 32 + lane]
+                                  : __ldg(a.x + (size_t)t * H + bb * 32 + lane);
       // the maximum of non-negative floats is the maximum of their bit patterns
       const float d = fdiv(__uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(v)))), 127.0f);
-      a.xq[b * 32 + lane] = (int8_t)q8_code(v, d);
-      if (lane == 0) a.xd[b] = d;
+      a.xq[(size_t)t * H + bb * 32 + lane] = (int8_t)q8_code(v, d);
+      if (lane == 0) a.xd[(size_t)t * HB + bb] = d;
     }
   }
-  // grid-wide: every CTA's logits are written before any CTA reads them (the
-  // barrier orders this CTA's writes before thread 0's release)
+  // grid-wide: every CTA's logits and codes are written before any CTA reads
+  // them (the barrier orders this CTA's writes before thread 0's release)
   __syncthreads();
   if (tid == 0) {
     red_release_add_u32(a.arrivals, 1u);
@@ -256,7 +281,6 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   }
   __syncthreads();
   if (*s_abort) return;  // nothing in flight: the staging copies have landed
-  }  // !a.routed: the routing record and the Q8_0 codes of x come from the workspace
 
   // the Q8_0 codes of a token (every CTA's share, from L2) into this CTA's
   // activation chunks, with the block scales and code sums; threads
@@ -286,50 +310,48 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   };
   if (warp != 0) load_token(0, 32, kFuThreads - 32);
 
-  // top-k, softmax and the union of every token -- the same in every CTA
-  if (warp == 0) {
-    for (int t = 0; t < NT; ++t) {
-      int *su = t_uni + t * SW, *sp = t_ppos + t * SW, *si = t_idx + t * SW, *so = t_own + t * SW;
-      int *sbp = t_bpos + t * SW;
-      float *sw = t_w + t * SW;
-      int e_sel = 0;
-      if (a.routed) {
-        if (lane < K) {
-          e_sel = a.idx[(size_t)t * K + lane];
-          si[lane] = e_sel;
-          sw[lane] = a.w[(size_t)t * K + lane];
-        }
-      } else {
-        float l_sel;
-        warp_topk(a.logits, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red));
-        warp_softmax_store(0, K, lane, e_sel, l_sel, si, sw, blockIdx.x == 0 ? a.route_counts : nullptr,
-                           nullptr);
+  // top-k and softmax of every token (one warp per token) -- the same in
+  // every CTA; CTA 0 counts the routes
+  for (int t = warp; t < NT; t += kFuWarps) {
+    int e_sel;
+    float l_sel;
+    warp_topk(a.logits + (size_t)t * E, E, K, lane, e_sel, l_sel, reinterpret_cast<uint32_t *>(red) + warp * 128);
+    warp_softmax_store(t, K, lane, e_sel, l_sel, t_idx, t_w, blockIdx.x == 0 ? a.route_counts : nullptr, nullptr);
+  }
+  // one token: the same warp builds its table; a batch: every token's top-k first
+  if (MULTI) __syncthreads(); else __syncwarp();
+  // each token's union (its k experts in ascending order: pair s at slot
+  // 1 + rank(e_s), the shared expert at slot 0), the rows its h codes take in
+  // the batch's pair order (the counting sort of the T k pairs by expert), and
+  // the slots this call computes (expert parallelism: the shared expert on one
+  // rank, the routed experts in [e_lo, e_hi); by default all of them)
+  for (int t = warp; t < NT; t += kFuWarps) {
+    int *su = t_uni + t * SW, *sp = t_ppos + t * SW, *so = t_own + t * SW, *sbp = t_bpos + t * SW;
+    const int *si = t_idx + t * K;
+    if (lane < K) {
+      const int e = si[lane], me = t * K + lane;
+      int rank = 0;
+      for (int q = 0; q < K; ++q) rank += si[q] < e ? 1 : 0;
+      int bpos = 0;
+      for (int q = 0; q < NT * K; ++q) {
+        const int eq = t_idx[q];
+        bpos += (eq < e || (eq == e && q < me)) ? 1 : 0;
       }
-      __syncwarp();
-      // one token: the union is the k selected experts in ascending order;
-      // pair s sits at slot 1 + rank(e_s), the shared expert at slot 0
-      if (lane < K) {
-        int rank = 0;
-        for (int q = 0; q < K; ++q) rank += si[q] < e_sel ? 1 : 0;
-        su[1 + rank] = e_sel;
-        sp[lane] = rank;
-        sbp[1 + rank] = a.routed ? a.pos_t[(size_t)t * K + lane] : rank;
-      }
-      if (lane == 0) {
-        su[0] = E;
-        sbp[0] = a.routed ? a.shared_pos + t : K;
-      }
-      __syncwarp();
-      // the slots this call computes (expert parallelism: the shared expert on
-      // one rank, the routed experts in [e_lo, e_hi); by default all of them)
-      if (lane == 0) {
-        int n = 0;
-        if (a.with_shared) so[n++] = 0;
-        for (int i = 1; i <= K; ++i)
-          if (su[i] >= a.e_lo && su[i] < a.e_hi) so[n++] = i;
-        t_nsl[t] = n;
-      }
-      __syncwarp();
+      su[1 + rank] = e;
+      sp[lane] = rank;
+      sbp[1 + rank] = bpos;
+    }
+    if (lane == 0) {
+      su[0] = E;
+      sbp[0] = NT * K + t;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      int n = 0;
+      if (a.with_shared) so[n++] = 0;
+      for (int i = 1; i <= K; ++i)
+        if (su[i] >= a.e_lo && su[i] < a.e_hi) so[n++] = i;
+      t_nsl[t] = n;
     }
   }
   __syncthreads();
@@ -645,8 +667,8 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     named_sync(kBarEnd, NCT);
     if (!*s_abort) {
       // combine, in the layer's order: shared expert, then the pairs by weight
-      const int *si = t_idx + t * SW, *sp = t_ppos + t * SW;
-      const float *sw = t_w + t * SW;
+      const int *si = t_idx + t * K, *sp = t_ppos + t * SW;
+      const float *sw = t_w + t * K;
       for (int i = tid; i < nrows; i += NCT) {
         float o = a.with_shared ? ysm[(size_t)K * a.rows_max + i] : 0.0f;
         for (int q = 0; q < K; ++q)
@@ -656,16 +678,21 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     }
   }
   if (*s_abort) return;
-  if (!a.routed && blockIdx.x == 0 && warp == 0) {
+  if (blockIdx.x == 0 && warp == 0) {
     // the routing record of the workspace, as the routing kernel writes it
     // (read by no one in this kernel: written last)
-    if (lane < K) {
-      a.idx[lane] = t_idx[lane];
-      a.w[lane] = t_w[lane];
+    for (int i = lane; i < NT * K; i += 32) {
+      a.idx[i] = t_idx[i];
+      a.w[i] = t_w[i];
     }
     __syncwarp();
-    bucket_small_counts(E, K, t_idx, a.cnt, a.off, 0, 1);
-    bucket_small(E, K, 1, t_idx, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos, a.pair_tok);
+    if (NT * K <= 32) {
+      bucket_small_counts(E, NT * K, t_idx, a.cnt, a.off, 0, 1);
+      bucket_small(E, K, NT, t_idx, a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos, a.pair_tok);
+    } else {
+      bucket_warp(E, K, NT, t_idx, reinterpret_cast<int *>(red), a.cnt, a.off, a.uni, a.n_uni, a.perm, a.pos,
+                  a.pair_tok);
+    }
   }
   prof_end(a.prof, 2);
 }
@@ -704,10 +731,10 @@ bool fused_plan(int H, int I, int E, int k, int grid, FusedArgs *a, size_t *smem
   return false;
 }
 
-template <int CSZG, int CSZD, int FMT>
-static cudaError_t launch_fu(const FusedArgs &a, int grid, size_t smem, cudaStream_t s) {
+template <int CSZG, int CSZD, int FMT, bool MULTI>
+static cudaError_t launch_fu_m(const FusedArgs &a, int grid, size_t smem, cudaStream_t s) {
   static int smem_set[64] = {0};
-  cudaError_t err = ensure_smem(k_decode_fused<CSZG, CSZD, FMT>, smem, smem_set);
+  cudaError_t err = ensure_smem(k_decode_fused<CSZG, CSZD, FMT, MULTI>, smem, smem_set);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -719,18 +746,31 @@ static cudaError_t launch_fu(const FusedArgs &a, int grid, size_t smem, cudaStre
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_decode_fused<CSZG, CSZD, FMT>, a);
+  return cudaLaunchKernelEx(&cfg, k_decode_fused<CSZG, CSZD, FMT, MULTI>, a);
 }
 
 template <int CSZG, int CSZD, int FMT>
-static int ctas_fu(size_t smem) {
+static cudaError_t launch_fu(const FusedArgs &a, int grid, size_t smem, cudaStream_t s) {
+  return a.ntok > 1 ? launch_fu_m<CSZG, CSZD, FMT, true>(a, grid, smem, s)
+                    : launch_fu_m<CSZG, CSZD, FMT, false>(a, grid, smem, s);
+}
+
+template <int CSZG, int CSZD, int FMT, bool MULTI>
+static int ctas_fu_m(size_t smem) {
   static int smem_set[64] = {0};
-  if (ensure_smem(k_decode_fused<CSZG, CSZD, FMT>, smem, smem_set) != cudaSuccess) return 0;
+  if (ensure_smem(k_decode_fused<CSZG, CSZD, FMT, MULTI>, smem, smem_set) != cudaSuccess) return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_fused<CSZG, CSZD, FMT>, kFuThreads, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k_decode_fused<CSZG, CSZD, FMT, MULTI>, kFuThreads, smem) !=
       cudaSuccess)
     return 0;
   return n;
+}
+
+// CTAs per SM that both instantiations (one token, a batch) reach
+template <int CSZG, int CSZD, int FMT>
+static int ctas_fu(size_t smem) {
+  const int a = ctas_fu_m<CSZG, CSZD, FMT, false>(smem), b = ctas_fu_m<CSZG, CSZD, FMT, true>(smem);
+  return a < b ? a : b;
 }
 
 #define MOE_FU_CASES(FN, F, ...)                                           \

@@ -262,17 +262,10 @@ struct FusedArgs {
   int e_lo, e_hi;          // routed experts this call computes (expert parallelism)
   int with_shared;         // and the shared expert
   int fmt;                 // kFmtInt4 or kFmtMxfp4
-  // routed mode (a batch of ntok tokens in one launch, streamed token after
-  // token): the routing kernel has written the batch's record; this launch
-  // takes each token's Q8_0 codes (xq, xd: [ntok] rows), top-k (idx, w) and
-  // pair positions (pos_t [ntok][k]; the shared expert's pair of token t at
-  // shared_pos + t) from it, writes h at those positions, out [ntok][H], uses
-  // the control words slot_done + kCtrlWords t for token t, and leaves the
-  // record as it is
-  int routed;
+  // tokens of the launch (1 .. kDecodeTMax): x, xq, xd, logits [ntok] rows,
+  // idx, w [ntok][k], out [ntok][H]; token t's gate/up counters at
+  // slot_done + kCtrlWords t; the record (cnt .. pair_tok) covers the batch
   int ntok;
-  const int32_t *pos_t;
-  int shared_pos;
   long long wait_limit;
   unsigned long long *prof;
 };

@@ -195,77 +195,6 @@ __device__ void bucket_block(int E, int k, int T, const int32_t *idx, int *s_wor
 }
 
 // =====================================================================
-// The same stable counting sort by a single warp (no block barriers): for
-// the decode batch (P = T*k <= 512 pairs).  s_work: >= 2E ints of shared
-// memory; idx may live in shared memory.
-// =====================================================================
-__device__ void bucket_warp(int E, int k, int T, const int32_t *idx, int *s_work, int32_t *cnt,
-                            int32_t *off, int32_t *uni, int32_t *n_uni, int32_t *perm,
-                            int32_t *pos, int32_t *pair_tok) {
-  const int lane = threadIdx.x & 31;
-  const int P = T * k;
-  int *s_cnt = s_work;      // [E]
-  int *s_cur = s_work + E;  // [E]
-  for (int e = lane; e < E; e += 32) s_cnt[e] = 0;
-  __syncwarp();
-  for (int p = lane; p < P; p += 32) atomicAdd(&s_cnt[idx[p]], 1);
-  __syncwarp();
-  // exclusive scans of the counts and of the union flags; lane owns a range
-  const int per = (E + 31) / 32;
-  const int b0 = min(E, lane * per), b1 = min(E, b0 + per);
-  int lc = 0, lf = 0;
-  for (int e = b0; e < b1; ++e) {
-    lc += s_cnt[e];
-    lf += s_cnt[e] > 0 ? 1 : 0;
-  }
-  int ic = lc, jf = lf;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int vc = __shfl_up_sync(0xffffffffu, ic, o);
-    const int vf = __shfl_up_sync(0xffffffffu, jf, o);
-    if (lane >= o) {
-      ic += vc;
-      jf += vf;
-    }
-  }
-  int run = ic - lc, runf = jf - lf;
-  for (int e = b0; e < b1; ++e) {
-    const int c = s_cnt[e];
-    cnt[e] = c;
-    off[e] = run;
-    s_cur[e] = run;
-    run += c;
-    if (c > 0) uni[runf++] = e;
-  }
-  const int nu = __shfl_sync(0xffffffffu, jf, 31);
-  if (lane == 0) {
-    off[E] = P;
-    *n_uni = nu;
-    uni[nu] = E;  // the shared expert follows the union
-  }
-  __syncwarp();
-  const unsigned lt = (1u << lane) - 1u;
-  for (int c0 = 0; c0 < P; c0 += 32) {
-    const int p = c0 + lane;
-    const bool has = p < P;
-    const int e = has ? idx[p] : -1 - lane;  // distinct dummies never match
-    const unsigned peers = __match_any_sync(0xffffffffu, e);
-    const int base = has ? s_cur[e] : 0;
-    __syncwarp();
-    if (has && lane == __ffs(peers) - 1) s_cur[e] = base + __popc(peers);
-    if (has) {
-      const int q = base + __popc(peers & lt);
-      perm[q] = p;
-      if (pos) pos[p] = q;
-      if (pair_tok) pair_tok[q] = p / k;
-    }
-    __syncwarp();
-  }
-  if (pair_tok)
-    for (int t = lane; t < T; t += 32) pair_tok[P + t] = t;
-}
-
-// =====================================================================
 // Router for small batches: Q8_0 of x (grid-stride), logits of epc experts
 // per CTA from shared-memory copies of their Wr rows and of x (TMA bulk),
 // then the last CTA to finish takes top-k + softmax and the batch union.

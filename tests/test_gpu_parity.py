@@ -320,8 +320,8 @@ def test_fused_one_token_equals_three_kernel_path(H, I, E, k, seed):
     x, Wr, blobs = mi.make_layer(w, 0, DEV)
     d = moe.dims(H, I, E, k)
     assert moe.moe_layer_launches(d, 1) == 1
-    assert moe.moe_layer_launches(d, 2) == 2          # routing kernel + one fused launch for the batch
-    assert moe.moe_layer_launches(d, 5) == 2
+    assert moe.moe_layer_launches(d, 2) == 1          # one fused launch for the batch, routing included
+    assert moe.moe_layer_launches(d, 5) == 1
     assert moe.moe_layer_launches(d, 2, 1) == 3       # MOE_PATH_DECODE: routing, gate/up, down
     out_f, ws_f, _ = gpu_layer(w, x, Wr, blobs)
     ws_s = moe.alloc_workspace(d, 1)
@@ -362,13 +362,13 @@ def test_fused_route_counts_and_repeat():
 # ----------------------------------------------------------------- small batches, token by token
 @pytest.mark.parametrize("name,T", [("medium", 2), ("medium", 5), ("tiny", 7), ("glm", 4), ("glm", 16)])
 def test_batch_token_by_token_equals_union_kernels(name, T):
-    """2 <= T <= 16 on the auto path: the routing kernel writes the batch's
-    record, then one fused launch (routed mode) streams the tokens' experts one
-    token after the other and writes each pair's h codes at the batch
-    position.  MOE_PATH_DECODE runs the same batch through the union's gate/up
-    and down kernels.  Both compute every (token, slot) pair with the same
-    per-row code and order, so the outputs, the routing record and the h codes
-    agree bit for bit."""
+    """2 <= T <= 16 on the auto path: one fused launch routes the batch and
+    streams the tokens' experts one token after the other, writing each pair's
+    h codes at its row in the batch's pair order.  MOE_PATH_DECODE runs the
+    same batch through the routing kernel and the union's gate/up and down
+    kernels.  Both compute every (token, slot) pair with the same per-row code
+    and order, so the outputs, the routing record and the h codes agree bit
+    for bit."""
     moe = _moe()
     from tests._common import ws_trace
     if name == "glm":
