@@ -365,16 +365,16 @@ def run_native(args, ws_n, rank, local):
            "what": "expert bytes ((|U|+1) blobs) / device time from the union known to the last output"}
     if fused:
         launch_b = my_bytes + K * (router_b + x_b)
-        roofline = {"bound": "hbm", "kernel": "k_decode_fused", "achieved": round(gbs(launch_b, call_ms), 1),
+        roofline = {"bound": "hbm", "kernel": "k_decode_fused1", "achieved": round(gbs(launch_b, call_ms), 1),
                     "peak": peak, "unit": "GB/s", "frac": round(gbs(launch_b, call_ms) / peak, 4),
                     "peak_source": peak_src,
-                    "traffic": profiled_traffic("k_decode_fused_glm_T1",
+                    "traffic": profiled_traffic("k_decode_fused1_glm_T1",
                                                 "int4_routed_expert_softmax_b200/csrc/moe_fused.cu"),
                     "bytes_per_launch": round(launch_b / K), "us_per_launch": round(call_ms / K * 1e3, 2),
                     "bytes_what": "(|U|+1) x 20,054,016 expert bytes + 6,291,456 router bytes + x",
                     "ffn": ffn}
         kernels = {
-            "k_decode_fused": {"us": round(call_ms / K * 1e3, 2), "GB/s": round(gbs(launch_b, call_ms), 1)},
+            "k_decode_fused1": {"us": round(call_ms / K * 1e3, 2), "GB/s": round(gbs(launch_b, call_ms), 1)},
             "phases_us": {"routing": round(rt_ms / K * 1e3, 2), "gate_up": round(gu_ms / K * 1e3, 2),
                           "down": round(dn_ms / K * 1e3, 2)},
             "timing": "device %globaltimer stamps per phase of the one kernel (first CTA start, last CTA end): "
