@@ -667,19 +667,26 @@ def run_stacked(args, ws_n, rank, local):
             nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
             out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
             layer_ms, layer_b = [], []
+            # events and union sizes stay on the device during a step (no host
+            # synchronisation between the chained layers); read once per step
+            nuni_hist = torch.zeros(L, dtype=torch.int32, device=dev)
             for it in range(args.warmup + args.steps):
                 x = mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1), dev)
+                evs = []
                 for l in range(L):
                     a = torch.cuda.Event(enable_timing=True)
                     b = torch.cuda.Event(enable_timing=True)
                     a.record(stream)
                     moe.moe_layer_forward(d, x, routers[l], tables[l], out, ws)
                     b.record(stream)
-                    b.synchronize()
-                    if it >= args.warmup:
-                        layer_ms.append(a.elapsed_time(b))
-                        layer_b.append((int(nuni_t.item()) + 1) * w.blob_bytes)
+                    nuni_hist[l:l + 1].copy_(nuni_t)
+                    evs.append((a, b))
                     x = chain_next_dev(x, out)
+                torch.cuda.synchronize()
+                if it >= args.warmup:
+                    for l, (a, b) in enumerate(evs):
+                        layer_ms.append(a.elapsed_time(b))
+                    layer_b.extend((int(u) + 1) * w.blob_bytes for u in nuni_hist.tolist())
             ms = allreduce_max(sum(layer_ms), ws_n)
             bts = allreduce_sum(float(sum(layer_b)), ws_n)
             res[f"T={T}"] = {"us_per_layer": round(ms / len(layer_ms) * 1e3, 2),
