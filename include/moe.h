@@ -56,7 +56,7 @@ extern "C" {
 #define MOE_GROUP 64 /* int4 weights per fp16 scale */
 #define MOE_BLOCK 32 /* int8 activations per fp32 scale */
 #define MOE_MAX_E 1024
-#define MOE_DECODE_T_MAX 16 /* largest batch the decode (GEMV) kernels take */
+#define MOE_DECODE_T_MAX 16 /* largest batch the decode kernels take in one call */
 
 enum moe_status {
   MOE_OK = 0,
@@ -81,7 +81,7 @@ typedef struct moe_dims {
 
 enum moe_path {
   MOE_PATH_AUTO = 0,    /* decode kernels for T <= MOE_DECODE_T_MAX, else prefill */
-  MOE_PATH_DECODE = 1,  /* GEMV kernels, T processed in chunks of MOE_DECODE_T_MAX */
+  MOE_PATH_DECODE = 1,  /* union GEMV kernels, T in chunks of MOE_DECODE_T_MAX */
   MOE_PATH_PREFILL = 2  /* grouped GEMM over the expert union */
 };
 
@@ -143,12 +143,13 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
  * Q8_0 code of SiLU(g)*u differing by one where h lies within rounding of a
  * code boundary.  Each path is deterministic: the same call gives the same
  * bits.
- * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): GEMV kernels that
- * stream each union expert's bytes once per 16 tokens, the expert sums in the
- * kernels' own fixed fp32 order.  One token runs in a single cooperative
- * kernel (routing, union, gate/up, down and combine, one CTA per SM) when the
- * shape fits it; larger batches run three kernels per 16 tokens (routing,
- * gate/up, down + combine).  Both give the same bits.
+ * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): one cooperative
+ * kernel (one CTA per SM) routes the batch and streams each token's experts in
+ * turn -- routing, gate/up, down and combine, the expert sums in the kernels'
+ * own fixed fp32 order -- when the shape fits it.  MOE_PATH_DECODE (and a
+ * shape the cooperative kernel does not fit) runs three kernels per 16 tokens
+ * over the batch union instead (routing, gate/up, down + combine), each union
+ * expert's bytes streamed once.  Both give the same bits.
  * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
  * union on the tensor cores (the int4 weights, exact in fp16, times an fp16
  * hi + lo split of the dequantised Q8_0 activations, 22 significant bits;
@@ -221,10 +222,10 @@ int moe_layer_forward_static(const moe_dims *dims, int32_t T, const float *x, co
  * N*K/32 E8M0 exponent bytes, one per 32-block of a row (weight =
  * e2m1 * 2^(E - 127), E = 255 outside the contract): the same byte count as
  * int4 gs64.  Activations stay Q8_0, so every block sum is exact in integers
- * (2 * e2m1 is an integer).  Decode path only, in the one-token fused kernel:
- * a batch runs token by token, each token a full pass over its experts (the
- * workspace's union record then holds the last token's).  MOE_ERR_SHAPE if
- * the shape does not fit the fused kernel.  Other arguments as
+ * (2 * e2m1 is an integer).  Decode path only, in the fused kernel: up to
+ * MOE_DECODE_T_MAX tokens in one launch (the workspace holds the batch's
+ * routing record); larger batches token by token (the record then holds the
+ * last token's).  MOE_ERR_SHAPE if the shape does not fit the fused kernel.  Other arguments as
  * moe_layer_forward (workspace: moe_workspace_bytes_path(dims, T,
  * MOE_PATH_DECODE)). */
 int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, const float *Wr,
@@ -245,7 +246,8 @@ int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, con
  * on one rank (an all-reduce) gives the layer's output within its float
  * tolerance.  expert_table entries outside the range (and entry E when
  * !with_shared) are never read and may be NULL.  Always the decode path
- * (chunks of MOE_DECODE_T_MAX tokens; one token in the fused kernel).
+ * (up to MOE_DECODE_T_MAX tokens in the fused kernel, larger batches in
+ * chunks of MOE_DECODE_T_MAX on the union kernels).
  * MOE_ERR_BAD_ARG unless 0 <= expert_lo <= expert_hi <= E.  Other arguments
  * as moe_layer_forward; workspace: moe_workspace_bytes_path(dims, T,
  * MOE_PATH_DECODE). */
@@ -425,8 +427,9 @@ int moe_device_binary_version(void);
 
 /* Number of this library's kernels one moe_layer_forward call of T tokens on
  * `path` enqueues on the current device (plus one workspace memset), or a
- * negative status: 1 for a one-token decode call that the fused kernel runs,
- * 3 per 16-token chunk on the three-kernel decode path, 9 on the prefill path. */
+ * negative status: 1 for a decode call of up to MOE_DECODE_T_MAX tokens that
+ * the fused kernel runs, 3 per 16-token chunk on the union kernels, 9 on the
+ * prefill path. */
 int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path);
 
 /* Number of streaming multiprocessors the kernels size their grids for
