@@ -240,7 +240,7 @@ def moe_layer_forward(d: MoeDims, x, Wr, table, out, ws, route_counts=None,
 
 
 def moe_layer_forward_mxfp4(d: MoeDims, x, Wr, table, out, ws, route_counts=None, stream=None):
-    """The layer with MXFP4 expert blobs (decode path, token by token)."""
+    """The layer with MXFP4 expert blobs (decode path: the fused kernel, up to 16 tokens per launch)."""
     T = _rows(x, "x", d.H)
     _arg(Wr, "Wr", torch.float32, d.E * d.H)
     _arg(table, "table", torch.int64, d.E + 1)
