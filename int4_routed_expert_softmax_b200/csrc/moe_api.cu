@@ -1,6 +1,7 @@
 // moe_api.cu -- the C ABI of libmoe (declared in include/moe.h): argument
 // checks, workspace carving and the launch sequence of the layer.
 #include <atomic>
+#include <chrono>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -29,6 +30,17 @@ int device_sms() {
     g_sms[dev] = n;
   }
   return g_sms[dev];
+}
+
+// Sequence numbers of fused-kernel launches: unique within the process and
+// never 0 (the ready word's idle value).  The start is drawn from the clock so
+// that a workspace holding another process's last number does not match.
+unsigned long long next_call_seq() {
+  static std::atomic<unsigned long long> seq{
+      (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull};
+  unsigned long long v = seq.fetch_add(1, std::memory_order_relaxed);
+  while (v == 0) v = seq.fetch_add(1, std::memory_order_relaxed);
+  return v;
 }
 
 bool dims_shape_ok(const moe_dims &d) {
@@ -299,7 +311,7 @@ bool fused_usable(const moe_dims &d, int fmt, FusedArgs *fa, size_t *smem, int *
 int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const float *Wr,
                   const void *const *table, float *out, void *ws, int32_t *counts,
                   unsigned long long *prof, const Owned &ow, cudaStream_t s, int fmt = kFmtInt4,
-                  int T = 1) {
+                  int T = 1, bool fresh = true) {
   FusedArgs fa{};
   size_t smem = 0;
   int sms = 0;
@@ -326,8 +338,14 @@ int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const fl
   fa.hqs = p.hqs;
   fa.hd = p.hd;
   fa.status = p.status;
-  fa.arrivals = at<unsigned int>(ws, L.ctrl) + 1;
-  fa.slot_done = at<int32_t>(ws, L.ctrl) + kCtrlSlot0;
+  // no memset: the kernel zeroes its control words (and, on a call's first
+  // launch, the status word) itself
+  fa.ctrl = at<int32_t>(ws, L.ctrl);
+  fa.arrivals = reinterpret_cast<unsigned int *>(fa.ctrl + 1);
+  fa.slot_done = fa.ctrl + kCtrlSlot0;
+  fa.ready = reinterpret_cast<unsigned long long *>(fa.ctrl + kCtrlReady);
+  fa.seq = next_call_seq();
+  fa.fresh = fresh ? 1 : 0;
   fa.e_lo = ow.lo;
   fa.e_hi = ow.hi;
   fa.with_shared = ow.shared;
@@ -335,6 +353,14 @@ int fused_forward(const moe_dims &d, const WsLayout &L, const float *x, const fl
   fa.prof = prof;
   fa.ntok = T;
   return cuda_status(launch_decode_fused(fa, sms, smem, s));
+}
+
+// The fused kernel runs this shape and weight format on the current device.
+bool fused_fits(const moe_dims &d, int fmt) {
+  FusedArgs fa{};
+  size_t smem = 0;
+  int grid = 0;
+  return fused_usable(d, fmt, &fa, &smem, &grid);
 }
 
 bool use_prefill(int T, int path) {
@@ -676,25 +702,24 @@ static int forward_checked(const moe_dims &d, int32_t T, const float *x, const f
                     float *out, void *ws, int32_t *route_counts_opt, bool pf, const WsLayout &L, bool zeroed,
                     cudaStream_t s, const Owned &ow, bool auto_path = true) {
   int rc = MOE_OK;
+  const moe_dims *dims = &d;
+  // One token, or a small batch on the auto path: one fused launch streams
+  // the tokens' experts one token after the other.  At these sizes the batch
+  // union is nearly the sum of the tokens' selections, so per-token streaming
+  // costs few extra bytes and runs at the fused kernel's rate.  The kernel
+  // zeroes its own control words and status word: no memset before it.
+  if (!pf && (T == 1 || (auto_path && T <= kDecodeTMax)) && fused_fits(d, kFmtInt4))
+  {
+    rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof_next(), ow, s, kFmtInt4, T);
+    return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
+  }
   if (!zeroed) {
     // status word and the router's arrival counter start at zero on every call
     cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
     if (err != cudaSuccess) return cuda_status(err);
   }
-  const moe_dims *dims = &d;
   if (pf) return prefill_forward(*dims, T, x, Wr, expert_table, out, ws, L, route_counts_opt, s);
   unsigned long long *prof = prof_next();
-  if (T == 1) {
-    rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s);
-    if (rc != kFusedNA) return rc;
-  } else if (auto_path && T <= kDecodeTMax) {
-    // a small batch: one fused launch streams the tokens' experts one token
-    // after the other.  At these sizes the batch union is nearly the sum of
-    // the tokens' selections, so per-token streaming costs few extra bytes
-    // and runs at the fused kernel's rate.
-    rc = fused_forward(d, L, x, Wr, expert_table, out, ws, route_counts_opt, prof, ow, s, kFmtInt4, T);
-    if (rc != kFusedNA) return rc;
-  }
   for (int t0 = 0; t0 < T; t0 += kDecodeTMax) {
     const int Tc = (T - t0) < kDecodeTMax ? (T - t0) : kDecodeTMax;
     rc = route_chunk(*dims, t0, Tc, L, x, Wr, ws, route_counts_opt, prof, ow, s);
@@ -734,24 +759,14 @@ int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, con
   if (!aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   const WsLayout L = ws_layout(*dims, T, false);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  {
-    FusedArgs fa{};
-    size_t smem = 0;
-    int grid = 0;
-    if (!fused_usable(*dims, kFmtMxfp4, &fa, &smem, &grid)) return MOE_ERR_SHAPE;
-  }
+  if (!fused_fits(*dims, kFmtMxfp4)) return MOE_ERR_SHAPE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  cudaError_t err = cudaMemsetAsync(ws, 0, L.xin, s);
-  if (err != cudaSuccess) return cuda_status(err);
   unsigned long long *prof = prof_next();
   if (T == 1 || T > kDecodeTMax) {
-    // token by token with the kernel's own routing (every token's control
-    // words zeroed before its launch)
+    // token by token with the kernel's own routing; every launch zeroes its
+    // control words, the first one the status word too (a later launch
+    // keeps an earlier one's error)
     for (int t = 0; t < T; ++t) {
-      if (t > 0) {
-        err = cudaMemsetAsync(at<unsigned char>(ws, L.ctrl), 0, L.xin - L.ctrl, s);
-        if (err != cudaSuccess) return cuda_status(err);
-      }
       // token t in the per-token rows of the workspace; the pair rows are reused
       WsLayout Lt = L;
       Lt.xq += (size_t)t * dims->H;
@@ -760,7 +775,7 @@ int moe_layer_forward_mxfp4(const moe_dims *dims, int32_t T, const float *x, con
       Lt.idx += (size_t)t * dims->k * 4;
       Lt.w += (size_t)t * dims->k * 4;
       rc = fused_forward(*dims, Lt, x + (size_t)t * dims->H, Wr, expert_table, out + (size_t)t * dims->H, ws,
-                         route_counts_opt, t == 0 ? prof : nullptr, all_owned(*dims), s, kFmtMxfp4);
+                         route_counts_opt, t == 0 ? prof : nullptr, all_owned(*dims), s, kFmtMxfp4, 1, t == 0);
       if (rc != MOE_OK) return rc == kFusedNA ? MOE_ERR_SHAPE : rc;
     }
     return MOE_OK;

@@ -154,6 +154,57 @@ __device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int *p) {
   return v;
 }
 
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ void st_relaxed_u64(unsigned long long *p, unsigned long long v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// The call's control words start at zero without a memset launched before
+// the kernel.  CTA 0 zeroes the first `nctl` of them (and the status word on a
+// call's first launch) as it starts, then publishes the call's sequence number
+// in the ready word; every other CTA waits for that number before it arrives
+// at the grid barrier, its first use of a control word.  (A status that one of
+// them sets before CTA 0's zeroing can be lost, but such a CTA never arrives,
+// so CTA 0's own barrier wait runs out and reports.)  CTA 0 puts the ready word
+// back to 0 once every CTA has arrived (so has seen it), or when it leaves
+// before the barrier, so that a replay of the same launch (a CUDA graph: the
+// same sequence number) waits for its own zeroing again.
+// ctrl_zero: every thread of CTA 0, after the barrier init.
+__device__ __forceinline__ void ctrl_zero(const FusedArgs &a, int nctl) {
+  const int tid = threadIdx.x;
+  for (int i = tid; i < nctl; i += blockDim.x)
+    if (i != kCtrlReady && i != kCtrlReady + 1) a.ctrl[i] = 0;
+  if (a.fresh && tid < 4) a.status[tid] = 0;
+  __syncthreads();
+  if (tid == 0) st_release_u64(a.ready, a.seq);  // after the CTA's zeroing (bar.sync, then release)
+}
+
+// Thread 0 of any CTA before its arrival: false if the wait ran out.
+__device__ __forceinline__ bool ctrl_ready(const FusedArgs &a, long long lim) {
+  if (blockIdx.x == 0 || ld_acquire_u64(a.ready) == a.seq) return true;
+  const long long t0 = clock64();
+  while (ld_acquire_u64(a.ready) != a.seq) {
+    if (clock64() - t0 > lim) {
+      set_status(a.status, MOE_ERR_TIMEOUT, kDetFuReady);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// CTA 0, thread 0: the ready word back to 0.
+__device__ __forceinline__ void ctrl_close(const FusedArgs &a) {
+  if (blockIdx.x == 0 && threadIdx.x == 0) st_relaxed_u64(a.ready, 0ull);
+}
+
 // Waits (bounded by `limit` SM clocks) until the counter at p reaches `target`.
 __device__ __forceinline__ bool wait_count(const int32_t *p, int32_t target, long long limit) {
   if (ld_acquire(p) >= target) return true;
@@ -235,12 +286,14 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
     if (nr > 0) bulk_g2s(rw, a.Wr + (size_t)e0 * H, (uint32_t)nr * (uint32_t)H * 4u, rbar);
     bulk_g2s(rx, a.x, (uint32_t)nx * (uint32_t)H * 4u, rbar);
   }
+  if (blockIdx.x == 0) ctrl_zero(a, NT * kCtrlWords);
   const int nlp = nr * NT;  // (row, token) pairs of logits
   for (int c0 = 0, ph = 0; c0 < NT; c0 += xcap, ph ^= 1) {
     const int nx = NT - c0 < xcap ? NT - c0 : xcap;
     const bool ok = mbar_wait(rbar, (uint32_t)ph, a.status, kDetFuRoute, lim);
     if (!__syncthreads_and(ok)) {
       if (tid == 0) mbar_drain(rbar, (uint32_t)ph, a.status, kDetFuRouteDrain);  // the copies land before exit
+      ctrl_close(a);
       return;
     }
     if (c0 == 0 && warp == PROD && lane == 0 && a.with_shared) {
@@ -302,18 +355,23 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused(FusedArgs a) {
   // them (the barrier orders this CTA's writes before thread 0's release)
   __syncthreads();
   if (tid == 0) {
-    red_release_add_u32(a.arrivals, 1u);
-    if (ld_acquire_u32(a.arrivals) < (unsigned)G) {
-      const long long t0 = clock64();
-      while (ld_acquire_u32(a.arrivals) < (unsigned)G) {
-        if (clock64() - t0 > lim) {
-          set_status(a.status, MOE_ERR_TIMEOUT, kDetFuGrid);
-          *s_abort = 1;
-          break;
+    if (!ctrl_ready(a, lim)) {
+      *s_abort = 1;
+    } else {
+      red_release_add_u32(a.arrivals, 1u);
+      if (ld_acquire_u32(a.arrivals) < (unsigned)G) {
+        const long long t0 = clock64();
+        while (ld_acquire_u32(a.arrivals) < (unsigned)G) {
+          if (clock64() - t0 > lim) {
+            set_status(a.status, MOE_ERR_TIMEOUT, kDetFuGrid);
+            *s_abort = 1;
+            break;
+          }
+          __nanosleep(32);
         }
-        __nanosleep(32);
       }
     }
+    ctrl_close(a);  // every CTA has arrived, so has seen the ready word (or the wait ran out)
   }
   __syncthreads();
   if (*s_abort) return;  // nothing in flight: the staging copies have landed
@@ -796,9 +854,11 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused1(FusedArgs a) {
   }
   // the expert table, for the stream that follows the union
   for (int e = tid; e <= E; e += kFuThreads) s_tab[e] = static_cast<const unsigned char *>(a.table[e]);
+  if (blockIdx.x == 0) ctrl_zero(a, kCtrlWords);
   const bool ok = mbar_wait(rbar, 0, a.status, kDetFuRoute, lim);
   if (!__syncthreads_and(ok)) {
     if (tid == 0) mbar_drain(rbar, 0, a.status, kDetFuRouteDrain);  // the copies land before exit
+    ctrl_close(a);
     return;
   }
   if (warp == PROD && lane == 0 && a.with_shared) {
@@ -843,18 +903,23 @@ __global__ void __launch_bounds__(kFuThreads, 1) k_decode_fused1(FusedArgs a) {
   // barrier orders this CTA's writes before thread 0's release)
   __syncthreads();
   if (tid == 0) {
-    red_release_add_u32(a.arrivals, 1u);
-    if (ld_acquire_u32(a.arrivals) < (unsigned)G) {
-      const long long t0 = clock64();
-      while (ld_acquire_u32(a.arrivals) < (unsigned)G) {
-        if (clock64() - t0 > lim) {
-          set_status(a.status, MOE_ERR_TIMEOUT, kDetFuGrid);
-          *s_abort = 1;
-          break;
+    if (!ctrl_ready(a, lim)) {
+      *s_abort = 1;
+    } else {
+      red_release_add_u32(a.arrivals, 1u);
+      if (ld_acquire_u32(a.arrivals) < (unsigned)G) {
+        const long long t0 = clock64();
+        while (ld_acquire_u32(a.arrivals) < (unsigned)G) {
+          if (clock64() - t0 > lim) {
+            set_status(a.status, MOE_ERR_TIMEOUT, kDetFuGrid);
+            *s_abort = 1;
+            break;
+          }
+          __nanosleep(32);
         }
-        __nanosleep(32);
       }
     }
+    ctrl_close(a);  // every CTA has arrived, so has seen the ready word (or the wait ran out)
   }
   __syncthreads();
   if (*s_abort) return;  // nothing in flight: the staging copies have landed

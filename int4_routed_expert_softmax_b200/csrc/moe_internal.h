@@ -19,9 +19,13 @@ constexpr int kMaxSmem = 227 * 1024 - 1024;            // dynamic shared memory 
 constexpr int kPfMaxCtas = 256;                        // prefill GEMM grid bound (one CTA per SM)
 constexpr int kProfSlots = 1024;                       // per-call profiling records kept per device
 constexpr int kProfWords = 8;                          // per record: 4 phases x (~first start, last end) in ns
-// Control words of the workspace (zeroed at the start of every call): [0] the
+// Control words of the workspace, zero at the start of every call: [0] the
 // routing kernel's arrival ticket, [1] the fused kernel's routing arrivals,
-// [kCtrlSlot0 + s] gate/up units completed for union slot s (fused kernel).
+// [kCtrlReady, +1] the fused kernel's 64-bit ready word, [kCtrlSlot0 + s]
+// gate/up units completed for union slot s (fused kernel).  The memset before
+// the other paths' launches zeroes them; the fused kernel zeroes its own (CTA 0,
+// then the call's sequence number in the ready word).
+constexpr int kCtrlReady = 2;
 constexpr int kCtrlSlot0 = 4;
 // Control words per token of a decode batch (token t's block at kCtrlWords t;
 // the fused kernel's per-token launches each use their own block).
@@ -56,6 +60,7 @@ enum Detail : int32_t {
   kDetFuDrain = 45,
   kDetFuSlot = 46,
   kDetFuAlign = 47,
+  kDetFuReady = 48,
 };
 
 // The wait limit kernels launched now take for their work waits (set by
@@ -253,8 +258,12 @@ struct FusedArgs {
   int32_t *hqs;
   float *hd;
   int32_t *status;
-  unsigned int *arrivals;  // routing arrivals of the grid (zeroed per call)
-  int32_t *slot_done;      // [k + 1] gate/up units completed per union slot (zeroed per call)
+  unsigned int *arrivals;  // routing arrivals of the grid (zeroed per call by CTA 0)
+  int32_t *slot_done;      // [k + 1] gate/up units completed per union slot (zeroed per call by CTA 0)
+  int32_t *ctrl;           // the control words (arrivals and slot_done point into them)
+  unsigned long long *ready;  // ctrl + kCtrlReady: the call's sequence number once CTA 0 has zeroed
+  unsigned long long seq;     // this call's sequence number (never 0)
+  int fresh;               // the first launch of a call: CTA 0 zeroes the status word too
   int nstage;              // ring stages
   int rows_max;            // down: most output rows a CTA owns
   int rg;                  // down: row granularity (scale bytes of rg rows: a multiple of 16)

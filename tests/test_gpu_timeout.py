@@ -20,7 +20,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 SHORT = 200                       # SM clocks: shorter than any copy from HBM takes
 MOE_ERR_TIMEOUT = -7
-ROUTE_DETAILS = {1, 40, 42}       # the routing kernel's staging wait; the fused kernel's, its grid arrival
+ROUTE_DETAILS = {1, 40, 42, 48}   # the routing kernel's staging wait; the fused kernel's, its grid
+                                  # arrival, its wait for CTA 0's zeroed control words
 EXPERT_DETAILS = {10, 11, 20, 21}  # gate/up and down: stage landed / stage freed
 PREFILL_DETAILS = {31, 32, 33, 34}  # grouped GEMM: operands landed / freed, accumulators
 
