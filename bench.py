@@ -665,28 +665,41 @@ def run_stacked(args, ws_n, rank, local):
             ws = moe.alloc_workspace(d, T, dev)
             view = moe.moe_workspace_view(d, T, ws)
             nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
-            out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
+            x_buf = mi.make_x(T, w.H, mi.sub_seed(seed, 100, 1), dev).clone()
+            outs = [torch.empty((T, w.H), dtype=torch.float32, device=dev) for _ in range(L)]
             layer_ms, layer_b = [], []
-            # events and union sizes stay on the device during a step (no host
-            # synchronisation between the chained layers); read once per step
+            # One step (the L chained layers, the glue between them, a copy of
+            # each layer's union size) is one CUDA graph, with an event pair
+            # around every layer call: the Python glue would otherwise leave the
+            # GPU waiting for the host between layers.  Read once per step.
             nuni_hist = torch.zeros(L, dtype=torch.int32, device=dev)
-            for it in range(args.warmup + args.steps):
-                x = mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1), dev)
-                evs = []
+            evs = [(torch.cuda.Event(enable_timing=True, external=True),
+                    torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):  # the library's one-time setup, outside the capture
+                moe.moe_layer_forward(d, x_buf, routers[0], tables[0], outs[0], ws)
+            stream.wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                gs = torch.cuda.current_stream()
+                x = x_buf
                 for l in range(L):
-                    a = torch.cuda.Event(enable_timing=True)
-                    b = torch.cuda.Event(enable_timing=True)
-                    a.record(stream)
-                    moe.moe_layer_forward(d, x, routers[l], tables[l], out, ws)
-                    b.record(stream)
+                    evs[l][0].record(gs)
+                    moe.moe_layer_forward(d, x, routers[l], tables[l], outs[l], ws)
+                    evs[l][1].record(gs)
                     nuni_hist[l:l + 1].copy_(nuni_t)
-                    evs.append((a, b))
-                    x = chain_next_dev(x, out)
+                    x = chain_next_dev(x, outs[l])
+            for it in range(args.warmup + args.steps):
+                x_buf.copy_(mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1), dev))
+                graph.replay()
                 torch.cuda.synchronize()
                 if it >= args.warmup:
-                    for l, (a, b) in enumerate(evs):
+                    for a, b in evs:
                         layer_ms.append(a.elapsed_time(b))
                     layer_b.extend((int(u) + 1) * w.blob_bytes for u in nuni_hist.tolist())
+            del graph
             ms = allreduce_max(sum(layer_ms), ws_n)
             bts = allreduce_sum(float(sum(layer_b)), ws_n)
             res[f"T={T}"] = {"us_per_layer": round(ms / len(layer_ms) * 1e3, 2),
@@ -702,7 +715,9 @@ def run_stacked(args, ws_n, rank, local):
                 config={"workload": "stacked: 8 GLM-5.2-shaped layers resident in HBM (41.2 GB), batches of "
                                     + ", ".join(str(t) for t in w.T_list) + " tokens, layers chained",
                         "layers": L, "T_list": list(w.T_list),
-                        "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)"},
+                        "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)",
+                        "timing": "one CUDA graph per step (layers, glue, union-size copies), "
+                                  "CUDA events around each layer call inside it"},
                 by_batch=res, clocks=clk.summary(),
                 gpu_launches=sum(moe.moe_layer_launches(d, T) for T in w.T_list) * L * args.steps)
 

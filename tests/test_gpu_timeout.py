@@ -57,8 +57,7 @@ def test_wait_limit_setter_round_trip():
 
 @pytest.mark.parametrize("name", ["tiny", "medium"])
 def test_routing_wait_runs_out_then_recovers(name):
-    """tiny: four tokens, the three-kernel path; medium: one token, the fused
-    cooperative kernel."""
+    """tiny: four tokens; medium: one token (the auto path's decode kernels)."""
     moe = _moe()
     w = mi.WORKLOADS["tiny"] if name == "tiny" else _medium()
     x, Wr, blobs = mi.make_layer(w, 0, DEV)
