@@ -56,7 +56,7 @@ def parse():
     ap.add_argument("--experts", type=int, default=None,
                     help="routed experts per layer (profiling: a small pool, same per-step work)")
     ap.add_argument("--tokens", type=int, default=None,
-                    help="prefill batch size (profiling a small case; default: the workload's 2048)")
+                    help="tokens per layer call: decode 1-16 (default 1), prefill (default 2048)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="default workload: leave out the prefill sub-object of the line")
     return ap.parse_args()
@@ -225,8 +225,8 @@ def host_cpu() -> dict:
 
 def decode_config(w: mi.Workload, ws_n: int) -> dict:
     """The decode workload's config record (the native and the reference arm print the same)."""
-    return {"workload": "decode: one GLM-5.2-shaped MoE layer, H=6144, 256 routed experts x "
-                        "SwiGLU I=2048 + 1 shared, top-8 softmax, batch 1, all experts resident",
+    return {"workload": f"decode: one GLM-5.2-shaped MoE layer, H={w.H}, {w.E} routed experts x "
+                        f"SwiGLU I={w.I} + 1 shared, top-{w.k} softmax, batch {w.T}, all experts resident",
             "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T, "global_batch": w.T * ws_n,
             "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
             "x_pool": POOL}
@@ -278,6 +278,10 @@ def run_native(args, ws_n, rank, local):
     w = mi.WORKLOADS[args.workload]
     if args.experts:
         w = mi.shrink(w, E=args.experts)
+    if args.tokens:
+        if not 1 <= args.tokens <= 16:
+            raise SystemExit("--tokens: the decode line takes 1 to 16 tokens per call")
+        w = mi.shrink(w, T=args.tokens)
     seed = rank_seed(w, rank)
     wl = mi.shrink(w, seed=seed)
     T = w.T
@@ -364,17 +368,23 @@ def run_native(args, ws_n, rank, local):
            "achieved": round(gbs(my_bytes, ffn_ms), 1), "frac": round(gbs(my_bytes, ffn_ms) / peak, 4),
            "what": "expert bytes ((|U|+1) blobs) / device time from the union known to the last output"}
     if fused:
+        # one token: k_decode_fused1; 2-16 tokens: k_decode_fused, which streams
+        # each token's k + 1 blobs in turn (the algorithmic bytes count every
+        # union expert once, as the union kernels read it)
+        kname = "k_decode_fused1" if T == 1 else "k_decode_fused"
         launch_b = my_bytes + K * (router_b + x_b)
-        roofline = {"bound": "hbm", "kernel": "k_decode_fused1", "achieved": round(gbs(launch_b, call_ms), 1),
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": round(gbs(launch_b, call_ms), 1),
                     "peak": peak, "unit": "GB/s", "frac": round(gbs(launch_b, call_ms) / peak, 4),
                     "peak_source": peak_src,
-                    "traffic": profiled_traffic("k_decode_fused1_glm_T1",
+                    "traffic": profiled_traffic(f"{kname}_glm_T{T}",
                                                 "int4_routed_expert_softmax_b200/csrc/moe_fused.cu"),
                     "bytes_per_launch": round(launch_b / K), "us_per_launch": round(call_ms / K * 1e3, 2),
-                    "bytes_what": "(|U|+1) x 20,054,016 expert bytes + 6,291,456 router bytes + x",
+                    "bytes_what": "(|U|+1) x 20,054,016 expert bytes + E x H x 4 router bytes + x",
                     "ffn": ffn}
+        if T > 1:
+            roofline["streamed_bytes_per_launch"] = T * (w.k + 1) * blob_b + router_b + x_b
         kernels = {
-            "k_decode_fused1": {"us": round(call_ms / K * 1e3, 2), "GB/s": round(gbs(launch_b, call_ms), 1)},
+            kname: {"us": round(call_ms / K * 1e3, 2), "GB/s": round(gbs(launch_b, call_ms), 1)},
             "phases_us": {"routing": round(rt_ms / K * 1e3, 2), "gate_up": round(gu_ms / K * 1e3, 2),
                           "down": round(dn_ms / K * 1e3, 2)},
             "timing": "device %globaltimer stamps per phase of the one kernel (first CTA start, last CTA end): "
@@ -847,6 +857,12 @@ def run_reference(args, ws_n, rank):
     if args.workload == "prefill":
         return run_reference_prefill(args, ws_n)
     w = mi.WORKLOADS[args.workload]
+    if args.workload == "decode":
+        # the native line's --experts / --tokens, so that both arms name one config
+        if args.experts:
+            w = mi.shrink(w, E=args.experts)
+        if args.tokens:
+            w = mi.shrink(w, T=args.tokens)
     seed = w.seed
     Wr = mi.make_router(w.E, w.H, mi.sub_seed(seed, 0, 2), "cpu").numpy()
     xpool = mi.make_x(POOL * w.T, w.H, mi.sub_seed(seed, 0, 1), "cpu").numpy()
