@@ -59,7 +59,10 @@ def parse():
                     help="tokens per layer call: decode 1-16 (default 1), prefill (default 2048)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="default workload: leave out the prefill sub-object of the line")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.workload == "decode" and args.tokens is not None and not 1 <= args.tokens <= 16:
+        ap.error("--tokens: the decode line takes 1 to 16 tokens per call")
+    return args
 
 
 def peaks():
@@ -279,8 +282,6 @@ def run_native(args, ws_n, rank, local):
     if args.experts:
         w = mi.shrink(w, E=args.experts)
     if args.tokens:
-        if not 1 <= args.tokens <= 16:
-            raise SystemExit("--tokens: the decode line takes 1 to 16 tokens per call")
         w = mi.shrink(w, T=args.tokens)
     seed = rank_seed(w, rank)
     wl = mi.shrink(w, seed=seed)

@@ -53,3 +53,28 @@ def test_reference_arm_prints_one_line_per_workload():
         assert d["impl"] == "reference" and d["unit"] == unit and d["value"] > 0
         assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
         assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_decode_config_names_the_batch_and_expert_count():
+    """--tokens / --experts change the decode line's config on both arms; the
+    default line keeps the GLM-5.2 layer with batch 1."""
+    import json
+    import subprocess
+    import sys
+    import moe_inputs as mi
+    d0 = bench.decode_config(mi.WORKLOADS["decode"], 1)
+    assert "256 routed experts" in d0["workload"] and "batch 1," in d0["workload"] and d0["T"] == 1
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference",
+                        "--tokens", "4", "--experts", "64", "--steps", "1", "--warmup", "0",
+                        "--cpu-seconds", "1"],
+                       capture_output=True, text=True, timeout=600,
+                       env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert r.returncode == 0, r.stderr[-2000:]
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    assert d["config"]["T"] == 4 and d["config"]["E"] == 64 and d["config"]["global_batch"] == 4
+    assert "64 routed experts" in d["config"]["workload"] and "batch 4," in d["config"]["workload"]
+    bad = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--tokens", "17"],
+                         capture_output=True, text=True, timeout=600,
+                         env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert bad.returncode != 0 and "1 to 16 tokens" in bad.stderr
