@@ -57,6 +57,8 @@ def parse():
                     help="routed experts per layer (profiling: a small pool, same per-step work)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per layer call: decode 1-16 (default 1), prefill (default 2048)")
+    ap.add_argument("--path", choices=["auto", "decode"], default="auto",
+                    help="decode line: the library's choice (fused kernel) or MOE_PATH_DECODE (union kernels)")
     ap.add_argument("--no-prefill", action="store_true",
                     help="default workload: leave out the prefill sub-object of the line")
     args = ap.parse_args()
@@ -226,13 +228,16 @@ def host_cpu() -> dict:
     return {"cpu_model": model, "nproc": os.cpu_count()}
 
 
-def decode_config(w: mi.Workload, ws_n: int) -> dict:
+def decode_config(w: mi.Workload, ws_n: int, path: str = "auto") -> dict:
     """The decode workload's config record (the native and the reference arm print the same)."""
-    return {"workload": f"decode: one GLM-5.2-shaped MoE layer, H={w.H}, {w.E} routed experts x "
-                        f"SwiGLU I={w.I} + 1 shared, top-{w.k} softmax, batch {w.T}, all experts resident",
-            "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T, "global_batch": w.T * ws_n,
-            "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
-            "x_pool": POOL}
+    c = {"workload": f"decode: one GLM-5.2-shaped MoE layer, H={w.H}, {w.E} routed experts x "
+                     f"SwiGLU I={w.I} + 1 shared, top-{w.k} softmax, batch {w.T}, all experts resident",
+         "H": w.H, "I": w.I, "E": w.E, "k": w.k, "T": w.T, "global_batch": w.T * ws_n,
+         "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
+         "x_pool": POOL}
+    if path != "auto":
+        c["path"] = "MOE_PATH_DECODE (routing, gate/up and down kernels over the batch union)"
+    return c
 
 
 def prefill_config(w: mi.Workload, ws_n: int) -> dict:
@@ -290,7 +295,8 @@ def run_native(args, ws_n, rank, local):
     blobs = mi.make_blobs(w.H, w.I, w.E + 1, mi.sub_seed(seed, 0, 3), dev)
     xpool = mi.make_x(POOL * T, w.H, mi.sub_seed(seed, 0, 1), dev).view(POOL, T, w.H)
     d = moe.dims(w.H, w.I, w.E, w.k)
-    ws = moe.alloc_workspace(d, T, dev)
+    path = moe.MOE_PATH_DECODE if args.path == "decode" else moe.MOE_PATH_AUTO
+    ws = moe.alloc_workspace(d, T, dev, path=path)
     table = moe.expert_table(blobs)
     out = torch.empty((T, w.H), dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -304,7 +310,7 @@ def run_native(args, ws_n, rank, local):
     stream = torch.cuda.current_stream()
 
     def step(i):
-        moe.moe_layer_forward(d, xpool[i % POOL], Wr, table, out, ws)
+        moe.moe_layer_forward(d, xpool[i % POOL], Wr, table, out, ws, path=path)
 
     moe.moe_profile_enable(True)
     for i in range(args.warmup):
@@ -352,7 +358,7 @@ def run_native(args, ws_n, rank, local):
     value = all_bytes / (max_ms * 1e-3) / 1e9
     ms_per_step = max_ms / K
 
-    launches = moe.moe_layer_launches(d, T)
+    launches = moe.moe_layer_launches(d, T, path)
     fused = launches == 1
     rt_ms = sum(p[0] for p in prof)
     gu_ms = sum(p[1] for p in prof)
@@ -395,7 +401,7 @@ def run_native(args, ws_n, rank, local):
         roofline = {"bound": "hbm", "kernel": "k_gateup_decode", "achieved": round(gbs(gu_bytes, gu_ms), 1),
                     "peak": peak, "unit": "GB/s", "frac": round(gbs(gu_bytes, gu_ms) / peak, 4),
                     "peak_source": peak_src,
-                    "traffic": profiled_traffic("k_gateup_decode_glm_T1",
+                    "traffic": profiled_traffic(f"k_gateup_decode_glm_T{T}",
                                                 "int4_routed_expert_softmax_b200/csrc/moe_decode.cu"),
                     "bytes_per_launch": round(gu_bytes / K), "us_per_launch": round(gu_ms / K * 1e3, 2),
                     "down": {"achieved": round(gbs(dn_bytes, dn_ms), 1),
@@ -416,7 +422,7 @@ def run_native(args, ws_n, rank, local):
         xh = xpool.cpu().pin_memory()
         oh = torch.empty((T, w.H), dtype=torch.float32).pin_memory()
         for i in range(args.warmup):
-            moe.moe_layer_forward_host(d, xh[i % POOL], Wr, table, oh, ws)
+            moe.moe_layer_forward_host(d, xh[i % POOL], Wr, table, oh, ws, path=path)
         torch.cuda.synchronize()
         e_ms, e_bytes = 0.0, 0
         barrier(ws_n)
@@ -426,7 +432,7 @@ def run_native(args, ws_n, rank, local):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
-            moe.moe_layer_forward_host(d, xh[(args.warmup + i) % POOL], Wr, table, oh, ws)
+            moe.moe_layer_forward_host(d, xh[(args.warmup + i) % POOL], Wr, table, oh, ws, path=path)
             b.record(stream)
             b.synchronize()
             e_ms += a.elapsed_time(b)
@@ -455,7 +461,7 @@ def run_native(args, ws_n, rank, local):
         metric=METRIC, value=round(value, 1), unit="GB/s", n_gpus=ws_n, steps=K, warmup=args.warmup,
         ms_per_step=round(ms_per_step, 5), higher_is_better=True, scaling="weak", vs_baseline=None,
         dtype="int4xint8->fp32", data="synthetic",
-        config=decode_config(w, ws_n),
+        config=decode_config(w, ws_n, args.path),
         us_per_token_layer=round(ms_per_step / T * 1e3, 2),
         union_mean=round(sum(nuni) / len(nuni), 2),
         roofline=roofline, kernels=kernels, e2e=e2e, cpu_baseline=cpu, clocks=clocks,
@@ -893,7 +899,7 @@ def run_reference(args, ws_n, rank):
         steps=args.steps, warmup=args.warmup, ms_per_step=round(ts / max(1, tn) * 1e3, 3),
         higher_is_better=True, scaling="weak", vs_baseline=None, dtype="int4xint8->fp32",
         data="synthetic",
-        config=decode_config(w, ws_n),
+        config=decode_config(w, ws_n, args.path),
         us_per_token_layer=round(ts / max(1, tn) * 1e6, 1), cpu_baseline=cpu,
         e2e={"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 
