@@ -146,10 +146,14 @@ int moe_bucket(const moe_dims *dims, int32_t T, const int32_t *idx, int32_t *cnt
  * Decode path (T <= MOE_DECODE_T_MAX under MOE_PATH_AUTO): one cooperative
  * kernel (one CTA per SM) routes the batch and streams each token's experts in
  * turn -- routing, gate/up, down and combine, the expert sums in the kernels'
- * own fixed fp32 order -- when the shape fits it.  MOE_PATH_DECODE (and a
- * shape the cooperative kernel does not fit) runs three kernels per 16 tokens
- * over the batch union instead (routing, gate/up, down + combine), each union
- * expert's bytes streamed once.  Both give the same bits.
+ * own fixed fp32 order -- when the shape fits it.  That kernel zeroes its own
+ * control words (nothing else is enqueued), so the call can be captured in a
+ * CUDA graph and replayed; make one call with the same dims on the device
+ * before capturing (it sets the kernels' attributes).  MOE_PATH_DECODE at 2 or
+ * more tokens (and a shape the cooperative kernel does not fit) runs three
+ * kernels per 16 tokens over the batch union instead (routing, gate/up, down +
+ * combine), each union expert's bytes streamed once; one token takes the
+ * cooperative kernel on either path.  Both give the same bits.
  * Prefill path: router GEMM, top-k, bucketing, then a grouped GEMM over the
  * union on the tensor cores (the int4 weights, exact in fp16, times an fp16
  * hi + lo split of the dequantised Q8_0 activations, 22 significant bits;
