@@ -57,6 +57,9 @@ def parse():
                     help="routed experts per layer (profiling: a small pool, same per-step work)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="tokens per layer call: decode 1-16 (default 1), prefill (default 2048)")
+    ap.add_argument("--chain", action="store_true",
+                    help="stacked workload: each layer's input from the previous layer's output "
+                         "(default: hidden states drawn independently per layer and step)")
     ap.add_argument("--path", choices=["auto", "decode"], default="auto",
                     help="decode line: the library's choice (fused kernel) or MOE_PATH_DECODE (union kernels)")
     ap.add_argument("--no-prefill", action="store_true",
@@ -663,8 +666,10 @@ def chain_next_dev(x: torch.Tensor, out: torch.Tensor, gamma: float = 0.5, zipf:
 
 def run_stacked(args, ws_n, rank, local):
     """8 stacked GLM-5.2-shaped layers resident in HBM; batches of 1, 2, 3, 4 and
-    16 tokens (2-3: draft-verification sizes) with independently drawn hidden
-    states; per-layer us and union-weighted expert GB/s."""
+    16 tokens (2-3: draft-verification sizes) with hidden states N(0, 1) drawn
+    independently per layer and step (so the union per layer spans 8 to 128),
+    or with --chain each layer's input made from the previous layer's output;
+    per-layer us and union-weighted expert GB/s."""
     import int4_routed_expert_softmax_b200 as moe
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
@@ -682,34 +687,38 @@ def run_stacked(args, ws_n, rank, local):
             ws = moe.alloc_workspace(d, T, dev)
             view = moe.moe_workspace_view(d, T, ws)
             nuni_t = moe.ws_slice(ws, view.n_uni, (1,), torch.int32)
-            x_buf = mi.make_x(T, w.H, mi.sub_seed(seed, 100, 1), dev).clone()
+            x_bufs = [mi.make_x(T, w.H, mi.sub_seed(seed, 100, 1 + l), dev).clone() for l in range(L)]
             outs = [torch.empty((T, w.H), dtype=torch.float32, device=dev) for _ in range(L)]
             layer_ms, layer_b = [], []
-            # One step (the L chained layers, the glue between them, a copy of
-            # each layer's union size) is one CUDA graph, with an event pair
-            # around every layer call: the Python glue would otherwise leave the
-            # GPU waiting for the host between layers.  Read once per step.
+            # One step (the L layers, with --chain the glue between them, a copy
+            # of each layer's union size) is one CUDA graph, with an event pair
+            # around every layer call: Python between the layers would otherwise
+            # leave the GPU waiting for the host.  Read once per step.
             nuni_hist = torch.zeros(L, dtype=torch.int32, device=dev)
             evs = [(torch.cuda.Event(enable_timing=True, external=True),
                     torch.cuda.Event(enable_timing=True, external=True)) for _ in range(L)]
             side = torch.cuda.Stream(device=dev)
             side.wait_stream(stream)
             with torch.cuda.stream(side):  # the library's one-time setup, outside the capture
-                moe.moe_layer_forward(d, x_buf, routers[0], tables[0], outs[0], ws)
+                moe.moe_layer_forward(d, x_bufs[0], routers[0], tables[0], outs[0], ws)
             stream.wait_stream(side)
             torch.cuda.synchronize()
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
                 gs = torch.cuda.current_stream()
-                x = x_buf
+                x = x_bufs[0]
                 for l in range(L):
+                    if not args.chain:
+                        x = x_bufs[l]
                     evs[l][0].record(gs)
                     moe.moe_layer_forward(d, x, routers[l], tables[l], outs[l], ws)
                     evs[l][1].record(gs)
                     nuni_hist[l:l + 1].copy_(nuni_t)
-                    x = chain_next_dev(x, outs[l])
+                    if args.chain:
+                        x = chain_next_dev(x, outs[l])
             for it in range(args.warmup + args.steps):
-                x_buf.copy_(mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1), dev))
+                for l in range(1 if args.chain else L):
+                    x_bufs[l].copy_(mi.make_x(T, w.H, mi.sub_seed(seed, 100 + it, 1 + l), dev))
                 graph.replay()
                 torch.cuda.synchronize()
                 if it >= args.warmup:
@@ -730,10 +739,12 @@ def run_stacked(args, ws_n, rank, local):
                 warmup=args.warmup, ms_per_step=round(tot_ms / args.steps, 4), higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="int4xint8->fp32", data="synthetic",
                 config={"workload": "stacked: 8 GLM-5.2-shaped layers resident in HBM (41.2 GB), batches of "
-                                    + ", ".join(str(t) for t in w.T_list) + " tokens, layers chained",
+                                    + ", ".join(str(t) for t in w.T_list) + " tokens, "
+                                    + ("layers chained (each layer's input from the previous output)" if args.chain
+                                       else "hidden states N(0,1) drawn independently per layer and step"),
                         "layers": L, "T_list": list(w.T_list),
                         "parallelism": f"replicas x{ws_n}", "l2": "each layer streams its own experts (> L2)",
-                        "timing": "one CUDA graph per step (layers, glue, union-size copies), "
+                        "timing": "one CUDA graph per step (layers, glue if chained, union-size copies), "
                                   "CUDA events around each layer call inside it"},
                 by_batch=res, clocks=clk.summary(),
                 gpu_launches=sum(moe.moe_layer_launches(d, T) for T in w.T_list) * L * args.steps)
