@@ -857,7 +857,8 @@ def run_tiered(args, ws_n, rank, local):
                 device_us_per_layer=dict(device_us, calls=len(prof),
                                          what="device stamps: routing kernel, gate/up, down, and the "
                                               "span from routing's first CTA to down's last (misses' "
-                                              "copies and the host's acquire fall inside it)"),
+                                              "copies and the host's acquire fall inside it); the first "
+                                              "layer calls of the timed region, up to the ring's 1024"),
                 clocks=clk.summary(),
                 # per token: every layer's routing, gate/up and down kernels, plus the
                 # next layer's prediction router for all but the last layer

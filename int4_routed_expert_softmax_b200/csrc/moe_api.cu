@@ -71,7 +71,11 @@ unsigned long long *prof_next() {
   std::lock_guard<std::mutex> lock(g_prof_mu);
   if (!g_prof) return nullptr;
   const int dev = current_device();
-  if (dev < 0 || g_prof_buf[dev] == nullptr || g_prof_n[dev] >= kProfSlots) return nullptr;
+  if (dev < 0) return nullptr;
+  if (g_prof_buf[dev] == nullptr || g_prof_n[dev] >= kProfSlots) {
+    g_prof_cur[dev] = nullptr;  // the experts half of this call goes unrecorded too
+    return nullptr;
+  }
   g_prof_cur[dev] = g_prof_buf[dev] + (size_t)(g_prof_n[dev]++) * kProfWords;
   return g_prof_cur[dev];
 }

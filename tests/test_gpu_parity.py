@@ -395,3 +395,33 @@ def test_batch_token_by_token_equals_union_kernels(name, T):
     assert np.array_equal(counts.cpu().numpy(), np.bincount(ta["idx"].reshape(-1), minlength=w.E))
     if name != "glm":
         _check_layer(w, x, Wr, blobs)
+
+
+def test_profile_ring_full_leaves_later_split_calls_unrecorded():
+    """Past the ring's 1024 records a call goes unrecorded, and so does the
+    experts half of a split layer (route, then experts): no later call stamps
+    into the last record."""
+    moe = _moe()
+    from int4_routed_expert_softmax_b200 import _cache as C
+    w = mi.WORKLOADS["tiny"]
+    x, Wr, blobs = mi.make_layer(w, 0, DEV)
+    T = x.shape[0]
+    _, ws, d = gpu_layer(w, x, Wr, blobs, path=1)
+    table = moe.expert_table(blobs)
+    out = torch.empty((T, w.H), device=DEV)
+    moe.moe_profile_enable(True)
+    try:
+        for _ in range(1024):
+            C.moe_layer_route(d, x, Wr, ws)
+            C.moe_layer_experts(d, T, table, out, ws)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(50_000_000)   # ~25 ms on the stream before the unrecorded calls
+        for _ in range(4):
+            C.moe_layer_route(d, x, Wr, ws)
+            C.moe_layer_experts(d, T, table, out, ws)
+        rec = moe.moe_profile_read(1024)
+    finally:
+        moe.moe_profile_enable(False)
+    assert len(rec) == 1024
+    spans = [r[3] for r in rec]
+    assert max(spans) < 5.0, max(spans)   # milliseconds: no record spans the sleep
