@@ -46,8 +46,9 @@ POOL = 64
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 50; tiered: 462 timed tokens, the rest of a 512-token sequence)")
+    ap.add_argument("--warmup", type=int, default=None, help="untimed steps (default 5; tiered: 50)")
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "stacked", "tiered"])
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="oracle sample budget")
@@ -65,6 +66,11 @@ def parse():
     ap.add_argument("--no-prefill", action="store_true",
                     help="default workload: leave out the prefill sub-object of the line")
     args = ap.parse_args()
+    tiered = args.workload == "tiered"
+    if args.steps is None:
+        args.steps = 462 if tiered else 50
+    if args.warmup is None:
+        args.warmup = 50 if tiered else 5
     if args.workload == "decode" and args.tokens is not None and not 1 <= args.tokens <= 16:
         ap.error("--tokens: the decode line takes 1 to 16 tokens per call")
     return args
