@@ -134,6 +134,12 @@ int copy_blob(moe_cache *c, int layer, int e, int slot, cudaStream_t s) {
       int rc = cuda_err(cudaStreamWaitEvent(s, ly.released, 0));
       if (rc) return rc;
     }
+    if (c->slot_ready_valid[slot]) {
+      // a copy into this slot may still be in flight, and on another stream
+      // (acquire and prefetch take the caller's streams): this one follows it
+      int rc = cuda_err(cudaStreamWaitEvent(s, c->slot_ready[slot], 0));
+      if (rc) return rc;
+    }
     int rc = cuda_err(cudaMemcpyAsync(dst, src, c->blob, cudaMemcpyHostToDevice, s));
     if (rc) {
       c->st.copy_errors++;
