@@ -430,10 +430,11 @@ int64_t moe_set_wait_limit(int64_t cycles);
 int moe_device_binary_version(void);
 
 /* Number of this library's kernels one moe_layer_forward call of T tokens on
- * `path` enqueues on the current device (plus one workspace memset), or a
- * negative status: 1 for a decode call of up to MOE_DECODE_T_MAX tokens that
- * the fused kernel runs, 3 per 16-token chunk on the union kernels, 9 on the
- * prefill path. */
+ * `path` enqueues on the current device, or a negative status: 1 for a
+ * decode call of up to MOE_DECODE_T_MAX tokens that the fused kernel runs
+ * (nothing else is enqueued), 3 per 16-token chunk on the union kernels and 9
+ * on the prefill path (each of those two also enqueues one workspace
+ * memset). */
 int moe_layer_launches(const moe_dims *dims, int32_t T, int32_t path);
 
 /* Number of streaming multiprocessors the kernels size their grids for
