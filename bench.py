@@ -245,7 +245,8 @@ def decode_config(w: mi.Workload, ws_n: int, path: str = "auto") -> dict:
          "parallelism": f"replicas x{ws_n}", "l2": "flushed (256 MiB write) before each step",
          "x_pool": POOL}
     if path != "auto":
-        c["path"] = "MOE_PATH_DECODE (routing, gate/up and down kernels over the batch union)"
+        c["path"] = ("MOE_PATH_DECODE (routing, gate/up and down kernels over the batch union)" if w.T > 1
+                     else "MOE_PATH_DECODE (one token: the fused kernel, as on every path)")
     return c
 
 
